@@ -1,0 +1,499 @@
+"""Benchmark of the gated delta-rule library on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workloads a,b,...]
+                    [--impl ours|reference]
+
+Prints ONE JSON line on rank 0.  The headline (`value`) is the first
+workload (default: the GDN prefill, 1 x 8192 tokens x 16 heads, d = 128,
+bf16).  Further workloads (default: the 256-sequence x 512-step GDN decode)
+are reported under "workloads" with the same fields.
+
+A "step" is one pass of the whole hot path over one batch of synthetic input:
+one gdr_prefill_chunked call for a prefill workload, the 512 consecutive
+gdr_decode_step calls for a decode workload.  Timing: W untimed warm-up
+steps, then K steps each timed with CUDA events on the stream the kernels are
+launched on; an L2 flush (a 512 MiB write) precedes every timed step and is
+not timed.  Barrier + synchronize bracket the timed region; the time is the
+max over ranks.  For N > 1 every rank runs its own independent batch (heads
+and sequences are independent; no collective on the data path) and `value`
+is the sum of tokens over ranks divided by that time ("weak" scaling).
+
+--impl reference times the fp64 CPU oracle (the reference this library is
+checked against) on a bounded sample of the same workload, on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from gated_delta_rule_151_b200 import gdr  # noqa: E402
+from gated_delta_rule_151_b200 import inputs as I  # noqa: E402
+
+METRIC = "gated delta-rule tokens/s (prefill, decode) and % roofline at 1 B200"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+CHUNK = 64
+
+
+# ------------------------------------------------------------ plumbing ----
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while running."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.t.join(timeout=2)
+
+    def summary(self):
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, val in zip(names, f[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def l2_flusher(device):
+    buf = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=device)
+
+    def flush():
+        buf.fill_(1)
+    return flush
+
+
+# ------------------------------------------------------- work per step ----
+
+def io_bytes(dtype):
+    return 2 if dtype == torch.bfloat16 else 4
+
+
+def prefill_work(inp):
+    """Algorithmic bytes and flops of one prefill launch (per-token-head
+    figures: q, k, v read, o written, beta and g read; plus 64 KiB of fp32
+    state written per (sequence, head), and read when an initial state is
+    given)."""
+    T, H, dk, dv, N = inp.total_T, inp.H, inp.d_k, inp.d_v, inp.num_seqs
+    e = io_bytes(inp.io_dtype)
+    gate = 4 * (dk if inp.gate_mode == I.CHANNEL else 1)
+    per_th = e * (2 * dk + 2 * dv) + 4 + gate
+    state = 4 * dk * dv * N * H * (2 if inp.h0 is not None else 1)
+    byts = T * H * per_th + state
+    flops = T * H * (5 * CHUNK * max(dk, dv) + 6 * dk * dv)
+    return byts, flops
+
+
+def decode_work(inp):
+    """Algorithmic bytes of one decode launch (one token per sequence): the
+    fp32 state read and written once, q/k/v/beta/g read, o written."""
+    N, H, dk, dv = inp.num_seqs, inp.H, inp.d_k, inp.d_v
+    e = io_bytes(inp.io_dtype)
+    gate = 4 * (dk if inp.gate_mode == I.CHANNEL else 1)
+    return N * H * (2 * 4 * dk * dv + e * (2 * dk + 2 * dv) + 4 + gate)
+
+
+class PrefillCase:
+    kind = "prefill"
+
+    def __init__(self, name, device, seed):
+        self.name = name
+        self.inp = inp = I.workload(name, seed=seed)
+        self.dev = device
+        self.d = {k: (None if v is None else v.to(device)) for k, v in dict(
+            q=inp.q, k=inp.k, v=inp.v, g=inp.g, beta=inp.beta, h0=inp.h0,
+            cu=inp.cu_seqlens).items()}
+        self.o = torch.empty((inp.total_T, inp.H, inp.d_v), dtype=inp.io_dtype, device=device)
+        self.fin = torch.empty((inp.num_seqs, inp.H, inp.d_v, inp.d_k), dtype=torch.float32,
+                               device=device)
+        gate = gdr.GDR_GATE_CHANNEL if inp.gate_mode == I.CHANNEL else gdr.GDR_GATE_SCALAR
+        io = gdr.GDR_BF16 if inp.io_dtype == torch.bfloat16 else gdr.GDR_F32
+        self.path = gdr.gdr_prefill_path(inp.d_k, inp.d_v, gate, io)
+        nbytes = gdr.gdr_prefill_workspace_size(inp.num_seqs, inp.total_T, inp.H, inp.d_k,
+                                                inp.d_v, gate, io)
+        self.ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=device) if nbytes else None
+        self.bytes, self.flops = prefill_work(inp)
+        self.tokens = inp.total_T
+        self.launches = 1
+
+    def step(self, stream=None):
+        d = self.d
+        gdr.gdr_prefill_chunked(d["q"], d["k"], d["v"], d["g"], d["beta"], d["h0"], d["cu"],
+                                o=self.o, final_state=self.fin, workspace=self.ws, stream=stream)
+
+    def host_inputs(self):
+        inp = self.inp
+        xs = dict(q=inp.q, k=inp.k, v=inp.v, g=inp.g, beta=inp.beta, cu=inp.cu_seqlens)
+        if inp.h0 is not None:
+            xs["h0"] = inp.h0
+        return {k: v.pin_memory() for k, v in xs.items()}
+
+    def e2e_step(self, host, host_o, host_fin, stream):
+        dev = {k: v.to(self.dev, non_blocking=True) for k, v in host.items()}
+        gdr.gdr_prefill_chunked(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"],
+                                dev.get("h0"), dev["cu"], o=self.o, final_state=self.fin,
+                                workspace=self.ws, stream=stream)
+        host_o.copy_(self.o, non_blocking=True)
+        host_fin.copy_(self.fin, non_blocking=True)
+
+    def e2e_buffers(self):
+        host = self.host_inputs()
+        h2d = sum(v.numel() * v.element_size() for v in host.values())
+        ho = torch.empty(self.o.shape, dtype=self.o.dtype).pin_memory()
+        hf = torch.empty(self.fin.shape, dtype=self.fin.dtype).pin_memory()
+        d2h = ho.numel() * ho.element_size() + hf.numel() * hf.element_size()
+        return host, ho, hf, h2d, d2h
+
+    def dtype_label(self):
+        if self.path == gdr.GDR_PATH_TCGEN05:
+            return "bf16/tf32 tensor-core operands, fp32 accumulate and state"
+        return "f32"
+
+
+class DecodeCase:
+    kind = "decode"
+
+    def __init__(self, name, device, seed):
+        self.name = name
+        self.inp = inp = I.workload(name, seed=seed)
+        self.dev = device
+        N = inp.num_seqs
+        self.steps = inp.total_T // N
+        self.q, self.k, self.v = (I.decode_view(x, N).to(device) for x in (inp.q, inp.k, inp.v))
+        self.g = I.decode_view(inp.g, N).to(device)
+        self.beta = I.decode_view(inp.beta, N).to(device)
+        self.state = inp.h0.to(device).clone()
+        self.o = torch.empty((self.steps, N, inp.H, inp.d_v), dtype=inp.io_dtype, device=device)
+        self.bytes = decode_work(inp)          # per launch
+        self.flops = 0
+        self.tokens = inp.total_T              # N * steps per bench step
+        self.launches = self.steps
+        self.path = None
+
+    def step(self, stream=None):
+        for t in range(self.steps):
+            gdr.gdr_decode_step(self.q[t], self.k[t], self.v[t], self.g[t], self.beta[t],
+                                self.state, o=self.o[t], stream=stream)
+
+    def e2e_buffers(self):
+        host = {k: v.cpu().pin_memory() for k, v in
+                dict(q=self.q, k=self.k, v=self.v, g=self.g, beta=self.beta).items()}
+        ho = torch.empty(self.o.shape, dtype=self.o.dtype).pin_memory()
+        h2d = sum(v.numel() * v.element_size() for v in host.values())
+        d2h = ho.numel() * ho.element_size()
+        self._dev_tok = {k: torch.empty(v.shape[1:], dtype=v.dtype, device=self.dev)
+                         for k, v in host.items()}
+        return host, ho, None, h2d, d2h
+
+    def e2e_step(self, host, host_o, host_fin, stream):
+        dt = self._dev_tok
+        for t in range(self.steps):
+            for key in dt:
+                dt[key].copy_(host[key][t], non_blocking=True)
+            gdr.gdr_decode_step(dt["q"], dt["k"], dt["v"], dt["g"], dt["beta"], self.state,
+                                o=self.o[t], stream=stream)
+            host_o[t].copy_(self.o[t], non_blocking=True)
+
+    def dtype_label(self):
+        return "f32"
+
+
+def make_case(name, device, seed):
+    if name.startswith("decode"):
+        return DecodeCase(name, device, seed)
+    return PrefillCase(name, device, seed)
+
+
+# ----------------------------------------------------------- measuring ----
+
+def timed_steps(fn, K, flush, stream):
+    """K steps, each bracketed by CUDA events on `stream` after an untimed
+    L2 flush; returns the per-step times in ms."""
+    times = []
+    for _ in range(K):
+        flush()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        times.append((a, b))
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in times]
+
+
+def max_over_ranks(x, ws):
+    if ws == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+def load_traffic(case):
+    """DRAM bytes per launch of the dominant kernel from a committed ncu
+    capture, if it was taken on the kernel sources as they are now."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        d = json.load(open(p))
+        ent = d.get(case.name)
+        if not ent:
+            return None
+        import hashlib
+        h = hashlib.sha256()
+        for rel in ent["sources"]:
+            h.update(open(os.path.join(ROOT, rel), "rb").read())
+        if h.hexdigest() != ent["sources_sha256"]:
+            return None
+        return float(ent["bytes_per_launch"])
+    except Exception:
+        return None
+
+
+def bench_case(case, args, ws, rank, flush, stream, pk, pk_kind):
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            case.step(stream)
+        torch.cuda.synchronize()
+        barrier(ws)
+        with ClockSampler(torch.cuda.current_device()) as clk:
+            times = timed_steps(lambda: case.step(stream), args.steps, flush, stream)
+        barrier(ws)
+    ms = max_over_ranks(sum(times) / len(times), ws)
+    tokens_all = case.tokens * ws
+    value = tokens_all / (ms / 1e3)
+    launch_ms = ms / case.launches
+    achieved = case.bytes / (launch_ms / 1e3) / 1e9
+    hbm_peak = float(pk["hbm_gbs"])
+    roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
+            "frac": round(achieved / hbm_peak, 4), "traffic": load_traffic(case),
+            "peak_source": f"{pk_kind} HBM copy bandwidth"}
+    if case.kind == "prefill":
+        tc_peak = float(pk["bf16_tflops"]) / 2.0   # tf32 = half the bf16 rate
+        roof["flops_per_launch"] = case.flops
+        roof["tensor_tflops"] = round(case.flops / (launch_ms / 1e3) / 1e12, 2)
+        roof["tensor_frac_of_tf32_peak"] = round(case.flops / (launch_ms / 1e3) / 1e12 / tc_peak, 4)
+        roof["algorithmic_bytes_per_launch"] = case.bytes
+    else:
+        roof["algorithmic_bytes_per_launch"] = case.bytes
+        roof["frac_of_8TBps_nominal"] = round(achieved / 8000.0, 4)
+
+    # end to end: pinned host buffers, copies inside the timed region
+    host, ho, hf, h2d, d2h = case.e2e_buffers()
+    with torch.cuda.stream(stream):
+        case.e2e_step(host, ho, hf, stream)
+        torch.cuda.synchronize()
+        barrier(ws)
+        e2e_times = timed_steps(lambda: case.e2e_step(host, ho, hf, stream), args.steps, flush,
+                                stream)
+        barrier(ws)
+    e2e_ms = max_over_ranks(sum(e2e_times) / len(e2e_times), ws)
+    inp = case.inp
+    cfg = {"workload": case.name, "num_seqs": inp.num_seqs, "total_T": inp.total_T,
+           "H": inp.H, "d_k": inp.d_k, "d_v": inp.d_v, "gate": inp.gate_mode,
+           "io": str(inp.io_dtype).replace("torch.", ""),
+           "h0": inp.h0 is not None, "l2": "flushed (512 MiB write) before every timed step",
+           "kernel": ("decode" if case.kind == "decode" else
+                      ("tcgen05" if case.path == gdr.GDR_PATH_TCGEN05 else "simt"))}
+    if case.kind == "decode":
+        cfg["steps_per_bench_step"] = case.steps
+    return {
+        "value": value, "ms_per_step": ms, "tokens_per_step": tokens_all,
+        "dtype": case.dtype_label(), "config": cfg, "roofline": roof,
+        "e2e": {"value": tokens_all / (e2e_ms / 1e3), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": case.launches * args.steps, "clocks": clk.summary(),
+    }
+
+
+def cpu_baseline(name, budget_s=20.0):
+    """The oracle, as it stands, on a bounded sample of the workload: whole
+    heads (all tokens of every sequence) until the estimated cost reaches the
+    budget.  Returns tokens/s scaled to the full workload's head count."""
+    import oracle
+    inp = I.workload(name)
+    cores = oracle.loop.default_threads()
+    per_head_flop = 7.0 * inp.d_k * inp.d_v * inp.total_T
+    est_rate = 1.2e9 * cores                      # fp64 flop/s, rough
+    nh = int(max(1, min(inp.H, budget_s * est_rate / per_head_flop)))
+    heads = list(range(nh))
+    t = time.perf_counter()
+    oracle.loop.run_inputs(inp, heads=heads, nthreads=cores)
+    dt = time.perf_counter() - t
+    value = inp.total_T * (nh / inp.H) / dt
+    return {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{name}: {nh} of {inp.H} heads, all {inp.total_T} tokens, "
+                      f"fp64 C loop, {dt:.2f} s"}
+
+
+def run_reference(args, ws, rank):
+    """--impl reference: the fp64 oracle timed on the host cores."""
+    if rank != 0:
+        return
+    import oracle
+    name = args.workloads.split(",")[0]
+    inp = I.workload(name)
+    cores = oracle.loop.default_threads()
+    per_head_flop = 7.0 * inp.d_k * inp.d_v * inp.total_T
+    nh = int(max(1, min(inp.H, 8.0 * 1.2e9 * cores / per_head_flop)))
+    heads = list(range(nh))
+    for _ in range(args.warmup if args.warmup < 2 else 1):
+        oracle.loop.run_inputs(inp, heads=heads[:1], nthreads=cores)
+    times = []
+    for _ in range(args.steps):
+        t = time.perf_counter()
+        oracle.loop.run_inputs(inp, heads=heads, nthreads=cores)
+        times.append(time.perf_counter() - t)
+    dt = sum(times) / len(times)
+    value = inp.total_T * (nh / inp.H) / dt
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": name, "sample_heads": nh, "H": inp.H, "total_T": inp.total_T},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"{name}: {nh} of {inp.H} heads per step"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workloads", default="gdn_prefill,decode_gdn",
+                    help="comma list from: " + ",".join(I.WORKLOADS) + " (or 'all')")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.workloads == "all":
+        args.workloads = "gdn_prefill,kda_prefill,varlen_gdn,decode_gdn,decode_kda"
+    if args.warmup < 3:
+        args.warmup = 3
+    ws, rank, local = dist_env()
+
+    if args.impl == "reference":
+        run_reference(args, ws, rank)
+        return
+
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+    gdr.load_library()
+    pk, pk_kind = peaks()
+    flush = l2_flusher(device)
+    stream = torch.cuda.Stream(device=device)
+    names = [w for w in args.workloads.split(",") if w]
+    results = {}
+    for i, name in enumerate(names):
+        case = make_case(name, device, seed=rank)
+        results[name] = bench_case(case, args, ws, rank, flush, stream, pk, pk_kind)
+        del case
+        torch.cuda.empty_cache()
+
+    if rank == 0:
+        head = results[names[0]]
+        line = {
+            "metric": METRIC, "value": head["value"], "unit": UNIT, "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": head["dtype"], "data": "synthetic (seeded PCG64; see inputs.py)",
+            "config": head["config"], "roofline": head["roofline"], "e2e": head["e2e"],
+            "gpu_launches": sum(r["gpu_launches"] for r in results.values()),
+            "clocks": head["clocks"],
+        }
+        if ws == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(names[0])
+        line["workloads"] = {n: r for n, r in results.items() if n != names[0]}
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,138 @@
+// C ABI of libgdr: argument validation, workspace sizing and kernel dispatch.
+// Every check runs on the host before any launch; on error nothing is
+// enqueued.  See include/gdr.h for the contract.
+#include <cstdint>
+
+#include "common.cuh"
+#include "gdr.h"
+#include "internal.h"
+
+namespace {
+
+bool valid_dim(int32_t d) { return d == 16 || d == 32 || d == 64 || d == 128; }
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool ok_ptr(const void *p) { return p != nullptr && aligned16(p); }
+
+bool ok_opt_ptr(const void *p) { return p == nullptr || aligned16(p); }
+
+gdr_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? GDR_OK : GDR_ERR_CUDA; }
+
+bool uses_tcgen05(int32_t d_k, int32_t d_v, gdr_gate_mode_t gate_mode, gdr_dtype_t io_dtype) {
+    (void)gate_mode;
+    return gdr::tcgen05_prefill_available() && io_dtype == GDR_BF16 && d_k == 128 && d_v == 128;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *gdr_status_string(gdr_status_t status) {
+    switch (status) {
+        case GDR_OK: return "GDR_OK";
+        case GDR_ERR_INVALID_ARG: return "GDR_ERR_INVALID_ARG: invalid argument";
+        case GDR_ERR_UNSUPPORTED: return "GDR_ERR_UNSUPPORTED: unsupported request";
+        case GDR_ERR_WORKSPACE: return "GDR_ERR_WORKSPACE: workspace missing or too small";
+        case GDR_ERR_CUDA: return "GDR_ERR_CUDA: a CUDA call or kernel launch failed";
+        case GDR_ERR_DEVICE_TIMEOUT: return "GDR_ERR_DEVICE_TIMEOUT: a device-side wait gave up";
+    }
+    return "GDR_ERR_UNKNOWN";
+}
+
+gdr_status_t gdr_prefill_path(int32_t d_k, int32_t d_v, gdr_gate_mode_t gate_mode,
+                              gdr_dtype_t io_dtype, gdr_prefill_path_t *path) {
+    if (path == nullptr || !valid_dim(d_k) || !valid_dim(d_v)) return GDR_ERR_INVALID_ARG;
+    if (gate_mode != GDR_GATE_SCALAR && gate_mode != GDR_GATE_CHANNEL) return GDR_ERR_INVALID_ARG;
+    if (io_dtype != GDR_F32 && io_dtype != GDR_BF16) return GDR_ERR_INVALID_ARG;
+    *path = uses_tcgen05(d_k, d_v, gate_mode, io_dtype) ? GDR_PATH_TCGEN05 : GDR_PATH_SIMT;
+    return GDR_OK;
+}
+
+gdr_status_t gdr_prefill_workspace_size(int32_t num_seqs, int32_t total_T, int32_t H,
+                                        int32_t d_k, int32_t d_v, gdr_gate_mode_t gate_mode,
+                                        gdr_dtype_t io_dtype, size_t *bytes) {
+    gdr_prefill_path_t path;
+    if (bytes == nullptr || num_seqs < 0 || total_T < 0 || H < 0) return GDR_ERR_INVALID_ARG;
+    gdr_status_t st = gdr_prefill_path(d_k, d_v, gate_mode, io_dtype, &path);
+    if (st != GDR_OK) return st;
+    *bytes = path == GDR_PATH_TCGEN05 ? gdr::tcgen05_workspace_bytes(num_seqs, total_T, H) : 0;
+    return GDR_OK;
+}
+
+gdr_status_t gdr_prefill_chunked(const void *q, const void *k, const void *v, const float *g,
+                                 const float *beta, const float *initial_state,
+                                 const int32_t *cu_seqlens, int32_t num_seqs, int32_t total_T,
+                                 int32_t H, int32_t d_k, int32_t d_v, gdr_gate_mode_t gate_mode,
+                                 gdr_dtype_t io_dtype, void *o, float *final_state,
+                                 void *workspace, size_t workspace_bytes, void *stream) {
+    if (num_seqs < 0 || total_T < 0 || H < 1) return GDR_ERR_INVALID_ARG;
+    if (!valid_dim(d_k) || !valid_dim(d_v)) return GDR_ERR_INVALID_ARG;
+    if (gate_mode != GDR_GATE_SCALAR && gate_mode != GDR_GATE_CHANNEL) return GDR_ERR_INVALID_ARG;
+    if (io_dtype != GDR_F32 && io_dtype != GDR_BF16) return GDR_ERR_INVALID_ARG;
+    if (num_seqs == 0 && total_T != 0) return GDR_ERR_INVALID_ARG;
+    if (cu_seqlens == nullptr && num_seqs > 0 && total_T % num_seqs != 0) return GDR_ERR_INVALID_ARG;
+    if (total_T > 0) {
+        if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(g) || !ok_ptr(beta) || !ok_ptr(o))
+            return GDR_ERR_INVALID_ARG;
+    } else if (!ok_opt_ptr(q) || !ok_opt_ptr(k) || !ok_opt_ptr(v) || !ok_opt_ptr(g) ||
+               !ok_opt_ptr(beta) || !ok_opt_ptr(o)) {
+        return GDR_ERR_INVALID_ARG;
+    }
+    if (!ok_opt_ptr(initial_state) || !ok_opt_ptr(final_state) || !ok_opt_ptr(cu_seqlens))
+        return GDR_ERR_INVALID_ARG;
+    // Element counts must stay addressable with 64-bit offsets and the
+    // kernels' 32-bit token indices.
+    if ((int64_t)total_T * H > (int64_t)INT32_MAX) return GDR_ERR_INVALID_ARG;
+
+    size_t need = 0;
+    gdr_status_t st = gdr_prefill_workspace_size(num_seqs, total_T, H, d_k, d_v, gate_mode,
+                                                 io_dtype, &need);
+    if (st != GDR_OK) return st;
+    if (need > 0 && (workspace == nullptr || workspace_bytes < need || !aligned16(workspace)))
+        return GDR_ERR_WORKSPACE;
+    if (num_seqs == 0) return GDR_OK;
+
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const bool channel = gate_mode == GDR_GATE_CHANNEL;
+    if (uses_tcgen05(d_k, d_v, gate_mode, io_dtype))
+        return from_cuda(gdr::launch_prefill_tcgen05(q, k, v, g, beta, initial_state, cu_seqlens,
+                                                      num_seqs, total_T, H, channel, o,
+                                                      final_state, workspace, s));
+    return from_cuda(gdr::launch_prefill_simt(q, k, v, g, beta, initial_state, cu_seqlens,
+                                              num_seqs, total_T, H, d_k, d_v, channel,
+                                              io_dtype == GDR_BF16, o, final_state, s));
+}
+
+gdr_status_t gdr_prefill_check_workspace(const void *workspace, size_t workspace_bytes,
+                                         void *stream) {
+    if (workspace == nullptr || workspace_bytes == 0) return GDR_OK;
+    if (workspace_bytes < sizeof(uint32_t) || !aligned16(workspace)) return GDR_ERR_INVALID_ARG;
+    uint32_t word = 0;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return GDR_ERR_CUDA;
+    return word == 0 ? GDR_OK : GDR_ERR_DEVICE_TIMEOUT;
+}
+
+gdr_status_t gdr_decode_step(const void *q, const void *k, const void *v, const float *g,
+                             const float *beta, float *state, int32_t N, int32_t H, int32_t d_k,
+                             int32_t d_v, gdr_gate_mode_t gate_mode, gdr_dtype_t io_dtype,
+                             void *o, void *stream) {
+    if (N < 0 || H < 0) return GDR_ERR_INVALID_ARG;
+    if (!valid_dim(d_k) || !valid_dim(d_v)) return GDR_ERR_INVALID_ARG;
+    if (gate_mode != GDR_GATE_SCALAR && gate_mode != GDR_GATE_CHANNEL) return GDR_ERR_INVALID_ARG;
+    if (io_dtype != GDR_F32 && io_dtype != GDR_BF16) return GDR_ERR_INVALID_ARG;
+    if ((int64_t)N * H > (int64_t)INT32_MAX) return GDR_ERR_INVALID_ARG;
+    if ((int64_t)N * H == 0) return GDR_OK;
+    if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(g) || !ok_ptr(beta) || !ok_ptr(state) ||
+        !ok_ptr(o))
+        return GDR_ERR_INVALID_ARG;
+    return from_cuda(gdr::launch_decode_step(q, k, v, g, beta, state, N, H, d_k, d_v,
+                                             gate_mode == GDR_GATE_CHANNEL,
+                                             io_dtype == GDR_BF16, o,
+                                             static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,29 @@
+// Host-side launchers behind the C ABI (arguments already validated).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace gdr {
+
+cudaError_t launch_decode_step(const void *q, const void *k, const void *v, const float *g,
+                               const float *beta, float *state, int N, int H, int DK, int DV,
+                               bool channel, bool bf16, void *o, cudaStream_t stream);
+
+cudaError_t launch_prefill_simt(const void *q, const void *k, const void *v, const float *g,
+                                const float *beta, const float *h0, const int32_t *cu,
+                                int num_seqs, int total_T, int H, int DK, int DV, bool channel,
+                                bool bf16, void *o, float *fin, cudaStream_t stream);
+
+size_t prefill_simt_smem_bytes(int DK, int DV);
+
+// tcgen05 prefill: bf16 I/O, d_k = d_v = 128.
+bool tcgen05_prefill_available();
+size_t tcgen05_workspace_bytes(int num_seqs, int total_T, int H);
+cudaError_t launch_prefill_tcgen05(const void *q, const void *k, const void *v, const float *g,
+                                   const float *beta, const float *h0, const int32_t *cu,
+                                   int num_seqs, int total_T, int H, bool channel, void *o,
+                                   float *fin, void *workspace, cudaStream_t stream);
+
+}  // namespace gdr

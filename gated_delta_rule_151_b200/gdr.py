@@ -1,0 +1,221 @@
+"""Python binding of libgdr (ctypes).  Argument marshalling only: every step of
+the recurrence runs in the library's CUDA kernels.
+
+The functions carry the C ABI's names (include/gdr.h) and take torch CUDA
+tensors; they check dtype, device and contiguity, pass raw pointers and the
+current CUDA stream, and raise ``GdrError`` on any non-OK status.  There is no
+fallback: if libgdr.so is missing or fails to load, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libgdr.so")
+
+GDR_OK = 0
+GDR_ERR_INVALID_ARG = 1
+GDR_ERR_UNSUPPORTED = 2
+GDR_ERR_WORKSPACE = 3
+GDR_ERR_CUDA = 4
+GDR_ERR_DEVICE_TIMEOUT = 5
+
+GDR_GATE_SCALAR = 0
+GDR_GATE_CHANNEL = 1
+GDR_F32 = 0
+GDR_BF16 = 1
+GDR_PATH_SIMT = 0
+GDR_PATH_TCGEN05 = 1
+
+# Every symbol include/gdr.h declares.
+EXPORTED = ("gdr_status_string", "gdr_prefill_workspace_size", "gdr_prefill_path",
+            "gdr_prefill_chunked", "gdr_prefill_check_workspace", "gdr_decode_step")
+
+
+class GdrError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {gdr_status_string(status)}")
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def load_library():
+    """Load libgdr.so once (raises if it is missing: there is no fallback)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libgdr.so not built ({LIB_PATH}); run "
+                               "`python -m gated_delta_rule_151_b200.build`")
+        lib = ctypes.CDLL(LIB_PATH)
+        P, I32, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+        ST = ctypes.c_int
+        lib.gdr_status_string.argtypes = [ST]
+        lib.gdr_status_string.restype = ctypes.c_char_p
+        lib.gdr_prefill_workspace_size.argtypes = [I32, I32, I32, I32, I32, ST, ST,
+                                                   ctypes.POINTER(SZ)]
+        lib.gdr_prefill_workspace_size.restype = ST
+        lib.gdr_prefill_path.argtypes = [I32, I32, ST, ST, ctypes.POINTER(ctypes.c_int)]
+        lib.gdr_prefill_path.restype = ST
+        lib.gdr_prefill_chunked.argtypes = [P, P, P, P, P, P, P, I32, I32, I32, I32, I32, ST, ST,
+                                            P, P, P, SZ, P]
+        lib.gdr_prefill_chunked.restype = ST
+        lib.gdr_prefill_check_workspace.argtypes = [P, SZ, P]
+        lib.gdr_prefill_check_workspace.restype = ST
+        lib.gdr_decode_step.argtypes = [P, P, P, P, P, P, I32, I32, I32, I32, ST, ST, P, P]
+        lib.gdr_decode_step.restype = ST
+        _lib = lib
+        return lib
+
+
+def gdr_status_string(status: int) -> str:
+    return load_library().gdr_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str):
+    if status != GDR_OK:
+        raise GdrError(status, where)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_ptr(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, int):
+        return ctypes.c_void_p(stream)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _io_code(dtype: torch.dtype) -> int:
+    if dtype == torch.bfloat16:
+        return GDR_BF16
+    if dtype == torch.float32:
+        return GDR_F32
+    raise TypeError(f"io dtype must be bfloat16 or float32, got {dtype}")
+
+
+def _need(t, name, dtype=None, ndim=None):
+    if t is None:
+        raise ValueError(f"{name} is required")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got {t.dim()}")
+
+
+def gdr_prefill_workspace_size(num_seqs, total_T, H, d_k, d_v, gate_mode, io_dtype) -> int:
+    out = ctypes.c_size_t(0)
+    _check(load_library().gdr_prefill_workspace_size(num_seqs, total_T, H, d_k, d_v, gate_mode,
+                                                     io_dtype, ctypes.byref(out)),
+           "gdr_prefill_workspace_size")
+    return int(out.value)
+
+
+def gdr_prefill_path(d_k, d_v, gate_mode, io_dtype) -> int:
+    out = ctypes.c_int(0)
+    _check(load_library().gdr_prefill_path(d_k, d_v, gate_mode, io_dtype, ctypes.byref(out)),
+           "gdr_prefill_path")
+    return int(out.value)
+
+
+def gdr_prefill_chunked(q, k, v, g, beta, initial_state=None, cu_seqlens=None, *,
+                        num_seqs=None, o=None, final_state=None, output_final_state=True,
+                        workspace=None, stream=None):
+    """Chunked prefill (see include/gdr.h).  Returns (o, final_state).
+
+    q, k [T, H, d_k], v [T, H, d_v] (bf16 or fp32); g [T, H] or [T, H, d_k]
+    fp32; beta [T, H] fp32; initial_state [N, H, d_v, d_k] fp32 or None;
+    cu_seqlens int32 [N + 1] on the device, or None with ``num_seqs`` equal
+    sequences (default 1).  ``final_state`` may be given (it may be the same
+    tensor as initial_state); otherwise one is allocated when
+    ``output_final_state``.
+    """
+    _need(q, "q", ndim=3)
+    io = q.dtype
+    _need(k, "k", io, 3)
+    _need(v, "v", io, 3)
+    _need(beta, "beta", torch.float32, 2)
+    _need(g, "g", torch.float32)
+    T, H, dk = q.shape
+    dv = v.shape[2]
+    if g.dim() == 2:
+        gate = GDR_GATE_SCALAR
+    elif g.dim() == 3:
+        gate = GDR_GATE_CHANNEL
+    else:
+        raise ValueError("g must be [T, H] or [T, H, d_k]")
+    if cu_seqlens is not None:
+        _need(cu_seqlens, "cu_seqlens", torch.int32, 1)
+        N = cu_seqlens.numel() - 1
+    else:
+        N = 1 if num_seqs is None else int(num_seqs)
+    if initial_state is not None:
+        _need(initial_state, "initial_state", torch.float32, 4)
+    if o is None:
+        o = torch.empty((T, H, dv), dtype=io, device=q.device)
+    _need(o, "o", io, 3)
+    if final_state is None and output_final_state:
+        final_state = torch.empty((N, H, dv, dk), dtype=torch.float32, device=q.device)
+    if final_state is not None:
+        _need(final_state, "final_state", torch.float32, 4)
+    io_code = _io_code(io)
+    ws_bytes = gdr_prefill_workspace_size(N, T, H, dk, dv, gate, io_code)
+    if ws_bytes and workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    st = load_library().gdr_prefill_chunked(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(initial_state), _ptr(cu_seqlens),
+        N, T, H, dk, dv, gate, io_code, _ptr(o), _ptr(final_state), _ptr(workspace),
+        workspace.numel() if workspace is not None else 0, _stream_ptr(stream))
+    _check(st, "gdr_prefill_chunked")
+    return o, final_state
+
+
+def gdr_prefill_check_workspace(workspace, stream=None):
+    _check(load_library().gdr_prefill_check_workspace(
+        _ptr(workspace), workspace.numel() if workspace is not None else 0, _stream_ptr(stream)),
+        "gdr_prefill_check_workspace")
+
+
+def gdr_decode_step(q, k, v, g, beta, state, *, o=None, stream=None):
+    """One decode step (see include/gdr.h): state is updated in place.
+
+    q, k [N, H, d_k], v [N, H, d_v] (bf16 or fp32); g [N, H] or [N, H, d_k]
+    fp32; beta [N, H] fp32; state [N, H, d_v, d_k] fp32.  Returns o [N, H, d_v].
+    """
+    _need(q, "q", ndim=3)
+    io = q.dtype
+    _need(k, "k", io, 3)
+    _need(v, "v", io, 3)
+    _need(beta, "beta", torch.float32, 2)
+    _need(g, "g", torch.float32)
+    _need(state, "state", torch.float32, 4)
+    N, H, dk = q.shape
+    dv = v.shape[2]
+    gate = GDR_GATE_SCALAR if g.dim() == 2 else GDR_GATE_CHANNEL
+    if o is None:
+        o = torch.empty((N, H, dv), dtype=io, device=q.device)
+    _need(o, "o", io, 3)
+    st = load_library().gdr_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                        _ptr(state), N, H, dk, dv, gate, _io_code(io), _ptr(o),
+                                        _stream_ptr(stream))
+    _check(st, "gdr_decode_step")
+    return o

@@ -1,0 +1,169 @@
+/*
+ * gdr.h -- C ABI of libgdr, the gated delta-rule recurrence for NVIDIA B200
+ * (sm_100a).
+ *
+ * The recurrence (page "How the New Flash Models Work: Inside GLM-5.3-Flash
+ * and Qwen3.8-Flash-Next", section "Linear attention: a fixed-size memory in
+ * place of the cache", Gated DeltaNet and Kimi Delta Attention equations):
+ *
+ *     S_t = S_{t-1} D_t (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,   o_t = S_t q_t
+ *
+ * per (sequence, head), with S_t a d_v x d_k fp32 matrix (row r = value
+ * channel r, column j = key channel j) and D_t = alpha_t I (GDR_GATE_SCALAR,
+ * Gated DeltaNet: one gate per head and token) or D_t = Diag(alpha_t)
+ * (GDR_GATE_CHANNEL, Kimi Delta Attention: one gate per key channel).
+ * With D_t = I this is the ungated rule S_t = S_{t-1} + beta_t (v_t - S_{t-1} k_t) k_t^T
+ * (page "Qwen3.8-Flash vs GLM-5.3-Flash", section "The 3:1 Blueprint").
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Gates are passed as their logarithm g = log(alpha) <= 0, in fp32
+ *   (gates and decays stay in high precision; page "How the New Flash Models
+ *   Work", section on precision).  g = -inf (alpha = 0) is allowed and resets
+ *   the state; the kernels clamp g at -20 per token (alpha >= 2e-9), which
+ *   changes no result by more than 2e-9 |S|.
+ * - beta is fp32, any finite value.  q and k are used as given: the library
+ *   neither normalises them nor scales q.
+ * - Tensors are dense, row-major and contiguous, token-major:
+ *     q, k     [T, H, d_k]        io dtype
+ *     v, o     [T, H, d_v]        io dtype
+ *     g        [T, H]             fp32 (scalar gate)
+ *              [T, H, d_k]        fp32 (channel gate)
+ *     beta     [T, H]             fp32
+ *     state    [N, H, d_v, d_k]   fp32
+ * - d_k and d_v are each one of 16, 32, 64, 128.  Every pointer must be
+ *   16-byte aligned.
+ * - All pointers are DEVICE pointers owned by the caller.  The library
+ *   allocates nothing, keeps no global state beyond cached kernel
+ *   attributes, and never synchronises the device: work is enqueued on
+ *   `stream` (a cudaStream_t passed as void*; NULL = legacy default stream)
+ *   and runs asynchronously.
+ * - Arguments are validated on the host before anything is launched.  On any
+ *   error nothing is launched and no output is written.  Launch failures
+ *   return GDR_ERR_CUDA.  Device-side faults from invalid device pointers
+ *   cannot be detected by the library.
+ * - Outputs must not overlap inputs, except final_state == initial_state
+ *   (in-place state update), which is supported.
+ */
+#ifndef GDR_H
+#define GDR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define GDR_API __attribute__((visibility("default")))
+#else
+#define GDR_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GDR_OK = 0,
+    GDR_ERR_INVALID_ARG = 1,    /* null pointer, bad size, misalignment, ... */
+    GDR_ERR_UNSUPPORTED = 2,    /* valid request this build does not serve   */
+    GDR_ERR_WORKSPACE = 3,      /* workspace missing or too small            */
+    GDR_ERR_CUDA = 4,           /* a CUDA runtime call or launch failed      */
+    GDR_ERR_DEVICE_TIMEOUT = 5  /* a bounded device-side wait gave up        */
+} gdr_status_t;
+
+typedef enum {
+    GDR_GATE_SCALAR = 0,   /* Gated DeltaNet: g [T, H]           */
+    GDR_GATE_CHANNEL = 1   /* Kimi Delta Attention: g [T, H, d_k] */
+} gdr_gate_mode_t;
+
+typedef enum {
+    GDR_F32 = 0,   /* q, k, v and o in fp32     */
+    GDR_BF16 = 1   /* q, k, v and o in bfloat16 */
+} gdr_dtype_t;
+
+/* Which prefill kernel serves a request. */
+typedef enum {
+    GDR_PATH_SIMT = 0,     /* fp32 CUDA-core chunked kernel (any d, any io dtype) */
+    GDR_PATH_TCGEN05 = 1   /* tcgen05/TMEM/TMA chunked kernel (bf16, d_k = d_v = 128) */
+} gdr_prefill_path_t;
+
+/* Human-readable name of a status code (static storage, never NULL). */
+GDR_API const char *gdr_status_string(gdr_status_t status);
+
+/*
+ * Bytes of device workspace gdr_prefill_chunked needs for this problem
+ * (written to *bytes; may be 0).  Pure host function.
+ */
+GDR_API gdr_status_t gdr_prefill_workspace_size(int32_t num_seqs, int32_t total_T, int32_t H,
+                                        int32_t d_k, int32_t d_v,
+                                        gdr_gate_mode_t gate_mode, gdr_dtype_t io_dtype,
+                                        size_t *bytes);
+
+/* The kernel gdr_prefill_chunked launches for this shape/dtype (host only). */
+GDR_API gdr_status_t gdr_prefill_path(int32_t d_k, int32_t d_v, gdr_gate_mode_t gate_mode,
+                              gdr_dtype_t io_dtype, gdr_prefill_path_t *path);
+
+/*
+ * Chunked prefill over packed variable-length sequences.
+ *
+ * Runs the recurrence over every token of every sequence and head, in
+ * chunks of 64 tokens that never straddle a sequence boundary; within a chunk
+ * the tokens are combined in the UT/WY form (cumulative gate products, the
+ * unit-lower-triangular inverse of (I + strictly-lower(beta K K^T)) weighted by
+ * the gate ratios, and the chunk contractions), and the fp32 state is carried
+ * on-chip from chunk to chunk.  Results equal the token loop up to rounding.
+ *
+ * q, k, v, g, beta   inputs, layouts above, T = total_T.
+ * initial_state      [num_seqs, H, d_v, d_k] fp32, or NULL for zeros.
+ * cu_seqlens         DEVICE int32 [num_seqs + 1]: cu[0] = 0, non-decreasing,
+ *                    cu[num_seqs] = total_T; sequence n is tokens
+ *                    [cu[n], cu[n+1]).  NULL means num_seqs equal sequences of
+ *                    total_T / num_seqs tokens (total_T must divide).  The
+ *                    contents cannot be checked on the host: the kernels clamp
+ *                    every range into [0, total_T] and treat a negative length
+ *                    as empty, so a malformed array gives wrong results but no
+ *                    out-of-bounds access.
+ * o                  [total_T, H, d_v] output, io dtype.
+ * final_state        [num_seqs, H, d_v, d_k] fp32 state after each sequence's
+ *                    last token, or NULL.  May equal initial_state.  An empty
+ *                    sequence yields its initial state (or zeros).
+ * workspace          device scratch of at least gdr_prefill_workspace_size()
+ *                    bytes (NULL allowed when that size is 0).
+ */
+GDR_API gdr_status_t gdr_prefill_chunked(const void *q, const void *k, const void *v,
+                                 const float *g, const float *beta,
+                                 const float *initial_state, const int32_t *cu_seqlens,
+                                 int32_t num_seqs, int32_t total_T, int32_t H,
+                                 int32_t d_k, int32_t d_v, gdr_gate_mode_t gate_mode,
+                                 gdr_dtype_t io_dtype, void *o, float *final_state,
+                                 void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * After gdr_prefill_chunked's work on `stream` has finished, reports whether a
+ * bounded device-side wait in it gave up (GDR_ERR_DEVICE_TIMEOUT) or not
+ * (GDR_OK).  Synchronises `stream` and copies one word from `workspace`.
+ */
+GDR_API gdr_status_t gdr_prefill_check_workspace(const void *workspace, size_t workspace_bytes,
+                                         void *stream);
+
+/*
+ * One decode step: one new token for each of N sequences.
+ *
+ * q, k [N, H, d_k], v [N, H, d_v] (io dtype); g [N, H] or [N, H, d_k] fp32;
+ * beta [N, H] fp32; state [N, H, d_v, d_k] fp32, read and overwritten in place
+ * with S_t; o [N, H, d_v] (io dtype) receives o_t = S_t q_t.  The state makes
+ * one pass through HBM (one read, one write); the serving split that hands a
+ * prefill's final state to decode (page "How the New Flash Models Work",
+ * section "Serving: prefill and decode are different problems") is the
+ * caller passing final_state here.
+ */
+GDR_API gdr_status_t gdr_decode_step(const void *q, const void *k, const void *v,
+                             const float *g, const float *beta, float *state,
+                             int32_t N, int32_t H, int32_t d_k, int32_t d_v,
+                             gdr_gate_mode_t gate_mode, gdr_dtype_t io_dtype,
+                             void *o, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDR_H */

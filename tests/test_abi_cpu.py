@@ -1,0 +1,108 @@
+"""The C ABI library on a machine without a GPU: it loads, exports every
+symbol include/gdr.h declares, and rejects invalid arguments on the host
+before touching CUDA (no compute call is made here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from gated_delta_rule_151_b200 import gdr
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gdr.h")
+
+A = 0x7f0000000000          # a 16-byte aligned fake device address (never dereferenced)
+MIS = A + 4                 # misaligned
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"GDR_API\s+[\w\s\*]+?\b(gdr_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return gdr.load_library()
+
+
+def test_header_declares_the_binding_names():
+    assert declared_symbols() == sorted(gdr.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    raw = ctypes.CDLL(gdr.LIB_PATH)
+    for name in declared_symbols():
+        assert hasattr(raw, name), name
+
+
+def test_status_strings(lib):
+    for s in range(6):
+        assert gdr.gdr_status_string(s).startswith("GDR_")
+    assert "UNKNOWN" in gdr.gdr_status_string(99)
+
+
+def _prefill(lib, **kw):
+    args = dict(q=A, k=A, v=A, g=A, beta=A, h0=None, cu=None, N=1, T=64, H=2, dk=16, dv=16,
+                gate=0, io=0, o=A, fin=A, ws=None, wsb=0, stream=None)
+    args.update(kw)
+    P = lambda x: None if x is None else ctypes.c_void_p(x)
+    return lib.gdr_prefill_chunked(P(args["q"]), P(args["k"]), P(args["v"]), P(args["g"]),
+                                   P(args["beta"]), P(args["h0"]), P(args["cu"]), args["N"],
+                                   args["T"], args["H"], args["dk"], args["dv"], args["gate"],
+                                   args["io"], P(args["o"]), P(args["fin"]), P(args["ws"]),
+                                   args["wsb"], args["stream"])
+
+
+@pytest.mark.parametrize("kw", [
+    dict(q=None), dict(k=None), dict(v=None), dict(g=None), dict(beta=None), dict(o=None),
+    dict(q=MIS), dict(v=MIS), dict(o=MIS), dict(fin=MIS), dict(h0=MIS), dict(cu=MIS),
+    dict(dk=48), dict(dv=256), dict(dk=0), dict(H=0), dict(T=-1), dict(N=-1),
+    dict(N=3, T=64),              # 64 tokens do not split into 3 equal sequences
+    dict(N=0, T=64), dict(gate=2), dict(io=5),
+])
+def test_prefill_rejects_invalid_arguments(lib, kw):
+    assert _prefill(lib, **kw) == gdr.GDR_ERR_INVALID_ARG
+
+
+def test_prefill_empty_problem_is_a_no_op(lib):
+    assert _prefill(lib, N=0, T=0, q=None, k=None, v=None, g=None, beta=None, o=None) == gdr.GDR_OK
+
+
+def _decode(lib, **kw):
+    args = dict(q=A, k=A, v=A, g=A, beta=A, state=A, N=4, H=2, dk=128, dv=128, gate=0, io=1,
+                o=A, stream=None)
+    args.update(kw)
+    P = lambda x: None if x is None else ctypes.c_void_p(x)
+    return lib.gdr_decode_step(P(args["q"]), P(args["k"]), P(args["v"]), P(args["g"]),
+                               P(args["beta"]), P(args["state"]), args["N"], args["H"], args["dk"],
+                               args["dv"], args["gate"], args["io"], P(args["o"]), args["stream"])
+
+
+@pytest.mark.parametrize("kw", [
+    dict(q=None), dict(state=None), dict(o=None), dict(state=MIS), dict(k=MIS), dict(dk=100),
+    dict(dv=8), dict(N=-1), dict(H=-2), dict(gate=7), dict(io=3),
+])
+def test_decode_rejects_invalid_arguments(lib, kw):
+    assert _decode(lib, **kw) == gdr.GDR_ERR_INVALID_ARG
+
+
+def test_decode_empty_batch_is_a_no_op(lib):
+    assert _decode(lib, N=0) == gdr.GDR_OK
+
+
+def test_workspace_and_path_queries(lib):
+    assert gdr.gdr_prefill_workspace_size(1, 64, 2, 16, 16, 0, 0) == 0
+    assert gdr.gdr_prefill_path(16, 16, 0, gdr.GDR_F32) == gdr.GDR_PATH_SIMT
+    assert gdr.gdr_prefill_path(128, 128, 1, gdr.GDR_F32) == gdr.GDR_PATH_SIMT
+    with pytest.raises(gdr.GdrError):
+        gdr.gdr_prefill_path(12, 16, 0, 0)
+    with pytest.raises(gdr.GdrError):
+        gdr.gdr_prefill_workspace_size(-1, 64, 2, 16, 16, 0, 0)
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    x = torch.zeros(4, 2, 16)
+    with pytest.raises(ValueError):
+        gdr.gdr_prefill_chunked(x, x, x, torch.zeros(4, 2), torch.zeros(4, 2))

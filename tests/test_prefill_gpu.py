@@ -1,0 +1,196 @@
+"""Chunked prefill on the GPU against the fp64 oracle, element by element,
+at sizes that span several 64-token chunks and a ragged tail, plus the
+full-size workloads on sampled (sequence, head) pairs, the edge cases
+(empty and one-token sequences, g = -inf, in-place state) and memory-safety
+canaries (guard bands, NaN-poisoned outputs)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gated_delta_rule_151_b200 import gdr
+from gated_delta_rule_151_b200 import inputs as I
+from _util import check, gpu_prefill, oracle_prefill, to_device, TOL_BF16_O
+
+pytestmark = pytest.mark.gpu
+
+
+def test_tiny_workload_fp32():
+    inp = I.workload("tiny_gdn")
+    o, fin = gpu_prefill(inp)
+    o_ref, fin_ref = oracle_prefill(inp)
+    check(inp, o, fin, o_ref, fin_ref, "tiny_gdn")
+
+
+@pytest.mark.parametrize("T", [1, 63, 64, 65, 127, 129, 300])
+@pytest.mark.parametrize("mode", [I.SCALAR, I.CHANNEL])
+def test_ragged_lengths_bf16_d128(T, mode):
+    inp = I.make_inputs(total_T=T, H=3, d_k=128, gate_mode=mode, io_dtype=torch.bfloat16,
+                        c=0.1, h0_std=0.02, seed=T)
+    o, fin = gpu_prefill(inp)
+    o_ref, fin_ref = oracle_prefill(inp)
+    check(inp, o, fin, o_ref, fin_ref, f"T={T} {mode}")
+
+
+@pytest.mark.parametrize("dk,dv", [(16, 16), (32, 32), (64, 64), (16, 128), (128, 32), (64, 16)])
+@pytest.mark.parametrize("mode", [I.SCALAR, I.CHANNEL])
+@pytest.mark.parametrize("io", [torch.float32, torch.bfloat16])
+def test_head_dims(dk, dv, mode, io):
+    inp = I.make_inputs(total_T=130, H=2, d_k=dk, d_v=dv, gate_mode=mode, io_dtype=io, c=0.2,
+                        h0_std=0.05, seed=dk * 7 + dv)
+    o, fin = gpu_prefill(inp)
+    o_ref, fin_ref = oracle_prefill(inp)
+    check(inp, o, fin, o_ref, fin_ref, f"dk={dk} dv={dv} {mode} {io}")
+
+
+@pytest.mark.parametrize("mode", [I.SCALAR, I.CHANNEL])
+@pytest.mark.parametrize("d,io", [(128, torch.bfloat16), (32, torch.float32)])
+def test_varlen_with_empty_and_short_sequences(mode, d, io):
+    lens = [0, 5, 64, 0, 130, 1, 77]
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    inp = I.make_inputs(total_T=int(cu[-1]), H=2, d_k=d, cu_seqlens=cu, gate_mode=mode,
+                        io_dtype=io, c=0.1, h0_std=0.03, seed=3)
+    o, fin = gpu_prefill(inp)
+    o_ref, fin_ref = oracle_prefill(inp)
+    check(inp, o, fin, o_ref, fin_ref, "varlen")
+    # empty sequences hand back their initial state exactly
+    for n in (0, 3):
+        assert torch.equal(fin[n].cpu(), inp.h0[n])
+
+
+def test_equal_lengths_without_cu_seqlens():
+    inp = I.make_inputs(total_T=3 * 100, H=2, d_k=128, num_seqs=3, io_dtype=torch.bfloat16,
+                        h0_std=0.02, seed=8)
+    o1, f1 = gpu_prefill(inp, use_cu=True)
+    o2, f2 = gpu_prefill(inp, use_cu=False)
+    assert torch.equal(o1, o2) and torch.equal(f1, f2)
+
+
+def test_no_initial_state_means_zeros_and_no_final_state_is_allowed():
+    inp = I.make_inputs(total_T=200, H=2, d_k=64, io_dtype=torch.float32, seed=5)
+    d = to_device(inp)
+    o, fin = gdr.gdr_prefill_chunked(d["q"], d["k"], d["v"], d["g"], d["beta"], None, d["cu"])
+    o2, fin2 = gdr.gdr_prefill_chunked(d["q"], d["k"], d["v"], d["g"], d["beta"],
+                                       torch.zeros_like(fin), d["cu"])
+    o3, none = gdr.gdr_prefill_chunked(d["q"], d["k"], d["v"], d["g"], d["beta"], None, d["cu"],
+                                       output_final_state=False)
+    torch.cuda.synchronize()
+    assert none is None
+    assert torch.equal(o, o2) and torch.equal(fin, fin2) and torch.equal(o, o3)
+
+
+@pytest.mark.parametrize("d,io", [(128, torch.bfloat16), (16, torch.float32)])
+def test_in_place_state(d, io):
+    inp = I.make_inputs(total_T=150, H=2, d_k=d, num_seqs=1, io_dtype=io, h0_std=0.05, seed=6)
+    dv = to_device(inp)
+    o_sep, f_sep = gdr.gdr_prefill_chunked(dv["q"], dv["k"], dv["v"], dv["g"], dv["beta"],
+                                           dv["h0"], dv["cu"])
+    state = dv["h0"].clone()
+    o_in, f_in = gdr.gdr_prefill_chunked(dv["q"], dv["k"], dv["v"], dv["g"], dv["beta"], state,
+                                         dv["cu"], final_state=state)
+    torch.cuda.synchronize()
+    assert f_in.data_ptr() == state.data_ptr()
+    assert torch.equal(o_sep, o_in) and torch.equal(f_sep, state)
+
+
+@pytest.mark.parametrize("mode", [I.SCALAR, I.CHANNEL])
+def test_gate_minus_infinity(mode):
+    inp = I.make_inputs(total_T=140, H=2, d_k=128, gate_mode=mode, io_dtype=torch.bfloat16,
+                        h0_std=0.05, seed=9)
+    g = inp.g.clone()
+    g[::17] = -float("inf")       # hard resets inside and across chunks
+    inp.g = g
+    o, fin = gpu_prefill(inp)
+    o_ref, fin_ref = oracle_prefill(inp)
+    check(inp, o, fin, o_ref, fin_ref, "g=-inf")
+
+
+@pytest.mark.parametrize("mode", [I.SCALAR, I.CHANNEL])
+def test_guard_bands_and_poisoned_outputs(mode):
+    """Outputs live inside larger buffers whose margins hold a sentinel and
+    whose interior starts as NaN: every output element must be written and
+    nothing outside may change."""
+    inp = I.make_inputs(total_T=197, H=3, d_k=128, gate_mode=mode, io_dtype=torch.bfloat16,
+                        cu_seqlens=[0, 61, 61, 197], h0_std=0.02, seed=10)
+    d = to_device(inp)
+    T, H, D, N = inp.total_T, inp.H, 128, inp.num_seqs
+    pad = 4096
+    sentinel = 12345.0
+    obuf = torch.full((pad + T * H * D + pad,), sentinel, dtype=torch.bfloat16, device="cuda")
+    fbuf = torch.full((pad + N * H * D * D + pad,), sentinel, dtype=torch.float32, device="cuda")
+    o = obuf[pad:pad + T * H * D].view(T, H, D)
+    f = fbuf[pad:pad + N * H * D * D].view(N, H, D, D)
+    o.fill_(float("nan"))
+    f.fill_(float("nan"))
+    gdr.gdr_prefill_chunked(d["q"], d["k"], d["v"], d["g"], d["beta"], d["h0"], d["cu"], o=o,
+                            final_state=f)
+    torch.cuda.synchronize()
+    assert torch.all(obuf[:pad] == sentinel) and torch.all(obuf[-pad:] == sentinel)
+    assert torch.all(fbuf[:pad] == sentinel) and torch.all(fbuf[-pad:] == sentinel)
+    assert not torch.isnan(o.float()).any() and not torch.isnan(f).any()
+    o_ref, fin_ref = oracle_prefill(inp)
+    check(inp, o, f, o_ref, fin_ref, "guard")
+
+
+@pytest.mark.parametrize("mode", [I.SCALAR, I.CHANNEL])
+def test_split_prefill_with_state_handoff(mode):
+    inp = I.make_inputs(total_T=300, H=2, d_k=128, gate_mode=mode, io_dtype=torch.bfloat16,
+                        h0_std=0.02, seed=11)
+    d = to_device(inp)
+    o_full, f_full = gdr.gdr_prefill_chunked(d["q"], d["k"], d["v"], d["g"], d["beta"], d["h0"])
+    T1 = 131
+    oa, fa = gdr.gdr_prefill_chunked(d["q"][:T1].contiguous(), d["k"][:T1].contiguous(),
+                                     d["v"][:T1].contiguous(), d["g"][:T1].contiguous(),
+                                     d["beta"][:T1].contiguous(), d["h0"])
+    ob, fb = gdr.gdr_prefill_chunked(d["q"][T1:].contiguous(), d["k"][T1:].contiguous(),
+                                     d["v"][T1:].contiguous(), d["g"][T1:].contiguous(),
+                                     d["beta"][T1:].contiguous(), fa)
+    torch.cuda.synchronize()
+    o_ref, fin_ref = oracle_prefill(inp)
+    check(inp, torch.cat([oa, ob]), fb, o_ref, fin_ref, "split")
+    check(inp, o_full, f_full, o_ref, fin_ref, "full")
+
+
+def test_prefill_then_decode_handoff():
+    """Prefill the first tokens, hand the state to the decode step for the
+    rest: the same outputs as the oracle's single pass."""
+    T, T1 = 80, 70
+    inp = I.make_inputs(total_T=T, H=2, d_k=128, io_dtype=torch.bfloat16, gate_mode=I.CHANNEL,
+                        h0_std=0.02, seed=12)
+    d = to_device(inp)
+    oa, state = gdr.gdr_prefill_chunked(d["q"][:T1].contiguous(), d["k"][:T1].contiguous(),
+                                        d["v"][:T1].contiguous(), d["g"][:T1].contiguous(),
+                                        d["beta"][:T1].contiguous(), d["h0"])
+    outs = [oa]
+    for t in range(T1, T):
+        outs.append(gdr.gdr_decode_step(d["q"][t:t + 1], d["k"][t:t + 1], d["v"][t:t + 1],
+                                        d["g"][t:t + 1], d["beta"][t:t + 1], state))
+    torch.cuda.synchronize()
+    o_ref, fin_ref = oracle_prefill(inp)
+    check(inp, torch.cat(outs), state, o_ref, fin_ref, "prefill->decode")
+
+
+# ------------------------------------------------ full-size workloads ----
+
+def _sampled(name, heads, seqs=None):
+    inp = I.workload(name)
+    o, fin = gpu_prefill(inp)
+    o_ref, fin_ref = oracle_prefill(inp, heads=heads, seqs=seqs)
+    cu = inp.cu_seqlens.numpy()
+    seqs = list(range(inp.num_seqs)) if seqs is None else seqs
+    tok = np.concatenate([np.arange(cu[s], cu[s + 1]) for s in seqs])
+    o_sel = o[torch.from_numpy(tok).cuda()][:, heads]
+    f_sel = fin[seqs][:, heads]
+    return check(inp, o_sel, f_sel, o_ref, fin_ref, name)
+
+
+def test_full_size_gdn_prefill_sampled():
+    _sampled("gdn_prefill", heads=[0, 7, 15])
+
+
+def test_full_size_kda_prefill_sampled():
+    _sampled("kda_prefill", heads=[0, 31], seqs=[0, 1])
+
+
+def test_full_size_varlen_prefill_sampled():
+    _sampled("varlen_gdn", heads=[5])
