@@ -84,6 +84,9 @@ class ClockSampler:
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
+            t_end = time.time() + 5.0            # let the sampler come up first
+            while not self.lines and time.time() < t_end and self.proc.poll() is None:
+                time.sleep(0.05)
         except (OSError, FileNotFoundError):
             self.proc = None
         return self

@@ -17,6 +17,15 @@ bool ok_ptr(const void *p) { return p != nullptr && aligned16(p); }
 
 bool ok_opt_ptr(const void *p) { return p == nullptr || aligned16(p); }
 
+// beta and scalar-mode g are read one element at a time: 4-byte alignment.
+bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+bool ok_gate_ptr(const void *p, gdr_gate_mode_t mode) {
+    return p != nullptr && (mode == GDR_GATE_CHANNEL ? aligned16(p) : aligned4(p));
+}
+
+bool ok_beta_ptr(const void *p) { return p != nullptr && aligned4(p); }
+
 gdr_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? GDR_OK : GDR_ERR_CUDA; }
 
 bool uses_tcgen05(int32_t d_k, int32_t d_v, gdr_gate_mode_t gate_mode, gdr_dtype_t io_dtype) {
@@ -73,10 +82,10 @@ gdr_status_t gdr_prefill_chunked(const void *q, const void *k, const void *v, co
     if (num_seqs == 0 && total_T != 0) return GDR_ERR_INVALID_ARG;
     if (cu_seqlens == nullptr && num_seqs > 0 && total_T % num_seqs != 0) return GDR_ERR_INVALID_ARG;
     if (total_T > 0) {
-        if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(g) || !ok_ptr(beta) || !ok_ptr(o))
+        if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_gate_ptr(g, gate_mode) ||
+            !ok_beta_ptr(beta) || !ok_ptr(o))
             return GDR_ERR_INVALID_ARG;
-    } else if (!ok_opt_ptr(q) || !ok_opt_ptr(k) || !ok_opt_ptr(v) || !ok_opt_ptr(g) ||
-               !ok_opt_ptr(beta) || !ok_opt_ptr(o)) {
+    } else if (!ok_opt_ptr(q) || !ok_opt_ptr(k) || !ok_opt_ptr(v) || !ok_opt_ptr(o)) {
         return GDR_ERR_INVALID_ARG;
     }
     if (!ok_opt_ptr(initial_state) || !ok_opt_ptr(final_state) || !ok_opt_ptr(cu_seqlens))
@@ -126,8 +135,8 @@ gdr_status_t gdr_decode_step(const void *q, const void *k, const void *v, const 
     if (io_dtype != GDR_F32 && io_dtype != GDR_BF16) return GDR_ERR_INVALID_ARG;
     if ((int64_t)N * H > (int64_t)INT32_MAX) return GDR_ERR_INVALID_ARG;
     if ((int64_t)N * H == 0) return GDR_OK;
-    if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(g) || !ok_ptr(beta) || !ok_ptr(state) ||
-        !ok_ptr(o))
+    if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_gate_ptr(g, gate_mode) ||
+        !ok_beta_ptr(beta) || !ok_ptr(state) || !ok_ptr(o))
         return GDR_ERR_INVALID_ARG;
     return from_cuda(gdr::launch_decode_step(q, k, v, g, beta, state, N, H, d_k, d_v,
                                              gate_mode == GDR_GATE_CHANNEL,

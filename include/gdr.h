@@ -31,8 +31,9 @@
  *              [T, H, d_k]        fp32 (channel gate)
  *     beta     [T, H]             fp32
  *     state    [N, H, d_v, d_k]   fp32
- * - d_k and d_v are each one of 16, 32, 64, 128.  Every pointer must be
- *   16-byte aligned.
+ * - d_k and d_v are each one of 16, 32, 64, 128.  q, k, v, o, the states and
+ *   channel-mode g must be 16-byte aligned; beta and scalar-mode g need
+ *   4-byte alignment.
  * - All pointers are DEVICE pointers owned by the caller.  The library
  *   allocates nothing, keeps no global state beyond cached kernel
  *   attributes, and never synchronises the device: work is enqueued on

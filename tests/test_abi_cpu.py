@@ -57,12 +57,20 @@ def _prefill(lib, **kw):
 @pytest.mark.parametrize("kw", [
     dict(q=None), dict(k=None), dict(v=None), dict(g=None), dict(beta=None), dict(o=None),
     dict(q=MIS), dict(v=MIS), dict(o=MIS), dict(fin=MIS), dict(h0=MIS), dict(cu=MIS),
+    dict(beta=A + 2), dict(g=A + 2), dict(g=A + 4, gate=1),
     dict(dk=48), dict(dv=256), dict(dk=0), dict(H=0), dict(T=-1), dict(N=-1),
     dict(N=3, T=64),              # 64 tokens do not split into 3 equal sequences
     dict(N=0, T=64), dict(gate=2), dict(io=5),
 ])
 def test_prefill_rejects_invalid_arguments(lib, kw):
     assert _prefill(lib, **kw) == gdr.GDR_ERR_INVALID_ARG
+
+
+def test_scalar_gate_and_beta_need_only_element_alignment(lib):
+    # a valid request would launch a kernel, so only the validation outcome is
+    # observed: anything but INVALID_ARG means the pointers were accepted
+    assert _prefill(lib, N=0, T=0, beta=A + 4, g=A + 4, q=None, k=None, v=None,
+                    o=None) == gdr.GDR_OK
 
 
 def test_prefill_empty_problem_is_a_no_op(lib):
@@ -81,6 +89,7 @@ def _decode(lib, **kw):
 
 @pytest.mark.parametrize("kw", [
     dict(q=None), dict(state=None), dict(o=None), dict(state=MIS), dict(k=MIS), dict(dk=100),
+    dict(beta=A + 1), dict(g=A + 8, gate=1),
     dict(dv=8), dict(N=-1), dict(H=-2), dict(gate=7), dict(io=3),
 ])
 def test_decode_rejects_invalid_arguments(lib, kw):
