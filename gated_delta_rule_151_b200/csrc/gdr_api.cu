@@ -29,8 +29,8 @@ bool ok_beta_ptr(const void *p) { return p != nullptr && aligned4(p); }
 gdr_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? GDR_OK : GDR_ERR_CUDA; }
 
 bool uses_tcgen05(int32_t d_k, int32_t d_v, gdr_gate_mode_t gate_mode, gdr_dtype_t io_dtype) {
-    (void)gate_mode;
-    return gdr::tcgen05_prefill_available() && io_dtype == GDR_BF16 && d_k == 128 && d_v == 128;
+    return gdr::tcgen05_prefill_available() && io_dtype == GDR_BF16 && d_k == 128 &&
+           d_v == 128 && gdr::tcgen05_prefill_serves(gate_mode == GDR_GATE_CHANNEL);
 }
 
 }  // namespace

@@ -20,6 +20,7 @@ size_t prefill_simt_smem_bytes(int DK, int DV);
 
 // tcgen05 prefill: bf16 I/O, d_k = d_v = 128.
 bool tcgen05_prefill_available();
+bool tcgen05_prefill_serves(bool channel);
 size_t tcgen05_workspace_bytes(int num_seqs, int total_T, int H);
 cudaError_t launch_prefill_tcgen05(const void *q, const void *k, const void *v, const float *g,
                                    const float *beta, const float *h0, const int32_t *cu,

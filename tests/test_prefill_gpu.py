@@ -194,3 +194,20 @@ def test_full_size_kda_prefill_sampled():
 
 def test_full_size_varlen_prefill_sampled():
     _sampled("varlen_gdn", heads=[5])
+
+
+def test_tensor_core_path_is_used_and_reports_no_timeout():
+    """bf16, d = 128, scalar gate runs on the tcgen05 kernel; its workspace
+    word (set by a bounded wait that gives up) stays clear."""
+    assert gdr.gdr_prefill_path(128, 128, gdr.GDR_GATE_SCALAR, gdr.GDR_BF16) == gdr.GDR_PATH_TCGEN05
+    inp = I.make_inputs(total_T=333, H=4, d_k=128, num_seqs=3, cu_seqlens=[0, 100, 101, 333],
+                        io_dtype=torch.bfloat16, h0_std=0.02, seed=13)
+    d = to_device(inp)
+    nb = gdr.gdr_prefill_workspace_size(3, 333, 4, 128, 128, gdr.GDR_GATE_SCALAR, gdr.GDR_BF16)
+    assert nb >= 4
+    ws = torch.full((nb,), 0xFF, dtype=torch.uint8, device="cuda")
+    o, fin = gdr.gdr_prefill_chunked(d["q"], d["k"], d["v"], d["g"], d["beta"], d["h0"], d["cu"],
+                                     workspace=ws)
+    gdr.gdr_prefill_check_workspace(ws)
+    o_ref, fin_ref = oracle_prefill(inp)
+    check(inp, o, fin, o_ref, fin_ref, "tcgen05")
