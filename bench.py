@@ -292,13 +292,23 @@ def timed_steps(fn, K, flush, stream):
     return [a.elapsed_time(b) for a, b in times]
 
 
-def max_over_ranks(x, ws):
+def max_over_ranks(x, ws, device="cuda"):
+    """Max of a per-rank scalar over all ranks (timing only; no data-path
+    collective exists)."""
     if ws == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def aggregate_throughput(tokens_per_rank, ms_local, ws, device="cuda"):
+    """Weak scaling: every rank processes its own batch of `tokens_per_rank`
+    tokens; the job's throughput is all ranks' tokens over the slowest rank's
+    time.  Returns (tokens/s, max ms)."""
+    ms = max_over_ranks(ms_local, ws, device)
+    return tokens_per_rank * ws / (ms / 1e3), ms
 
 
 def barrier(ws):
@@ -339,9 +349,8 @@ def bench_case(case, args, ws, rank, flush, stream, pk, pk_kind):
         with ClockSampler(torch.cuda.current_device()) as clk:
             times = timed_steps(lambda: case.step(stream), args.steps, flush, stream)
         barrier(ws)
-    ms = max_over_ranks(sum(times) / len(times), ws)
+    value, ms = aggregate_throughput(case.tokens, sum(times) / len(times), ws)
     tokens_all = case.tokens * ws
-    value = tokens_all / (ms / 1e3)
     launch_ms = ms / case.launches
     achieved = case.bytes / (launch_ms / 1e3) / 1e9
     hbm_peak = float(pk["hbm_gbs"])
