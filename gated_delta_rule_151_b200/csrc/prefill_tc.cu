@@ -39,7 +39,10 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <mutex>
+
 #include "common.cuh"
+#include "gdr.h"
 #include "internal.h"
 #include "tc_ptx.cuh"
 
@@ -596,3 +599,64 @@ cudaError_t launch_prefill_tcgen05(const void *q, const void *k, const void *v, 
 }
 
 }  // namespace gdr
+
+// ----------------------------------------------- allocation-free variant ----
+//
+// Some callers cannot hand the library a workspace: they run where calling
+// cudaMalloc is not allowed or not acceptable (inside a host framework that
+// owns every device allocation through its own pool, in a latency-critical
+// loop where an allocation would synchronise the device, or in plugin code
+// with no allocator of its own).  For them the prefill's scratch -- the
+// error word the tensor-core kernel's bounded waits write -- lives in the
+// fixed-size device array below, which every GPU that loads this library
+// holds until the process exits.
+
+namespace gdr {
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = 256;
+constexpr int kNoAllocMaxDevices = 64;
+
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mutex;
+void *g_noalloc_addr[kNoAllocMaxDevices] = {};
+
+// Device address of the scratch array on the current device, looked up once
+// per device (host code only sees a stand-in symbol for the array).
+cudaError_t noalloc_scratch_address(void **out) {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kNoAllocMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (g_noalloc_addr[dev] == nullptr) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return e;
+        g_noalloc_addr[dev] = p;
+    }
+    *out = g_noalloc_addr[dev];
+    return cudaSuccess;
+}
+
+}  // namespace
+}  // namespace gdr
+
+extern "C" gdr_status_t gdr_prefill_chunked_noalloc(
+    const void *q, const void *k, const void *v, const float *g, const float *beta,
+    const float *initial_state, const int32_t *cu_seqlens, int32_t num_seqs, int32_t total_T,
+    int32_t H, int32_t d_k, int32_t d_v, gdr_gate_mode_t gate_mode, gdr_dtype_t io_dtype, void *o,
+    float *final_state, void *stream) {
+    size_t need = 0;
+    gdr_status_t st = gdr_prefill_workspace_size(num_seqs, total_T, H, d_k, d_v, gate_mode,
+                                                 io_dtype, &need);
+    if (st != GDR_OK) return st;
+    if (need > gdr::kNoAllocScratchBytes) return GDR_ERR_WORKSPACE;
+    void *scratch = nullptr;
+    if (gdr::noalloc_scratch_address(&scratch) != cudaSuccess) return GDR_ERR_CUDA;
+    return gdr_prefill_chunked(q, k, v, g, beta, initial_state, cu_seqlens, num_seqs, total_T, H,
+                               d_k, d_v, gate_mode, io_dtype, o, final_state, scratch,
+                               gdr::kNoAllocScratchBytes, stream);
+}
+

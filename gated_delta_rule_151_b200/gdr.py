@@ -33,7 +33,8 @@ GDR_PATH_TCGEN05 = 1
 
 # Every symbol include/gdr.h declares.
 EXPORTED = ("gdr_status_string", "gdr_prefill_workspace_size", "gdr_prefill_path",
-            "gdr_prefill_chunked", "gdr_prefill_check_workspace", "gdr_decode_step")
+            "gdr_prefill_chunked", "gdr_prefill_check_workspace", "gdr_decode_step",
+            "gdr_prefill_chunked_noalloc")
 
 
 class GdrError(RuntimeError):
@@ -72,6 +73,9 @@ def load_library():
         lib.gdr_prefill_check_workspace.restype = ST
         lib.gdr_decode_step.argtypes = [P, P, P, P, P, P, I32, I32, I32, I32, ST, ST, P, P]
         lib.gdr_decode_step.restype = ST
+        lib.gdr_prefill_chunked_noalloc.argtypes = [P, P, P, P, P, P, P, I32, I32, I32, I32, I32,
+                                                    ST, ST, P, P, P]
+        lib.gdr_prefill_chunked_noalloc.restype = ST
         _lib = lib
         return lib
 
@@ -219,3 +223,34 @@ def gdr_decode_step(q, k, v, g, beta, state, *, o=None, stream=None):
                                         _stream_ptr(stream))
     _check(st, "gdr_decode_step")
     return o
+
+
+def gdr_prefill_chunked_noalloc(q, k, v, g, beta, initial_state=None, cu_seqlens=None, *,
+                                num_seqs=None, o=None, final_state=None, stream=None):
+    """gdr_prefill_chunked without a workspace: the library's own fixed device
+    scratch is used instead (see include/gdr.h for who needs this and the
+    rules that come with it).  ``o`` and ``final_state`` must be given."""
+    _need(q, "q", ndim=3)
+    io = q.dtype
+    _need(k, "k", io, 3)
+    _need(v, "v", io, 3)
+    _need(beta, "beta", torch.float32, 2)
+    _need(g, "g", torch.float32)
+    _need(o, "o", io, 3)
+    T, H, dk = q.shape
+    dv = v.shape[2]
+    gate = GDR_GATE_SCALAR if g.dim() == 2 else GDR_GATE_CHANNEL
+    if cu_seqlens is not None:
+        _need(cu_seqlens, "cu_seqlens", torch.int32, 1)
+        N = cu_seqlens.numel() - 1
+    else:
+        N = 1 if num_seqs is None else int(num_seqs)
+    if initial_state is not None:
+        _need(initial_state, "initial_state", torch.float32, 4)
+    if final_state is not None:
+        _need(final_state, "final_state", torch.float32, 4)
+    st = load_library().gdr_prefill_chunked_noalloc(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(initial_state), _ptr(cu_seqlens),
+        N, T, H, dk, dv, gate, _io_code(io), _ptr(o), _ptr(final_state), _stream_ptr(stream))
+    _check(st, "gdr_prefill_chunked_noalloc")
+    return o, final_state

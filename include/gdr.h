@@ -147,6 +147,35 @@ GDR_API gdr_status_t gdr_prefill_check_workspace(const void *workspace, size_t w
                                          void *stream);
 
 /*
+ * gdr_prefill_chunked for callers that cannot allocate device memory.
+ *
+ * Same arguments, layouts, results and errors as gdr_prefill_chunked, minus
+ * the workspace.  The published method has no counterpart to this entry
+ * point: it exists for callers that may not call cudaMalloc -- code whose
+ * device memory is all owned by a host framework's pool, latency-critical
+ * loops where an allocation would synchronise the device, plugins with no
+ * allocator of their own.  Instead of a caller-provided workspace, the
+ * scratch the prefill needs lives in a fixed 256-byte device array inside
+ * libgdr, present on every GPU that loads the library until the process
+ * exits.  A problem whose gdr_prefill_workspace_size() exceeds 256 bytes is
+ * rejected with GDR_ERR_WORKSPACE (this build needs 16 bytes or none).
+ *
+ * The first call on each device looks up the array's device address with
+ * that device current (a one-time set-up); make that first call before any
+ * stream capture on the device.  All calls share the one array and clear
+ * what must start at zero themselves, so calls whose GPU work overlaps (on
+ * different streams or devices sharing nothing else) race on it: serialise
+ * them.  Calls no cudaMalloc, cudaFree or allocating library routine.
+ */
+GDR_API gdr_status_t gdr_prefill_chunked_noalloc(const void *q, const void *k, const void *v,
+                                         const float *g, const float *beta,
+                                         const float *initial_state, const int32_t *cu_seqlens,
+                                         int32_t num_seqs, int32_t total_T, int32_t H,
+                                         int32_t d_k, int32_t d_v, gdr_gate_mode_t gate_mode,
+                                         gdr_dtype_t io_dtype, void *o, float *final_state,
+                                         void *stream);
+
+/*
  * One decode step: one new token for each of N sequences.
  *
  * q, k [N, H, d_k], v [N, H, d_v] (io dtype); g [N, H] or [N, H, d_k] fp32;
