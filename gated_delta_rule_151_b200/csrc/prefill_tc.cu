@@ -1,44 +1,62 @@
 // Chunked prefill of the gated delta rule on the sm_100a tensor cores
 // (tcgen05 MMA with TMEM accumulators, operands staged by TMA), bf16 I/O,
-// d_k = d_v = 128, scalar gate (Gated DeltaNet).
+// d_k = d_v = 128, scalar gate (Gated DeltaNet) or per-key-channel gate
+// (Kimi Delta Attention).
 //
 // The algebra is the exact chunk rearrangement of the recurrence on the page
 // "How the New Flash Models Work: Inside GLM-5.3-Flash and Qwen3.8-Flash-Next"
 // (section "Linear attention: a fixed-size memory in place of the cache",
-// Gated DeltaNet equation).  For a chunk of C = 64 tokens entering with state
-// S (d_v x d_k), within-chunk cumulative log-gate G_i and γ_i = exp(G_i):
+// Gated DeltaNet and Kimi Delta Attention equations).  For a chunk of C = 64
+// tokens entering with state S (d_v x d_k), within-chunk cumulative log-gate
+// G_i (a scalar, or one value per key channel) and Γ_i = exp(G_i):
 //
-//   A  = strictly-lower( diag(β) (K K^T) ⊙ exp(G_i - G_j) ),  T = (I + A)^-1
-//   W  = T diag(βγ) K,   Ũ = T diag(β) V
-//   U  = Ũ - W S^T                                  (corrected values)
-//   O  = diag(γ) Q S^T + (P ⊙ causal) U,  P_ij = exp(G_i - G_j) q_i . k_j
-//   S' = γ_C S + U^T K̂,   K̂_j = exp(G_C - G_j) k_j
+//   A_ij = β_i k_i^T Diag(exp(G_i - G_j)) k_j  (j < i),   T = (I + A)^-1
+//   W    = T diag(β) (K ⊙ Γ),   Ũ = T diag(β) V
+//   U    = Ũ - W S^T                                (corrected values)
+//   O    = (Q ⊙ Γ) S^T + (P ⊙ causal) U,  P_ij = q_i^T Diag(exp(G_i - G_j)) k_j
+//   S'   = S Diag(Γ_C) + U^T K̂,   K̂_j = k_j ⊙ exp(G_C - G_j)
 //
-// Every exponent is <= 0.  The MMAs are written transposed so that the
-// 128-wide d_v / d_k dimension is the M = 128 dimension (TMEM lane = row):
+// Every exponent in these formulas is <= 0.  The MMAs are written transposed
+// so that the 128-wide d_v / d_k dimension is the M = 128 dimension (TMEM
+// lane = matrix row):
 //
-//   P1  [K;Q] K^T      bf16  M=128 N=64  K=128  -> K K^T (lanes 0-63), Q K^T (64-127)
-//   P2  W^T = K'^T T^T tf32  M=128 N=64  K=64   (K' = diag(βγ) K)
-//       Ũ^T = V'^T T^T tf32  M=128 N=64  K=64   (V' = diag(β) V), into the U accumulator
-//   S1  U^T += S (-W)^T      A = S from TMEM, M=128 N=64 K=128
-//   S1' O^T  = S Q̃^T         A = S from TMEM (Q̃ = diag(γ) Q)
-//   S3  ΔS   = U^T K̂         A = U from TMEM, M=128 N=128 K=64
-//   S2  O^T += U^T (P⊙causal)^T
+//   P1  [K;Q] K^T  M=128 N=64  -> rows 0-63 give A (with β and decay),
+//                                 rows 64-127 give P
+//   P2  W^T = K'^T T^T, Ũ^T = V'^T T^T           (tf32)
+//   S1  U^T += S (-W)^T       S1'  O^T = S Q̃^T    (tf32, A = S from TMEM)
+//   S3  ΔS = U^T K̂            S2   O^T += U^T P^T (tf32, A = U from TMEM)
 //
-// The fp32 master state lives in registers (thread = row of S, 64 columns);
-// a tf32-rounded copy in TMEM is the A operand of S1/S1'.  Operands that feed
-// the state update are tf32 (round-to-nearest) to keep the state within its
-// error budget over thousands of chunks; Q K^T and K K^T use the exact bf16
-// inputs.  CUDA cores apply the gates, build the operands in the 128-byte
-// swizzled layout, and invert I + A (blocked 16 x 16 forward substitution).
+// Gated DeltaNet runs P1 on the exact bf16 inputs and applies the scalar
+// decays afterwards in fp32.  Kimi Delta Attention folds the per-channel
+// decays into the operands around a mid-chunk reference R (token 31):
+// [K ⊙ e^{G-R}; Q ⊙ e^{G-R}] (K ⊙ e^{R-G})^T, in fp16 (11-bit significand,
+// as precise as tf32 at half the footprint).  A chunk whose scaled operands
+// would leave fp16's range instead computes A and P exactly on CUDA cores.
 //
-// One CTA (8 warps) per (sequence, head).  Rows past a sequence's end get
-// β = 0 and g = 0, which makes their A rows, u and gate increments vanish.
-// Every mbarrier wait is bounded; on timeout the CTA records an error bit in
-// the workspace word and stops.
+// Operands that feed the state are tf32, rounded to nearest: bf16 would put
+// ~2^-9 relative error into every chunk's update.  The fp32 master state
+// lives in registers (thread = row of S, 64 columns); a tf32 copy in TMEM is
+// the A operand of S1/S1'.
+//
+// One CTA of 16 warps per (sequence, head), split into two groups that run
+// one chunk apart:
+//   * the chain group (warps 0-7) owns the state and runs only the
+//     state-dependent steps S1/S1', the rounding of U, S3/S2, the state
+//     update and the output store;
+//   * the prep group (warps 8-15) runs every chunk-local step for the next
+//     chunk: TMA loads, gates, P1, A and P, the 64 x 64 unit-triangular
+//     inverse (blocked 16 x 16 forward substitution), the tf32 operands, P2
+//     and -W.
+// They hand off through mbarriers; Ũ (TMEM) and P (shared memory) are
+// double-buffered so the prep of chunk c+1 overlaps the chain of chunk c.
+// Rows past a sequence's end get β = 0 and g = 0, which makes their A rows,
+// u and gate increments vanish.  Every mbarrier wait is bounded; on timeout
+// the CTA records an error bit in the workspace word and stops.
 #include <cuda.h>
 #include <cudaTypedefs.h>
+#include <cuda_fp16.h>
 
+#include <cstddef>
 #include <mutex>
 
 #include "common.cuh"
@@ -53,44 +71,53 @@ using namespace tc;
 
 constexpr int C = 64;
 constexpr int D = 128;
-constexpr int kThreads = 256;
+constexpr int kThreads = 512;
 
-// Shared-memory map (byte offsets from a 1024-aligned base).
-constexpr uint32_t OFF_KQ = 0;            // [K dk0-63][Q dk0-63][K dk64-127][Q dk64-127], bf16 8 KiB each
-constexpr uint32_t OFF_V = 32768;         // [V dv0-63][V dv64-127]
-constexpr uint32_t OFF_X1 = 49152;        // K'^T [dk][tok] tf32, then -W [tok][dk]
-constexpr uint32_t OFF_X2 = 81920;        // V'^T [dv][tok] tf32
-constexpr uint32_t OFF_KH = 114688;       // K̂^T [dk][tok] tf32 (A in fp32 before that)
-constexpr uint32_t OFF_QT = 147456;       // Q̃ [tok][dk] tf32 (T in fp32 before that)
-constexpr uint32_t OFF_PM = 180224;       // P [i][j] tf32
-constexpr uint32_t OFF_TM = 196608;       // T [i][j] tf32
-constexpr uint32_t OFF_MISC = 212992;
-constexpr uint32_t SMEM_BYTES = OFF_MISC + 2048 + 1024;  // + misc + alignment slack
-
-constexpr int AF_LD = 65;                 // padded row stride of the fp32 scratch matrices
+// Shared-memory map (byte offsets from the 1024-aligned dynamic base).
+constexpr uint32_t OFF_KQ = 0;        // bf16 tiles [K d0-63][Q d0-63][K d64-127][Q d64-127], 8 KiB each
+constexpr uint32_t OFF_V = 32768;     // bf16 tiles [V d0-63][V d64-127]
+constexpr uint32_t OFF_X1 = 49152;    // K'^T [dk][tok] tf32, then -W [tok][dk] tf32
+constexpr uint32_t OFF_X2 = 81920;    // scratch (A, T fp32 / KDA fp16 P1 operand / G), then V'^T
+constexpr uint32_t OFF_KH = 114688;   // K̂^T [dk][tok] tf32
+constexpr uint32_t OFF_QT = 147456;   // Q̃ [tok][dk] tf32
+constexpr uint32_t OFF_PM = 180224;   // P [i][j] tf32, two slots of 16 KiB
+constexpr uint32_t OFF_TM = 212992;   // T [i][j] tf32 (scratch before that)
+constexpr uint32_t OFF_MISC = 229376;
+constexpr uint32_t SMEM_BYTES = OFF_MISC + 3072;   // 232448: the per-block maximum
 
 // TMEM columns.
-constexpr uint32_t TM_P1 = 0, TM_W = 64, TM_U = 128, TM_O = 192, TM_DS = 256, TM_S = 384;
+constexpr uint32_t TM_P1W = 0, TM_U0 = 64, TM_O = 192, TM_DS = 256, TM_S = 384;
 constexpr uint32_t TMEM_COLS = 512;
 
-constexpr uint32_t IDESC_P1 = make_idesc(1, 128, 64);    // bf16
-constexpr uint32_t IDESC_N64 = make_idesc(2, 128, 64);   // tf32
-constexpr uint32_t IDESC_N128 = make_idesc(2, 128, 128); // tf32
+constexpr uint32_t IDESC_BF16 = make_idesc(1, 128, 64);
+constexpr uint32_t IDESC_F16 = make_idesc(0, 128, 64);
+constexpr uint32_t IDESC_N64 = make_idesc(2, 128, 64);
+constexpr uint32_t IDESC_N128 = make_idesc(2, 128, 128);
 
-constexpr uint32_t ERR_TIMEOUT_TMA = 1u, ERR_TIMEOUT_MMA = 2u;
+constexpr uint32_t ERR_TIMEOUT_TMA = 1u, ERR_TIMEOUT_MMA = 2u, ERR_TIMEOUT_HANDOFF = 4u,
+                   ERR_SMEM_ALIGN = 8u;
+
+constexpr float kF16Limit = 60000.f;   // largest magnitude let into an fp16 operand
 
 struct Misc {
-    uint64_t bar_tma;
-    uint64_t bar_mma;
+    uint64_t bar_tma, bar_p, bar_ready, bar_s1, bar_s3;
     uint32_t tmem_base;
     int abort_flag;
-    float G[C];      // cumulative log-gate
-    float beta[C];
-    float gam[C];    // exp(G_i)
-    float kp[C];     // beta_i * exp(G_i)
-    float kh[C];     // exp(G_C - G_i)
-    float gC;        // exp(G_C)
+    int slow;
+    int wide;                          // Gated DeltaNet: chunk decay beyond e^-80
+    union alignas(16) {
+        struct {                       // Gated DeltaNet, per chunk (prep only)
+            float beta[C], G[C], gam[C], kp[C], kh[C], ieg[C];
+        } s;
+        struct {                       // Kimi Delta Attention, per chunk (prep only)
+            float beta[C], T0[D], T1[D];
+        } c;
+    } u;                               // beta comes first in both layouts
+    alignas(16) float gcb[2][D];       // exp(G_C) handed to the chain, per chunk slot
 };
+static_assert(sizeof(Misc) <= 3072, "misc area overflow");
+// float4 reads of the per-token arrays need 16-byte alignment
+static_assert(offsetof(Misc, u) % 16 == 0 && (C * 4) % 16 == 0, "misc arrays misaligned");
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
                                              uint32_t d) {
@@ -98,17 +125,23 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
                  "r"(d)
                  : "memory");
 }
-
 __device__ __forceinline__ void st_shared_b32(uint32_t addr, uint32_t a) {
     asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(a) : "memory");
 }
-
+__device__ __forceinline__ void st_shared_b16(uint32_t addr, uint16_t a) {
+    asm volatile("st.shared.b16 [%0], %1;" ::"r"(addr), "h"(a) : "memory");
+}
 __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
     uint4 v;
     asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
                  : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                  : "r"(addr));
     return v;
+}
+__device__ __forceinline__ float ld_shared_bf16(uint32_t addr) {
+    uint16_t v;
+    asm volatile("ld.shared.b16 %0, [%1];" : "=h"(v) : "r"(addr));
+    return __uint_as_float(static_cast<uint32_t>(v) << 16);
 }
 
 __device__ __forceinline__ void bf16x8_to_f32(const uint4 &v, float (&f)[8]) {
@@ -120,48 +153,176 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4 &v, float (&f)[8]) {
     }
 }
 
-// Wait on an mbarrier phase; every thread takes part so that all agree on
-// whether to stop.  Returns false when the CTA must stop.
-__device__ __forceinline__ bool cta_wait(uint64_t *bar, uint32_t phase, Misc *m, uint32_t *err,
-                                         uint32_t code) {
+// Named barrier over one 256-thread warp group (ids 1 and 2; 0 is __syncthreads).
+__device__ __forceinline__ void group_sync(int id) {
+    asm volatile("bar.sync %0, 256;" ::"r"(id) : "memory");
+}
+
+// Element (i, j) of a 64 x 64 fp32 scratch matrix: rows of 64 floats whose
+// 16-byte chunks are XOR-swizzled by the row, so float4 accesses by eight
+// threads on eight different rows hit eight different bank groups.
+__device__ __forceinline__ int ax(int i, int j) {
+    return i * 64 + ((((j >> 2) ^ (i & 15))) << 2) + (j & 3);
+}
+__device__ __forceinline__ float4 ld4(const float *base, int i, int j) {
+    return *reinterpret_cast<const float4 *>(base + ax(i, j));
+}
+__device__ __forceinline__ void st4(float *base, int i, int j, float4 v) {
+    *reinterpret_cast<float4 *>(base + ax(i, j)) = v;
+}
+
+// Bounded wait inside one group; all threads of the group agree on stopping.
+__device__ __forceinline__ bool group_wait(uint64_t *bar, uint32_t phase, Misc *m, uint32_t *err,
+                                           uint32_t code, int gid) {
     const bool ok = mbar_wait(bar, phase);
     if (!ok) {
         m->abort_flag = 1;
         atomicOr(err, code);
     }
-    __syncthreads();
+    group_sync(gid);
     return m->abort_flag == 0;
 }
 
+// acc[0..3] += sum_{s<16} X[xi][xj + s] * Y[yi + s][yj .. yj+3] for 16 x 16
+// blocks of the swizzled scratch (Y may also be a plain 16 x 16 block).
+template <bool Y_PLAIN>
+__device__ __forceinline__ void block_row_times(float (&acc)[4], const float *X, int xi, int xj,
+                                                const float *Y, int yi, int yj) {
+#pragma unroll
+    for (int s4 = 0; s4 < 16; s4 += 4) {
+        const float4 a = ld4(X, xi, xj + s4);
+        const float av[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float4 t = Y_PLAIN ? *reinterpret_cast<const float4 *>(Y + (s4 + e) * 16 + yj)
+                                     : ld4(Y, yi + s4 + e, yj);
+            acc[0] = fmaf(av[e], t.x, acc[0]);
+            acc[1] = fmaf(av[e], t.y, acc[1]);
+            acc[2] = fmaf(av[e], t.z, acc[2]);
+            acc[3] = fmaf(av[e], t.w, acc[3]);
+        }
+    }
+}
+
+// T = (I + A)^-1 for the strictly lower 64 x 64 A (fp32 scratch), recursively
+// on halves: with A = [[A_a, 0], [A_ba, A_b]] (32 x 32 blocks),
+//   T = [[T_a, 0], [-T_b A_ba T_a, T_b]],
+// and the same on each 32 x 32 half down to 16 x 16 diagonal blocks, which
+// are inverted by forward substitution (one thread per column).  Four
+// dependent matrix steps after the diagonal blocks; writes T as the tf32
+// operand [i][j] (128-byte swizzled rows, zero above the diagonal).
+// Xs: 4 KiB plain scratch (four 16 x 16 blocks).
+__device__ __forceinline__ void unit_lower_inverse(const float *Af, float *Tf, float *Xs,
+                                                   uint32_t tm_addr, int p) {
+    // diagonal 16 x 16 blocks, column c of block `blk`
+    if (p < 64) {
+        const int blk = p >> 4, c = p & 15, o = blk * 16;
+        float x[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+            float a[16];
+#pragma unroll
+            for (int s4 = 0; s4 < 16; s4 += 4) {
+                if (s4 < r) {
+                    const float4 v = ld4(Af, o + r, o + s4);
+                    a[s4] = v.x; a[s4 + 1] = v.y; a[s4 + 2] = v.z; a[s4 + 3] = v.w;
+                }
+            }
+            float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll
+            for (int s = 0; s < r; ++s) {
+                if (s & 1) acc1 = fmaf(a[s], x[s], acc1);
+                else acc0 = fmaf(a[s], x[s], acc0);
+            }
+            const float v = -(acc0 + acc1);
+            x[r] = (r < c) ? 0.f : ((r == c) ? 1.f : v);
+        }
+#pragma unroll
+        for (int r = 0; r < 16; ++r) Tf[ax(o + r, o + c)] = x[r];
+    }
+    group_sync(2);
+    const int r = (p >> 2) & 15, cq = (p & 3) * 4;
+    // T_10 = -T_11 A_10 T_00 and T_32 = -T_33 A_32 T_22
+    if (p < 128) {
+        const int I = (p >> 6) ? 3 : 1, J = I - 1;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        block_row_times<false>(acc, Af, 16 * I + r, 16 * J, Tf, 16 * J, 16 * J + cq);
+        *reinterpret_cast<float4 *>(Xs + (p >> 6) * 256 + r * 16 + cq) =
+            make_float4(acc[0], acc[1], acc[2], acc[3]);
+    }
+    group_sync(2);
+    if (p < 128) {
+        const int I = (p >> 6) ? 3 : 1, J = I - 1;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        block_row_times<true>(acc, Tf, 16 * I + r, 16 * I, Xs + (p >> 6) * 256, 0, cq);
+        st4(Tf, 16 * I + r, 16 * J + cq, make_float4(-acc[0], -acc[1], -acc[2], -acc[3]));
+    }
+    group_sync(2);
+    // Y = A_ba T_a: blocks (I, J) in {2,3} x {0,1}
+    {
+        const int b = p >> 6, I = 2 + (b >> 1), J = b & 1;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int K = J; K < 2; ++K)
+            block_row_times<false>(acc, Af, 16 * I + r, 16 * K, Tf, 16 * K, 16 * J + cq);
+        *reinterpret_cast<float4 *>(Xs + b * 256 + r * 16 + cq) =
+            make_float4(acc[0], acc[1], acc[2], acc[3]);
+    }
+    group_sync(2);
+    // T_ba = -T_b Y
+    {
+        const int b = p >> 6, I = 2 + (b >> 1), J = b & 1;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int K = 2; K <= I; ++K)
+            block_row_times<true>(acc, Tf, 16 * I + r, 16 * K, Xs + ((K - 2) * 2 + J) * 256, 0, cq);
+        st4(Tf, 16 * I + r, 16 * J + cq, make_float4(-acc[0], -acc[1], -acc[2], -acc[3]));
+    }
+    group_sync(2);
+    // T -> tf32 operand [i][j]
+    for (int e = p; e < C * 16; e += 256) {
+        const int i = e >> 4, q = e & 15, j0 = q * 4;
+        const float4 t = ld4(Tf, i, j0);
+        const float tv[4] = {t.x, t.y, t.z, t.w};
+        uint32_t w[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) w[k] = to_tf32(j0 + k <= i ? tv[k] : 0.f);
+        st_shared_v4(tm_addr + (j0 >> 5) * 8192 + sw128_offset(i, (j0 & 31) >> 2), w[0], w[1], w[2],
+                     w[3]);
+    }
+}
+
+template <bool CHANNEL>
 __global__ void __launch_bounds__(kThreads, 1)
-prefill_tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q,
-                      const __grid_constant__ CUtensorMap tm_k,
-                      const __grid_constant__ CUtensorMap tm_v, const float *__restrict__ g,
-                      const float *__restrict__ beta, const float *h0,
-                      const int32_t *__restrict__ cu, int num_seqs, int total_T, int H,
-                      __nv_bfloat16 *__restrict__ o, float *fin, uint32_t *err) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *sm = reinterpret_cast<uint8_t *>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    const uint32_t sbase = smem_u32(sm);
+prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, const float *__restrict__ g,
+                  const float *__restrict__ beta, const float *h0,
+                  const int32_t *__restrict__ cu, int num_seqs, int total_T, int H,
+                  __nv_bfloat16 *__restrict__ o, float *fin, uint32_t *err) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const uint32_t sbase = smem_u32(smem_raw);
+    if ((sbase & 1023u) != 0) {
+        if (threadIdx.x == 0) atomicOr(err, ERR_SMEM_ALIGN);
+        return;
+    }
+    uint8_t *sm = smem_raw;
     Misc *m = reinterpret_cast<Misc *>(sm + OFF_MISC);
-    float *Af = reinterpret_cast<float *>(sm + OFF_KH);            // [64][65]
-    float *Tf = reinterpret_cast<float *>(sm + OFF_QT);            // [64][65]
-    float *Xt = reinterpret_cast<float *>(sm + OFF_QT + 64 * AF_LD * 4);  // [3][16][16]
 
     const int h = blockIdx.x % H;
     const int n = blockIdx.x / H;
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
-    const int sub = warp & 3;          // TMEM sub-partition (lanes 32*sub .. +31)
-    const int half = warp >> 2;        // which half of the columns this warp handles
-    const int row = sub * 32 + lane;   // TMEM lane = matrix row
+    const int sub = warp & 3;           // TMEM sub-partition of this warp
+    const int half = (warp >> 2) & 1;   // column half handled inside the group
+    const int row = sub * 32 + lane;    // TMEM lane = matrix row
     const uint32_t lane_off = static_cast<uint32_t>(sub * 32) << 16;
 
     if (tid == 0) {
         mbar_init(&m->bar_tma, 1);
-        mbar_init(&m->bar_mma, 1);
+        mbar_init(&m->bar_p, 1);
+        mbar_init(&m->bar_ready, 1);
+        mbar_init(&m->bar_s1, 1);
+        mbar_init(&m->bar_s3, 1);
         m->abort_flag = 0;
+        m->slow = 0;
         fence_barrier_init();
         prefetch_tensormap(&tm_q);
         prefetch_tensormap(&tm_k);
@@ -178,38 +339,196 @@ prefill_tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q,
 
     int t0, len;
     sequence_range(cu, n, num_seqs, total_T, t0, len);
+    const int nchunks = (len + C - 1) / C;
 
-    // ---- initial state: thread owns row `row`, columns half*64 .. +63 ------
-    const size_t sbase_g = (((size_t)n * H + h) * D + row) * D + half * 64;
-    float S[64];
+    if (tid < 256) {
+        // ===================================================== chain group ====
+        const size_t sg = (((size_t)n * H + h) * D + row) * D + half * 64;
+        float S[64];
 #pragma unroll
-    for (int j = 0; j < 64; j += 4) {
-        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (h0 != nullptr) x = *reinterpret_cast<const float4 *>(h0 + sbase_g + j);
-        S[j] = x.x; S[j + 1] = x.y; S[j + 2] = x.z; S[j + 3] = x.w;
-    }
-    {
-        uint32_t r[32];
-#pragma unroll
-        for (int part = 0; part < 2; ++part) {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) r[j] = to_tf32(S[part * 32 + j]);
-            tmem_st32(tmem + lane_off + TM_S + half * 64 + part * 32, r);
+        for (int j = 0; j < 64; j += 4) {
+            float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (h0 != nullptr) x = *reinterpret_cast<const float4 *>(h0 + sg + j);
+            S[j] = x.x; S[j + 1] = x.y; S[j + 2] = x.z; S[j + 3] = x.w;
         }
-        tmem_wait_st();
-    }
-    tc_fence_before();
-    __syncthreads();
+        {
+            uint32_t r[32];
+#pragma unroll
+            for (int part = 0; part < 2; ++part) {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) r[j] = to_tf32(S[part * 32 + j]);
+                tmem_st32(tmem + lane_off + TM_S + half * 64 + part * 32, r);
+            }
+            tmem_wait_st();
+        }
+        tc_fence_before();
+        group_sync(1);
 
-    uint32_t ph_tma = 0, ph_mma = 0;
-    bool alive = true;
+        // output epilogue of a finished chunk: lane = value channel, columns = tokens
+        auto store_o = [&](int cc) {
+            const int tok0 = t0 + cc * C;
+            const int cl = min(C, len - cc * C);
+            uint32_t x[32];
+            tmem_ld32(tmem + lane_off + TM_O + half * 32, x);
+            tmem_wait_ld();
+#pragma unroll
+            for (int ii = 0; ii < 32; ++ii) {
+                const int i = half * 32 + ii;
+                if (i < cl)
+                    o[((size_t)(tok0 + i) * H + h) * D + row] =
+                        __float2bfloat16_rn(__uint_as_float(x[ii]));
+            }
+        };
+        bool done_ok = true;
+        for (int c = 0; c < nchunks; ++c) {
+            const uint32_t par = c & 1;
+            const uint32_t tmU = TM_U0 + par * 64;
+            if (!group_wait(&m->bar_ready, par, m, err, ERR_TIMEOUT_HANDOFF, 1)) { done_ok = false; break; }
+            tc_fence_after();
+            // S1: U^T += S (-W)^T -- the only product on the state's critical path
+            if (tid == 0) {
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    const uint32_t off = (k >> 2) * 8192 + (k & 3) * 32;
+                    mma_tf32_ts(tmem + tmU, tmem + TM_S + k * 8,
+                                sw128_kmajor_desc(sbase + OFF_X1 + off), IDESC_N64, 1);
+                }
+                mma_commit(&m->bar_s1);
+            }
+            if (c >= 1) store_o(c - 1);   // overlaps S1
+            if (!group_wait(&m->bar_s1, par, m, err, ERR_TIMEOUT_MMA, 1)) { done_ok = false; break; }
+            tc_fence_after();
+            {   // round U to tf32 in place: it is the A operand of S3 and S2
+                uint32_t x[32];
+                tmem_ld32(tmem + lane_off + tmU + half * 32, x);
+                tmem_wait_ld();
+#pragma unroll
+                for (int jj = 0; jj < 32; ++jj) x[jj] = to_tf32(__uint_as_float(x[jj]));
+                tmem_st32(tmem + lane_off + tmU + half * 32, x);
+                tmem_wait_st();
+            }
+            tc_fence_before();
+            group_sync(1);
+            if (tid == 0) {
+                tc_fence_after();
+                // S3: ΔS = U^T K̂ (state) first, then the output products
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const uint32_t kb = k >> 2, kk = k & 3;
+                    mma_tf32_ts(tmem + TM_DS, tmem + tmU + k * 8,
+                                sw128_kmajor_desc(sbase + OFF_KH + kb * 16384 + kk * 32),
+                                IDESC_N128, k != 0);
+                }
+                // S1': O^T = S Q̃^T ; S2: O^T += U^T (P⊙causal)^T
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    const uint32_t off = (k >> 2) * 8192 + (k & 3) * 32;
+                    mma_tf32_ts(tmem + TM_O, tmem + TM_S + k * 8,
+                                sw128_kmajor_desc(sbase + OFF_QT + off), IDESC_N64, k != 0);
+                }
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const uint32_t kb = k >> 2, kk = k & 3;
+                    mma_tf32_ts(tmem + TM_O, tmem + tmU + k * 8,
+                                sw128_kmajor_desc(sbase + OFF_PM + par * 16384 + kb * 8192 + kk * 32),
+                                IDESC_N64, 1);
+                }
+                mma_commit(&m->bar_s3);
+            }
+            if (!group_wait(&m->bar_s3, par, m, err, ERR_TIMEOUT_MMA, 1)) { done_ok = false; break; }
+            tc_fence_after();
+            {   // S = S Diag(exp(G_C)) + ΔS (fp32 master), tf32 copy back to TMEM
+                const float *gcb = m->gcb[par];
+#pragma unroll
+                for (int part = 0; part < 2; ++part) {
+                    uint32_t x[32];
+                    tmem_ld32(tmem + lane_off + TM_DS + half * 64 + part * 32, x);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int jj = 0; jj < 32; ++jj) {
+                        const float gc = CHANNEL ? gcb[half * 64 + part * 32 + jj] : gcb[0];
+                        const float sv = fmaf(gc, S[part * 32 + jj], __uint_as_float(x[jj]));
+                        S[part * 32 + jj] = sv;
+                        x[jj] = to_tf32(sv);
+                    }
+                    tmem_st32(tmem + lane_off + TM_S + half * 64 + part * 32, x);
+                }
+                tmem_wait_st();
+            }
+            tc_fence_before();
+            group_sync(1);
+        }
+        if (done_ok && nchunks > 0) {
+            tc_fence_after();
+            store_o(nchunks - 1);
+        }
+        if (fin != nullptr) {
+#pragma unroll
+            for (int j = 0; j < 64; j += 4)
+                *reinterpret_cast<float4 *>(fin + sg + j) =
+                    make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+        }
+    } else {
+        // ====================================================== prep group ====
+        const int p = tid - 256;
+        bool tma_pending = false;
+        uint32_t ph_tma = 0, ph_p = 0;
 
-    for (int c0 = 0; c0 < len && alive; c0 += C) {
-        const int cl = min(C, len - c0);
-        const int tok0 = t0 + c0;
-
-        // ---- a1: stage the chunk tiles (TMA) and the masked gates ---------
-        if (tid == 0) {
+        // gates and beta run ahead of the tiles: scalar gates two chunks ahead in
+        // registers (prep warp 0), channel gates one chunk ahead in registers and
+        // two chunks ahead in L2
+        float gs0 = 0.f, gs1 = 0.f, bs0 = 0.f, bs1 = 0.f;   // chunk c (prep warp 0)
+        float fg0 = 0.f, fg1 = 0.f, fb0 = 0.f, fb1 = 0.f;   // chunk c + 1 (scalar gates)
+        float gr[32];                                        // channel gates (KDA)
+#pragma unroll
+        for (int k = 0; k < 32; ++k) gr[k] = 0.f;
+        const int ch = p & 127, hh = p >> 7;                 // KDA: channel, token half
+        auto load_scalar = [&](int c, float &ga, float &gb, float &ba, float &bb) {
+            if (p < 32 && c < nchunks) {
+                const int tok0 = t0 + c * C;
+                const int cl = min(C, len - c * C);
+                const int i0 = 2 * p, i1 = 2 * p + 1;
+                const size_t r0 = (size_t)(tok0 + i0) * H + h, r1 = (size_t)(tok0 + i1) * H + h;
+                ba = i0 < cl ? beta[r0] : 0.f;
+                bb = i1 < cl ? beta[r1] : 0.f;
+                if (!CHANNEL) {   // raw values: clamped where used, so nothing waits here
+                    ga = i0 < cl ? g[r0] : 0.f;
+                    gb = i1 < cl ? g[r1] : 0.f;
+                }
+            }
+        };
+        auto load_channel = [&](int c) {
+            if (CHANNEL && c < nchunks) {
+                const int tok0 = t0 + c * C;
+                const int cl = min(C, len - c * C);
+#pragma unroll
+                for (int k = 0; k < 32; ++k) {
+                    const int i = hh * 32 + k;
+                    gr[k] = i < cl ? g[((size_t)(tok0 + i) * H + h) * D + ch] : 0.f;
+                }
+            }
+        };
+        auto l2_channel = [&](int c) {   // one 128-byte line of chunk c's gate rows per thread
+            if (CHANNEL && c < nchunks) {
+                const int tok0 = t0 + c * C;
+                const int i = p >> 2;
+                if (i < len - c * C) {
+                    const float *a = g + ((size_t)(tok0 + i) * H + h) * D + (p & 3) * 32;
+                    asm volatile("prefetch.global.L2 [%0];" ::"l"(a));
+                }
+            }
+        };
+        auto issue_tma = [&](int c) {
+            const int tok0 = t0 + c * C;
+            if (c + 1 < nchunks) {       // warm L2 with the chunk after this one
+                const int t1 = tok0 + C;
+                tma_prefetch_l2_3d(&tm_k, 0, h, t1);
+                tma_prefetch_l2_3d(&tm_k, 64, h, t1);
+                tma_prefetch_l2_3d(&tm_q, 0, h, t1);
+                tma_prefetch_l2_3d(&tm_q, 64, h, t1);
+                tma_prefetch_l2_3d(&tm_v, 0, h, t1);
+                tma_prefetch_l2_3d(&tm_v, 64, h, t1);
+            }
             fence_proxy_async();
             mbar_arrive_expect_tx(&m->bar_tma, 6 * 8192);
             tma_load_3d(sm + OFF_KQ + 0, &tm_k, &m->bar_tma, 0, h, tok0);
@@ -218,309 +537,329 @@ prefill_tc_gdn_kernel(const __grid_constant__ CUtensorMap tm_q,
             tma_load_3d(sm + OFF_KQ + 24576, &tm_q, &m->bar_tma, 64, h, tok0);
             tma_load_3d(sm + OFF_V + 0, &tm_v, &m->bar_tma, 0, h, tok0);
             tma_load_3d(sm + OFF_V + 8192, &tm_v, &m->bar_tma, 64, h, tok0);
-        }
-        if (warp == 0) {
-            // a2: within-chunk cumulative log-gate (lane holds tokens 2l, 2l+1)
-            const int i0 = 2 * lane, i1 = 2 * lane + 1;
-            const size_t r0 = (size_t)(tok0 + i0) * H + h, r1 = (size_t)(tok0 + i1) * H + h;
-            const float g0 = i0 < cl ? clamp_log_gate(g[r0]) : 0.f;
-            const float g1 = i1 < cl ? clamp_log_gate(g[r1]) : 0.f;
-            const float b0 = i0 < cl ? beta[r0] : 0.f;
-            const float b1 = i1 < cl ? beta[r1] : 0.f;
-            float pair = g0 + g1;
-            float incl = pair;
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const float y = __shfl_up_sync(0xffffffffu, incl, off);
-                if (lane >= off) incl += y;
+        };
+        if (nchunks > 0) {
+            if (p == 0) {
+                issue_tma(0);
+                tma_pending = true;
             }
-            const float excl = incl - pair;
-            const float G0 = excl + g0, G1 = incl;
-            const float GC = __shfl_sync(0xffffffffu, incl, 31);
-            m->G[i0] = G0; m->G[i1] = G1;
-            m->beta[i0] = b0; m->beta[i1] = b1;
-            const float e0 = __expf(G0), e1 = __expf(G1);
-            m->gam[i0] = e0; m->gam[i1] = e1;
-            m->kp[i0] = b0 * e0; m->kp[i1] = b1 * e1;
-            m->kh[i0] = __expf(GC - G0); m->kh[i1] = __expf(GC - G1);
-            if (lane == 0) m->gC = __expf(GC);
+            load_scalar(0, gs0, gs1, bs0, bs1);
+            load_scalar(1, fg0, fg1, fb0, fb1);
+            l2_channel(0);
+            l2_channel(1);
         }
-        alive = cta_wait(&m->bar_tma, ph_tma, m, err, ERR_TIMEOUT_TMA);
-        ph_tma ^= 1;
-        if (!alive) break;
 
-        // ---- a3 (tensor part): P1 = [K;Q] K^T --------------------------------
-        if (tid == 0) {
-            tc_fence_after();
-#pragma unroll
-            for (int kb = 0; kb < 2; ++kb)
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    const uint32_t a = sbase + OFF_KQ + kb * 16384 + kk * 32;
-                    mma_f16_ss(tmem + TM_P1, sw128_kmajor_desc(a), sw128_kmajor_desc(a), IDESC_P1,
-                               (kb | kk) != 0);
-                }
-            mma_commit(&m->bar_mma);
-        }
-        alive = cta_wait(&m->bar_mma, ph_mma, m, err, ERR_TIMEOUT_MMA);
-        ph_mma ^= 1;
-        if (!alive) break;
-        tc_fence_after();
+        for (int c = 0; c < nchunks; ++c) {
+            const uint32_t par = c & 1;
+            float GC = 0.f, R = 0.f;
 
-        // ---- a3 (gates): A (fp32 scratch) and P (tf32 operand) -------------
-        {
-            uint32_t x[32];
-            tmem_ld32(tmem + lane_off + TM_P1 + half * 32, x);
-            tmem_wait_ld();
-            if (row < C) {
-                const int i = row;
-                const float Gi = m->G[i], bi = m->beta[i];
+            // ---- a2: gates ----------------------------------------------------
+            if (p < 32) {
+                m->u.s.beta[2 * p] = bs0;       // beta is first in both layouts
+                m->u.s.beta[2 * p + 1] = bs1;
+            }
+            if (p == 0) m->slow = 0;
+            if (!CHANNEL) {
+                if (p < 32) {
+                    const int i0 = 2 * p, i1 = 2 * p + 1;
+                    gs0 = clamp_log_gate(gs0);
+                    gs1 = clamp_log_gate(gs1);
+                    const float pair = gs0 + gs1;
+                    float incl = pair;
 #pragma unroll
-                for (int jj = 0; jj < 32; ++jj) {
-                    const int j = half * 32 + jj;
-                    const float a = (j < i) ? bi * __expf(Gi - m->G[j]) * __uint_as_float(x[jj]) : 0.f;
-                    Af[i * AF_LD + j] = a;
+                    for (int off = 1; off < 32; off <<= 1) {
+                        const float y = __shfl_up_sync(0xffffffffu, incl, off);
+                        if (lane >= off) incl += y;
+                    }
+                    const float G0 = incl - pair + gs0, G1 = incl;
+                    const float Gl = __shfl_sync(0xffffffffu, incl, 31);
+                    m->u.s.G[i0] = G0; m->u.s.G[i1] = G1;
+                    const float e0 = __expf(G0), e1 = __expf(G1);
+                    m->u.s.gam[i0] = e0; m->u.s.gam[i1] = e1;
+                    m->u.s.kp[i0] = bs0 * e0; m->u.s.kp[i1] = bs1 * e1;
+                    m->u.s.kh[i0] = __expf(Gl - G0); m->u.s.kh[i1] = __expf(Gl - G1);
+                    m->u.s.ieg[i0] = __expf(-G0); m->u.s.ieg[i1] = __expf(-G1);
+                    if (p == 0) m->wide = (Gl < -80.f) ? 1 : 0;
                 }
             } else {
-                const int i = row - C;
-                const float Gi = m->G[i];
-                const uint32_t rowaddr = sbase + OFF_PM + half * 8192;
+                // this chunk's channel gates (L2-resident: prefetched two chunks ago),
+                // then the inclusive cumsum of this thread's 32 tokens of channel ch
+                load_channel(c);
+                gr[0] = clamp_log_gate(gr[0]);
+#pragma unroll
+                for (int k = 1; k < 32; ++k) gr[k] = clamp_log_gate(gr[k]) + gr[k - 1];
+                if (hh == 0) m->u.c.T0[ch] = gr[31];
+                else m->u.c.T1[ch] = gr[31];
+            }
+            // roll the scalar pipeline: chunk c+1 moves up, chunk c+2 is requested
+            gs0 = fg0; gs1 = fg1; bs0 = fb0; bs1 = fb1;
+            load_scalar(c + 2, fg0, fg1, fb0, fb1);
+            if (!group_wait(&m->bar_tma, ph_tma, m, err, ERR_TIMEOUT_TMA, 2)) break;
+            ph_tma ^= 1;
+            tma_pending = false;
+
+            if (CHANNEL) {
+                // chunk-cumulative gate of this thread's tokens; reference R = G_31
+                const float T0 = m->u.c.T0[ch], T1 = m->u.c.T1[ch];
+                if (hh == 1) {
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) gr[k] += T0;
+                }
+                R = T0;
+                GC = T0 + T1;
+                // fp16 P1 operands: rows [K e^{G-R}; Q e^{G-R}] (X2), K e^{R-G} (TM)
+                bool bad = false;
+                const uint32_t kcol = (ch >> 6) * 16384, bcol = (ch >> 6) * 8192;
+                const uint32_t cch = (ch & 63) >> 3, cel = (ch & 7) * 2;
+#pragma unroll 4
+                for (int k = 0; k < 32; ++k) {
+                    const int i = hh * 32 + k;
+                    const uint32_t src = sbase + OFF_KQ + kcol + sw128_offset(i, cch) + cel;
+                    const float kv = ld_shared_bf16(src), qv = ld_shared_bf16(src + 8192);
+                    const float up = __expf(gr[k] - R), dn = __expf(R - gr[k]);
+                    const float a = kv * up, b = qv * up, e = kv * dn;
+                    bad |= !(fabsf(a) < kF16Limit) || !(fabsf(b) < kF16Limit) ||
+                           !(fabsf(e) < kF16Limit);
+                    st_shared_b16(sbase + OFF_X2 + kcol + sw128_offset(i, cch) + cel,
+                                  __half_as_ushort(__float2half_rn(a)));
+                    st_shared_b16(sbase + OFF_X2 + kcol + sw128_offset(64 + i, cch) + cel,
+                                  __half_as_ushort(__float2half_rn(b)));
+                    st_shared_b16(sbase + OFF_TM + bcol + sw128_offset(i, cch) + cel,
+                                  __half_as_ushort(__float2half_rn(e)));
+                }
+                if (bad) m->slow = 1;
+                fence_proxy_async();
+                group_sync(2);
+            }
+            const bool slow = CHANNEL && m->slow != 0;
+
+            // ---- a3: P1 ---------------------------------------------------------
+            if (!slow) {
+                if (p == 0) {
+                    tc_fence_after();
+#pragma unroll
+                    for (int kb = 0; kb < 2; ++kb)
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk) {
+                            if (CHANNEL) {
+                                mma_f16_ss(tmem + TM_P1W,
+                                           sw128_kmajor_desc(sbase + OFF_X2 + kb * 16384 + kk * 32),
+                                           sw128_kmajor_desc(sbase + OFF_TM + kb * 8192 + kk * 32),
+                                           IDESC_F16, (kb | kk) != 0);
+                            } else {
+                                const uint32_t a = sbase + OFF_KQ + kb * 16384 + kk * 32;
+                                mma_f16_ss(tmem + TM_P1W, sw128_kmajor_desc(a), sw128_kmajor_desc(a),
+                                           IDESC_BF16, (kb | kk) != 0);
+                            }
+                        }
+                    mma_commit(&m->bar_p);
+                }
+                if (!group_wait(&m->bar_p, ph_p, m, err, ERR_TIMEOUT_MMA, 2)) break;
+                ph_p ^= 1;
+                tc_fence_after();
+            }
+            // P slot `par` and U slot `par` were last used by chunk c-2's chain;
+            // chunk c-1's S1 completing implies that chain finished.
+            if (c >= 1 && !group_wait(&m->bar_s1, (c - 1) & 1, m, err, ERR_TIMEOUT_HANDOFF, 2)) break;
+
+            float *Af;
+            float *Tf;
+            float *Xs;
+            const uint32_t pm = sbase + OFF_PM + par * 16384;
+            if (!slow) {
+                Af = reinterpret_cast<float *>(sm + OFF_X2);
+                Tf = reinterpret_cast<float *>(sm + OFF_X2 + 16384);
+                Xs = reinterpret_cast<float *>(sm + OFF_TM);
+                uint32_t x[32];
+                tmem_ld32(tmem + lane_off + TM_P1W + half * 32, x);
+                tmem_wait_ld();
+                // decay factor exp(G_i - G_j): a product of per-row and per-column
+                // factors when the chunk's total decay stays within e^-80 (the
+                // factors are then finite normals), else one exponential each
+                const bool wide = !CHANNEL && m->wide != 0;
+                const int i = row < C ? row : row - C;
+                const float Gi = CHANNEL ? 0.f : m->u.s.G[i];
+                const float rowf = (row < C ? m->u.s.beta[i] : 1.f) * (CHANNEL ? 1.f : m->u.s.gam[i]);
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
-                    uint32_t w[4];
+                    const int j0 = half * 32 + q * 4;
+                    float cf[4] = {1.f, 1.f, 1.f, 1.f};
+                    if (!CHANNEL) {
+                        const float4 t = *reinterpret_cast<const float4 *>(&m->u.s.ieg[j0]);
+                        cf[0] = t.x; cf[1] = t.y; cf[2] = t.z; cf[3] = t.w;
+                    }
+                    float v4[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const int jj = q * 4 + e, j = half * 32 + jj;
-                        const float p = (j <= i) ? __expf(Gi - m->G[j]) * __uint_as_float(x[jj]) : 0.f;
-                        w[e] = to_tf32(p);
+                        const int j = j0 + e;
+                        float f = rowf * cf[e];
+                        if (wide) f = (row < C ? m->u.s.beta[i] : 1.f) * __expf(Gi - m->u.s.G[j]);
+                        const bool keep = row < C ? (j < i) : (j <= i);
+                        v4[e] = keep ? f * __uint_as_float(x[q * 4 + e]) : 0.f;
                     }
-                    st_shared_v4(rowaddr + sw128_offset(i, q), w[0], w[1], w[2], w[3]);
+                    if (row < C) {
+                        st4(Af, i, j0, make_float4(v4[0], v4[1], v4[2], v4[3]));
+                    } else {
+                        st_shared_v4(pm + half * 8192 + sw128_offset(i, q), to_tf32(v4[0]),
+                                     to_tf32(v4[1]), to_tf32(v4[2]), to_tf32(v4[3]));
+                    }
+                }
+            } else {
+                // exact A and P on CUDA cores: G [64][128] fp32 in X2, A in TM
+                float *Gs = reinterpret_cast<float *>(sm + OFF_X2);
+                Af = reinterpret_cast<float *>(sm + OFF_TM);
+                Tf = reinterpret_cast<float *>(sm + OFF_X2);
+                Xs = reinterpret_cast<float *>(sm + OFF_X2 + 16384);
+#pragma unroll
+                for (int k = 0; k < 32; ++k) Gs[(hh * 32 + k) * D + ch] = gr[k];
+                group_sync(2);
+                for (int pr = p; pr < C * (C + 1) / 2; pr += 256) {
+                    int i = (int)((sqrtf(8.f * (float)pr + 1.f) - 1.f) * 0.5f);
+                    while (i * (i + 1) / 2 > pr) --i;
+                    while ((i + 1) * (i + 2) / 2 <= pr) ++i;
+                    const int j = pr - i * (i + 1) / 2;
+                    float dk = 0.f, dq = 0.f;
+                    for (int cc = 0; cc < D; ++cc) {
+                        const uint32_t kc = (cc >> 6) * 16384, chk = (cc & 63) >> 3, el = (cc & 7) * 2;
+                        const float ki = ld_shared_bf16(sbase + OFF_KQ + kc + sw128_offset(i, chk) + el);
+                        const float qi = ld_shared_bf16(sbase + OFF_KQ + kc + 8192 + sw128_offset(i, chk) + el);
+                        const float kj = ld_shared_bf16(sbase + OFF_KQ + kc + sw128_offset(j, chk) + el);
+                        const float e = __expf(Gs[i * D + cc] - Gs[j * D + cc]) * kj;
+                        dk = fmaf(ki, e, dk);
+                        dq = fmaf(qi, e, dq);
+                    }
+                    Af[ax(i, j)] = (j < i) ? m->u.c.beta[i] * dk : 0.f;
+                    st_shared_b32(pm + (j >> 5) * 8192 + sw128_offset(i, (j & 31) >> 2) + (j & 3) * 4,
+                                  to_tf32(dq));
+                }
+                for (int e = p; e < C * C; e += 256) {
+                    const int i = e >> 6, j = e & 63;
+                    if (j > i) {
+                        Af[ax(i, j)] = 0.f;
+                        st_shared_b32(pm + (j >> 5) * 8192 + sw128_offset(i, (j & 31) >> 2) + (j & 3) * 4,
+                                      0u);
+                    }
                 }
             }
-        }
-        __syncthreads();
+            group_sync(2);
 
-        // ---- a4: T = (I + A)^-1 (blocked 16 x 16 forward substitution) -----
-        if (tid < 64) {
-            const int blk = tid >> 4, c = tid & 15, col = blk * 16 + c;
-            for (int r = 0; r < 16; ++r) {
-                const int ri = blk * 16 + r;
-                float x;
-                if (r < c) {
-                    x = 0.f;
-                } else if (r == c) {
-                    x = 1.f;
-                } else {
-                    float acc = 0.f;
-                    for (int s = c; s < r; ++s) acc = fmaf(Af[ri * AF_LD + blk * 16 + s], Tf[(blk * 16 + s) * AF_LD + col], acc);
-                    x = -acc;
-                }
-                Tf[ri * AF_LD + col] = x;
-            }
-        }
-        __syncthreads();
-        for (int d = 1; d < 4; ++d) {
-            const int nblk = 4 - d;
-            for (int e = tid; e < nblk * 256; e += kThreads) {
-                const int bi = e >> 8, r = (e >> 4) & 15, c = e & 15;
-                const int I = d + bi, J = I - d;
-                float acc = 0.f;
-                for (int K = J; K < I; ++K)
-#pragma unroll
-                    for (int s = 0; s < 16; ++s)
-                        acc = fmaf(Af[(I * 16 + r) * AF_LD + K * 16 + s], Tf[(K * 16 + s) * AF_LD + J * 16 + c], acc);
-                Xt[bi * 256 + r * 16 + c] = acc;
-            }
-            __syncthreads();
-            for (int e = tid; e < nblk * 256; e += kThreads) {
-                const int bi = e >> 8, r = (e >> 4) & 15, c = e & 15;
-                const int I = d + bi, J = I - d;
-                float acc = 0.f;
-                for (int s = 0; s <= r; ++s)
-                    acc = fmaf(Tf[(I * 16 + r) * AF_LD + I * 16 + s], Xt[bi * 256 + s * 16 + c], acc);
-                Tf[(I * 16 + r) * AF_LD + J * 16 + c] = -acc;
-            }
-            __syncthreads();
-        }
-        // T -> tf32 operand [i][j] (zero above the diagonal)
-        for (int e = tid; e < C * 16; e += kThreads) {
-            const int i = e >> 4, q = e & 15, j0 = q * 4;
-            uint32_t w[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int j = j0 + k;
-                w[k] = to_tf32(j <= i ? Tf[i * AF_LD + j] : 0.f);
-            }
-            st_shared_v4(sbase + OFF_TM + (j0 >> 5) * 8192 + sw128_offset(i, (j0 & 31) >> 2), w[0], w[1], w[2], w[3]);
-        }
-        __syncthreads();
+            // ---- a4: T = (I + A)^-1 -------------------------------------------------
+            unit_lower_inverse(Af, Tf, Xs, sbase + OFF_TM, p);
+            group_sync(2);
 
-        // ---- a5 operands: K'^T, V'^T, K̂^T (transposed) and Q̃ -------------
-        {
-            const int i = tid & 63;
-            const float kp = m->kp[i], bt = m->beta[i], kh = m->kh[i], gq = m->gam[i];
-            const uint32_t tcol = (i >> 5) * 16384;          // token block of the [d][tok] tiles
-            const uint32_t tchunk = (i & 31) >> 2, tel = (i & 3) * 4;
+            // ---- a5 operands (X1, QT, KH are free once chunk c-1's S3 is done) --------
+            if (c >= 1 && !group_wait(&m->bar_s3, (c - 1) & 1, m, err, ERR_TIMEOUT_HANDOFF, 2)) break;
+            if (!CHANNEL) {
+                if (p == 0) m->gcb[par][0] = __expf(m->u.s.G[C - 1]);
+                const int i = p & 63;
+                const float kp = m->u.s.kp[i], bt = m->u.s.beta[i], kh = m->u.s.kh[i],
+                            gq = m->u.s.gam[i];
+                const uint32_t tcol = (i >> 5) * 16384;
+                const uint32_t tchunk = (i & 31) >> 2, tel = (i & 3) * 4;
 #pragma unroll 1
-            for (int it = 0; it < 4; ++it) {
-                const int jc = (tid >> 6) + 4 * it;          // 8-wide d chunk 0..15
-                const uint32_t kb = jc >> 3, ch = jc & 7;
-                float kf[8], qf[8], vf[8];
-                bf16x8_to_f32(ld_shared_v4(sbase + OFF_KQ + kb * 16384 + sw128_offset(i, ch)), kf);
-                bf16x8_to_f32(ld_shared_v4(sbase + OFF_KQ + kb * 16384 + 8192 + sw128_offset(i, ch)), qf);
-                bf16x8_to_f32(ld_shared_v4(sbase + OFF_V + kb * 8192 + sw128_offset(i, ch)), vf);
+                for (int it = 0; it < 4; ++it) {
+                    const int jc = (p >> 6) + 4 * it;
+                    const uint32_t kb = jc >> 3, chk = jc & 7;
+                    float kf[8], qf[8], vf[8];
+                    bf16x8_to_f32(ld_shared_v4(sbase + OFF_KQ + kb * 16384 + sw128_offset(i, chk)), kf);
+                    bf16x8_to_f32(ld_shared_v4(sbase + OFF_KQ + kb * 16384 + 8192 + sw128_offset(i, chk)), qf);
+                    bf16x8_to_f32(ld_shared_v4(sbase + OFF_V + kb * 8192 + sw128_offset(i, chk)), vf);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const uint32_t j = jc * 8 + e;
-                    const uint32_t off = tcol + sw128_offset(j, tchunk) + tel;
-                    st_shared_b32(sbase + OFF_X1 + off, to_tf32(kp * kf[e]));
-                    st_shared_b32(sbase + OFF_X2 + off, to_tf32(bt * vf[e]));
-                    st_shared_b32(sbase + OFF_KH + off, to_tf32(kh * kf[e]));
+                    for (int e = 0; e < 8; ++e) {
+                        const uint32_t j = jc * 8 + e;
+                        const uint32_t off = tcol + sw128_offset(j, tchunk) + tel;
+                        st_shared_b32(sbase + OFF_X1 + off, to_tf32(kp * kf[e]));
+                        st_shared_b32(sbase + OFF_X2 + off, to_tf32(bt * vf[e]));
+                        st_shared_b32(sbase + OFF_KH + off, to_tf32(kh * kf[e]));
+                    }
+                    const uint32_t qb = sbase + OFF_QT + (jc >> 2) * 8192;
+                    const uint32_t qc = (jc & 3) * 2;
+                    st_shared_v4(qb + sw128_offset(i, qc), to_tf32(gq * qf[0]), to_tf32(gq * qf[1]),
+                                 to_tf32(gq * qf[2]), to_tf32(gq * qf[3]));
+                    st_shared_v4(qb + sw128_offset(i, qc + 1), to_tf32(gq * qf[4]), to_tf32(gq * qf[5]),
+                                 to_tf32(gq * qf[6]), to_tf32(gq * qf[7]));
                 }
-                const uint32_t qb = sbase + OFF_QT + (jc >> 2) * 8192;
-                const uint32_t qc = (jc & 3) * 2;
-                st_shared_v4(qb + sw128_offset(i, qc), to_tf32(gq * qf[0]), to_tf32(gq * qf[1]),
-                             to_tf32(gq * qf[2]), to_tf32(gq * qf[3]));
-                st_shared_v4(qb + sw128_offset(i, qc + 1), to_tf32(gq * qf[4]), to_tf32(gq * qf[5]),
-                             to_tf32(gq * qf[6]), to_tf32(gq * qf[7]));
+            } else {
+                if (hh == 0) m->gcb[par][ch] = __expf(GC);
+                const uint32_t kcol = (ch >> 6) * 16384, cch = (ch & 63) >> 3, cel = (ch & 7) * 2;
+                const uint32_t vcol = (ch >> 6) * 8192;
+                const uint32_t rowblk = hh * 16384;
+                const uint32_t qaddr = sbase + OFF_QT + (ch >> 5) * 8192 + (ch & 3) * 4;
+                const uint32_t qch = (ch & 31) >> 2;
+#pragma unroll
+                for (int q4 = 0; q4 < 8; ++q4) {
+                    uint32_t wk[4], wh[4], wv[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int k = q4 * 4 + e, i = hh * 32 + k;
+                        const uint32_t src = sbase + OFF_KQ + kcol + sw128_offset(i, cch) + cel;
+                        const float kv = ld_shared_bf16(src), qv = ld_shared_bf16(src + 8192);
+                        const float vv = ld_shared_bf16(sbase + OFF_V + vcol + sw128_offset(i, cch) + cel);
+                        const float bi = m->u.c.beta[i];
+                        const float eg = __expf(gr[k]);
+                        wk[e] = to_tf32(bi * kv * eg);
+                        wh[e] = to_tf32(kv * __expf(GC - gr[k]));
+                        wv[e] = to_tf32(bi * vv);
+                        st_shared_b32(qaddr + sw128_offset(i, qch), to_tf32(qv * eg));
+                    }
+                    st_shared_v4(sbase + OFF_X1 + rowblk + sw128_offset(ch, q4), wk[0], wk[1], wk[2], wk[3]);
+                    st_shared_v4(sbase + OFF_KH + rowblk + sw128_offset(ch, q4), wh[0], wh[1], wh[2], wh[3]);
+                    st_shared_v4(sbase + OFF_X2 + rowblk + sw128_offset(ch, q4), wv[0], wv[1], wv[2], wv[3]);
+                }
             }
-        }
-        fence_proxy_async();
-        __syncthreads();
+            fence_proxy_async();
+            group_sync(2);
 
-        // ---- a5 (tensor part): W^T and Ũ^T ----------------------------------
-        if (tid == 0) {
+            // ---- a5 (tensor part): W^T, Ũ^T -------------------------------------------
+            if (p == 0) {
+                tc_fence_after();
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const uint32_t kb = k >> 2, kk = k & 3;
+                    const uint64_t bd = sw128_kmajor_desc(sbase + OFF_TM + kb * 8192 + kk * 32);
+                    mma_tf32_ss(tmem + TM_P1W, sw128_kmajor_desc(sbase + OFF_X1 + kb * 16384 + kk * 32),
+                                bd, IDESC_N64, k != 0);
+                    mma_tf32_ss(tmem + TM_U0 + par * 64,
+                                sw128_kmajor_desc(sbase + OFF_X2 + kb * 16384 + kk * 32), bd, IDESC_N64,
+                                k != 0);
+                }
+                mma_commit(&m->bar_p);
+            }
+            // the chunk tiles are consumed: stage the next chunk while P2 runs
+            if (c + 1 < nchunks) {
+                if (p == 0) {
+                    issue_tma(c + 1);
+                    tma_pending = true;
+                }
+                l2_channel(c + 2);
+            }
+            if (!group_wait(&m->bar_p, ph_p, m, err, ERR_TIMEOUT_MMA, 2)) break;
+            ph_p ^= 1;
             tc_fence_after();
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const uint32_t kb = k >> 2, kk = k & 3;
-                const uint64_t bd = sw128_kmajor_desc(sbase + OFF_TM + kb * 8192 + kk * 32);
-                mma_tf32_ss(tmem + TM_W, sw128_kmajor_desc(sbase + OFF_X1 + kb * 16384 + kk * 32), bd,
-                            IDESC_N64, k != 0);
-                mma_tf32_ss(tmem + TM_U, sw128_kmajor_desc(sbase + OFF_X2 + kb * 16384 + kk * 32), bd,
-                            IDESC_N64, k != 0);
-            }
-            mma_commit(&m->bar_mma);
-        }
-        alive = cta_wait(&m->bar_mma, ph_mma, m, err, ERR_TIMEOUT_MMA);
-        ph_mma ^= 1;
-        if (!alive) break;
-        tc_fence_after();
 
-        // -W -> [tok][dk] tf32 operand (thread = dk row of W^T)
-        {
-            uint32_t x[32];
-            tmem_ld32(tmem + lane_off + TM_W + half * 32, x);
-            tmem_wait_ld();
-            const uint32_t j = row;
-            const uint32_t base = sbase + OFF_X1 + (j >> 5) * 8192;
-#pragma unroll
-            for (int ii = 0; ii < 32; ++ii) {
-                const uint32_t i = half * 32 + ii;
-                st_shared_b32(base + sw128_offset(i, (j & 31) >> 2) + (j & 3) * 4,
-                              to_tf32(-__uint_as_float(x[ii])));
-            }
-        }
-        fence_proxy_async();
-        tc_fence_before();
-        __syncthreads();
-
-        // ---- a6/a7 (state part): U^T += S (-W)^T ; O^T = S Q̃^T ----------------
-        if (tid == 0) {
-            tc_fence_after();
-#pragma unroll
-            for (int k = 0; k < 16; ++k) {
-                const uint32_t off = (k >> 2) * 8192 + (k & 3) * 32;
-                mma_tf32_ts(tmem + TM_U, tmem + TM_S + k * 8, sw128_kmajor_desc(sbase + OFF_X1 + off),
-                            IDESC_N64, 1);
-            }
-#pragma unroll
-            for (int k = 0; k < 16; ++k) {
-                const uint32_t off = (k >> 2) * 8192 + (k & 3) * 32;
-                mma_tf32_ts(tmem + TM_O, tmem + TM_S + k * 8, sw128_kmajor_desc(sbase + OFF_QT + off),
-                            IDESC_N64, k != 0);
-            }
-            mma_commit(&m->bar_mma);
-        }
-        alive = cta_wait(&m->bar_mma, ph_mma, m, err, ERR_TIMEOUT_MMA);
-        ph_mma ^= 1;
-        if (!alive) break;
-        tc_fence_after();
-
-        // round U to tf32 in place (A operand of S2/S3)
-        {
-            uint32_t x[32];
-            tmem_ld32(tmem + lane_off + TM_U + half * 32, x);
-            tmem_wait_ld();
-#pragma unroll
-            for (int jj = 0; jj < 32; ++jj) x[jj] = to_tf32(__uint_as_float(x[jj]));
-            tmem_st32(tmem + lane_off + TM_U + half * 32, x);
-            tmem_wait_st();
-        }
-        tc_fence_before();
-        __syncthreads();
-
-        // ---- a8 + a7: ΔS = U^T K̂ ; O^T += U^T (P⊙causal)^T -------------------
-        if (tid == 0) {
-            tc_fence_after();
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const uint32_t kb = k >> 2, kk = k & 3;
-                mma_tf32_ts(tmem + TM_DS, tmem + TM_U + k * 8,
-                            sw128_kmajor_desc(sbase + OFF_KH + kb * 16384 + kk * 32), IDESC_N128,
-                            k != 0);
-            }
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const uint32_t kb = k >> 2, kk = k & 3;
-                mma_tf32_ts(tmem + TM_O, tmem + TM_U + k * 8,
-                            sw128_kmajor_desc(sbase + OFF_PM + kb * 8192 + kk * 32), IDESC_N64, 1);
-            }
-            mma_commit(&m->bar_mma);
-        }
-        alive = cta_wait(&m->bar_mma, ph_mma, m, err, ERR_TIMEOUT_MMA);
-        ph_mma ^= 1;
-        if (!alive) break;
-        tc_fence_after();
-
-        // state update S = γ_C S + ΔS (fp32 master), tf32 copy back to TMEM
-        {
-            const float gC = m->gC;
-#pragma unroll
-            for (int part = 0; part < 2; ++part) {
+            // -W -> [tok][dk] tf32 operand (thread = d_k row of W^T)
+            {
                 uint32_t x[32];
-                tmem_ld32(tmem + lane_off + TM_DS + half * 64 + part * 32, x);
+                tmem_ld32(tmem + lane_off + TM_P1W + half * 32, x);
                 tmem_wait_ld();
+                const uint32_t j = row;
+                const uint32_t base = sbase + OFF_X1 + (j >> 5) * 8192;
 #pragma unroll
-                for (int jj = 0; jj < 32; ++jj) {
-                    const float s = fmaf(gC, S[part * 32 + jj], __uint_as_float(x[jj]));
-                    S[part * 32 + jj] = s;
-                    x[jj] = to_tf32(s);
+                for (int ii = 0; ii < 32; ++ii) {
+                    const uint32_t i = half * 32 + ii;
+                    st_shared_b32(base + sw128_offset(i, (j & 31) >> 2) + (j & 3) * 4,
+                                  to_tf32(-__uint_as_float(x[ii])));
                 }
-                tmem_st32(tmem + lane_off + TM_S + half * 64 + part * 32, x);
             }
-            // outputs: lane = value channel, columns = tokens
-            uint32_t x[32];
-            tmem_ld32(tmem + lane_off + TM_O + half * 32, x);
-            tmem_wait_ld();
-#pragma unroll
-            for (int ii = 0; ii < 32; ++ii) {
-                const int i = half * 32 + ii;
-                if (i < cl)
-                    o[((size_t)(tok0 + i) * H + h) * D + row] = __float2bfloat16_rn(__uint_as_float(x[ii]));
-            }
-            tmem_wait_st();
+            fence_proxy_async();
+            tc_fence_before();
+            group_sync(2);
+            if (p == 0) mbar_arrive(&m->bar_ready);
         }
-        tc_fence_before();
-        __syncthreads();
+        // never leave a TMA load in flight into this CTA's shared memory
+        if (p == 0 && tma_pending) (void)mbar_wait(&m->bar_tma, ph_tma);
     }
 
-    // ---- a9: final state ----------------------------------------------------
-    if (fin != nullptr) {
-#pragma unroll
-        for (int j = 0; j < 64; j += 4)
-            *reinterpret_cast<float4 *>(fin + sbase_g + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
-    }
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
@@ -566,7 +905,7 @@ bool make_map(CUtensorMap *map, const void *base, int total_T, int H) {
 
 bool tcgen05_prefill_available() { return true; }
 
-bool tcgen05_prefill_serves(bool channel) { return !channel; }
+bool tcgen05_prefill_serves(bool) { return true; }
 
 size_t tcgen05_workspace_bytes(int, int, int) { return 16; }
 
@@ -574,7 +913,6 @@ cudaError_t launch_prefill_tcgen05(const void *q, const void *k, const void *v, 
                                    const float *beta, const float *h0, const int32_t *cu,
                                    int num_seqs, int total_T, int H, bool channel, void *o,
                                    float *fin, void *workspace, cudaStream_t stream) {
-    if (channel) return cudaErrorNotSupported;
     uint32_t *err = static_cast<uint32_t *>(workspace);
     cudaError_t e = cudaMemsetAsync(err, 0, sizeof(uint32_t), stream);
     if (e != cudaSuccess) return e;
@@ -587,12 +925,12 @@ cudaError_t launch_prefill_tcgen05(const void *q, const void *k, const void *v, 
     CUtensorMap mq, mk, mv;
     if (!make_map(&mq, q, total_T, H) || !make_map(&mk, k, total_T, H) || !make_map(&mv, v, total_T, H))
         return cudaErrorInvalidValue;
-    e = cudaFuncSetAttribute(prefill_tc_gdn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)SMEM_BYTES);
+    auto kern = channel ? prefill_tc_kernel<true> : prefill_tc_kernel<false>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
     const size_t blocks = (size_t)num_seqs * H;
     if (blocks > 0x7fffffffull) return cudaErrorInvalidConfiguration;
-    prefill_tc_gdn_kernel<<<(unsigned)blocks, kThreads, SMEM_BYTES, stream>>>(
+    kern<<<(unsigned)blocks, kThreads, SMEM_BYTES, stream>>>(
         mq, mk, mv, g, beta, h0, cu, num_seqs, total_T, H, static_cast<__nv_bfloat16 *>(o), fin,
         err);
     return cudaGetLastError();

@@ -211,3 +211,17 @@ def test_tensor_core_path_is_used_and_reports_no_timeout():
     gdr.gdr_prefill_check_workspace(ws)
     o_ref, fin_ref = oracle_prefill(inp)
     check(inp, o, fin, o_ref, fin_ref, "tcgen05")
+
+
+@pytest.mark.parametrize("c_gate", [0.02, 0.3, 1.5, 6.0])
+def test_channel_gate_decay_strengths(c_gate):
+    """Kimi Delta Attention on the tensor-core kernel across decay strengths:
+    weak and moderate decays take the fp16 scaled-operand path for the
+    intra-chunk products, strong ones push the scaled operands past fp16's
+    range and take the exact CUDA-core path; both must match the oracle."""
+    assert gdr.gdr_prefill_path(128, 128, gdr.GDR_GATE_CHANNEL, gdr.GDR_BF16) == gdr.GDR_PATH_TCGEN05
+    inp = I.make_inputs(total_T=320, H=2, d_k=128, gate_mode=I.CHANNEL, io_dtype=torch.bfloat16,
+                        c=c_gate, h0_std=0.02, seed=31)
+    o, fin = gpu_prefill(inp)
+    o_ref, fin_ref = oracle_prefill(inp)
+    check(inp, o, fin, o_ref, fin_ref, f"kda c={c_gate}")
