@@ -40,7 +40,12 @@ decode_gdn/kda     256 sequences, H=32, d=128, 512 steps of one bf16 token,
                    c=0.1, h0 ~ N(0, 0.02^2) (state 512 MiB fp32)
 varlen_gdn         8 packed sequences, 262144 tokens, H=16, d=128, bf16,
                    scalar gate c=0.1, h0=0
+gqa_prefill        1 sequence, 8192 tokens, 16 query/key heads shared by 48
+                   value heads (3 each), d=128, bf16, scalar gate c=0.05
 =================  ==========================================================
+
+With grouped heads (``H_qk`` < ``H``), q and k carry ``H_qk`` heads and value
+head h reads query/key head ``h // (H // H_qk)``.
 """
 from __future__ import annotations
 
@@ -112,7 +117,7 @@ def _softplus(x: np.ndarray) -> np.ndarray:
 class Inputs:
     """One workload's rounded inputs as CPU torch tensors.
 
-    q, k: [total_T, H, d_k]; v: [total_T, H, d_v] in ``io_dtype``;
+    q, k: [total_T, H_qk, d_k]; v: [total_T, H, d_v] in ``io_dtype``;
     g: [total_T, H] (scalar) or [total_T, H, d_k] (channel) float32;
     beta: [total_T, H] float32; h0: [num_seqs, H, d_v, d_k] float32 or None;
     cu_seqlens: int32 [num_seqs + 1] (always filled in, also for equal
@@ -140,6 +145,10 @@ class Inputs:
 
     @property
     def H(self) -> int:
+        return int(self.v.shape[1])
+
+    @property
+    def H_qk(self) -> int:
         return int(self.q.shape[1])
 
     @property
@@ -173,6 +182,7 @@ def random_cu_seqlens(seed: int, total_T: int, num_seqs: int) -> np.ndarray:
 
 
 def make_inputs(*, total_T: int, H: int, d_k: int, d_v: int | None = None,
+                H_qk: int | None = None,
                 num_seqs: int = 1, cu_seqlens=None, gate_mode: str = SCALAR,
                 io_dtype: torch.dtype = torch.bfloat16, c: float = 0.05,
                 h0_std: float = 0.0, seed: int = 0, meta: dict | None = None) -> Inputs:
@@ -182,6 +192,9 @@ def make_inputs(*, total_T: int, H: int, d_k: int, d_v: int | None = None,
     from 0 to total_T); otherwise ``num_seqs`` equal sequences are used.
     """
     d_v = d_k if d_v is None else d_v
+    H_qk = H if H_qk is None else H_qk
+    if H_qk < 1 or H % H_qk:
+        raise ValueError("H_qk must divide H")
     if gate_mode not in (SCALAR, CHANNEL):
         raise ValueError(f"gate_mode {gate_mode!r}")
     if io_dtype not in (torch.bfloat16, torch.float32):
@@ -196,8 +209,8 @@ def make_inputs(*, total_T: int, H: int, d_k: int, d_v: int | None = None,
         if cu[0] != 0 or cu[-1] != total_T or np.any(np.diff(cu) < 0):
             raise ValueError("cu_seqlens must run from 0 to total_T, non-decreasing")
 
-    q = _fill(seed, "q", (total_T, H, d_k), _l2norm, np.float32)
-    k = _fill(seed, "k", (total_T, H, d_k), _l2norm, np.float32)
+    q = _fill(seed, "q", (total_T, H_qk, d_k), _l2norm, np.float32)
+    k = _fill(seed, "k", (total_T, H_qk, d_k), _l2norm, np.float32)
     v = _fill(seed, "v", (total_T, H, d_v), lambda x: x, np.float32)
     beta = _fill(seed, "beta", (total_T, H), _sigmoid, np.float32)
     gshape = (total_T, H) if gate_mode == SCALAR else (total_T, H, d_k)
@@ -226,7 +239,7 @@ def make_inputs(*, total_T: int, H: int, d_k: int, d_v: int | None = None,
 # ---------------------------------------------------------------------------
 
 WORKLOADS = ("tiny_gdn", "gdn_prefill", "kda_prefill", "decode_gdn",
-             "decode_kda", "varlen_gdn")
+             "decode_kda", "varlen_gdn", "gqa_prefill")
 
 DECODE_SEQS, DECODE_HEADS, DECODE_D, DECODE_STEPS = 256, 32, 128, 512
 
@@ -256,6 +269,10 @@ def workload(name: str, seed: int = 0) -> Inputs:
                            d_k=DECODE_D, num_seqs=DECODE_SEQS, gate_mode=mode,
                            io_dtype=torch.bfloat16, c=0.1, h0_std=0.02, seed=seed,
                            meta={"workload": name, "steps": DECODE_STEPS})
+    if name == "gqa_prefill":
+        return make_inputs(total_T=8192, H=48, H_qk=16, d_k=128, num_seqs=1,
+                           gate_mode=SCALAR, io_dtype=torch.bfloat16, c=0.05, seed=seed,
+                           meta={"workload": name})
     if name == "varlen_gdn":
         cu = random_cu_seqlens(seed, 262144, 8)
         return make_inputs(total_T=262144, H=16, d_k=128, cu_seqlens=cu,

@@ -35,10 +35,17 @@
  * its own initial state (or zero) and the final state after its last token is
  * returned; an empty sequence returns its initial state unchanged.
  *
- * Layouts (all row-major, fp64): q, k [total_T][H][d_k]; v, o
+ * Layouts (all row-major, fp64): q, k [total_T][H_qk][d_k]; v, o
  * [total_T][H][d_v]; g [total_T][H] (scalar mode) or [total_T][H][d_k]
  * (channel mode); beta [total_T][H]; h0, final [num_seqs][H][d_v][d_k];
  * cu_seqlens [num_seqs + 1] int64, 0 = cu[0] <= ... <= cu[num_seqs] = total_T.
+ *
+ * Head mapping: H value heads each own a state; the query/key heads may be
+ * fewer (H_qk dividing H), each shared by H / H_qk consecutive value heads,
+ * value head h reading query/key head h / (H / H_qk).  This is the grouping
+ * of the Qwen Gated DeltaNet layer (16 query-key heads, 48 value heads;
+ * page "Qwen3.8-Flash-Next and GLM-5.3-Flash ...", section "Gated DeltaNet
+ * carries most of the sequence").  H_qk = H is the plain one-to-one case.
  */
 #include <math.h>
 #include <pthread.h>
@@ -49,7 +56,7 @@
 typedef struct {
     const double *q, *k, *v, *g, *beta, *h0;
     const int64_t *cu;
-    int64_t num_seqs, H, dk, dv;
+    int64_t num_seqs, H, H_qk, dk, dv;
     int channel_gate;
     double *o, *final_state;
     int64_t next;                 /* next (sequence, head) pair to take */
@@ -61,6 +68,7 @@ static void run_pair(const oracle_job *J, int64_t n, int64_t h, double *S, doubl
                      double *a)
 {
     const int64_t H = J->H, dk = J->dk, dv = J->dv;
+    const int64_t hq = h / (H / J->H_qk);           /* query/key head of value head h */
     const int64_t SS = dv * dk;
     double *Sfin = J->final_state ? J->final_state + (n * H + h) * SS : NULL;
 
@@ -70,8 +78,8 @@ static void run_pair(const oracle_job *J, int64_t n, int64_t h, double *S, doubl
         memset(S, 0, sizeof(double) * (size_t)SS);
 
     for (int64_t t = J->cu[n]; t < J->cu[n + 1]; ++t) {
-        const double *qt = J->q + (t * H + h) * dk;
-        const double *kt = J->k + (t * H + h) * dk;
+        const double *qt = J->q + (t * J->H_qk + hq) * dk;
+        const double *kt = J->k + (t * J->H_qk + hq) * dk;
         const double *vt = J->v + (t * H + h) * dv;
         const double bt = J->beta[t * H + h];
         double *ot = J->o + (t * H + h) * dv;
@@ -147,11 +155,11 @@ static void *worker(void *arg)
 int gdr_oracle_run(const double *q, const double *k, const double *v,
                    const double *g, const double *beta, const double *h0,
                    const int64_t *cu_seqlens, int64_t num_seqs, int64_t H,
-                   int64_t d_k, int64_t d_v, int channel_gate, double *o,
+                   int64_t H_qk, int64_t d_k, int64_t d_v, int channel_gate, double *o,
                    double *final_state, int nthreads)
 {
     if (!q || !k || !v || !g || !beta || !cu_seqlens || !o || num_seqs < 0 ||
-        H < 0 || d_k < 1 || d_v < 1)
+        H < 0 || H_qk < 1 || d_k < 1 || d_v < 1 || (H > 0 && H % H_qk != 0))
         return -1;
     for (int64_t n = 0; n < num_seqs; ++n)
         if (cu_seqlens[n + 1] < cu_seqlens[n] || cu_seqlens[n] < 0)
@@ -161,7 +169,7 @@ int gdr_oracle_run(const double *q, const double *k, const double *v,
 
     oracle_job J;
     J.q = q; J.k = k; J.v = v; J.g = g; J.beta = beta; J.h0 = h0;
-    J.cu = cu_seqlens; J.num_seqs = num_seqs; J.H = H; J.dk = d_k; J.dv = d_v;
+    J.cu = cu_seqlens; J.num_seqs = num_seqs; J.H = H; J.H_qk = H_qk; J.dk = d_k; J.dv = d_v;
     J.channel_gate = channel_gate ? 1 : 0;
     J.o = o; J.final_state = final_state; J.next = 0;
     pthread_mutex_init(&J.lock, NULL);

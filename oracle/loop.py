@@ -46,7 +46,7 @@ def _load():
             lib = ctypes.CDLL(_LIB)
             P = ctypes.c_void_p
             I64 = ctypes.c_int64
-            lib.gdr_oracle_run.argtypes = [P, P, P, P, P, P, P, I64, I64, I64, I64,
+            lib.gdr_oracle_run.argtypes = [P, P, P, P, P, P, P, I64, I64, I64, I64, I64,
                                            ctypes.c_int, P, P, ctypes.c_int]
             lib.gdr_oracle_run.restype = ctypes.c_int
             _lib = lib
@@ -76,13 +76,15 @@ def run(q, k, v, g, beta, h0=None, cu_seqlens=None, *, channel_gate: bool | None
         nthreads: int | None = None):
     """Evaluate the recurrence in float64.
 
-    q, k: [T, H, d_k]; v: [T, H, d_v]; g: [T, H] (scalar gate) or [T, H, d_k]
-    (channel gate); beta: [T, H]; h0: [N, H, d_v, d_k] or None (zeros);
-    cu_seqlens: [N + 1] or None (one sequence of length T).
+    q, k: [T, H_qk, d_k]; v: [T, H, d_v]; g: [T, H] (scalar gate) or
+    [T, H, d_k] (channel gate); beta: [T, H]; h0: [N, H, d_v, d_k] or None
+    (zeros); cu_seqlens: [N + 1] or None (one sequence of length T).  H_qk
+    divides H; value head h reads query/key head h // (H // H_qk).
     Returns (o [T, H, d_v], final_state [N, H, d_v, d_k]) as float64 arrays.
     """
     q, k, v, g, beta, h0 = (_f64(x) for x in (q, k, v, g, beta, h0))
-    T, H, dk = q.shape
+    T, Hqk, dk = q.shape
+    H = v.shape[1]
     dv = v.shape[2]
     if channel_gate is None:
         channel_gate = g.ndim == 3
@@ -94,7 +96,8 @@ def run(q, k, v, g, beta, h0=None, cu_seqlens=None, *, channel_gate: bool | None
         cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int64))
     N = len(cu) - 1
     exp_g = (T, H, dk) if channel_gate else (T, H)
-    if k.shape != (T, H, dk) or v.shape[:2] != (T, H) or g.shape != exp_g or beta.shape != (T, H):
+    if (k.shape != (T, Hqk, dk) or v.shape[:2] != (T, H) or g.shape != exp_g
+            or beta.shape != (T, H) or Hqk < 1 or H % Hqk):
         raise ValueError("oracle: inconsistent shapes")
     if h0 is not None and h0.shape != (N, H, dv, dk):
         raise ValueError("oracle: h0 shape")
@@ -103,7 +106,7 @@ def run(q, k, v, g, beta, h0=None, cu_seqlens=None, *, channel_gate: bool | None
     o = np.empty((T, H, dv), dtype=np.float64)
     fin = np.empty((N, H, dv, dk), dtype=np.float64)
     rc = _load().gdr_oracle_run(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0),
-                                _ptr(cu), N, H, dk, dv, int(bool(channel_gate)),
+                                _ptr(cu), N, H, Hqk, dk, dv, int(bool(channel_gate)),
                                 _ptr(o), _ptr(fin), int(nthreads or default_threads()))
     if rc != 0:
         raise RuntimeError(f"gdr_oracle_run failed ({rc})")
@@ -127,15 +130,19 @@ def run_inputs(inp, heads=None, seqs=None, nthreads=None):
     ti = np.asarray(tok, dtype=np.int64)
     hi = np.asarray(heads, dtype=np.int64)
 
-    def pick(x):
+    grp = inp.H // int(inp.q.shape[1])
+    hq = hi // grp              # query/key head of each selected value head
+
+    def pick(x, heads=hi):
         if hasattr(x, "detach"):
             import torch
-            x = x.index_select(0, torch.from_numpy(ti)).index_select(1, torch.from_numpy(hi))
+            x = x.index_select(0, torch.from_numpy(ti)).index_select(1, torch.from_numpy(heads))
             return x.float().numpy()
-        return np.asarray(x)[ti][:, hi]
+        return np.asarray(x)[ti][:, heads]
 
     h0 = None
     if inp.h0 is not None:
         h0 = inp.h0.numpy()[np.asarray(seqs, dtype=np.int64)][:, hi]
-    return run(pick(inp.q), pick(inp.k), pick(inp.v), pick(inp.g), pick(inp.beta), h0, sub_cu,
+    # one q/k head per selected value head (a replicated copy where heads share)
+    return run(pick(inp.q, hq), pick(inp.k, hq), pick(inp.v), pick(inp.g), pick(inp.beta), h0, sub_cu,
                channel_gate=(inp.gate_mode == "channel"), nthreads=nthreads)

@@ -40,7 +40,7 @@ def _compile(src_text, tmpdir, name):
                            "-lpthread", "-lm"])
     lib = ctypes.CDLL(so)
     P, I64 = ctypes.c_void_p, ctypes.c_int64
-    lib.gdr_oracle_run.argtypes = [P, P, P, P, P, P, P, I64, I64, I64, I64, ctypes.c_int,
+    lib.gdr_oracle_run.argtypes = [P, P, P, P, P, P, P, I64, I64, I64, I64, I64, ctypes.c_int,
                                    P, P, ctypes.c_int]
     lib.gdr_oracle_run.restype = ctypes.c_int
     return lib
@@ -55,7 +55,7 @@ def _run(lib, q, k, v, g, beta, S0, channel):
     o = np.empty((T, dv))
     fin = np.empty((dv, dk))
     p = lambda a: a.ctypes.data_as(ctypes.c_void_p)
-    rc = lib.gdr_oracle_run(p(q), p(k), p(v), p(g), p(beta), p(S0), p(cu), 1, 1, dk, dv,
+    rc = lib.gdr_oracle_run(p(q), p(k), p(v), p(g), p(beta), p(S0), p(cu), 1, 1, 1, dk, dv,
                             int(channel), p(o), p(fin), 1)
     assert rc == 0
     return o, fin

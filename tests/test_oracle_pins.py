@@ -284,3 +284,26 @@ def test_rejects_bad_arguments():
         oracle.run(z, z, z, np.zeros((4, 1)), np.zeros((4, 1)), None, [0, 3])
     with pytest.raises(ValueError):
         oracle.run(z, z, z, np.zeros((4, 2)), np.zeros((4, 1)))
+
+
+@pytest.mark.parametrize("channel", [False, True])
+def test_grouped_heads_equal_replicated_query_key_heads(channel):
+    """Value heads sharing a query/key head give exactly the result of giving
+    each value head its own copy of that head (the grouping is an index map,
+    not arithmetic)."""
+    rng = np.random.default_rng(15)
+    T, Hqk, grp, dk, dv = 37, 2, 3, 8, 6
+    H = Hqk * grp
+    q = rng.standard_normal((T, Hqk, dk)); k = rng.standard_normal((T, Hqk, dk))
+    k /= np.linalg.norm(k, axis=2, keepdims=True)
+    v = rng.standard_normal((T, H, dv))
+    beta = 1 / (1 + np.exp(-rng.standard_normal((T, H))))
+    g = -np.logaddexp(0, rng.standard_normal((T, H, dk) if channel else (T, H))) * 0.3
+    h0 = rng.standard_normal((1, H, dv, dk)) * 0.1
+    o1, f1 = oracle.run(q, k, v, g, beta, h0, channel_gate=channel)
+    rep = np.arange(H) // grp
+    o2, f2 = oracle.run(q[:, rep], k[:, rep], v, g, beta, h0, channel_gate=channel)
+    assert np.array_equal(o1, o2) and np.array_equal(f1, f2)
+    with pytest.raises(ValueError):
+        oracle.run(q[:, :1].repeat(4, axis=1), k[:, :1].repeat(4, axis=1), v, g, beta, h0,
+                   channel_gate=channel)   # 4 query/key heads do not divide 6 value heads
