@@ -147,9 +147,10 @@ def prefill_work(inp):
     T, H, dk, dv, N = inp.total_T, inp.H, inp.d_k, inp.d_v, inp.num_seqs
     e = io_bytes(inp.io_dtype)
     gate = 4 * (dk if inp.gate_mode == I.CHANNEL else 1)
-    per_th = e * (2 * dk + 2 * dv) + 4 + gate
+    # q and k per query/key head; v, o, beta, g per value head
+    per_t = inp.H_qk * e * 2 * dk + H * (e * 2 * dv + 4 + gate)
     state = 4 * dk * dv * N * H * (2 if inp.h0 is not None else 1)
-    byts = T * H * per_th + state
+    byts = T * per_t + state
     flops = T * H * (5 * CHUNK * max(dk, dv) + 6 * dk * dv)
     return byts, flops
 
@@ -186,10 +187,13 @@ class PrefillCase:
         self.tokens = inp.total_T
         self.launches = 1
 
+    def _fn(self):
+        return gdr.gdr_prefill_chunked if self.inp.H_qk == self.inp.H else gdr.gdr_prefill_chunked_gqa
+
     def step(self, stream=None):
         d = self.d
-        gdr.gdr_prefill_chunked(d["q"], d["k"], d["v"], d["g"], d["beta"], d["h0"], d["cu"],
-                                o=self.o, final_state=self.fin, workspace=self.ws, stream=stream)
+        self._fn()(d["q"], d["k"], d["v"], d["g"], d["beta"], d["h0"], d["cu"], o=self.o,
+                   final_state=self.fin, workspace=self.ws, stream=stream)
 
     def host_inputs(self):
         inp = self.inp
@@ -200,9 +204,8 @@ class PrefillCase:
 
     def e2e_step(self, host, host_o, host_fin, stream):
         dev = {k: v.to(self.dev, non_blocking=True) for k, v in host.items()}
-        gdr.gdr_prefill_chunked(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"],
-                                dev.get("h0"), dev["cu"], o=self.o, final_state=self.fin,
-                                workspace=self.ws, stream=stream)
+        self._fn()(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"], dev.get("h0"), dev["cu"],
+                   o=self.o, final_state=self.fin, workspace=self.ws, stream=stream)
         host_o.copy_(self.o, non_blocking=True)
         host_fin.copy_(self.fin, non_blocking=True)
 
@@ -379,7 +382,7 @@ def bench_case(case, args, ws, rank, flush, stream, pk, pk_kind):
     e2e_ms = max_over_ranks(sum(e2e_times) / len(e2e_times), ws)
     inp = case.inp
     cfg = {"workload": case.name, "num_seqs": inp.num_seqs, "total_T": inp.total_T,
-           "H": inp.H, "d_k": inp.d_k, "d_v": inp.d_v, "gate": inp.gate_mode,
+           "H": inp.H, "H_qk": inp.H_qk, "d_k": inp.d_k, "d_v": inp.d_v, "gate": inp.gate_mode,
            "io": str(inp.io_dtype).replace("torch.", ""),
            "h0": inp.h0 is not None, "l2": "flushed (512 MiB write) before every timed step",
            "kernel": ("decode" if case.kind == "decode" else
@@ -459,7 +462,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.workloads == "all":
-        args.workloads = "gdn_prefill,kda_prefill,varlen_gdn,decode_gdn,decode_kda"
+        args.workloads = "gdn_prefill,kda_prefill,varlen_gdn,gqa_prefill,decode_gdn,decode_kda"
     if args.warmup < 3:
         args.warmup = 3
     ws, rank, local = dist_env()

@@ -46,14 +46,15 @@ template <int DK, bool CHANNEL, typename IoT>
 __global__ void __launch_bounds__(kDecodeThreads, 2)
 decode_step_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k,
                    const IoT *__restrict__ v, const float *__restrict__ g,
-                   const float *__restrict__ beta, float *__restrict__ state, int DV,
-                   IoT *__restrict__ o) {
+                   const float *__restrict__ beta, float *__restrict__ state, int Hqk, int H,
+                   int DV, IoT *__restrict__ o) {
     constexpr int LPR = DK / 16;                      // lanes per state row
     constexpr int RP = kDecodeThreads / LPR;          // rows per pass
     constexpr int MAXP = (LPR / 2 > 0) ? LPR / 2 : 1; // passes cover d_v <= 128
     static_assert(MAXP * RP >= 128, "passes must cover 128 rows");
 
-    const size_t nh = blockIdx.x;
+    const size_t nh = blockIdx.x;                       // (sequence, value head)
+    const size_t qh = (nh / H) * Hqk + (nh % H) / (H / Hqk);   // its query/key head
     const int tid = threadIdx.x;
     const int p = tid % LPR;
     const int rg = tid / LPR;
@@ -78,8 +79,8 @@ decode_step_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k,
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
         const int col = 4 * (p + LPR * m);
-        load4(k + nh * DK + col, kf + 4 * m);
-        load4(q + nh * DK + col, qf + 4 * m);
+        load4(k + qh * DK + col, kf + 4 * m);
+        load4(q + qh * DK + col, qf + 4 * m);
     }
     float af[CHANNEL ? 16 : 1];
     if constexpr (CHANNEL) {
@@ -140,24 +141,24 @@ decode_step_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k,
 
 template <int DK, bool CHANNEL, typename IoT>
 cudaError_t launch_dk(const void *q, const void *k, const void *v, const float *g,
-                      const float *beta, float *state, int N, int H, int DV, void *o,
+                      const float *beta, float *state, int N, int Hqk, int H, int DV, void *o,
                       cudaStream_t stream) {
     const unsigned blocks = (unsigned)((size_t)N * H);
     decode_step_kernel<DK, CHANNEL, IoT><<<blocks, kDecodeThreads, 0, stream>>>(
         static_cast<const IoT *>(q), static_cast<const IoT *>(k), static_cast<const IoT *>(v), g,
-        beta, state, DV, static_cast<IoT *>(o));
+        beta, state, Hqk, H, DV, static_cast<IoT *>(o));
     return cudaGetLastError();
 }
 
 template <bool CHANNEL, typename IoT>
 cudaError_t launch_mode(const void *q, const void *k, const void *v, const float *g,
-                        const float *beta, float *state, int N, int H, int DK, int DV,
-                        void *o, cudaStream_t stream) {
+                        const float *beta, float *state, int N, int Hqk, int H, int DK,
+                        int DV, void *o, cudaStream_t stream) {
     switch (DK) {
-        case 16: return launch_dk<16, CHANNEL, IoT>(q, k, v, g, beta, state, N, H, DV, o, stream);
-        case 32: return launch_dk<32, CHANNEL, IoT>(q, k, v, g, beta, state, N, H, DV, o, stream);
-        case 64: return launch_dk<64, CHANNEL, IoT>(q, k, v, g, beta, state, N, H, DV, o, stream);
-        default: return launch_dk<128, CHANNEL, IoT>(q, k, v, g, beta, state, N, H, DV, o, stream);
+        case 16: return launch_dk<16, CHANNEL, IoT>(q, k, v, g, beta, state, N, Hqk, H, DV, o, stream);
+        case 32: return launch_dk<32, CHANNEL, IoT>(q, k, v, g, beta, state, N, Hqk, H, DV, o, stream);
+        case 64: return launch_dk<64, CHANNEL, IoT>(q, k, v, g, beta, state, N, Hqk, H, DV, o, stream);
+        default: return launch_dk<128, CHANNEL, IoT>(q, k, v, g, beta, state, N, Hqk, H, DV, o, stream);
     }
 }
 
@@ -165,14 +166,14 @@ cudaError_t launch_mode(const void *q, const void *k, const void *v, const float
 
 // Host launcher (arguments already validated by the C ABI layer).
 cudaError_t launch_decode_step(const void *q, const void *k, const void *v, const float *g,
-                               const float *beta, float *state, int N, int H, int DK, int DV,
-                               bool channel, bool bf16, void *o, cudaStream_t stream) {
+                               const float *beta, float *state, int N, int Hqk, int H, int DK,
+                               int DV, bool channel, bool bf16, void *o, cudaStream_t stream) {
     if (N == 0 || H == 0) return cudaSuccess;
     if (channel)
-        return bf16 ? launch_mode<true, __nv_bfloat16>(q, k, v, g, beta, state, N, H, DK, DV, o, stream)
-                    : launch_mode<true, float>(q, k, v, g, beta, state, N, H, DK, DV, o, stream);
-    return bf16 ? launch_mode<false, __nv_bfloat16>(q, k, v, g, beta, state, N, H, DK, DV, o, stream)
-                : launch_mode<false, float>(q, k, v, g, beta, state, N, H, DK, DV, o, stream);
+        return bf16 ? launch_mode<true, __nv_bfloat16>(q, k, v, g, beta, state, N, Hqk, H, DK, DV, o, stream)
+                    : launch_mode<true, float>(q, k, v, g, beta, state, N, Hqk, H, DK, DV, o, stream);
+    return bf16 ? launch_mode<false, __nv_bfloat16>(q, k, v, g, beta, state, N, Hqk, H, DK, DV, o, stream)
+                : launch_mode<false, float>(q, k, v, g, beta, state, N, Hqk, H, DK, DV, o, stream);
 }
 
 }  // namespace gdr

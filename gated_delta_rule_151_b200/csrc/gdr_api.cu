@@ -69,13 +69,15 @@ gdr_status_t gdr_prefill_workspace_size(int32_t num_seqs, int32_t total_T, int32
     return GDR_OK;
 }
 
-gdr_status_t gdr_prefill_chunked(const void *q, const void *k, const void *v, const float *g,
-                                 const float *beta, const float *initial_state,
-                                 const int32_t *cu_seqlens, int32_t num_seqs, int32_t total_T,
-                                 int32_t H, int32_t d_k, int32_t d_v, gdr_gate_mode_t gate_mode,
-                                 gdr_dtype_t io_dtype, void *o, float *final_state,
-                                 void *workspace, size_t workspace_bytes, void *stream) {
-    if (num_seqs < 0 || total_T < 0 || H < 1) return GDR_ERR_INVALID_ARG;
+gdr_status_t gdr_prefill_chunked_gqa(const void *q, const void *k, const void *v,
+                                     const float *g, const float *beta,
+                                     const float *initial_state, const int32_t *cu_seqlens,
+                                     int32_t num_seqs, int32_t total_T, int32_t H_qk, int32_t H,
+                                     int32_t d_k, int32_t d_v, gdr_gate_mode_t gate_mode,
+                                     gdr_dtype_t io_dtype, void *o, float *final_state,
+                                     void *workspace, size_t workspace_bytes, void *stream) {
+    if (num_seqs < 0 || total_T < 0 || H < 1 || H_qk < 1 || H % H_qk != 0)
+        return GDR_ERR_INVALID_ARG;
     if (!valid_dim(d_k) || !valid_dim(d_v)) return GDR_ERR_INVALID_ARG;
     if (gate_mode != GDR_GATE_SCALAR && gate_mode != GDR_GATE_CHANNEL) return GDR_ERR_INVALID_ARG;
     if (io_dtype != GDR_F32 && io_dtype != GDR_BF16) return GDR_ERR_INVALID_ARG;
@@ -106,11 +108,22 @@ gdr_status_t gdr_prefill_chunked(const void *q, const void *k, const void *v, co
     const bool channel = gate_mode == GDR_GATE_CHANNEL;
     if (uses_tcgen05(d_k, d_v, gate_mode, io_dtype))
         return from_cuda(gdr::launch_prefill_tcgen05(q, k, v, g, beta, initial_state, cu_seqlens,
-                                                      num_seqs, total_T, H, channel, o,
+                                                      num_seqs, total_T, H_qk, H, channel, o,
                                                       final_state, workspace, s));
     return from_cuda(gdr::launch_prefill_simt(q, k, v, g, beta, initial_state, cu_seqlens,
-                                              num_seqs, total_T, H, d_k, d_v, channel,
+                                              num_seqs, total_T, H_qk, H, d_k, d_v, channel,
                                               io_dtype == GDR_BF16, o, final_state, s));
+}
+
+gdr_status_t gdr_prefill_chunked(const void *q, const void *k, const void *v, const float *g,
+                                 const float *beta, const float *initial_state,
+                                 const int32_t *cu_seqlens, int32_t num_seqs, int32_t total_T,
+                                 int32_t H, int32_t d_k, int32_t d_v, gdr_gate_mode_t gate_mode,
+                                 gdr_dtype_t io_dtype, void *o, float *final_state,
+                                 void *workspace, size_t workspace_bytes, void *stream) {
+    return gdr_prefill_chunked_gqa(q, k, v, g, beta, initial_state, cu_seqlens, num_seqs, total_T,
+                                   H, H, d_k, d_v, gate_mode, io_dtype, o, final_state, workspace,
+                                   workspace_bytes, stream);
 }
 
 gdr_status_t gdr_prefill_check_workspace(const void *workspace, size_t workspace_bytes,
@@ -125,11 +138,11 @@ gdr_status_t gdr_prefill_check_workspace(const void *workspace, size_t workspace
     return word == 0 ? GDR_OK : GDR_ERR_DEVICE_TIMEOUT;
 }
 
-gdr_status_t gdr_decode_step(const void *q, const void *k, const void *v, const float *g,
-                             const float *beta, float *state, int32_t N, int32_t H, int32_t d_k,
-                             int32_t d_v, gdr_gate_mode_t gate_mode, gdr_dtype_t io_dtype,
-                             void *o, void *stream) {
-    if (N < 0 || H < 0) return GDR_ERR_INVALID_ARG;
+gdr_status_t gdr_decode_step_gqa(const void *q, const void *k, const void *v, const float *g,
+                                 const float *beta, float *state, int32_t N, int32_t H_qk,
+                                 int32_t H, int32_t d_k, int32_t d_v, gdr_gate_mode_t gate_mode,
+                                 gdr_dtype_t io_dtype, void *o, void *stream) {
+    if (N < 0 || H < 0 || H_qk < 1 || (H > 0 && H % H_qk != 0)) return GDR_ERR_INVALID_ARG;
     if (!valid_dim(d_k) || !valid_dim(d_v)) return GDR_ERR_INVALID_ARG;
     if (gate_mode != GDR_GATE_SCALAR && gate_mode != GDR_GATE_CHANNEL) return GDR_ERR_INVALID_ARG;
     if (io_dtype != GDR_F32 && io_dtype != GDR_BF16) return GDR_ERR_INVALID_ARG;
@@ -138,10 +151,19 @@ gdr_status_t gdr_decode_step(const void *q, const void *k, const void *v, const 
     if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_gate_ptr(g, gate_mode) ||
         !ok_beta_ptr(beta) || !ok_ptr(state) || !ok_ptr(o))
         return GDR_ERR_INVALID_ARG;
-    return from_cuda(gdr::launch_decode_step(q, k, v, g, beta, state, N, H, d_k, d_v,
+    return from_cuda(gdr::launch_decode_step(q, k, v, g, beta, state, N, H_qk, H, d_k, d_v,
                                              gate_mode == GDR_GATE_CHANNEL,
                                              io_dtype == GDR_BF16, o,
                                              static_cast<cudaStream_t>(stream)));
+}
+
+gdr_status_t gdr_decode_step(const void *q, const void *k, const void *v, const float *g,
+                             const float *beta, float *state, int32_t N, int32_t H, int32_t d_k,
+                             int32_t d_v, gdr_gate_mode_t gate_mode, gdr_dtype_t io_dtype,
+                             void *o, void *stream) {
+    if (H < 0) return GDR_ERR_INVALID_ARG;
+    return gdr_decode_step_gqa(q, k, v, g, beta, state, N, H > 0 ? H : 1, H, d_k, d_v, gate_mode,
+                               io_dtype, o, stream);
 }
 
 }  // extern "C"

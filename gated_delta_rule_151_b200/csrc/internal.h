@@ -7,14 +7,17 @@
 
 namespace gdr {
 
+// H counts value heads (one state each); the Hqk query/key heads each serve
+// H / Hqk consecutive value heads.
 cudaError_t launch_decode_step(const void *q, const void *k, const void *v, const float *g,
-                               const float *beta, float *state, int N, int H, int DK, int DV,
-                               bool channel, bool bf16, void *o, cudaStream_t stream);
+                               const float *beta, float *state, int N, int Hqk, int H, int DK,
+                               int DV, bool channel, bool bf16, void *o, cudaStream_t stream);
 
 cudaError_t launch_prefill_simt(const void *q, const void *k, const void *v, const float *g,
                                 const float *beta, const float *h0, const int32_t *cu,
-                                int num_seqs, int total_T, int H, int DK, int DV, bool channel,
-                                bool bf16, void *o, float *fin, cudaStream_t stream);
+                                int num_seqs, int total_T, int Hqk, int H, int DK, int DV,
+                                bool channel, bool bf16, void *o, float *fin,
+                                cudaStream_t stream);
 
 size_t prefill_simt_smem_bytes(int DK, int DV);
 
@@ -24,7 +27,7 @@ bool tcgen05_prefill_serves(bool channel);
 size_t tcgen05_workspace_bytes(int num_seqs, int total_T, int H);
 cudaError_t launch_prefill_tcgen05(const void *q, const void *k, const void *v, const float *g,
                                    const float *beta, const float *h0, const int32_t *cu,
-                                   int num_seqs, int total_T, int H, bool channel, void *o,
-                                   float *fin, void *workspace, cudaStream_t stream);
+                                   int num_seqs, int total_T, int Hqk, int H, bool channel,
+                                   void *o, float *fin, void *workspace, cudaStream_t stream);
 
 }  // namespace gdr

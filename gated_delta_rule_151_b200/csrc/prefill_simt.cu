@@ -76,11 +76,12 @@ __global__ void __launch_bounds__(kSimtThreads)
 prefill_simt_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k,
                     const IoT *__restrict__ v, const float *__restrict__ g,
                     const float *__restrict__ beta, const float *h0,
-                    const int32_t *__restrict__ cu, int num_seqs, int total_T, int H, int DK,
-                    int DV, int VS, int nslabs, IoT *__restrict__ o, float *fin) {
+                    const int32_t *__restrict__ cu, int num_seqs, int total_T, int Hqk, int H,
+                    int DK, int DV, int VS, int nslabs, IoT *__restrict__ o, float *fin) {
     const int slab = blockIdx.x % nslabs;
-    const int h = (blockIdx.x / nslabs) % H;
+    const int h = (blockIdx.x / nslabs) % H;          // value head
     const int n = blockIdx.x / (nslabs * H);
+    const int hq = h / (H / Hqk);                      // its query/key head
     const int r0 = slab * VS;
     const int nv = min(VS, DV - r0);
     const int tid = threadIdx.x;
@@ -111,8 +112,9 @@ prefill_simt_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k,
             const int i = idx / DK, c = idx % DK;
             const bool ok = i < cl;
             const size_t row = ((size_t)(t0 + c0 + i) * H + h);
-            Ks[i * KS + c] = ok ? to_f32(k[row * DK + c]) : 0.f;
-            Qs[i * KS + c] = ok ? to_f32(q[row * DK + c]) : 0.f;
+            const size_t qrow = ((size_t)(t0 + c0 + i) * Hqk + hq);
+            Ks[i * KS + c] = ok ? to_f32(k[qrow * DK + c]) : 0.f;
+            Qs[i * KS + c] = ok ? to_f32(q[qrow * DK + c]) : 0.f;
             if (CHANNEL) Xs[i * KS + c] = ok ? clamp_log_gate(g[row * DK + c]) : 0.f;
         }
         for (int idx = tid; idx < C * VS; idx += kSimtThreads) {
@@ -243,7 +245,7 @@ prefill_simt_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k,
 template <bool CHANNEL, typename IoT>
 cudaError_t launch_typed(const void *q, const void *k, const void *v, const float *g,
                          const float *beta, const float *h0, const int32_t *cu, int num_seqs,
-                         int total_T, int H, int DK, int DV, void *o, float *fin,
+                         int total_T, int Hqk, int H, int DK, int DV, void *o, float *fin,
                          cudaStream_t stream) {
     const int VS = DV < 32 ? DV : 32;
     const int nslabs = (DV + VS - 1) / VS;
@@ -257,7 +259,7 @@ cudaError_t launch_typed(const void *q, const void *k, const void *v, const floa
     if (blocks > 0x7fffffffull) return cudaErrorInvalidConfiguration;
     kern<<<(unsigned)blocks, kSimtThreads, L.total, stream>>>(
         static_cast<const IoT *>(q), static_cast<const IoT *>(k), static_cast<const IoT *>(v), g,
-        beta, h0, cu, num_seqs, total_T, H, DK, DV, VS, nslabs, static_cast<IoT *>(o), fin);
+        beta, h0, cu, num_seqs, total_T, Hqk, H, DK, DV, VS, nslabs, static_cast<IoT *>(o), fin);
     return cudaGetLastError();
 }
 
@@ -265,13 +267,14 @@ cudaError_t launch_typed(const void *q, const void *k, const void *v, const floa
 
 cudaError_t launch_prefill_simt(const void *q, const void *k, const void *v, const float *g,
                                 const float *beta, const float *h0, const int32_t *cu,
-                                int num_seqs, int total_T, int H, int DK, int DV, bool channel,
-                                bool bf16, void *o, float *fin, cudaStream_t stream) {
+                                int num_seqs, int total_T, int Hqk, int H, int DK, int DV,
+                                bool channel, bool bf16, void *o, float *fin,
+                                cudaStream_t stream) {
     if (channel)
-        return bf16 ? launch_typed<true, __nv_bfloat16>(q, k, v, g, beta, h0, cu, num_seqs, total_T, H, DK, DV, o, fin, stream)
-                    : launch_typed<true, float>(q, k, v, g, beta, h0, cu, num_seqs, total_T, H, DK, DV, o, fin, stream);
-    return bf16 ? launch_typed<false, __nv_bfloat16>(q, k, v, g, beta, h0, cu, num_seqs, total_T, H, DK, DV, o, fin, stream)
-                : launch_typed<false, float>(q, k, v, g, beta, h0, cu, num_seqs, total_T, H, DK, DV, o, fin, stream);
+        return bf16 ? launch_typed<true, __nv_bfloat16>(q, k, v, g, beta, h0, cu, num_seqs, total_T, Hqk, H, DK, DV, o, fin, stream)
+                    : launch_typed<true, float>(q, k, v, g, beta, h0, cu, num_seqs, total_T, Hqk, H, DK, DV, o, fin, stream);
+    return bf16 ? launch_typed<false, __nv_bfloat16>(q, k, v, g, beta, h0, cu, num_seqs, total_T, Hqk, H, DK, DV, o, fin, stream)
+                : launch_typed<false, float>(q, k, v, g, beta, h0, cu, num_seqs, total_T, Hqk, H, DK, DV, o, fin, stream);
 }
 
 size_t prefill_simt_smem_bytes(int DK, int DV) {

@@ -295,7 +295,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const float *__restrict__ g,
                   const float *__restrict__ beta, const float *h0,
-                  const int32_t *__restrict__ cu, int num_seqs, int total_T, int H,
+                  const int32_t *__restrict__ cu, int num_seqs, int total_T, int Hqk, int H,
                   __nv_bfloat16 *__restrict__ o, float *fin, uint32_t *err) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t sbase = smem_u32(smem_raw);
@@ -306,8 +306,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     uint8_t *sm = smem_raw;
     Misc *m = reinterpret_cast<Misc *>(sm + OFF_MISC);
 
-    const int h = blockIdx.x % H;
+    const int h = blockIdx.x % H;          // value head
     const int n = blockIdx.x / H;
+    const int hq = h / (H / Hqk);          // its query/key head
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
     const int sub = warp & 3;           // TMEM sub-partition of this warp
@@ -522,19 +523,19 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             const int tok0 = t0 + c * C;
             if (c + 1 < nchunks) {       // warm L2 with the chunk after this one
                 const int t1 = tok0 + C;
-                tma_prefetch_l2_3d(&tm_k, 0, h, t1);
-                tma_prefetch_l2_3d(&tm_k, 64, h, t1);
-                tma_prefetch_l2_3d(&tm_q, 0, h, t1);
-                tma_prefetch_l2_3d(&tm_q, 64, h, t1);
+                tma_prefetch_l2_3d(&tm_k, 0, hq, t1);
+                tma_prefetch_l2_3d(&tm_k, 64, hq, t1);
+                tma_prefetch_l2_3d(&tm_q, 0, hq, t1);
+                tma_prefetch_l2_3d(&tm_q, 64, hq, t1);
                 tma_prefetch_l2_3d(&tm_v, 0, h, t1);
                 tma_prefetch_l2_3d(&tm_v, 64, h, t1);
             }
             fence_proxy_async();
             mbar_arrive_expect_tx(&m->bar_tma, 6 * 8192);
-            tma_load_3d(sm + OFF_KQ + 0, &tm_k, &m->bar_tma, 0, h, tok0);
-            tma_load_3d(sm + OFF_KQ + 16384, &tm_k, &m->bar_tma, 64, h, tok0);
-            tma_load_3d(sm + OFF_KQ + 8192, &tm_q, &m->bar_tma, 0, h, tok0);
-            tma_load_3d(sm + OFF_KQ + 24576, &tm_q, &m->bar_tma, 64, h, tok0);
+            tma_load_3d(sm + OFF_KQ + 0, &tm_k, &m->bar_tma, 0, hq, tok0);
+            tma_load_3d(sm + OFF_KQ + 16384, &tm_k, &m->bar_tma, 64, hq, tok0);
+            tma_load_3d(sm + OFF_KQ + 8192, &tm_q, &m->bar_tma, 0, hq, tok0);
+            tma_load_3d(sm + OFF_KQ + 24576, &tm_q, &m->bar_tma, 64, hq, tok0);
             tma_load_3d(sm + OFF_V + 0, &tm_v, &m->bar_tma, 0, h, tok0);
             tma_load_3d(sm + OFF_V + 8192, &tm_v, &m->bar_tma, 64, h, tok0);
         };
@@ -911,19 +912,20 @@ size_t tcgen05_workspace_bytes(int, int, int) { return 16; }
 
 cudaError_t launch_prefill_tcgen05(const void *q, const void *k, const void *v, const float *g,
                                    const float *beta, const float *h0, const int32_t *cu,
-                                   int num_seqs, int total_T, int H, bool channel, void *o,
-                                   float *fin, void *workspace, cudaStream_t stream) {
+                                   int num_seqs, int total_T, int Hqk, int H, bool channel,
+                                   void *o, float *fin, void *workspace, cudaStream_t stream) {
     uint32_t *err = static_cast<uint32_t *>(workspace);
     cudaError_t e = cudaMemsetAsync(err, 0, sizeof(uint32_t), stream);
     if (e != cudaSuccess) return e;
     if ((size_t)num_seqs * H == 0) return cudaSuccess;
     if (total_T == 0) {
         // nothing to stage: the state passes through unchanged
-        return launch_prefill_simt(q, k, v, g, beta, h0, cu, num_seqs, total_T, H, D, D, channel,
-                                   true, o, fin, stream);
+        return launch_prefill_simt(q, k, v, g, beta, h0, cu, num_seqs, total_T, Hqk, H, D, D,
+                                   channel, true, o, fin, stream);
     }
     CUtensorMap mq, mk, mv;
-    if (!make_map(&mq, q, total_T, H) || !make_map(&mk, k, total_T, H) || !make_map(&mv, v, total_T, H))
+    if (!make_map(&mq, q, total_T, Hqk) || !make_map(&mk, k, total_T, Hqk) ||
+        !make_map(&mv, v, total_T, H))
         return cudaErrorInvalidValue;
     auto kern = channel ? prefill_tc_kernel<true> : prefill_tc_kernel<false>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
@@ -931,8 +933,8 @@ cudaError_t launch_prefill_tcgen05(const void *q, const void *k, const void *v, 
     const size_t blocks = (size_t)num_seqs * H;
     if (blocks > 0x7fffffffull) return cudaErrorInvalidConfiguration;
     kern<<<(unsigned)blocks, kThreads, SMEM_BYTES, stream>>>(
-        mq, mk, mv, g, beta, h0, cu, num_seqs, total_T, H, static_cast<__nv_bfloat16 *>(o), fin,
-        err);
+        mq, mk, mv, g, beta, h0, cu, num_seqs, total_T, Hqk, H, static_cast<__nv_bfloat16 *>(o),
+        fin, err);
     return cudaGetLastError();
 }
 

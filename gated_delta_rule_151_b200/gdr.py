@@ -34,7 +34,7 @@ GDR_PATH_TCGEN05 = 1
 # Every symbol include/gdr.h declares.
 EXPORTED = ("gdr_status_string", "gdr_prefill_workspace_size", "gdr_prefill_path",
             "gdr_prefill_chunked", "gdr_prefill_check_workspace", "gdr_decode_step",
-            "gdr_prefill_chunked_noalloc")
+            "gdr_prefill_chunked_noalloc", "gdr_prefill_chunked_gqa", "gdr_decode_step_gqa")
 
 
 class GdrError(RuntimeError):
@@ -76,6 +76,11 @@ def load_library():
         lib.gdr_prefill_chunked_noalloc.argtypes = [P, P, P, P, P, P, P, I32, I32, I32, I32, I32,
                                                     ST, ST, P, P, P]
         lib.gdr_prefill_chunked_noalloc.restype = ST
+        lib.gdr_prefill_chunked_gqa.argtypes = [P, P, P, P, P, P, P, I32, I32, I32, I32, I32, I32,
+                                                ST, ST, P, P, P, SZ, P]
+        lib.gdr_prefill_chunked_gqa.restype = ST
+        lib.gdr_decode_step_gqa.argtypes = [P, P, P, P, P, P, I32, I32, I32, I32, I32, ST, ST, P, P]
+        lib.gdr_decode_step_gqa.restype = ST
         _lib = lib
         return lib
 
@@ -141,26 +146,16 @@ def gdr_prefill_path(d_k, d_v, gate_mode, io_dtype) -> int:
     return int(out.value)
 
 
-def gdr_prefill_chunked(q, k, v, g, beta, initial_state=None, cu_seqlens=None, *,
-                        num_seqs=None, o=None, final_state=None, output_final_state=True,
-                        workspace=None, stream=None):
-    """Chunked prefill (see include/gdr.h).  Returns (o, final_state).
-
-    q, k [T, H, d_k], v [T, H, d_v] (bf16 or fp32); g [T, H] or [T, H, d_k]
-    fp32; beta [T, H] fp32; initial_state [N, H, d_v, d_k] fp32 or None;
-    cu_seqlens int32 [N + 1] on the device, or None with ``num_seqs`` equal
-    sequences (default 1).  ``final_state`` may be given (it may be the same
-    tensor as initial_state); otherwise one is allocated when
-    ``output_final_state``.
-    """
+def _prefill(name, q, k, v, g, beta, initial_state, cu_seqlens, num_seqs, o, final_state,
+             output_final_state, workspace, stream):
     _need(q, "q", ndim=3)
     io = q.dtype
     _need(k, "k", io, 3)
     _need(v, "v", io, 3)
     _need(beta, "beta", torch.float32, 2)
     _need(g, "g", torch.float32)
-    T, H, dk = q.shape
-    dv = v.shape[2]
+    T, Hqk, dk = q.shape
+    H, dv = v.shape[1], v.shape[2]
     if g.dim() == 2:
         gate = GDR_GATE_SCALAR
     elif g.dim() == 3:
@@ -185,12 +180,41 @@ def gdr_prefill_chunked(q, k, v, g, beta, initial_state=None, cu_seqlens=None, *
     ws_bytes = gdr_prefill_workspace_size(N, T, H, dk, dv, gate, io_code)
     if ws_bytes and workspace is None:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
-    st = load_library().gdr_prefill_chunked(
+    lib = load_library()
+    heads = (Hqk, H) if name == "gdr_prefill_chunked_gqa" else (H,)
+    if name == "gdr_prefill_chunked" and Hqk != H:
+        raise ValueError("q/k and v head counts differ: use gdr_prefill_chunked_gqa")
+    st = getattr(lib, name)(
         _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(initial_state), _ptr(cu_seqlens),
-        N, T, H, dk, dv, gate, io_code, _ptr(o), _ptr(final_state), _ptr(workspace),
+        N, T, *heads, dk, dv, gate, io_code, _ptr(o), _ptr(final_state), _ptr(workspace),
         workspace.numel() if workspace is not None else 0, _stream_ptr(stream))
-    _check(st, "gdr_prefill_chunked")
+    _check(st, name)
     return o, final_state
+
+
+def gdr_prefill_chunked(q, k, v, g, beta, initial_state=None, cu_seqlens=None, *,
+                        num_seqs=None, o=None, final_state=None, output_final_state=True,
+                        workspace=None, stream=None):
+    """Chunked prefill (see include/gdr.h).  Returns (o, final_state).
+
+    q, k [T, H, d_k], v [T, H, d_v] (bf16 or fp32); g [T, H] or [T, H, d_k]
+    fp32; beta [T, H] fp32; initial_state [N, H, d_v, d_k] fp32 or None;
+    cu_seqlens int32 [N + 1] on the device, or None with ``num_seqs`` equal
+    sequences (default 1).  ``final_state`` may be given (it may be the same
+    tensor as initial_state); otherwise one is allocated when
+    ``output_final_state``.
+    """
+    return _prefill("gdr_prefill_chunked", q, k, v, g, beta, initial_state, cu_seqlens, num_seqs,
+                    o, final_state, output_final_state, workspace, stream)
+
+
+def gdr_prefill_chunked_gqa(q, k, v, g, beta, initial_state=None, cu_seqlens=None, *,
+                            num_seqs=None, o=None, final_state=None, output_final_state=True,
+                            workspace=None, stream=None):
+    """Chunked prefill with grouped query/key heads: q, k [T, H_qk, d_k],
+    everything else per value head [T, H, ...]; H_qk divides H."""
+    return _prefill("gdr_prefill_chunked_gqa", q, k, v, g, beta, initial_state, cu_seqlens,
+                    num_seqs, o, final_state, output_final_state, workspace, stream)
 
 
 def gdr_prefill_check_workspace(workspace, stream=None):
@@ -199,12 +223,7 @@ def gdr_prefill_check_workspace(workspace, stream=None):
         "gdr_prefill_check_workspace")
 
 
-def gdr_decode_step(q, k, v, g, beta, state, *, o=None, stream=None):
-    """One decode step (see include/gdr.h): state is updated in place.
-
-    q, k [N, H, d_k], v [N, H, d_v] (bf16 or fp32); g [N, H] or [N, H, d_k]
-    fp32; beta [N, H] fp32; state [N, H, d_v, d_k] fp32.  Returns o [N, H, d_v].
-    """
+def _decode(name, q, k, v, g, beta, state, o, stream):
     _need(q, "q", ndim=3)
     io = q.dtype
     _need(k, "k", io, 3)
@@ -212,17 +231,34 @@ def gdr_decode_step(q, k, v, g, beta, state, *, o=None, stream=None):
     _need(beta, "beta", torch.float32, 2)
     _need(g, "g", torch.float32)
     _need(state, "state", torch.float32, 4)
-    N, H, dk = q.shape
-    dv = v.shape[2]
+    N, Hqk, dk = q.shape
+    H, dv = v.shape[1], v.shape[2]
     gate = GDR_GATE_SCALAR if g.dim() == 2 else GDR_GATE_CHANNEL
     if o is None:
         o = torch.empty((N, H, dv), dtype=io, device=q.device)
     _need(o, "o", io, 3)
-    st = load_library().gdr_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
-                                        _ptr(state), N, H, dk, dv, gate, _io_code(io), _ptr(o),
-                                        _stream_ptr(stream))
-    _check(st, "gdr_decode_step")
+    if name == "gdr_decode_step" and Hqk != H:
+        raise ValueError("q/k and v head counts differ: use gdr_decode_step_gqa")
+    heads = (Hqk, H) if name == "gdr_decode_step_gqa" else (H,)
+    st = getattr(load_library(), name)(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                       _ptr(state), N, *heads, dk, dv, gate, _io_code(io), _ptr(o),
+                                       _stream_ptr(stream))
+    _check(st, name)
     return o
+
+
+def gdr_decode_step(q, k, v, g, beta, state, *, o=None, stream=None):
+    """One decode step (see include/gdr.h): state is updated in place.
+
+    q, k [N, H, d_k], v [N, H, d_v] (bf16 or fp32); g [N, H] or [N, H, d_k]
+    fp32; beta [N, H] fp32; state [N, H, d_v, d_k] fp32.  Returns o [N, H, d_v].
+    """
+    return _decode("gdr_decode_step", q, k, v, g, beta, state, o, stream)
+
+
+def gdr_decode_step_gqa(q, k, v, g, beta, state, *, o=None, stream=None):
+    """One decode step with grouped query/key heads: q, k [N, H_qk, d_k]."""
+    return _decode("gdr_decode_step_gqa", q, k, v, g, beta, state, o, stream)
 
 
 def gdr_prefill_chunked_noalloc(q, k, v, g, beta, initial_state=None, cu_seqlens=None, *,

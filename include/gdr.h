@@ -139,6 +139,24 @@ GDR_API gdr_status_t gdr_prefill_chunked(const void *q, const void *k, const voi
                                  void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * gdr_prefill_chunked with grouped query/key heads: q and k are
+ * [T, H_qk, d_k] while v, o, g, beta and the states carry H value heads
+ * (H_qk divides H); value head h reads query/key head h / (H / H_qk).  This
+ * is the head layout of the Qwen Gated DeltaNet layer, 16 query-key heads for
+ * 48 value heads (page "Qwen3.8-Flash-Next and GLM-5.3-Flash ...", section
+ * "Gated DeltaNet carries most of the sequence").  H_qk == H is exactly
+ * gdr_prefill_chunked.  The workspace size is the one
+ * gdr_prefill_workspace_size reports for H value heads.
+ */
+GDR_API gdr_status_t gdr_prefill_chunked_gqa(const void *q, const void *k, const void *v,
+                                     const float *g, const float *beta,
+                                     const float *initial_state, const int32_t *cu_seqlens,
+                                     int32_t num_seqs, int32_t total_T, int32_t H_qk, int32_t H,
+                                     int32_t d_k, int32_t d_v, gdr_gate_mode_t gate_mode,
+                                     gdr_dtype_t io_dtype, void *o, float *final_state,
+                                     void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * After gdr_prefill_chunked's work on `stream` has finished, reports whether a
  * bounded device-side wait in it gave up (GDR_ERR_DEVICE_TIMEOUT) or not
  * (GDR_OK).  Synchronises `stream` and copies one word from `workspace`.
@@ -191,6 +209,18 @@ GDR_API gdr_status_t gdr_decode_step(const void *q, const void *k, const void *v
                              int32_t N, int32_t H, int32_t d_k, int32_t d_v,
                              gdr_gate_mode_t gate_mode, gdr_dtype_t io_dtype,
                              void *o, void *stream);
+
+/*
+ * gdr_decode_step with grouped query/key heads: q, k [N, H_qk, d_k];
+ * v, o [N, H, d_v]; g, beta, state per value head (H_qk divides H); value
+ * head h reads query/key head h / (H / H_qk) -- the same grouping as
+ * gdr_prefill_chunked_gqa.  H_qk == H is exactly gdr_decode_step.
+ */
+GDR_API gdr_status_t gdr_decode_step_gqa(const void *q, const void *k, const void *v,
+                                 const float *g, const float *beta, float *state, int32_t N,
+                                 int32_t H_qk, int32_t H, int32_t d_k, int32_t d_v,
+                                 gdr_gate_mode_t gate_mode, gdr_dtype_t io_dtype, void *o,
+                                 void *stream);
 
 #ifdef __cplusplus
 }

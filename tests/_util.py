@@ -32,9 +32,9 @@ def to_device(inp, device="cuda"):
 def gpu_prefill(inp, use_cu=True, initial_state="h0", final_state=None):
     d = to_device(inp)
     h0 = d["h0"] if initial_state == "h0" else initial_state
-    o, fin = gdr.gdr_prefill_chunked(d["q"], d["k"], d["v"], d["g"], d["beta"], h0,
-                                     d["cu"] if use_cu else None,
-                                     num_seqs=inp.num_seqs, final_state=final_state)
+    fn = gdr.gdr_prefill_chunked if inp.H_qk == inp.H else gdr.gdr_prefill_chunked_gqa
+    o, fin = fn(d["q"], d["k"], d["v"], d["g"], d["beta"], h0, d["cu"] if use_cu else None,
+                num_seqs=inp.num_seqs, final_state=final_state)
     torch.cuda.synchronize()
     return o, fin
 

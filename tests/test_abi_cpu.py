@@ -115,3 +115,18 @@ def test_binding_refuses_cpu_tensors():
     x = torch.zeros(4, 2, 16)
     with pytest.raises(ValueError):
         gdr.gdr_prefill_chunked(x, x, x, torch.zeros(4, 2), torch.zeros(4, 2))
+
+
+def _prefill_gqa(lib, Hqk, H):
+    P = ctypes.c_void_p
+    return lib.gdr_prefill_chunked_gqa(P(A), P(A), P(A), P(A), P(A), None, None, 1, 64, Hqk, H,
+                                       128, 128, 0, 1, P(A), P(A), None, 0, None)
+
+
+@pytest.mark.parametrize("Hqk,H", [(0, 4), (3, 4), (8, 4), (-1, 2)])
+def test_grouped_heads_must_divide(lib, Hqk, H):
+    assert _prefill_gqa(lib, Hqk, H) == gdr.GDR_ERR_INVALID_ARG
+    P = ctypes.c_void_p
+    st = lib.gdr_decode_step_gqa(P(A), P(A), P(A), P(A), P(A), P(A), 2, Hqk, H, 128, 128, 0, 1,
+                                 P(A), None)
+    assert st == gdr.GDR_ERR_INVALID_ARG
