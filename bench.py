@@ -271,7 +271,62 @@ class DecodeCase:
         return "f32"
 
 
+class SpecDecodeCase(DecodeCase):
+    """Draft verification: each launch applies SPEC_DRAFT consecutive tokens of
+    every sequence (gdr_decode_multi); a step is the 512 tokens of each
+    sequence, i.e. 512 / SPEC_DRAFT launches."""
+
+    def __init__(self, name, device, seed):
+        self.name = name
+        self.inp = inp = I.workload(name, seed=seed)
+        self.dev = device
+        N, T = inp.num_seqs, I.SPEC_DRAFT
+        L = inp.total_T // N
+        self.T, self.steps = T, L // T
+
+        def grp(x):   # [N*L, ...] -> [steps, N, T, ...] contiguous per launch
+            return x.reshape(N, self.steps, T, *x.shape[1:]).transpose(0, 1).contiguous().to(device)
+        self.q, self.k, self.v, self.g, self.beta = (grp(x) for x in (inp.q, inp.k, inp.v, inp.g,
+                                                                      inp.beta))
+        self.state = inp.h0.to(device).clone()
+        self.o = torch.empty((self.steps, N, T, inp.H, inp.d_v), dtype=inp.io_dtype, device=device)
+        e = io_bytes(inp.io_dtype)
+        gate = 4 * (inp.d_k if inp.gate_mode == I.CHANNEL else 1)
+        self.bytes = N * inp.H * (2 * 4 * inp.d_k * inp.d_v +
+                                  T * (e * (2 * inp.d_k + 2 * inp.d_v) + 4 + gate))
+        self.flops = 0
+        self.tokens = inp.total_T
+        self.launches = self.steps
+        self.path = None
+
+    def step(self, stream=None):
+        for t in range(self.steps):
+            gdr.gdr_decode_multi(self.q[t], self.k[t], self.v[t], self.g[t], self.beta[t],
+                                 self.state, o=self.o[t], stream=stream)
+
+    def e2e_buffers(self):
+        host = {k: v.cpu().pin_memory() for k, v in
+                dict(q=self.q, k=self.k, v=self.v, g=self.g, beta=self.beta).items()}
+        ho = torch.empty(self.o.shape, dtype=self.o.dtype).pin_memory()
+        h2d = sum(v.numel() * v.element_size() for v in host.values())
+        d2h = ho.numel() * ho.element_size()
+        self._dev_tok = {k: torch.empty(v.shape[1:], dtype=v.dtype, device=self.dev)
+                         for k, v in host.items()}
+        return host, ho, None, h2d, d2h
+
+    def e2e_step(self, host, host_o, host_fin, stream):
+        dt = self._dev_tok
+        for t in range(self.steps):
+            for key in dt:
+                dt[key].copy_(host[key][t], non_blocking=True)
+            gdr.gdr_decode_multi(dt["q"], dt["k"], dt["v"], dt["g"], dt["beta"], self.state,
+                                 o=self.o[t], stream=stream)
+            host_o[t].copy_(self.o[t], non_blocking=True)
+
+
 def make_case(name, device, seed):
+    if name == "decode_spec_gdn":
+        return SpecDecodeCase(name, device, seed)
     if name.startswith("decode"):
         return DecodeCase(name, device, seed)
     return PrefillCase(name, device, seed)
@@ -388,7 +443,8 @@ def bench_case(case, args, ws, rank, flush, stream, pk, pk_kind):
            "kernel": ("decode" if case.kind == "decode" else
                       ("tcgen05" if case.path == gdr.GDR_PATH_TCGEN05 else "simt"))}
     if case.kind == "decode":
-        cfg["steps_per_bench_step"] = case.steps
+        cfg["launches_per_bench_step"] = case.steps
+        cfg["tokens_per_sequence_per_launch"] = getattr(case, "T", 1)
     return {
         "value": value, "ms_per_step": ms, "tokens_per_step": tokens_all,
         "dtype": case.dtype_label(), "config": cfg, "roofline": roof,
@@ -462,7 +518,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.workloads == "all":
-        args.workloads = "gdn_prefill,kda_prefill,varlen_gdn,gqa_prefill,decode_gdn,decode_kda"
+        args.workloads = ("gdn_prefill,kda_prefill,varlen_gdn,gqa_prefill,decode_gdn,decode_kda,"
+                          "decode_spec_gdn")
     if args.warmup < 3:
         args.warmup = 3
     ws, rank, local = dist_env()

@@ -166,4 +166,25 @@ gdr_status_t gdr_decode_step(const void *q, const void *k, const void *v, const 
                                io_dtype, o, stream);
 }
 
+gdr_status_t gdr_decode_multi(const void *q, const void *k, const void *v, const float *g,
+                              const float *beta, float *state, int32_t N, int32_t T,
+                              int32_t H_qk, int32_t H, int32_t d_k, int32_t d_v,
+                              gdr_gate_mode_t gate_mode, gdr_dtype_t io_dtype, void *o,
+                              float *snapshots, void *stream) {
+    if (N < 0 || T < 0 || T > 16 || H < 0 || H_qk < 1 || (H > 0 && H % H_qk != 0))
+        return GDR_ERR_INVALID_ARG;
+    if (!valid_dim(d_k) || !valid_dim(d_v)) return GDR_ERR_INVALID_ARG;
+    if (gate_mode != GDR_GATE_SCALAR && gate_mode != GDR_GATE_CHANNEL) return GDR_ERR_INVALID_ARG;
+    if (io_dtype != GDR_F32 && io_dtype != GDR_BF16) return GDR_ERR_INVALID_ARG;
+    if ((int64_t)N * T * H > (int64_t)INT32_MAX) return GDR_ERR_INVALID_ARG;
+    if ((int64_t)N * H * T == 0) return GDR_OK;
+    if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_gate_ptr(g, gate_mode) ||
+        !ok_beta_ptr(beta) || !ok_ptr(state) || !ok_ptr(o) || !ok_opt_ptr(snapshots))
+        return GDR_ERR_INVALID_ARG;
+    return from_cuda(gdr::launch_decode_multi(q, k, v, g, beta, state, N, T, H_qk, H, d_k, d_v,
+                                              gate_mode == GDR_GATE_CHANNEL,
+                                              io_dtype == GDR_BF16, o, snapshots,
+                                              static_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

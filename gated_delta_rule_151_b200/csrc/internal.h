@@ -13,6 +13,12 @@ cudaError_t launch_decode_step(const void *q, const void *k, const void *v, cons
                                const float *beta, float *state, int N, int Hqk, int H, int DK,
                                int DV, bool channel, bool bf16, void *o, cudaStream_t stream);
 
+// T consecutive tokens per sequence in one pass over the state (T <= 16).
+cudaError_t launch_decode_multi(const void *q, const void *k, const void *v, const float *g,
+                                const float *beta, float *state, int N, int T, int Hqk, int H,
+                                int DK, int DV, bool channel, bool bf16, void *o, float *snap,
+                                cudaStream_t stream);
+
 cudaError_t launch_prefill_simt(const void *q, const void *k, const void *v, const float *g,
                                 const float *beta, const float *h0, const int32_t *cu,
                                 int num_seqs, int total_T, int Hqk, int H, int DK, int DV,

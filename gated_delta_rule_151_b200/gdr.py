@@ -34,7 +34,8 @@ GDR_PATH_TCGEN05 = 1
 # Every symbol include/gdr.h declares.
 EXPORTED = ("gdr_status_string", "gdr_prefill_workspace_size", "gdr_prefill_path",
             "gdr_prefill_chunked", "gdr_prefill_check_workspace", "gdr_decode_step",
-            "gdr_prefill_chunked_noalloc", "gdr_prefill_chunked_gqa", "gdr_decode_step_gqa")
+            "gdr_prefill_chunked_noalloc", "gdr_prefill_chunked_gqa", "gdr_decode_step_gqa",
+            "gdr_decode_multi")
 
 
 class GdrError(RuntimeError):
@@ -81,6 +82,9 @@ def load_library():
         lib.gdr_prefill_chunked_gqa.restype = ST
         lib.gdr_decode_step_gqa.argtypes = [P, P, P, P, P, P, I32, I32, I32, I32, I32, ST, ST, P, P]
         lib.gdr_decode_step_gqa.restype = ST
+        lib.gdr_decode_multi.argtypes = [P, P, P, P, P, P, I32, I32, I32, I32, I32, I32, ST, ST, P,
+                                         P, P]
+        lib.gdr_decode_multi.restype = ST
         _lib = lib
         return lib
 
@@ -290,3 +294,33 @@ def gdr_prefill_chunked_noalloc(q, k, v, g, beta, initial_state=None, cu_seqlens
         N, T, H, dk, dv, gate, _io_code(io), _ptr(o), _ptr(final_state), _stream_ptr(stream))
     _check(st, "gdr_prefill_chunked_noalloc")
     return o, final_state
+
+
+def gdr_decode_multi(q, k, v, g, beta, state, *, o=None, snapshots=None, stream=None):
+    """T consecutive decode steps per sequence in one pass (see include/gdr.h).
+
+    q, k [N, T, H_qk, d_k]; v [N, T, H, d_v]; g [N, T, H] or [N, T, H, d_k];
+    beta [N, T, H]; state [N, H, d_v, d_k] updated in place; optional
+    snapshots [N, T, H, d_v, d_k] receive the state after every token.
+    Returns o [N, T, H, d_v].
+    """
+    _need(q, "q", ndim=4)
+    io = q.dtype
+    _need(k, "k", io, 4)
+    _need(v, "v", io, 4)
+    _need(beta, "beta", torch.float32, 3)
+    _need(g, "g", torch.float32)
+    _need(state, "state", torch.float32, 4)
+    N, T, Hqk, dk = q.shape
+    H, dv = v.shape[2], v.shape[3]
+    gate = GDR_GATE_SCALAR if g.dim() == 3 else GDR_GATE_CHANNEL
+    if o is None:
+        o = torch.empty((N, T, H, dv), dtype=io, device=q.device)
+    _need(o, "o", io, 4)
+    if snapshots is not None:
+        _need(snapshots, "snapshots", torch.float32, 5)
+    st = load_library().gdr_decode_multi(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                         _ptr(state), N, T, Hqk, H, dk, dv, gate, _io_code(io),
+                                         _ptr(o), _ptr(snapshots), _stream_ptr(stream))
+    _check(st, "gdr_decode_multi")
+    return o

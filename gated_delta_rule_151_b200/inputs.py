@@ -38,6 +38,8 @@ kda_prefill        2 sequences x 32768, H=32, d=128, bf16, channel gate
                    c=0.05, h0 ~ N(0, 0.02^2)
 decode_gdn/kda     256 sequences, H=32, d=128, 512 steps of one bf16 token,
                    c=0.1, h0 ~ N(0, 0.02^2) (state 512 MiB fp32)
+decode_spec_gdn    the decode_gdn tokens verified 4 at a time (128 steps of
+                   4 draft tokens per sequence)
 varlen_gdn         8 packed sequences, 262144 tokens, H=16, d=128, bf16,
                    scalar gate c=0.1, h0=0
 gqa_prefill        1 sequence, 8192 tokens, 16 query/key heads shared by 48
@@ -239,7 +241,9 @@ def make_inputs(*, total_T: int, H: int, d_k: int, d_v: int | None = None,
 # ---------------------------------------------------------------------------
 
 WORKLOADS = ("tiny_gdn", "gdn_prefill", "kda_prefill", "decode_gdn",
-             "decode_kda", "varlen_gdn", "gqa_prefill")
+             "decode_kda", "varlen_gdn", "gqa_prefill", "decode_spec_gdn")
+
+SPEC_DRAFT = 4   # tokens verified per sequence per step in decode_spec_gdn
 
 DECODE_SEQS, DECODE_HEADS, DECODE_D, DECODE_STEPS = 256, 32, 128, 512
 
@@ -263,8 +267,8 @@ def workload(name: str, seed: int = 0) -> Inputs:
         return make_inputs(total_T=65536, H=32, d_k=128, num_seqs=2, gate_mode=CHANNEL,
                            io_dtype=torch.bfloat16, c=0.05, h0_std=0.02, seed=seed,
                            meta={"workload": name})
-    if name in ("decode_gdn", "decode_kda"):
-        mode = SCALAR if name == "decode_gdn" else CHANNEL
+    if name in ("decode_gdn", "decode_kda", "decode_spec_gdn"):
+        mode = CHANNEL if name == "decode_kda" else SCALAR
         return make_inputs(total_T=DECODE_SEQS * DECODE_STEPS, H=DECODE_HEADS,
                            d_k=DECODE_D, num_seqs=DECODE_SEQS, gate_mode=mode,
                            io_dtype=torch.bfloat16, c=0.1, h0_std=0.02, seed=seed,

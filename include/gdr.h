@@ -222,6 +222,28 @@ GDR_API gdr_status_t gdr_decode_step_gqa(const void *q, const void *k, const voi
                                  gdr_gate_mode_t gate_mode, gdr_dtype_t io_dtype, void *o,
                                  void *stream);
 
+/*
+ * T consecutive decode steps per sequence in one pass over the state -- the
+ * verification step of speculative decoding, where a draft model proposes a
+ * few tokens per sequence (the pages' multi-token-prediction drafting uses
+ * 4-5; page "How the New Flash Models Work", multi-token prediction
+ * section).  1 <= T <= 16.
+ *
+ * q, k [N, T, H_qk, d_k]; v [N, T, H, d_v] (io dtype); g [N, T, H] or
+ * [N, T, H, d_k]; beta [N, T, H] (fp32): token t of sequence n is row
+ * n*T + t.  state [N, H, d_v, d_k] fp32 is read once and overwritten with the
+ * state after all T tokens; o [N, T, H, d_v] receives every token's output.
+ * The results equal T calls of gdr_decode_step_gqa (same arithmetic, same
+ * order).  snapshots, if not NULL, is [N, T, H, d_v, d_k] fp32 and receives
+ * the state after each token (snapshot t = state after tokens 0..t), so a
+ * caller that accepts only the first m drafts restores snapshot m-1.
+ */
+GDR_API gdr_status_t gdr_decode_multi(const void *q, const void *k, const void *v,
+                              const float *g, const float *beta, float *state, int32_t N,
+                              int32_t T, int32_t H_qk, int32_t H, int32_t d_k, int32_t d_v,
+                              gdr_gate_mode_t gate_mode, gdr_dtype_t io_dtype, void *o,
+                              float *snapshots, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -130,3 +130,14 @@ def test_grouped_heads_must_divide(lib, Hqk, H):
     st = lib.gdr_decode_step_gqa(P(A), P(A), P(A), P(A), P(A), P(A), 2, Hqk, H, 128, 128, 0, 1,
                                  P(A), None)
     assert st == gdr.GDR_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("T,Hqk,H", [(17, 2, 2), (-1, 2, 2), (4, 3, 4), (4, 0, 2)])
+def test_decode_multi_rejects_invalid_arguments(lib, T, Hqk, H):
+    P = ctypes.c_void_p
+    st = lib.gdr_decode_multi(P(A), P(A), P(A), P(A), P(A), P(A), 2, T, Hqk, H, 128, 128, 0, 1,
+                              P(A), None, None)
+    assert st == gdr.GDR_ERR_INVALID_ARG
+    st = lib.gdr_decode_multi(P(A), P(A), P(A), P(A), P(A), P(A), 2, 4, 2, 2, 128, 128, 0, 1,
+                              P(A), P(MIS), None)
+    assert st == gdr.GDR_ERR_INVALID_ARG     # misaligned snapshot buffer
