@@ -164,6 +164,16 @@ def decode_work(inp):
     return N * H * (2 * 4 * dk * dv + e * (2 * dk + 2 * dv) + 4 + gate)
 
 
+def split_launches(inp):
+    """Kernel launches of the chunk-parallel plan: a prep and a chain kernel
+    per window of chunks (the library bounds the chunk records of one window
+    to 1 GiB at 147,968 bytes per chunk and head)."""
+    chains = inp.num_seqs * inp.H
+    max_chunks = -(-inp.total_T // 64)
+    window = max(1, min(max_chunks, (1 << 30) // (chains * 147968)))
+    return 2 * (-(-max_chunks // window))
+
+
 class PrefillCase:
     kind = "prefill"
 
@@ -179,13 +189,14 @@ class PrefillCase:
                                device=device)
         gate = gdr.GDR_GATE_CHANNEL if inp.gate_mode == I.CHANNEL else gdr.GDR_GATE_SCALAR
         io = gdr.GDR_BF16 if inp.io_dtype == torch.bfloat16 else gdr.GDR_F32
-        self.path = gdr.gdr_prefill_path(inp.d_k, inp.d_v, gate, io)
         nbytes = gdr.gdr_prefill_workspace_size(inp.num_seqs, inp.total_T, inp.H, inp.d_k,
                                                 inp.d_v, gate, io)
         self.ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=device) if nbytes else None
+        self.path = gdr.gdr_prefill_plan(inp.num_seqs, inp.total_T, inp.H, inp.d_k, inp.d_v,
+                                         gate, io, nbytes)
         self.bytes, self.flops = prefill_work(inp)
         self.tokens = inp.total_T
-        self.launches = 1
+        self.launches = split_launches(inp) if self.path == gdr.GDR_PATH_TCGEN05_SPLIT else 1
 
     def _fn(self):
         return gdr.gdr_prefill_chunked if self.inp.H_qk == self.inp.H else gdr.gdr_prefill_chunked_gqa
@@ -218,7 +229,7 @@ class PrefillCase:
         return host, ho, hf, h2d, d2h
 
     def dtype_label(self):
-        if self.path == gdr.GDR_PATH_TCGEN05:
+        if self.path in (gdr.GDR_PATH_TCGEN05, gdr.GDR_PATH_TCGEN05_SPLIT):
             return "bf16/tf32 tensor-core operands, fp32 accumulate and state"
         return "f32"
 
@@ -409,7 +420,9 @@ def bench_case(case, args, ws, rank, flush, stream, pk, pk_kind):
         barrier(ws)
     value, ms = aggregate_throughput(case.tokens, sum(times) / len(times), ws)
     tokens_all = case.tokens * ws
-    launch_ms = ms / case.launches
+    # decode: bytes per launch over the time per launch; prefill: the whole
+    # step's bytes (every kernel of the plan) over the step time
+    launch_ms = ms if case.kind == "prefill" else ms / case.launches
     achieved = case.bytes / (launch_ms / 1e3) / 1e9
     hbm_peak = float(pk["hbm_gbs"])
     roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
@@ -441,7 +454,11 @@ def bench_case(case, args, ws, rank, flush, stream, pk, pk_kind):
            "io": str(inp.io_dtype).replace("torch.", ""),
            "h0": inp.h0 is not None, "l2": "flushed (512 MiB write) before every timed step",
            "kernel": ("decode" if case.kind == "decode" else
-                      ("tcgen05" if case.path == gdr.GDR_PATH_TCGEN05 else "simt"))}
+                      {gdr.GDR_PATH_TCGEN05: "tcgen05",
+                       gdr.GDR_PATH_TCGEN05_SPLIT: "tcgen05 chunk-parallel (prep + chain)"}.get(
+                           case.path, "simt"))}
+    if case.kind == "prefill":
+        cfg["launches_per_step"] = case.launches
     if case.kind == "decode":
         cfg["launches_per_bench_step"] = case.steps
         cfg["tokens_per_sequence_per_launch"] = getattr(case, "T", 1)

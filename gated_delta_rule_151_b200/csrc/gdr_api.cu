@@ -65,7 +65,29 @@ gdr_status_t gdr_prefill_workspace_size(int32_t num_seqs, int32_t total_T, int32
     if (bytes == nullptr || num_seqs < 0 || total_T < 0 || H < 0) return GDR_ERR_INVALID_ARG;
     gdr_status_t st = gdr_prefill_path(d_k, d_v, gate_mode, io_dtype, &path);
     if (st != GDR_OK) return st;
-    *bytes = path == GDR_PATH_TCGEN05 ? gdr::tcgen05_workspace_bytes(num_seqs, total_T, H) : 0;
+    *bytes = 0;
+    if (path == GDR_PATH_TCGEN05) {
+        const size_t split = gdr::tcgen05_split_workspace_bytes(num_seqs, total_T, H);
+        const size_t single = gdr::tcgen05_workspace_bytes(num_seqs, total_T, H);
+        *bytes = split > single ? split : single;
+    }
+    return GDR_OK;
+}
+
+gdr_status_t gdr_prefill_plan(int32_t num_seqs, int32_t total_T, int32_t H, int32_t d_k,
+                              int32_t d_v, gdr_gate_mode_t gate_mode, gdr_dtype_t io_dtype,
+                              size_t workspace_bytes, gdr_prefill_path_t *path) {
+    if (path == nullptr || num_seqs < 0 || total_T < 0 || H < 0) return GDR_ERR_INVALID_ARG;
+    gdr_prefill_path_t family;
+    gdr_status_t st = gdr_prefill_path(d_k, d_v, gate_mode, io_dtype, &family);
+    if (st != GDR_OK) return st;
+    *path = family;
+    if (family == GDR_PATH_TCGEN05) {
+        if (workspace_bytes < gdr::tcgen05_workspace_bytes(num_seqs, total_T, H))
+            return GDR_ERR_WORKSPACE;
+        const size_t split = gdr::tcgen05_split_workspace_bytes(num_seqs, total_T, H);
+        if (split > 0 && workspace_bytes >= split) *path = GDR_PATH_TCGEN05_SPLIT;
+    }
     return GDR_OK;
 }
 
@@ -96,17 +118,24 @@ gdr_status_t gdr_prefill_chunked_gqa(const void *q, const void *k, const void *v
     // kernels' 32-bit token indices.
     if ((int64_t)total_T * H > (int64_t)INT32_MAX) return GDR_ERR_INVALID_ARG;
 
-    size_t need = 0;
-    gdr_status_t st = gdr_prefill_workspace_size(num_seqs, total_T, H, d_k, d_v, gate_mode,
-                                                 io_dtype, &need);
-    if (st != GDR_OK) return st;
-    if (need > 0 && (workspace == nullptr || workspace_bytes < need || !aligned16(workspace)))
+    // The single-kernel tcgen05 plan needs a few bytes; with the (larger) size
+    // gdr_prefill_workspace_size reports, the chunk-parallel plan runs where it
+    // applies.
+    gdr_prefill_path_t plan;
+    if (workspace_bytes > 0 && (workspace == nullptr || !aligned16(workspace)))
         return GDR_ERR_WORKSPACE;
+    gdr_status_t st = gdr_prefill_plan(num_seqs, total_T, H, d_k, d_v, gate_mode, io_dtype,
+                                       workspace == nullptr ? 0 : workspace_bytes, &plan);
+    if (st != GDR_OK) return st;
     if (num_seqs == 0) return GDR_OK;
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const bool channel = gate_mode == GDR_GATE_CHANNEL;
-    if (uses_tcgen05(d_k, d_v, gate_mode, io_dtype))
+    if (plan == GDR_PATH_TCGEN05_SPLIT)
+        return from_cuda(gdr::launch_prefill_split(q, k, v, g, beta, initial_state, cu_seqlens,
+                                                    num_seqs, total_T, H_qk, H, channel, o,
+                                                    final_state, workspace, s));
+    if (plan == GDR_PATH_TCGEN05)
         return from_cuda(gdr::launch_prefill_tcgen05(q, k, v, g, beta, initial_state, cu_seqlens,
                                                       num_seqs, total_T, H_qk, H, channel, o,
                                                       final_state, workspace, s));

@@ -36,4 +36,12 @@ cudaError_t launch_prefill_tcgen05(const void *q, const void *k, const void *v, 
                                    int num_seqs, int total_T, int Hqk, int H, bool channel,
                                    void *o, float *fin, void *workspace, cudaStream_t stream);
 
+// Two-kernel chunk-parallel plan of the tcgen05 prefill: workspace bytes it
+// needs (0 when the plan does not apply to this shape), and its launcher.
+size_t tcgen05_split_workspace_bytes(int num_seqs, int total_T, int H);
+cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, const float *g,
+                                 const float *beta, const float *h0, const int32_t *cu,
+                                 int num_seqs, int total_T, int Hqk, int H, bool channel, void *o,
+                                 float *fin, void *workspace, cudaStream_t stream);
+
 }  // namespace gdr

@@ -30,12 +30,13 @@ GDR_F32 = 0
 GDR_BF16 = 1
 GDR_PATH_SIMT = 0
 GDR_PATH_TCGEN05 = 1
+GDR_PATH_TCGEN05_SPLIT = 2
 
 # Every symbol include/gdr.h declares.
 EXPORTED = ("gdr_status_string", "gdr_prefill_workspace_size", "gdr_prefill_path",
             "gdr_prefill_chunked", "gdr_prefill_check_workspace", "gdr_decode_step",
             "gdr_prefill_chunked_noalloc", "gdr_prefill_chunked_gqa", "gdr_decode_step_gqa",
-            "gdr_decode_multi")
+            "gdr_decode_multi", "gdr_prefill_plan")
 
 
 class GdrError(RuntimeError):
@@ -67,6 +68,9 @@ def load_library():
         lib.gdr_prefill_workspace_size.restype = ST
         lib.gdr_prefill_path.argtypes = [I32, I32, ST, ST, ctypes.POINTER(ctypes.c_int)]
         lib.gdr_prefill_path.restype = ST
+        lib.gdr_prefill_plan.argtypes = [I32, I32, I32, I32, I32, ST, ST, SZ,
+                                         ctypes.POINTER(ctypes.c_int)]
+        lib.gdr_prefill_plan.restype = ST
         lib.gdr_prefill_chunked.argtypes = [P, P, P, P, P, P, P, I32, I32, I32, I32, I32, ST, ST,
                                             P, P, P, SZ, P]
         lib.gdr_prefill_chunked.restype = ST
@@ -147,6 +151,17 @@ def gdr_prefill_path(d_k, d_v, gate_mode, io_dtype) -> int:
     out = ctypes.c_int(0)
     _check(load_library().gdr_prefill_path(d_k, d_v, gate_mode, io_dtype, ctypes.byref(out)),
            "gdr_prefill_path")
+    return int(out.value)
+
+
+def gdr_prefill_plan(num_seqs, total_T, H, d_k, d_v, gate_mode, io_dtype,
+                     workspace_bytes) -> int:
+    """The plan gdr_prefill_chunked runs with this much workspace:
+    GDR_PATH_SIMT, GDR_PATH_TCGEN05 or GDR_PATH_TCGEN05_SPLIT."""
+    out = ctypes.c_int(0)
+    _check(load_library().gdr_prefill_plan(num_seqs, total_T, H, d_k, d_v, gate_mode, io_dtype,
+                                           workspace_bytes, ctypes.byref(out)),
+           "gdr_prefill_plan")
     return int(out.value)
 
 

@@ -81,27 +81,53 @@ typedef enum {
     GDR_BF16 = 1   /* q, k, v and o in bfloat16 */
 } gdr_dtype_t;
 
-/* Which prefill kernel serves a request. */
+/* Which prefill kernel(s) serve a request. */
 typedef enum {
-    GDR_PATH_SIMT = 0,     /* fp32 CUDA-core chunked kernel (any d, any io dtype) */
-    GDR_PATH_TCGEN05 = 1   /* tcgen05/TMEM/TMA chunked kernel (bf16, d_k = d_v = 128) */
+    GDR_PATH_SIMT = 0,          /* fp32 CUDA-core chunked kernel (any d, any io dtype)     */
+    GDR_PATH_TCGEN05 = 1,       /* tcgen05/TMEM/TMA chunked kernel (bf16, d_k = d_v = 128):
+                                   one CTA per (sequence, head) runs every chunk step     */
+    GDR_PATH_TCGEN05_SPLIT = 2  /* same arithmetic as two kernels: every chunk's local
+                                   operands in parallel into the workspace, then one CTA
+                                   per (sequence, head) runs the state chain over them    */
 } gdr_prefill_path_t;
 
 /* Human-readable name of a status code (static storage, never NULL). */
 GDR_API const char *gdr_status_string(gdr_status_t status);
 
 /*
- * Bytes of device workspace gdr_prefill_chunked needs for this problem
- * (written to *bytes; may be 0).  Pure host function.
+ * Bytes of device workspace for the fastest plan gdr_prefill_chunked has for
+ * this problem (written to *bytes; may be 0).  Pure host function.
+ *
+ * The tcgen05 kernels take two plans.  The single-kernel plan needs 16 bytes
+ * (an error word).  With fewer (sequence, head) pairs than 149, the
+ * chunk-parallel plan (GDR_PATH_TCGEN05_SPLIT) keeps all SMs busy; it needs
+ * 144.5 KiB per (chunk, sequence, head) of its chunk records, capped at
+ * 1 GiB by running long problems in windows of chunks (plus 64 KiB of state
+ * per (sequence, head) between windows).  The size reported here is the
+ * larger one where both apply; gdr_prefill_chunked runs the chunk-parallel
+ * plan when given at least that much and the single-kernel plan when given
+ * at least 16 bytes.  Both give the same results up to rounding order.
  */
 GDR_API gdr_status_t gdr_prefill_workspace_size(int32_t num_seqs, int32_t total_T, int32_t H,
                                         int32_t d_k, int32_t d_v,
                                         gdr_gate_mode_t gate_mode, gdr_dtype_t io_dtype,
                                         size_t *bytes);
 
-/* The kernel gdr_prefill_chunked launches for this shape/dtype (host only). */
+/* The kernel family gdr_prefill_chunked uses for this shape/dtype (host only):
+ * GDR_PATH_SIMT or GDR_PATH_TCGEN05. */
 GDR_API gdr_status_t gdr_prefill_path(int32_t d_k, int32_t d_v, gdr_gate_mode_t gate_mode,
                               gdr_dtype_t io_dtype, gdr_prefill_path_t *path);
+
+/*
+ * The plan gdr_prefill_chunked runs for this problem given `workspace_bytes`
+ * of workspace (host only): GDR_PATH_SIMT, GDR_PATH_TCGEN05 or
+ * GDR_PATH_TCGEN05_SPLIT.  GDR_ERR_WORKSPACE if that workspace is below the
+ * minimum; GDR_ERR_INVALID_ARG for an invalid shape or mode.
+ */
+GDR_API gdr_status_t gdr_prefill_plan(int32_t num_seqs, int32_t total_T, int32_t H,
+                              int32_t d_k, int32_t d_v, gdr_gate_mode_t gate_mode,
+                              gdr_dtype_t io_dtype, size_t workspace_bytes,
+                              gdr_prefill_path_t *path);
 
 /*
  * Chunked prefill over packed variable-length sequences.
@@ -127,8 +153,11 @@ GDR_API gdr_status_t gdr_prefill_path(int32_t d_k, int32_t d_v, gdr_gate_mode_t 
  * final_state        [num_seqs, H, d_v, d_k] fp32 state after each sequence's
  *                    last token, or NULL.  May equal initial_state.  An empty
  *                    sequence yields its initial state (or zeros).
- * workspace          device scratch of at least gdr_prefill_workspace_size()
- *                    bytes (NULL allowed when that size is 0).
+ * workspace          device scratch, 16-byte aligned: gdr_prefill_workspace_size()
+ *                    bytes run the fastest plan; fewer bytes run the plan
+ *                    gdr_prefill_plan reports for them (GDR_ERR_WORKSPACE
+ *                    below the minimum).  NULL allowed when the minimum is 0.
+ *                    Word 0 receives the device-side error bits.
  */
 GDR_API gdr_status_t gdr_prefill_chunked(const void *q, const void *k, const void *v,
                                  const float *g, const float *beta,
@@ -175,8 +204,9 @@ GDR_API gdr_status_t gdr_prefill_check_workspace(const void *workspace, size_t w
  * allocator of their own.  Instead of a caller-provided workspace, the
  * scratch the prefill needs lives in a fixed 256-byte device array inside
  * libgdr, present on every GPU that loads the library until the process
- * exits.  A problem whose gdr_prefill_workspace_size() exceeds 256 bytes is
- * rejected with GDR_ERR_WORKSPACE (this build needs 16 bytes or none).
+ * exits.  The array serves the single-kernel plans (16 bytes of workspace or
+ * none); a problem whose minimum exceeds 256 bytes is rejected with
+ * GDR_ERR_WORKSPACE.
  *
  * The first call on each device looks up the array's device address with
  * that device current (a one-time set-up); make that first call before any

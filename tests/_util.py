@@ -29,13 +29,28 @@ def to_device(inp, device="cuda"):
     return d
 
 
-def gpu_prefill(inp, use_cu=True, initial_state="h0", final_state=None):
+# Workspace that selects each tcgen05 plan: None lets the binding allocate the
+# reported size (the chunk-parallel plan where it applies); 16 bytes is the
+# single-kernel plan's minimum.
+PLANS = ("split", "single")
+
+
+def plan_workspace(plan):
+    if plan == "single":
+        return torch.zeros(16, dtype=torch.uint8, device="cuda")
+    return None
+
+
+def gpu_prefill(inp, use_cu=True, initial_state="h0", final_state=None, plan="split"):
     d = to_device(inp)
     h0 = d["h0"] if initial_state == "h0" else initial_state
     fn = gdr.gdr_prefill_chunked if inp.H_qk == inp.H else gdr.gdr_prefill_chunked_gqa
+    ws = plan_workspace(plan)
     o, fin = fn(d["q"], d["k"], d["v"], d["g"], d["beta"], h0, d["cu"] if use_cu else None,
-                num_seqs=inp.num_seqs, final_state=final_state)
+                num_seqs=inp.num_seqs, final_state=final_state, workspace=ws)
     torch.cuda.synchronize()
+    if ws is not None:
+        gdr.gdr_prefill_check_workspace(ws)
     return o, fin
 
 

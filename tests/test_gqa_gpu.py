@@ -8,30 +8,32 @@ import torch
 import oracle
 from gated_delta_rule_151_b200 import gdr
 from gated_delta_rule_151_b200 import inputs as I
-from _util import TOL_BF16_O, TOL_BF16_STATE_REL, TOL_F32, check, gpu_prefill, oracle_prefill, rel_frob
+from _util import PLANS, TOL_BF16_O, TOL_BF16_STATE_REL, TOL_F32, check, gpu_prefill, oracle_prefill, rel_frob
 
 pytestmark = pytest.mark.gpu
 
 
 @pytest.mark.parametrize("mode", [I.SCALAR, I.CHANNEL])
-@pytest.mark.parametrize("d,io", [(128, torch.bfloat16), (32, torch.float32)])
-def test_prefill_grouped_heads(mode, d, io):
+@pytest.mark.parametrize("d,io,plan", [(128, torch.bfloat16, "split"), (128, torch.bfloat16, "single"),
+                                       (32, torch.float32, "split")])
+def test_prefill_grouped_heads(mode, d, io, plan):
     inp = I.make_inputs(total_T=211, H=6, H_qk=2, d_k=d, gate_mode=mode, io_dtype=io,
                         cu_seqlens=[0, 90, 90, 211], c=0.1, h0_std=0.03, seed=41)
-    o, fin = gpu_prefill(inp)
+    o, fin = gpu_prefill(inp, plan=plan)
     o_ref, fin_ref = oracle_prefill(inp)
     check(inp, o, fin, o_ref, fin_ref, f"gqa {mode} d={d}")
 
 
-def test_prefill_grouped_equals_replicated_heads():
+@pytest.mark.parametrize("plan", PLANS)
+def test_prefill_grouped_equals_replicated_heads(plan):
     """The kernels' head mapping is an index map: replicating each query/key
     head over its value heads must give bit-identical results."""
     inp = I.make_inputs(total_T=150, H=6, H_qk=3, d_k=128, io_dtype=torch.bfloat16,
                         h0_std=0.02, seed=42)
-    o1, f1 = gpu_prefill(inp)
+    o1, f1 = gpu_prefill(inp, plan=plan)
     rep = torch.arange(6) // 2
     inp.q, inp.k = inp.q[:, rep].contiguous(), inp.k[:, rep].contiguous()
-    o2, f2 = gpu_prefill(inp)
+    o2, f2 = gpu_prefill(inp, plan=plan)
     assert torch.equal(o1, o2) and torch.equal(f1, f2)
 
 

@@ -10,7 +10,7 @@ import torch
 import oracle
 from gated_delta_rule_151_b200 import gdr
 from gated_delta_rule_151_b200 import inputs as I
-from _util import check, gpu_prefill, oracle_prefill, to_device, TOL_BF16_O
+from _util import PLANS, check, gpu_prefill, oracle_prefill, plan_workspace, to_device, TOL_BF16_O
 
 pytestmark = pytest.mark.gpu
 
@@ -24,10 +24,11 @@ def test_tiny_workload_fp32():
 
 @pytest.mark.parametrize("T", [1, 63, 64, 65, 127, 129, 300])
 @pytest.mark.parametrize("mode", [I.SCALAR, I.CHANNEL])
-def test_ragged_lengths_bf16_d128(T, mode):
+@pytest.mark.parametrize("plan", PLANS)
+def test_ragged_lengths_bf16_d128(T, mode, plan):
     inp = I.make_inputs(total_T=T, H=3, d_k=128, gate_mode=mode, io_dtype=torch.bfloat16,
                         c=0.1, h0_std=0.02, seed=T)
-    o, fin = gpu_prefill(inp)
+    o, fin = gpu_prefill(inp, plan=plan)
     o_ref, fin_ref = oracle_prefill(inp)
     check(inp, o, fin, o_ref, fin_ref, f"T={T} {mode}")
 
@@ -44,13 +45,14 @@ def test_head_dims(dk, dv, mode, io):
 
 
 @pytest.mark.parametrize("mode", [I.SCALAR, I.CHANNEL])
-@pytest.mark.parametrize("d,io", [(128, torch.bfloat16), (32, torch.float32)])
-def test_varlen_with_empty_and_short_sequences(mode, d, io):
+@pytest.mark.parametrize("d,io,plan", [(128, torch.bfloat16, "split"), (128, torch.bfloat16, "single"),
+                                       (32, torch.float32, "split")])
+def test_varlen_with_empty_and_short_sequences(mode, d, io, plan):
     lens = [0, 5, 64, 0, 130, 1, 77]
     cu = np.concatenate([[0], np.cumsum(lens)])
     inp = I.make_inputs(total_T=int(cu[-1]), H=2, d_k=d, cu_seqlens=cu, gate_mode=mode,
                         io_dtype=io, c=0.1, h0_std=0.03, seed=3)
-    o, fin = gpu_prefill(inp)
+    o, fin = gpu_prefill(inp, plan=plan)
     o_ref, fin_ref = oracle_prefill(inp)
     check(inp, o, fin, o_ref, fin_ref, "varlen")
     # empty sequences hand back their initial state exactly
@@ -79,34 +81,37 @@ def test_no_initial_state_means_zeros_and_no_final_state_is_allowed():
     assert torch.equal(o, o2) and torch.equal(fin, fin2) and torch.equal(o, o3)
 
 
-@pytest.mark.parametrize("d,io", [(128, torch.bfloat16), (16, torch.float32)])
-def test_in_place_state(d, io):
+@pytest.mark.parametrize("d,io,plan", [(128, torch.bfloat16, "split"), (128, torch.bfloat16, "single"),
+                                       (16, torch.float32, "split")])
+def test_in_place_state(d, io, plan):
     inp = I.make_inputs(total_T=150, H=2, d_k=d, num_seqs=1, io_dtype=io, h0_std=0.05, seed=6)
     dv = to_device(inp)
     o_sep, f_sep = gdr.gdr_prefill_chunked(dv["q"], dv["k"], dv["v"], dv["g"], dv["beta"],
-                                           dv["h0"], dv["cu"])
+                                           dv["h0"], dv["cu"], workspace=plan_workspace(plan))
     state = dv["h0"].clone()
     o_in, f_in = gdr.gdr_prefill_chunked(dv["q"], dv["k"], dv["v"], dv["g"], dv["beta"], state,
-                                         dv["cu"], final_state=state)
+                                         dv["cu"], final_state=state, workspace=plan_workspace(plan))
     torch.cuda.synchronize()
     assert f_in.data_ptr() == state.data_ptr()
     assert torch.equal(o_sep, o_in) and torch.equal(f_sep, state)
 
 
 @pytest.mark.parametrize("mode", [I.SCALAR, I.CHANNEL])
-def test_gate_minus_infinity(mode):
+@pytest.mark.parametrize("plan", PLANS)
+def test_gate_minus_infinity(mode, plan):
     inp = I.make_inputs(total_T=140, H=2, d_k=128, gate_mode=mode, io_dtype=torch.bfloat16,
                         h0_std=0.05, seed=9)
     g = inp.g.clone()
     g[::17] = -float("inf")       # hard resets inside and across chunks
     inp.g = g
-    o, fin = gpu_prefill(inp)
+    o, fin = gpu_prefill(inp, plan=plan)
     o_ref, fin_ref = oracle_prefill(inp)
     check(inp, o, fin, o_ref, fin_ref, "g=-inf")
 
 
 @pytest.mark.parametrize("mode", [I.SCALAR, I.CHANNEL])
-def test_guard_bands_and_poisoned_outputs(mode):
+@pytest.mark.parametrize("plan", PLANS)
+def test_guard_bands_and_poisoned_outputs(mode, plan):
     """Outputs live inside larger buffers whose margins hold a sentinel and
     whose interior starts as NaN: every output element must be written and
     nothing outside may change."""
@@ -123,7 +128,7 @@ def test_guard_bands_and_poisoned_outputs(mode):
     o.fill_(float("nan"))
     f.fill_(float("nan"))
     gdr.gdr_prefill_chunked(d["q"], d["k"], d["v"], d["g"], d["beta"], d["h0"], d["cu"], o=o,
-                            final_state=f)
+                            final_state=f, workspace=plan_workspace(plan))
     torch.cuda.synchronize()
     assert torch.all(obuf[:pad] == sentinel) and torch.all(obuf[-pad:] == sentinel)
     assert torch.all(fbuf[:pad] == sentinel) and torch.all(fbuf[-pad:] == sentinel)
@@ -172,9 +177,9 @@ def test_prefill_then_decode_handoff():
 
 # ------------------------------------------------ full-size workloads ----
 
-def _sampled(name, heads, seqs=None):
+def _sampled(name, heads, seqs=None, plan="split"):
     inp = I.workload(name)
-    o, fin = gpu_prefill(inp)
+    o, fin = gpu_prefill(inp, plan=plan)
     o_ref, fin_ref = oracle_prefill(inp, heads=heads, seqs=seqs)
     cu = inp.cu_seqlens.numpy()
     seqs = list(range(inp.num_seqs)) if seqs is None else seqs
@@ -184,8 +189,9 @@ def _sampled(name, heads, seqs=None):
     return check(inp, o_sel, f_sel, o_ref, fin_ref, name)
 
 
-def test_full_size_gdn_prefill_sampled():
-    _sampled("gdn_prefill", heads=[0, 7, 15])
+@pytest.mark.parametrize("plan", PLANS)
+def test_full_size_gdn_prefill_sampled(plan):
+    _sampled("gdn_prefill", heads=[0, 7, 15], plan=plan)
 
 
 def test_full_size_kda_prefill_sampled():
@@ -205,6 +211,8 @@ def test_tensor_core_path_is_used_and_reports_no_timeout():
     d = to_device(inp)
     nb = gdr.gdr_prefill_workspace_size(3, 333, 4, 128, 128, gdr.GDR_GATE_SCALAR, gdr.GDR_BF16)
     assert nb >= 4
+    assert gdr.gdr_prefill_plan(3, 333, 4, 128, 128, gdr.GDR_GATE_SCALAR, gdr.GDR_BF16,
+                                nb) == gdr.GDR_PATH_TCGEN05_SPLIT
     ws = torch.full((nb,), 0xFF, dtype=torch.uint8, device="cuda")
     o, fin = gdr.gdr_prefill_chunked(d["q"], d["k"], d["v"], d["g"], d["beta"], d["h0"], d["cu"],
                                      workspace=ws)
@@ -214,7 +222,8 @@ def test_tensor_core_path_is_used_and_reports_no_timeout():
 
 
 @pytest.mark.parametrize("c_gate", [0.02, 0.3, 1.5, 6.0])
-def test_channel_gate_decay_strengths(c_gate):
+@pytest.mark.parametrize("plan", PLANS)
+def test_channel_gate_decay_strengths(c_gate, plan):
     """Kimi Delta Attention on the tensor-core kernel across decay strengths:
     weak and moderate decays take the fp16 scaled-operand path for the
     intra-chunk products, strong ones push the scaled operands past fp16's
@@ -222,6 +231,41 @@ def test_channel_gate_decay_strengths(c_gate):
     assert gdr.gdr_prefill_path(128, 128, gdr.GDR_GATE_CHANNEL, gdr.GDR_BF16) == gdr.GDR_PATH_TCGEN05
     inp = I.make_inputs(total_T=320, H=2, d_k=128, gate_mode=I.CHANNEL, io_dtype=torch.bfloat16,
                         c=c_gate, h0_std=0.02, seed=31)
-    o, fin = gpu_prefill(inp)
+    o, fin = gpu_prefill(inp, plan=plan)
     o_ref, fin_ref = oracle_prefill(inp)
     check(inp, o, fin, o_ref, fin_ref, f"kda c={c_gate}")
+
+
+@pytest.mark.parametrize("mode", [I.SCALAR, I.CHANNEL])
+def test_chunk_parallel_plan_in_windows(mode):
+    """148 heads x 3,840 tokens: the chunk records exceed the 1 GiB window,
+    so the chunk-parallel plan runs in two windows of chunks with the state
+    handed between them through the workspace (sequence of 60 chunks, a
+    window of 49).  Sampled heads against the oracle, in-place state."""
+    T, H = 3840, 148
+    nb = gdr.gdr_prefill_workspace_size(1, T, H, 128, 128, 0 if mode == I.SCALAR else 1,
+                                        gdr.GDR_BF16)
+    assert nb > (1 << 30)
+    inp = I.make_inputs(total_T=T, H=H, d_k=128, gate_mode=mode, io_dtype=torch.bfloat16,
+                        c=0.1, h0_std=0.02, seed=51)
+    d = to_device(inp)
+    state = d["h0"].clone()
+    ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    o, fin = gdr.gdr_prefill_chunked(d["q"], d["k"], d["v"], d["g"], d["beta"], state, d["cu"],
+                                     final_state=state, workspace=ws)
+    gdr.gdr_prefill_check_workspace(ws)
+    heads = [0, 77, 147]
+    o_ref, fin_ref = oracle_prefill(inp, heads=heads)
+    check(inp, o[:, heads], fin[:, heads], o_ref, fin_ref, "windows")
+
+
+@pytest.mark.parametrize("mode", [I.SCALAR, I.CHANNEL])
+def test_plans_agree(mode):
+    """Both tcgen05 plans compute the same chunk algebra in the same
+    precisions: their outputs agree far inside the oracle tolerance."""
+    inp = I.make_inputs(total_T=1000, H=4, d_k=128, gate_mode=mode, io_dtype=torch.bfloat16,
+                        cu_seqlens=[0, 333, 334, 1000], c=0.1, h0_std=0.02, seed=52)
+    o1, f1 = gpu_prefill(inp, plan="split")
+    o2, f2 = gpu_prefill(inp, plan="single")
+    assert float((o1.float() - o2.float()).abs().max()) <= 4e-3
+    assert float((f1 - f2).norm() / f2.norm()) <= 1e-4
