@@ -838,10 +838,11 @@ chain_kernel(const uint8_t *__restrict__ recs, const float *h0, float *fin, floa
 // with U_b = Ũ_b + X (tf32) and S_b^T = S_b^T Diag(exp(G_C)) + ΔS_b^T kept in
 // fp32 registers (thread = d_k row).  N = 32 for every product.  Warp roles:
 // 0-3 own the state block, 4-5 form U, 6-7 store the output, 8 issues the
-// MMAs and the record loads; they hand off through mbarriers only.
+// MMAs, 9 loads the records; they hand off through mbarriers only (MMA
+// completion frees record buffers through tcgen05.commit).
 constexpr int kNB = 32;                       // value channels per CTA
 constexpr int kSplitParts = D / kNB;          // CTAs per (sequence, head)
-constexpr int kSplitThreads = 288;
+constexpr int kSplitThreads = 320;
 constexpr uint32_t VO_A1 = 0;                 // [-W; Q̃], two stages of 64 KiB
 constexpr uint32_t VO_KH = 131072;            // K̂^T, 32 KiB
 constexpr uint32_t VO_A4 = 163840;            // per 16 KiB block: rows 0-63 a Ũ stage, rows 64-127 P
@@ -854,6 +855,7 @@ constexpr uint32_t IDESC_N32 = make_idesc(2, 128, 32);
 
 struct VMisc {
     uint64_t full_a1[2], full_u[2], full_k, full_p;   // record parts landed
+    uint64_t empty_a1[2], empty_u[2], empty_kp;       // record buffers free
     uint64_t bar1, bar2, bar4[2];                     // M1 / M2 / M4 done
     uint64_t u_ready, s_ready, o_free[2];             // role hand-offs
     uint32_t tmem_base;
@@ -911,11 +913,14 @@ chain_split_kernel(const uint8_t *__restrict__ recs, const float *h0, float *fin
         for (int s = 0; s < 2; ++s) {
             mbar_init(&m->full_a1[s], 1);
             mbar_init(&m->full_u[s], 1);
+            mbar_init(&m->empty_a1[s], 1);
+            mbar_init(&m->empty_u[s], 64);
             mbar_init(&m->bar4[s], 1);
             mbar_init(&m->o_free[s], 64);
         }
         mbar_init(&m->full_k, 1);
         mbar_init(&m->full_p, 1);
+        mbar_init(&m->empty_kp, 1);
         mbar_init(&m->bar1, 1);
         mbar_init(&m->bar2, 1);
         mbar_init(&m->u_ready, 64);
@@ -1004,6 +1009,7 @@ chain_split_kernel(const uint8_t *__restrict__ recs, const float *h0, float *fin
             fence_proxy_async();
             tc_fence_before();
             mbar_arrive(&m->u_ready);
+            mbar_arrive(&m->empty_u[s]);   // the Ũ stage is read
         }
     } else if (warp < 8) {
         // ================================ output rows (token i), 32 channels ====
@@ -1034,8 +1040,51 @@ chain_split_kernel(const uint8_t *__restrict__ recs, const float *h0, float *fin
                 }
             }
         }
+    } else if (warp == 8) {
+        // ======================================================= MMA issuer ====
+        if (lane == 0) {
+            const uint64_t d_sb = sw128_kmajor_desc(sbase + VO_SB);
+            const uint64_t d_ub = sw128_kmajor_desc(sbase + VO_UB);
+            const uint64_t d_kh = sw128_kmajor_desc(sbase + VO_KH);
+            const uint64_t d_a4 = sw128_kmajor_desc(sbase + VO_A4);
+            for (int lc = 0; lc < nl; ++lc) {
+                if (*abort_flag) break;
+                const uint32_t s = lc & 1, sph = (lc >> 1) & 1;
+                // the buffers are normally ready long before the state block
+                if (!mbar_wait_sleep(&m->full_a1[s], sph)) { fail(ERR_TIMEOUT_TMA); break; }
+                if (lc >= 2 && !mbar_wait_sleep(&m->o_free[s], ((lc - 2) >> 1) & 1)) { fail(ERR_TIMEOUT_HANDOFF); break; }
+                if (!mbar_wait_sleep(&m->s_ready, lc & 1)) { fail(ERR_TIMEOUT_HANDOFF); break; }
+                tc_fence_after();
+                const uint64_t d_a1 = sw128_kmajor_desc(sbase + VO_A1 + s * 65536);
+                const uint32_t d1 = tmem + VT_D1 + s * 32;
+                // descriptors advance by (bytes >> 4) in their start-address field
+#pragma unroll
+                for (int k = 0; k < 16; ++k)
+                    mma_tf32_ss(d1, d_a1 + (((k >> 2) * 16384 + (k & 3) * 32) >> 4),
+                                d_sb + (((k >> 2) * 4096 + (k & 3) * 32) >> 4), IDESC_N32, k != 0);
+                mma_commit(&m->bar1);
+                mma_commit(&m->empty_a1[s]);
+                if (!mbar_wait_sleep(&m->full_k, lc & 1) || !mbar_wait_sleep(&m->full_p, lc & 1)) {
+                    fail(ERR_TIMEOUT_TMA);
+                    break;
+                }
+                if (!mbar_wait_sleep(&m->u_ready, lc & 1)) { fail(ERR_TIMEOUT_HANDOFF); break; }
+                tc_fence_after();
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    mma_tf32_ss(tmem + VT_DS, d_kh + (((k >> 2) * 16384 + (k & 3) * 32) >> 4),
+                                d_ub + (((k >> 2) * 4096 + (k & 3) * 32) >> 4), IDESC_N32, k != 0);
+                mma_commit(&m->bar2);
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    mma_tf32_ss(d1, d_a4 + (((k >> 2) * 16384 + (k & 3) * 32) >> 4),
+                                d_ub + (((k >> 2) * 4096 + (k & 3) * 32) >> 4), IDESC_N32, 1);
+                mma_commit(&m->bar4[s]);
+                mma_commit(&m->empty_kp);
+            }
+        }
     } else if (lane == 0) {
-        // ========================================== MMA and record issuer ====
+        // ==================================================== record loader ====
         uint32_t issued[6] = {0, 0, 0, 0, 0, 0};
         uint64_t *bars[6] = {&m->full_a1[0], &m->full_a1[1], &m->full_u[0], &m->full_u[1],
                              &m->full_k, &m->full_p};
@@ -1069,61 +1118,30 @@ chain_split_kernel(const uint8_t *__restrict__ recs, const float *h0, float *fin
             }
         };
         load_a1(0);
-        load_u(0);
         load_kp(0);
+        load_u(0);
         if (nl > 1) {
             load_a1(1);
             load_u(1);
         }
         prefetch_rec(1);
         prefetch_rec(2);
+        // each buffer is refilled as soon as the step reading it has finished,
+        // in the order those steps finish within a chunk
         for (int lc = 0; lc < nl; ++lc) {
             if (*abort_flag) break;
             const uint32_t s = lc & 1, sph = (lc >> 1) & 1;
-            if (!mbar_wait(&m->s_ready, lc & 1)) { fail(ERR_TIMEOUT_HANDOFF); break; }
-            if (lc >= 2 && !mbar_wait(&m->o_free[s], ((lc - 2) >> 1) & 1)) { fail(ERR_TIMEOUT_HANDOFF); break; }
-            if (!mbar_wait(&m->full_a1[s], sph)) { fail(ERR_TIMEOUT_TMA); break; }
-            tc_fence_after();
-            const uint32_t a1 = sbase + VO_A1 + s * 65536;
-#pragma unroll
-            for (int k = 0; k < 16; ++k)
-                mma_tf32_ss(tmem + VT_D1 + s * 32,
-                            sw128_kmajor_desc(a1 + (k >> 2) * 16384 + (k & 3) * 32),
-                            sw128_kmajor_desc(sbase + VO_SB + (k >> 2) * 4096 + (k & 3) * 32),
-                            IDESC_N32, k != 0);
-            mma_commit(&m->bar1);
-            if (!mbar_wait(&m->u_ready, lc & 1)) { fail(ERR_TIMEOUT_HANDOFF); break; }
-            if (lc + 2 < nl) load_u(lc + 2);          // this Ũ stage is consumed
-            if (!mbar_wait(&m->full_k, lc & 1) || !mbar_wait(&m->full_p, lc & 1)) {
-                fail(ERR_TIMEOUT_TMA);
-                break;
-            }
-            tc_fence_after();
-#pragma unroll
-            for (int k = 0; k < 8; ++k)
-                mma_tf32_ss(tmem + VT_DS,
-                            sw128_kmajor_desc(sbase + VO_KH + (k >> 2) * 16384 + (k & 3) * 32),
-                            sw128_kmajor_desc(sbase + VO_UB + (k >> 2) * 4096 + (k & 3) * 32),
-                            IDESC_N32, k != 0);
-            mma_commit(&m->bar2);
-#pragma unroll
-            for (int k = 0; k < 8; ++k)
-                mma_tf32_ss(tmem + VT_D1 + s * 32,
-                            sw128_kmajor_desc(sbase + VO_A4 + (k >> 2) * 16384 + (k & 3) * 32),
-                            sw128_kmajor_desc(sbase + VO_UB + (k >> 2) * 4096 + (k & 3) * 32),
-                            IDESC_N32, 1);
-            mma_commit(&m->bar4[s]);
-            // M1 done (the U warps saw it): this A1 stage takes chunk lc + 2
-            if (!mbar_wait(&m->bar1, lc & 1)) { fail(ERR_TIMEOUT_MMA); break; }
+            if (!mbar_wait_sleep(&m->empty_a1[s], sph)) { fail(ERR_TIMEOUT_MMA); break; }
             if (lc + 2 < nl) load_a1(lc + 2);
-            // M2 and M4 done: K̂ and P take chunk lc + 1
-            if (!mbar_wait(&m->bar4[s], sph)) { fail(ERR_TIMEOUT_MMA); break; }
+            if (!mbar_wait_sleep(&m->empty_u[s], sph)) { fail(ERR_TIMEOUT_HANDOFF); break; }
+            if (lc + 2 < nl) load_u(lc + 2);
+            if (!mbar_wait_sleep(&m->empty_kp, lc & 1)) { fail(ERR_TIMEOUT_MMA); break; }
             if (lc + 1 < nl) load_kp(lc + 1);
             prefetch_rec(lc + 3);
         }
         // never leave a bulk copy in flight into this CTA's shared memory
         for (int b = 0; b < 6; ++b)
-            if (issued[b] > 0) (void)mbar_wait(bars[b], (issued[b] - 1) & 1);
+            if (issued[b] > 0) (void)mbar_wait_sleep(bars[b], (issued[b] - 1) & 1);
     }
 
     tc_fence_before();

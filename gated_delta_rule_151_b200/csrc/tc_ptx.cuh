@@ -51,6 +51,28 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t phase) {
     return ok != 0;
 }
 
+// try_wait that lets the hardware suspend the thread until the phase
+// completes or `ns` nanoseconds pass, so waiting warps take no issue slots.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t phase, uint32_t ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(phase), "r"(ns)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait that sleeps in hardware between checks: at most 2^16 checks of
+// up to 20 us each (about 1.3 s) before it reports failure.
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t *bar, uint32_t phase) {
+    for (uint32_t it = 0; it < (1u << 16); ++it)
+        if (mbar_try_wait_sleep(bar, phase, 20000u)) return true;
+    return false;
+}
+
 // Bounded wait for the phase with parity `phase` to complete.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t phase) {
     for (uint32_t it = 0; it < kSpinLimit; ++it) {
