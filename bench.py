@@ -167,10 +167,10 @@ def decode_work(inp):
 def split_launches(inp):
     """Kernel launches of the chunk-parallel plan: a prep and a chain kernel
     per window of chunks (the library bounds the chunk records of one window
-    to 1 GiB at 147,968 bytes per chunk and head)."""
+    to 1 GiB at 90,640 bytes per chunk and head)."""
     chains = inp.num_seqs * inp.H
     max_chunks = -(-inp.total_T // 64)
-    window = max(1, min(max_chunks, (1 << 30) // (chains * 147968)))
+    window = max(1, min(max_chunks, (1 << 30) // (chains * 90640)))
     return 2 * (-(-max_chunks // window))
 
 

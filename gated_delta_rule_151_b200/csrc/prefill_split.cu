@@ -19,23 +19,22 @@
 //                 stages the bf16 tiles with TMA, forms A and P with one
 //                 tcgen05 MMA, inverts I + A on CUDA cores, builds the tf32
 //                 operands and forms W and Ũ with two more MMAs.  It writes a
-//                 chunk record to the workspace: -W, Q̃ = Q ⊙ Γ, K̂^T and
-//                 P ⊙ causal as ready-made 128-byte-swizzled shared-memory
-//                 images, Ũ as plain fp32 rows, and exp(G_C).
-//   chain kernel  one CTA per (sequence, head).  It keeps the fp32 state in
-//                 registers (tf32 copy in TMEM) and, per chunk, bulk-copies
-//                 the record into shared memory and runs only the products
-//                 that need the state:
-//                   S1  X^T = S (-W)^T           U^T = Ũ^T + X^T (tf32)
-//                   S1' O^T = S Q̃^T              S3  ΔS = U^T K̂
-//                   S2  O^T += U^T (P ⊙ causal)^T,   S = S Diag(exp(G_C)) + ΔS
-//                 with the record of the next chunks already in flight.
+//                 chunk record to the workspace: [-W; Q̃], K̂^T and P ⊙ causal
+//                 as ready-made fp16 shared-memory operand images, each with a
+//                 power-of-two scale, Ũ as fp32 rows, and exp(G_C).
+//   chain kernel  one CTA per NB value channels of a (sequence, head), NB =
+//                 32, 64 or 128 so that all chain CTAs fit the GPU at once.
+//                 Per chunk it bulk-copies the record and runs only the
+//                 products that need the state (fp16 operands, fp32
+//                 accumulation, the state itself in fp32 registers), with the
+//                 next records already in flight.
 //
-// The chain kernel does per chunk what the single-kernel plan's chain group
-// does; the prep work that bounds that plan's chunk period moves to
-// otherwise idle SMs.  Records take 144.5 KiB per (chunk, head); problems
-// whose records exceed 1 GiB run in windows of chunks, the state passing
-// between windows through the workspace.
+// fp16 with a per-block power-of-two scale keeps the 11-bit significand of
+// tf32 at half the bytes and twice the MMA depth; the chain is bound by the
+// shared-memory traffic of its operands, so halving them is what counts.
+// Records take 90,640 bytes per (chunk, head); problems whose records exceed
+// 1 GiB run in windows of chunks, the state passing between windows through
+// the workspace.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_fp16.h>
@@ -57,22 +56,51 @@ constexpr uint32_t ERR_TIMEOUT_TMA = 1u, ERR_TIMEOUT_MMA = 2u, ERR_TIMEOUT_HANDO
                    ERR_SMEM_ALIGN = 8u;
 
 // ----------------------------------------------------------- chunk record ----
-// Byte offsets inside one record.  The images use the layout the chain
-// kernel's MMA descriptors read (128-byte rows, 16-byte chunks XOR-swizzled
-// by row % 8, blocks 1024-byte aligned).
-constexpr uint32_t REC_A1 = 0;          // [-W; Q̃] [tok][dk] tf32: per 32-dk block (16 KiB) the
-                                        //   64 rows of -W, then the 64 rows of Q̃ (128 x 128 B)
-constexpr uint32_t REC_KH = 65536;      // K̂^T [dk][tok] tf32: 2 blocks (32 tok) of 128 x 128 B
-constexpr uint32_t REC_PM = 98304;      // P ⊙ causal [i][j] tf32: 2 blocks (32 j) of 64 x 128 B
-constexpr uint32_t REC_UT = 114688;     // Ũ fp32: 4 blocks of 32 dv, each [tok][32] with the
+// Byte offsets inside one record.  The operand images are fp16 in the layout
+// the chain kernel's MMA descriptors read: rows of 64 halves (128 bytes) whose
+// 16-byte chunks are XOR-swizzled by row % 8, blocks 1024-byte aligned.  Each
+// image block is scaled by a power of two 2^s chosen so that its largest
+// magnitude lies in [2^14, 2^15): fp16 then carries the same 11-bit
+// significand as tf32 for every value above 2^-29 of the block maximum, and
+// the exponents s travel in the record.
+constexpr uint32_t REC_A1 = 0;          // [-W; Q̃] [tok][dk]: 2 blocks (64 dk) of 128 rows,
+                                        //   rows 0-63 -W (scale s_W), rows 64-127 Q̃ (s_Q)
+constexpr uint32_t REC_KH = 32768;      // K̂^T [dk][tok]: 128 rows (s_K)
+constexpr uint32_t REC_PM = 49152;      // P ⊙ causal [i][j]: 64 rows (s_P)
+constexpr uint32_t REC_UT = 57344;      // Ũ fp32: 4 blocks of 32 dv, each [tok][32] with the
                                         //   16-byte chunks of row i XOR-swizzled by i % 8
-constexpr uint32_t REC_GC = 147456;     // exp(G_C): 1 float (scalar) or 128 (channel)
-constexpr uint32_t REC_BYTES = 147968;
-static_assert(REC_BYTES % 16 == 0 && REC_GC + 512 == REC_BYTES, "record layout");
+constexpr uint32_t REC_GC = 90112;      // exp(G_C): 1 float (scalar) or 128 (channel)
+constexpr uint32_t REC_EX = 90624;      // int32 {s_W, s_Q, s_K, s_P}
+constexpr uint32_t REC_BYTES = 90640;
+static_assert(REC_BYTES % 16 == 0 && REC_EX + 16 == REC_BYTES, "record layout");
+
+// Byte offset of fp16 element (r, c) (c < 64) inside a block of 128-byte rows.
+__host__ __device__ constexpr uint32_t h16_offset(uint32_t r, uint32_t c) {
+    return r * 128u + ((((c >> 3) ^ (r & 7u)) & 7u) << 4) + (c & 7u) * 2u;
+}
 
 // Byte offset of Ũ[i][dv] inside the record.
 __host__ __device__ constexpr uint32_t rec_ut_offset(uint32_t i, uint32_t dv) {
     return REC_UT + (dv >> 5) * 8192 + i * 128 + (((((dv & 31) >> 2) ^ (i & 7)) << 4) | ((dv & 3) << 2));
+}
+
+// Scale exponent s for a block whose largest magnitude is mx: mx 2^s lies in
+// [2^14, 2^15).  Zero, subnormal-only or non-finite maxima give safe values;
+// s is clamped to [-100, 100] so that 2^s and 2^-s stay normal floats.
+__device__ __forceinline__ int scale_exp(float mx) {
+    if (!(mx > 0.f) || !(mx < 3.0e38f)) return 0;
+    const int e = (int)((__float_as_uint(mx) >> 23) & 255u) - 127;
+    return min(max(14 - e, -100), 100);
+}
+
+// 2^s for |s| <= 126.
+__device__ __forceinline__ float exp2i(int s) { return __int_as_float((127 + s) << 23); }
+
+__device__ __forceinline__ uint16_t f2h_bits(float x) { return __half_as_ushort(__float2half_rn(x)); }
+
+__device__ __forceinline__ uint32_t f2h2_bits(float a, float b) {
+    const __half2 h = __floats2half2_rn(a, b);
+    return *reinterpret_cast<const uint32_t *>(&h);
 }
 
 // ------------------------------------------------------------ prep kernel ----
@@ -99,6 +127,7 @@ struct PrepMisc {
             float beta[C], T0[D], T1[D];
         } c;
     } u;                               // beta comes first in both layouts
+    float red[2][8];                   // per-warp maxima for the image scales
 };
 static_assert(sizeof(PrepMisc) <= 2048, "prep misc area overflow");
 static_assert(offsetof(PrepMisc, u) % 16 == 0, "prep misc arrays misaligned");
@@ -107,8 +136,30 @@ __device__ __forceinline__ void st_global_v4(uint8_t *p, uint32_t a, uint32_t b,
                                              uint32_t d) {
     *reinterpret_cast<uint4 *>(p) = make_uint4(a, b, c, d);
 }
-__device__ __forceinline__ void st_global_b32(uint8_t *p, uint32_t a) {
-    *reinterpret_cast<uint32_t *>(p) = a;
+__device__ __forceinline__ void st_global_b16(uint8_t *p, uint16_t a) {
+    *reinterpret_cast<uint16_t *>(p) = a;
+}
+
+// Scale exponents of two blocks from every thread's largest |value| of each
+// (a, b >= 0); all 256 threads call it (two __syncthreads inside).
+__device__ __forceinline__ void block_scale2(float a, float b, float (*red)[8], int &sa, int &sb) {
+    const uint32_t ua = __reduce_max_sync(0xffffffffu, __float_as_uint(a));
+    const uint32_t ub = __reduce_max_sync(0xffffffffu, __float_as_uint(b));
+    const int w = threadIdx.x >> 5;
+    if ((threadIdx.x & 31) == 0) {
+        red[0][w] = __uint_as_float(ua);
+        red[1][w] = __uint_as_float(ub);
+    }
+    __syncthreads();
+    float ma = 0.f, mb = 0.f;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        ma = fmaxf(ma, red[0][k]);
+        mb = fmaxf(mb, red[1][k]);
+    }
+    __syncthreads();
+    sa = scale_exp(ma);
+    sb = scale_exp(mb);
 }
 
 // Bounded wait by every thread of the block; all threads agree on stopping.
@@ -292,7 +343,8 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             tc_fence_after();
         }
 
-        // ---- A (fp32 scratch) and P ⊙ causal (record image, tf32) -----------
+        // ---- A (fp32 scratch) and P ⊙ causal (record image, fp16) -----------
+        int sP = 0, sQ = 0, sK = 0, sW = 0;   // record image scale exponents
         float *Af;
         float *Tf;
         float *Xs;
@@ -309,6 +361,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             const int i = row < C ? row : row - C;
             const float Gi = CHANNEL ? 0.f : m->u.s.G[i];
             const float rowf = (row < C ? m->u.s.beta[i] : 1.f) * (CHANNEL ? 1.f : m->u.s.gam[i]);
+            float pv[32];   // P row i, columns half*32 .. +31 (rows 64-127 of P1)
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
                 const int j0 = half * 32 + q * 4;
@@ -326,11 +379,29 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     const bool keep = row < C ? (j < i) : (j <= i);
                     v4[e] = keep ? f * __uint_as_float(x[q * 4 + e]) : 0.f;
                 }
-                if (row < C)
+                if (row < C) {
                     st4(Af, i, j0, make_float4(v4[0], v4[1], v4[2], v4[3]));
-                else
-                    st_global_v4(rec + REC_PM + half * 8192 + sw128_offset(i, q), to_tf32(v4[0]),
-                                 to_tf32(v4[1]), to_tf32(v4[2]), to_tf32(v4[3]));
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) pv[q * 4 + e] = v4[e];
+                }
+            }
+            float pm = 0.f;
+            if (row >= C) {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) pm = fmaxf(pm, fabsf(pv[e]));
+            }
+            int unused;
+            block_scale2(pm, 0.f, m->red, sP, unused);
+            if (row >= C) {
+                const float f = exp2i(sP);
+#pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4) {
+                    const float *v = pv + c4 * 8;
+                    st_global_v4(rec + REC_PM + i * 128 + ((((half * 4 + c4) ^ (i & 7)) & 7) << 4),
+                                 f2h2_bits(v[0] * f, v[1] * f), f2h2_bits(v[2] * f, v[3] * f),
+                                 f2h2_bits(v[4] * f, v[5] * f), f2h2_bits(v[6] * f, v[7] * f));
+                }
             }
         } else {
             // exact A and P on CUDA cores: G [64][128] fp32 in X1, A in TM
@@ -341,32 +412,56 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 #pragma unroll
             for (int k = 0; k < 32; ++k) Gs[(hh * 32 + k) * D + ch] = gr[k];
             __syncthreads();
-            for (int pr = tid; pr < C * (C + 1) / 2; pr += kPrepThreads) {
-                int i = (int)((sqrtf(8.f * (float)pr + 1.f) - 1.f) * 0.5f);
+            // pair pr = i (i + 1) / 2 + j (j <= i); each thread keeps its P values
+            // until the block's scale is known
+            constexpr int kPairIters = (C * (C + 1) / 2 + kPrepThreads - 1) / kPrepThreads;
+            auto pair_ij = [](int pr, int &i, int &j) {
+                i = (int)((sqrtf(8.f * (float)pr + 1.f) - 1.f) * 0.5f);
                 while (i * (i + 1) / 2 > pr) --i;
                 while ((i + 1) * (i + 2) / 2 <= pr) ++i;
-                const int j = pr - i * (i + 1) / 2;
-                float dk = 0.f, dq = 0.f;
-                for (int cc = 0; cc < D; ++cc) {
-                    const uint32_t kc = (cc >> 6) * 16384, chk = (cc & 63) >> 3, el = (cc & 7) * 2;
-                    const float ki = ld_shared_bf16(sbase + PO_KQ + kc + sw128_offset(i, chk) + el);
-                    const float qi = ld_shared_bf16(sbase + PO_KQ + kc + 8192 + sw128_offset(i, chk) + el);
-                    const float kj = ld_shared_bf16(sbase + PO_KQ + kc + sw128_offset(j, chk) + el);
-                    const float e = __expf(Gs[i * D + cc] - Gs[j * D + cc]) * kj;
-                    dk = fmaf(ki, e, dk);
-                    dq = fmaf(qi, e, dq);
+                j = pr - i * (i + 1) / 2;
+            };
+            float dqs[kPairIters];
+            float pm = 0.f;
+#pragma unroll
+            for (int it = 0; it < kPairIters; ++it) {
+                const int pr = tid + it * kPrepThreads;
+                dqs[it] = 0.f;
+                if (pr < C * (C + 1) / 2) {
+                    int i, j;
+                    pair_ij(pr, i, j);
+                    float dk = 0.f, dq = 0.f;
+                    for (int cc = 0; cc < D; ++cc) {
+                        const uint32_t kc = (cc >> 6) * 16384, chk = (cc & 63) >> 3, el = (cc & 7) * 2;
+                        const float ki = ld_shared_bf16(sbase + PO_KQ + kc + sw128_offset(i, chk) + el);
+                        const float qi = ld_shared_bf16(sbase + PO_KQ + kc + 8192 + sw128_offset(i, chk) + el);
+                        const float kj = ld_shared_bf16(sbase + PO_KQ + kc + sw128_offset(j, chk) + el);
+                        const float e = __expf(Gs[i * D + cc] - Gs[j * D + cc]) * kj;
+                        dk = fmaf(ki, e, dk);
+                        dq = fmaf(qi, e, dq);
+                    }
+                    Af[ax(i, j)] = (j < i) ? m->u.c.beta[i] * dk : 0.f;
+                    dqs[it] = dq;
+                    pm = fmaxf(pm, fabsf(dq));
                 }
-                Af[ax(i, j)] = (j < i) ? m->u.c.beta[i] * dk : 0.f;
-                st_global_b32(rec + REC_PM + (j >> 5) * 8192 + sw128_offset(i, (j & 31) >> 2) + (j & 3) * 4,
-                              to_tf32(dq));
             }
             for (int e = tid; e < C * C; e += kPrepThreads) {
                 const int i = e >> 6, j = e & 63;
                 if (j > i) {
                     Af[ax(i, j)] = 0.f;
-                    st_global_b32(rec + REC_PM + (j >> 5) * 8192 + sw128_offset(i, (j & 31) >> 2) +
-                                      (j & 3) * 4,
-                                  0u);
+                    st_global_b16(rec + REC_PM + h16_offset(i, j), 0);
+                }
+            }
+            int unused;
+            block_scale2(pm, 0.f, m->red, sP, unused);
+            const float f = exp2i(sP);
+#pragma unroll
+            for (int it = 0; it < kPairIters; ++it) {
+                const int pr = tid + it * kPrepThreads;
+                if (pr < C * (C + 1) / 2) {
+                    int i, j;
+                    pair_ij(pr, i, j);
+                    st_global_b16(rec + REC_PM + h16_offset(i, j), f2h_bits(dqs[it] * f));
                 }
             }
         }
@@ -376,10 +471,27 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         unit_lower_inverse(Af, Tf, Xs, sbase + PO_TM, tid);
         __syncthreads();
 
-        // ---- operands, pass 1: K'^T (X1), K̂^T and Q̃ (record) from K and Q ----
+        // ---- operands, pass 1: K'^T (X1, tf32), K̂^T and Q̃ (record, fp16) ------
         if (!CHANNEL) {
             const int i = tid & 63;
             const float kp = m->u.s.kp[i], kh = m->u.s.kh[i], gq = m->u.s.gam[i];
+            // the chunk's largest |K̂| and |Q̃| set their image scales
+            float mk = 0.f, mq = 0.f;
+#pragma unroll 1
+            for (int it = 0; it < 4; ++it) {
+                const int jc = (tid >> 6) + 4 * it;
+                const uint32_t kb = jc >> 3, chk = jc & 7;
+                float kf[8], qf[8];
+                bf16x8_to_f32(ld_shared_v4(sbase + PO_KQ + kb * 16384 + sw128_offset(i, chk)), kf);
+                bf16x8_to_f32(ld_shared_v4(sbase + PO_KQ + kb * 16384 + 8192 + sw128_offset(i, chk)), qf);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    mk = fmaxf(mk, fabsf(kh * kf[e]));
+                    mq = fmaxf(mq, fabsf(gq * qf[e]));
+                }
+            }
+            block_scale2(mk, mq, m->red, sK, sQ);
+            const float fk = exp2i(sK), fq = exp2i(sQ);
             const uint32_t tcol = (i >> 5) * 16384;
             const uint32_t tchunk = (i & 31) >> 2, tel = (i & 3) * 4;
 #pragma unroll 1
@@ -392,37 +504,53 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     const uint32_t j = jc * 8 + e;
-                    const uint32_t off = tcol + sw128_offset(j, tchunk) + tel;
-                    st_shared_b32(sbase + PO_X1 + off, to_tf32(kp * kf[e]));
-                    st_global_b32(rec + REC_KH + off, to_tf32(kh * kf[e]));
+                    st_shared_b32(sbase + PO_X1 + tcol + sw128_offset(j, tchunk) + tel, to_tf32(kp * kf[e]));
+                    st_global_b16(rec + REC_KH + h16_offset(j, i), f2h_bits(kh * kf[e] * fk));
                 }
-                uint8_t *qb = rec + REC_A1 + (jc >> 2) * 16384 + 8192;
-                const uint32_t qc = (jc & 3) * 2;
-                st_global_v4(qb + sw128_offset(i, qc), to_tf32(gq * qf[0]), to_tf32(gq * qf[1]),
-                             to_tf32(gq * qf[2]), to_tf32(gq * qf[3]));
-                st_global_v4(qb + sw128_offset(i, qc + 1), to_tf32(gq * qf[4]), to_tf32(gq * qf[5]),
-                             to_tf32(gq * qf[6]), to_tf32(gq * qf[7]));
+                // Q̃ row 64 + i, channels jc*8 .. +7: one 16-byte chunk
+                st_global_v4(rec + REC_A1 + kb * 16384 + (64 + i) * 128 + (((chk ^ (i & 7)) & 7) << 4),
+                             f2h2_bits(gq * qf[0] * fq, gq * qf[1] * fq),
+                             f2h2_bits(gq * qf[2] * fq, gq * qf[3] * fq),
+                             f2h2_bits(gq * qf[4] * fq, gq * qf[5] * fq),
+                             f2h2_bits(gq * qf[6] * fq, gq * qf[7] * fq));
             }
         } else {
             const uint32_t kcol = (ch >> 6) * 16384, cch = (ch & 63) >> 3, cel = (ch & 7) * 2;
+            float mk = 0.f, mq = 0.f;
+#pragma unroll 4
+            for (int k = 0; k < 32; ++k) {
+                const int i = hh * 32 + k;
+                const uint32_t src = sbase + PO_KQ + kcol + sw128_offset(i, cch) + cel;
+                mk = fmaxf(mk, fabsf(ld_shared_bf16(src) * __expf(GC - gr[k])));
+                mq = fmaxf(mq, fabsf(ld_shared_bf16(src + 8192) * __expf(gr[k])));
+            }
+            block_scale2(mk, mq, m->red, sK, sQ);
+            const float fk = exp2i(sK), fq = exp2i(sQ);
             const uint32_t rowblk = hh * 16384;
-            const uint32_t qoff = REC_A1 + (ch >> 5) * 16384 + 8192 + (ch & 3) * 4;
-            const uint32_t qch = (ch & 31) >> 2;
+            uint8_t *qdst = rec + REC_A1 + (ch >> 6) * 16384;
 #pragma unroll
-            for (int q4 = 0; q4 < 8; ++q4) {
-                uint32_t wk[4], wh[4];
+            for (int c8 = 0; c8 < 4; ++c8) {   // tokens hh*32 + c8*8 .. +7
+                float wh[8];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int k = q4 * 4 + e, i = hh * 32 + k;
-                    const uint32_t src = sbase + PO_KQ + kcol + sw128_offset(i, cch) + cel;
-                    const float kv = ld_shared_bf16(src), qv = ld_shared_bf16(src + 8192);
-                    const float eg = __expf(gr[k]);
-                    wk[e] = to_tf32(m->u.c.beta[i] * kv * eg);
-                    wh[e] = to_tf32(kv * __expf(GC - gr[k]));
-                    st_global_b32(rec + qoff + sw128_offset(i, qch), to_tf32(qv * eg));
+                for (int q2 = 0; q2 < 2; ++q2) {
+                    const int q4 = c8 * 2 + q2;
+                    uint32_t wk[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int k = q4 * 4 + e, i = hh * 32 + k;
+                        const uint32_t src = sbase + PO_KQ + kcol + sw128_offset(i, cch) + cel;
+                        const float kv = ld_shared_bf16(src), qv = ld_shared_bf16(src + 8192);
+                        const float eg = __expf(gr[k]);
+                        wk[e] = to_tf32(m->u.c.beta[i] * kv * eg);
+                        wh[q2 * 4 + e] = kv * __expf(GC - gr[k]) * fk;
+                        st_global_b16(qdst + h16_offset(64 + i, ch & 63), f2h_bits(qv * eg * fq));
+                    }
+                    st_shared_v4(sbase + PO_X1 + rowblk + sw128_offset(ch, q4), wk[0], wk[1], wk[2], wk[3]);
                 }
-                st_shared_v4(sbase + PO_X1 + rowblk + sw128_offset(ch, q4), wk[0], wk[1], wk[2], wk[3]);
-                st_global_v4(rec + REC_KH + rowblk + sw128_offset(ch, q4), wh[0], wh[1], wh[2], wh[3]);
+                // K̂^T row ch, tokens hh*32 + c8*8 .. +7: one 16-byte chunk
+                st_global_v4(rec + REC_KH + ch * 128 + ((((hh * 4 + c8) ^ (ch & 7)) & 7) << 4),
+                             f2h2_bits(wh[0], wh[1]), f2h2_bits(wh[2], wh[3]), f2h2_bits(wh[4], wh[5]),
+                             f2h2_bits(wh[6], wh[7]));
             }
         }
         __syncthreads();   // K and Q are consumed: V'^T takes their place
@@ -481,17 +609,24 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         if (!block_wait(&m->bar_mma, slow ? 0 : 1, &m->abort_flag, err, ERR_TIMEOUT_MMA)) break;
         tc_fence_after();
 
-        // ---- -W (image) and Ũ (rows) into the record; thread = d row -----------
+        // ---- -W (fp16 image) and Ũ (fp32 rows) into the record; thread = d row --
         {
             uint32_t x[32];
             tmem_ld32(tmem + lane_off + PT_W + half * 32, x);
             tmem_wait_ld();
+            float mw = 0.f;
+#pragma unroll
+            for (int ii = 0; ii < 32; ++ii) mw = fmaxf(mw, fabsf(__uint_as_float(x[ii])));
+            int unused;
+            block_scale2(mw, 0.f, m->red, sW, unused);
+            const float fw = -exp2i(sW);
             const uint32_t j = row;
-            uint8_t *base = rec + REC_A1 + (j >> 5) * 16384 + (j & 3) * 4;
+            uint8_t *base = rec + REC_A1 + (j >> 6) * 16384;
 #pragma unroll
             for (int ii = 0; ii < 32; ++ii)
-                st_global_b32(base + sw128_offset(half * 32 + ii, (j & 31) >> 2),
-                              to_tf32(-__uint_as_float(x[ii])));
+                st_global_b16(base + h16_offset(half * 32 + ii, j & 63), f2h_bits(__uint_as_float(x[ii]) * fw));
+            if (tid == 0)
+                *reinterpret_cast<int4 *>(rec + REC_EX) = make_int4(sW, sQ, sK, sP);
             tmem_ld32(tmem + lane_off + PT_U + half * 32, x);
             tmem_wait_ld();
 #pragma unroll
@@ -509,377 +644,112 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     }
 }
 
-// ------------------------------------------- chain kernel, one head per CTA ----
-// Transposed products (TMEM lane = value channel), 256 threads: thread
-// (lane group, half) owns one row of S, 64 columns.
-constexpr int kChainThreads = 256;
-constexpr uint32_t CO_A1 = 0;         // [-W; Q̃] record images, two stages of 64 KiB
-constexpr uint32_t CO_PM = 131072;    // P, two stages of 16 KiB
-constexpr uint32_t CO_KH = 163840;    // K̂^T, 32 KiB
-constexpr uint32_t CO_UT = 196608;    // Ũ, 32 KiB
-constexpr uint32_t CO_MISC = 229376;
-constexpr uint32_t CHAIN_SMEM = CO_MISC + 2048;   // 231424
-// TMEM columns: O (two buffers), U, ΔS, tf32 copy of S.
-constexpr uint32_t CT_O = 0, CT_U = 128, CT_DS = 256, CT_S = 384, CHAIN_TMEM_COLS = 512;
+// ----------------------------------------------------------- chain kernel ----
+// Each CTA owns NB value channels (a column block of S^T) of one (sequence,
+// head); the (D / NB) CTAs of a head run in lockstep on the same records.
+// Every product keeps the 128-row M dimension on [W; Q̃] or on d_k, with
+// fp16 operands (K = 16 per MMA) and fp32 accumulators:
+//
+//   M1  D1 = [-W; Q̃] S_b^T          rows 0-63: X = -W S_b^T
+//                                   rows 64-127: the inter-chunk output Q̃ S_b^T
+//   M2  D2 = K̂^T U_b                ΔS_b^T
+//   M4  D4 = [junk; P ⊙ causal] U_b rows 64-127: the intra-chunk output
+//
+// U_b = Ũ_b + X and S_b^T = S_b^T Diag(exp(G_C)) + ΔS_b^T are formed in fp32
+// (the state block stays in registers, thread = d_k row) and written back as
+// fp16 images with a fresh power-of-two scale each chunk; every accumulator
+// is unscaled by the exponents of its two operands.  Warp roles: state
+// block, U (tokens 0-63 of D1), output (tokens 64-127 of D1 and D4), the MMA
+// issuer and the record loader, handing off through mbarriers only; record
+// buffers are freed by tcgen05.commit of the MMAs that read them.
+template <int NB>
+struct Chain {
+    static constexpr int kSW = NB <= 64 ? 4 : 8;         // state warps
+    static constexpr int kCS = NB * 4 / kSW;              // state columns per thread
+    static constexpr int kSets = NB <= 64 ? 1 : 2;        // sets of (2 U warps, 2 output warps)
+    static constexpr int kCU = NB / kSets;                // U / output columns per thread
+    static constexpr int kIssuer = kSW + 4 * kSets;       // MMA issuer warp; the loader follows
+    static constexpr int kThreads = 32 * (kIssuer + 2);
+    static constexpr bool kDB = NB <= 64;                 // two K̂/P stages and O buffers
+    static constexpr int kStages = kDB ? 2 : 1;
+    static constexpr uint32_t A1 = 0;                     // [-W; Q̃], 2 stages of 32 KiB
+    static constexpr uint32_t KH = 65536;                 // K̂^T, 16 KiB per stage
+    static constexpr uint32_t A4 = KH + kStages * 16384;  // [junk; P], 16 KiB per stage
+    static constexpr uint32_t UT = A4 + kStages * 16384;  // Ũ fp32, 2 stages of 256 NB bytes
+    static constexpr uint32_t SB = UT + 512 * NB;         // S_b image [NB][128], 256 NB bytes
+    static constexpr uint32_t UB = SB + 256 * NB;         // U_b^T image [NB][64], 128 NB bytes
+    static constexpr uint32_t MISC = UB + 128 * NB;
+    static constexpr uint32_t SMEM = MISC + 1024;
+    static constexpr uint32_t TD1 = 0;                    // per O buffer
+    static constexpr uint32_t TD4 = kStages * NB;         // per O buffer
+    static constexpr uint32_t TD2 = 2 * kStages * NB;
+    static constexpr uint32_t TCOLS = TD2 + NB <= 256 ? 256 : 512;
+    static constexpr uint32_t IDESC = make_idesc(0, 128, NB);   // fp16 x fp16 -> fp32
+    static_assert(SMEM <= 232448 && TD2 + NB <= 512, "chain kernel does not fit");
+};
 
 struct ChainMisc {
-    uint64_t full_a1[2], full_p[2], full_u, full_k;   // record parts landed
-    uint64_t bar_s1, bar_s3, bar_o;                   // MMA groups done
+    uint64_t full_a1[2], full_u[2], full_kp[2];     // record parts landed
+    uint64_t empty_a1[2], empty_u[2], empty_kp[2];  // record buffers free
+    uint64_t bar1, bar2, bar4[2];                   // M1 / M2 / M4 done
+    uint64_t s_ready, u_ready, o_free[2], osc_full[2];
     uint32_t tmem_base;
     int abort_flag;
-    alignas(16) float gam[2][D];                      // exp(G_C), with the P stage
+    int es[4];                  // S image exponent, per chunk mod 4
+    int dsx[2][2];              // {s_K, s_U}, per chunk parity
+    int osx[2][4];              // {s_Q, s_S, s_P, s_U}, per chunk parity
+    alignas(16) int ex[2][4];   // record exponents {s_W, s_Q, s_K, s_P}, with the Ũ stage
+    float red_s[2][8], red_u[2][4];
 };
-static_assert(sizeof(ChainMisc) <= 2048, "chain misc area overflow");
-
-// Bounded wait by all 256 threads; all agree on stopping.
-__device__ __forceinline__ bool chain_wait(uint64_t *bar, uint32_t phase, ChainMisc *m,
-                                           uint32_t *err, uint32_t code) {
-    if (!mbar_wait(bar, phase)) {
-        m->abort_flag = 1;
-        atomicOr(err, code);
-    }
-    group_sync(1);
-    return *reinterpret_cast<volatile int *>(&m->abort_flag) == 0;
-}
-
-template <bool CHANNEL>
-__global__ void __launch_bounds__(kChainThreads, 1)
-chain_kernel(const uint8_t *__restrict__ recs, const float *h0, float *fin, float *ws_state,
-             const int32_t *__restrict__ cu, int num_seqs, int total_T, int H, int c_begin,
-             int c_end, __nv_bfloat16 *__restrict__ o, uint32_t *err) {
-    extern __shared__ __align__(1024) uint8_t smem_raw[];
-    const uint32_t sbase = smem_u32(smem_raw);
-    const int chain = blockIdx.x, chains = gridDim.x;
-    const int h = chain % H, n = chain / H;
-    int t0, len;
-    sequence_range(cu, n, num_seqs, total_T, t0, len);
-    const int nchunks = (len + C - 1) / C;
-    if (c_begin > 0 && c_begin >= nchunks) return;   // finished in an earlier window
-    const int c_stop = min(c_end, nchunks);
-    const int nl = max(c_stop - c_begin, 0);
-    const float *s_in = c_begin == 0 ? h0 : ws_state;
-    float *s_out = c_stop == nchunks ? fin : ws_state;
-
-    const int tid = threadIdx.x;
-    const int warp = tid >> 5, lane = tid & 31;
-    const int sub = warp & 3;
-    const int half = warp >> 2;          // state columns half*64 .. +63
-    const int row = sub * 32 + lane;     // TMEM lane = value channel
-    const uint32_t lane_off = static_cast<uint32_t>(sub * 32) << 16;
-    const size_t sg = (((size_t)n * H + h) * D + row) * D + half * 64;
-
-    float S[64];
-#pragma unroll
-    for (int j = 0; j < 64; j += 4) {
-        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (s_in != nullptr) x = *reinterpret_cast<const float4 *>(s_in + sg + j);
-        S[j] = x.x; S[j + 1] = x.y; S[j + 2] = x.z; S[j + 3] = x.w;
-    }
-    if (nl == 0) {   // empty sequence: the state passes through
-        if (s_out != nullptr) {
-#pragma unroll
-            for (int j = 0; j < 64; j += 4)
-                *reinterpret_cast<float4 *>(s_out + sg + j) =
-                    make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
-        }
-        return;
-    }
-    if ((sbase & 1023u) != 0) {
-        if (tid == 0) atomicOr(err, ERR_SMEM_ALIGN);
-        return;
-    }
-    uint8_t *sm = smem_raw;
-    ChainMisc *m = reinterpret_cast<ChainMisc *>(sm + CO_MISC);
-    if (tid == 0) {
-        mbar_init(&m->full_a1[0], 1);
-        mbar_init(&m->full_a1[1], 1);
-        mbar_init(&m->full_p[0], 1);
-        mbar_init(&m->full_p[1], 1);
-        mbar_init(&m->full_u, 1);
-        mbar_init(&m->full_k, 1);
-        mbar_init(&m->bar_s1, 1);
-        mbar_init(&m->bar_s3, 1);
-        mbar_init(&m->bar_o, 1);
-        m->abort_flag = 0;
-        fence_barrier_init();
-    }
-    if (warp == 0) {
-        tmem_alloc(&m->tmem_base, CHAIN_TMEM_COLS);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = m->tmem_base;
-
-    {   // tf32 copy of the entering state: A operand of S1 and S1'
-        uint32_t r[32];
-#pragma unroll
-        for (int part = 0; part < 2; ++part) {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) r[j] = to_tf32(S[part * 32 + j]);
-            tmem_st32(tmem + lane_off + CT_S + half * 64 + part * 32, r);
-        }
-        tmem_wait_st();
-    }
-
-    // Record loads, issued by thread 0 as soon as the buffer they overwrite is
-    // free.  Loads per buffer are counted so that an aborted run can wait for
-    // the ones still in flight before the CTA exits.
-    const uint32_t gbytes = CHANNEL ? 512u : 16u;
-    uint32_t issued[6] = {0, 0, 0, 0, 0, 0};
-    uint64_t *bars[6] = {&m->full_a1[0], &m->full_a1[1], &m->full_p[0], &m->full_p[1], &m->full_u,
-                         &m->full_k};
-    auto rec_of = [&](int lc) {
-        return recs + ((size_t)lc * chains + chain) * REC_BYTES;
-    };
-    auto load_a1 = [&](int lc) {
-        const int s = lc & 1;
-        mbar_arrive_expect_tx(&m->full_a1[s], 65536);
-        bulk_load(sm + CO_A1 + s * 65536, rec_of(lc) + REC_A1, 65536, &m->full_a1[s]);
-        ++issued[s];
-    };
-    auto load_p = [&](int lc) {
-        const int s = lc & 1;
-        const uint8_t *r = rec_of(lc);
-        mbar_arrive_expect_tx(&m->full_p[s], 16384 + gbytes);
-        bulk_load(sm + CO_PM + s * 16384, r + REC_PM, 16384, &m->full_p[s]);
-        bulk_load(m->gam[s], r + REC_GC, gbytes, &m->full_p[s]);
-        ++issued[2 + s];
-    };
-    auto load_u = [&](int lc) {
-        mbar_arrive_expect_tx(&m->full_u, 32768);
-        bulk_load(sm + CO_UT, rec_of(lc) + REC_UT, 32768, &m->full_u);
-        ++issued[4];
-    };
-    auto load_k = [&](int lc) {
-        mbar_arrive_expect_tx(&m->full_k, 32768);
-        bulk_load(sm + CO_KH, rec_of(lc) + REC_KH, 32768, &m->full_k);
-        ++issued[5];
-    };
-    auto prefetch_rec = [&](int lc) {
-        if (lc < nl) {
-            const uint8_t *r = rec_of(lc);
-#pragma unroll
-            for (int part = 0; part < 4; ++part) bulk_prefetch_l2(r + part * 36992, 36992);
-        }
-    };
-    if (tid == 0) {
-        load_a1(0);
-        load_p(0);
-        load_u(0);
-        load_k(0);
-        if (nl > 1) {
-            load_a1(1);
-            load_p(1);
-        }
-        prefetch_rec(2);
-        prefetch_rec(3);
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-
-    // output of a finished chunk: lane = value channel, TMEM columns = tokens
-    auto store_o = [&](int cc, uint32_t col) {
-        const int tok0 = t0 + cc * C;
-        const int cl = min(C, len - cc * C);
-        uint32_t x[32];
-        tmem_ld32(tmem + lane_off + col + half * 32, x);
-        tmem_wait_ld();
-#pragma unroll
-        for (int ii = 0; ii < 32; ++ii) {
-            const int i = half * 32 + ii;
-            if (i < cl)
-                o[((size_t)(tok0 + i) * H + h) * D + row] = __float2bfloat16_rn(__uint_as_float(x[ii]));
-        }
-    };
-    auto fail = [&](uint32_t code) {
-        m->abort_flag = 1;
-        atomicOr(err, code);
-    };
-
-    bool ok = true;
-    for (int lc = 0; lc < nl; ++lc) {
-        const uint32_t par = lc & 1, sph = (lc >> 1) & 1;
-        const uint32_t tmO = CT_O + par * 64;
-        const uint32_t a1 = sbase + CO_A1 + par * 65536;
-        // The previous chunk's S1'/S2 are done: its O is readable, U (TMEM) may
-        // be overwritten and its P stage takes the chunk after this one.
-        if (lc >= 1) {
-            if (!chain_wait(&m->bar_o, (lc - 1) & 1, m, err, ERR_TIMEOUT_MMA)) { ok = false; break; }
-            tc_fence_after();
-            if (tid == 0 && lc + 1 < nl) load_p(lc + 1);
-        }
-        if (tid == 0) {
-            if (!mbar_wait(&m->full_a1[par], sph)) {
-                fail(ERR_TIMEOUT_TMA);
-            } else {
-                tc_fence_after();
-                // S1: X^T = S (-W)^T, the only product on the state's path
-#pragma unroll
-                for (int k = 0; k < 16; ++k)
-                    mma_tf32_ts(tmem + CT_U, tmem + CT_S + k * 8,
-                                sw128_kmajor_desc(a1 + (k >> 2) * 16384 + (k & 3) * 32), IDESC_N64,
-                                k != 0);
-                mma_commit(&m->bar_s1);
-                // S1': O^T = S Q̃^T (runs while U is formed)
-#pragma unroll
-                for (int k = 0; k < 16; ++k)
-                    mma_tf32_ts(tmem + tmO, tmem + CT_S + k * 8,
-                                sw128_kmajor_desc(a1 + (k >> 2) * 16384 + 8192 + (k & 3) * 32),
-                                IDESC_N64, k != 0);
-            }
-        }
-        if (lc >= 1) store_o(c_begin + lc - 1, CT_O + (par ^ 1) * 64);
-        if (!chain_wait(&m->bar_s1, par, m, err, ERR_TIMEOUT_MMA)) { ok = false; break; }
-        tc_fence_after();
-        if (!chain_wait(&m->full_u, par, m, err, ERR_TIMEOUT_TMA)) { ok = false; break; }
-        {   // U = Ũ + X, rounded to tf32 in place: A operand of S3 and S2
-            uint32_t x[32];
-            tmem_ld32(tmem + lane_off + CT_U + half * 32, x);
-            tmem_wait_ld();
-#pragma unroll
-            for (int jj = 0; jj < 32; ++jj)
-                x[jj] = to_tf32(__uint_as_float(x[jj]) +
-                                *reinterpret_cast<const float *>(
-                                    sm + CO_UT + rec_ut_offset(half * 32 + jj, row) - REC_UT));
-            tmem_st32(tmem + lane_off + CT_U + half * 32, x);
-            tmem_wait_st();
-        }
-        tc_fence_before();
-        group_sync(1);
-        if (tid == 0) {
-            if (lc + 1 < nl) load_u(lc + 1);
-            tc_fence_after();
-            if (!mbar_wait(&m->full_k, par) || !mbar_wait(&m->full_p[par], sph)) {
-                fail(ERR_TIMEOUT_TMA);
-            } else {
-                // S3: ΔS = U^T K̂, then S2: O^T += U^T (P ⊙ causal)^T
-#pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    mma_tf32_ts(tmem + CT_DS, tmem + CT_U + k * 8,
-                                sw128_kmajor_desc(sbase + CO_KH + (k >> 2) * 16384 + (k & 3) * 32),
-                                IDESC_N128, k != 0);
-                mma_commit(&m->bar_s3);
-#pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    mma_tf32_ts(tmem + tmO, tmem + CT_U + k * 8,
-                                sw128_kmajor_desc(sbase + CO_PM + par * 16384 + (k >> 2) * 8192 + (k & 3) * 32),
-                                IDESC_N64, 1);
-                mma_commit(&m->bar_o);
-            }
-        }
-        if (!chain_wait(&m->bar_s3, par, m, err, ERR_TIMEOUT_MMA)) { ok = false; break; }
-        tc_fence_after();
-        if (tid == 0) {
-            // S3 done: K̂ and (S1' before it) this A1 stage are consumed
-            if (lc + 1 < nl) load_k(lc + 1);
-            if (lc + 2 < nl) load_a1(lc + 2);
-            prefetch_rec(lc + 4);
-        }
-        // exp(G_C) of this chunk came with its P stage
-        if (!chain_wait(&m->full_p[par], sph, m, err, ERR_TIMEOUT_TMA)) { ok = false; break; }
-        {   // S = S Diag(exp(G_C)) + ΔS (fp32 master), tf32 copy back to TMEM
-            const float *gcb = m->gam[par];
-#pragma unroll
-            for (int part = 0; part < 2; ++part) {
-                uint32_t x[32];
-                tmem_ld32(tmem + lane_off + CT_DS + half * 64 + part * 32, x);
-                tmem_wait_ld();
-#pragma unroll
-                for (int jj = 0; jj < 32; ++jj) {
-                    const float gc = CHANNEL ? gcb[half * 64 + part * 32 + jj] : gcb[0];
-                    const float sv = fmaf(gc, S[part * 32 + jj], __uint_as_float(x[jj]));
-                    S[part * 32 + jj] = sv;
-                    x[jj] = to_tf32(sv);
-                }
-                tmem_st32(tmem + lane_off + CT_S + half * 64 + part * 32, x);
-            }
-            tmem_wait_st();
-        }
-        tc_fence_before();
-        group_sync(1);
-    }
-    if (ok) {
-        if (chain_wait(&m->bar_o, (nl - 1) & 1, m, err, ERR_TIMEOUT_MMA)) {
-            tc_fence_after();
-            store_o(c_begin + nl - 1, CT_O + ((nl - 1) & 1) * 64);
-        }
-    }
-    if (s_out != nullptr) {
-#pragma unroll
-        for (int j = 0; j < 64; j += 4)
-            *reinterpret_cast<float4 *>(s_out + sg + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
-    }
-    // never leave a bulk copy in flight into this CTA's shared memory: wait for
-    // the last load of every buffer (a completed phase returns at once)
-    if (tid == 0) {
-        for (int b = 0; b < 6; ++b)
-            if (issued[b] > 0) (void)mbar_wait(bars[b], (issued[b] - 1) & 1);
-    }
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 0) {
-        tc_fence_after();
-        tmem_dealloc(tmem, CHAIN_TMEM_COLS);
-    }
-}
-
-// ------------------------------------- chain kernel, d_v split over 4 CTAs ----
-// Each CTA owns 32 value channels (a column block of S^T) of one (sequence,
-// head); the products keep the 128-row M dimension on d_k or on [W; Q̃]:
-//
-//   M1  D1 = [-W; Q̃] S_b^T     (M = 128: rows 0-63 give X = -W S_b^T, rows 64-127
-//                                give the inter-chunk output Q̃ S_b^T)
-//   M2  ΔS_b^T = K̂^T U_b       (M = 128 = d_k)
-//   M4  D1 += [junk; P ⊙ causal] U_b   (rows 64-127: the intra-chunk output)
-//
-// with U_b = Ũ_b + X (tf32) and S_b^T = S_b^T Diag(exp(G_C)) + ΔS_b^T kept in
-// fp32 registers (thread = d_k row).  N = 32 for every product.  Warp roles:
-// 0-3 own the state block, 4-5 form U, 6-7 store the output, 8 issues the
-// MMAs, 9 loads the records; they hand off through mbarriers only (MMA
-// completion frees record buffers through tcgen05.commit).
-constexpr int kNB = 32;                       // value channels per CTA
-constexpr int kSplitParts = D / kNB;          // CTAs per (sequence, head)
-constexpr int kSplitThreads = 320;
-constexpr uint32_t VO_A1 = 0;                 // [-W; Q̃], two stages of 64 KiB
-constexpr uint32_t VO_KH = 131072;            // K̂^T, 32 KiB
-constexpr uint32_t VO_A4 = 163840;            // per 16 KiB block: rows 0-63 a Ũ stage, rows 64-127 P
-constexpr uint32_t VO_SB = 196608;            // S_b [32 dv][128 dk] tf32 image, 4 blocks of 4 KiB
-constexpr uint32_t VO_UB = 212992;            // U_b^T [32 dv][64 tok] tf32 image, 2 blocks of 4 KiB
-constexpr uint32_t VO_MISC = 221184;
-constexpr uint32_t VSPLIT_SMEM = VO_MISC + 1024;   // 222208
-constexpr uint32_t VT_D1 = 0, VT_DS = 64, VSPLIT_TMEM_COLS = 128;   // D1 buffers at 0 and 32
-constexpr uint32_t IDESC_N32 = make_idesc(2, 128, 32);
-
-struct VMisc {
-    uint64_t full_a1[2], full_u[2], full_k, full_p;   // record parts landed
-    uint64_t empty_a1[2], empty_u[2], empty_kp;       // record buffers free
-    uint64_t bar1, bar2, bar4[2];                     // M1 / M2 / M4 done
-    uint64_t u_ready, s_ready, o_free[2];             // role hand-offs
-    uint32_t tmem_base;
-    int abort_flag;
-};
-static_assert(sizeof(VMisc) <= 1024, "split misc area overflow");
+static_assert(sizeof(ChainMisc) <= 1024, "chain misc area overflow");
 
 // Bounded wait by a whole warp; the lanes agree on the outcome, so the
 // warp-wide TMEM accesses after it stay convergent.
 __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t phase) {
-    return __all_sync(0xffffffffu, mbar_wait(bar, phase));
+    return __all_sync(0xffffffffu, mbar_wait_sleep(bar, phase));
 }
 
-template <bool CHANNEL>
-__global__ void __launch_bounds__(kSplitThreads, 1)
-chain_split_kernel(const uint8_t *__restrict__ recs, const float *h0, float *fin, float *ws_state,
-                   const int32_t *__restrict__ cu, int num_seqs, int total_T, int H, int c_begin,
-                   int c_end, __nv_bfloat16 *__restrict__ o, uint32_t *err) {
+// Named barrier over `nthreads` threads that also ORs a flag across them.
+__device__ __forceinline__ bool named_sync_or(int id, int nthreads, bool flag) {
+    uint32_t any;
+    asm volatile(
+        "{\n\t.reg .pred pc, pr;\n\t"
+        "setp.ne.u32 pc, %1, 0;\n\t"
+        "barrier.red.or.pred pr, %2, %3, pc;\n\t"
+        "selp.u32 %0, 1, 0, pr;\n\t}"
+        : "=r"(any)
+        : "r"((uint32_t)flag), "r"(id), "r"(nthreads)
+        : "memory");
+    return any != 0;
+}
+
+// Largest |value| over a role's warps -> the role-wide scale exponent.  The
+// barrier also agrees on stopping: every warp of the role calls this once
+// per chunk, even after a failed wait, and all of them see `stop` true if
+// any thread passed stop = true or the CTA's abort flag was set before.
+__device__ __forceinline__ int role_scale(float mx, float *slots, int slot, int nwarps, int bar_id,
+                                          bool &stop, volatile int *abort_flag) {
+    const uint32_t wm = __reduce_max_sync(0xffffffffu, __float_as_uint(mx));
+    if ((threadIdx.x & 31) == 0) slots[slot] = __uint_as_float(wm);
+    stop = named_sync_or(bar_id, nwarps * 32, stop || *abort_flag != 0);
+    float bm = 0.f;
+    for (int w = 0; w < nwarps; ++w) bm = fmaxf(bm, slots[w]);
+    return scale_exp(bm);
+}
+
+template <bool CHANNEL, int NB>
+__global__ void __launch_bounds__(Chain<NB>::kThreads, 1)
+chain_kernel(const uint8_t *__restrict__ recs, const float *h0, float *fin, float *ws_state,
+             const int32_t *__restrict__ cu, int num_seqs, int total_T, int H, int c_begin,
+             int c_end, __nv_bfloat16 *__restrict__ o, uint32_t *err) {
+    using K = Chain<NB>;
+    constexpr int kParts = D / NB;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t sbase = smem_u32(smem_raw);
-    const int chain = blockIdx.x / kSplitParts, part = blockIdx.x % kSplitParts;
-    const int chains = gridDim.x / kSplitParts;
+    const int chain = blockIdx.x / kParts, part = blockIdx.x % kParts;
+    const int chains = gridDim.x / kParts;
     const int h = chain % H, n = chain / H;
-    const int dv0 = part * kNB;
+    const int dv0 = part * NB;
     int t0, len;
     sequence_range(cu, n, num_seqs, total_T, t0, len);
     const int nchunks = (len + C - 1) / C;
@@ -891,15 +761,13 @@ chain_split_kernel(const uint8_t *__restrict__ recs, const float *h0, float *fin
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
-    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    // state entry (dv0 + j, t) of this (sequence, head) for state thread t
-    const size_t sbase_g = (((size_t)n * H + h) * D + dv0) * D;
+    // entry (dv0 + j, t) of this (sequence, head)'s state
+    const size_t sg = (((size_t)n * H + h) * D + dv0) * D;
 
     if (nl == 0) {   // empty sequence: the state block passes through
         if (s_out != nullptr && tid < D) {
-#pragma unroll 4
-            for (int j = 0; j < kNB; ++j)
-                s_out[sbase_g + (size_t)j * D + tid] = s_in != nullptr ? s_in[sbase_g + (size_t)j * D + tid] : 0.f;
+            for (int j = 0; j < NB; ++j)
+                s_out[sg + (size_t)j * D + tid] = s_in != nullptr ? s_in[sg + (size_t)j * D + tid] : 0.f;
         }
         return;
     }
@@ -908,28 +776,28 @@ chain_split_kernel(const uint8_t *__restrict__ recs, const float *h0, float *fin
         return;
     }
     uint8_t *sm = smem_raw;
-    VMisc *m = reinterpret_cast<VMisc *>(sm + VO_MISC);
+    ChainMisc *m = reinterpret_cast<ChainMisc *>(sm + K::MISC);
     if (tid == 0) {
         for (int s = 0; s < 2; ++s) {
             mbar_init(&m->full_a1[s], 1);
             mbar_init(&m->full_u[s], 1);
+            mbar_init(&m->full_kp[s], 1);
             mbar_init(&m->empty_a1[s], 1);
-            mbar_init(&m->empty_u[s], 64);
+            mbar_init(&m->empty_u[s], 64 * K::kSets);
+            mbar_init(&m->empty_kp[s], 1);
             mbar_init(&m->bar4[s], 1);
-            mbar_init(&m->o_free[s], 64);
+            mbar_init(&m->o_free[s], 64 * K::kSets);
+            mbar_init(&m->osc_full[s], 64 * K::kSets);
         }
-        mbar_init(&m->full_k, 1);
-        mbar_init(&m->full_p, 1);
-        mbar_init(&m->empty_kp, 1);
         mbar_init(&m->bar1, 1);
         mbar_init(&m->bar2, 1);
-        mbar_init(&m->u_ready, 64);
-        mbar_init(&m->s_ready, 128);
+        mbar_init(&m->s_ready, 32 * K::kSW);
+        mbar_init(&m->u_ready, 64 * K::kSets);
         m->abort_flag = 0;
         fence_barrier_init();
     }
     if (warp == 0) {
-        tmem_alloc(&m->tmem_base, VSPLIT_TMEM_COLS);
+        tmem_alloc(&m->tmem_base, K::TCOLS);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -945,184 +813,268 @@ chain_split_kernel(const uint8_t *__restrict__ recs, const float *h0, float *fin
         return recs + ((size_t)lc * chains + chain) * REC_BYTES;
     };
 
-    if (warp < 4) {
-        // ====================================== state block S_b^T, row t ====
-        const int t = tid;
-        float S[kNB];
+    if (warp < K::kSW) {
+        // ================================== state block S_b^T, thread = d_k row ====
+        const int sub = warp & 3, cg = warp >> 2;
+        const int t = sub * 32 + lane;
+        const int c0 = cg * K::kCS;
+        const uint32_t lane_off = static_cast<uint32_t>(sub * 32) << 16;
+        float S[K::kCS];
 #pragma unroll
-        for (int j = 0; j < kNB; ++j)
-            S[j] = s_in != nullptr ? s_in[sbase_g + (size_t)j * D + t] : 0.f;
-        const uint32_t sb = sbase + VO_SB + (t >> 5) * 4096 + (t & 3) * 4;
-        const uint32_t sch = (t & 31) >> 2;
+        for (int j = 0; j < K::kCS; ++j)
+            S[j] = s_in != nullptr ? s_in[sg + (size_t)(c0 + j) * D + t] : 0.f;
+        // fp16 image of the state block for chunk lc, with its scale exponent
+        const uint32_t scol = sbase + K::SB + (t >> 6) * (NB * 128) + (t & 7) * 2;
+        const uint32_t schk = (t & 63) >> 3;
+        bool stop = false;
+        auto publish = [&](int lc) {
+            float mx = 0.f;
 #pragma unroll
-        for (int j = 0; j < kNB; ++j) st_shared_b32(sb + sw128_offset(j, sch), to_tf32(S[j]));
-        fence_proxy_async();
-        mbar_arrive(&m->s_ready);
-        for (int lc = 0; lc < nl; ++lc) {
-            if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
-            const uint8_t *r = rec_of(lc);
-            const float gc = *reinterpret_cast<const float *>(r + REC_GC + (CHANNEL ? t * 4 : 0));
-            if (!warp_wait(&m->bar2, lc & 1)) { fail(ERR_TIMEOUT_MMA); break; }
-            tc_fence_after();
-            uint32_t x[32];
-            tmem_ld32(tmem + lane_off + VT_DS, x);
-            tmem_wait_ld();
+            for (int j = 0; j < K::kCS; ++j) mx = fmaxf(mx, fabsf(S[j]));
+            const int sS = role_scale(mx, m->red_s[lc & 1], warp, K::kSW, 1, stop, abort_flag);
+            const float f = exp2i(sS);
 #pragma unroll
-            for (int j = 0; j < kNB; ++j) {
-                S[j] = fmaf(gc, S[j], __uint_as_float(x[j]));
-                st_shared_b32(sb + sw128_offset(j, sch), to_tf32(S[j]));
-            }
+            for (int j = 0; j < K::kCS; ++j) st_shared_b16(scol + sw128_offset(c0 + j, schk), f2h_bits(S[j] * f));
+            if (tid == 0) m->es[lc & 3] = sS;
             fence_proxy_async();
-            tc_fence_before();
             mbar_arrive(&m->s_ready);
+        };
+        publish(0);
+        for (int lc = 0; lc < nl && !stop; ++lc) {
+            const float gc =
+                *reinterpret_cast<const float *>(rec_of(lc) + REC_GC + (CHANNEL ? t * 4 : 0));
+            // u_ready publishes the ΔS exponents; M2 done gives ΔS.  A failed wait
+            // still takes part in the role's barrier below.
+            if (!warp_wait(&m->u_ready, lc & 1)) { fail(ERR_TIMEOUT_HANDOFF); stop = true; }
+            if (!stop && !warp_wait(&m->bar2, lc & 1)) { fail(ERR_TIMEOUT_MMA); stop = true; }
+            if (!stop) {
+                tc_fence_after();
+                const float f1 = exp2i(-m->dsx[lc & 1][0]), f2 = exp2i(-m->dsx[lc & 1][1]);
+#pragma unroll
+                for (int p = 0; p < K::kCS / 16; ++p) {
+                    uint32_t x[16];
+                    tmem_ld16(tmem + lane_off + K::TD2 + c0 + p * 16, x);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int jj = 0; jj < 16; ++jj)
+                        S[p * 16 + jj] = fmaf(gc, S[p * 16 + jj], __uint_as_float(x[jj]) * f1 * f2);
+                }
+                tc_fence_before();
+            }
+            if (lc + 1 < nl) publish(lc + 1);
         }
         if (s_out != nullptr) {
 #pragma unroll
-            for (int j = 0; j < kNB; ++j) s_out[sbase_g + (size_t)j * D + t] = S[j];
+            for (int j = 0; j < K::kCS; ++j) s_out[sg + (size_t)(c0 + j) * D + t] = S[j];
         }
-    } else if (warp < 6) {
-        // ======================================== U_b = Ũ_b + X, token i ====
-        const int i = tid - 128;
-        const uint32_t ub = sbase + VO_UB + (i >> 5) * 4096 + (i & 3) * 4;
-        const uint32_t uch = (i & 31) >> 2;
-        for (int lc = 0; lc < nl; ++lc) {
-            if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
-            const uint32_t s = lc & 1;
-            if (!warp_wait(&m->full_u[s], (lc >> 1) & 1)) { fail(ERR_TIMEOUT_TMA); break; }
-            if (!warp_wait(&m->bar1, lc & 1)) { fail(ERR_TIMEOUT_MMA); break; }
-            tc_fence_after();
-            uint32_t x[32];
-            tmem_ld32(tmem + lane_off + VT_D1 + s * 32, x);
-            // Ũ row i of this block, 16-byte chunks swizzled by i % 8
-            const uint32_t urow = sbase + VO_A4 + s * 16384 + i * 128;
-            float u[kNB];
+    } else if (warp < K::kIssuer) {
+        const int set = (warp - K::kSW) >> 2, r = (warp - K::kSW) & 3;
+        const int c0 = set * K::kCU;
+        const uint32_t lane_off = static_cast<uint32_t>(r * 32) << 16;
+        if (r < 2) {
+            // ===================================== U_b = Ũ_b + X, thread = token i ====
+            const int i = r * 32 + lane;
+            const uint32_t ucol = sbase + K::UB + (i & 7) * 2;
+            const uint32_t uchk = i >> 3;
+            bool stop = false;
+            for (int lc = 0; lc < nl && !stop; ++lc) {
+                const uint32_t s = lc & 1;
+                const uint32_t b = K::kDB ? (lc & 1) : 0;
+                // a failed wait still takes part in the role's barrier below
+                if (!warp_wait(&m->full_u[s], (lc >> 1) & 1)) { fail(ERR_TIMEOUT_TMA); stop = true; }
+                if (!stop && !warp_wait(&m->s_ready, lc & 1)) { fail(ERR_TIMEOUT_HANDOFF); stop = true; }
+                if (!stop && !warp_wait(&m->bar1, lc & 1)) { fail(ERR_TIMEOUT_MMA); stop = true; }
+                if (!stop) tc_fence_after();
+                const int sW = m->ex[s][0], sQ = m->ex[s][1], sK = m->ex[s][2], sP = m->ex[s][3];
+                const int sS = m->es[lc & 3];
+                const float fa = exp2i(-sW), fb = exp2i(-sS);
+                // U = Ũ + X in fp32, written back over this thread's Ũ row (the stage
+                // is read only here) until the block's scale is known
+                float mx = 0.f;
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                const uint4 v = ld_shared_v4(urow + ((q ^ (i & 7)) << 4));
-                u[4 * q] = __uint_as_float(v.x); u[4 * q + 1] = __uint_as_float(v.y);
-                u[4 * q + 2] = __uint_as_float(v.z); u[4 * q + 3] = __uint_as_float(v.w);
-            }
-            tmem_wait_ld();
+                for (int p = 0; p < K::kCU / 32 && !stop; ++p) {
+                    uint32_t x[32];
+                    tmem_ld32(tmem + lane_off + K::TD1 + b * NB + c0 + p * 32, x);
+                    const uint32_t urow =
+                        sbase + K::UT + s * (256 * NB) + ((c0 + p * 32) >> 5) * 8192 + i * 128;
+                    tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < kNB; ++j)
-                st_shared_b32(ub + sw128_offset(j, uch), to_tf32(u[j] + __uint_as_float(x[j])));
-            fence_proxy_async();
-            tc_fence_before();
-            mbar_arrive(&m->u_ready);
-            mbar_arrive(&m->empty_u[s]);   // the Ũ stage is read
-        }
-    } else if (warp < 8) {
-        // ================================ output rows (token i), 32 channels ====
-        const int i = tid - 192;
-        for (int lc = 0; lc < nl; ++lc) {
-            if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
-            const uint32_t s = lc & 1;
-            if (!warp_wait(&m->bar4[s], (lc >> 1) & 1)) { fail(ERR_TIMEOUT_MMA); break; }
-            tc_fence_after();
-            uint32_t x[32];
-            tmem_ld32(tmem + lane_off + VT_D1 + s * 32, x);
-            tmem_wait_ld();
-            tc_fence_before();
-            mbar_arrive(&m->o_free[s]);
-            const int cc = c_begin + lc;
-            if (i < min(C, len - cc * C)) {
-                uint4 *dst = reinterpret_cast<uint4 *>(o + ((size_t)(t0 + cc * C + i) * H + h) * D + dv0);
+                    for (int q = 0; q < 8; ++q) {
+                        const uint32_t a = urow + ((q ^ (i & 7)) << 4);
+                        const uint4 v = ld_shared_v4(a);
+                        float w[4] = {__uint_as_float(v.x), __uint_as_float(v.y),
+                                      __uint_as_float(v.z), __uint_as_float(v.w)};
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    uint32_t w[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(x[8 * q + 2 * e]),
-                                                                        __uint_as_float(x[8 * q + 2 * e + 1]));
-                        w[e] = *reinterpret_cast<const uint32_t *>(&b2);
+                        for (int e = 0; e < 4; ++e) {
+                            w[e] += __uint_as_float(x[q * 4 + e]) * fa * fb;
+                            mx = fmaxf(mx, fabsf(w[e]));
+                        }
+                        st_shared_v4(a, __float_as_uint(w[0]), __float_as_uint(w[1]),
+                                     __float_as_uint(w[2]), __float_as_uint(w[3]));
                     }
-                    dst[q] = make_uint4(w[0], w[1], w[2], w[3]);
                 }
+                const int sU = role_scale(mx, m->red_u[lc & 1], set * 2 + r, 2 * K::kSets, 2, stop,
+                                          abort_flag);
+                if (stop) break;
+                const float fu = exp2i(sU);
+#pragma unroll
+                for (int p = 0; p < K::kCU / 32; ++p) {
+                    const uint32_t urow =
+                        sbase + K::UT + s * (256 * NB) + ((c0 + p * 32) >> 5) * 8192 + i * 128;
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        const uint4 v = ld_shared_v4(urow + ((q ^ (i & 7)) << 4));
+                        const float w[4] = {__uint_as_float(v.x), __uint_as_float(v.y),
+                                            __uint_as_float(v.z), __uint_as_float(v.w)};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            st_shared_b16(ucol + sw128_offset(c0 + p * 32 + q * 4 + e, uchk),
+                                          f2h_bits(w[e] * fu));
+                    }
+                }
+                if (i == 0 && set == 0) {
+                    m->dsx[lc & 1][0] = sK;
+                    m->dsx[lc & 1][1] = sU;
+                    m->osx[lc & 1][0] = sQ;
+                    m->osx[lc & 1][1] = sS;
+                    m->osx[lc & 1][2] = sP;
+                    m->osx[lc & 1][3] = sU;
+                }
+                fence_proxy_async();
+                tc_fence_before();
+                mbar_arrive(&m->u_ready);
+                mbar_arrive(&m->empty_u[s]);   // this Ũ stage (and its exponents) is read
+                mbar_arrive(&m->osc_full[lc & 1]);
+            }
+        } else {
+            // ====================== output rows (token i = TMEM lane - 64), NB/kSets channels ====
+            const int i = (r - 2) * 32 + lane;
+            for (int lc = 0; lc < nl; ++lc) {
+                if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
+                const uint32_t b = K::kDB ? (lc & 1) : 0;
+                const uint32_t bph = K::kDB ? ((lc >> 1) & 1) : (lc & 1);
+                if (!warp_wait(&m->osc_full[lc & 1], (lc >> 1) & 1)) { fail(ERR_TIMEOUT_HANDOFF); break; }
+                if (!warp_wait(&m->bar4[b], bph)) { fail(ERR_TIMEOUT_MMA); break; }
+                tc_fence_after();
+                const int *sx = m->osx[lc & 1];
+                const float fq1 = exp2i(-sx[0]), fq2 = exp2i(-sx[1]);
+                const float fp1 = exp2i(-sx[2]), fp2 = exp2i(-sx[3]);
+                const int cc = c_begin + lc;
+                const bool live = i < min(C, len - cc * C);
+                uint4 *dst = reinterpret_cast<uint4 *>(o + ((size_t)(t0 + cc * C + i) * H + h) * D + dv0 + c0);
+#pragma unroll
+                for (int p = 0; p < K::kCU / 32; ++p) {
+                    uint32_t x1[32], x4[32];
+                    tmem_ld32(tmem + lane_off + K::TD1 + b * NB + c0 + p * 32, x1);
+                    tmem_ld32(tmem + lane_off + K::TD4 + b * NB + c0 + p * 32, x4);
+                    tmem_wait_ld();
+                    if (live) {
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            uint32_t w[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int j = q * 8 + 2 * e;
+                                const float a = __uint_as_float(x1[j]) * fq1 * fq2 + __uint_as_float(x4[j]) * fp1 * fp2;
+                                const float c2 = __uint_as_float(x1[j + 1]) * fq1 * fq2 + __uint_as_float(x4[j + 1]) * fp1 * fp2;
+                                const __nv_bfloat162 b2 = __floats2bfloat162_rn(a, c2);
+                                w[e] = *reinterpret_cast<const uint32_t *>(&b2);
+                            }
+                            dst[p * 4 + q] = make_uint4(w[0], w[1], w[2], w[3]);
+                        }
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive(&m->o_free[b]);
             }
         }
-    } else if (warp == 8) {
+    } else if (warp == K::kIssuer) {
         // ======================================================= MMA issuer ====
         if (lane == 0) {
-            const uint64_t d_sb = sw128_kmajor_desc(sbase + VO_SB);
-            const uint64_t d_ub = sw128_kmajor_desc(sbase + VO_UB);
-            const uint64_t d_kh = sw128_kmajor_desc(sbase + VO_KH);
-            const uint64_t d_a4 = sw128_kmajor_desc(sbase + VO_A4);
+            const uint64_t d_sb = sw128_kmajor_desc(sbase + K::SB);
+            const uint64_t d_ub = sw128_kmajor_desc(sbase + K::UB);
             for (int lc = 0; lc < nl; ++lc) {
                 if (*abort_flag) break;
                 const uint32_t s = lc & 1, sph = (lc >> 1) & 1;
+                const uint32_t b = K::kDB ? (lc & 1) : 0;                 // K̂/P stage = O buffer
+                const uint32_t bph = K::kDB ? ((lc >> 1) & 1) : (lc & 1);
                 // the buffers are normally ready long before the state block
                 if (!mbar_wait_sleep(&m->full_a1[s], sph)) { fail(ERR_TIMEOUT_TMA); break; }
-                if (lc >= 2 && !mbar_wait_sleep(&m->o_free[s], ((lc - 2) >> 1) & 1)) { fail(ERR_TIMEOUT_HANDOFF); break; }
-                if (!mbar_wait_sleep(&m->s_ready, lc & 1)) { fail(ERR_TIMEOUT_HANDOFF); break; }
-                tc_fence_after();
-                const uint64_t d_a1 = sw128_kmajor_desc(sbase + VO_A1 + s * 65536);
-                const uint32_t d1 = tmem + VT_D1 + s * 32;
-                // descriptors advance by (bytes >> 4) in their start-address field
-#pragma unroll
-                for (int k = 0; k < 16; ++k)
-                    mma_tf32_ss(d1, d_a1 + (((k >> 2) * 16384 + (k & 3) * 32) >> 4),
-                                d_sb + (((k >> 2) * 4096 + (k & 3) * 32) >> 4), IDESC_N32, k != 0);
-                mma_commit(&m->bar1);
-                mma_commit(&m->empty_a1[s]);
-                if (!mbar_wait_sleep(&m->full_k, lc & 1) || !mbar_wait_sleep(&m->full_p, lc & 1)) {
-                    fail(ERR_TIMEOUT_TMA);
+                const int prev = K::kDB ? lc - 2 : lc - 1;                // last user of O buffer b
+                if (prev >= 0 && !mbar_wait_sleep(&m->o_free[b], K::kDB ? ((prev >> 1) & 1) : (prev & 1))) {
+                    fail(ERR_TIMEOUT_HANDOFF);
                     break;
                 }
+                if (!mbar_wait_sleep(&m->s_ready, lc & 1)) { fail(ERR_TIMEOUT_HANDOFF); break; }
+                tc_fence_after();
+                const uint64_t d_a1 = sw128_kmajor_desc(sbase + K::A1 + s * 32768);
+                // descriptors advance by (bytes >> 4) in their start-address field
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    mma_f16_ss(tmem + K::TD1 + b * NB, d_a1 + (((k >> 2) * 16384 + (k & 3) * 32) >> 4),
+                               d_sb + (((k >> 2) * (NB * 128) + (k & 3) * 32) >> 4), K::IDESC, k != 0);
+                mma_commit(&m->bar1);
+                mma_commit(&m->empty_a1[s]);
+                if (!mbar_wait_sleep(&m->full_kp[b], bph)) { fail(ERR_TIMEOUT_TMA); break; }
                 if (!mbar_wait_sleep(&m->u_ready, lc & 1)) { fail(ERR_TIMEOUT_HANDOFF); break; }
                 tc_fence_after();
+                const uint64_t d_kh = sw128_kmajor_desc(sbase + K::KH + b * 16384);
+                const uint64_t d_a4 = sw128_kmajor_desc(sbase + K::A4 + b * 16384);
 #pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    mma_tf32_ss(tmem + VT_DS, d_kh + (((k >> 2) * 16384 + (k & 3) * 32) >> 4),
-                                d_ub + (((k >> 2) * 4096 + (k & 3) * 32) >> 4), IDESC_N32, k != 0);
+                for (int k = 0; k < 4; ++k)
+                    mma_f16_ss(tmem + K::TD2, d_kh + ((k * 32) >> 4), d_ub + ((k * 32) >> 4), K::IDESC, k != 0);
                 mma_commit(&m->bar2);
 #pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    mma_tf32_ss(d1, d_a4 + (((k >> 2) * 16384 + (k & 3) * 32) >> 4),
-                                d_ub + (((k >> 2) * 4096 + (k & 3) * 32) >> 4), IDESC_N32, 1);
-                mma_commit(&m->bar4[s]);
-                mma_commit(&m->empty_kp);
+                for (int k = 0; k < 4; ++k)
+                    mma_f16_ss(tmem + K::TD4 + b * NB, d_a4 + ((k * 32) >> 4), d_ub + ((k * 32) >> 4), K::IDESC,
+                               k != 0);
+                mma_commit(&m->bar4[b]);
+                mma_commit(&m->empty_kp[b]);
             }
         }
     } else if (lane == 0) {
         // ==================================================== record loader ====
         uint32_t issued[6] = {0, 0, 0, 0, 0, 0};
         uint64_t *bars[6] = {&m->full_a1[0], &m->full_a1[1], &m->full_u[0], &m->full_u[1],
-                             &m->full_k, &m->full_p};
+                             &m->full_kp[0], &m->full_kp[1]};
         auto load_a1 = [&](int lc) {
             const int s = lc & 1;
-            mbar_arrive_expect_tx(&m->full_a1[s], 65536);
-            bulk_load(sm + VO_A1 + s * 65536, rec_of(lc) + REC_A1, 65536, &m->full_a1[s]);
+            mbar_arrive_expect_tx(&m->full_a1[s], 32768);
+            bulk_load(sm + K::A1 + s * 32768, rec_of(lc) + REC_A1, 32768, &m->full_a1[s]);
             ++issued[s];
         };
-        auto load_u = [&](int lc) {   // this CTA's 32-channel block of Ũ
+        auto load_u = [&](int lc) {   // this CTA's channel blocks of Ũ, and the exponents
             const int s = lc & 1;
-            mbar_arrive_expect_tx(&m->full_u[s], 8192);
-            bulk_load(sm + VO_A4 + s * 16384, rec_of(lc) + REC_UT + part * 8192, 8192, &m->full_u[s]);
+            const uint8_t *r = rec_of(lc);
+            mbar_arrive_expect_tx(&m->full_u[s], 256 * NB + 16);
+            bulk_load(sm + K::UT + s * (256 * NB), r + REC_UT + part * (NB / 32) * 8192, 256 * NB,
+                      &m->full_u[s]);
+            bulk_load(m->ex[s], r + REC_EX, 16, &m->full_u[s]);
             ++issued[2 + s];
         };
         auto load_kp = [&](int lc) {
+            const int b = K::kDB ? (lc & 1) : 0;
             const uint8_t *r = rec_of(lc);
-            mbar_arrive_expect_tx(&m->full_k, 32768);
-            bulk_load(sm + VO_KH, r + REC_KH, 32768, &m->full_k);
-            mbar_arrive_expect_tx(&m->full_p, 16384);
-            bulk_load(sm + VO_A4 + 8192, r + REC_PM, 8192, &m->full_p);
-            bulk_load(sm + VO_A4 + 16384 + 8192, r + REC_PM + 8192, 8192, &m->full_p);
-            ++issued[4];
-            ++issued[5];
+            mbar_arrive_expect_tx(&m->full_kp[b], 16384 + 8192);
+            bulk_load(sm + K::KH + b * 16384, r + REC_KH, 16384, &m->full_kp[b]);
+            bulk_load(sm + K::A4 + b * 16384 + 8192, r + REC_PM, 8192, &m->full_kp[b]);
+            ++issued[4 + b];
         };
         auto prefetch_rec = [&](int lc) {
             if (lc < nl) {
                 const uint8_t *r = rec_of(lc);
 #pragma unroll
-                for (int q = 0; q < 4; ++q) bulk_prefetch_l2(r + q * 36992, 36992);
+                for (int q = 0; q < 5; ++q) bulk_prefetch_l2(r + q * 18128, 18128);
             }
         };
+        constexpr int kKPAhead = K::kDB ? 2 : 1;   // K̂/P stages in flight
         load_a1(0);
         load_kp(0);
         load_u(0);
         if (nl > 1) {
             load_a1(1);
             load_u(1);
+            if (K::kDB) load_kp(1);
         }
         prefetch_rec(1);
         prefetch_rec(2);
@@ -1131,24 +1083,411 @@ chain_split_kernel(const uint8_t *__restrict__ recs, const float *h0, float *fin
         for (int lc = 0; lc < nl; ++lc) {
             if (*abort_flag) break;
             const uint32_t s = lc & 1, sph = (lc >> 1) & 1;
+            const uint32_t b = K::kDB ? (lc & 1) : 0;
+            const uint32_t bph = K::kDB ? ((lc >> 1) & 1) : (lc & 1);
             if (!mbar_wait_sleep(&m->empty_a1[s], sph)) { fail(ERR_TIMEOUT_MMA); break; }
             if (lc + 2 < nl) load_a1(lc + 2);
             if (!mbar_wait_sleep(&m->empty_u[s], sph)) { fail(ERR_TIMEOUT_HANDOFF); break; }
             if (lc + 2 < nl) load_u(lc + 2);
-            if (!mbar_wait_sleep(&m->empty_kp, lc & 1)) { fail(ERR_TIMEOUT_MMA); break; }
-            if (lc + 1 < nl) load_kp(lc + 1);
+            if (!mbar_wait_sleep(&m->empty_kp[b], bph)) { fail(ERR_TIMEOUT_MMA); break; }
+            if (lc + kKPAhead < nl) load_kp(lc + kKPAhead);
             prefetch_rec(lc + 3);
         }
         // never leave a bulk copy in flight into this CTA's shared memory
-        for (int b = 0; b < 6; ++b)
-            if (issued[b] > 0) (void)mbar_wait_sleep(bars[b], (issued[b] - 1) & 1);
+        for (int q = 0; q < 6; ++q)
+            if (issued[q] > 0) (void)mbar_wait_sleep(bars[q], (issued[q] - 1) & 1);
     }
 
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
-        tmem_dealloc(tmem, VSPLIT_TMEM_COLS);
+        tmem_dealloc(tmem, K::TCOLS);
+    }
+}
+
+// ------------------------------------------- chain kernel, transposed form ----
+// One CTA per (sequence, head).  The products are written transposed so that
+// the value channel n is the TMEM lane and the state-side operand is the A
+// operand, read from TMEM as packed fp16:
+//
+//   M1  D1^T = S_h [-W; Q̃]^T      (A = S fp16 in TMEM, B = the record's [-W; Q̃])
+//                                  columns 0-63: X^T, 64-127: inter-chunk output
+//   M2  ΔS   = U^T_h K̂            (A = U^T fp16 in TMEM, B = the record's K̂^T)
+//   M4  O4^T = U^T_h (P ⊙ causal)^T   (B = the record's P)
+//
+// Each row of an fp16 A operand (one value channel) carries its own
+// power-of-two scale, so the threads that share a row only exchange one
+// value; there are no shared-memory operand writes.  4 kRQ row warps (warp
+// w: lanes of sub-partition w % 4, part w / 4 of each row) run U, the state
+// update and the output, meeting at one barrier per step that also carries
+// the decision to stop; the next warp issues the MMAs, the last one loads the
+// records.  The output tile goes through shared memory so that it leaves in
+// 16-byte row segments.
+// TMEM loads / stores of N consecutive columns (N = 8, 16 or 32), as many
+// calls as needed for larger N.
+template <int N>
+__device__ __forceinline__ void tmem_ldn(uint32_t taddr, uint32_t (&r)[N]) {
+    if constexpr (N == 16) {
+        tmem_ld16(taddr, r);
+    } else {
+        static_assert(N % 32 == 0, "column count");
+#pragma unroll
+        for (int p = 0; p < N / 32; ++p) tmem_ld32(taddr + p * 32, *reinterpret_cast<uint32_t (*)[32]>(r + p * 32));
+    }
+}
+template <int N>
+__device__ __forceinline__ void tmem_stn(uint32_t taddr, const uint32_t (&r)[N]) {
+    if constexpr (N == 8) {
+        tmem_st8(taddr, r);
+    } else if constexpr (N == 16) {
+        tmem_st16(taddr, r);
+    } else {
+        static_assert(N % 32 == 0, "column count");
+#pragma unroll
+        for (int p = 0; p < N / 32; ++p)
+            tmem_st32(taddr + p * 32, *reinterpret_cast<const uint32_t (*)[32]>(r + p * 32));
+    }
+}
+
+constexpr int kRQ = 2;                     // threads per row (value channel)
+constexpr int kRowWarps = 4 * kRQ;
+constexpr int kRowThreads = 32 * kRowWarps;
+constexpr int kSC = D / kRQ;               // state columns per thread
+constexpr int kTK = C / kRQ;               // tokens per thread (U and output)
+constexpr int kTThreads = kRowThreads + 64;
+constexpr uint32_t TO_A1 = 0;          // [-W; Q̃] fp16 images, 2 stages of 32 KiB
+constexpr uint32_t TO_KH = 65536;      // K̂^T fp16, 2 stages of 16 KiB
+constexpr uint32_t TO_PM = 98304;      // P fp16, 2 stages of 8 KiB
+constexpr uint32_t TO_UT = 114688;     // Ũ fp32, 2 stages of 32 KiB
+constexpr uint32_t TO_OS = 180224;     // output tile [64 tok][128 ch] bf16, 2 buffers of 16 KiB
+constexpr uint32_t TO_MISC = 212992;
+constexpr uint32_t TSMEM = TO_MISC + 12288;
+constexpr uint32_t TT_D1 = 0, TT_DS = 128, TT_O4 = 256, TT_SA = 320, TT_UA = 384, TT_COLS = 512;
+constexpr uint32_t IDESC_H128 = make_idesc(0, 128, 128), IDESC_H64 = make_idesc(0, 128, 64);
+
+struct TMisc {
+    uint64_t full_a1[2], full_u[2], full_kp[2];
+    uint64_t empty_a1[2], empty_u[2], empty_kp[2];
+    uint64_t bar1, bar2, bar4;
+    uint64_t u_ready, s_ready;
+    uint32_t tmem_base;
+    int abort_flag;
+    alignas(16) int ex[2][4];      // record exponents {s_W, s_Q, s_K, s_P}, with the Ũ stage
+    alignas(16) float gam[2][D];   // exp(G_C), with the Ũ stage
+    float xu[2][kRQ * D], xs[2][kRQ * D];   // part-row maxima exchanged between a row's threads
+};
+static_assert(sizeof(TMisc) <= 12288 && TSMEM <= 232448, "chain smem overflow");
+
+template <bool CHANNEL>
+__global__ void __launch_bounds__(kTThreads, 1)
+chain_t_kernel(const uint8_t *__restrict__ recs, const float *h0, float *fin, float *ws_state,
+               const int32_t *__restrict__ cu, int num_seqs, int total_T, int H, int c_begin,
+               int c_end, __nv_bfloat16 *__restrict__ o, uint32_t *err) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const uint32_t sbase = smem_u32(smem_raw);
+    const int chain = blockIdx.x, chains = gridDim.x;
+    const int h = chain % H, n = chain / H;
+    int t0, len;
+    sequence_range(cu, n, num_seqs, total_T, t0, len);
+    const int nchunks = (len + C - 1) / C;
+    if (c_begin > 0 && c_begin >= nchunks) return;   // finished in an earlier window
+    const int c_stop = min(c_end, nchunks);
+    const int nl = max(c_stop - c_begin, 0);
+    const float *s_in = c_begin == 0 ? h0 : ws_state;
+    float *s_out = c_stop == nchunks ? fin : ws_state;
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
+    const int sub = warp & 3, qp = (warp >> 2) % kRQ;   // TMEM sub-partition, row quarter
+    const int row = sub * 32 + lane;                     // value channel = TMEM lane
+    const uint32_t lane_off = static_cast<uint32_t>(sub * 32) << 16;
+    const size_t sg = (((size_t)n * H + h) * D + row) * D + qp * kSC;
+
+    if (nl == 0) {   // empty sequence: the state passes through
+        if (s_out != nullptr && warp < kRowWarps) {
+#pragma unroll
+            for (int j = 0; j < kSC; j += 4) {
+                float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (s_in != nullptr) x = *reinterpret_cast<const float4 *>(s_in + sg + j);
+                *reinterpret_cast<float4 *>(s_out + sg + j) = x;
+            }
+        }
+        return;
+    }
+    if ((sbase & 1023u) != 0) {
+        if (tid == 0) atomicOr(err, ERR_SMEM_ALIGN);
+        return;
+    }
+    uint8_t *sm = smem_raw;
+    TMisc *m = reinterpret_cast<TMisc *>(sm + TO_MISC);
+    if (tid == 0) {
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&m->full_a1[s], 1);
+            mbar_init(&m->full_u[s], 1);
+            mbar_init(&m->full_kp[s], 1);
+            mbar_init(&m->empty_a1[s], 1);
+            mbar_init(&m->empty_u[s], kRowThreads);
+            mbar_init(&m->empty_kp[s], 1);
+        }
+        mbar_init(&m->bar1, 1);
+        mbar_init(&m->bar2, 1);
+        mbar_init(&m->bar4, 1);
+        mbar_init(&m->u_ready, kRowThreads);
+        mbar_init(&m->s_ready, kRowThreads);
+        m->abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(&m->tmem_base, TT_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = m->tmem_base;
+    volatile int *abort_flag = &m->abort_flag;
+    auto fail = [&](uint32_t code) {
+        *abort_flag = 1;
+        atomicOr(err, code);
+    };
+    auto rec_of = [&](int lc) {
+        return recs + ((size_t)lc * chains + chain) * REC_BYTES;
+    };
+
+    if (warp < kRowWarps) {
+        // ============================= row warps: channel `row`, quarter `qp` ====
+        bool stop = false;
+        // Barrier over the row warps; every row warp passes the same sequence of
+        // them, and `stop` leaves it the same in all threads.
+        auto rows_sync = [&]() { stop = named_sync_or(1, kRowThreads, stop || *abort_flag != 0); };
+        // the row's largest |value| over its kRQ parts
+        auto row_max = [&](float mx, float *slots) {
+            slots[qp * D + row] = mx;
+            rows_sync();
+#pragma unroll
+            for (int k = 0; k < kRQ; ++k) mx = fmaxf(mx, slots[k * D + row]);
+            return mx;
+        };
+        float S[kSC];
+#pragma unroll
+        for (int j = 0; j < kSC; j += 4) {
+            float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (s_in != nullptr) x = *reinterpret_cast<const float4 *>(s_in + sg + j);
+            S[j] = x.x; S[j + 1] = x.y; S[j + 2] = x.z; S[j + 3] = x.w;
+        }
+        // fp16 copy of the state row (A of M1) with the row's own scale
+        auto publish = [&](int lc) {
+            float mx = 0.f;
+#pragma unroll
+            for (int j = 0; j < kSC; ++j) mx = fmaxf(mx, fabsf(S[j]));
+            const int sS = scale_exp(row_max(mx, m->xs[lc & 1]));
+            const float f = exp2i(sS);
+            uint32_t w[kSC / 2];
+#pragma unroll
+            for (int j = 0; j < kSC / 2; ++j) w[j] = f2h2_bits(S[2 * j] * f, S[2 * j + 1] * f);
+            tmem_stn<kSC / 2>(tmem + lane_off + TT_SA + qp * (kSC / 2), w);
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&m->s_ready);
+            return sS;
+        };
+        int sS = publish(0);
+        for (int lc = 0; lc < nl && !stop; ++lc) {
+            const uint32_t s = lc & 1, sph = (lc >> 1) & 1;
+            // (a) D1^T: X^T and the inter-chunk output of this thread's tokens
+            if (!warp_wait(&m->bar1, lc & 1)) { fail(ERR_TIMEOUT_MMA); stop = true; }
+            if (!stop && !warp_wait(&m->full_u[s], sph)) { fail(ERR_TIMEOUT_TMA); stop = true; }
+            uint32_t x[kTK], oi[kTK];
+            int sW = 0, sQ = 0, sK = 0, sP = 0;
+            float mx = 0.f;
+            if (!stop) {
+                tc_fence_after();
+                tmem_ldn<kTK>(tmem + lane_off + TT_D1 + qp * kTK, x);
+                tmem_ldn<kTK>(tmem + lane_off + TT_D1 + 64 + qp * kTK, oi);
+                sW = m->ex[s][0]; sQ = m->ex[s][1]; sK = m->ex[s][2]; sP = m->ex[s][3];
+                const float fa = exp2i(-sW), fb = exp2i(-sS);
+                const uint8_t *ut = sm + TO_UT + s * 32768 - REC_UT;
+                tmem_wait_ld();
+#pragma unroll
+                for (int jj = 0; jj < kTK; ++jj) {
+                    const float u = *reinterpret_cast<const float *>(ut + rec_ut_offset(qp * kTK + jj, row)) +
+                                    __uint_as_float(x[jj]) * fa * fb;
+                    x[jj] = __float_as_uint(u);
+                    mx = fmaxf(mx, fabsf(u));
+                }
+            }
+            const int sU = scale_exp(row_max(mx, m->xu[lc & 1]));
+            if (stop) break;
+            {   // U^T row part (A of M2 and M4): kTK tokens = kTK / 2 packed columns
+                const float f = exp2i(sU);
+                uint32_t w[kTK / 2];
+#pragma unroll
+                for (int j = 0; j < kTK / 2; ++j)
+                    w[j] = f2h2_bits(__uint_as_float(x[2 * j]) * f, __uint_as_float(x[2 * j + 1]) * f);
+                tmem_stn<kTK / 2>(tmem + lane_off + TT_UA + qp * (kTK / 2), w);
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(&m->u_ready);
+            }
+            // (b) S = S Diag(exp(G_C)) + ΔS
+            if (!warp_wait(&m->bar2, lc & 1)) { fail(ERR_TIMEOUT_MMA); stop = true; }
+            if (!stop) {
+                tc_fence_after();
+                const float f1 = exp2i(-sK), f2 = exp2i(-sU);
+                const float *gam = m->gam[s] + qp * kSC;
+                uint32_t d[kSC];
+                tmem_ldn<kSC>(tmem + lane_off + TT_DS + qp * kSC, d);
+                tmem_wait_ld();
+#pragma unroll
+                for (int jj = 0; jj < kSC; ++jj) {
+                    const float gc = CHANNEL ? gam[jj] : m->gam[s][0];
+                    S[jj] = fmaf(gc, S[jj], __uint_as_float(d[jj]) * f1 * f2);
+                }
+                tc_fence_before();
+                mbar_arrive(&m->empty_u[s]);   // Ũ, exponents and gate of this stage are read
+            }
+            // (stop may differ between warps here; the barrier in (c) settles it)
+            const int sS_next = (lc + 1 < nl) ? publish(lc + 1) : 0;
+            // (c) output rows: O^T = O_inter^T + O4^T, unscaled, for this thread's
+            //     tokens, staged as a [token][channel] tile
+            if (!warp_wait(&m->bar4, lc & 1)) { fail(ERR_TIMEOUT_MMA); stop = true; }
+            if (!stop) {
+                uint32_t o4[kTK];
+                tc_fence_after();
+                tmem_ldn<kTK>(tmem + lane_off + TT_O4 + qp * kTK, o4);
+                tmem_wait_ld();
+                const float fq1 = exp2i(-sQ), fq2 = exp2i(-sS), fp1 = exp2i(-sP), fp2 = exp2i(-sU);
+                const uint32_t stile = sbase + TO_OS + s * 16384 + qp * kTK * 256 + row * 2;
+#pragma unroll
+                for (int jj = 0; jj < kTK; ++jj) {
+                    const __nv_bfloat16 b = __float2bfloat16_rn(__uint_as_float(oi[jj]) * fq1 * fq2 +
+                                                                __uint_as_float(o4[jj]) * fp1 * fp2);
+                    st_shared_b16(stile + jj * 256, *reinterpret_cast<const uint16_t *>(&b));
+                }
+            }
+            rows_sync();
+            if (stop) break;
+            {   // 64 rows x 256 bytes leave as 16-byte segments; rows past the end stay
+                const int cc = c_begin + lc;
+                const int cl = min(C, len - cc * C);
+                const uint32_t tile = sbase + TO_OS + s * 16384;
+#pragma unroll
+                for (int q = 0; q < 1024 / kRowThreads; ++q) {
+                    const int e = q * kRowThreads + tid;   // segment: row e / 16, 16 bytes e % 16
+                    const int i = e >> 4, seg = e & 15;
+                    if (i < cl) {
+                        const uint4 v = ld_shared_v4(tile + i * 256 + seg * 16);
+                        *reinterpret_cast<uint4 *>(o + ((size_t)(t0 + cc * C + i) * H + h) * D + seg * 8) = v;
+                    }
+                }
+            }
+            sS = sS_next;
+        }
+        if (s_out != nullptr) {
+#pragma unroll
+            for (int j = 0; j < kSC; j += 4)
+                *reinterpret_cast<float4 *>(s_out + sg + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+        }
+    } else if (warp == kRowWarps) {
+        // ======================================================= MMA issuer ====
+        if (lane == 0) {
+            for (int lc = 0; lc < nl; ++lc) {
+                if (*abort_flag) break;
+                const uint32_t s = lc & 1, sph = (lc >> 1) & 1;
+                if (!mbar_wait_sleep(&m->full_a1[s], sph)) { fail(ERR_TIMEOUT_TMA); break; }
+                if (!mbar_wait_sleep(&m->s_ready, lc & 1)) { fail(ERR_TIMEOUT_HANDOFF); break; }
+                tc_fence_after();
+                const uint64_t d_a1 = sw128_kmajor_desc(sbase + TO_A1 + s * 32768);
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    mma_f16_ts(tmem + TT_D1, tmem + TT_SA + k * 8,
+                               d_a1 + (((k >> 2) * 16384 + (k & 3) * 32) >> 4), IDESC_H128, k != 0);
+                mma_commit(&m->bar1);
+                mma_commit(&m->empty_a1[s]);
+                if (!mbar_wait_sleep(&m->full_kp[s], sph)) { fail(ERR_TIMEOUT_TMA); break; }
+                if (!mbar_wait_sleep(&m->u_ready, lc & 1)) { fail(ERR_TIMEOUT_HANDOFF); break; }
+                tc_fence_after();
+                const uint64_t d_kh = sw128_kmajor_desc(sbase + TO_KH + s * 16384);
+                const uint64_t d_pm = sw128_kmajor_desc(sbase + TO_PM + s * 8192);
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    mma_f16_ts(tmem + TT_DS, tmem + TT_UA + k * 8, d_kh + ((k * 32) >> 4), IDESC_H128, k != 0);
+                mma_commit(&m->bar2);
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    mma_f16_ts(tmem + TT_O4, tmem + TT_UA + k * 8, d_pm + ((k * 32) >> 4), IDESC_H64, k != 0);
+                mma_commit(&m->bar4);
+                mma_commit(&m->empty_kp[s]);
+            }
+        }
+    } else if (lane == 0) {
+        // ==================================================== record loader ====
+        const uint32_t gbytes = CHANNEL ? 512u : 16u;
+        uint32_t issued[6] = {0, 0, 0, 0, 0, 0};
+        uint64_t *bars[6] = {&m->full_a1[0], &m->full_a1[1], &m->full_u[0], &m->full_u[1],
+                             &m->full_kp[0], &m->full_kp[1]};
+        auto load_a1 = [&](int lc) {
+            const int s = lc & 1;
+            mbar_arrive_expect_tx(&m->full_a1[s], 32768);
+            bulk_load(sm + TO_A1 + s * 32768, rec_of(lc) + REC_A1, 32768, &m->full_a1[s]);
+            ++issued[s];
+        };
+        auto load_u = [&](int lc) {
+            const int s = lc & 1;
+            const uint8_t *r = rec_of(lc);
+            mbar_arrive_expect_tx(&m->full_u[s], 32768 + 16 + gbytes);
+            bulk_load(sm + TO_UT + s * 32768, r + REC_UT, 32768, &m->full_u[s]);
+            bulk_load(m->ex[s], r + REC_EX, 16, &m->full_u[s]);
+            bulk_load(m->gam[s], r + REC_GC, gbytes, &m->full_u[s]);
+            ++issued[2 + s];
+        };
+        auto load_kp = [&](int lc) {
+            const int s = lc & 1;
+            const uint8_t *r = rec_of(lc);
+            mbar_arrive_expect_tx(&m->full_kp[s], 16384 + 8192);
+            bulk_load(sm + TO_KH + s * 16384, r + REC_KH, 16384, &m->full_kp[s]);
+            bulk_load(sm + TO_PM + s * 8192, r + REC_PM, 8192, &m->full_kp[s]);
+            ++issued[4 + s];
+        };
+        auto prefetch_rec = [&](int lc) {
+            if (lc < nl) {
+                const uint8_t *r = rec_of(lc);
+#pragma unroll
+                for (int q = 0; q < 5; ++q) bulk_prefetch_l2(r + q * 18128, 18128);
+            }
+        };
+        load_a1(0);
+        load_kp(0);
+        load_u(0);
+        if (nl > 1) {
+            load_a1(1);
+            load_u(1);
+            load_kp(1);
+        }
+        prefetch_rec(2);
+        prefetch_rec(3);
+        for (int lc = 0; lc < nl; ++lc) {
+            if (*abort_flag) break;
+            const uint32_t s = lc & 1, sph = (lc >> 1) & 1;
+            if (!mbar_wait_sleep(&m->empty_a1[s], sph)) { fail(ERR_TIMEOUT_MMA); break; }
+            if (lc + 2 < nl) load_a1(lc + 2);
+            if (!mbar_wait_sleep(&m->empty_kp[s], sph)) { fail(ERR_TIMEOUT_MMA); break; }
+            if (lc + 2 < nl) load_kp(lc + 2);
+            if (!mbar_wait_sleep(&m->empty_u[s], sph)) { fail(ERR_TIMEOUT_HANDOFF); break; }
+            if (lc + 2 < nl) load_u(lc + 2);
+            prefetch_rec(lc + 4);
+        }
+        // never leave a bulk copy in flight into this CTA's shared memory
+        for (int q = 0; q < 6; ++q)
+            if (issued[q] > 0) (void)mbar_wait_sleep(bars[q], (issued[q] - 1) & 1);
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TT_COLS);
     }
 }
 
@@ -1156,8 +1495,11 @@ chain_split_kernel(const uint8_t *__restrict__ recs, const float *h0, float *fin
 
 constexpr size_t kHeaderBytes = 256;                        // error word
 constexpr size_t kMaxRecordBytes = size_t(1) << 30;         // records per window
-constexpr int kSplitMaxChains = 148;                        // one chain CTA per SM
-constexpr int kSplitDvMaxChains = 148 / kSplitParts;        // d_v split: 4 CTAs a chain
+// Up to 64 chains the two kernels beat the single-kernel plan: its chunk
+// period is set by the chunk-local work, which the prep kernel spreads over
+// all SMs.  With more chains that plan already keeps most SMs busy and the
+// prep kernel's extra record traffic no longer pays (measured on B200).
+constexpr int kSplitMaxChains = 64;
 
 struct SplitPlan {
     int chains = 0, max_chunks = 0, window = 0, windows = 0;
@@ -1178,6 +1520,22 @@ bool make_split_plan(int num_seqs, int total_T, int H, SplitPlan &p) {
     p.rec_off = (kHeaderBytes + state + 1023) & ~size_t(1023);
     p.bytes = p.rec_off + (size_t)p.window * per;
     return true;
+}
+
+// Value channels per chain CTA: as few as keep every chain CTA on its own SM.
+int channels_per_cta(int chains) { return chains * 4 <= 148 ? 32 : (chains * 2 <= 148 ? 64 : 128); }
+
+template <int NB>
+cudaError_t launch_chain(bool channel, int chains, const uint8_t *recs, const float *h0, float *fin,
+                         float *state, const int32_t *cu, int num_seqs, int total_T, int H, int c0,
+                         int c1, __nv_bfloat16 *o, uint32_t *err, cudaStream_t stream) {
+    using K = Chain<NB>;
+    auto kern = channel ? chain_kernel<true, NB> : chain_kernel<false, NB>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)K::SMEM);
+    if (e != cudaSuccess) return e;
+    kern<<<(unsigned)(chains * (D / NB)), K::kThreads, K::SMEM, stream>>>(
+        recs, h0, fin, state, cu, num_seqs, total_T, H, c0, c1, o, err);
+    return cudaGetLastError();
 }
 
 }  // namespace
@@ -1201,22 +1559,18 @@ cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, co
     if (!make_map(&mq, q, total_T, Hqk) || !make_map(&mk, k, total_T, Hqk) ||
         !make_map(&mv, v, total_T, H))
         return cudaErrorInvalidValue;
-    const bool dv_split = p.chains <= kSplitDvMaxChains;
     auto prep = channel ? prep_kernel<true> : prep_kernel<false>;
-    auto chain = channel ? chain_kernel<true> : chain_kernel<false>;
-    auto chain_dv = channel ? chain_split_kernel<true> : chain_split_kernel<false>;
     e = cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PREP_SMEM);
-    if (e != cudaSuccess) return e;
-    if (dv_split)
-        e = cudaFuncSetAttribute(chain_dv, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)VSPLIT_SMEM);
-    else
-        e = cudaFuncSetAttribute(chain, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)CHAIN_SMEM);
     if (e != cudaSuccess) return e;
     float *state = p.windows > 1 ? reinterpret_cast<float *>(ws + p.state_off) : nullptr;
     uint8_t *recs = ws + p.rec_off;
     __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(o);
+    // Few chains: split d_v over four CTAs each (NB = 32), so that more SMs
+    // share the chain work; otherwise one CTA per chain, transposed form.
+    const bool dv_split = p.chains * 4 <= 148;
+    auto chain_t = channel ? chain_t_kernel<true> : chain_t_kernel<false>;
+    e = cudaFuncSetAttribute(chain_t, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TSMEM);
+    if (e != cudaSuccess) return e;
     for (int w = 0; w < p.windows; ++w) {
         const int c0 = w * p.window;
         const int c1 = c0 + p.window < p.max_chunks ? c0 + p.window : p.max_chunks;
@@ -1224,13 +1578,14 @@ cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, co
             mq, mk, mv, g, beta, cu, num_seqs, total_T, Hqk, H, c0, recs, err);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
-        if (dv_split)
-            chain_dv<<<(unsigned)(p.chains * kSplitParts), kSplitThreads, VSPLIT_SMEM, stream>>>(
-                recs, h0, fin, state, cu, num_seqs, total_T, H, c0, c1, out, err);
-        else
-            chain<<<(unsigned)p.chains, kChainThreads, CHAIN_SMEM, stream>>>(
-                recs, h0, fin, state, cu, num_seqs, total_T, H, c0, c1, out, err);
-        e = cudaGetLastError();
+        if (dv_split) {
+            e = launch_chain<32>(channel, p.chains, recs, h0, fin, state, cu, num_seqs, total_T, H, c0, c1,
+                                 out, err, stream);
+        } else {
+            chain_t<<<(unsigned)p.chains, kTThreads, TSMEM, stream>>>(recs, h0, fin, state, cu, num_seqs,
+                                                                     total_T, H, c0, c1, out, err);
+            e = cudaGetLastError();
+        }
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;

@@ -99,9 +99,9 @@ GDR_API const char *gdr_status_string(gdr_status_t status);
  * this problem (written to *bytes; may be 0).  Pure host function.
  *
  * The tcgen05 kernels take two plans.  The single-kernel plan needs 16 bytes
- * (an error word).  With fewer (sequence, head) pairs than 149, the
+ * (an error word).  With at most 64 (sequence, head) pairs, the
  * chunk-parallel plan (GDR_PATH_TCGEN05_SPLIT) keeps all SMs busy; it needs
- * 144.5 KiB per (chunk, sequence, head) of its chunk records, capped at
+ * 90,640 bytes per (chunk, sequence, head) of its chunk records, capped at
  * 1 GiB by running long problems in windows of chunks (plus 64 KiB of state
  * per (sequence, head) between windows).  The size reported here is the
  * larger one where both apply; gdr_prefill_chunked runs the chunk-parallel

@@ -112,10 +112,10 @@ def test_workspace_and_path_queries(lib):
 
 def test_plan_selection_and_workspace_sizes(lib):
     """The tcgen05 family runs as two plans: the chunk-parallel one with the
-    reported workspace (144.5 KiB of chunk records per chunk and head, in
+    reported workspace (90,640 bytes of chunk records per chunk and head, in
     windows of at most 1 GiB), the single-kernel one with 16 bytes."""
     S, CH, BF = gdr.GDR_GATE_SCALAR, gdr.GDR_GATE_CHANNEL, gdr.GDR_BF16
-    rec = 147968
+    rec = 90640
     nb = gdr.gdr_prefill_workspace_size(1, 8192, 16, 128, 128, S, BF)
     assert nb == 1024 + 128 * 16 * rec
     assert gdr.gdr_prefill_plan(1, 8192, 16, 128, 128, S, BF, nb) == gdr.GDR_PATH_TCGEN05_SPLIT
@@ -124,17 +124,18 @@ def test_plan_selection_and_workspace_sizes(lib):
     assert gdr.gdr_prefill_plan(1, 8192, 16, 128, 128, S, BF, 16) == gdr.GDR_PATH_TCGEN05
     with pytest.raises(gdr.GdrError):
         gdr.gdr_prefill_plan(1, 8192, 16, 128, 128, S, BF, 8)
-    # more (sequence, head) pairs than SMs: the single-kernel plan only
-    assert gdr.gdr_prefill_workspace_size(2, 8192, 128, 128, 128, S, BF) == 16
-    assert gdr.gdr_prefill_plan(2, 8192, 128, 128, 128, S, BF, 1 << 40) == gdr.GDR_PATH_TCGEN05
+    # more than 64 (sequence, head) pairs: the single-kernel plan only
+    assert gdr.gdr_prefill_workspace_size(2, 8192, 33, 128, 128, S, BF) == 16
+    assert gdr.gdr_prefill_plan(2, 8192, 33, 128, 128, S, BF, 1 << 40) == gdr.GDR_PATH_TCGEN05
+    assert gdr.gdr_prefill_workspace_size(1, 8192, 64, 128, 128, S, BF) > 16
     # fp32 I/O and other head sizes: the CUDA-core kernel, no workspace
     assert gdr.gdr_prefill_plan(1, 8192, 16, 128, 128, S, gdr.GDR_F32, 0) == gdr.GDR_PATH_SIMT
     assert gdr.gdr_prefill_plan(1, 8192, 16, 64, 64, S, BF, 0) == gdr.GDR_PATH_SIMT
-    # 148 heads x 60 chunks: records beyond 1 GiB -> windows of 49 chunks with
+    # 64 heads x 250 chunks: records beyond 1 GiB -> windows of 185 chunks with
     # 64 KiB of state per head between them
-    nb = gdr.gdr_prefill_workspace_size(1, 3840, 148, 128, 128, S, BF)
-    state = 148 * 128 * 128 * 4
-    assert nb == ((256 + state + 1023) // 1024) * 1024 + 49 * 148 * rec
+    nb = gdr.gdr_prefill_workspace_size(1, 16000, 64, 128, 128, S, BF)
+    state = 64 * 128 * 128 * 4
+    assert nb == ((256 + state + 1023) // 1024) * 1024 + 185 * 64 * rec
     # a tcgen05 problem without any workspace is refused before any launch
     assert _prefill(lib, dk=128, dv=128, io=1) == gdr.GDR_ERR_WORKSPACE
 
