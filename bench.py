@@ -388,8 +388,9 @@ def barrier(ws):
 
 
 def load_traffic(case):
-    """DRAM bytes per launch of the dominant kernel from a committed ncu
-    capture, if it was taken on the kernel sources as they are now."""
+    """DRAM bytes per launch (single-kernel plans) or per step (the two-kernel
+    chunk-parallel plan) from a committed ncu capture, if it was taken on the
+    kernel sources as they are now."""
     p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if not os.path.exists(p):
         return None
@@ -404,7 +405,8 @@ def load_traffic(case):
             h.update(open(os.path.join(ROOT, rel), "rb").read())
         if h.hexdigest() != ent["sources_sha256"]:
             return None
-        return float(ent["bytes_per_launch"])
+        # one kernel: DRAM bytes per launch; a multi-kernel plan: per step
+        return float(ent.get("bytes_per_step", ent.get("bytes_per_launch")))
     except Exception:
         return None
 
