@@ -167,11 +167,14 @@ def decode_work(inp):
 def split_launches(inp):
     """Kernel launches of the chunk-parallel plan: a prep and a chain kernel
     per window of chunks (the library bounds the chunk records of one window
-    to 1 GiB at 90,640 bytes per chunk and head)."""
+    to 1 GiB at 90,640 bytes per chunk and head), and per pipeline piece when
+    a single window is cut into pieces."""
     chains = inp.num_seqs * inp.H
     max_chunks = -(-inp.total_T // 64)
     window = max(1, min(max_chunks, (1 << 30) // (chains * 90640)))
-    return 2 * (-(-max_chunks // window))
+    windows = -(-max_chunks // window)
+    pieces = min(4, max(1, max_chunks // 32)) if windows == 1 else 1   # pipelined pieces
+    return 2 * windows * pieces
 
 
 class PrefillCase:

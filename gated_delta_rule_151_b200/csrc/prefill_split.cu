@@ -39,7 +39,9 @@
 #include <cudaTypedefs.h>
 #include <cuda_fp16.h>
 
+#include <algorithm>
 #include <cstddef>
+#include <mutex>
 
 #include "common.cuh"
 #include "gdr.h"
@@ -1503,6 +1505,7 @@ constexpr int kSplitMaxChains = 64;
 
 struct SplitPlan {
     int chains = 0, max_chunks = 0, window = 0, windows = 0;
+    int pieces = 1;   // pipeline pieces of a single window (prep of piece k + 1 beside chain k)
     size_t state_off = 0, rec_off = 0, bytes = 0;
 };
 
@@ -1515,15 +1518,48 @@ bool make_split_plan(int num_seqs, int total_T, int H, SplitPlan &p) {
     const size_t fit = kMaxRecordBytes / per;
     p.window = (int)(fit < 1 ? 1 : (fit < (size_t)p.max_chunks ? fit : (size_t)p.max_chunks));
     p.windows = (p.max_chunks + p.window - 1) / p.window;
-    const size_t state = p.windows > 1 ? (size_t)p.chains * D * D * sizeof(float) : 0;
+    p.pieces = p.windows == 1 ? std::min(4, std::max(1, p.max_chunks / 32)) : 1;
+    const size_t state =
+        (p.windows > 1 || p.pieces > 1) ? (size_t)p.chains * D * D * sizeof(float) : 0;
     p.state_off = kHeaderBytes;
     p.rec_off = (kHeaderBytes + state + 1023) & ~size_t(1023);
     p.bytes = p.rec_off + (size_t)p.window * per;
     return true;
 }
 
-// Value channels per chain CTA: as few as keep every chain CTA on its own SM.
-int channels_per_cta(int chains) { return chains * 4 <= 148 ? 32 : (chains * 2 <= 148 ? 64 : 128); }
+
+// Per-device helper streams for the pipelined plan: chain kernels on a
+// high-priority stream, prep kernels on a low-priority one, forked from and
+// joined back into the caller's stream with events (capturable in a graph).
+struct Helpers {
+    bool ready = false;
+    cudaStream_t chain_s = nullptr, prep_s = nullptr;
+    cudaEvent_t fork = nullptr, prep_done = nullptr, join = nullptr;
+};
+constexpr int kMaxDevices = 64;
+std::mutex g_helpers_mutex;
+Helpers g_helpers[kMaxDevices];
+
+cudaError_t get_helpers(Helpers **out) {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    Helpers &hs = g_helpers[dev];
+    if (!hs.ready) {
+        int least = 0, greatest = 0;
+        e = cudaDeviceGetStreamPriorityRange(&least, &greatest);
+        if (e == cudaSuccess) e = cudaStreamCreateWithPriority(&hs.chain_s, cudaStreamNonBlocking, greatest);
+        if (e == cudaSuccess) e = cudaStreamCreateWithPriority(&hs.prep_s, cudaStreamNonBlocking, least);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&hs.fork, cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&hs.prep_done, cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&hs.join, cudaEventDisableTiming);
+        if (e != cudaSuccess) return e;
+        hs.ready = true;
+    }
+    *out = &hs;
+    return cudaSuccess;
+}
 
 template <int NB>
 cudaError_t launch_chain(bool channel, int chains, const uint8_t *recs, const float *h0, float *fin,
@@ -1562,7 +1598,7 @@ cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, co
     auto prep = channel ? prep_kernel<true> : prep_kernel<false>;
     e = cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PREP_SMEM);
     if (e != cudaSuccess) return e;
-    float *state = p.windows > 1 ? reinterpret_cast<float *>(ws + p.state_off) : nullptr;
+    float *state = (p.windows > 1 || p.pieces > 1) ? reinterpret_cast<float *>(ws + p.state_off) : nullptr;
     uint8_t *recs = ws + p.rec_off;
     __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(o);
     // Few chains: split d_v over four CTAs each (NB = 32), so that more SMs
@@ -1571,21 +1607,48 @@ cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, co
     auto chain_t = channel ? chain_t_kernel<true> : chain_t_kernel<false>;
     e = cudaFuncSetAttribute(chain_t, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TSMEM);
     if (e != cudaSuccess) return e;
+    auto run_chain = [&](int c0, int c1, const uint8_t *r, cudaStream_t st) {
+        if (dv_split)
+            return launch_chain<32>(channel, p.chains, r, h0, fin, state, cu, num_seqs, total_T, H, c0, c1,
+                                    out, err, st);
+        chain_t<<<(unsigned)p.chains, kTThreads, TSMEM, st>>>(r, h0, fin, state, cu, num_seqs, total_T, H,
+                                                                c0, c1, out, err);
+        return cudaGetLastError();
+    };
+    auto run_prep = [&](int c0, int c1, uint8_t *r, cudaStream_t st) {
+        prep<<<dim3((unsigned)(c1 - c0), (unsigned)p.chains), kPrepThreads, PREP_SMEM, st>>>(
+            mq, mk, mv, g, beta, cu, num_seqs, total_T, Hqk, H, c0, r, err);
+        return cudaGetLastError();
+    };
+    if (p.pieces > 1) {
+        // every record has its own slot: the prep kernel of piece k + 1 runs on
+        // the SMs the chain kernel of piece k leaves free
+        std::lock_guard<std::mutex> lock(g_helpers_mutex);
+        Helpers *hs = nullptr;
+        e = get_helpers(&hs);
+        if (e != cudaSuccess) return e;
+        const int per = (p.max_chunks + p.pieces - 1) / p.pieces;
+        e = cudaEventRecord(hs->fork, stream);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(hs->prep_s, hs->fork, 0);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(hs->chain_s, hs->fork, 0);
+        for (int k = 0; k < p.pieces && e == cudaSuccess; ++k) {
+            const int c0 = k * per, c1 = std::min(c0 + per, p.max_chunks);
+            uint8_t *r = recs + (size_t)c0 * p.chains * REC_BYTES;
+            e = run_prep(c0, c1, r, hs->prep_s);
+            if (e == cudaSuccess) e = cudaEventRecord(hs->prep_done, hs->prep_s);
+            if (e == cudaSuccess) e = cudaStreamWaitEvent(hs->chain_s, hs->prep_done, 0);
+            if (e == cudaSuccess) e = run_chain(c0, c1, r, hs->chain_s);
+        }
+        if (e == cudaSuccess) e = cudaEventRecord(hs->join, hs->chain_s);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(stream, hs->join, 0);
+        return e;
+    }
     for (int w = 0; w < p.windows; ++w) {
         const int c0 = w * p.window;
         const int c1 = c0 + p.window < p.max_chunks ? c0 + p.window : p.max_chunks;
-        prep<<<dim3((unsigned)(c1 - c0), (unsigned)p.chains), kPrepThreads, PREP_SMEM, stream>>>(
-            mq, mk, mv, g, beta, cu, num_seqs, total_T, Hqk, H, c0, recs, err);
-        e = cudaGetLastError();
+        e = run_prep(c0, c1, recs, stream);
         if (e != cudaSuccess) return e;
-        if (dv_split) {
-            e = launch_chain<32>(channel, p.chains, recs, h0, fin, state, cu, num_seqs, total_T, H, c0, c1,
-                                 out, err, stream);
-        } else {
-            chain_t<<<(unsigned)p.chains, kTThreads, TSMEM, stream>>>(recs, h0, fin, state, cu, num_seqs,
-                                                                     total_T, H, c0, c1, out, err);
-            e = cudaGetLastError();
-        }
+        e = run_chain(c0, c1, recs, stream);
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;

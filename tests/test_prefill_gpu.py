@@ -269,3 +269,20 @@ def test_plans_agree(mode):
     o2, f2 = gpu_prefill(inp, plan="single")
     assert float((o1.float() - o2.float()).abs().max()) <= 4e-3
     assert float((f1 - f2).norm() / f2.norm()) <= 1e-4
+
+
+@pytest.mark.parametrize("mode", [I.SCALAR, I.CHANNEL])
+def test_chunk_parallel_plan_in_pipelined_pieces(mode):
+    """100 chunks of records fit one window, which runs as three pipelined
+    pieces (prep of the next piece beside the chain of this one, the state
+    handed between pieces through the workspace).  Sequences of 32 chunks, one
+    token and 69 chunks, so pieces end inside and after sequences."""
+    inp = I.make_inputs(total_T=6400, H=4, d_k=128, gate_mode=mode, io_dtype=torch.bfloat16,
+                        cu_seqlens=[0, 2048, 2049, 6400], c=0.1, h0_std=0.02, seed=53)
+    nb = gdr.gdr_prefill_workspace_size(3, 6400, 4, 128, 128, 0 if mode == I.SCALAR else 1,
+                                        gdr.GDR_BF16)
+    assert gdr.gdr_prefill_plan(3, 6400, 4, 128, 128, 0 if mode == I.SCALAR else 1, gdr.GDR_BF16,
+                                nb) == gdr.GDR_PATH_TCGEN05_SPLIT
+    o, fin = gpu_prefill(inp)
+    o_ref, fin_ref = oracle_prefill(inp)
+    check(inp, o, fin, o_ref, fin_ref, "pieces")
