@@ -284,6 +284,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         if (!block_wait(&m->bar_tma, 0, &m->abort_flag, err, ERR_TIMEOUT_TMA)) break;
 
         float GC = 0.f;
+        float kmax = 0.f, qmax = 0.f;   // channel gate: this thread's largest |k| and |q|
         if (CHANNEL) {
             // chunk-cumulative gate of this thread's tokens; reference R = G_31
             const float T0 = m->u.c.T0[ch], T1 = m->u.c.T1[ch];
@@ -303,6 +304,8 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 const int i = hh * 32 + k;
                 const uint32_t src = sbase + PO_KQ + kcol + sw128_offset(i, cch) + cel;
                 const float kv = ld_shared_bf16(src), qv = ld_shared_bf16(src + 8192);
+                kmax = fmaxf(kmax, fabsf(kv));
+                qmax = fmaxf(qmax, fabsf(qv));
                 const float up = __expf(gr[k] - R), dn = __expf(R - gr[k]);
                 const float a = kv * up, b = qv * up, e = kv * dn;
                 bad |= !(fabsf(a) < kF16Limit) || !(fabsf(b) < kF16Limit) ||
@@ -518,15 +521,16 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             }
         } else {
             const uint32_t kcol = (ch >> 6) * 16384, cch = (ch & 63) >> 3, cel = (ch & 7) * 2;
-            float mk = 0.f, mq = 0.f;
-#pragma unroll 4
+            // scales from bounds: |K̂| <= max|k| e^{max(G_C - G)}, |Q̃| <= max|q| e^{max G};
+            // a bound above the true maximum only moves values down within fp16's
+            // normal range, so the precision is the same
+            float dk = -3.0e38f, dq = -3.0e38f;
+#pragma unroll
             for (int k = 0; k < 32; ++k) {
-                const int i = hh * 32 + k;
-                const uint32_t src = sbase + PO_KQ + kcol + sw128_offset(i, cch) + cel;
-                mk = fmaxf(mk, fabsf(ld_shared_bf16(src) * __expf(GC - gr[k])));
-                mq = fmaxf(mq, fabsf(ld_shared_bf16(src + 8192) * __expf(gr[k])));
+                dk = fmaxf(dk, GC - gr[k]);
+                dq = fmaxf(dq, gr[k]);
             }
-            block_scale2(mk, mq, m->red, sK, sQ);
+            block_scale2(kmax * __expf(dk), qmax * __expf(dq), m->red, sK, sQ);
             const float fk = exp2i(sK), fq = exp2i(sQ);
             const uint32_t rowblk = hh * 16384;
             uint8_t *qdst = rec + REC_A1 + (ch >> 6) * 16384;
@@ -1627,12 +1631,20 @@ cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, co
         Helpers *hs = nullptr;
         e = get_helpers(&hs);
         if (e != cudaSuccess) return e;
-        const int per = (p.max_chunks + p.pieces - 1) / p.pieces;
+        // a short first piece: only its prep runs before any chain work
+        const int first = std::min(8, p.max_chunks);
+        const int per = (p.max_chunks - first + p.pieces - 2) / (p.pieces - 1);
+        auto piece = [&](int k, int &c0, int &c1) {
+            c0 = k == 0 ? 0 : first + (k - 1) * per;
+            c1 = std::min(k == 0 ? first : c0 + per, p.max_chunks);
+        };
         e = cudaEventRecord(hs->fork, stream);
         if (e == cudaSuccess) e = cudaStreamWaitEvent(hs->prep_s, hs->fork, 0);
         if (e == cudaSuccess) e = cudaStreamWaitEvent(hs->chain_s, hs->fork, 0);
         for (int k = 0; k < p.pieces && e == cudaSuccess; ++k) {
-            const int c0 = k * per, c1 = std::min(c0 + per, p.max_chunks);
+            int c0, c1;
+            piece(k, c0, c1);
+            if (c0 >= c1) break;
             uint8_t *r = recs + (size_t)c0 * p.chains * REC_BYTES;
             e = run_prep(c0, c1, r, hs->prep_s);
             if (e == cudaSuccess) e = cudaEventRecord(hs->prep_done, hs->prep_s);
