@@ -690,8 +690,11 @@ struct Chain {
     static constexpr uint32_t TD4 = kStages * NB;         // per O buffer
     static constexpr uint32_t TD2 = 2 * kStages * NB;
     static constexpr uint32_t TCOLS = TD2 + NB <= 256 ? 256 : 512;
-    static constexpr uint32_t IDESC = make_idesc(0, 128, NB);   // fp16 x fp16 -> fp32
+    // fp16 x fp16 -> fp32, B (the S and U images) MN-major
+    static constexpr uint32_t IDESC = make_idesc(0, 128, NB) | (1u << 16);
     static_assert(SMEM <= 232448 && TD2 + NB <= 512, "chain kernel does not fit");
+    // the S and U images are MN-major with one 64-byte row (32 channels) per K index
+    static_assert(NB == 32, "MN-major images hold 32 value channels");
 };
 
 struct ChainMisc {
@@ -829,9 +832,9 @@ chain_kernel(const uint8_t *__restrict__ recs, const float *h0, float *fin, floa
 #pragma unroll
         for (int j = 0; j < K::kCS; ++j)
             S[j] = s_in != nullptr ? s_in[sg + (size_t)(c0 + j) * D + t] : 0.f;
-        // fp16 image of the state block for chunk lc, with its scale exponent
-        const uint32_t scol = sbase + K::SB + (t >> 6) * (NB * 128) + (t & 7) * 2;
-        const uint32_t schk = (t & 63) >> 3;
+        // fp16 image of the state block for chunk lc (MN-major: row t holds the 32
+        // channels of d_k index t), with its scale exponent
+        const uint32_t srow = sbase + K::SB + t * 64;
         bool stop = false;
         auto publish = [&](int lc) {
             float mx = 0.f;
@@ -840,7 +843,10 @@ chain_kernel(const uint8_t *__restrict__ recs, const float *h0, float *fin, floa
             const int sS = role_scale(mx, m->red_s[lc & 1], warp, K::kSW, 1, stop, abort_flag);
             const float f = exp2i(sS);
 #pragma unroll
-            for (int j = 0; j < K::kCS; ++j) st_shared_b16(scol + sw128_offset(c0 + j, schk), f2h_bits(S[j] * f));
+            for (int c = 0; c < 4; ++c)
+                st_shared_v4(srow + ((c ^ ((t >> 1) & 3)) << 4), f2h2_bits(S[8 * c] * f, S[8 * c + 1] * f),
+                             f2h2_bits(S[8 * c + 2] * f, S[8 * c + 3] * f), f2h2_bits(S[8 * c + 4] * f, S[8 * c + 5] * f),
+                             f2h2_bits(S[8 * c + 6] * f, S[8 * c + 7] * f));
             if (tid == 0) m->es[lc & 3] = sS;
             fence_proxy_async();
             mbar_arrive(&m->s_ready);
@@ -880,8 +886,7 @@ chain_kernel(const uint8_t *__restrict__ recs, const float *h0, float *fin, floa
         if (r < 2) {
             // ===================================== U_b = Ũ_b + X, thread = token i ====
             const int i = r * 32 + lane;
-            const uint32_t ucol = sbase + K::UB + (i & 7) * 2;
-            const uint32_t uchk = i >> 3;
+            const uint32_t urow_img = sbase + K::UB + i * 64;   // MN-major: row i = token
             bool stop = false;
             for (int lc = 0; lc < nl && !stop; ++lc) {
                 const uint32_t s = lc & 1;
@@ -894,29 +899,24 @@ chain_kernel(const uint8_t *__restrict__ recs, const float *h0, float *fin, floa
                 const int sW = m->ex[s][0], sQ = m->ex[s][1], sK = m->ex[s][2], sP = m->ex[s][3];
                 const int sS = m->es[lc & 3];
                 const float fa = exp2i(-sW), fb = exp2i(-sS);
-                // U = Ũ + X in fp32, written back over this thread's Ũ row (the stage
-                // is read only here) until the block's scale is known
+                // U = Ũ + X in fp32 (this thread's token row, 32 channels)
+                float u[32];
                 float mx = 0.f;
-#pragma unroll
-                for (int p = 0; p < K::kCU / 32 && !stop; ++p) {
+                if (!stop) {
                     uint32_t x[32];
-                    tmem_ld32(tmem + lane_off + K::TD1 + b * NB + c0 + p * 32, x);
-                    const uint32_t urow =
-                        sbase + K::UT + s * (256 * NB) + ((c0 + p * 32) >> 5) * 8192 + i * 128;
+                    tmem_ld32(tmem + lane_off + K::TD1 + b * NB, x);
+                    const uint32_t urow = sbase + K::UT + s * (256 * NB) + i * 128;
                     tmem_wait_ld();
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {
-                        const uint32_t a = urow + ((q ^ (i & 7)) << 4);
-                        const uint4 v = ld_shared_v4(a);
-                        float w[4] = {__uint_as_float(v.x), __uint_as_float(v.y),
-                                      __uint_as_float(v.z), __uint_as_float(v.w)};
+                        const uint4 v = ld_shared_v4(urow + ((q ^ (i & 7)) << 4));
+                        const float w[4] = {__uint_as_float(v.x), __uint_as_float(v.y),
+                                            __uint_as_float(v.z), __uint_as_float(v.w)};
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
-                            w[e] += __uint_as_float(x[q * 4 + e]) * fa * fb;
-                            mx = fmaxf(mx, fabsf(w[e]));
+                            u[q * 4 + e] = w[e] + __uint_as_float(x[q * 4 + e]) * fa * fb;
+                            mx = fmaxf(mx, fabsf(u[q * 4 + e]));
                         }
-                        st_shared_v4(a, __float_as_uint(w[0]), __float_as_uint(w[1]),
-                                     __float_as_uint(w[2]), __float_as_uint(w[3]));
                     }
                 }
                 const int sU = role_scale(mx, m->red_u[lc & 1], set * 2 + r, 2 * K::kSets, 2, stop,
@@ -924,20 +924,11 @@ chain_kernel(const uint8_t *__restrict__ recs, const float *h0, float *fin, floa
                 if (stop) break;
                 const float fu = exp2i(sU);
 #pragma unroll
-                for (int p = 0; p < K::kCU / 32; ++p) {
-                    const uint32_t urow =
-                        sbase + K::UT + s * (256 * NB) + ((c0 + p * 32) >> 5) * 8192 + i * 128;
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const uint4 v = ld_shared_v4(urow + ((q ^ (i & 7)) << 4));
-                        const float w[4] = {__uint_as_float(v.x), __uint_as_float(v.y),
-                                            __uint_as_float(v.z), __uint_as_float(v.w)};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            st_shared_b16(ucol + sw128_offset(c0 + p * 32 + q * 4 + e, uchk),
-                                          f2h_bits(w[e] * fu));
-                    }
-                }
+                for (int c = 0; c < 4; ++c)
+                    st_shared_v4(urow_img + ((c ^ ((i >> 1) & 3)) << 4), f2h2_bits(u[8 * c] * fu, u[8 * c + 1] * fu),
+                                 f2h2_bits(u[8 * c + 2] * fu, u[8 * c + 3] * fu),
+                                 f2h2_bits(u[8 * c + 4] * fu, u[8 * c + 5] * fu),
+                                 f2h2_bits(u[8 * c + 6] * fu, u[8 * c + 7] * fu));
                 if (i == 0 && set == 0) {
                     m->dsx[lc & 1][0] = sK;
                     m->dsx[lc & 1][1] = sU;
@@ -997,8 +988,9 @@ chain_kernel(const uint8_t *__restrict__ recs, const float *h0, float *fin, floa
     } else if (warp == K::kIssuer) {
         // ======================================================= MMA issuer ====
         if (lane == 0) {
-            const uint64_t d_sb = sw128_kmajor_desc(sbase + K::SB);
-            const uint64_t d_ub = sw128_kmajor_desc(sbase + K::UB);
+            // MN-major images: 8-row K groups 512 bytes apart, 16 K rows per MMA
+            const uint64_t d_sb = sw64_mnmajor_desc(sbase + K::SB, 8192, 512);
+            const uint64_t d_ub = sw64_mnmajor_desc(sbase + K::UB, 8192, 512);
             for (int lc = 0; lc < nl; ++lc) {
                 if (*abort_flag) break;
                 const uint32_t s = lc & 1, sph = (lc >> 1) & 1;
@@ -1018,7 +1010,7 @@ chain_kernel(const uint8_t *__restrict__ recs, const float *h0, float *fin, floa
 #pragma unroll
                 for (int k = 0; k < 8; ++k)
                     mma_f16_ss(tmem + K::TD1 + b * NB, d_a1 + (((k >> 2) * 16384 + (k & 3) * 32) >> 4),
-                               d_sb + (((k >> 2) * (NB * 128) + (k & 3) * 32) >> 4), K::IDESC, k != 0);
+                               d_sb + ((k * 1024) >> 4), K::IDESC, k != 0);
                 mma_commit(&m->bar1);
                 mma_commit(&m->empty_a1[s]);
                 if (!mbar_wait_sleep(&m->full_kp[b], bph)) { fail(ERR_TIMEOUT_TMA); break; }
@@ -1028,11 +1020,11 @@ chain_kernel(const uint8_t *__restrict__ recs, const float *h0, float *fin, floa
                 const uint64_t d_a4 = sw128_kmajor_desc(sbase + K::A4 + b * 16384);
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
-                    mma_f16_ss(tmem + K::TD2, d_kh + ((k * 32) >> 4), d_ub + ((k * 32) >> 4), K::IDESC, k != 0);
+                    mma_f16_ss(tmem + K::TD2, d_kh + ((k * 32) >> 4), d_ub + ((k * 1024) >> 4), K::IDESC, k != 0);
                 mma_commit(&m->bar2);
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
-                    mma_f16_ss(tmem + K::TD4 + b * NB, d_a4 + ((k * 32) >> 4), d_ub + ((k * 32) >> 4), K::IDESC,
+                    mma_f16_ss(tmem + K::TD4 + b * NB, d_a4 + ((k * 32) >> 4), d_ub + ((k * 1024) >> 4), K::IDESC,
                                k != 0);
                 mma_commit(&m->bar4[b]);
                 mma_commit(&m->empty_kp[b]);

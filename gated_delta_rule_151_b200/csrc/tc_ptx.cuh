@@ -293,6 +293,21 @@ __device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t addr) {
     return d;
 }
 
+// Shared-memory matrix descriptor for an MN-major 16-bit operand in the
+// 64-byte swizzled canonical layout: rows of 64 bytes (32 elements along M or
+// N), one row per K index, 16-byte chunks XOR-swizzled by (row / 2) % 4;
+// `sbo` is the byte distance between groups of 8 rows along K, `lbo` the
+// distance between 32-element blocks along M/N (unused for 32 elements).
+__device__ __forceinline__ uint64_t sw64_mnmajor_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+    uint64_t d = 0;
+    d |= (uint64_t)((addr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1u << 46;                       // descriptor version (sm_100)
+    d |= (uint64_t)4u << 61;                       // layout: 64-byte swizzle
+    return d;
+}
+
 // Instruction descriptor: fp32 accumulate, K-major A and B.
 // ab_format: 1 = bf16, 2 = tf32.
 __host__ __device__ constexpr uint32_t make_idesc(uint32_t ab_format, uint32_t M, uint32_t N) {
