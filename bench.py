@@ -173,7 +173,13 @@ def split_launches(inp):
     max_chunks = -(-inp.total_T // 64)
     window = max(1, min(max_chunks, (1 << 30) // (chains * 90640)))
     windows = -(-max_chunks // window)
-    pieces = min(4, max(1, max_chunks // 32)) if windows == 1 else 1   # pipelined pieces
+    pieces = 1
+    if windows == 1:   # pipelined pieces of 12, 16, 21, 27, ... chunks (1.3x growth)
+        pieces, c, size = 0, 0, 12
+        while c < max_chunks and pieces < 32:
+            c = max_chunks if pieces + 1 == 32 else min(c + size, max_chunks)
+            pieces += 1
+            size = (size * 13 + 9) // 10
     return 2 * windows * pieces
 
 

@@ -7,7 +7,36 @@
 
 #include "gdr.h"
 
+#include <mutex>
+#include <vector>
+
 namespace gdr {
+
+// cudaFuncSetAttribute(MaxDynamicSharedMemorySize) only when a kernel needs
+// more than it was last given on this device: the call costs host time on
+// every launch otherwise, and launches of short kernels are host-bound.
+inline cudaError_t ensure_dynamic_smem(const void *fn, int bytes) {
+    struct Entry {
+        const void *fn;
+        int dev;
+        int bytes;
+    };
+    static std::mutex mu;
+    static std::vector<Entry> done;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lock(mu);
+    Entry *hit = nullptr;
+    for (auto &d : done)
+        if (d.fn == fn && d.dev == dev) hit = &d;
+    if (hit != nullptr && hit->bytes >= bytes) return cudaSuccess;
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return e;
+    if (hit != nullptr) hit->bytes = bytes;
+    else done.push_back(Entry{fn, dev, bytes});
+    return cudaSuccess;
+}
 
 // Log-gates are clamped at this value per token: alpha >= e^-20 ~ 2e-9, so
 // every exponent difference the chunked form takes stays finite.

@@ -297,8 +297,7 @@ cudaError_t launch_multi_dk(const void *q, const void *k, const void *v, const f
     const size_t smem = sizeof(float) * (size_t)T * (2 * DK + DV + (CHANNEL ? DK : 1) + 1);
     auto kern = decode_multi_kernel<DK, CHANNEL, IoT>;
     if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)smem);
+        cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void *>(kern), (int)smem);
         if (e != cudaSuccess) return e;
     }
     const unsigned blocks = (unsigned)((size_t)N * H);

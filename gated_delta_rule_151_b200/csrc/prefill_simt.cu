@@ -251,8 +251,7 @@ cudaError_t launch_typed(const void *q, const void *k, const void *v, const floa
     const int nslabs = (DV + VS - 1) / VS;
     const SimtLayout L(DK, VS);
     auto kern = prefill_simt_kernel<CHANNEL, IoT>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)L.total);
+    cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void *>(kern), (int)L.total);
     if (e != cudaSuccess) return e;
     const size_t blocks = (size_t)nslabs * H * num_seqs;
     if (blocks == 0) return cudaSuccess;

@@ -1505,6 +1505,23 @@ struct SplitPlan {
     size_t state_off = 0, rec_off = 0, bytes = 0;
 };
 
+// Pipeline pieces of one window: the prep kernel of piece k + 1 runs beside
+// the chain kernel of piece k, and on the SMs the chain leaves free a chunk's
+// prep takes about 3/4 of a chunk's chain step, so each piece may be 1.3 times
+// the one before: 12, 16, 21, 27, 35, ... chunks, the last one the remainder.
+// Writes the piece boundaries (count + 1 of them) and returns the count.
+constexpr int kMaxPieces = 32;
+int piece_schedule(int max_chunks, int *bounds) {
+    int n = 0, c = 0, size = 12;
+    bounds[0] = 0;
+    while (c < max_chunks && n < kMaxPieces) {
+        c = (n + 1 == kMaxPieces) ? max_chunks : std::min(c + size, max_chunks);
+        bounds[++n] = c;
+        size = (size * 13 + 9) / 10;
+    }
+    return n;
+}
+
 bool make_split_plan(int num_seqs, int total_T, int H, SplitPlan &p) {
     const long long chains = (long long)num_seqs * H;
     if (chains < 1 || chains > kSplitMaxChains || total_T <= 0) return false;
@@ -1514,7 +1531,8 @@ bool make_split_plan(int num_seqs, int total_T, int H, SplitPlan &p) {
     const size_t fit = kMaxRecordBytes / per;
     p.window = (int)(fit < 1 ? 1 : (fit < (size_t)p.max_chunks ? fit : (size_t)p.max_chunks));
     p.windows = (p.max_chunks + p.window - 1) / p.window;
-    p.pieces = p.windows == 1 ? std::min(4, std::max(1, p.max_chunks / 32)) : 1;
+    int bounds[kMaxPieces + 1];
+    p.pieces = p.windows == 1 ? piece_schedule(p.max_chunks, bounds) : 1;
     const size_t state =
         (p.windows > 1 || p.pieces > 1) ? (size_t)p.chains * D * D * sizeof(float) : 0;
     p.state_off = kHeaderBytes;
@@ -1563,7 +1581,7 @@ cudaError_t launch_chain(bool channel, int chains, const uint8_t *recs, const fl
                          int c1, __nv_bfloat16 *o, uint32_t *err, cudaStream_t stream) {
     using K = Chain<NB>;
     auto kern = channel ? chain_kernel<true, NB> : chain_kernel<false, NB>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)K::SMEM);
+    cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void *>(kern), (int)K::SMEM);
     if (e != cudaSuccess) return e;
     kern<<<(unsigned)(chains * (D / NB)), K::kThreads, K::SMEM, stream>>>(
         recs, h0, fin, state, cu, num_seqs, total_T, H, c0, c1, o, err);
@@ -1592,7 +1610,7 @@ cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, co
         !make_map(&mv, v, total_T, H))
         return cudaErrorInvalidValue;
     auto prep = channel ? prep_kernel<true> : prep_kernel<false>;
-    e = cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PREP_SMEM);
+    e = ensure_dynamic_smem(reinterpret_cast<const void *>(prep), (int)PREP_SMEM);
     if (e != cudaSuccess) return e;
     float *state = (p.windows > 1 || p.pieces > 1) ? reinterpret_cast<float *>(ws + p.state_off) : nullptr;
     uint8_t *recs = ws + p.rec_off;
@@ -1601,7 +1619,7 @@ cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, co
     // share the chain work; otherwise one CTA per chain, transposed form.
     const bool dv_split = p.chains * 4 <= 148;
     auto chain_t = channel ? chain_t_kernel<true> : chain_t_kernel<false>;
-    e = cudaFuncSetAttribute(chain_t, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TSMEM);
+    e = ensure_dynamic_smem(reinterpret_cast<const void *>(chain_t), (int)TSMEM);
     if (e != cudaSuccess) return e;
     auto run_chain = [&](int c0, int c1, const uint8_t *r, cudaStream_t st) {
         if (dv_split)
@@ -1623,20 +1641,13 @@ cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, co
         Helpers *hs = nullptr;
         e = get_helpers(&hs);
         if (e != cudaSuccess) return e;
-        // a short first piece: only its prep runs before any chain work
-        const int first = std::min(8, p.max_chunks);
-        const int per = (p.max_chunks - first + p.pieces - 2) / (p.pieces - 1);
-        auto piece = [&](int k, int &c0, int &c1) {
-            c0 = k == 0 ? 0 : first + (k - 1) * per;
-            c1 = std::min(k == 0 ? first : c0 + per, p.max_chunks);
-        };
+        int bounds[kMaxPieces + 1];
+        piece_schedule(p.max_chunks, bounds);
         e = cudaEventRecord(hs->fork, stream);
         if (e == cudaSuccess) e = cudaStreamWaitEvent(hs->prep_s, hs->fork, 0);
         if (e == cudaSuccess) e = cudaStreamWaitEvent(hs->chain_s, hs->fork, 0);
         for (int k = 0; k < p.pieces && e == cudaSuccess; ++k) {
-            int c0, c1;
-            piece(k, c0, c1);
-            if (c0 >= c1) break;
+            const int c0 = bounds[k], c1 = bounds[k + 1];
             uint8_t *r = recs + (size_t)c0 * p.chains * REC_BYTES;
             e = run_prep(c0, c1, r, hs->prep_s);
             if (e == cudaSuccess) e = cudaEventRecord(hs->prep_done, hs->prep_s);

@@ -731,7 +731,7 @@ cudaError_t launch_prefill_tcgen05(const void *q, const void *k, const void *v, 
         !make_map(&mv, v, total_T, H))
         return cudaErrorInvalidValue;
     auto kern = channel ? prefill_tc_kernel<true> : prefill_tc_kernel<false>;
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    e = ensure_dynamic_smem(reinterpret_cast<const void *>(kern), (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
     const size_t blocks = (size_t)num_seqs * H;
     if (blocks > 0x7fffffffull) return cudaErrorInvalidConfiguration;
