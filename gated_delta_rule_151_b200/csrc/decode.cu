@@ -42,6 +42,59 @@ __device__ __forceinline__ void load4(const __nv_bfloat16 *p, float out[4]) {
     out[0] = a.x; out[1] = a.y; out[2] = b.x; out[3] = b.y;
 }
 
+// A lane's 16 columns of a row, or of k, q or a, are 8 column pairs: pair
+// 2m holds columns 4(p + LPR m) + {0, 1}, pair 2m + 1 columns + {2, 3}, with
+// p the lane's place in its row group.  The arithmetic runs on the packed
+// fp32x2 units, two columns per instruction.
+__device__ __forceinline__ void split4(float4 x, float2 &lo, float2 &hi) {
+    lo = make_float2(x.x, x.y);
+    hi = make_float2(x.z, x.w);
+}
+
+__device__ __forceinline__ float4 join4(float2 lo, float2 hi) {
+    return make_float4(lo.x, lo.y, hi.x, hi.y);
+}
+
+template <int LPR>
+__device__ __forceinline__ float group_sum(float x) {
+#pragma unroll
+    for (int off = LPR / 2; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+    return x;
+}
+
+// kappa = k . q over the row group.
+template <int LPR>
+__device__ __forceinline__ float head_kappa(const float2 (&k)[8], const float2 (&q)[8]) {
+    float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc = __ffma2_rn(k[j], q[j], acc);
+    return group_sum<LPR>(acc.x + acc.y);
+}
+
+// One token applied to one state row (the lane's 16 columns in e); returns
+// o_r.  Every decode kernel goes through this routine, so several tokens in
+// one pass give bit for bit the results of as many single steps.
+template <int LPR, bool CHANNEL>
+__device__ __forceinline__ float row_token(float2 (&e)[8], const float2 (&k)[8],
+                                           const float2 (&q)[8],
+                                           const float2 (&a)[CHANNEL ? 8 : 1], float b, float vr,
+                                           float kappa) {
+    float2 x2 = make_float2(0.f, 0.f), y2 = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        e[j] = __fmul2_rn(e[j], CHANNEL ? a[j] : a[0]);
+        x2 = __ffma2_rn(e[j], k[j], x2);
+        y2 = __ffma2_rn(e[j], q[j], y2);
+    }
+    const float x = group_sum<LPR>(x2.x + x2.y);
+    const float y = group_sum<LPR>(y2.x + y2.y);
+    const float u = b * (vr - x);
+    const float2 u2 = make_float2(u, u);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) e[j] = __ffma2_rn(u2, k[j], e[j]);
+    return fmaf(u, kappa, y);
+}
+
 template <int DK, bool CHANNEL, typename IoT>
 __global__ void __launch_bounds__(kDecodeThreads, 2)
 decode_step_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k,
@@ -62,79 +115,55 @@ decode_step_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k,
     float4 *S = reinterpret_cast<float4 *>(state + nh * (size_t)DV * DK);
 
     // Issue all state loads of this thread first.
-    float4 s[MAXP][4];
+    float2 s[MAXP][8];
 #pragma unroll
     for (int pp = 0; pp < MAXP; ++pp) {
         const int r = pp * RP + rg;
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
-            if (r < DV)
-                s[pp][m] = __ldcs(S + (size_t)r * (DK / 4) + p + LPR * m);
-            else
-                s[pp][m] = make_float4(0.f, 0.f, 0.f, 0.f);
+            const float4 x = (r < DV) ? __ldcs(S + (size_t)r * (DK / 4) + p + LPR * m)
+                                      : make_float4(0.f, 0.f, 0.f, 0.f);
+            split4(x, s[pp][2 * m], s[pp][2 * m + 1]);
         }
     }
 
-    float kf[16], qf[16];
+    float2 kf[8], qf[8], af[CHANNEL ? 8 : 1];
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
         const int col = 4 * (p + LPR * m);
-        load4(k + qh * DK + col, kf + 4 * m);
-        load4(q + qh * DK + col, qf + 4 * m);
+        float t[4];
+        load4(k + qh * DK + col, t);
+        kf[2 * m] = make_float2(t[0], t[1]);
+        kf[2 * m + 1] = make_float2(t[2], t[3]);
+        load4(q + qh * DK + col, t);
+        qf[2 * m] = make_float2(t[0], t[1]);
+        qf[2 * m + 1] = make_float2(t[2], t[3]);
     }
-    float af[CHANNEL ? 16 : 1];
     if constexpr (CHANNEL) {
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
             const int col = 4 * (p + LPR * m);
-            float4 gg = *reinterpret_cast<const float4 *>(g + nh * DK + col);
-            af[4 * m + 0] = __expf(clamp_log_gate(gg.x));
-            af[4 * m + 1] = __expf(clamp_log_gate(gg.y));
-            af[4 * m + 2] = __expf(clamp_log_gate(gg.z));
-            af[4 * m + 3] = __expf(clamp_log_gate(gg.w));
+            const float4 gg = *reinterpret_cast<const float4 *>(g + nh * DK + col);
+            af[2 * m] = make_float2(__expf(clamp_log_gate(gg.x)), __expf(clamp_log_gate(gg.y)));
+            af[2 * m + 1] = make_float2(__expf(clamp_log_gate(gg.z)), __expf(clamp_log_gate(gg.w)));
         }
     } else {
-        af[0] = __expf(clamp_log_gate(g[nh]));
+        const float a = __expf(clamp_log_gate(g[nh]));
+        af[0] = make_float2(a, a);
     }
     const float b = beta[nh];
-
-    // kappa = k . q, shared by every row of the head.
-    float kappa = 0.f;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) kappa = fmaf(kf[i], qf[i], kappa);
-#pragma unroll
-    for (int off = LPR / 2; off > 0; off >>= 1) kappa += __shfl_xor_sync(0xffffffffu, kappa, off);
+    const float kappa = head_kappa<LPR>(kf, qf);
 
 #pragma unroll
     for (int pp = 0; pp < MAXP; ++pp) {
         const int r = pp * RP + rg;
-        float x = 0.f, y = 0.f;
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-            float *e = reinterpret_cast<float *>(&s[pp][m]);
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const float a = CHANNEL ? af[4 * m + c] : af[0];
-                e[c] *= a;
-                x = fmaf(e[c], kf[4 * m + c], x);
-                y = fmaf(e[c], qf[4 * m + c], y);
-            }
-        }
-#pragma unroll
-        for (int off = LPR / 2; off > 0; off >>= 1) {
-            x += __shfl_xor_sync(0xffffffffu, x, off);
-            y += __shfl_xor_sync(0xffffffffu, y, off);
-        }
+        const float vr = (r < DV) ? to_f32(v[nh * DV + r]) : 0.f;
+        const float out = row_token<LPR, CHANNEL>(s[pp], kf, qf, af, b, vr, kappa);
         if (r < DV) {
-            const float u = b * (to_f32(v[nh * DV + r]) - x);
 #pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                float *e = reinterpret_cast<float *>(&s[pp][m]);
-#pragma unroll
-                for (int c = 0; c < 4; ++c) e[c] = fmaf(u, kf[4 * m + c], e[c]);
-                __stcs(S + (size_t)r * (DK / 4) + p + LPR * m, s[pp][m]);
-            }
-            if (p == 0) store_io(o + nh * DV + r, fmaf(u, kappa, y));
+            for (int m = 0; m < 4; ++m)
+                __stcs(S + (size_t)r * (DK / 4) + p + LPR * m, join4(s[pp][2 * m], s[pp][2 * m + 1]));
+            if (p == 0) store_io(o + nh * DV + r, out);
         }
     }
 }
@@ -167,143 +196,288 @@ cudaError_t launch_mode(const void *q, const void *k, const void *v, const float
 // T consecutive tokens of each sequence in one pass over the state (draft
 // verification in speculative decoding): every state row is read once, the
 // T updates are applied in registers token after token, and the row is
-// written once, so the state traffic per token falls by T.  The T tokens'
-// q/k/v/gates/beta of the (sequence, head) are staged in shared memory while
-// the state loads are in flight.  Optionally the state after every token is
-// stored to a snapshot buffer, from which a caller rolls back to the last
-// accepted draft token.
+// written once, so the state traffic per token falls by T.  Optionally the
+// state after every token is stored to a snapshot buffer, from which a
+// caller rolls back to the last accepted draft token.
+//
+// With T updates per row the arithmetic is no longer small next to the
+// bytes, so the kernel overlaps the two: it is persistent, and each CTA walks
+// over slabs of RB state rows of one (sequence, head) -- RB * d_k * 4
+// contiguous bytes -- with a ring of kMultiStages shared-memory stages that
+// cp.async fills kMultiStages - 1 slabs ahead.  A stage holds the slab's
+// state rows and the T tokens' k, q, the slab's v entries, the gates and
+// beta.  Data in flight costs no registers, so a few CTAs per SM keep the
+// HBM pipe full while the arithmetic of the current slab runs.
+constexpr int kMultiThreads = 128;
+constexpr int kMultiStages = 3;
+
+template <int DK>
+struct MultiShape {
+    static constexpr int LPR = DK / 16;                       // lanes per row
+    static constexpr int RP = kMultiThreads / LPR;            // rows per pass
+    static constexpr int MAXP = (LPR / 2 > 0) ? LPR / 2 : 1;  // passes per slab
+    static constexpr int RB = RP * MAXP;                      // rows per slab
+};
+
+__host__ __device__ constexpr int align16(int x) { return (x + 15) & ~15; }
+
+// Byte offsets inside a stage, the stage stride, and the fp32 operand
+// buffer (k, q converted once per slab; exp of the gates) after the ring.
+struct MultiLayout {
+    int st, kq, v, g, b, stage, conv_kq, conv_a, total;
+};
+
+__host__ __device__ inline MultiLayout multi_layout(int T, int DK, int RB, int io_bytes, int GD) {
+    MultiLayout L;
+    L.st = 0;
+    L.kq = RB * DK * 4;
+    L.v = L.kq + align16(T * 2 * DK * io_bytes);
+    L.g = L.v + align16(T * RB * io_bytes);
+    L.b = L.g + align16(T * GD * 4);
+    L.stage = (L.b + T * 4 + 127) & ~127;
+    L.conv_kq = kMultiStages * L.stage;
+    L.conv_a = L.conv_kq + T * 2 * DK * 4;
+    L.total = L.conv_a + align16(T * GD * 4);
+    return L;
+}
+
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(
+                     static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+                 "l"(src)
+                 : "memory");
+}
+
+__device__ __forceinline__ void cp_async4(void *dst, const void *src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(
+                     static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+                 "l"(src)
+                 : "memory");
+}
+
+__device__ __forceinline__ void cp_async_commit() {
+    asm volatile("cp.async.commit_group;\n" ::: "memory");
+}
+
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
+}
+
+// Slab s = (sequence, head) * nblk + row block.
+struct Slab {
+    size_t nh, n;
+    int h, r0, rows;
+};
+
+__device__ __forceinline__ Slab slab_of(long long s, int nblk, int H, int RB, int DV) {
+    Slab x;
+    x.nh = (size_t)(s / nblk);
+    x.r0 = (int)(s % nblk) * RB;
+    x.n = x.nh / H;
+    x.h = (int)(x.nh % H);
+    x.rows = min(RB, DV - x.r0);
+    return x;
+}
+
+// Start the copies of one slab into a stage (every thread takes a share).
+// All sources are 16-byte aligned (the C ABI checks the base pointers; rows
+// are multiples of 16 elements), except scalar gates and beta: 4-byte copies.
 template <int DK, bool CHANNEL, typename IoT>
-__global__ void __launch_bounds__(kDecodeThreads, 2)
+__device__ __forceinline__ void issue_slab(uint8_t *stg, const MultiLayout &L, const Slab &x,
+                                           const IoT *q, const IoT *k, const IoT *v,
+                                           const float *g, const float *beta, const float *state,
+                                           int T, int Hqk, int H, int DV) {
+    constexpr int RB = MultiShape<DK>::RB;
+    const int tid = threadIdx.x;
+    const size_t hq = (size_t)(x.h / (H / Hqk));
+    const float *src = state + (x.nh * DV + x.r0) * DK;
+    const int ns = x.rows * DK / 4;
+    for (int i = tid; i < ns; i += kMultiThreads) cp_async16(stg + L.st + 16 * i, src + 4 * i);
+    constexpr int KG = DK * (int)sizeof(IoT) / 16;     // 16-byte pieces of a k or q row
+    for (int i = tid; i < T * 2 * KG; i += kMultiThreads) {
+        const int t = i / (2 * KG), w = (i / KG) % 2, c = i % KG;
+        const IoT *row = (w == 0 ? k : q) + ((x.n * T + t) * Hqk + hq) * DK;
+        cp_async16(stg + L.kq + (2 * t + w) * DK * (int)sizeof(IoT) + 16 * c,
+                   reinterpret_cast<const uint8_t *>(row) + 16 * c);
+    }
+    const int VG = x.rows * (int)sizeof(IoT) / 16;
+    for (int i = tid; i < T * VG; i += kMultiThreads) {
+        const int t = i / VG, c = i % VG;
+        const IoT *row = v + ((x.n * T + t) * H + x.h) * DV + x.r0;
+        cp_async16(stg + L.v + t * RB * (int)sizeof(IoT) + 16 * c,
+                   reinterpret_cast<const uint8_t *>(row) + 16 * c);
+    }
+    if constexpr (CHANNEL) {
+        for (int i = tid; i < T * (DK / 4); i += kMultiThreads) {
+            const int t = i / (DK / 4), c = i % (DK / 4);
+            cp_async16(stg + L.g + (t * DK + 4 * c) * 4, g + ((x.n * T + t) * H + x.h) * DK + 4 * c);
+        }
+    } else {
+        for (int t = tid; t < T; t += kMultiThreads)
+            cp_async4(stg + L.g + 4 * t, g + (x.n * T + t) * H + x.h);
+    }
+    for (int t = tid; t < T; t += kMultiThreads)
+        cp_async4(stg + L.b + 4 * t, beta + (x.n * T + t) * H + x.h);
+}
+
+template <int DK, bool CHANNEL, typename IoT>
+__global__ void __launch_bounds__(kMultiThreads, 3)
 decode_multi_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k,
                     const IoT *__restrict__ v, const float *__restrict__ g,
                     const float *__restrict__ beta, float *__restrict__ state, int T, int Hqk,
-                    int H, int DV, IoT *__restrict__ o, float *__restrict__ snap) {
-    constexpr int LPR = DK / 16;
-    constexpr int RP = kDecodeThreads / LPR;
-    constexpr int MAXP = (LPR / 2 > 0) ? LPR / 2 : 1;
+                    int H, int DV, int nblk, long long slabs, IoT *__restrict__ o,
+                    float *__restrict__ snap) {
+    using Sh = MultiShape<DK>;
+    constexpr int LPR = Sh::LPR, RP = Sh::RP, MAXP = Sh::MAXP, RB = Sh::RB;
     constexpr int GD = CHANNEL ? DK : 1;
-    extern __shared__ float sh[];
-
-    const size_t nh = blockIdx.x;                 // (sequence, value head)
-    const size_t n = nh / H, h = nh % H;
-    const size_t hq = h / (H / Hqk);
+    extern __shared__ __align__(128) uint8_t smem[];
+    const MultiLayout L = multi_layout(T, DK, RB, (int)sizeof(IoT), GD);
     const int tid = threadIdx.x;
     const int p = tid % LPR;
     const int rg = tid / LPR;
+    const long long first = blockIdx.x, stride = gridDim.x;
+    const int mine = slabs > first ? (int)((slabs - 1 - first) / stride + 1) : 0;
+    float *kqf = reinterpret_cast<float *>(smem + L.conv_kq);   // [T][2][DK]  k, q
+    float *af = reinterpret_cast<float *>(smem + L.conv_a);     // [T][GD]     exp(g)
 
-    float4 *S = reinterpret_cast<float4 *>(state + nh * (size_t)DV * DK);
-    float4 s[MAXP][4];
 #pragma unroll
-    for (int pp = 0; pp < MAXP; ++pp) {
-        const int r = pp * RP + rg;
-#pragma unroll
-        for (int m = 0; m < 4; ++m)
-            s[pp][m] = (r < DV) ? __ldcs(S + (size_t)r * (DK / 4) + p + LPR * m)
-                                : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j = 0; j < kMultiStages - 1; ++j) {
+        if (j < mine)
+            issue_slab<DK, CHANNEL, IoT>(smem + j * L.stage, L,
+                                         slab_of(first + j * stride, nblk, H, RB, DV), q, k, v,
+                                         g, beta, state, T, Hqk, H, DV);
+        cp_async_commit();
     }
 
-    float *kq = sh;                       // [T][2][DK]  k, q
-    float *vs = kq + (size_t)T * 2 * DK;  // [T][DV]
-    float *as = vs + (size_t)T * DV;      // [T][GD]     exp(g)
-    float *bs = as + (size_t)T * GD;      // [T]
-    for (int idx = tid; idx < T * DK; idx += kDecodeThreads) {
-        const int t = idx / DK, c = idx % DK;
-        const size_t qrow = (n * T + t) * Hqk + hq;
-        kq[(2 * t) * DK + c] = to_f32(k[qrow * DK + c]);
-        kq[(2 * t + 1) * DK + c] = to_f32(q[qrow * DK + c]);
-    }
-    for (int idx = tid; idx < T * DV; idx += kDecodeThreads) {
-        const int t = idx / DV, r = idx % DV;
-        vs[idx] = to_f32(v[((n * T + t) * H + h) * DV + r]);
-    }
-    for (int idx = tid; idx < T * GD; idx += kDecodeThreads) {
-        const int t = idx / GD, c = idx % GD;
-        as[idx] = __expf(clamp_log_gate(g[((n * T + t) * H + h) * GD + c]));
-    }
-    for (int t = tid; t < T; t += kDecodeThreads) bs[t] = beta[(n * T + t) * H + h];
-    __syncthreads();
+    for (int j = 0; j < mine; ++j) {
+        const int jn = j + kMultiStages - 1;
+        if (jn < mine)
+            issue_slab<DK, CHANNEL, IoT>(smem + (jn % kMultiStages) * L.stage, L,
+                                         slab_of(first + jn * stride, nblk, H, RB, DV), q, k, v,
+                                         g, beta, state, T, Hqk, H, DV);
+        cp_async_commit();
+        cp_async_wait<kMultiStages - 1>();   // slab j has landed (groups complete in order)
+        __syncthreads();
 
-    for (int t = 0; t < T; ++t) {
-        float kf[16], qf[16], af[CHANNEL ? 16 : 1];
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-            const int col = 4 * (p + LPR * m);
-            const float4 kk = *reinterpret_cast<const float4 *>(kq + (2 * t) * DK + col);
-            const float4 qq = *reinterpret_cast<const float4 *>(kq + (2 * t + 1) * DK + col);
-            kf[4 * m] = kk.x; kf[4 * m + 1] = kk.y; kf[4 * m + 2] = kk.z; kf[4 * m + 3] = kk.w;
-            qf[4 * m] = qq.x; qf[4 * m + 1] = qq.y; qf[4 * m + 2] = qq.z; qf[4 * m + 3] = qq.w;
-            if constexpr (CHANNEL) {
-                const float4 aa = *reinterpret_cast<const float4 *>(as + t * DK + col);
-                af[4 * m] = aa.x; af[4 * m + 1] = aa.y; af[4 * m + 2] = aa.z; af[4 * m + 3] = aa.w;
-            }
-        }
-        if constexpr (!CHANNEL) af[0] = as[t];
-        const float b = bs[t];
-        float kappa = 0.f;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) kappa = fmaf(kf[i], qf[i], kappa);
-#pragma unroll
-        for (int off = LPR / 2; off > 0; off >>= 1) kappa += __shfl_xor_sync(0xffffffffu, kappa, off);
+        const uint8_t *stg = smem + (j % kMultiStages) * L.stage;
+        const Slab x = slab_of(first + j * stride, nblk, H, RB, DV);
+        const IoT *kq_raw = reinterpret_cast<const IoT *>(stg + L.kq);
+        for (int i = tid; i < T * 2 * DK; i += kMultiThreads) kqf[i] = to_f32(kq_raw[i]);
+        const float *g_raw = reinterpret_cast<const float *>(stg + L.g);
+        for (int i = tid; i < T * GD; i += kMultiThreads) af[i] = __expf(clamp_log_gate(g_raw[i]));
 
-        const size_t vrow = (n * T + t) * H + h;
+        const float4 *st4 = reinterpret_cast<const float4 *>(stg + L.st);
+        float2 s[MAXP][8];
 #pragma unroll
         for (int pp = 0; pp < MAXP; ++pp) {
-            const int r = pp * RP + rg;
-            float x = 0.f, y = 0.f;
+            const int rl = pp * RP + rg;
 #pragma unroll
             for (int m = 0; m < 4; ++m) {
-                float *e = reinterpret_cast<float *>(&s[pp][m]);
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    e[c] *= CHANNEL ? af[4 * m + c] : af[0];
-                    x = fmaf(e[c], kf[4 * m + c], x);
-                    y = fmaf(e[c], qf[4 * m + c], y);
-                }
-            }
-#pragma unroll
-            for (int off = LPR / 2; off > 0; off >>= 1) {
-                x += __shfl_xor_sync(0xffffffffu, x, off);
-                y += __shfl_xor_sync(0xffffffffu, y, off);
-            }
-            if (r < DV) {
-                const float u = b * (vs[t * DV + r] - x);
-#pragma unroll
-                for (int m = 0; m < 4; ++m) {
-                    float *e = reinterpret_cast<float *>(&s[pp][m]);
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) e[c] = fmaf(u, kf[4 * m + c], e[c]);
-                    if (snap != nullptr)
-                        __stcs(reinterpret_cast<float4 *>(snap + (vrow * DV + r) * DK) + p + LPR * m,
-                               s[pp][m]);
-                }
-                if (p == 0) store_io(o + vrow * DV + r, fmaf(u, kappa, y));
+                const float4 e4 = (rl < x.rows) ? st4[rl * (DK / 4) + p + LPR * m]
+                                                : make_float4(0.f, 0.f, 0.f, 0.f);
+                split4(e4, s[pp][2 * m], s[pp][2 * m + 1]);
             }
         }
-    }
+        __syncthreads();   // converted operands visible
+
+        const IoT *v_raw = reinterpret_cast<const IoT *>(stg + L.v);
+        const float *b_raw = reinterpret_cast<const float *>(stg + L.b);
+        for (int t = 0; t < T; ++t) {
+            float2 kf[8], qf[8], a2[CHANNEL ? 8 : 1];
 #pragma unroll
-    for (int pp = 0; pp < MAXP; ++pp) {
-        const int r = pp * RP + rg;
-        if (r < DV) {
+            for (int m = 0; m < 4; ++m) {
+                const int col = 4 * (p + LPR * m);
+                split4(*reinterpret_cast<const float4 *>(kqf + (2 * t) * DK + col), kf[2 * m],
+                       kf[2 * m + 1]);
+                split4(*reinterpret_cast<const float4 *>(kqf + (2 * t + 1) * DK + col), qf[2 * m],
+                       qf[2 * m + 1]);
+                if constexpr (CHANNEL)
+                    split4(*reinterpret_cast<const float4 *>(af + t * DK + col), a2[2 * m],
+                           a2[2 * m + 1]);
+            }
+            if constexpr (!CHANNEL) a2[0] = make_float2(af[t], af[t]);
+            const float b = b_raw[t];
+            const float kappa = head_kappa<LPR>(kf, qf);
+            const size_t vrow = (x.n * T + t) * H + x.h;
 #pragma unroll
-            for (int m = 0; m < 4; ++m) __stcs(S + (size_t)r * (DK / 4) + p + LPR * m, s[pp][m]);
+            for (int pp = 0; pp < MAXP; ++pp) {
+                const int rl = pp * RP + rg;
+                const float vr = (rl < x.rows) ? to_f32(v_raw[t * RB + rl]) : 0.f;
+                const float out = row_token<LPR, CHANNEL>(s[pp], kf, qf, a2, b, vr, kappa);
+                if (rl < x.rows) {
+                    const int r = x.r0 + rl;
+                    if (snap != nullptr) {
+#pragma unroll
+                        for (int m = 0; m < 4; ++m)
+                            __stcs(reinterpret_cast<float4 *>(snap + (vrow * DV + r) * DK) + p + LPR * m,
+                                   join4(s[pp][2 * m], s[pp][2 * m + 1]));
+                    }
+                    if (p == 0) store_io(o + vrow * DV + r, out);
+                }
+            }
         }
+        float4 *S = reinterpret_cast<float4 *>(state + (x.nh * DV + x.r0) * DK);
+#pragma unroll
+        for (int pp = 0; pp < MAXP; ++pp) {
+            const int rl = pp * RP + rg;
+            if (rl < x.rows) {
+#pragma unroll
+                for (int m = 0; m < 4; ++m)
+                    __stcs(S + (size_t)rl * (DK / 4) + p + LPR * m, join4(s[pp][2 * m], s[pp][2 * m + 1]));
+            }
+        }
+        __syncthreads();   // the stage and the operand buffer are free again
     }
+    cp_async_wait<0>();
+}
+
+// CTAs per SM the multi-token kernel reaches with a given shared memory
+// size (cached: the occupancy query costs host time on every launch).
+inline cudaError_t resident_ctas(const void *fn, int threads, int smem, int *out) {
+    struct Entry {
+        const void *fn;
+        int dev, smem, ctas;
+    };
+    static std::mutex mu;
+    static std::vector<Entry> done;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lock(mu);
+    for (auto &d : done)
+        if (d.fn == fn && d.dev == dev && d.smem == smem) {
+            *out = d.ctas;
+            return cudaSuccess;
+        }
+    int sms = 0, per = 0;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, fn, threads, smem);
+    if (e != cudaSuccess) return e;
+    if (per < 1) return cudaErrorInvalidConfiguration;
+    done.push_back(Entry{fn, dev, smem, sms * per});
+    *out = sms * per;
+    return cudaSuccess;
 }
 
 template <int DK, bool CHANNEL, typename IoT>
 cudaError_t launch_multi_dk(const void *q, const void *k, const void *v, const float *g,
                             const float *beta, float *state, int N, int T, int Hqk, int H, int DV,
                             void *o, float *snap, cudaStream_t stream) {
-    const size_t smem = sizeof(float) * (size_t)T * (2 * DK + DV + (CHANNEL ? DK : 1) + 1);
+    using Sh = MultiShape<DK>;
+    const MultiLayout L = multi_layout(T, DK, Sh::RB, (int)sizeof(IoT), CHANNEL ? DK : 1);
     auto kern = decode_multi_kernel<DK, CHANNEL, IoT>;
-    if (smem > 48 * 1024) {
-        cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void *>(kern), (int)smem);
-        if (e != cudaSuccess) return e;
-    }
-    const unsigned blocks = (unsigned)((size_t)N * H);
-    kern<<<blocks, kDecodeThreads, smem, stream>>>(
+    cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void *>(kern), L.total);
+    if (e != cudaSuccess) return e;
+    int ctas = 0;
+    e = resident_ctas(reinterpret_cast<const void *>(kern), kMultiThreads, L.total, &ctas);
+    if (e != cudaSuccess) return e;
+    const int nblk = (DV + Sh::RB - 1) / Sh::RB;
+    const long long slabs = (long long)N * H * nblk;
+    const unsigned grid = (unsigned)(slabs < ctas ? slabs : ctas);
+    kern<<<grid, kMultiThreads, L.total, stream>>>(
         static_cast<const IoT *>(q), static_cast<const IoT *>(k), static_cast<const IoT *>(v), g,
-        beta, state, T, Hqk, H, DV, static_cast<IoT *>(o), snap);
+        beta, state, T, Hqk, H, DV, nblk, slabs, static_cast<IoT *>(o), snap);
     return cudaGetLastError();
 }
 
