@@ -209,7 +209,7 @@ cudaError_t launch_mode(const void *q, const void *k, const void *v, const float
 // beta.  Data in flight costs no registers, so a few CTAs per SM keep the
 // HBM pipe full while the arithmetic of the current slab runs.
 constexpr int kMultiThreads = 128;
-constexpr int kMultiStages = 3;
+constexpr int kMultiStages = 2;
 
 template <int DK>
 struct MultiShape {
@@ -399,12 +399,18 @@ decode_multi_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k,
             if constexpr (!CHANNEL) a2[0] = make_float2(af[t], af[t]);
             const float b = b_raw[t];
             const float kappa = head_kappa<LPR>(kf, qf);
-            const size_t vrow = (x.n * T + t) * H + x.h;
+            // every row first (their dependency chains interleave), then the stores
+            float out[MAXP];
 #pragma unroll
             for (int pp = 0; pp < MAXP; ++pp) {
                 const int rl = pp * RP + rg;
                 const float vr = (rl < x.rows) ? to_f32(v_raw[t * RB + rl]) : 0.f;
-                const float out = row_token<LPR, CHANNEL>(s[pp], kf, qf, a2, b, vr, kappa);
+                out[pp] = row_token<LPR, CHANNEL>(s[pp], kf, qf, a2, b, vr, kappa);
+            }
+            const size_t vrow = (x.n * T + t) * H + x.h;
+#pragma unroll
+            for (int pp = 0; pp < MAXP; ++pp) {
+                const int rl = pp * RP + rg;
                 if (rl < x.rows) {
                     const int r = x.r0 + rl;
                     if (snap != nullptr) {
@@ -413,7 +419,7 @@ decode_multi_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k,
                             __stcs(reinterpret_cast<float4 *>(snap + (vrow * DV + r) * DK) + p + LPR * m,
                                    join4(s[pp][2 * m], s[pp][2 * m + 1]));
                     }
-                    if (p == 0) store_io(o + vrow * DV + r, out);
+                    if (p == 0) store_io(o + vrow * DV + r, out[pp]);
                 }
             }
         }
