@@ -40,6 +40,10 @@ decode_gdn/kda     256 sequences, H=32, d=128, 512 steps of one bf16 token,
                    c=0.1, h0 ~ N(0, 0.02^2) (state 512 MiB fp32)
 decode_spec_gdn    the decode_gdn tokens verified 4 at a time (128 steps of
                    4 draft tokens per sequence)
+prologue_gdn       raw prologue inputs at the gdn_prefill shape (1 x 8192
+                   tokens, H=16, d=128, bf16): x_q, x_k, x_v ~ N(0, 1), taps
+                   ~ N(0, 0.5^2), convolution state ~ N(0, 1), x_g, x_beta
+                   ~ N(0, 1), gate coefficient c=0.05 per head
 varlen_gdn         8 packed sequences, 262144 tokens, H=16, d=128, bf16,
                    scalar gate c=0.1, h0=0
 gqa_prefill        1 sequence, 8192 tokens, 16 query/key heads shared by 48
@@ -60,7 +64,10 @@ import torch
 
 BLOCK_ELEMS = 1 << 21
 
-_ID = {"q": 0, "k": 1, "v": 2, "beta": 3, "gate": 4, "h0": 5, "cuts": 6}
+_ID = {"q": 0, "k": 1, "v": 2, "beta": 3, "gate": 4, "h0": 5, "cuts": 6,
+       # raw inputs of the prologue (before the convolution and the maps)
+       "xq": 7, "xk": 8, "xv": 9, "wq": 10, "wk": 11, "wv": 12, "xg": 13, "xb": 14,
+       "conv": 15}
 
 SCALAR = "scalar"    # Gated DeltaNet: one gate per head and token
 CHANNEL = "channel"  # Kimi Delta Attention: one gate per key channel
@@ -236,12 +243,99 @@ def make_inputs(*, total_T: int, H: int, d_k: int, d_v: int | None = None,
                   gate_mode=gate_mode, io_dtype=io_dtype, meta=m)
 
 
+@dataclass
+class PrologueInputs:
+    """Raw inputs of the input-side prologue as CPU torch tensors.
+
+    xq, xk: [total_T, H_qk, d_k]; xv: [total_T, H, d_v] in ``io_dtype``;
+    wq, wk: [H_qk d_k, 4]; wv: [H d_v, 4] float32 taps (tap 3 takes the current
+    token); xg: [total_T, H] or [total_T, H, d_k] and xb: [total_T, H] float32;
+    gscale: [H] float32; conv_state: [num_seqs, 2 H_qk d_k + H d_v, 3]
+    float32 or None; cu_seqlens: int32 [num_seqs + 1].
+    """
+
+    xq: torch.Tensor
+    xk: torch.Tensor
+    xv: torch.Tensor
+    wq: torch.Tensor
+    wk: torch.Tensor
+    wv: torch.Tensor
+    xg: torch.Tensor
+    gscale: torch.Tensor
+    xb: torch.Tensor
+    conv_state: torch.Tensor | None
+    cu_seqlens: torch.Tensor
+    gate_mode: str
+    io_dtype: torch.dtype
+    meta: dict = field(default_factory=dict)
+
+    @property
+    def num_seqs(self) -> int:
+        return int(self.cu_seqlens.numel() - 1)
+
+    @property
+    def total_T(self) -> int:
+        return int(self.xq.shape[0])
+
+
+def make_prologue_inputs(*, total_T: int, H: int, d_k: int, d_v: int | None = None,
+                         H_qk: int | None = None, num_seqs: int = 1, cu_seqlens=None,
+                         gate_mode: str = SCALAR, io_dtype: torch.dtype = torch.bfloat16,
+                         c: float = 0.05, tap_std: float = 0.5, state_std: float = 1.0,
+                         seed: int = 0, meta: dict | None = None) -> PrologueInputs:
+    """Draw raw prologue inputs: standard normals (taps and state scaled by
+    their standard deviations), rounded once to the I/O precision."""
+    d_v = d_k if d_v is None else d_v
+    H_qk = H if H_qk is None else H_qk
+    if H_qk < 1 or H % H_qk:
+        raise ValueError("H_qk must divide H")
+    if cu_seqlens is None:
+        if num_seqs < 1 or total_T % num_seqs:
+            raise ValueError("total_T must divide into num_seqs equal sequences")
+        cu = np.arange(num_seqs + 1, dtype=np.int64) * (total_T // num_seqs)
+    else:
+        cu = np.asarray(cu_seqlens, dtype=np.int64)
+        num_seqs = len(cu) - 1
+        if cu[0] != 0 or cu[-1] != total_T or np.any(np.diff(cu) < 0):
+            raise ValueError("cu_seqlens must run from 0 to total_T, non-decreasing")
+    ident = lambda x: x  # noqa: E731
+    xq = _fill(seed, "xq", (total_T, H_qk, d_k), ident, np.float32)
+    xk = _fill(seed, "xk", (total_T, H_qk, d_k), ident, np.float32)
+    xv = _fill(seed, "xv", (total_T, H, d_v), ident, np.float32)
+    taps = lambda x: x * tap_std  # noqa: E731
+    wq = _fill(seed, "wq", (H_qk * d_k, 4), taps, np.float32)
+    wk = _fill(seed, "wk", (H_qk * d_k, 4), taps, np.float32)
+    wv = _fill(seed, "wv", (H * d_v, 4), taps, np.float32)
+    gshape = (total_T, H) if gate_mode == SCALAR else (total_T, H, d_k)
+    xg = _fill(seed, "xg", gshape, ident, np.float32)
+    xb = _fill(seed, "xb", (total_T, H), ident, np.float32)
+    conv = None
+    if state_std > 0.0:
+        conv = torch.from_numpy(_fill(seed, "conv", (num_seqs, 2 * H_qk * d_k + H * d_v, 3),
+                                      lambda x: x * state_std, np.float32))
+
+    def io(a):
+        t = torch.from_numpy(a)
+        return t.to(io_dtype) if io_dtype != torch.float32 else t
+
+    m = {"seed": seed, "c": c, "tap_std": tap_std, "state_std": state_std,
+         "gate_mode": gate_mode, "io_dtype": str(io_dtype).replace("torch.", "")}
+    if meta:
+        m.update(meta)
+    return PrologueInputs(xq=io(xq), xk=io(xk), xv=io(xv), wq=torch.from_numpy(wq),
+                          wk=torch.from_numpy(wk), wv=torch.from_numpy(wv),
+                          xg=torch.from_numpy(xg), gscale=torch.full((H,), c, dtype=torch.float32),
+                          xb=torch.from_numpy(xb), conv_state=conv,
+                          cu_seqlens=torch.from_numpy(cu.astype(np.int32)),
+                          gate_mode=gate_mode, io_dtype=io_dtype, meta=m)
+
+
 # ---------------------------------------------------------------------------
 # The benchmark workloads.
 # ---------------------------------------------------------------------------
 
 WORKLOADS = ("tiny_gdn", "gdn_prefill", "kda_prefill", "decode_gdn",
-             "decode_kda", "varlen_gdn", "gqa_prefill", "decode_spec_gdn")
+             "decode_kda", "varlen_gdn", "gqa_prefill", "decode_spec_gdn", "prologue_gdn")
 
 SPEC_DRAFT = 4   # tokens verified per sequence per step in decode_spec_gdn
 
@@ -283,6 +377,15 @@ def workload(name: str, seed: int = 0) -> Inputs:
                            gate_mode=SCALAR, io_dtype=torch.bfloat16, c=0.1,
                            seed=seed, meta={"workload": name})
     raise KeyError(name)
+
+
+def prologue_workload(name: str = "prologue_gdn", seed: int = 0) -> PrologueInputs:
+    """Raw prologue inputs at the gdn_prefill shape (module docstring table)."""
+    if name != "prologue_gdn":
+        raise KeyError(name)
+    return make_prologue_inputs(total_T=8192, H=16, d_k=128, num_seqs=1, gate_mode=SCALAR,
+                                io_dtype=torch.bfloat16, c=0.05, tap_std=0.5, state_std=1.0,
+                                seed=seed, meta={"workload": name})
 
 
 def decode_view(x: torch.Tensor, num_seqs: int) -> torch.Tensor:

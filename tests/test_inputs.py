@@ -63,3 +63,17 @@ def test_decode_view_roundtrip():
     dv = I.decode_view(x, 3)
     assert dv.shape == (4, 3, 2)
     assert torch.equal(dv[1, 2], x[2 * 4 + 1])
+
+
+def test_prologue_inputs_shapes_and_determinism():
+    a = I.make_prologue_inputs(total_T=10, H=4, H_qk=2, d_k=16, d_v=32, cu_seqlens=[0, 3, 3, 10],
+                               gate_mode=I.CHANNEL, io_dtype=torch.float32, seed=3)
+    b = I.make_prologue_inputs(total_T=10, H=4, H_qk=2, d_k=16, d_v=32, cu_seqlens=[0, 3, 3, 10],
+                               gate_mode=I.CHANNEL, io_dtype=torch.float32, seed=3)
+    assert a.xq.shape == (10, 2, 16) and a.xv.shape == (10, 4, 32)
+    assert a.wq.shape == (32, 4) and a.wv.shape == (128, 4) and a.xg.shape == (10, 4, 16)
+    assert a.conv_state.shape == (3, 2 * 32 + 128, 3) and a.num_seqs == 3
+    assert torch.equal(a.xq, b.xq) and torch.equal(a.conv_state, b.conv_state)
+    assert not torch.equal(a.xq, a.xk)
+    p = I.prologue_workload()
+    assert p.xq.dtype == torch.bfloat16 and p.total_T == 8192 and p.gscale.shape == (16,)
