@@ -10,10 +10,14 @@ are reported under "workloads" with the same fields.
 
 A "step" is one pass of the whole hot path over one batch of synthetic input:
 one gdr_prefill_chunked call for a prefill workload, the 512 consecutive
-gdr_decode_step calls for a decode workload.  Timing: W untimed warm-up
-steps, then K steps each timed with CUDA events on the stream the kernels are
-launched on; an L2 flush (a 512 MiB write) precedes every timed step and is
-not timed.  Barrier + synchronize bracket the timed region; the time is the
+gdr_decode_step calls for a decode workload, one gdr_prologue call for the
+prologue workload.  Timing: W untimed warm-up steps, then one step is
+captured as a CUDA graph, and K replays of it are each timed with CUDA events
+on the stream the kernels are launched on (--no-graph times eager calls
+instead, which adds the host's per-call time whenever it exceeds the GPU's);
+an L2 flush (a 512 MiB write) precedes every timed step and is not timed.
+The end-to-end figure (`e2e`) always goes through the Python binding with
+pinned host buffers, host/device copies inside its timed region.  Barrier + synchronize bracket the timed region; the time is the
 max over ranks.  For N > 1 every rank runs its own independent batch (heads
 and sequences are independent; no collective on the data path) and `value`
 is the sum of tokens over ranks divided by that time ("weak" scaling).
@@ -344,7 +348,70 @@ class SpecDecodeCase(DecodeCase):
             host_o[t].copy_(self.o[t], non_blocking=True)
 
 
+class PrologueCase:
+    """The input-side prologue at the gdn_prefill shape: one gdr_prologue
+    launch per step (convolution with state, SiLU, q/k normalisation, gate
+    and beta maps)."""
+    kind = "prologue"
+    kernel_label = "prologue"
+
+    def __init__(self, name, device, seed):
+        self.name = name
+        self.inp = inp = I.prologue_workload(name, seed=seed)
+        self.dev = device
+        self.d = {k: getattr(inp, k).to(device) for k in
+                  ("xq", "xk", "xv", "wq", "wk", "wv", "xg", "gscale", "xb", "conv_state")}
+        N = inp.num_seqs
+        self.Call = inp.wq.shape[0] * 2 + inp.wv.shape[0]
+        self.state_out = torch.empty((N, self.Call, 3), dtype=torch.float32, device=device)
+        e = io_bytes(inp.io_dtype)
+        T, Call = inp.total_T, self.Call
+        gate = inp.xg.numel() * 4
+        # read x (q, k, v), taps, gate and beta inputs, state; write the same shapes back
+        self.bytes = (2 * T * Call * e + Call * 16 + 2 * gate + 2 * T * inp.H * 4 + inp.H * 4
+                      + 2 * N * Call * 12)
+        self.flops = 0
+        self.tokens = T
+        self.launches = 1
+        self.path = None
+        self.out = None
+
+    def _call(self, d, stream):
+        self.out = gdr.gdr_prologue(d["xq"], d["xk"], d["xv"], d["wq"], d["wk"], d["wv"], d["xg"],
+                                    d["gscale"], d["xb"], d["conv_state"], None,
+                                    num_seqs=self.inp.num_seqs, conv_state_out=self.state_out,
+                                    silu=True, normalize_qk=True,
+                                    **({} if self.out is None else dict(
+                                        q=self.out[0], k=self.out[1], v=self.out[2],
+                                        g=self.out[3], beta=self.out[4])),
+                                    stream=stream)
+
+    def step(self, stream=None):
+        self._call(self.d, stream)
+
+    def e2e_buffers(self):
+        host = {k: v.cpu().pin_memory() for k, v in self.d.items()}
+        if self.out is None:
+            self.step()
+        outs = list(self.out) + [self.state_out]
+        ho = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
+        h2d = sum(v.numel() * v.element_size() for v in host.values())
+        d2h = sum(o.numel() * o.element_size() for o in ho)
+        return host, ho, None, h2d, d2h
+
+    def e2e_step(self, host, host_o, host_fin, stream):
+        dev = {k: v.to(self.dev, non_blocking=True) for k, v in host.items()}
+        self._call(dev, stream)
+        for h, o in zip(host_o, list(self.out) + [self.state_out]):
+            h.copy_(o, non_blocking=True)
+
+    def dtype_label(self):
+        return "f32 arithmetic, bf16 in and out"
+
+
 def make_case(name, device, seed):
+    if name == "prologue_gdn":
+        return PrologueCase(name, device, seed)
     if name == "decode_spec_gdn":
         return SpecDecodeCase(name, device, seed)
     if name.startswith("decode"):
@@ -420,15 +487,32 @@ def load_traffic(case):
         return None
 
 
+def capture_step(case, stream):
+    """One step captured as a CUDA graph (after warm-up, so every kernel
+    attribute and helper stream already exists): replaying it runs exactly the
+    step's kernels, back to back, without the host's per-call Python and
+    argument-checking time between them."""
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        case.step(stream)
+    torch.cuda.synchronize()
+    return g
+
+
 def bench_case(case, args, ws, rank, flush, stream, pk, pk_kind):
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
             case.step(stream)
         torch.cuda.synchronize()
+        graph = None if args.no_graph else capture_step(case, stream)
+        run = graph.replay if graph is not None else (lambda: case.step(stream))
+        run()
+        torch.cuda.synchronize()
         barrier(ws)
         with ClockSampler(torch.cuda.current_device()) as clk:
-            times = timed_steps(lambda: case.step(stream), args.steps, flush, stream)
+            times = timed_steps(run, args.steps, flush, stream)
         barrier(ws)
+        del graph
     value, ms = aggregate_throughput(case.tokens, sum(times) / len(times), ws)
     tokens_all = case.tokens * ws
     # decode: bytes per launch over the time per launch; prefill: the whole
@@ -464,10 +548,13 @@ def bench_case(case, args, ws, rank, flush, stream, pk, pk_kind):
            "H": inp.H, "H_qk": inp.H_qk, "d_k": inp.d_k, "d_v": inp.d_v, "gate": inp.gate_mode,
            "io": str(inp.io_dtype).replace("torch.", ""),
            "h0": inp.h0 is not None, "l2": "flushed (512 MiB write) before every timed step",
-           "kernel": ("decode" if case.kind == "decode" else
-                      {gdr.GDR_PATH_TCGEN05: "tcgen05",
-                       gdr.GDR_PATH_TCGEN05_SPLIT: "tcgen05 chunk-parallel (prep + chain)"}.get(
-                           case.path, "simt"))}
+           "kernel": getattr(case, "kernel_label", None) or (
+               "decode" if case.kind == "decode" else
+               {gdr.GDR_PATH_TCGEN05: "tcgen05",
+                gdr.GDR_PATH_TCGEN05_SPLIT: "tcgen05 chunk-parallel (prep + chain)"}.get(
+                   case.path, "simt"))}
+    cfg["launch"] = ("the step's kernels replayed from a CUDA graph captured after warm-up"
+                     if not args.no_graph else "eager calls through the Python binding")
     if case.kind == "prefill":
         cfg["launches_per_step"] = case.launches
     if case.kind == "decode":
@@ -544,10 +631,12 @@ def main():
                     help="comma list from: " + ",".join(I.WORKLOADS) + " (or 'all')")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="time eager calls instead of a CUDA-graph replay of the step")
     args = ap.parse_args()
     if args.workloads == "all":
         args.workloads = ("gdn_prefill,kda_prefill,varlen_gdn,gqa_prefill,decode_gdn,decode_kda,"
-                          "decode_spec_gdn")
+                          "decode_spec_gdn,prologue_gdn")
     if args.warmup < 3:
         args.warmup = 3
     ws, rank, local = dist_env()

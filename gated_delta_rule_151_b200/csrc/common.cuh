@@ -7,6 +7,7 @@
 
 #include "gdr.h"
 
+#include <algorithm>
 #include <mutex>
 #include <vector>
 

@@ -216,4 +216,67 @@ gdr_status_t gdr_decode_multi(const void *q, const void *k, const void *v, const
                                               static_cast<cudaStream_t>(stream)));
 }
 
+gdr_status_t gdr_prologue(const void *xq, const void *xk, const void *xv, const float *wq,
+                          const float *wk, const float *wv, const float *xg, const float *gscale,
+                          const float *xb, const float *conv_state_in, float *conv_state_out,
+                          const int32_t *cu_seqlens, int32_t num_seqs, int32_t total_T,
+                          int32_t H_qk, int32_t H, int32_t d_k, int32_t d_v,
+                          gdr_gate_mode_t gate_mode, gdr_dtype_t io_dtype, uint32_t flags,
+                          void *q, void *k, void *v, float *g, float *beta, void *stream) {
+    if (num_seqs < 1 || total_T < 0 || H < 1 || H_qk < 1 || H % H_qk != 0)
+        return GDR_ERR_INVALID_ARG;
+    if (!valid_dim(d_k) || !valid_dim(d_v)) return GDR_ERR_INVALID_ARG;
+    if (gate_mode != GDR_GATE_SCALAR && gate_mode != GDR_GATE_CHANNEL) return GDR_ERR_INVALID_ARG;
+    if (io_dtype != GDR_F32 && io_dtype != GDR_BF16) return GDR_ERR_INVALID_ARG;
+    if ((flags & ~(GDR_PROLOGUE_SILU | GDR_PROLOGUE_NORMALIZE_QK)) != 0) return GDR_ERR_INVALID_ARG;
+    if (cu_seqlens == nullptr && total_T % num_seqs != 0) return GDR_ERR_INVALID_ARG;
+    const int64_t Cq = (int64_t)H_qk * d_k, Cv = (int64_t)H * d_v, Call = 2 * Cq + Cv;
+    if ((int64_t)total_T * Call > ((int64_t)1 << 40) || (int64_t)num_seqs * Call > INT32_MAX)
+        return GDR_ERR_INVALID_ARG;
+    if (conv_state_out != nullptr && !aligned4(conv_state_out)) return GDR_ERR_INVALID_ARG;
+    if (conv_state_in != nullptr && !aligned4(conv_state_in)) return GDR_ERR_INVALID_ARG;
+    if (!ok_ptr(wq) || !ok_ptr(wk) || !ok_ptr(wv)) return GDR_ERR_INVALID_ARG;
+    if (total_T > 0) {
+        if (!ok_ptr(xq) || !ok_ptr(xk) || !ok_ptr(xv) || !ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) ||
+            !ok_gate_ptr(xg, gate_mode) || !ok_gate_ptr(g, gate_mode) || !ok_beta_ptr(xb) ||
+            !ok_beta_ptr(beta) || gscale == nullptr || !aligned4(gscale))
+            return GDR_ERR_INVALID_ARG;
+    }
+    // no output may overlap an input (the convolution reads neighbouring tokens)
+    const size_t e = io_dtype == GDR_BF16 ? 2 : 4;
+    const size_t T = (size_t)total_T, gsz = T * H * (gate_mode == GDR_GATE_CHANNEL ? d_k : 1) * 4;
+    const size_t ssz = (size_t)num_seqs * Call * 3 * 4;
+    struct Range {
+        const void *p;
+        size_t n;
+    };
+    const Range in[] = {{xq, T * Cq * e}, {xk, T * Cq * e}, {xv, T * Cv * e},
+                        {wq, (size_t)Cq * 16}, {wk, (size_t)Cq * 16}, {wv, (size_t)Cv * 16},
+                        {xg, gsz}, {gscale, (size_t)H * 4}, {xb, T * H * 4},
+                        {conv_state_in, ssz},
+                        {cu_seqlens, cu_seqlens ? ((size_t)num_seqs + 1) * 4 : 0}};
+    const Range out[] = {{q, T * Cq * e}, {k, T * Cq * e}, {v, T * Cv * e}, {g, gsz},
+                         {beta, T * H * 4}, {conv_state_out, ssz}};
+    for (const Range &o : out) {
+        if (o.p == nullptr || o.n == 0) continue;
+        const uintptr_t o0 = reinterpret_cast<uintptr_t>(o.p), o1 = o0 + o.n;
+        for (const Range &i : in) {
+            if (i.p == nullptr || i.n == 0) continue;
+            const uintptr_t i0 = reinterpret_cast<uintptr_t>(i.p), i1 = i0 + i.n;
+            if (o0 < i1 && i0 < o1) return GDR_ERR_INVALID_ARG;
+        }
+        for (const Range &o2 : out) {
+            if (&o2 == &o || o2.p == nullptr || o2.n == 0) continue;
+            const uintptr_t a0 = reinterpret_cast<uintptr_t>(o2.p), a1 = a0 + o2.n;
+            if (o0 < a1 && a0 < o1) return GDR_ERR_INVALID_ARG;
+        }
+    }
+    if (total_T == 0 && conv_state_out == nullptr) return GDR_OK;
+    return from_cuda(gdr::launch_prologue(
+        xq, xk, xv, wq, wk, wv, xg, gscale, xb, conv_state_in, conv_state_out, cu_seqlens,
+        num_seqs, total_T, H_qk, H, d_k, d_v, gate_mode == GDR_GATE_CHANNEL, io_dtype == GDR_BF16,
+        (flags & GDR_PROLOGUE_SILU) != 0, (flags & GDR_PROLOGUE_NORMALIZE_QK) != 0, q, k, v, g,
+        beta, static_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

@@ -13,6 +13,16 @@ cudaError_t launch_decode_step(const void *q, const void *k, const void *v, cons
                                const float *beta, float *state, int N, int Hqk, int H, int DK,
                                int DV, bool channel, bool bf16, void *o, cudaStream_t stream);
 
+// Input-side prologue: short causal convolution with state, q/k
+// normalisation, gate and beta maps (arguments validated by the C ABI).
+cudaError_t launch_prologue(const void *xq, const void *xk, const void *xv, const float *wq,
+                            const float *wk, const float *wv, const float *xg,
+                            const float *gscale, const float *xb, const float *state_in,
+                            float *state_out, const int32_t *cu, int num_seqs, int total_T,
+                            int Hqk, int H, int dk, int dv, bool channel, bool bf16, bool silu,
+                            bool norm, void *q, void *k, void *v, float *g, float *beta,
+                            cudaStream_t stream);
+
 // T consecutive tokens per sequence in one pass over the state (T <= 16).
 cudaError_t launch_decode_multi(const void *q, const void *k, const void *v, const float *g,
                                 const float *beta, float *state, int N, int T, int Hqk, int H,

@@ -31,12 +31,14 @@ GDR_BF16 = 1
 GDR_PATH_SIMT = 0
 GDR_PATH_TCGEN05 = 1
 GDR_PATH_TCGEN05_SPLIT = 2
+GDR_PROLOGUE_SILU = 1
+GDR_PROLOGUE_NORMALIZE_QK = 2
 
 # Every symbol include/gdr.h declares.
 EXPORTED = ("gdr_status_string", "gdr_prefill_workspace_size", "gdr_prefill_path",
             "gdr_prefill_chunked", "gdr_prefill_check_workspace", "gdr_decode_step",
             "gdr_prefill_chunked_noalloc", "gdr_prefill_chunked_gqa", "gdr_decode_step_gqa",
-            "gdr_decode_multi", "gdr_prefill_plan")
+            "gdr_decode_multi", "gdr_prefill_plan", "gdr_prologue")
 
 
 class GdrError(RuntimeError):
@@ -89,6 +91,8 @@ def load_library():
         lib.gdr_decode_multi.argtypes = [P, P, P, P, P, P, I32, I32, I32, I32, I32, I32, ST, ST, P,
                                          P, P]
         lib.gdr_decode_multi.restype = ST
+        lib.gdr_prologue.argtypes = [P] * 12 + [I32] * 6 + [ST, ST, ctypes.c_uint32] + [P] * 6
+        lib.gdr_prologue.restype = ST
         _lib = lib
         return lib
 
@@ -339,3 +343,51 @@ def gdr_decode_multi(q, k, v, g, beta, state, *, o=None, snapshots=None, stream=
                                          _ptr(o), _ptr(snapshots), _stream_ptr(stream))
     _check(st, "gdr_decode_multi")
     return o
+
+
+def gdr_prologue(xq, xk, xv, wq, wk, wv, xg, gscale, xb, conv_state_in=None, cu_seqlens=None, *,
+                 num_seqs=None, conv_state_out=None, silu=False, normalize_qk=True, q=None,
+                 k=None, v=None, g=None, beta=None, stream=None):
+    """Input-side prologue (see include/gdr.h): short causal convolution with
+    state, optional SiLU, q/k L2 normalisation, beta and log-gate maps.
+
+    xq, xk [T, H_qk, d_k]; xv [T, H, d_v] (bf16 or fp32); wq, wk [H_qk d_k, 4];
+    wv [H d_v, 4]; xg [T, H] or [T, H, d_k]; gscale [H]; xb [T, H];
+    conv_state_in / conv_state_out [N, 2 H_qk d_k + H d_v, 3] fp32 or None.
+    Returns (q, k, v, g, beta).
+    """
+    _need(xq, "xq", ndim=3)
+    io = xq.dtype
+    _need(xk, "xk", io, 3)
+    _need(xv, "xv", io, 3)
+    for t, name in ((wq, "wq"), (wk, "wk"), (wv, "wv")):
+        _need(t, name, torch.float32, 2)
+    _need(xg, "xg", torch.float32)
+    _need(gscale, "gscale", torch.float32, 1)
+    _need(xb, "xb", torch.float32, 2)
+    T, Hqk, dk = xq.shape
+    H, dv = xv.shape[1], xv.shape[2]
+    gate = GDR_GATE_SCALAR if xg.dim() == 2 else GDR_GATE_CHANNEL
+    if cu_seqlens is not None:
+        _need(cu_seqlens, "cu_seqlens", torch.int32, 1)
+        n = cu_seqlens.numel() - 1
+    else:
+        n = 1 if num_seqs is None else int(num_seqs)
+    if conv_state_in is not None:
+        _need(conv_state_in, "conv_state_in", torch.float32, 3)
+    if conv_state_out is not None:
+        _need(conv_state_out, "conv_state_out", torch.float32, 3)
+    dev = xq.device
+    q = torch.empty_like(xq) if q is None else q
+    k = torch.empty_like(xk) if k is None else k
+    v = torch.empty_like(xv) if v is None else v
+    g = torch.empty(xg.shape, dtype=torch.float32, device=dev) if g is None else g
+    beta = torch.empty(xb.shape, dtype=torch.float32, device=dev) if beta is None else beta
+    flags = (GDR_PROLOGUE_SILU if silu else 0) | (GDR_PROLOGUE_NORMALIZE_QK if normalize_qk else 0)
+    st = load_library().gdr_prologue(
+        _ptr(xq), _ptr(xk), _ptr(xv), _ptr(wq), _ptr(wk), _ptr(wv), _ptr(xg), _ptr(gscale),
+        _ptr(xb), _ptr(conv_state_in), _ptr(conv_state_out), _ptr(cu_seqlens), n, T, Hqk, H, dk,
+        dv, gate, _io_code(io), flags, _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+        _stream_ptr(stream))
+    _check(st, "gdr_prologue")
+    return q, k, v, g, beta

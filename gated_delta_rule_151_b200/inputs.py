@@ -277,6 +277,26 @@ class PrologueInputs:
     def total_T(self) -> int:
         return int(self.xq.shape[0])
 
+    @property
+    def H(self) -> int:
+        return int(self.xv.shape[1])
+
+    @property
+    def H_qk(self) -> int:
+        return int(self.xq.shape[1])
+
+    @property
+    def d_k(self) -> int:
+        return int(self.xq.shape[2])
+
+    @property
+    def d_v(self) -> int:
+        return int(self.xv.shape[2])
+
+    @property
+    def h0(self):
+        return None
+
 
 def make_prologue_inputs(*, total_T: int, H: int, d_k: int, d_v: int | None = None,
                          H_qk: int | None = None, num_seqs: int = 1, cu_seqlens=None,

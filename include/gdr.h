@@ -274,6 +274,59 @@ GDR_API gdr_status_t gdr_decode_multi(const void *q, const void *k, const void *
                               gdr_gate_mode_t gate_mode, gdr_dtype_t io_dtype, void *o,
                               float *snapshots, void *stream);
 
+/*
+ * Input-side prologue of a gated delta-rule layer: turns the raw q/k/v
+ * projections and raw gate/beta activations into the recurrence's inputs.
+ *
+ *  - Short causal convolution, kernel size 4 (page "Qwen3.8-Flash-Next and
+ *    GLM-5.3-Flash share a 3:1 long-context pattern", section "Kimi Delta
+ *    Attention extends recurrent memory control"), depthwise: each channel of
+ *    x_q, x_k and x_v has its own four taps,
+ *        y_t[c] = w[c][0] x_{t-3}[c] + w[c][1] x_{t-2}[c] + w[c][2] x_{t-1}[c] + w[c][3] x_t[c],
+ *    causal within each sequence.  Before a sequence's first token the inputs
+ *    come from conv_state_in (zeros when it is NULL); conv_state_out receives
+ *    each sequence's last three inputs, the state a decode call continuing
+ *    the sequence starts from (page "How the New Flash Models Work", section
+ *    "Serving: prefill and decode are different problems").
+ *  - Optional SiLU y <- y / (1 + e^-y) (flag GDR_PROLOGUE_SILU).
+ *  - Optional L2 normalisation of every q and k head over its d_k channels,
+ *    y <- y / sqrt(sum y^2 + 1e-6) (flag GDR_PROLOGUE_NORMALIZE_QK).
+ *  - beta = sigmoid(x_beta); log-gate g = -gscale[h] * softplus(x_g).
+ *
+ * Layouts (row-major, token-major like the other entry points):
+ *   xq, xk, q, k   [total_T, H_qk, d_k]   io dtype
+ *   xv, v          [total_T, H, d_v]      io dtype
+ *   wq, wk         [H_qk * d_k, 4]        fp32 taps; tap 3 takes the current token
+ *   wv             [H * d_v, 4]           fp32
+ *   xg, g          [total_T, H] (GDR_GATE_SCALAR) or [total_T, H, d_k] (GDR_GATE_CHANNEL), fp32
+ *   gscale         [H]                    fp32, > 0 for a decaying gate
+ *   xb, beta       [total_T, H]           fp32
+ *   conv_state_*   [num_seqs, 2 H_qk d_k + H d_v, 3] fp32: channels of q, then
+ *                  k, then v; per channel the three inputs before (in) or at
+ *                  the end of (out) the sequence, oldest first.  Either may be
+ *                  NULL; they must not overlap.
+ * cu_seqlens as for gdr_prefill_chunked (NULL = num_seqs equal sequences).
+ * A sequence shorter than three tokens carries part of conv_state_in over to
+ * conv_state_out; an empty one copies it.  For decode, pass one token per
+ * sequence (cu_seqlens NULL, total_T = num_seqs).
+ * Pointers: x*, q, k, v, w* and channel-mode xg/g 16-byte aligned; the rest
+ * 4-byte aligned.  Outputs must not overlap the inputs (the convolution reads
+ * neighbouring tokens).  Errors: GDR_ERR_INVALID_ARG for a bad size, pointer,
+ * flag or overlap, before anything is launched; GDR_ERR_CUDA on launch
+ * failure.
+ */
+#define GDR_PROLOGUE_SILU 1u
+#define GDR_PROLOGUE_NORMALIZE_QK 2u
+
+GDR_API gdr_status_t gdr_prologue(const void *xq, const void *xk, const void *xv,
+                                  const float *wq, const float *wk, const float *wv,
+                                  const float *xg, const float *gscale, const float *xb,
+                                  const float *conv_state_in, float *conv_state_out,
+                                  const int32_t *cu_seqlens, int32_t num_seqs, int32_t total_T,
+                                  int32_t H_qk, int32_t H, int32_t d_k, int32_t d_v,
+                                  gdr_gate_mode_t gate_mode, gdr_dtype_t io_dtype, uint32_t flags,
+                                  void *q, void *k, void *v, float *g, float *beta, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

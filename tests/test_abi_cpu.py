@@ -173,3 +173,42 @@ def test_decode_multi_rejects_invalid_arguments(lib, T, Hqk, H):
     st = lib.gdr_decode_multi(P(A), P(A), P(A), P(A), P(A), P(A), 2, 4, 2, 2, 128, 128, 0, 1,
                               P(A), P(MIS), None)
     assert st == gdr.GDR_ERR_INVALID_ARG     # misaligned snapshot buffer
+
+
+_PRO_BASE = 1 << 40
+_PRO_NAMES = ("xq", "xk", "xv", "wq", "wk", "wv", "xg", "gs", "xb", "sin", "sout", "cu",
+              "q", "k", "v", "g", "beta")
+_PRO = {n: _PRO_BASE + (i << 30) for i, n in enumerate(_PRO_NAMES)}   # 1 GiB apart
+
+
+def _prologue(lib, **kw):
+    args = dict(_PRO)
+    args.update(cu=None, sin=None, sout=None, N=1, T=64, Hqk=2, H=2, dk=16, dv=16, gate=0, io=0,
+                flags=2)
+    args.update(kw)
+    P = lambda x: None if x is None else ctypes.c_void_p(x)
+    return lib.gdr_prologue(*(P(args[n]) for n in _PRO_NAMES[:12]), args["N"], args["T"],
+                            args["Hqk"], args["H"], args["dk"], args["dv"], args["gate"],
+                            args["io"], args["flags"], *(P(args[n]) for n in _PRO_NAMES[12:]), None)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(xq=None), dict(xv=None), dict(q=None), dict(wq=None), dict(gs=None), dict(xb=None),
+    dict(beta=None), dict(g=None),
+    dict(xq=_PRO["xq"] + 2), dict(q=_PRO["q"] + 8), dict(wv=_PRO["wv"] + 4),
+    dict(xg=_PRO["xg"] + 2), dict(xg=_PRO["xg"] + 4, gate=1), dict(g=_PRO["g"] + 4, gate=1),
+    dict(sin=_PRO["sin"] + 2), dict(sout=_PRO["sout"] + 1),
+    dict(dk=48), dict(dv=256), dict(H=0), dict(Hqk=3), dict(N=0), dict(T=-1),
+    dict(N=3, T=64), dict(gate=2), dict(io=5), dict(flags=4),
+    # outputs overlapping inputs or each other
+    dict(q=_PRO["xq"]), dict(v=_PRO["xv"] + 64), dict(g=_PRO["xg"]), dict(beta=_PRO["xb"]),
+    dict(sin=_PRO["sin"], sout=_PRO["sin"] + 12), dict(k=_PRO["q"] + 16),
+    dict(sout=_PRO["wq"]),
+])
+def test_prologue_rejects_invalid_arguments(lib, kw):
+    assert _prologue(lib, **kw) == gdr.GDR_ERR_INVALID_ARG
+
+
+def test_prologue_empty_problem_is_a_no_op(lib):
+    assert _prologue(lib, T=0, xq=None, xk=None, xv=None, q=None, k=None, v=None, xg=None,
+                     g=None, xb=None, beta=None) == gdr.GDR_OK
