@@ -17,16 +17,16 @@
 // The pass is HBM-bound: per token and head it reads the raw q/k/v
 // projections once and writes the recurrence's q/k/v once.  Roles by block:
 //
-//   conv blocks   persistent blocks over (tensor, 128-channel block, 64-token
-//                 tile) items.  A three-stage cp.async ring brings each tile's
-//                 rows (and the three before it) into shared memory two tiles
-//                 ahead of the one computed, so the bytes in flight cost no
-//                 registers.  Lane l of a warp owns channels 4l..4l+3; a warp
-//                 takes a run of eight consecutive tokens, reads the run's
-//                 eleven window rows once, and interleaves the eight norms,
-//                 xor-shuffle sums over the d_k / 4 lanes of a head.  Loads and
-//                 stores are contiguous 256-byte (bf16) or 512-byte (fp32) row
-//                 pieces per warp.
+//   conv blocks   persistent warps over (tensor, 128-channel block, run of
+//                 eight tokens) items.  Each warp keeps its own three-stage
+//                 cp.async ring of window rows (the run's eight and the three
+//                 before it) in shared memory, two runs ahead of the one it
+//                 computes, so the bytes in flight cost no registers and no
+//                 block barrier couples the warps.  Lane l owns channels
+//                 4l..4l+3; the run's outputs are computed on the packed
+//                 fp32x2 units and its eight head norms reduced together.
+//                 Loads and stores are contiguous 256-byte (bf16) or 512-byte
+//                 (fp32) row pieces per warp.
 //   gate blocks   grid-stride over the g and beta elements.
 //   state blocks  one thread per (sequence, channel) writes the three inputs
 //                 before the sequence's end (falling back to the incoming
@@ -37,13 +37,15 @@
 namespace gdr {
 namespace {
 
-constexpr int kProWarps = 8;                  // warps per conv block
-constexpr int kProTile = 64;                  // tokens per work item
-constexpr int kProRun = kProTile / kProWarps;  // consecutive tokens per warp
-// a stage: the tile's rows and the three before it, 128 channels of fp32 at most
-constexpr int kProStageBytes = (kProTile + 3) * 128 * 4;
-constexpr int kProStages = 3;
+constexpr int kProWarps = 4;                  // warps per block
+constexpr int kProRun = 8;                    // consecutive tokens per work item
+static_assert(kProRun == 8, "the norm butterfly spreads eight tokens over the xor-16/8/4 steps");
+constexpr int kProRows = kProRun + 3;         // a run's window rows
+constexpr int kProStages = 3;                 // per-warp cp.async ring
 constexpr int kProThreads = 32 * kProWarps;
+// shared memory of one block: every warp's ring of window rows, 128 channels
+template <typename IoT>
+constexpr int pro_smem_bytes() { return kProWarps * kProStages * kProRows * 128 * (int)sizeof(IoT); }
 constexpr float kNormEps = 1e-6f;
 
 struct ProArgs {
@@ -58,7 +60,7 @@ struct ProArgs {
     int num_seqs, total_T, Hqk, H, dk, dv;
     int Cq, Cv, Call;                     // channels of q (= of k), of v, of all three
     int nbq, nbv, nball;                  // 128-channel blocks: q (= k), v, all
-    int tiles;                            // token tiles
+    int runs;                             // runs of kProRun tokens
     int conv_blocks, gate_blocks, state_blocks;
     bool channel, silu, norm;
 };
@@ -110,7 +112,40 @@ __device__ __forceinline__ int seq_of(const ProArgs &A, int t, int &a, int &b) {
     return lo;
 }
 
-__device__ __forceinline__ float silu_f(float y) { return __fdividef(y, 1.0f + __expf(-y)); }
+// Single-instruction approximations (denormals flushed: every operand here is
+// either normal or its exact result is 0 or 1 to fp32 precision).
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ float rcp_approx(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ float rsqrt_approx(float x) {   // x >= 1e-6 here
+    float y;
+    asm("rsqrt.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+// SiLU y / (1 + e^-y) = y * 1 / (1 + 2^(-y log2 e)), on a pair of channels.
+// For y -> -inf the power overflows to inf and the reciprocal to 0.
+__device__ __forceinline__ float2 silu2(float2 y) {
+    float2 t = __fmul2_rn(y, make_float2(-kLog2e, -kLog2e));
+    t = make_float2(ex2_approx(t.x), ex2_approx(t.y));
+    t = __fadd2_rn(t, make_float2(1.f, 1.f));
+    return __fmul2_rn(y, make_float2(rcp_approx(t.x), rcp_approx(t.y)));
+}
+
+__device__ __forceinline__ float silu_f(float y) {
+    return y * rcp_approx(1.0f + ex2_approx(-kLog2e * y));
+}
 
 __device__ __forceinline__ void cp_async16(void *dst, const void *src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(
@@ -128,54 +163,54 @@ __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
 }
 
-// One work item: (tensor, 128-channel block, token tile).
+// One work item: (tensor, 128-channel block, run of kProRun tokens).
 struct ProItem {
-    int which, cb, t0, t1, C;
+    int which, cb, tr, te, C;
 };
 
 __device__ __forceinline__ ProItem item_of(const ProArgs &A, int item) {
     ProItem it;
-    const int tile = item / A.nball, cbg = item % A.nball;
+    const int run = item / A.nball, cbg = item % A.nball;
     if (cbg < A.nbq) { it.which = 0; it.cb = cbg; }
     else if (cbg < 2 * A.nbq) { it.which = 1; it.cb = cbg - A.nbq; }
     else { it.which = 2; it.cb = cbg - 2 * A.nbq; }
     it.C = it.which == 2 ? A.Cv : A.Cq;
-    it.t0 = tile * kProTile;
-    it.t1 = min(it.t0 + kProTile, A.total_T);
+    it.tr = run * kProRun;
+    it.te = min(it.tr + kProRun, A.total_T);
     return it;
 }
 
-// Copy rows t0-3 .. t1-1 (those inside [0, total_T)) of the item's 128
-// channels into a stage: row r holds token t0 - 3 + r.
+// One warp copies the rows tr-3 .. te-1 (those inside [0, total_T)) of the
+// item's 128 channels into one of its stages: row r holds token tr - 3 + r.
 template <typename IoT>
-__device__ __forceinline__ void issue_tile(const ProArgs &A, const ProItem &it, uint8_t *stage) {
+__device__ __forceinline__ void issue_run(const ProArgs &A, const ProItem &it, uint8_t *stage,
+                                          int lane) {
     const IoT *x = static_cast<const IoT *>(it.which == 0 ? A.xq : it.which == 1 ? A.xk : A.xv);
     const int width = min(128, it.C - it.cb * 128);          // channels (multiple of 16)
     constexpr int kRowBytes = 128 * (int)sizeof(IoT);
-    const int pieces = width * (int)sizeof(IoT) / 16;        // 16-byte pieces per row
-    const int rows = it.t1 - it.t0 + 3;
-    for (int i = threadIdx.x; i < rows * pieces; i += kProThreads) {
-        const int r = i / pieces, p = i % pieces;
-        const int t = it.t0 - 3 + r;
-        if (t < 0) continue;
-        const uint8_t *src = reinterpret_cast<const uint8_t *>(x + (size_t)t * it.C + it.cb * 128);
-        cp_async16(stage + r * kRowBytes + 16 * p, src + 16 * p);
+    constexpr int kPieces = kRowBytes / 16;                  // 16-byte pieces of a full row
+    const int pieces = width * (int)sizeof(IoT) / 16;        // of this block's rows
+    const uint8_t *base = reinterpret_cast<const uint8_t *>(x + it.cb * 128);
+    const size_t pitch = (size_t)it.C * sizeof(IoT);
+    for (int i = lane; i < kProRows * kPieces; i += 32) {
+        const int r = i / kPieces, p = i % kPieces;
+        const int t = it.tr - 3 + r;
+        if (t < 0 || t >= it.te || p >= pieces) continue;
+        cp_async16(stage + r * kRowBytes + 16 * p, base + (size_t)t * pitch + 16 * p);
     }
 }
 
 __device__ __forceinline__ void lds4(const float *p, float (&x)[4]) { load4(p, x); }
 __device__ __forceinline__ void lds4(const __nv_bfloat16 *p, float (&x)[4]) { load4(p, x); }
 
-// Outputs of the item's tokens: warp w takes the kProRun consecutive tokens
-// t0 + kProRun w ..., loads their kProRun + 3 window rows from the stage once,
-// computes the outputs in place (token s reads rows s..s+3 only, so oldest
-// first frees row s), and interleaves the kProRun norms, xor-shuffle sums over
-// the d_k / 4 lanes of a head.  Inputs before a token's sequence come from the
+// Outputs of a run's tokens: the warp loads the run's kProRun + 3 window rows
+// from its stage once, computes the outputs in place (token s reads rows
+// s..s+3 only, so oldest first frees row s), and reduces the kProRun head
+// norms together, xor-shuffle sums over the d_k / 4 lanes of a head.  Inputs before a token's sequence come from the
 // incoming state (zeros without one).
 template <typename IoT>
-__device__ __forceinline__ void compute_tile(const ProArgs &A, const ProItem &it,
-                                             const uint8_t *stage) {
-    const int lane = threadIdx.x % 32, warp = threadIdx.x / 32;
+__device__ __forceinline__ void compute_run(const ProArgs &A, const ProItem &it,
+                                            const uint8_t *stage, int lane) {
     const int c = it.cb * 128 + 4 * lane;
     const bool live = c < it.C;
     const bool normed = A.norm && it.which < 2;
@@ -184,8 +219,7 @@ __device__ __forceinline__ void compute_tile(const ProArgs &A, const ProItem &it
     const float *w = it.which == 0 ? A.wq : it.which == 1 ? A.wk : A.wv;
     IoT *y = static_cast<IoT *>(it.which == 0 ? A.q : it.which == 1 ? A.k : A.v);
     const IoT *rows = reinterpret_cast<const IoT *>(stage);
-    const int tr = it.t0 + kProRun * warp;           // the run's first token
-    if (tr >= it.t1) return;                         // warp-uniform
+    const int tr = it.tr, te = it.te;
 
     float tap[4][4];
 #pragma unroll
@@ -200,12 +234,11 @@ __device__ __forceinline__ void compute_tile(const ProArgs &A, const ProItem &it
     for (int r = 0; r < kProRun + 3; ++r) {
 #pragma unroll
         for (int j = 0; j < 4; ++j) xr[r][j] = 0.f;
-        if (live) lds4(rows + (tr - it.t0 + r) * 128 + 4 * lane, xr[r]);
+        if (live) lds4(rows + r * 128 + 4 * lane, xr[r]);
     }
     // rows before a token's sequence: the incoming state, or zeros
     int a0, b0;
     const int n0 = seq_of(A, tr, a0, b0);
-    const int te = min(tr + kProRun, it.t1);
     if (!(tr >= a0 + 3 && te <= b0)) {
 #pragma unroll
         for (int s = 0; s < kProRun; ++s) {
@@ -244,11 +277,12 @@ __device__ __forceinline__ void compute_tile(const ProArgs &A, const ProItem &it
                 o[j] = A.silu ? silu_f(acc) : acc;
             }
             if (normed) {
-                float ss = o[0] * o[0];
-#pragma unroll
-                for (int j = 1; j < 4; ++j) ss = fmaf(o[j], o[j], ss);
+                // the same pairing as the packed path: the two paths agree bit for bit
+                const float2 lo = make_float2(o[0], o[1]), hi = make_float2(o[2], o[3]);
+                const float2 q2 = __ffma2_rn(hi, hi, __fmul2_rn(lo, lo));
+                float ss = q2.x + q2.y;
                 for (int off = group / 2; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-                const float r = rsqrtf(ss + kNormEps);
+                const float r = rsqrt_approx(ss + kNormEps);
 #pragma unroll
                 for (int j = 0; j < 4; ++j) o[j] *= r;
             }
@@ -256,68 +290,116 @@ __device__ __forceinline__ void compute_tile(const ProArgs &A, const ProItem &it
         }
         return;
     }
-    // the whole run lies at least three tokens inside one sequence
+    // the whole run lies at least three tokens inside one sequence: pairs of
+    // channels on the packed fp32x2 units
+    float2 tp[2][4];                                 // [channel pair][tap]
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) tp[h][i] = make_float2(tap[2 * h][i], tap[2 * h + 1][i]);
+    float2 xp[kProRun + 3][2];
+#pragma unroll
+    for (int r = 0; r < kProRun + 3; ++r) {
+        xp[r][0] = make_float2(xr[r][0], xr[r][1]);
+        xp[r][1] = make_float2(xr[r][2], xr[r][3]);
+    }
+    float ss[kProRun];
 #pragma unroll
     for (int s = 0; s < kProRun; ++s) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            float acc = tap[j][0] * xr[s][j];
-            acc = fmaf(tap[j][1], xr[s + 1][j], acc);
-            acc = fmaf(tap[j][2], xr[s + 2][j], acc);
-            acc = fmaf(tap[j][3], xr[s + 3][j], acc);
-            xr[s][j] = A.silu ? silu_f(acc) : acc;
+        for (int h = 0; h < 2; ++h) {
+            float2 acc = __fmul2_rn(tp[h][0], xp[s][h]);
+            acc = __ffma2_rn(tp[h][1], xp[s + 1][h], acc);
+            acc = __ffma2_rn(tp[h][2], xp[s + 2][h], acc);
+            acc = __ffma2_rn(tp[h][3], xp[s + 3][h], acc);
+            xp[s][h] = A.silu ? silu2(acc) : acc;    // row s is not read again
         }
+        const float2 q2 = __ffma2_rn(xp[s][1], xp[s][1], __fmul2_rn(xp[s][0], xp[s][0]));
+        ss[s] = q2.x + q2.y;
     }
     if (normed) {
-        float ss[kProRun];
+        float tot[kProRun];
+        if (group == 32) {
+            // transposed butterfly: halve the tokens a lane carries at each of
+            // the xor-16/8/4 steps, finish with xor 2/1, then fetch each
+            // token's total from a lane that holds it (token of lane l:
+            // 4 bit4(l) + 2 bit3(l) + bit2(l))
+            const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
+            float v4[4], v2[2];
 #pragma unroll
-        for (int s = 0; s < kProRun; ++s) {
-            ss[s] = xr[s][0] * xr[s][0];
+            for (int k = 0; k < 4; ++k) {
+                const float send = b4 ? ss[k] : ss[k + 4], keep = b4 ? ss[k + 4] : ss[k];
+                v4[k] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+            }
 #pragma unroll
-            for (int j = 1; j < 4; ++j) ss[s] = fmaf(xr[s][j], xr[s][j], ss[s]);
+            for (int k = 0; k < 2; ++k) {
+                const float send = b3 ? v4[k] : v4[k + 2], keep = b3 ? v4[k + 2] : v4[k];
+                v2[k] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+            }
+            float v = (b2 ? v2[1] : v2[0]) + __shfl_xor_sync(0xffffffffu, b2 ? v2[0] : v2[1], 4);
+            v += __shfl_xor_sync(0xffffffffu, v, 2);
+            v += __shfl_xor_sync(0xffffffffu, v, 1);
+#pragma unroll
+            for (int k = 0; k < kProRun; ++k)
+                tot[k] = __shfl_sync(0xffffffffu, v, ((k >> 2) & 1) * 16 + ((k >> 1) & 1) * 8 + (k & 1) * 4);
+        } else {
+#pragma unroll
+            for (int k = 0; k < kProRun; ++k) tot[k] = ss[k];
+            for (int off = group / 2; off > 0; off >>= 1) {
+#pragma unroll
+                for (int k = 0; k < kProRun; ++k) tot[k] += __shfl_xor_sync(0xffffffffu, tot[k], off);
+            }
         }
-        for (int off = group / 2; off > 0; off >>= 1) {
 #pragma unroll
-            for (int s = 0; s < kProRun; ++s) ss[s] += __shfl_xor_sync(0xffffffffu, ss[s], off);
-        }
-#pragma unroll
-        for (int s = 0; s < kProRun; ++s) {
-            const float r = rsqrtf(ss[s] + kNormEps);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) xr[s][j] *= r;
+        for (int k = 0; k < kProRun; ++k) {
+            const float r = rsqrt_approx(tot[k] + kNormEps);
+            xp[k][0] = __fmul2_rn(xp[k][0], make_float2(r, r));
+            xp[k][1] = __fmul2_rn(xp[k][1], make_float2(r, r));
         }
     }
     if (live) {
+        IoT *out = y + (size_t)tr * it.C + c;
 #pragma unroll
-        for (int s = 0; s < kProRun; ++s)
-            if (tr + s < te) store4(y + (size_t)(tr + s) * it.C + c, xr[s]);
+        for (int k = 0; k < kProRun; ++k) {
+            if (tr + k < te) {
+                const float o4[4] = {xp[k][0].x, xp[k][0].y, xp[k][1].x, xp[k][1].y};
+                store4(out, o4);
+            }
+            out += it.C;
+        }
     }
 }
 
-// Persistent conv blocks: a cp.async ring of kProStages tiles over the
-// block's items, the copies of the next kProStages - 1 tiles in flight while
-// this one is computed.
+// Persistent warps: each walks over its work items with its own ring of
+// kProStages stages, the copies of its next kProStages - 1 runs in flight
+// while it computes this one.  cp.async groups belong to the issuing thread,
+// so a warp waits for its own copies and needs no block barrier; __syncwarp
+// makes the lanes' copies visible to each other and protects a stage until
+// every lane is done with it.
 template <typename IoT>
-__device__ void conv_blocks(const ProArgs &A, uint8_t *smem) {
-    const int items = A.tiles * A.nball;
-    const int first = blockIdx.x, stride = A.conv_blocks;
+__device__ void conv_warps(const ProArgs &A, uint8_t *smem) {
+    constexpr int kStageBytes = kProRows * 128 * (int)sizeof(IoT);
+    const int lane = threadIdx.x % 32, warp = threadIdx.x / 32;
+    uint8_t *ring = smem + warp * kProStages * kStageBytes;
+    const int items = A.runs * A.nball;
+    const int first = blockIdx.x * kProWarps + warp, stride = A.conv_blocks * kProWarps;
     const int mine = items > first ? (items - 1 - first) / stride + 1 : 0;
 #pragma unroll
     for (int j = 0; j < kProStages - 1; ++j) {
-        if (j < mine) issue_tile<IoT>(A, item_of(A, first + j * stride), smem + j * kProStageBytes);
+        if (j < mine) issue_run<IoT>(A, item_of(A, first + j * stride), ring + j * kStageBytes, lane);
         cp_async_commit();
     }
     for (int j = 0; j < mine; ++j) {
         const int jn = j + kProStages - 1;
         if (jn < mine)
-            issue_tile<IoT>(A, item_of(A, first + jn * stride),
-                            smem + (jn % kProStages) * kProStageBytes);
+            issue_run<IoT>(A, item_of(A, first + jn * stride), ring + (jn % kProStages) * kStageBytes,
+                           lane);
         cp_async_commit();
-        cp_async_wait<kProStages - 1>();   // tile j has landed (groups complete in order)
-        __syncthreads();
-        compute_tile<IoT>(A, item_of(A, first + j * stride),
-                          smem + (j % kProStages) * kProStageBytes);
-        __syncthreads();
+        cp_async_wait<kProStages - 1>();   // run j has landed (groups complete in order)
+        __syncwarp();
+        compute_run<IoT>(A, item_of(A, first + j * stride), ring + (j % kProStages) * kStageBytes,
+                         lane);
+        __syncwarp();
     }
 }
 
@@ -326,12 +408,12 @@ __device__ __forceinline__ float softplus_f(float x) {
 }
 
 template <typename IoT>
-__global__ void __launch_bounds__(kProThreads, 2)
+__global__ void __launch_bounds__(kProThreads, 4)
 prologue_kernel(const __grid_constant__ ProArgs A) {
     const int bid = blockIdx.x;
     if (bid < A.conv_blocks) {
         extern __shared__ __align__(128) uint8_t smem[];
-        conv_blocks<IoT>(A, smem);
+        conv_warps<IoT>(A, smem);
         return;
     }
     if (bid < A.conv_blocks + A.gate_blocks) {
@@ -392,17 +474,18 @@ cudaError_t launch_prologue(const void *xq, const void *xk, const void *xv, cons
     A.num_seqs = num_seqs; A.total_T = total_T; A.Hqk = Hqk; A.H = H; A.dk = dk; A.dv = dv;
     A.Cq = Hqk * dk; A.Cv = H * dv; A.Call = 2 * A.Cq + A.Cv;
     A.nbq = (A.Cq + 127) / 128; A.nbv = (A.Cv + 127) / 128; A.nball = 2 * A.nbq + A.nbv;
-    A.tiles = (total_T + kProTile - 1) / kProTile;
+    A.runs = (total_T + kProRun - 1) / kProRun;
     A.channel = channel; A.silu = silu; A.norm = norm;
-    const long long items = (long long)A.tiles * A.nball;
+    const long long items = (long long)A.runs * A.nball;
     if (items > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
     int dev = 0, sms = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
-    // two resident CTAs per SM (three stages of 34 KiB each): one wave of
-    // persistent blocks
-    A.conv_blocks = (int)std::min<long long>(items, 2LL * sms);
+    // one wave of persistent warps: four resident blocks of four warps per SM
+    // (shared memory allows three with fp32 rows)
+    const long long per_sm = bf16 ? 4 : 3;
+    A.conv_blocks = (int)std::min<long long>((items + kProWarps - 1) / kProWarps, per_sm * sms);
     const long long gate_elems = (long long)total_T * H * (channel ? dk : 1);
     A.gate_blocks = total_T > 0 ? (int)std::min<long long>((gate_elems + kProThreads - 1) / kProThreads, 1184) : 0;
     A.state_blocks = state_out != nullptr
@@ -411,12 +494,13 @@ cudaError_t launch_prologue(const void *xq, const void *xk, const void *xv, cons
     const long long blocks = (long long)A.conv_blocks + A.gate_blocks + A.state_blocks;
     if (blocks == 0) return cudaSuccess;
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-    constexpr int smem = kProStages * kProStageBytes;
     if (bf16) {
+        constexpr int smem = pro_smem_bytes<__nv_bfloat16>();
         e = ensure_dynamic_smem(reinterpret_cast<const void *>(prologue_kernel<__nv_bfloat16>), smem);
         if (e != cudaSuccess) return e;
         prologue_kernel<__nv_bfloat16><<<(unsigned)blocks, kProThreads, smem, stream>>>(A);
     } else {
+        constexpr int smem = pro_smem_bytes<float>();
         e = ensure_dynamic_smem(reinterpret_cast<const void *>(prologue_kernel<float>), smem);
         if (e != cudaSuccess) return e;
         prologue_kernel<float><<<(unsigned)blocks, kProThreads, smem, stream>>>(A);
