@@ -17,10 +17,12 @@
 // The pass is HBM-bound: per token and head it reads the raw q/k/v
 // projections once and writes the recurrence's q/k/v once.  Roles by block:
 //
-//   conv blocks   persistent warps over (tensor, 128-channel block, run of
-//                 eight tokens) items.  Each warp keeps its own three-stage
-//                 cp.async ring of window rows (the run's eight and the three
-//                 before it) in shared memory, two runs ahead of the one it
+//   conv blocks   persistent warps, each over a contiguous range of (tensor,
+//                 128-channel block, run of eight tokens) items numbered block
+//                 by block, so a warp walks along one channel block run after
+//                 run and carries each run's last three inputs into the next.
+//                 Each warp keeps its own three-stage cp.async ring of window
+//                 rows in shared memory, two runs ahead of the one it
 //                 computes, so the bytes in flight cost no registers and no
 //                 block barrier couples the warps.  Lane l owns channels
 //                 4l..4l+3; the run's outputs are computed on the packed
@@ -163,17 +165,20 @@ __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
 }
 
-// One work item: (tensor, 128-channel block, run of kProRun tokens).
+// One work item: (tensor, 128-channel block, run of kProRun tokens).  Items
+// are numbered channel block by channel block, so consecutive items are
+// consecutive runs of one block (and a new block starts at token 0).
 struct ProItem {
-    int which, cb, tr, te, C;
+    int cbg, which, cb, tr, te, C;
 };
 
 __device__ __forceinline__ ProItem item_of(const ProArgs &A, int item) {
     ProItem it;
-    const int run = item / A.nball, cbg = item % A.nball;
-    if (cbg < A.nbq) { it.which = 0; it.cb = cbg; }
-    else if (cbg < 2 * A.nbq) { it.which = 1; it.cb = cbg - A.nbq; }
-    else { it.which = 2; it.cb = cbg - 2 * A.nbq; }
+    const int run = item % A.runs;
+    it.cbg = item / A.runs;
+    if (it.cbg < A.nbq) { it.which = 0; it.cb = it.cbg; }
+    else if (it.cbg < 2 * A.nbq) { it.which = 1; it.cb = it.cbg - A.nbq; }
+    else { it.which = 2; it.cb = it.cbg - 2 * A.nbq; }
     it.C = it.which == 2 ? A.Cv : A.Cq;
     it.tr = run * kProRun;
     it.te = min(it.tr + kProRun, A.total_T);
@@ -182,9 +187,11 @@ __device__ __forceinline__ ProItem item_of(const ProArgs &A, int item) {
 
 // One warp copies the rows tr-3 .. te-1 (those inside [0, total_T)) of the
 // item's 128 channels into one of its stages: row r holds token tr - 3 + r.
+// Without `halo` the three rows before the run are skipped: the warp carries
+// them in registers from the run before.
 template <typename IoT>
 __device__ __forceinline__ void issue_run(const ProArgs &A, const ProItem &it, uint8_t *stage,
-                                          int lane) {
+                                          int lane, bool halo) {
     const IoT *x = static_cast<const IoT *>(it.which == 0 ? A.xq : it.which == 1 ? A.xk : A.xv);
     const int width = min(128, it.C - it.cb * 128);          // channels (multiple of 16)
     constexpr int kRowBytes = 128 * (int)sizeof(IoT);
@@ -192,7 +199,8 @@ __device__ __forceinline__ void issue_run(const ProArgs &A, const ProItem &it, u
     const int pieces = width * (int)sizeof(IoT) / 16;        // of this block's rows
     const uint8_t *base = reinterpret_cast<const uint8_t *>(x + it.cb * 128);
     const size_t pitch = (size_t)it.C * sizeof(IoT);
-    for (int i = lane; i < kProRows * kPieces; i += 32) {
+    const int r0 = halo ? 0 : 3;
+    for (int i = lane + r0 * kPieces; i < kProRows * kPieces; i += 32) {
         const int r = i / kPieces, p = i % kPieces;
         const int t = it.tr - 3 + r;
         if (t < 0 || t >= it.te || p >= pieces) continue;
@@ -203,43 +211,39 @@ __device__ __forceinline__ void issue_run(const ProArgs &A, const ProItem &it, u
 __device__ __forceinline__ void lds4(const float *p, float (&x)[4]) { load4(p, x); }
 __device__ __forceinline__ void lds4(const __nv_bfloat16 *p, float (&x)[4]) { load4(p, x); }
 
-// Outputs of a run's tokens: the warp loads the run's kProRun + 3 window rows
-// from its stage once, computes the outputs in place (token s reads rows
-// s..s+3 only, so oldest first frees row s), and reduces the kProRun head
-// norms together, xor-shuffle sums over the d_k / 4 lanes of a head.  Inputs before a token's sequence come from the
-// incoming state (zeros without one).
+// Outputs of a run's tokens: the warp takes the run's window rows (the three
+// before it carried from the run before unless `halo`), computes the kProRun
+// outputs (token s reads rows s..s+3 only), and reduces the kProRun head norms
+// together, xor-shuffle sums over the d_k / 4 lanes of a head.  Inputs before
+// a token's sequence come from the incoming state (zeros without one).  On
+// return rows 0..2 hold the run's last three inputs, the next run's carry.
 template <typename IoT>
 __device__ __forceinline__ void compute_run(const ProArgs &A, const ProItem &it,
-                                            const uint8_t *stage, int lane) {
+                                            const uint8_t *stage, int lane, bool halo,
+                                            const float (&tap)[4][4], float (&xr)[kProRows][4],
+                                            int &n0, int &a0, int &b0) {
     const int c = it.cb * 128 + 4 * lane;
     const bool live = c < it.C;
     const bool normed = A.norm && it.which < 2;
     const int group = A.dk / 4;
     const int choff = it.which * A.Cq;
-    const float *w = it.which == 0 ? A.wq : it.which == 1 ? A.wk : A.wv;
     IoT *y = static_cast<IoT *>(it.which == 0 ? A.q : it.which == 1 ? A.k : A.v);
     const IoT *rows = reinterpret_cast<const IoT *>(stage);
     const int tr = it.tr, te = it.te;
 
-    float tap[4][4];
+    // window rows: the three before the run from the stage (halo) or carried
+    // from the run before, the run's own from the stage
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        float t4[4] = {0.f, 0.f, 0.f, 0.f};
-        if (live) load4(w + (size_t)(c + j) * 4, t4);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) tap[j][i] = t4[i];
-    }
-    float xr[kProRun + 3][4];                        // tokens tr-3 .. tr+kProRun-1
-#pragma unroll
-    for (int r = 0; r < kProRun + 3; ++r) {
+    for (int r = 0; r < kProRows; ++r) {
+        if (r < 3 && !halo) continue;
 #pragma unroll
         for (int j = 0; j < 4; ++j) xr[r][j] = 0.f;
         if (live) lds4(rows + r * 128 + 4 * lane, xr[r]);
     }
     // rows before a token's sequence: the incoming state, or zeros
-    int a0, b0;
-    const int n0 = seq_of(A, tr, a0, b0);
-    if (!(tr >= a0 + 3 && te <= b0)) {
+    if (!(tr >= a0 && tr < b0)) n0 = seq_of(A, tr, a0, b0);   // cached across runs
+    const bool fast = tr >= a0 + 3 && te <= b0;
+    if (!fast) {
 #pragma unroll
         for (int s = 0; s < kProRun; ++s) {
             const int t = tr + s;
@@ -288,8 +292,7 @@ __device__ __forceinline__ void compute_run(const ProArgs &A, const ProItem &it,
             }
             if (live) store4(y + (size_t)t * it.C + c, o);
         }
-        return;
-    }
+    } else {
     // the whole run lies at least three tokens inside one sequence: pairs of
     // channels on the packed fp32x2 units
     float2 tp[2][4];                                 // [channel pair][tap]
@@ -368,37 +371,64 @@ __device__ __forceinline__ void compute_run(const ProArgs &A, const ProItem &it,
             out += it.C;
         }
     }
+    }
+    // carry: the inputs at tr+5 .. tr+7 are the next run's rows 0..2
+#pragma unroll
+    for (int r = 0; r < 3; ++r)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) xr[r][j] = xr[kProRun + r][j];
 }
 
-// Persistent warps: each walks over its work items with its own ring of
-// kProStages stages, the copies of its next kProStages - 1 runs in flight
-// while it computes this one.  cp.async groups belong to the issuing thread,
-// so a warp waits for its own copies and needs no block barrier; __syncwarp
-// makes the lanes' copies visible to each other and protects a stage until
-// every lane is done with it.
+// Persistent warps: warp g takes the contiguous items [g per, (g+1) per), so
+// it walks along one channel block run after run (a new block starts at
+// token 0) and carries each run's last three inputs into the next; only its
+// first item copies the three rows before the run.  Each warp has its own
+// ring of kProStages stages, the copies of its next kProStages - 1 runs in
+// flight while it computes this one.  cp.async groups belong to the issuing
+// thread, so a warp waits for its own copies and needs no block barrier;
+// __syncwarp makes the lanes' copies visible to each other and protects a
+// stage until every lane is done with it.
 template <typename IoT>
 __device__ void conv_warps(const ProArgs &A, uint8_t *smem) {
     constexpr int kStageBytes = kProRows * 128 * (int)sizeof(IoT);
     const int lane = threadIdx.x % 32, warp = threadIdx.x / 32;
     uint8_t *ring = smem + warp * kProStages * kStageBytes;
     const int items = A.runs * A.nball;
-    const int first = blockIdx.x * kProWarps + warp, stride = A.conv_blocks * kProWarps;
-    const int mine = items > first ? (items - 1 - first) / stride + 1 : 0;
+    const int nw = A.conv_blocks * kProWarps;
+    const int per = (items + nw - 1) / nw;
+    const int lo = min((blockIdx.x * kProWarps + warp) * per, items);
+    const int mine = min(lo + per, items) - lo;
 #pragma unroll
     for (int j = 0; j < kProStages - 1; ++j) {
-        if (j < mine) issue_run<IoT>(A, item_of(A, first + j * stride), ring + j * kStageBytes, lane);
+        if (j < mine) issue_run<IoT>(A, item_of(A, lo + j), ring + j * kStageBytes, lane, j == 0);
         cp_async_commit();
     }
+    float tap[4][4] = {};
+    float xr[kProRows][4] = {};
+    int tap_cbg = -1, n0 = 0, a0 = 0, b0 = -1;   // taps and sequence range held across runs
     for (int j = 0; j < mine; ++j) {
         const int jn = j + kProStages - 1;
         if (jn < mine)
-            issue_run<IoT>(A, item_of(A, first + jn * stride), ring + (jn % kProStages) * kStageBytes,
-                           lane);
+            issue_run<IoT>(A, item_of(A, lo + jn), ring + (jn % kProStages) * kStageBytes, lane,
+                           false);
         cp_async_commit();
         cp_async_wait<kProStages - 1>();   // run j has landed (groups complete in order)
         __syncwarp();
-        compute_run<IoT>(A, item_of(A, first + j * stride), ring + (j % kProStages) * kStageBytes,
-                         lane);
+        const ProItem it = item_of(A, lo + j);
+        if (it.cbg != tap_cbg) {
+            tap_cbg = it.cbg;
+            const float *w = it.which == 0 ? A.wq : it.which == 1 ? A.wk : A.wv;
+            const int c = it.cb * 128 + 4 * lane;
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                float t4[4] = {0.f, 0.f, 0.f, 0.f};
+                if (c < it.C) load4(w + (size_t)(c + jj) * 4, t4);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) tap[jj][i] = t4[i];
+            }
+        }
+        compute_run<IoT>(A, it, ring + (j % kProStages) * kStageBytes, lane, j == 0, tap, xr, n0,
+                         a0, b0);
         __syncwarp();
     }
 }
