@@ -8,6 +8,8 @@ the CUDA path, and nothing here imports it.
                      per core over independent (sequence, head) pairs).
 * ``brute_force`` -- an independent expansion of the recurrence into explicit
                      d_k x d_k transition matrices, used to pin the loop.
+* ``backward``    -- the gradient of the recurrence (reverse token sweep, numpy
+                     float64), pinned by finite differences of ``run``.
 * ``prologue``    -- the input-side prologue (short causal convolution with its
                      state, q/k L2 normalisation, gate and beta maps) in numpy
                      float64.
@@ -19,3 +21,4 @@ the cache" (Gated DeltaNet and Kimi Delta Attention equations).
 from .loop import run, build, library_path  # noqa: F401
 from . import brute_force  # noqa: F401
 from . import prologue  # noqa: F401
+from . import backward  # noqa: F401
