@@ -417,7 +417,69 @@ class PrologueCase:
         return "f32 arithmetic, bf16 in and out"
 
 
+class BackwardCase:
+    """The gradient of the recurrence at the gdn_prefill shape: one
+    gdr_backward call per step (upstream gradients dO and dS_final drawn by
+    the input module)."""
+    kind = "backward"
+    kernel_label = "backward (forward sweep with a checkpoint every 16 tokens, reverse sweep)"
+
+    def __init__(self, name, device, seed):
+        self.name = name
+        self.inp = inp = I.workload("gdn_prefill", seed=seed)
+        dO, dsf = I.make_grad_inputs(inp, seed=seed)
+        self.dev = device
+        self.d = {k: (None if v is None else v.to(device)) for k, v in dict(
+            q=inp.q, k=inp.k, v=inp.v, g=inp.g, beta=inp.beta, h0=inp.h0, cu=inp.cu_seqlens,
+            dO=dO, dsf=dsf).items()}
+        nbytes = gdr.gdr_backward_workspace_size(inp.num_seqs, inp.total_T, inp.H, inp.d_k,
+                                                 inp.d_v)
+        self.ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=device)
+        e = io_bytes(inp.io_dtype)
+        T, H, Hqk, dk, dv, N = inp.total_T, inp.H, inp.H_qk, inp.d_k, inp.d_v, inp.num_seqs
+        gate = inp.g.numel() * 4
+        state = N * H * dv * dk * 4
+        # read q, k, v, dO, g, beta, dS_final (h0 when given); write dq, dk, dv (fp32), dg,
+        # dbeta, d_initial_state
+        self.bytes = (T * (2 * Hqk * dk + 2 * H * dv) * e + 2 * gate + 2 * T * H * 4
+                      + (2 if inp.h0 is not None else 1) * state
+                      + T * (2 * Hqk * dk + H * dv) * 4 + state)
+        self.flops = 0
+        self.tokens = T
+        self.launches = 1
+        self.path = None
+        self.out = None
+
+    def _call(self, d, stream):
+        self.out = gdr.gdr_backward(d["q"], d["k"], d["v"], d["g"], d["beta"], d.get("h0"),
+                                    d["cu"], d_o=d["dO"], d_final_state=d.get("dsf"),
+                                    workspace=self.ws, stream=stream)
+
+    def step(self, stream=None):
+        self._call(self.d, stream)
+
+    def e2e_buffers(self):
+        host = {k: v.cpu().pin_memory() for k, v in self.d.items() if v is not None}
+        if self.out is None:
+            self.step()
+        ho = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in self.out if o is not None]
+        h2d = sum(v.numel() * v.element_size() for v in host.values())
+        d2h = sum(o.numel() * o.element_size() for o in ho)
+        return host, ho, None, h2d, d2h
+
+    def e2e_step(self, host, host_o, host_fin, stream):
+        dev = {k: v.to(self.dev, non_blocking=True) for k, v in host.items()}
+        self._call(dev, stream)
+        for h, o in zip(host_o, [o for o in self.out if o is not None]):
+            h.copy_(o, non_blocking=True)
+
+    def dtype_label(self):
+        return "f32 arithmetic and gradients, bf16 inputs"
+
+
 def make_case(name, device, seed):
+    if name == "backward_gdn":
+        return BackwardCase(name, device, seed)
     if name == "prologue_gdn":
         return PrologueCase(name, device, seed)
     if name == "decode_spec_gdn":
@@ -644,7 +706,7 @@ def main():
     args = ap.parse_args()
     if args.workloads == "all":
         args.workloads = ("gdn_prefill,kda_prefill,varlen_gdn,gqa_prefill,decode_gdn,decode_kda,"
-                          "decode_spec_gdn,prologue_gdn")
+                          "decode_spec_gdn,prologue_gdn,backward_gdn")
     if args.warmup < 3:
         args.warmup = 3
     ws, rank, local = dist_env()

@@ -279,4 +279,72 @@ gdr_status_t gdr_prologue(const void *xq, const void *xk, const void *xv, const 
         beta, static_cast<cudaStream_t>(stream)));
 }
 
+gdr_status_t gdr_backward_workspace_size(int32_t num_seqs, int32_t total_T, int32_t H,
+                                         int32_t d_k, int32_t d_v, size_t *bytes) {
+    if (bytes == nullptr || num_seqs < 0 || total_T < 0 || H < 0 || !valid_dim(d_k) ||
+        !valid_dim(d_v))
+        return GDR_ERR_INVALID_ARG;
+    *bytes = gdr::backward_workspace_bytes(num_seqs, total_T, H, d_k, d_v);
+    return GDR_OK;
+}
+
+gdr_status_t gdr_backward(const void *q, const void *k, const void *v, const float *g,
+                          const float *beta, const float *initial_state, const int32_t *cu_seqlens,
+                          int32_t num_seqs, int32_t total_T, int32_t H_qk, int32_t H, int32_t d_k,
+                          int32_t d_v, gdr_gate_mode_t gate_mode, gdr_dtype_t io_dtype,
+                          const void *d_o, const float *d_final_state, float *dq, float *dk,
+                          float *dv, float *dg, float *dbeta, float *d_initial_state,
+                          void *workspace, size_t workspace_bytes, void *stream) {
+    if (num_seqs < 1 || total_T < 0 || H < 1 || H_qk < 1 || H % H_qk != 0)
+        return GDR_ERR_INVALID_ARG;
+    if (!valid_dim(d_k) || !valid_dim(d_v)) return GDR_ERR_INVALID_ARG;
+    if (gate_mode != GDR_GATE_SCALAR && gate_mode != GDR_GATE_CHANNEL) return GDR_ERR_INVALID_ARG;
+    if (io_dtype != GDR_F32 && io_dtype != GDR_BF16) return GDR_ERR_INVALID_ARG;
+    if (cu_seqlens == nullptr && total_T % num_seqs != 0) return GDR_ERR_INVALID_ARG;
+    if ((int64_t)num_seqs * H * ((d_v + 15) / 16) > INT32_MAX) return GDR_ERR_INVALID_ARG;
+    if (!ok_opt_ptr(initial_state) || !ok_opt_ptr(d_final_state) || !ok_opt_ptr(d_initial_state))
+        return GDR_ERR_INVALID_ARG;
+    if (cu_seqlens != nullptr && !aligned4(cu_seqlens)) return GDR_ERR_INVALID_ARG;
+    if (total_T > 0) {
+        if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(d_o) || !ok_ptr(dq) || !ok_ptr(dk) ||
+            !ok_ptr(dv) || !ok_gate_ptr(g, gate_mode) || !ok_gate_ptr(dg, gate_mode) ||
+            !ok_beta_ptr(beta) || !ok_beta_ptr(dbeta))
+            return GDR_ERR_INVALID_ARG;
+    }
+    const size_t need = gdr::backward_workspace_bytes(num_seqs, total_T, H, d_k, d_v);
+    if (need > 0 && (workspace == nullptr || workspace_bytes < need || !aligned16(workspace)))
+        return GDR_ERR_WORKSPACE;
+    // no output may overlap an input or another output
+    const size_t e = io_dtype == GDR_BF16 ? 2 : 4, T = (size_t)total_T;
+    const size_t nq = T * H_qk * d_k, nv = T * H * d_v, ng = T * H * (gate_mode == GDR_GATE_CHANNEL ? d_k : 1);
+    const size_t ns = (size_t)num_seqs * H * d_v * d_k * 4;
+    struct Range {
+        const void *p;
+        size_t n;
+    };
+    const Range in[] = {{q, nq * e}, {k, nq * e}, {v, nv * e}, {g, ng * 4}, {beta, T * H * 4},
+                        {initial_state, ns}, {d_o, nv * e}, {d_final_state, ns},
+                        {cu_seqlens, cu_seqlens ? ((size_t)num_seqs + 1) * 4 : 0}};
+    const Range out[] = {{dq, nq * 4}, {dk, nq * 4}, {dv, nv * 4}, {dg, ng * 4},
+                         {dbeta, T * H * 4}, {d_initial_state, ns}, {workspace, need}};
+    for (const Range &o : out) {
+        if (o.p == nullptr || o.n == 0) continue;
+        const uintptr_t o0 = reinterpret_cast<uintptr_t>(o.p), o1 = o0 + o.n;
+        for (const Range &i : in) {
+            if (i.p == nullptr || i.n == 0) continue;
+            const uintptr_t i0 = reinterpret_cast<uintptr_t>(i.p), i1 = i0 + i.n;
+            if (o0 < i1 && i0 < o1) return GDR_ERR_INVALID_ARG;
+        }
+        for (const Range &o2 : out) {
+            if (&o2 == &o || o2.p == nullptr || o2.n == 0) continue;
+            const uintptr_t a0 = reinterpret_cast<uintptr_t>(o2.p), a1 = a0 + o2.n;
+            if (o0 < a1 && a0 < o1) return GDR_ERR_INVALID_ARG;
+        }
+    }
+    return from_cuda(gdr::launch_backward(
+        q, k, v, g, beta, initial_state, cu_seqlens, num_seqs, total_T, H_qk, H, d_k, d_v,
+        gate_mode == GDR_GATE_CHANNEL, io_dtype == GDR_BF16, d_o, d_final_state, dq, dk, dv, dg,
+        dbeta, d_initial_state, workspace, static_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

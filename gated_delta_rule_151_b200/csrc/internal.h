@@ -13,6 +13,15 @@ cudaError_t launch_decode_step(const void *q, const void *k, const void *v, cons
                                const float *beta, float *state, int N, int Hqk, int H, int DK,
                                int DV, bool channel, bool bf16, void *o, cudaStream_t stream);
 
+// Gradient of the recurrence: workspace for the state checkpoints, launcher.
+size_t backward_workspace_bytes(int num_seqs, int total_T, int H, int DK, int DV);
+cudaError_t launch_backward(const void *q, const void *k, const void *v, const float *g,
+                            const float *beta, const float *h0, const int32_t *cu, int num_seqs,
+                            int total_T, int Hqk, int H, int DK, int DV, bool channel, bool bf16,
+                            const void *dO, const float *dSf, float *dq, float *dk, float *dv,
+                            float *dg, float *dbeta, float *dh0, void *workspace,
+                            cudaStream_t stream);
+
 // Input-side prologue: short causal convolution with state, q/k
 // normalisation, gate and beta maps (arguments validated by the C ABI).
 cudaError_t launch_prologue(const void *xq, const void *xk, const void *xv, const float *wq,

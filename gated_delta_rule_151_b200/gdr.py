@@ -38,7 +38,8 @@ GDR_PROLOGUE_NORMALIZE_QK = 2
 EXPORTED = ("gdr_status_string", "gdr_prefill_workspace_size", "gdr_prefill_path",
             "gdr_prefill_chunked", "gdr_prefill_check_workspace", "gdr_decode_step",
             "gdr_prefill_chunked_noalloc", "gdr_prefill_chunked_gqa", "gdr_decode_step_gqa",
-            "gdr_decode_multi", "gdr_prefill_plan", "gdr_prologue")
+            "gdr_decode_multi", "gdr_prefill_plan", "gdr_prologue", "gdr_backward",
+            "gdr_backward_workspace_size")
 
 
 class GdrError(RuntimeError):
@@ -93,6 +94,10 @@ def load_library():
         lib.gdr_decode_multi.restype = ST
         lib.gdr_prologue.argtypes = [P] * 12 + [I32] * 6 + [ST, ST, ctypes.c_uint32] + [P] * 6
         lib.gdr_prologue.restype = ST
+        lib.gdr_backward_workspace_size.argtypes = [I32, I32, I32, I32, I32, ctypes.POINTER(SZ)]
+        lib.gdr_backward_workspace_size.restype = ST
+        lib.gdr_backward.argtypes = [P] * 7 + [I32] * 6 + [ST, ST] + [P] * 9 + [SZ, P]
+        lib.gdr_backward.restype = ST
         _lib = lib
         return lib
 
@@ -391,3 +396,60 @@ def gdr_prologue(xq, xk, xv, wq, wk, wv, xg, gscale, xb, conv_state_in=None, cu_
         _stream_ptr(stream))
     _check(st, "gdr_prologue")
     return q, k, v, g, beta
+
+
+def gdr_backward_workspace_size(num_seqs, total_T, H, d_k, d_v) -> int:
+    n = ctypes.c_size_t(0)
+    _check(load_library().gdr_backward_workspace_size(num_seqs, total_T, H, d_k, d_v,
+                                                      ctypes.byref(n)),
+           "gdr_backward_workspace_size")
+    return int(n.value)
+
+
+def gdr_backward(q, k, v, g, beta, initial_state=None, cu_seqlens=None, *, d_o,
+                 d_final_state=None, num_seqs=None, want_d_initial_state=True, workspace=None,
+                 stream=None):
+    """Gradient of <d_o, o> + <d_final_state, final_state> (see include/gdr.h).
+
+    Inputs as for gdr_prefill_chunked_gqa; d_o [T, H, d_v] in the io dtype;
+    d_final_state [N, H, d_v, d_k] fp32 or None.  Returns (dq, dk, dv, dg,
+    dbeta, d_initial_state) as fp32 tensors (the last None unless wanted).
+    """
+    _need(q, "q", ndim=3)
+    io = q.dtype
+    _need(k, "k", io, 3)
+    _need(v, "v", io, 3)
+    _need(d_o, "d_o", io, 3)
+    _need(beta, "beta", torch.float32, 2)
+    _need(g, "g", torch.float32)
+    T, Hqk, dk = q.shape
+    H, dv = v.shape[1], v.shape[2]
+    gate = GDR_GATE_SCALAR if g.dim() == 2 else GDR_GATE_CHANNEL
+    if cu_seqlens is not None:
+        _need(cu_seqlens, "cu_seqlens", torch.int32, 1)
+        n = cu_seqlens.numel() - 1
+    else:
+        n = 1 if num_seqs is None else int(num_seqs)
+    if initial_state is not None:
+        _need(initial_state, "initial_state", torch.float32, 4)
+    if d_final_state is not None:
+        _need(d_final_state, "d_final_state", torch.float32, 4)
+    dev = q.device
+    f32 = dict(dtype=torch.float32, device=dev)
+    dq = torch.empty((T, Hqk, dk), **f32)
+    dk_ = torch.empty((T, Hqk, dk), **f32)
+    dv_ = torch.empty((T, H, dv), **f32)
+    dg = torch.empty(g.shape, **f32)
+    db = torch.empty((T, H), **f32)
+    dh0 = torch.empty((n, H, dv, dk), **f32) if want_d_initial_state else None
+    need = gdr_backward_workspace_size(n, T, H, dk, dv)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    wsb = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = load_library().gdr_backward(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(initial_state), _ptr(cu_seqlens),
+        n, T, Hqk, H, dk, dv, gate, _io_code(io), _ptr(d_o), _ptr(d_final_state), _ptr(dq),
+        _ptr(dk_), _ptr(dv_), _ptr(dg), _ptr(db), _ptr(dh0), _ptr(workspace), wsb,
+        _stream_ptr(stream))
+    _check(st, "gdr_backward")
+    return dq, dk_, dv_, dg, db, dh0

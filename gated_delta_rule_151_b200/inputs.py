@@ -40,6 +40,8 @@ decode_gdn/kda     256 sequences, H=32, d=128, 512 steps of one bf16 token,
                    c=0.1, h0 ~ N(0, 0.02^2) (state 512 MiB fp32)
 decode_spec_gdn    the decode_gdn tokens verified 4 at a time (128 steps of
                    4 draft tokens per sequence)
+backward_gdn       the gdn_prefill inputs with upstream gradients dO ~ N(0, 1)
+                   (bf16) and dS_final ~ N(0, 1) for the gradient
 prologue_gdn       raw prologue inputs at the gdn_prefill shape (1 x 8192
                    tokens, H=16, d=128, bf16): x_q, x_k, x_v ~ N(0, 1), taps
                    ~ N(0, 0.5^2), convolution state ~ N(0, 1), x_g, x_beta
@@ -67,7 +69,9 @@ BLOCK_ELEMS = 1 << 21
 _ID = {"q": 0, "k": 1, "v": 2, "beta": 3, "gate": 4, "h0": 5, "cuts": 6,
        # raw inputs of the prologue (before the convolution and the maps)
        "xq": 7, "xk": 8, "xv": 9, "wq": 10, "wk": 11, "wv": 12, "xg": 13, "xb": 14,
-       "conv": 15}
+       "conv": 15,
+       # upstream gradients of the backward pass
+       "do": 16, "dsf": 17}
 
 SCALAR = "scalar"    # Gated DeltaNet: one gate per head and token
 CHANNEL = "channel"  # Kimi Delta Attention: one gate per key channel
@@ -355,7 +359,8 @@ def make_prologue_inputs(*, total_T: int, H: int, d_k: int, d_v: int | None = No
 # ---------------------------------------------------------------------------
 
 WORKLOADS = ("tiny_gdn", "gdn_prefill", "kda_prefill", "decode_gdn",
-             "decode_kda", "varlen_gdn", "gqa_prefill", "decode_spec_gdn", "prologue_gdn")
+             "decode_kda", "varlen_gdn", "gqa_prefill", "decode_spec_gdn", "prologue_gdn",
+             "backward_gdn")
 
 SPEC_DRAFT = 4   # tokens verified per sequence per step in decode_spec_gdn
 
@@ -397,6 +402,21 @@ def workload(name: str, seed: int = 0) -> Inputs:
                            gate_mode=SCALAR, io_dtype=torch.bfloat16, c=0.1,
                            seed=seed, meta={"workload": name})
     raise KeyError(name)
+
+
+def make_grad_inputs(inp: Inputs, seed: int = 0, dsf_std: float = 1.0):
+    """Upstream gradients for the backward pass of ``inp``: dO [total_T, H,
+    d_v] ~ N(0, 1) rounded to the I/O type, and dS_final [num_seqs, H, d_v,
+    d_k] ~ N(0, dsf_std^2) in float32 (None when dsf_std is 0)."""
+    dO = _fill(seed, "do", (inp.total_T, inp.H, inp.d_v), lambda x: x, np.float32)
+    dO = torch.from_numpy(dO)
+    if inp.io_dtype != torch.float32:
+        dO = dO.to(inp.io_dtype)
+    dsf = None
+    if dsf_std > 0.0:
+        dsf = torch.from_numpy(_fill(seed, "dsf", (inp.num_seqs, inp.H, inp.d_v, inp.d_k),
+                                     lambda x: x * dsf_std, np.float32))
+    return dO, dsf
 
 
 def prologue_workload(name: str = "prologue_gdn", seed: int = 0) -> PrologueInputs:

@@ -327,6 +327,44 @@ GDR_API gdr_status_t gdr_prologue(const void *xq, const void *xk, const void *xv
                                   gdr_gate_mode_t gate_mode, gdr_dtype_t io_dtype, uint32_t flags,
                                   void *q, void *k, void *v, float *g, float *beta, void *stream);
 
+/*
+ * Gradient of the recurrence (training).  The pages train these layers but
+ * print no backward pass; this is the gradient of the rule at the top of this
+ * header, for the loss
+ *
+ *     L = sum_t <d_o_t, o_t> + sum_n <d_final_state_n, final_state_n>
+ *
+ * with respect to q, k, v, g, beta and the initial state.  Inputs are those
+ * of gdr_prefill_chunked_gqa (same layouts, dtypes and cu_seqlens rules);
+ * d_o is [total_T, H, d_v] in the io dtype; d_final_state [N, H, d_v, d_k]
+ * fp32 or NULL (zeros).  Outputs, all fp32 and overwritten:
+ *   dq, dk            [total_T, H_qk, d_k]  (summed over the value heads of a group)
+ *   dv                [total_T, H, d_v]
+ *   dg                [total_T, H] or [total_T, H, d_k]   (zero where g was clamped at -20)
+ *   dbeta             [total_T, H]
+ *   d_initial_state   [N, H, d_v, d_k], or NULL to skip
+ * The workspace (gdr_backward_workspace_size bytes, 16-byte aligned) holds
+ * the state checkpointed every 16 tokens: (N + ceil(total_T / 16)) * H *
+ * d_v * d_k * 4 bytes.  Pointers: q, k, v, d_o, the states, dq, dk, dv and
+ * channel-mode g/dg 16-byte aligned; the rest 4-byte aligned.  Outputs must
+ * not overlap inputs.  Errors: GDR_ERR_INVALID_ARG (size, pointer, overlap),
+ * GDR_ERR_WORKSPACE (missing or too small), GDR_ERR_CUDA; nothing is launched
+ * on error.  Sums over rows use floating-point atomics, so the last bits of
+ * dq, dk, dg and dbeta may differ from run to run.
+ */
+GDR_API gdr_status_t gdr_backward_workspace_size(int32_t num_seqs, int32_t total_T, int32_t H,
+                                                 int32_t d_k, int32_t d_v, size_t *bytes);
+
+GDR_API gdr_status_t gdr_backward(const void *q, const void *k, const void *v, const float *g,
+                                  const float *beta, const float *initial_state,
+                                  const int32_t *cu_seqlens, int32_t num_seqs, int32_t total_T,
+                                  int32_t H_qk, int32_t H, int32_t d_k, int32_t d_v,
+                                  gdr_gate_mode_t gate_mode, gdr_dtype_t io_dtype,
+                                  const void *d_o, const float *d_final_state, float *dq,
+                                  float *dk, float *dv, float *dg, float *dbeta,
+                                  float *d_initial_state, void *workspace,
+                                  size_t workspace_bytes, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

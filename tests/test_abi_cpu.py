@@ -212,3 +212,42 @@ def test_prologue_rejects_invalid_arguments(lib, kw):
 def test_prologue_empty_problem_is_a_no_op(lib):
     assert _prologue(lib, T=0, xq=None, xk=None, xv=None, q=None, k=None, v=None, xg=None,
                      g=None, xb=None, beta=None) == gdr.GDR_OK
+
+
+_BW_NAMES = ("q", "k", "v", "g", "beta", "h0", "cu", "do", "dsf", "gq", "gk", "gv", "gg", "gb",
+             "gh0", "ws")   # gX: the gradient output for X
+_BW = {n: _PRO_BASE + ((i + 20) << 30) for i, n in enumerate(_BW_NAMES)}
+
+
+def _backward(lib, **kw):
+    args = dict(_BW)
+    args.update(h0=None, cu=None, dsf=None, gh0=None, N=1, T=64, Hqk=2, H=2, dk=16, dv=16,
+                gate=0, io=0, wsb=1 << 30)
+    args.update(kw)
+    P = lambda x: None if x is None else ctypes.c_void_p(x)
+    return lib.gdr_backward(*(P(args[n]) for n in _BW_NAMES[:7]), args["N"], args["T"],
+                            args["Hqk"], args["H"], args["dk"], args["dv"], args["gate"],
+                            args["io"], *(P(args[n]) for n in _BW_NAMES[7:]), args["wsb"], None)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(q=None), dict(do=None), dict(gq=None), dict(gv=None), dict(gg=None), dict(gb=None),
+    dict(q=_BW["q"] + 2), dict(gq=_BW["gq"] + 4), dict(g=_BW["g"] + 2),
+    dict(g=_BW["g"] + 4, gate=1), dict(gh0=_BW["gh0"] + 4), dict(cu=_BW["cu"] + 2),
+    dict(dk=48), dict(dv=256), dict(H=0), dict(Hqk=3), dict(N=0), dict(T=-1), dict(N=3),
+    dict(gate=2), dict(io=5),
+    dict(gq=_BW["q"]), dict(gv=_BW["v"] + 64), dict(gb=_BW["beta"]), dict(gh0=_BW["gq"]),
+])
+def test_backward_rejects_invalid_arguments(lib, kw):
+    assert _backward(lib, **kw) == gdr.GDR_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("kw", [dict(ws=None), dict(wsb=16), dict(ws=_BW["ws"] + 8)])
+def test_backward_rejects_a_missing_or_small_workspace(lib, kw):
+    assert _backward(lib, **kw) == gdr.GDR_ERR_WORKSPACE
+
+
+def test_backward_workspace_size(lib):
+    # one state checkpoint per 16 tokens of every sequence, plus one per sequence
+    assert gdr.gdr_backward_workspace_size(2, 100, 3, 64, 32) == (2 + 7) * 3 * 32 * 64 * 4
+    assert gdr.gdr_backward_workspace_size(1, 8192, 16, 128, 128) == (1 + 512) * 16 * 65536
