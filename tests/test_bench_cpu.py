@@ -1,0 +1,72 @@
+"""Host logic of bench.py on the CPU: the reference arm's JSON line, the
+launch accounting of the pipelined chunk-parallel plan, and the algorithmic
+byte counts of the workloads (the roofline numerators), each against a count
+done by hand here."""
+import json
+import os
+import subprocess
+import sys
+
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from gated_delta_rule_151_b200 import inputs as I  # noqa: E402
+
+
+def test_reference_arm_prints_one_contract_line():
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--steps", "1", "--warmup", "1", "--workloads", "tiny_gdn"],
+                       capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["value"] > 0 and d["dtype"] == "f64"
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+
+
+def test_pipelined_plan_launch_accounting():
+    # 128 chunks in one window: pieces of 12, 16, 21, 27, 35 and the last 17;
+    # each piece is one prep and one chain launch
+    assert bench.split_launches(I.workload("gdn_prefill")) == 12
+    # 64 chains of 90,640-byte records in 1 GiB windows: 185 chunks per
+    # window.  cu_seqlens lives on the device, so the plan bounds a
+    # sequence's chunks by total_T / 64 = 1024: 6 windows, one piece each
+    # (the last three hold no chunk of these two 512-chunk sequences)
+    kda = I.workload("kda_prefill")
+    window = (1 << 30) // (64 * 90640)
+    assert window == 185
+    assert bench.split_launches(kda) == 2 * -(-1024 // window) == 12
+
+
+def test_prologue_bytes_per_launch():
+    case = bench.PrologueCase("prologue_gdn", torch.device("cpu"), seed=0)
+    T, C = 8192, 3 * 16 * 128
+    expect = (2 * T * C * 2          # x_q, x_k, x_v in; q, k, v out (bf16)
+              + C * 4 * 4            # taps
+              + 2 * T * 16 * 4       # x_g in, g out
+              + 2 * T * 16 * 4       # x_beta in, beta out
+              + 16 * 4               # gate coefficients
+              + 2 * C * 3 * 4)       # convolution state in and out
+    assert case.bytes == expect
+
+
+def test_backward_bytes_per_launch():
+    case = bench.BackwardCase("backward_gdn", torch.device("cpu"), seed=0)
+    T, H, d = 8192, 16, 128
+    act = T * H * d
+    expect = (4 * act * 2            # q, k, v, dO (bf16)
+              + 2 * T * H * 4        # g in, dg out
+              + 2 * T * H * 4        # beta in, dbeta out
+              + H * d * d * 4        # dS_final
+              + 3 * act * 4          # dq, dk, dv (fp32)
+              + H * d * d * 4)       # d_initial_state
+    assert case.bytes == expect
+    assert case.ws.numel() == (1 + T // 16) * H * d * d * 4
