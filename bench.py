@@ -182,7 +182,10 @@ def split_launches(inp):
     to 1 GiB at 90,640 bytes per chunk and head), and per pipeline piece when
     a single window is cut into pieces."""
     chains = inp.num_seqs * inp.H
-    max_chunks = -(-inp.total_T // 64)
+    # equal lengths go without cu_seqlens, so the library knows each
+    # sequence's length; otherwise total_T bounds it
+    longest = inp.total_T // inp.num_seqs if inp.equal_lengths() else inp.total_T
+    max_chunks = -(-longest // 64)
     window = max(1, min(max_chunks, (1 << 30) // (chains * 90640)))
     windows = -(-max_chunks // window)
     pieces = 1
@@ -202,9 +205,12 @@ class PrefillCase:
         self.name = name
         self.inp = inp = I.workload(name, seed=seed)
         self.dev = device
+        # equal-length batches go in the dense layout (no cu_seqlens), as a
+        # caller with a [B, T, H, d] batch would pass them
+        self.equal = inp.equal_lengths()
         self.d = {k: (None if v is None else v.to(device)) for k, v in dict(
             q=inp.q, k=inp.k, v=inp.v, g=inp.g, beta=inp.beta, h0=inp.h0,
-            cu=inp.cu_seqlens).items()}
+            cu=None if self.equal else inp.cu_seqlens).items()}
         self.o = torch.empty((inp.total_T, inp.H, inp.d_v), dtype=inp.io_dtype, device=device)
         self.fin = torch.empty((inp.num_seqs, inp.H, inp.d_v, inp.d_k), dtype=torch.float32,
                                device=device)
@@ -224,20 +230,24 @@ class PrefillCase:
 
     def step(self, stream=None):
         d = self.d
-        self._fn()(d["q"], d["k"], d["v"], d["g"], d["beta"], d["h0"], d["cu"], o=self.o,
-                   final_state=self.fin, workspace=self.ws, stream=stream)
+        self._fn()(d["q"], d["k"], d["v"], d["g"], d["beta"], d["h0"], d["cu"],
+                   num_seqs=self.inp.num_seqs, o=self.o, final_state=self.fin,
+                   workspace=self.ws, stream=stream)
 
     def host_inputs(self):
         inp = self.inp
-        xs = dict(q=inp.q, k=inp.k, v=inp.v, g=inp.g, beta=inp.beta, cu=inp.cu_seqlens)
+        xs = dict(q=inp.q, k=inp.k, v=inp.v, g=inp.g, beta=inp.beta)
+        if not self.equal:
+            xs["cu"] = inp.cu_seqlens
         if inp.h0 is not None:
             xs["h0"] = inp.h0
         return {k: v.pin_memory() for k, v in xs.items()}
 
     def e2e_step(self, host, host_o, host_fin, stream):
         dev = {k: v.to(self.dev, non_blocking=True) for k, v in host.items()}
-        self._fn()(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"], dev.get("h0"), dev["cu"],
-                   o=self.o, final_state=self.fin, workspace=self.ws, stream=stream)
+        self._fn()(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"], dev.get("h0"), dev.get("cu"),
+                   num_seqs=self.inp.num_seqs, o=self.o, final_state=self.fin,
+                   workspace=self.ws, stream=stream)
         host_o.copy_(self.o, non_blocking=True)
         host_fin.copy_(self.fin, non_blocking=True)
 

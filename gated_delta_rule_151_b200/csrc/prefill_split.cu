@@ -1522,11 +1522,16 @@ int piece_schedule(int max_chunks, int *bounds) {
     return n;
 }
 
-bool make_split_plan(int num_seqs, int total_T, int H, SplitPlan &p) {
+// With equal lengths (no cu_seqlens) every sequence has total_T / num_seqs
+// tokens; otherwise the lengths live on the device and total_T bounds them.
+// The equal-length plan never needs more workspace than the general one (its
+// window is no larger, and it needs the state area only when that one does).
+bool make_split_plan(int num_seqs, int total_T, int H, SplitPlan &p, bool equal_lengths = false) {
     const long long chains = (long long)num_seqs * H;
     if (chains < 1 || chains > kSplitMaxChains || total_T <= 0) return false;
     p.chains = (int)chains;
-    p.max_chunks = (total_T + C - 1) / C;   // no sequence has more chunks
+    const int longest = equal_lengths ? total_T / num_seqs : total_T;
+    p.max_chunks = (longest + C - 1) / C;   // no sequence has more chunks
     const size_t per = (size_t)p.chains * REC_BYTES;
     const size_t fit = kMaxRecordBytes / per;
     p.window = (int)(fit < 1 ? 1 : (fit < (size_t)p.max_chunks ? fit : (size_t)p.max_chunks));
@@ -1600,7 +1605,7 @@ cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, co
                                  int num_seqs, int total_T, int Hqk, int H, bool channel, void *o,
                                  float *fin, void *workspace, cudaStream_t stream) {
     SplitPlan p;
-    if (!make_split_plan(num_seqs, total_T, H, p)) return cudaErrorInvalidValue;
+    if (!make_split_plan(num_seqs, total_T, H, p, cu == nullptr)) return cudaErrorInvalidValue;
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     uint32_t *err = reinterpret_cast<uint32_t *>(ws);
     cudaError_t e = cudaMemsetAsync(err, 0, sizeof(uint32_t), stream);

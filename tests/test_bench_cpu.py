@@ -37,13 +37,15 @@ def test_pipelined_plan_launch_accounting():
     # each piece is one prep and one chain launch
     assert bench.split_launches(I.workload("gdn_prefill")) == 12
     # 64 chains of 90,640-byte records in 1 GiB windows: 185 chunks per
-    # window.  cu_seqlens lives on the device, so the plan bounds a
-    # sequence's chunks by total_T / 64 = 1024: 6 windows, one piece each
-    # (the last three hold no chunk of these two 512-chunk sequences)
+    # window.  The two equal sequences go without cu_seqlens, so the plan
+    # knows each has 512 chunks: 3 windows, one piece each
     kda = I.workload("kda_prefill")
     window = (1 << 30) // (64 * 90640)
     assert window == 185
-    assert bench.split_launches(kda) == 2 * -(-1024 // window) == 12
+    assert bench.split_launches(kda) == 2 * -(-512 // window) == 6
+    # with packed lengths only total_T bounds a sequence: varlen has 128
+    # chains, beyond the plan, so only the counting is checked here
+    assert bench.split_launches(I.workload("gqa_prefill")) == 12
 
 
 def test_prologue_bytes_per_launch():

@@ -286,3 +286,19 @@ def test_chunk_parallel_plan_in_pipelined_pieces(mode):
     o, fin = gpu_prefill(inp)
     o_ref, fin_ref = oracle_prefill(inp)
     check(inp, o, fin, o_ref, fin_ref, "pieces")
+
+
+@pytest.mark.parametrize("mode", [I.SCALAR, I.CHANNEL])
+def test_equal_lengths_plan_knows_each_sequence_length(mode):
+    # 2 x 6000 tokens x 32 heads: with cu_seqlens the plan bounds a sequence
+    # by all 12000 tokens (188 chunks: two windows of 185); without it each
+    # sequence has 94 chunks (one window, pipelined pieces).  Both match the
+    # oracle, and the two runs agree.
+    inp = I.make_inputs(total_T=12000, H=32, d_k=128, num_seqs=2, gate_mode=mode,
+                        io_dtype=torch.bfloat16, c=0.05, h0_std=0.02, seed=90)
+    o1, f1 = gpu_prefill(inp, use_cu=True)
+    o2, f2 = gpu_prefill(inp, use_cu=False)
+    o_ref, fin_ref = oracle_prefill(inp)
+    check(inp, o1, f1, o_ref, fin_ref, "with cu_seqlens")
+    check(inp, o2, f2, o_ref, fin_ref, "equal lengths")
+    assert float((o1.float() - o2.float()).abs().max()) <= 2e-2
