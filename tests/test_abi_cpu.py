@@ -6,6 +6,7 @@ import os
 import re
 
 import pytest
+import torch
 
 from gated_delta_rule_151_b200 import gdr
 
@@ -251,3 +252,17 @@ def test_backward_workspace_size(lib):
     # one state checkpoint per 16 tokens of every sequence, plus one per sequence
     assert gdr.gdr_backward_workspace_size(2, 100, 3, 64, 32) == (2 + 7) * 3 * 32 * 64 * 4
     assert gdr.gdr_backward_workspace_size(1, 8192, 16, 128, 128) == (1 + 512) * 16 * 65536
+
+
+def test_bindings_reject_host_tensors_before_any_call():
+    # argument marshalling only: CPU tensors never reach the library
+    x = torch.zeros(8, 2, 16)
+    with pytest.raises(ValueError, match="CUDA"):
+        gdr.gdr_prologue(x, x, x, torch.zeros(32, 4), torch.zeros(32, 4), torch.zeros(32, 4),
+                         torch.zeros(8, 2), torch.ones(2), torch.zeros(8, 2))
+    with pytest.raises(ValueError, match="CUDA"):
+        gdr.gdr_backward(x, x, x, torch.zeros(8, 2), torch.zeros(8, 2), d_o=x)
+    with pytest.raises(ValueError, match="CUDA"):
+        gdr.gdr_decode_multi(torch.zeros(1, 2, 2, 16), torch.zeros(1, 2, 2, 16),
+                             torch.zeros(1, 2, 2, 16), torch.zeros(1, 2, 2), torch.zeros(1, 2, 2),
+                             torch.zeros(1, 2, 16, 16))
