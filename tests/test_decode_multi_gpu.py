@@ -68,3 +68,34 @@ def test_decode_multi_equals_single_steps(mode):
                                               b[:, t].contiguous(), s2) for t in range(T)], dim=1)
     torch.cuda.synchronize()
     assert torch.equal(o1, o2) and torch.equal(s1, s2)
+
+
+def test_full_size_draft_verification_sampled():
+    """The full 256 x 32 x 128 x 128 (512 MiB) state verified 4 drafts per
+    launch, 128 launches, in the launch configuration the benchmark times;
+    the oracle checks 16 sequences (all heads) at every token and their final
+    states."""
+    inp = I.workload("decode_spec_gdn")
+    N, T, H, dv = inp.num_seqs, I.SPEC_DRAFT, inp.H, inp.d_v
+    L = inp.total_T // N
+    steps = L // T
+    dev = "cuda"
+
+    def grp(x):   # [N*L, ...] -> [steps, N, T, ...]
+        return x.reshape(N, steps, T, *x.shape[1:]).transpose(0, 1).contiguous().to(dev)
+
+    q, k, v, g, b = (grp(x) for x in (inp.q, inp.k, inp.v, inp.g, inp.beta))
+    state = inp.h0.to(dev).clone()
+    o = torch.empty((steps, N, T, H, dv), dtype=inp.io_dtype, device=dev)
+    for s in range(steps):
+        gdr.gdr_decode_multi(q[s], k[s], v[s], g[s], b[s], state, o=o[s])
+    torch.cuda.synchronize()
+    seqs = list(range(0, N, N // 16))
+    o_ref, fin_ref = oracle.loop.run_inputs(inp, seqs=seqs)
+    o_ref = o_ref.reshape(len(seqs), L, H, dv)
+    o_gpu = o.permute(1, 0, 2, 3, 4).reshape(N, L, H, dv)[seqs].float().cpu().numpy()
+    err = float(np.max(np.abs(o_gpu - o_ref)))
+    assert err <= TOL_BF16_O, err
+    fin = state.cpu().numpy()
+    per = max(rel_frob(fin[s, h], fin_ref[i, h]) for i, s in enumerate(seqs) for h in range(H))
+    assert per <= TOL_BF16_STATE_REL, per
