@@ -72,3 +72,23 @@ def test_backward_bytes_per_launch():
               + H * d * d * 4)       # d_initial_state
     assert case.bytes == expect
     assert case.ws.numel() == (1 + T // 16) * H * d * d * 4
+
+
+def test_reference_arm_under_two_ranks_prints_once():
+    # launched like the multi-GPU bench: rank 0 alone times the oracle and
+    # prints; the other rank exits 0 without work
+    import socket
+    sock = socket.socket()
+    sock.bind(("127.0.0.1", 0))
+    port = sock.getsockname()[1]
+    sock.close()
+    r = subprocess.run([sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+                        "--nproc-per-node", "2", "--master-addr", "127.0.0.1", "--master-port",
+                        str(port), os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--gpus", "2", "--steps", "1", "--warmup", "1", "--workloads", "tiny_gdn"],
+                       capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["n_gpus"] == 2
