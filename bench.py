@@ -4,9 +4,13 @@
                     [--impl ours|reference]
 
 Prints ONE JSON line on rank 0.  The headline (`value`) is the first
-workload (default: the GDN prefill, 1 x 8192 tokens x 16 heads, d = 128,
-bf16).  Further workloads (default: the 256-sequence x 512-step GDN decode)
-are reported under "workloads" with the same fields.
+workload; by default that is the largest single-GPU configuration, the
+long-context variable-length GDN prefill (8 packed sequences, 262,144 tokens,
+16 heads, d = 128, bf16).  The other benchmark configurations (the 1 x 8192
+GDN prefill, the 2 x 32768 KDA prefill with an initial state, and the
+256-sequence x 512-step GDN and KDA decodes) follow under "workloads", each
+with the same fields: its own roofline, end-to-end figure, clock record and
+CPU baseline.
 
 A "step" is one pass of the whole hot path over one batch of synthetic input:
 one gdr_prefill_chunked call for a prefill workload, the 512 consecutive
@@ -51,6 +55,9 @@ METRIC = "gated delta-rule tokens/s (prefill, decode) and % roofline at 1 B200"
 UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 CHUNK = 64
+# the five benchmark configurations that run on the GPU (the tiny GDN case is
+# a parity-only configuration); the first is the headline
+DEFAULT_WORKLOADS = "varlen_gdn,gdn_prefill,kda_prefill,decode_gdn,decode_kda"
 
 
 # ------------------------------------------------------------ plumbing ----
@@ -68,6 +75,77 @@ def peaks():
         d = json.load(open(p))
         return d, "measured"
     return dict(FALLBACK_PEAKS), "fallback"
+
+
+class NvmlClockSampler:
+    """SM clock and clock-event reasons read through NVML every 20 ms while
+    running (read-only queries; no setting is changed).  Short timed regions
+    still get several samples."""
+
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40),
+               ("sw_thermal_slowdown", 0x20), ("sw_power_cap", 0x4))
+
+    def __init__(self, gpu_index: int, period_s: float = 0.02):
+        import pynvml
+        self.nv = pynvml
+        self.gpu = gpu_index
+        self.period = period_s
+        self.samples = []
+        self._stop = threading.Event()
+
+    def __enter__(self):
+        nv = self.nv
+        nv.nvmlInit()
+        uuid = torch.cuda.get_device_properties(self.gpu).uuid
+        self.h = None
+        try:
+            self.h = nv.nvmlDeviceGetHandleByUUID("GPU-" + str(uuid))
+        except Exception:
+            self.h = nv.nvmlDeviceGetHandleByIndex(self.gpu)
+        self.smax = nv.nvmlDeviceGetMaxClockInfo(self.h, nv.NVML_CLOCK_SM)
+        self.t = threading.Thread(target=self._run, daemon=True)
+        self.t.start()
+        return self
+
+    def _sample(self):
+        nv = self.nv
+        sm = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+        try:
+            r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        except AttributeError:
+            r = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+        self.samples.append((sm, r))
+
+    def _run(self):
+        while not self._stop.is_set():
+            self._sample()
+            time.sleep(self.period)
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        self.t.join(timeout=2)
+        self._sample()
+        try:
+            self.nv.nvmlShutdown()
+        except Exception:
+            pass
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        reasons = sorted({n for _, r in self.samples for n, bit in self.REASONS if r & bit})
+        return {"sm_mhz": statistics.median(s for s, _ in self.samples),
+                "sm_max_mhz": self.smax, "reasons": reasons, "samples": len(self.samples),
+                "source": "NVML every 20 ms during the timed region"}
+
+
+def clock_sampler(gpu_index: int):
+    """NVML sampler where NVML is importable, else nvidia-smi at 200 ms."""
+    try:
+        import pynvml  # noqa: F401
+        return NvmlClockSampler(gpu_index)
+    except Exception:
+        return ClockSampler(gpu_index)
 
 
 class ClockSampler:
@@ -572,11 +650,36 @@ def capture_step(case, stream):
     attribute and helper stream already exists): replaying it runs exactly the
     step's kernels, back to back, without the host's per-call Python and
     argument-checking time between them."""
-    g = torch.cuda.CUDAGraph()
+    try:
+        g = torch.cuda.CUDAGraph(keep_graph=True)   # keep the graph so its nodes can be counted
+    except TypeError:
+        g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=stream):
         case.step(stream)
     torch.cuda.synchronize()
     return g
+
+
+def graph_kernel_nodes(graph):
+    """Kernel nodes in a captured step (every kernel launch of the step is one
+    node), or None where the graph cannot be inspected."""
+    try:
+        from cuda.bindings import runtime as rt
+        g = rt.cudaGraph_t(init_value=int(graph.raw_cuda_graph()))
+        err, _, n = rt.cudaGraphGetNodes(g, 0)
+        if err != rt.cudaError_t.cudaSuccess:
+            return None
+        err, nodes, n = rt.cudaGraphGetNodes(g, n)
+        if err != rt.cudaError_t.cudaSuccess:
+            return None
+        kern = 0
+        for node in nodes[:n]:
+            err, kind = rt.cudaGraphNodeGetType(node)
+            if err == rt.cudaError_t.cudaSuccess and kind == rt.cudaGraphNodeType.cudaGraphNodeTypeKernel:
+                kern += 1
+        return kern
+    except Exception:
+        return None
 
 
 def bench_case(case, args, ws, rank, flush, stream, pk, pk_kind):
@@ -585,11 +688,14 @@ def bench_case(case, args, ws, rank, flush, stream, pk, pk_kind):
             case.step(stream)
         torch.cuda.synchronize()
         graph = None if args.no_graph else capture_step(case, stream)
+        counted = graph_kernel_nodes(graph) if graph is not None else None
+        if counted:
+            case.launches = counted
         run = graph.replay if graph is not None else (lambda: case.step(stream))
         run()
         torch.cuda.synchronize()
         barrier(ws)
-        with ClockSampler(torch.cuda.current_device()) as clk:
+        with clock_sampler(torch.cuda.current_device()) as clk:
             times = timed_steps(run, args.steps, flush, stream)
         barrier(ws)
         del graph
@@ -637,6 +743,8 @@ def bench_case(case, args, ws, rank, flush, stream, pk, pk_kind):
                      if not args.no_graph else "eager calls through the Python binding")
     if case.kind == "prefill":
         cfg["launches_per_step"] = case.launches
+    cfg["launch_count_source"] = ("kernel nodes of the captured step" if counted
+                                  else "the library's launch plan")
     if case.kind == "decode":
         cfg["launches_per_bench_step"] = case.steps
         cfg["tokens_per_sequence_per_launch"] = getattr(case, "T", 1)
@@ -649,10 +757,12 @@ def bench_case(case, args, ws, rank, flush, stream, pk, pk_kind):
     }
 
 
-def cpu_baseline(name, budget_s=20.0):
+def cpu_baseline(name, budget_s=10.0):
     """The oracle, as it stands, on a bounded sample of the workload: whole
     heads (all tokens of every sequence) until the estimated cost reaches the
-    budget.  Returns tokens/s scaled to the full workload's head count."""
+    budget.  Returns tokens/s scaled to the full workload's head count (a
+    decode workload's tokens are its sequences' tokens: the oracle runs the
+    same recurrence token by token)."""
     import oracle
     inp = I.workload(name)
     cores = oracle.loop.default_threads()
@@ -665,8 +775,14 @@ def cpu_baseline(name, budget_s=20.0):
     dt = time.perf_counter() - t
     value = inp.total_T * (nh / inp.H) / dt
     return {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-            "sample": f"{name}: {nh} of {inp.H} heads, all {inp.total_T} tokens, "
-                      f"fp64 C loop, {dt:.2f} s"}
+            "sample": f"{name}: {nh} of {inp.H} heads, all {inp.total_T} tokens of all "
+                      f"{inp.num_seqs} sequences, fp64 C loop, {dt:.2f} s"}
+
+
+# workloads whose recurrence the fp64 oracle runs (the prologue and the
+# backward have oracles of their own, not timed here)
+CPU_BASELINE_WORKLOADS = ("tiny_gdn", "gdn_prefill", "kda_prefill", "varlen_gdn", "gqa_prefill",
+                          "decode_gdn", "decode_kda", "decode_spec_gdn")
 
 
 def run_reference(args, ws, rank):
@@ -678,7 +794,7 @@ def run_reference(args, ws, rank):
     inp = I.workload(name)
     cores = oracle.loop.default_threads()
     per_head_flop = 7.0 * inp.d_k * inp.d_v * inp.total_T
-    nh = int(max(1, min(inp.H, 8.0 * 1.2e9 * cores / per_head_flop)))
+    nh = int(max(1, min(inp.H, 3.0 * 1.2e9 * cores / per_head_flop)))
     heads = list(range(nh))
     for _ in range(args.warmup if args.warmup < 2 else 1):
         oracle.loop.run_inputs(inp, heads=heads[:1], nthreads=cores)
@@ -707,7 +823,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workloads", default="gdn_prefill,decode_gdn",
+    ap.add_argument("--workloads", default=DEFAULT_WORKLOADS,
                     help="comma list from: " + ",".join(I.WORKLOADS) + " (or 'all')")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -743,6 +859,10 @@ def main():
         results[name] = bench_case(case, args, ws, rank, flush, stream, pk, pk_kind)
         del case
         torch.cuda.empty_cache()
+    if ws == 1 and rank == 0 and not args.no_cpu_baseline:
+        for name in names:
+            if name in CPU_BASELINE_WORKLOADS:
+                results[name]["cpu_baseline"] = cpu_baseline(name)
 
     if rank == 0:
         head = results[names[0]]
@@ -755,8 +875,8 @@ def main():
             "gpu_launches": sum(r["gpu_launches"] for r in results.values()),
             "clocks": head["clocks"],
         }
-        if ws == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_baseline(names[0])
+        if "cpu_baseline" in head:
+            line["cpu_baseline"] = head["cpu_baseline"]
         line["workloads"] = {n: r for n, r in results.items() if n != names[0]}
         print(json.dumps(line), flush=True)
     if ws > 1:

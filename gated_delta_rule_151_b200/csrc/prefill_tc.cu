@@ -783,8 +783,43 @@ cudaError_t noalloc_scratch_address(void **out) {
     return cudaSuccess;
 }
 
+// A wait on a flag that nothing sets, bounded by `polls` checks; when it
+// gives up it records the failure in the scratch's error word exactly as a
+// prefill kernel's bounded wait does.  The flag is a word of the scratch that
+// no code writes, so it stays zero.
+__global__ void noalloc_wait_probe_kernel(uint32_t polls) {
+    volatile uint32_t *flag = reinterpret_cast<volatile uint32_t *>(g_noalloc_scratch + 128);
+    uint32_t *err = reinterpret_cast<uint32_t *>(g_noalloc_scratch);
+    for (uint32_t it = 0; it < polls; ++it) {
+        if (*flag != 0u) return;
+        __nanosleep(64);
+    }
+    atomicOr(err, 1u);
+}
+
 }  // namespace
 }  // namespace gdr
+
+extern "C" gdr_status_t gdr_prefill_noalloc_check(void *stream) {
+    void *scratch = nullptr;
+    if (gdr::noalloc_scratch_address(&scratch) != cudaSuccess) return GDR_ERR_CUDA;
+    uint32_t word = 0;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemcpyAsync(&word, scratch, sizeof(word), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    // the word reports failures since the previous check: clear it
+    if (e == cudaSuccess && word != 0) e = cudaMemsetAsync(scratch, 0, sizeof(word), s);
+    if (e != cudaSuccess) return GDR_ERR_CUDA;
+    return word == 0 ? GDR_OK : GDR_ERR_DEVICE_TIMEOUT;
+}
+
+extern "C" gdr_status_t gdr_test_noalloc_wait_timeout(uint32_t polls, void *stream) {
+    if (polls == 0 || polls > (1u << 20)) return GDR_ERR_INVALID_ARG;
+    void *scratch = nullptr;
+    if (gdr::noalloc_scratch_address(&scratch) != cudaSuccess) return GDR_ERR_CUDA;
+    gdr::noalloc_wait_probe_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(polls);
+    return cudaGetLastError() == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
+}
 
 extern "C" gdr_status_t gdr_prefill_chunked_noalloc(
     const void *q, const void *k, const void *v, const float *g, const float *beta,

@@ -39,7 +39,8 @@ EXPORTED = ("gdr_status_string", "gdr_prefill_workspace_size", "gdr_prefill_path
             "gdr_prefill_chunked", "gdr_prefill_check_workspace", "gdr_decode_step",
             "gdr_prefill_chunked_noalloc", "gdr_prefill_chunked_gqa", "gdr_decode_step_gqa",
             "gdr_decode_multi", "gdr_prefill_plan", "gdr_prologue", "gdr_backward",
-            "gdr_backward_workspace_size")
+            "gdr_backward_workspace_size", "gdr_prefill_noalloc_check",
+            "gdr_test_noalloc_wait_timeout")
 
 
 class GdrError(RuntimeError):
@@ -84,6 +85,10 @@ def load_library():
         lib.gdr_prefill_chunked_noalloc.argtypes = [P, P, P, P, P, P, P, I32, I32, I32, I32, I32,
                                                     ST, ST, P, P, P]
         lib.gdr_prefill_chunked_noalloc.restype = ST
+        lib.gdr_prefill_noalloc_check.argtypes = [P]
+        lib.gdr_prefill_noalloc_check.restype = ST
+        lib.gdr_test_noalloc_wait_timeout.argtypes = [ctypes.c_uint32, P]
+        lib.gdr_test_noalloc_wait_timeout.restype = ST
         lib.gdr_prefill_chunked_gqa.argtypes = [P, P, P, P, P, P, P, I32, I32, I32, I32, I32, I32,
                                                 ST, ST, P, P, P, SZ, P]
         lib.gdr_prefill_chunked_gqa.restype = ST
@@ -293,7 +298,9 @@ def gdr_prefill_chunked_noalloc(q, k, v, g, beta, initial_state=None, cu_seqlens
                                 num_seqs=None, o=None, final_state=None, stream=None):
     """gdr_prefill_chunked without a workspace: the library's own fixed device
     scratch is used instead (see include/gdr.h for who needs this and the
-    rules that come with it).  ``o`` and ``final_state`` must be given."""
+    rules that come with it).  ``o`` must be given; ``final_state`` is
+    optional (None: the final state is not written, and None is returned for
+    it).  gdr_prefill_noalloc_check reports a device-side wait that gave up."""
     _need(q, "q", ndim=3)
     io = q.dtype
     _need(k, "k", io, 3)
@@ -318,6 +325,14 @@ def gdr_prefill_chunked_noalloc(q, k, v, g, beta, initial_state=None, cu_seqlens
         N, T, H, dk, dv, gate, _io_code(io), _ptr(o), _ptr(final_state), _stream_ptr(stream))
     _check(st, "gdr_prefill_chunked_noalloc")
     return o, final_state
+
+
+def gdr_prefill_noalloc_check(stream=None):
+    """Raise GdrError(GDR_ERR_DEVICE_TIMEOUT) if a bounded device-side wait of
+    a no-alloc prefill gave up since the previous check (synchronises the
+    stream; the error word is cleared once read)."""
+    _check(load_library().gdr_prefill_noalloc_check(_stream_ptr(stream)),
+           "gdr_prefill_noalloc_check")
 
 
 def gdr_decode_multi(q, k, v, g, beta, state, *, o=None, snapshots=None, stream=None):

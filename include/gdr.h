@@ -138,6 +138,13 @@ GDR_API gdr_status_t gdr_prefill_plan(int32_t num_seqs, int32_t total_T, int32_t
  * unit-lower-triangular inverse of (I + strictly-lower(beta K K^T)) weighted by
  * the gate ratios, and the chunk contractions), and the fp32 state is carried
  * on-chip from chunk to chunk.  Results equal the token loop up to rounding.
+ * The token loop is the pair of update rules on page "How the New Flash
+ * Models Work: Inside GLM-5.3-Flash and Qwen3.8-Flash-Next", section "Linear
+ * attention: a fixed-size memory in place of the cache": the Gated DeltaNet
+ * rule (scalar gate) and the Kimi Delta Attention rule (one gate per key
+ * channel), each with o_t read from the updated state.  Prefill is the phase
+ * that processes a whole prompt at once (same page, section "Serving:
+ * prefill and decode are different problems").
  *
  * q, k, v, g, beta   inputs, layouts above, T = total_T.
  * initial_state      [num_seqs, H, d_v, d_k] fp32, or NULL for zeros.
@@ -214,6 +221,10 @@ GDR_API gdr_status_t gdr_prefill_check_workspace(const void *workspace, size_t w
  * what must start at zero themselves, so calls whose GPU work overlaps (on
  * different streams or devices sharing nothing else) race on it: serialise
  * them.  Calls no cudaMalloc, cudaFree or allocating library routine.
+ *
+ * The device address of the array is kept per device for the life of the
+ * process: after cudaDeviceReset (or any teardown of the device's primary
+ * context) the library must not be used on that device again.
  */
 GDR_API gdr_status_t gdr_prefill_chunked_noalloc(const void *q, const void *k, const void *v,
                                          const float *g, const float *beta,
@@ -222,6 +233,27 @@ GDR_API gdr_status_t gdr_prefill_chunked_noalloc(const void *q, const void *k, c
                                          int32_t d_k, int32_t d_v, gdr_gate_mode_t gate_mode,
                                          gdr_dtype_t io_dtype, void *o, float *final_state,
                                          void *stream);
+
+/*
+ * The no-alloc counterpart of gdr_prefill_check_workspace.  The published
+ * method has no counterpart to it.  Synchronises `stream`, then reads the
+ * error word of the fixed array gdr_prefill_chunked_noalloc uses: it returns
+ * GDR_ERR_DEVICE_TIMEOUT if a bounded device-side wait of a no-alloc prefill
+ * (on this device, since the previous check) gave up -- that call's outputs
+ * are then not valid -- and GDR_OK otherwise.  A nonzero word is cleared
+ * after it is read, so each failure is reported once.  Allocates nothing.
+ */
+GDR_API gdr_status_t gdr_prefill_noalloc_check(void *stream);
+
+/*
+ * Test hook for gdr_prefill_noalloc_check; the published method has no
+ * counterpart to it.  Enqueues on `stream` one single-thread kernel that
+ * waits on a flag nothing sets, giving up after `polls` checks (1 to 2^20,
+ * about 100 ns each), and records the give-up in the no-alloc array's error
+ * word exactly as a prefill kernel's bounded wait does.  It cannot hang: the
+ * wait always ends.  GDR_ERR_INVALID_ARG for polls outside the range.
+ */
+GDR_API gdr_status_t gdr_test_noalloc_wait_timeout(uint32_t polls, void *stream);
 
 /*
  * One decode step: one new token for each of N sequences.

@@ -1,0 +1,75 @@
+"""Prefill edge cases the C ABI accepts but the workloads do not reach, on
+both tensor-core plans, against the fp64 oracle element by element:
+
+* write strengths beta in {0, 2}: beta = 0 leaves a token's write out, and
+  beta = 2 with a unit key makes the token's map S -> S (I - 2 k k^T) a
+  Householder reflection, which keeps ||S||_F (page "How the New Flash Models
+  Work", section "Linear attention: a fixed-size memory in place of the
+  cache": beta is a learned write strength, the rule itself puts no bound on
+  it);
+* the ungated rule, g = 0 for every token over thousands of tokens, where the
+  state never decays and every rounding error it picks up stays in it (page
+  "Qwen3.8-Flash vs GLM-5.3-Flash", section "The 3:1 Blueprint: Recurrent
+  Delta Rules and 2048-Token Indexing");
+* keys whose norm is not 1 (the rule does not normalise them; the library
+  leaves normalisation to the caller).
+"""
+import numpy as np
+import pytest
+import torch
+
+from gated_delta_rule_151_b200 import inputs as I
+from _util import PLANS, check, gpu_prefill, oracle_prefill
+
+pytestmark = pytest.mark.gpu
+
+MODES = [I.SCALAR, I.CHANNEL]
+
+
+def _rng(seed):
+    return np.random.default_rng(np.random.SeedSequence(seed, spawn_key=(99,)))
+
+
+@pytest.mark.parametrize("mode", MODES)
+@pytest.mark.parametrize("plan", PLANS)
+def test_beta_zero_and_two(mode, plan):
+    """Each token's beta is 0, 2 or its sigmoid draw, at random: skipped
+    writes and reflections mixed with ordinary writes inside every chunk."""
+    inp = I.make_inputs(total_T=700, H=3, d_k=128, gate_mode=mode, io_dtype=torch.bfloat16,
+                        cu_seqlens=[0, 260, 700], c=0.05, h0_std=0.05, seed=61)
+    pick = _rng(61).integers(0, 3, size=tuple(inp.beta.shape))
+    beta = inp.beta.numpy().copy()
+    beta[pick == 0] = 0.0
+    beta[pick == 1] = 2.0
+    inp.beta = torch.from_numpy(beta)
+    o, fin = gpu_prefill(inp, plan=plan)
+    o_ref, fin_ref = oracle_prefill(inp)
+    check(inp, o, fin, o_ref, fin_ref, f"beta in {{0, 2}} {mode} {plan}")
+
+
+@pytest.mark.parametrize("mode", MODES)
+@pytest.mark.parametrize("plan", PLANS)
+def test_ungated_rule_over_long_sequences(mode, plan):
+    """g = 0 for every token over 2,048 and 3,000 tokens: the state never
+    decays, so the chunk-to-chunk rounding of the state operands is never
+    forgotten.  The contract tolerances still hold."""
+    inp = I.make_inputs(total_T=5048, H=2, d_k=128, gate_mode=mode, io_dtype=torch.bfloat16,
+                        cu_seqlens=[0, 2048, 5048], c=0.05, h0_std=0.02, seed=63)
+    inp.g = torch.zeros_like(inp.g)
+    o, fin = gpu_prefill(inp, plan=plan)
+    o_ref, fin_ref = oracle_prefill(inp)
+    check(inp, o, fin, o_ref, fin_ref, f"ungated {mode} {plan}")
+
+
+@pytest.mark.parametrize("mode", MODES)
+@pytest.mark.parametrize("plan", PLANS)
+def test_keys_not_unit_norm(mode, plan):
+    """Keys scaled per token by a factor in [0.3, 1.4] (beta |k|^2 stays
+    below 2, so every token's map is still non-expansive)."""
+    inp = I.make_inputs(total_T=600, H=3, d_k=128, gate_mode=mode, io_dtype=torch.bfloat16,
+                        cu_seqlens=[0, 1, 333, 600], c=0.05, h0_std=0.05, seed=64)
+    s = _rng(64).uniform(0.3, 1.4, size=(inp.total_T, inp.H_qk, 1))
+    inp.k = (inp.k.double() * torch.from_numpy(s)).to(torch.bfloat16)
+    o, fin = gpu_prefill(inp, plan=plan)
+    o_ref, fin_ref = oracle_prefill(inp)
+    check(inp, o, fin, o_ref, fin_ref, f"key norms {mode} {plan}")
