@@ -257,14 +257,14 @@ def decode_work(inp):
 def split_launches(inp):
     """Kernel launches of the chunk-parallel plan: a prep and a chain kernel
     per window of chunks (the library bounds the chunk records of one window
-    to 1 GiB at 90,640 bytes per chunk and head), and per pipeline piece when
+    to 4 GiB at 98,848 bytes per chunk and head), and per pipeline piece when
     a single window is cut into pieces."""
     chains = inp.num_seqs * inp.H
     # equal lengths go without cu_seqlens, so the library knows each
     # sequence's length; otherwise total_T bounds it
     longest = inp.total_T // inp.num_seqs if inp.equal_lengths() else inp.total_T
     max_chunks = -(-longest // 64)
-    window = max(1, min(max_chunks, (1 << 30) // (chains * 90640)))
+    window = max(1, min(max_chunks, (4 << 30) // (chains * 98848)))
     windows = -(-max_chunks // window)
     pieces = 1
     if windows == 1:   # pipelined pieces of 12, 16, 21, 27, ... chunks (1.3x growth)

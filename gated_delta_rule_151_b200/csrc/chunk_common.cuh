@@ -106,11 +106,11 @@ __device__ __forceinline__ void block_row_times(float (&acc)[4], const float *X,
 //   T = [[T_a, 0], [-T_b A_ba T_a, T_b]],
 // and the same on each 32 x 32 half down to 16 x 16 diagonal blocks, which
 // are inverted by forward substitution (one thread per column).  Four
-// dependent matrix steps after the diagonal blocks; writes T as the tf32
-// operand [i][j] (128-byte swizzled rows, zero above the diagonal).
-// Xs: 4 KiB plain scratch (four 16 x 16 blocks).
-__device__ __forceinline__ void unit_lower_inverse(const float *Af, float *Tf, float *Xs,
-                                                   uint32_t tm_addr, int p) {
+// dependent matrix steps after the diagonal blocks.  T lands in Tf (fp32,
+// lower triangle and diagonal; the blocks above the diagonal are not
+// written).  Xs: 4 KiB plain scratch (four 16 x 16 blocks).  Called by 256
+// threads (p = thread index), which end synchronised.
+__device__ __forceinline__ void unit_lower_inverse_f32(const float *Af, float *Tf, float *Xs, int p) {
     // diagonal 16 x 16 blocks, column c of block `blk`
     if (p < 64) {
         const int blk = p >> 4, c = p & 15, o = blk * 16;
@@ -174,7 +174,13 @@ __device__ __forceinline__ void unit_lower_inverse(const float *Af, float *Tf, f
         st4(Tf, 16 * I + r, 16 * J + cq, make_float4(-acc[0], -acc[1], -acc[2], -acc[3]));
     }
     group_sync(2);
-    // T -> tf32 operand [i][j]
+}
+
+// unit_lower_inverse_f32, then T as the tf32 operand [i][j] (128-byte
+// swizzled rows, zero above the diagonal) at shared address tm_addr.
+__device__ __forceinline__ void unit_lower_inverse(const float *Af, float *Tf, float *Xs,
+                                                   uint32_t tm_addr, int p) {
+    unit_lower_inverse_f32(Af, Tf, Xs, p);
     for (int e = p; e < C * 16; e += 256) {
         const int i = e >> 4, q = e & 15, j0 = q * 4;
         const float4 t = ld4(Tf, i, j0);

@@ -1,42 +1,53 @@
 // Chunk-parallel plan of the tensor-core prefill (bf16 I/O, d_k = d_v = 128):
-// two kernels instead of one, for problems with fewer (sequence, head)
-// chains than the GPU has SMs.
+// a prep kernel over every chunk of every head, then a chain kernel that
+// carries the state from chunk to chunk with ONE tensor-core product on its
+// critical path.
 //
-// The chunk algebra is the one of the single-kernel plan (page "How the New
-// Flash Models Work: Inside GLM-5.3-Flash and Qwen3.8-Flash-Next", section
-// "Linear attention: a fixed-size memory in place of the cache", Gated
-// DeltaNet and Kimi Delta Attention equations, rearranged per chunk of C = 64
-// tokens):
+// The chunk algebra follows the recurrence on the page "How the New Flash
+// Models Work: Inside GLM-5.3-Flash and Qwen3.8-Flash-Next" (section "Linear
+// attention: a fixed-size memory in place of the cache", the Gated DeltaNet
+// and Kimi Delta Attention equations), rearranged per chunk of C = 64
+// tokens.  With S the state entering the chunk, G the within-chunk
+// cumulative log-gate and Γ = exp(G):
 //
-//   T = (I + A)^-1,  W = T diag(β)(K ⊙ Γ),  Ũ = T diag(β) V      chunk-local
-//   U = Ũ - W S^T,   O = (Q ⊙ Γ) S^T + (P ⊙ causal) U,
-//   S' = S Diag(Γ_C) + U^T K̂                                       state chain
+//   A_ij = β_i k_i^T Diag(e^{G_i - G_j}) k_j (j < i),  T = (I + A)^-1
+//   W = T diag(β)(K ⊙ Γ),  Ũ = T diag(β) V,  K̂_j = k_j ⊙ e^{G_C - G_j}
+//   P_ij = q_i^T Diag(e^{G_i - G_j}) k_j (j <= i),  Q̃_i = q_i ⊙ Γ_i
 //
-// Everything in the first line depends on one chunk only, so it runs for
-// every chunk of every head at once:
+// and the chunk's effect on the state is the affine map
 //
-//   prep kernel   one CTA per (chunk, sequence, head), two CTAs per SM.  It
-//                 stages the bf16 tiles with TMA, forms A and P with one
-//                 tcgen05 MMA, inverts I + A on CUDA cores, builds the tf32
-//                 operands and forms W and Ũ with two more MMAs.  It writes a
-//                 chunk record to the workspace: [-W; Q̃], K̂^T and P ⊙ causal
-//                 as ready-made fp16 shared-memory operand images, each with a
-//                 power-of-two scale, Ũ as fp32 rows, and exp(G_C).
-//   chain kernel  one CTA per NB value channels of a (sequence, head), NB =
-//                 32, 64 or 128 so that all chain CTAs fit the GPU at once.
-//                 Per chunk it bulk-copies the record and runs only the
-//                 products that need the state (fp16 operands, fp32
-//                 accumulation, the state itself in fp32 registers), with the
-//                 next records already in flight.
+//   S' = S Diag(Γ_C) + S N + B,     N = -W^T K̂,  B = Ũ^T K̂
+//   O  = S Q'^T + O⁰,               Q' = Q̃ - P W,  O⁰ = P Ũ
 //
-// fp16 with a per-block power-of-two scale keeps the 11-bit significand of
-// tf32 at half the bytes and twice the MMA depth; the chain is bound by the
-// shared-memory traffic of its operands, so halving them is what counts.
-// Records take 90,640 bytes per (chunk, head); problems whose records exceed
-// 1 GiB run in windows of chunks, the state passing between windows through
-// the workspace.
+// (the usual U = Ũ - W S^T, O = Q̃ S^T + P U, S' = S Diag(Γ_C) + U^T K̂,
+// with U substituted).  Everything except the products with S depends on
+// one chunk only:
+//
+//   prep kernel   one CTA per (chunk, sequence, head), two CTAs per SM.
+//                 TMA stages the bf16 tiles; tcgen05 MMAs form [K;Q] K^T
+//                 (A and P), then, after the 64 x 64 inverse on CUDA cores,
+//                 W^T and Ũ^T (the bf16 K and V tiles are the MN-major A
+//                 operands as TMA left them; T diag(β) is split into a bf16
+//                 high and low part), then N^T = K̂^T (-W) and P (-W) with W
+//                 split into fp16 high and low parts, then P Ũ.  It writes a
+//                 chunk record: N^T, the K̂ tile, Ũ^T, Q' and O⁰ as fp16
+//                 images with power-of-two scales, and exp(G_C).
+//   chain kernel  one CTA per (sequence, head).  Per chunk: D_B = Ũ^T K̂
+//                 (issued early, off the critical path), D_S = S N with S as
+//                 fp16 high + low parts in TMEM, D_O = S Q'^T; the state
+//                 warps form S' from D_S and D_B in fp32 and write the new
+//                 S halves back to TMEM, which starts the next chunk's D_S;
+//                 the output warps add O⁰ and store o.
+//
+// Splitting S, W and T diag(β) into high and low halves keeps the state's
+// rounding at about 2^-22 where a single fp16 or tf32 rounding per chunk
+// would be amplified by the conditioning of I + A (up to ~10 at beta = 2).
+// Records take 98,848 bytes per (chunk, head); problems whose records exceed
+// 4 GiB run in windows of chunks, the state passing between windows
+// through the workspace.
 #include <cuda.h>
 #include <cudaTypedefs.h>
+#include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
 #include <algorithm>
@@ -58,32 +69,24 @@ constexpr uint32_t ERR_TIMEOUT_TMA = 1u, ERR_TIMEOUT_MMA = 2u, ERR_TIMEOUT_HANDO
                    ERR_SMEM_ALIGN = 8u;
 
 // ----------------------------------------------------------- chunk record ----
-// Byte offsets inside one record.  The operand images are fp16 in the layout
-// the chain kernel's MMA descriptors read: rows of 64 halves (128 bytes) whose
-// 16-byte chunks are XOR-swizzled by row % 8, blocks 1024-byte aligned.  Each
-// image block is scaled by a power of two 2^s chosen so that its largest
-// magnitude lies in [2^14, 2^15): fp16 then carries the same 11-bit
-// significand as tf32 for every value above 2^-29 of the block maximum, and
-// the exponents s travel in the record.
-constexpr uint32_t REC_A1 = 0;          // [-W; Q̃] [tok][dk]: 2 blocks (64 dk) of 128 rows,
-                                        //   rows 0-63 -W (scale s_W), rows 64-127 Q̃ (s_Q)
-constexpr uint32_t REC_KH = 32768;      // K̂^T [dk][tok]: 128 rows (s_K)
-constexpr uint32_t REC_PM = 49152;      // P ⊙ causal [i][j]: 64 rows (s_P)
-constexpr uint32_t REC_UT = 57344;      // Ũ fp32: 4 blocks of 32 dv, each [tok][32] with the
-                                        //   16-byte chunks of row i XOR-swizzled by i % 8
-constexpr uint32_t REC_GC = 90112;      // exp(G_C): 1 float (scalar) or 128 (channel)
-constexpr uint32_t REC_EX = 90624;      // int32 {s_W, s_Q, s_K, s_P}
-constexpr uint32_t REC_BYTES = 90640;
-static_assert(REC_BYTES % 16 == 0 && REC_EX + 16 == REC_BYTES, "record layout");
+// Byte offsets inside one record.  The operand images are fp16 in the
+// 128-byte swizzled layouts the chain kernel's MMA descriptors read (rows of
+// 64 halves whose 16-byte chunks are XOR-swizzled by row % 8, blocks
+// 1024-byte aligned).  Each image carries its own power-of-two scale 2^s,
+// chosen so that its largest magnitude lies in [2^14, 2^15).
+constexpr uint32_t REC_NT = 0;        // N^T [j][i]: 2 K-blocks (i 0-63, 64-127) of 128 rows (s_N)
+constexpr uint32_t REC_KH = 32768;    // K̂ tile [t][j]: 2 blocks (j 0-63, 64-127) of 64 rows (s_K)
+constexpr uint32_t REC_UT = 49152;    // Ũ^T [r][t]: 128 rows (s_U)
+constexpr uint32_t REC_QP = 65536;    // Q' [t][j]: 2 K-blocks of 64 rows (s_Q)
+constexpr uint32_t REC_OZ = 81920;    // O⁰ [t][r]: plain rows of 256 bytes (s_O)
+constexpr uint32_t REC_GC = 98304;    // exp(G_C): 1 float (scalar gate) or 128 (channel gate)
+constexpr uint32_t REC_EX = 98816;    // int32 {s_N, s_K, s_U, s_Q, s_O, 0, 0, 0}
+constexpr uint32_t REC_BYTES = 98848;
+static_assert(REC_BYTES % 16 == 0 && REC_EX + 32 == REC_BYTES, "record layout");
 
 // Byte offset of fp16 element (r, c) (c < 64) inside a block of 128-byte rows.
 __host__ __device__ constexpr uint32_t h16_offset(uint32_t r, uint32_t c) {
     return r * 128u + ((((c >> 3) ^ (r & 7u)) & 7u) << 4) + (c & 7u) * 2u;
-}
-
-// Byte offset of Ũ[i][dv] inside the record.
-__host__ __device__ constexpr uint32_t rec_ut_offset(uint32_t i, uint32_t dv) {
-    return REC_UT + (dv >> 5) * 8192 + i * 128 + (((((dv & 31) >> 2) ^ (i & 7)) << 4) | ((dv & 3) << 2));
 }
 
 // Scale exponent s for a block whose largest magnitude is mx: mx 2^s lies in
@@ -105,15 +108,54 @@ __device__ __forceinline__ uint32_t f2h2_bits(float a, float b) {
     return *reinterpret_cast<const uint32_t *>(&h);
 }
 
+// fp16 high part of two values and the fp16 rounding of what it leaves.
+__device__ __forceinline__ void f2h2_hilo(float a, float b, uint32_t &hi, uint32_t &lo) {
+    const __half2 h = __floats2half2_rn(a, b);
+    const float2 back = __half22float2(h);
+    const __half2 l = __floats2half2_rn(a - back.x, b - back.y);
+    hi = *reinterpret_cast<const uint32_t *>(&h);
+    lo = *reinterpret_cast<const uint32_t *>(&l);
+}
+
+// bf16 high part of two values and the bf16 rounding of what it leaves.
+__device__ __forceinline__ void bf2_hilo(float a, float b, uint32_t &hi, uint32_t &lo) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    const float2 back = __bfloat1622float2(h);
+    const __nv_bfloat162 l = __floats2bfloat162_rn(a - back.x, b - back.y);
+    hi = *reinterpret_cast<const uint32_t *>(&h);
+    lo = *reinterpret_cast<const uint32_t *>(&l);
+}
+
+__device__ __forceinline__ uint16_t bf16_bits(float x) {
+    return __bfloat16_as_ushort(__float2bfloat16_rn(x));
+}
+
+__device__ __forceinline__ void st_global_v4(uint8_t *p, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+    *reinterpret_cast<uint4 *>(p) = make_uint4(a, b, c, d);
+}
+
 // ------------------------------------------------------------ prep kernel ----
 constexpr int kPrepThreads = 256;
-constexpr uint32_t PO_KQ = 0;       // bf16 [K d0-63][Q d0-63][K d64-127][Q d64-127]; then V'^T tf32
-constexpr uint32_t PO_V = 32768;    // bf16 [V d0-63][V d64-127]
-constexpr uint32_t PO_X1 = 49152;   // scratch (A, T fp32 / channel fp16 P1 operand / slow-path G); then K'^T tf32
-constexpr uint32_t PO_TM = 81920;   // inverse scratch / channel fp16 P1 operand; then T tf32
-constexpr uint32_t PO_MISC = 98304;
-constexpr uint32_t PREP_SMEM = PO_MISC + 2048;   // 100352: two CTAs per SM
-constexpr uint32_t PT_W = 0, PT_U = 64, PREP_TMEM_COLS = 128;
+// Shared memory (two CTAs per SM).  Regions and what they hold in turn:
+constexpr uint32_t PO_KQ = 0;       // bf16 [K d0-63][Q d0-63][K d64-127][Q d64-127] (TMA);
+                                    //   channel gate: K' = K ⊙ Γ (bf16 high) over K, Q̃ fp16 over Q
+constexpr uint32_t PO_V = 32768;    // bf16 [V d0-63][V d64-127] (TMA); after P2: Ũ^T fp16
+constexpr uint32_t PO_RA = 49152;   // A fp32 / channel P1 A operand (with RT) / slow-path G (with RT);
+                                    //   then T diag(.) bf16 high | low; after P2: -W^T fp16 high
+constexpr uint32_t PO_RT = 65536;   // T fp32; then the K̂ fp16 tile
+constexpr uint32_t PO_RX = 81920;   // inverse scratch / channel P1 B operand / slow-path A; then
+                                    //   scalar T diag(β) bf16 high | low, channel K' bf16 low;
+                                    //   after P2: -W^T fp16 low
+constexpr uint32_t PO_P = 98304;    // P fp16 [i][j] (rows 64-127 of the M = 128 A operand whose
+                                    //   rows 0-63 are the 8 KiB before it, never read back)
+constexpr uint32_t PO_MISC = 106496;
+constexpr uint32_t PREP_SMEM = PO_MISC + 2048;   // 108544: two CTAs per SM
+constexpr uint32_t PT_W = 0, PREP_TMEM_COLS = 256;   // P1 accumulates at column 0
+constexpr uint32_t IDESC_P2 = make_idesc(1, 128, 64) | kIdescAMN;     // bf16, A MN-major
+constexpr uint32_t IDESC_NT = make_idesc(0, 128, 128) | kIdescAMN;    // fp16, A MN-major
+constexpr uint32_t IDESC_H128 = make_idesc(0, 128, 128);              // fp16, K-major
+constexpr uint32_t IDESC_H64 = make_idesc(0, 128, 64);
 
 struct PrepMisc {
     uint64_t bar_tma, bar_mma;
@@ -129,18 +171,10 @@ struct PrepMisc {
             float beta[C], T0[D], T1[D];
         } c;
     } u;                               // beta comes first in both layouts
-    float red[2][8];                   // per-warp maxima for the image scales
+    float red[3][8];                   // per-warp maxima for the image scales
 };
 static_assert(sizeof(PrepMisc) <= 2048, "prep misc area overflow");
 static_assert(offsetof(PrepMisc, u) % 16 == 0, "prep misc arrays misaligned");
-
-__device__ __forceinline__ void st_global_v4(uint8_t *p, uint32_t a, uint32_t b, uint32_t c,
-                                             uint32_t d) {
-    *reinterpret_cast<uint4 *>(p) = make_uint4(a, b, c, d);
-}
-__device__ __forceinline__ void st_global_b16(uint8_t *p, uint16_t a) {
-    *reinterpret_cast<uint16_t *>(p) = a;
-}
 
 // Scale exponents of two blocks from every thread's largest |value| of each
 // (a, b >= 0); all 256 threads call it (two __syncthreads inside).
@@ -163,6 +197,29 @@ __device__ __forceinline__ void block_scale2(float a, float b, float (*red)[8], 
     sa = scale_exp(ma);
     sb = scale_exp(mb);
 }
+
+// Block-wide maxima of three per-thread values (all >= 0); all 256 threads
+// call it (two __syncthreads inside) and receive the same three results.
+__device__ __forceinline__ void block_max3(float (&v)[3], float (*red)[8]) {
+    const int w = threadIdx.x >> 5;
+#pragma unroll
+    for (int k = 0; k < 3; ++k) {
+        const uint32_t u = __reduce_max_sync(0xffffffffu, __float_as_uint(v[k]));
+        if ((threadIdx.x & 31) == 0) red[k][w] = __uint_as_float(u);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < 3; ++k) {
+        float mx = 0.f;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) mx = fmaxf(mx, red[k][q]);
+        v[k] = mx;
+    }
+    __syncthreads();
+}
+
+// 2^e for any integer e, saturated to the float range's normal powers.
+__device__ __forceinline__ float exp2c(int e) { return exp2i(min(max(e, -126), 126)); }
 
 // Bounded wait by every thread of the block; all threads agree on stopping.
 __device__ __forceinline__ bool block_wait(uint64_t *bar, uint32_t phase, int *abort_flag,
@@ -295,7 +352,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             const float R = T0;
             GC = T0 + T1;
             if (hh == 0) *reinterpret_cast<float *>(rec + REC_GC + ch * 4) = __expf(GC);
-            // fp16 P1 operands: rows [K e^{G-R}; Q e^{G-R}] (X1), K e^{R-G} (TM)
+            // fp16 P1 operands: rows [K e^{G-R}; Q e^{G-R}] (RA..RT), K e^{R-G} (RX)
             bool bad = false;
             const uint32_t kcol = (ch >> 6) * 16384, bcol = (ch >> 6) * 8192;
             const uint32_t cch = (ch & 63) >> 3, cel = (ch & 7) * 2;
@@ -310,11 +367,11 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 const float a = kv * up, b = qv * up, e = kv * dn;
                 bad |= !(fabsf(a) < kF16Limit) || !(fabsf(b) < kF16Limit) ||
                        !(fabsf(e) < kF16Limit);
-                st_shared_b16(sbase + PO_X1 + kcol + sw128_offset(i, cch) + cel,
+                st_shared_b16(sbase + PO_RA + kcol + sw128_offset(i, cch) + cel,
                               __half_as_ushort(__float2half_rn(a)));
-                st_shared_b16(sbase + PO_X1 + kcol + sw128_offset(64 + i, cch) + cel,
+                st_shared_b16(sbase + PO_RA + kcol + sw128_offset(64 + i, cch) + cel,
                               __half_as_ushort(__float2half_rn(b)));
-                st_shared_b16(sbase + PO_TM + bcol + sw128_offset(i, cch) + cel,
+                st_shared_b16(sbase + PO_RX + bcol + sw128_offset(i, cch) + cel,
                               __half_as_ushort(__float2half_rn(e)));
             }
             if (bad) m->slow = 1;
@@ -333,8 +390,8 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     for (int kk = 0; kk < 4; ++kk) {
                         if (CHANNEL) {
                             mma_f16_ss(tmem + PT_W,
-                                       sw128_kmajor_desc(sbase + PO_X1 + kb * 16384 + kk * 32),
-                                       sw128_kmajor_desc(sbase + PO_TM + kb * 8192 + kk * 32),
+                                       sw128_kmajor_desc(sbase + PO_RA + kb * 16384 + kk * 32),
+                                       sw128_kmajor_desc(sbase + PO_RX + kb * 8192 + kk * 32),
                                        IDESC_F16, (kb | kk) != 0);
                         } else {
                             const uint32_t a = sbase + PO_KQ + kb * 16384 + kk * 32;
@@ -350,13 +407,28 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 
         // ---- A (fp32 scratch) and P ⊙ causal (record image, fp16) -----------
         int sP = 0, sQ = 0, sK = 0, sW = 0;   // record image scale exponents
+        float kbound = 0.f, qbound = 0.f;      // bounds of |K̂| and |Q̃| over the chunk
+        // channel gate: this thread's bounds, |K̂| <= max|k| e^{max(G_C - G)} and
+        // |Q̃| <= max|q| e^{max G} over its tokens (a bound above the true
+        // maximum only moves values down within fp16's normal range)
+        float kbnd = 0.f, qbnd = 0.f;
+        if (CHANNEL) {
+            float dk = -3.0e38f, dq = -3.0e38f;
+#pragma unroll
+            for (int k = 0; k < 32; ++k) {
+                dk = fmaxf(dk, GC - gr[k]);
+                dq = fmaxf(dq, gr[k]);
+            }
+            kbnd = kmax * __expf(dk);
+            qbnd = qmax * __expf(dq);
+        }
         float *Af;
         float *Tf;
         float *Xs;
         if (!slow) {
-            Af = reinterpret_cast<float *>(sm + PO_X1);
-            Tf = reinterpret_cast<float *>(sm + PO_X1 + 16384);
-            Xs = reinterpret_cast<float *>(sm + PO_TM);
+            Af = reinterpret_cast<float *>(sm + PO_RA);
+            Tf = reinterpret_cast<float *>(sm + PO_RT);
+            Xs = reinterpret_cast<float *>(sm + PO_RX);
             uint32_t x[32];
             tmem_ld32(tmem + lane_off + PT_W + half * 32, x);
             tmem_wait_ld();
@@ -391,29 +463,52 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     for (int e = 0; e < 4; ++e) pv[q * 4 + e] = v4[e];
                 }
             }
-            float pm = 0.f;
+            float mx3[3] = {0.f, 0.f, 0.f};   // |P|; bounds of |K̂| and |Q̃| (see below)
             if (row >= C) {
 #pragma unroll
-                for (int e = 0; e < 32; ++e) pm = fmaxf(pm, fabsf(pv[e]));
+                for (int e = 0; e < 32; ++e) mx3[0] = fmaxf(mx3[0], fabsf(pv[e]));
             }
-            int unused;
-            block_scale2(pm, 0.f, m->red, sP, unused);
+            if (!CHANNEL) {
+                // |K̂| <= max |k| <= max ||k_i||, the diagonal of K K^T; |Q̃| <= max |q|
+                if (row < C) {
+                    const float kh = m->u.s.kh[i];
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        if (half * 32 + e == i) mx3[1] = __uint_as_float(x[e]) * kh * kh;
+                } else {
+                    const float gq = m->u.s.gam[i];
+#pragma unroll
+                    for (int c8 = 0; c8 < 8; ++c8) {
+                        float qf[8];
+                        bf16x8_to_f32(ld_shared_v4(sbase + PO_KQ + 8192 + half * 16384 + sw128_offset(i, c8)), qf);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) mx3[2] = fmaxf(mx3[2], fabsf(qf[e]) * gq);
+                    }
+                }
+            } else {
+                mx3[1] = kbnd;
+                mx3[2] = qbnd;
+            }
+            block_max3(mx3, m->red);
+            sP = scale_exp(mx3[0]);
+            kbound = CHANNEL ? mx3[1] : sqrtf(mx3[1]);
+            qbound = mx3[2];
             if (row >= C) {
                 const float f = exp2i(sP);
 #pragma unroll
                 for (int c4 = 0; c4 < 4; ++c4) {
                     const float *v = pv + c4 * 8;
-                    st_global_v4(rec + REC_PM + i * 128 + ((((half * 4 + c4) ^ (i & 7)) & 7) << 4),
+                    st_shared_v4(sbase + PO_P + i * 128 + ((((half * 4 + c4) ^ (i & 7)) & 7) << 4),
                                  f2h2_bits(v[0] * f, v[1] * f), f2h2_bits(v[2] * f, v[3] * f),
                                  f2h2_bits(v[4] * f, v[5] * f), f2h2_bits(v[6] * f, v[7] * f));
                 }
             }
         } else {
-            // exact A and P on CUDA cores: G [64][128] fp32 in X1, A in TM
-            float *Gs = reinterpret_cast<float *>(sm + PO_X1);
-            Af = reinterpret_cast<float *>(sm + PO_TM);
-            Tf = reinterpret_cast<float *>(sm + PO_X1);
-            Xs = reinterpret_cast<float *>(sm + PO_X1 + 16384);
+            // exact A and P on CUDA cores: G [64][128] fp32 in RA..RT, A in RX
+            float *Gs = reinterpret_cast<float *>(sm + PO_RA);
+            Af = reinterpret_cast<float *>(sm + PO_RX);
+            Tf = reinterpret_cast<float *>(sm + PO_RT);
+            Xs = reinterpret_cast<float *>(sm + PO_RA);
 #pragma unroll
             for (int k = 0; k < 32; ++k) Gs[(hh * 32 + k) * D + ch] = gr[k];
             __syncthreads();
@@ -454,11 +549,14 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 const int i = e >> 6, j = e & 63;
                 if (j > i) {
                     Af[ax(i, j)] = 0.f;
-                    st_global_b16(rec + REC_PM + h16_offset(i, j), 0);
+                    st_shared_b16(sbase + PO_P + h16_offset(i, j), 0);
                 }
             }
-            int unused;
-            block_scale2(pm, 0.f, m->red, sP, unused);
+            float mx3[3] = {pm, kbnd, qbnd};
+            block_max3(mx3, m->red);
+            sP = scale_exp(mx3[0]);
+            kbound = mx3[1];
+            qbound = mx3[2];
             const float f = exp2i(sP);
 #pragma unroll
             for (int it = 0; it < kPairIters; ++it) {
@@ -466,179 +564,282 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 if (pr < C * (C + 1) / 2) {
                     int i, j;
                     pair_ij(pr, i, j);
-                    st_global_b16(rec + REC_PM + h16_offset(i, j), f2h_bits(dqs[it] * f));
+                    st_shared_b16(sbase + PO_P + h16_offset(i, j), f2h_bits(dqs[it] * f));
                 }
             }
         }
         __syncthreads();
 
-        // ---- T = (I + A)^-1 -> tf32 [i][j] in TM ------------------------------
-        unit_lower_inverse(Af, Tf, Xs, sbase + PO_TM, tid);
-        __syncthreads();
+        // ---- T = (I + A)^-1 in fp32 (into RT on both paths) ---------------------
+        unit_lower_inverse_f32(Af, Tf, Xs, tid);
 
-        // ---- operands, pass 1: K'^T (X1, tf32), K̂^T and Q̃ (record, fp16) ------
-        if (!CHANNEL) {
-            const int i = tid & 63;
-            const float kp = m->u.s.kp[i], kh = m->u.s.kh[i], gq = m->u.s.gam[i];
-            // the chunk's largest |K̂| and |Q̃| set their image scales
-            float mk = 0.f, mq = 0.f;
-#pragma unroll 1
-            for (int it = 0; it < 4; ++it) {
-                const int jc = (tid >> 6) + 4 * it;
-                const uint32_t kb = jc >> 3, chk = jc & 7;
-                float kf[8], qf[8];
-                bf16x8_to_f32(ld_shared_v4(sbase + PO_KQ + kb * 16384 + sw128_offset(i, chk)), kf);
-                bf16x8_to_f32(ld_shared_v4(sbase + PO_KQ + kb * 16384 + 8192 + sw128_offset(i, chk)), qf);
+        // ---- B operands of P2: T diag(f) as bf16 high and low parts, rows t.
+        //      Scalar gate: f = β Γ for W (RA) and f = β for Ũ (RX); channel
+        //      gate: f = β for both (RA), Γ goes into the A operand ------------
+        {
+            const float *Tm = reinterpret_cast<const float *>(sm + PO_RT);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    mk = fmaxf(mk, fabsf(kh * kf[e]));
-                    mq = fmaxf(mq, fabsf(gq * qf[e]));
-                }
-            }
-            block_scale2(mk, mq, m->red, sK, sQ);
-            const float fk = exp2i(sK), fq = exp2i(sQ);
-            const uint32_t tcol = (i >> 5) * 16384;
-            const uint32_t tchunk = (i & 31) >> 2, tel = (i & 3) * 4;
-#pragma unroll 1
-            for (int it = 0; it < 4; ++it) {
-                const int jc = (tid >> 6) + 4 * it;
-                const uint32_t kb = jc >> 3, chk = jc & 7;
-                float kf[8], qf[8];
-                bf16x8_to_f32(ld_shared_v4(sbase + PO_KQ + kb * 16384 + sw128_offset(i, chk)), kf);
-                bf16x8_to_f32(ld_shared_v4(sbase + PO_KQ + kb * 16384 + 8192 + sw128_offset(i, chk)), qf);
+            for (int it = 0; it < 2; ++it) {
+                const int item = tid + it * kPrepThreads;
+                const int t = item >> 3, cq = item & 7;   // row t, columns 8 cq .. 8 cq + 7
+                const float4 a = ld4(Tm, t, cq * 8), b = ld4(Tm, t, cq * 8 + 4);
+                const float tv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+                uint32_t h1[4], l1[4], h2[4], l2[4];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const uint32_t j = jc * 8 + e;
-                    st_shared_b32(sbase + PO_X1 + tcol + sw128_offset(j, tchunk) + tel, to_tf32(kp * kf[e]));
-                    st_global_b16(rec + REC_KH + h16_offset(j, i), f2h_bits(kh * kf[e] * fk));
-                }
-                // Q̃ row 64 + i, channels jc*8 .. +7: one 16-byte chunk
-                st_global_v4(rec + REC_A1 + kb * 16384 + (64 + i) * 128 + (((chk ^ (i & 7)) & 7) << 4),
-                             f2h2_bits(gq * qf[0] * fq, gq * qf[1] * fq),
-                             f2h2_bits(gq * qf[2] * fq, gq * qf[3] * fq),
-                             f2h2_bits(gq * qf[4] * fq, gq * qf[5] * fq),
-                             f2h2_bits(gq * qf[6] * fq, gq * qf[7] * fq));
-            }
-        } else {
-            const uint32_t kcol = (ch >> 6) * 16384, cch = (ch & 63) >> 3, cel = (ch & 7) * 2;
-            // scales from bounds: |K̂| <= max|k| e^{max(G_C - G)}, |Q̃| <= max|q| e^{max G};
-            // a bound above the true maximum only moves values down within fp16's
-            // normal range, so the precision is the same
-            float dk = -3.0e38f, dq = -3.0e38f;
-#pragma unroll
-            for (int k = 0; k < 32; ++k) {
-                dk = fmaxf(dk, GC - gr[k]);
-                dq = fmaxf(dq, gr[k]);
-            }
-            block_scale2(kmax * __expf(dk), qmax * __expf(dq), m->red, sK, sQ);
-            const float fk = exp2i(sK), fq = exp2i(sQ);
-            const uint32_t rowblk = hh * 16384;
-            uint8_t *qdst = rec + REC_A1 + (ch >> 6) * 16384;
-#pragma unroll
-            for (int c8 = 0; c8 < 4; ++c8) {   // tokens hh*32 + c8*8 .. +7
-                float wh[8];
-#pragma unroll
-                for (int q2 = 0; q2 < 2; ++q2) {
-                    const int q4 = c8 * 2 + q2;
-                    uint32_t wk[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int k = q4 * 4 + e, i = hh * 32 + k;
-                        const uint32_t src = sbase + PO_KQ + kcol + sw128_offset(i, cch) + cel;
-                        const float kv = ld_shared_bf16(src), qv = ld_shared_bf16(src + 8192);
-                        const float eg = __expf(gr[k]);
-                        wk[e] = to_tf32(m->u.c.beta[i] * kv * eg);
-                        wh[q2 * 4 + e] = kv * __expf(GC - gr[k]) * fk;
-                        st_global_b16(qdst + h16_offset(64 + i, ch & 63), f2h_bits(qv * eg * fq));
+                for (int e = 0; e < 8; e += 2) {
+                    const int j = cq * 8 + e;
+                    const float x0 = j <= t ? tv[e] : 0.f, x1 = j + 1 <= t ? tv[e + 1] : 0.f;
+                    const float b0 = m->u.c.beta[j], b1 = m->u.c.beta[j + 1];
+                    if (CHANNEL) {
+                        bf2_hilo(x0 * b0, x1 * b1, h1[e / 2], l1[e / 2]);
+                    } else {
+                        bf2_hilo(x0 * m->u.s.kp[j], x1 * m->u.s.kp[j + 1], h1[e / 2], l1[e / 2]);
+                        bf2_hilo(x0 * b0, x1 * b1, h2[e / 2], l2[e / 2]);
                     }
-                    st_shared_v4(sbase + PO_X1 + rowblk + sw128_offset(ch, q4), wk[0], wk[1], wk[2], wk[3]);
                 }
-                // K̂^T row ch, tokens hh*32 + c8*8 .. +7: one 16-byte chunk
-                st_global_v4(rec + REC_KH + ch * 128 + ((((hh * 4 + c8) ^ (ch & 7)) & 7) << 4),
-                             f2h2_bits(wh[0], wh[1]), f2h2_bits(wh[2], wh[3]), f2h2_bits(wh[4], wh[5]),
-                             f2h2_bits(wh[6], wh[7]));
+                const uint32_t off = t * 128 + (((cq ^ (t & 7)) & 7) << 4);
+                st_shared_v4(sbase + PO_RA + off, h1[0], h1[1], h1[2], h1[3]);
+                st_shared_v4(sbase + PO_RA + 8192 + off, l1[0], l1[1], l1[2], l1[3]);
+                if (!CHANNEL) {
+                    st_shared_v4(sbase + PO_RX + off, h2[0], h2[1], h2[2], h2[3]);
+                    st_shared_v4(sbase + PO_RX + 8192 + off, l2[0], l2[1], l2[2], l2[3]);
+                }
             }
         }
-        __syncthreads();   // K and Q are consumed: V'^T takes their place
+        __syncthreads();   // T (RT) is consumed
 
-        // ---- operands, pass 2: V'^T = (diag(β) V)^T into the K/Q area --------
+        // ---- the K̂ tile (fp16, scale s_K) into RT.  Channel gate: also
+        //      K' = K ⊙ Γ as bf16 high (over K) and low (RX) parts, and
+        //      Q̃ = Q ⊙ Γ as fp16 (scale s_Q) over Q ------------------------------
+        sK = scale_exp(kbound);
+        if (CHANNEL) sQ = scale_exp(qbound);
         if (!CHANNEL) {
-            const int i = tid & 63;
-            const float bt = m->u.s.beta[i];
-            const uint32_t tcol = (i >> 5) * 16384;
-            const uint32_t tchunk = (i & 31) >> 2, tel = (i & 3) * 4;
-#pragma unroll 1
-            for (int it = 0; it < 4; ++it) {
-                const int jc = (tid >> 6) + 4 * it;
-                const uint32_t kb = jc >> 3, chk = jc & 7;
-                float vf[8];
-                bf16x8_to_f32(ld_shared_v4(sbase + PO_V + kb * 8192 + sw128_offset(i, chk)), vf);
+            const float fs = exp2i(sK);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const uint32_t j = jc * 8 + e;
-                    st_shared_b32(sbase + PO_KQ + tcol + sw128_offset(j, tchunk) + tel,
-                                  to_tf32(bt * vf[e]));
-                }
+            for (int it = 0; it < 4; ++it) {
+                const int item = tid + it * kPrepThreads;
+                const int blk = item >> 9, t = (item >> 3) & 63, cq = item & 7;
+                float kf[8];
+                bf16x8_to_f32(ld_shared_v4(sbase + PO_KQ + blk * 16384 + sw128_offset(t, cq)), kf);
+                const float f = m->u.s.kh[t] * fs;
+                st_shared_v4(sbase + PO_RT + blk * 8192 + sw128_offset(t, cq),
+                             f2h2_bits(kf[0] * f, kf[1] * f), f2h2_bits(kf[2] * f, kf[3] * f),
+                             f2h2_bits(kf[4] * f, kf[5] * f), f2h2_bits(kf[6] * f, kf[7] * f));
             }
         } else {
-            const uint32_t vcol = (ch >> 6) * 8192, cch = (ch & 63) >> 3, cel = (ch & 7) * 2;
-            const uint32_t rowblk = hh * 16384;
-#pragma unroll
-            for (int q4 = 0; q4 < 8; ++q4) {
-                uint32_t wv[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int i = hh * 32 + q4 * 4 + e;
-                    const float vv = ld_shared_bf16(sbase + PO_V + vcol + sw128_offset(i, cch) + cel);
-                    wv[e] = to_tf32(m->u.c.beta[i] * vv);
-                }
-                st_shared_v4(sbase + PO_KQ + rowblk + sw128_offset(ch, q4), wv[0], wv[1], wv[2], wv[3]);
+            const float fk = exp2i(sK), fq = exp2i(sQ);
+            const uint32_t kcol = (ch >> 6) * 16384, tcol = (ch >> 6) * 8192;
+            const uint32_t cch = (ch & 63) >> 3, cel = (ch & 7) * 2;
+#pragma unroll 4
+            for (int k = 0; k < 32; ++k) {
+                const int i = hh * 32 + k;
+                const uint32_t src = sbase + PO_KQ + kcol + sw128_offset(i, cch) + cel;
+                const uint32_t dst = tcol + sw128_offset(i, cch) + cel;
+                const float kv = ld_shared_bf16(src), qv = ld_shared_bf16(src + 8192);
+                const float eg = __expf(gr[k]);
+                st_shared_b16(sbase + PO_RT + dst, f2h_bits(kv * __expf(GC - gr[k]) * fk));
+                const float kp = kv * eg;
+                const uint16_t khi = bf16_bits(kp);
+                st_shared_b16(src, khi);
+                st_shared_b16(sbase + PO_RX + dst, bf16_bits(kp - __uint_as_float((uint32_t)khi << 16)));
+                st_shared_b16(src + 8192, f2h_bits(qv * eg * fq));
             }
         }
         fence_proxy_async();
         __syncthreads();
 
-        // ---- P2: W^T = K'^T T^T, Ũ^T = V'^T T^T --------------------------------
+        // ---- P2: W^T = K'^T (T diag(.))^T and Ũ^T = V^T (T diag(β))^T in bf16,
+        //      the K and V tiles (or K' high and low) as MN-major A operands ----
+        uint32_t mph = slow ? 0u : 1u;   // next phase of bar_mma
         if (tid == 0) {
             tc_fence_after();
+            const uint32_t tb_w = sbase + PO_RA, tb_u = sbase + (CHANNEL ? PO_RA : PO_RX);
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const uint32_t kb = k >> 2, kk = k & 3;
-                const uint64_t bd = sw128_kmajor_desc(sbase + PO_TM + kb * 8192 + kk * 32);
-                mma_tf32_ss(tmem + PT_W, sw128_kmajor_desc(sbase + PO_X1 + kb * 16384 + kk * 32),
-                            bd, IDESC_N64, k != 0);
-                mma_tf32_ss(tmem + PT_U, sw128_kmajor_desc(sbase + PO_KQ + kb * 16384 + kk * 32),
-                            bd, IDESC_N64, k != 0);
+            for (int k = 0; k < 4; ++k) {
+                const uint64_t ak = sw128_mnmajor_desc(sbase + PO_KQ + k * 2048, 16384, 1024);
+                mma_f16_ss(tmem + 0, ak, sw128_kmajor_desc(tb_w + k * 32), IDESC_P2, k != 0);
+                mma_f16_ss(tmem + 0, ak, sw128_kmajor_desc(tb_w + 8192 + k * 32), IDESC_P2, 1);
+                if (CHANNEL)
+                    mma_f16_ss(tmem + 0, sw128_mnmajor_desc(sbase + PO_RX + k * 2048, 8192, 1024),
+                               sw128_kmajor_desc(tb_w + k * 32), IDESC_P2, 1);
+                const uint64_t av = sw128_mnmajor_desc(sbase + PO_V + k * 2048, 8192, 1024);
+                mma_f16_ss(tmem + 64, av, sw128_kmajor_desc(tb_u + k * 32), IDESC_P2, k != 0);
+                mma_f16_ss(tmem + 64, av, sw128_kmajor_desc(tb_u + 8192 + k * 32), IDESC_P2, 1);
             }
             mma_commit(&m->bar_mma);
         }
-        if (!block_wait(&m->bar_mma, slow ? 0 : 1, &m->abort_flag, err, ERR_TIMEOUT_MMA)) break;
+        // the K̂ tile goes to the record while the MMAs run
+#pragma unroll
+        for (int it = 0; it < 4; ++it) {
+            const int e = tid + it * kPrepThreads;
+            *reinterpret_cast<uint4 *>(rec + REC_KH + e * 16) = ld_shared_v4(sbase + PO_RT + e * 16);
+        }
+        if (!block_wait(&m->bar_mma, mph, &m->abort_flag, err, ERR_TIMEOUT_MMA)) break;
+        mph ^= 1u;
         tc_fence_after();
 
-        // ---- -W (fp16 image) and Ũ (fp32 rows) into the record; thread = d row --
+        // ---- -W^T (fp16 high in RA, low in RX) and Ũ^T (fp16, RV and the
+        //      record), thread = row d of W^T / r of Ũ^T, tokens half*32 .. +31 -----
+        int sU = 0;
         {
-            uint32_t x[32];
-            tmem_ld32(tmem + lane_off + PT_W + half * 32, x);
+            uint32_t x[32], y[32];
+            tmem_ld32(tmem + lane_off + 0 + half * 32, x);
+            tmem_ld32(tmem + lane_off + 64 + half * 32, y);
             tmem_wait_ld();
-            float mw = 0.f;
+            float mw = 0.f, mu = 0.f;
 #pragma unroll
-            for (int ii = 0; ii < 32; ++ii) mw = fmaxf(mw, fabsf(__uint_as_float(x[ii])));
-            int unused;
-            block_scale2(mw, 0.f, m->red, sW, unused);
-            const float fw = -exp2i(sW);
-            const uint32_t j = row;
-            uint8_t *base = rec + REC_A1 + (j >> 6) * 16384;
+            for (int e = 0; e < 32; ++e) {
+                mw = fmaxf(mw, fabsf(__uint_as_float(x[e])));
+                mu = fmaxf(mu, fabsf(__uint_as_float(y[e])));
+            }
+            block_scale2(mw, mu, m->red, sW, sU);
+            const float fw = -exp2i(sW), fu = exp2i(sU);
 #pragma unroll
-            for (int ii = 0; ii < 32; ++ii)
-                st_global_b16(base + h16_offset(half * 32 + ii, j & 63), f2h_bits(__uint_as_float(x[ii]) * fw));
-            if (tid == 0)
-                *reinterpret_cast<int4 *>(rec + REC_EX) = make_int4(sW, sQ, sK, sP);
-            tmem_ld32(tmem + lane_off + PT_U + half * 32, x);
-            tmem_wait_ld();
+            for (int c4 = 0; c4 < 4; ++c4) {
+                const uint32_t off = row * 128 + ((((half * 4 + c4) ^ (row & 7)) & 7) << 4);
+                uint32_t hw[4], lw[4], hu[4];
 #pragma unroll
-            for (int ii = 0; ii < 32; ++ii)
-                *reinterpret_cast<float *>(rec + rec_ut_offset(half * 32 + ii, row)) =
-                    __uint_as_float(x[ii]);
+                for (int e = 0; e < 4; ++e) {
+                    const int i = c4 * 8 + 2 * e;
+                    f2h2_hilo(__uint_as_float(x[i]) * fw, __uint_as_float(x[i + 1]) * fw, hw[e], lw[e]);
+                    hu[e] = f2h2_bits(__uint_as_float(y[i]) * fu, __uint_as_float(y[i + 1]) * fu);
+                }
+                st_shared_v4(sbase + PO_RA + off, hw[0], hw[1], hw[2], hw[3]);
+                st_shared_v4(sbase + PO_RX + off, lw[0], lw[1], lw[2], lw[3]);
+                st_shared_v4(sbase + PO_V + off, hu[0], hu[1], hu[2], hu[3]);
+                st_global_v4(rec + REC_UT + off, hu[0], hu[1], hu[2], hu[3]);
+            }
+        }
+        fence_proxy_async();
+        tc_fence_before();
+        __syncthreads();
+
+        // ---- N^T = K̂^T (-W) (columns 0-127) and P (-W) (rows 64-127 of
+        //      columns 128-255), -W as fp16 high + low ------------------------------
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const uint64_t akh = sw128_mnmajor_desc(sbase + PO_RT + k * 2048, 8192, 1024);
+                mma_f16_ss(tmem + 0, akh, sw128_kmajor_desc(sbase + PO_RA + k * 32), IDESC_NT, k != 0);
+                mma_f16_ss(tmem + 0, akh, sw128_kmajor_desc(sbase + PO_RX + k * 32), IDESC_NT, 1);
+                const uint64_t ap = sw128_kmajor_desc(sbase + PO_P - 8192 + k * 32);
+                mma_f16_ss(tmem + 128, ap, sw128_kmajor_desc(sbase + PO_RA + k * 32), IDESC_H128, k != 0);
+                mma_f16_ss(tmem + 128, ap, sw128_kmajor_desc(sbase + PO_RX + k * 32), IDESC_H128, 1);
+            }
+            mma_commit(&m->bar_mma);
+        }
+        if (!block_wait(&m->bar_mma, mph, &m->abort_flag, err, ERR_TIMEOUT_MMA)) break;
+        mph ^= 1u;
+        tc_fence_after();
+
+        // ---- N^T (record, scale s_N): thread = row j, columns i = half*64 .. +63;
+        //      Q' = Q̃ - P W (record, scale s_Q'): rows t = row - 64 --------------
+        // Scales from bounds (every |operand| below 2^15 after its own scale):
+        // |N| <= 64 2^30 2^-(s_K + s_W), |P W| <= 64 2^30 2^-(s_P + s_W),
+        // |O⁰| <= 64 2^30 2^-(s_P + s_U); a bound above the true maximum only
+        // moves values down within fp16's normal range.
+        const int sN = min(max(sK + sW - 22, -100), 100);
+        const int sQP = scale_exp(qbound + exp2c(36 - sP - sW));
+        {
+            const float gn = exp2c(sN - sK - sW), fpw = exp2i(-sP) * exp2i(-sW), gq = exp2i(sQP);
+            const bool qrow = row >= C;            // warp-uniform (TMEM sub-partitions 2, 3)
+            const int t = row - C;
+            // Q̃ for columns half*64 + p*32 + 8*c8 .. +7 (p < 2, c8 < 4)
+            auto qtilde = [&](int p, int c8, float (&qv)[8]) {
+                const uint32_t a = sbase + PO_KQ + 8192 + half * 16384 + sw128_offset(t, p * 4 + c8);
+                if (CHANNEL) {
+                    const uint4 w = ld_shared_v4(a);
+                    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+                    const float f = exp2i(-sQ);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 v = __half22float2(*reinterpret_cast<const __half2 *>(&ww[e]));
+                        qv[2 * e] = v.x * f;
+                        qv[2 * e + 1] = v.y * f;
+                    }
+                } else {
+                    bf16x8_to_f32(ld_shared_v4(a), qv);
+                    const float gq2 = m->u.s.gam[t];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) qv[e] *= gq2;
+                }
+            };
+#pragma unroll
+            for (int p = 0; p < 2; ++p) {
+                uint32_t x[32];
+                tmem_ld32(tmem + lane_off + half * 64 + p * 32, x);
+                tmem_wait_ld();
+#pragma unroll
+                for (int c8 = 0; c8 < 4; ++c8) {
+                    uint32_t w[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        w[e] = f2h2_bits(__uint_as_float(x[c8 * 8 + 2 * e]) * gn,
+                                         __uint_as_float(x[c8 * 8 + 2 * e + 1]) * gn);
+                    st_global_v4(rec + REC_NT + half * 16384 + row * 128 +
+                                     ((((p * 4 + c8) ^ (row & 7)) & 7) << 4),
+                                 w[0], w[1], w[2], w[3]);
+                }
+                if (qrow) {
+                    tmem_ld32(tmem + lane_off + 128 + half * 64 + p * 32, x);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int c8 = 0; c8 < 4; ++c8) {
+                        float qv[8];
+                        qtilde(p, c8, qv);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            qv[e] = (qv[e] + __uint_as_float(x[c8 * 8 + e]) * fpw) * gq;
+                        st_global_v4(rec + REC_QP + half * 8192 + t * 128 +
+                                         ((((p * 4 + c8) ^ (t & 7)) & 7) << 4),
+                                     f2h2_bits(qv[0], qv[1]), f2h2_bits(qv[2], qv[3]),
+                                     f2h2_bits(qv[4], qv[5]), f2h2_bits(qv[6], qv[7]));
+                    }
+                }
+            }
+        }
+        tc_fence_before();
+        __syncthreads();   // TMEM columns 0-127 are read
+
+        // ---- O⁰ = P Ũ (rows 64-127 of columns 0-127) ------------------------------
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                mma_f16_ss(tmem + 0, sw128_kmajor_desc(sbase + PO_P - 8192 + k * 32),
+                           sw128_kmajor_desc(sbase + PO_V + k * 32), IDESC_H128, k != 0);
+            mma_commit(&m->bar_mma);
+        }
+        if (!block_wait(&m->bar_mma, mph, &m->abort_flag, err, ERR_TIMEOUT_MMA)) break;
+        mph ^= 1u;
+        tc_fence_after();
+        {
+            const int sO = min(max(sP + sU - 22, -100), 100);
+            const float go = exp2c(sO - sP - sU);
+            const int t = row - C;
+            if (row >= C) {
+#pragma unroll
+                for (int p = 0; p < 2; ++p) {
+                    uint32_t x[32];
+                    tmem_ld32(tmem + lane_off + half * 64 + p * 32, x);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int c8 = 0; c8 < 4; ++c8) {
+                        uint32_t w[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            w[e] = f2h2_bits(__uint_as_float(x[c8 * 8 + 2 * e]) * go,
+                                             __uint_as_float(x[c8 * 8 + 2 * e + 1]) * go);
+                        st_global_v4(rec + REC_OZ + t * 256 + (half * 64 + p * 32 + c8 * 8) * 2,
+                                     w[0], w[1], w[2], w[3]);
+                    }
+                }
+            }
+            if (tid == 0) {
+                *reinterpret_cast<int4 *>(rec + REC_EX) = make_int4(sN, sK, sU, sQP);
+                *reinterpret_cast<int4 *>(rec + REC_EX + 16) = make_int4(sO, 0, 0, 0);
+            }
         }
     } while (0);
 
@@ -651,66 +852,50 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 }
 
 // ----------------------------------------------------------- chain kernel ----
-// Each CTA owns NB value channels (a column block of S^T) of one (sequence,
-// head); the (D / NB) CTAs of a head run in lockstep on the same records.
-// Every product keeps the 128-row M dimension on [W; Q̃] or on d_k, with
-// fp16 operands (K = 16 per MMA) and fp32 accumulators:
+// One CTA per (sequence, head).  Per chunk, with S the state entering it:
 //
-//   M1  D1 = [-W; Q̃] S_b^T          rows 0-63: X = -W S_b^T
-//                                   rows 64-127: the inter-chunk output Q̃ S_b^T
-//   M2  D2 = K̂^T U_b                ΔS_b^T
-//   M4  D4 = [junk; P ⊙ causal] U_b rows 64-127: the intra-chunk output
+//   MMA_B  D_B = Ũ^T K̂        A = record Ũ^T, B = record K̂ tile (MN-major);
+//                              issued as soon as the last D_B was read
+//   MMA_S  D_S = S N           A = S as fp16 high + low parts in TMEM, one
+//                              power-of-two scale per row (value channel);
+//                              B = record N^T
+//   MMA_O  D_O = S Q'^T        A = the high part of S, B = record Q'
 //
-// U_b = Ũ_b + X and S_b^T = S_b^T Diag(exp(G_C)) + ΔS_b^T are formed in fp32
-// (the state block stays in registers, thread = d_k row) and written back as
-// fp16 images with a fresh power-of-two scale each chunk; every accumulator
-// is unscaled by the exponents of its two operands.  Warp roles: state
-// block, U (tokens 0-63 of D1), output (tokens 64-127 of D1 and D4), the MMA
-// issuer and the record loader, handing off through mbarriers only; record
-// buffers are freed by tcgen05.commit of the MMAs that read them.
-template <int NB>
-struct Chain {
-    static constexpr int kSW = NB <= 64 ? 4 : 8;         // state warps
-    static constexpr int kCS = NB * 4 / kSW;              // state columns per thread
-    static constexpr int kSets = NB <= 64 ? 1 : 2;        // sets of (2 U warps, 2 output warps)
-    static constexpr int kCU = NB / kSets;                // U / output columns per thread
-    static constexpr int kIssuer = kSW + 4 * kSets;       // MMA issuer warp; the loader follows
-    static constexpr int kThreads = 32 * (kIssuer + 2);
-    static constexpr bool kDB = NB <= 64;                 // two K̂/P stages and O buffers
-    static constexpr int kStages = kDB ? 2 : 1;
-    static constexpr uint32_t A1 = 0;                     // [-W; Q̃], 2 stages of 32 KiB
-    static constexpr uint32_t KH = 65536;                 // K̂^T, 16 KiB per stage
-    static constexpr uint32_t A4 = KH + kStages * 16384;  // [junk; P], 16 KiB per stage
-    static constexpr uint32_t UT = A4 + kStages * 16384;  // Ũ fp32, 2 stages of 256 NB bytes
-    static constexpr uint32_t SB = UT + 512 * NB;         // S_b image [NB][128], 256 NB bytes
-    static constexpr uint32_t UB = SB + 256 * NB;         // U_b^T image [NB][64], 128 NB bytes
-    static constexpr uint32_t MISC = UB + 128 * NB;
-    static constexpr uint32_t SMEM = MISC + 1024;
-    static constexpr uint32_t TD1 = 0;                    // per O buffer
-    static constexpr uint32_t TD4 = kStages * NB;         // per O buffer
-    static constexpr uint32_t TD2 = 2 * kStages * NB;
-    static constexpr uint32_t TCOLS = TD2 + NB <= 256 ? 256 : 512;
-    // fp16 x fp16 -> fp32, B (the S and U images) MN-major
-    static constexpr uint32_t IDESC = make_idesc(0, 128, NB) | (1u << 16);
-    static_assert(SMEM <= 232448 && TD2 + NB <= 512, "chain kernel does not fit");
-    // the S and U images are MN-major with one 64-byte row (32 channels) per K index
-    static_assert(NB == 32, "MN-major images hold 32 value channels");
-};
+//   S' = S Diag(exp(G_C)) + D_S + D_B          (fp32, state warps)
+//   O  = D_O^T + O⁰                             (output warps)
+//
+// MMA_S is the only product on the state's critical path: the state warps
+// write the new S halves into TMEM and MMA_S of the next chunk starts.
+// The high part of S alternates between two TMEM buffers, so the next
+// chunk's state can be written while this chunk's MMA_O still reads it.
+// Warps: 16 state warps (warp w: value channel r = 32 (w % 4) + lane, key
+// channels 32 (w / 4) .. +31; the fp32 state lives in registers), 4 output
+// warps (value channel r, all 64 tokens, through a shared-memory tile that
+// leaves in 16-byte row segments), an MMA issuer and a record loader (two
+// record stages, bulk copies, the records two chunks ahead prefetched to L2).
+constexpr int kStateWarps = 16, kOutWarps = 4;
+constexpr int kIssuerWarp = kStateWarps + kOutWarps, kLoaderWarp = kIssuerWarp + 1;
+constexpr int kChainThreads = 32 * (kLoaderWarp + 1);   // 704
+constexpr int kStateThreads = 32 * kStateWarps, kOutThreads = 32 * kOutWarps;
+constexpr uint32_t CSTAGE = 99328;                       // record slot (1024-byte multiple)
+constexpr uint32_t CO_OT = 2 * CSTAGE;                   // output tile [64 t][128 r] bf16
+constexpr uint32_t CO_MISC = CO_OT + 16384;
+constexpr uint32_t CHAIN_SMEM = CO_MISC + 8192;          // 223232
+// TMEM: D_S, D_B, D_O, the high part of S in two buffers (chunk parity), the low part
+constexpr uint32_t CT_DS = 0, CT_DB = 128, CT_DO = 256, CT_SH = 320, CT_SL = 448, CT_COLS = 512;
+constexpr uint32_t IDESC_DB = make_idesc(0, 128, 128) | kIdescBMN;
+static_assert(CHAIN_SMEM <= 232448 && REC_BYTES <= CSTAGE, "chain smem");
 
 struct ChainMisc {
-    uint64_t full_a1[2], full_u[2], full_kp[2];     // record parts landed
-    uint64_t empty_a1[2], empty_u[2], empty_kp[2];  // record buffers free
-    uint64_t bar1, bar2, bar4[2];                   // M1 / M2 / M4 done
-    uint64_t s_ready, u_ready, o_free[2], osc_full[2];
+    uint64_t full[2], empty[2];       // record stage landed / free
+    uint64_t bar_s, bar_o, bar_end;
+    uint64_t s_hi, s_lo, d_free, o_free;      // S high / low part in TMEM
     uint32_t tmem_base;
     int abort_flag;
-    int es[4];                  // S image exponent, per chunk mod 4
-    int dsx[2][2];              // {s_K, s_U}, per chunk parity
-    int osx[2][4];              // {s_Q, s_S, s_P, s_U}, per chunk parity
-    alignas(16) int ex[2][4];   // record exponents {s_W, s_Q, s_K, s_P}, with the Ũ stage
-    float red_s[2][8], red_u[2][4];
+    int rowscale[4][D];               // S row exponents, by chunk mod 4
+    float xs[2][4][D];                // row maxima of the four key-channel quarters, by chunk parity
 };
-static_assert(sizeof(ChainMisc) <= 1024, "chain misc area overflow");
+static_assert(sizeof(ChainMisc) <= 8192, "chain misc area overflow");
 
 // Bounded wait by a whole warp; the lanes agree on the outcome, so the
 // warp-wide TMEM accesses after it stay convergent.
@@ -732,456 +917,15 @@ __device__ __forceinline__ bool named_sync_or(int id, int nthreads, bool flag) {
     return any != 0;
 }
 
-// Largest |value| over a role's warps -> the role-wide scale exponent.  The
-// barrier also agrees on stopping: every warp of the role calls this once
-// per chunk, even after a failed wait, and all of them see `stop` true if
-// any thread passed stop = true or the CTA's abort flag was set before.
-__device__ __forceinline__ int role_scale(float mx, float *slots, int slot, int nwarps, int bar_id,
-                                          bool &stop, volatile int *abort_flag) {
-    const uint32_t wm = __reduce_max_sync(0xffffffffu, __float_as_uint(mx));
-    if ((threadIdx.x & 31) == 0) slots[slot] = __uint_as_float(wm);
-    stop = named_sync_or(bar_id, nwarps * 32, stop || *abort_flag != 0);
-    float bm = 0.f;
-    for (int w = 0; w < nwarps; ++w) bm = fmaxf(bm, slots[w]);
-    return scale_exp(bm);
+__device__ __forceinline__ void named_sync(int id, int nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
-template <bool CHANNEL, int NB>
-__global__ void __launch_bounds__(Chain<NB>::kThreads, 1)
+template <bool CHANNEL>
+__global__ void __launch_bounds__(kChainThreads, 1)
 chain_kernel(const uint8_t *__restrict__ recs, const float *h0, float *fin, float *ws_state,
              const int32_t *__restrict__ cu, int num_seqs, int total_T, int H, int c_begin,
              int c_end, __nv_bfloat16 *__restrict__ o, uint32_t *err) {
-    using K = Chain<NB>;
-    constexpr int kParts = D / NB;
-    extern __shared__ __align__(1024) uint8_t smem_raw[];
-    const uint32_t sbase = smem_u32(smem_raw);
-    const int chain = blockIdx.x / kParts, part = blockIdx.x % kParts;
-    const int chains = gridDim.x / kParts;
-    const int h = chain % H, n = chain / H;
-    const int dv0 = part * NB;
-    int t0, len;
-    sequence_range(cu, n, num_seqs, total_T, t0, len);
-    const int nchunks = (len + C - 1) / C;
-    if (c_begin > 0 && c_begin >= nchunks) return;   // finished in an earlier window
-    const int c_stop = min(c_end, nchunks);
-    const int nl = max(c_stop - c_begin, 0);
-    const float *s_in = c_begin == 0 ? h0 : ws_state;
-    float *s_out = c_stop == nchunks ? fin : ws_state;
-
-    const int tid = threadIdx.x;
-    const int warp = tid >> 5, lane = tid & 31;
-    // entry (dv0 + j, t) of this (sequence, head)'s state
-    const size_t sg = (((size_t)n * H + h) * D + dv0) * D;
-
-    if (nl == 0) {   // empty sequence: the state block passes through
-        if (s_out != nullptr && tid < D) {
-            for (int j = 0; j < NB; ++j)
-                s_out[sg + (size_t)j * D + tid] = s_in != nullptr ? s_in[sg + (size_t)j * D + tid] : 0.f;
-        }
-        return;
-    }
-    if ((sbase & 1023u) != 0) {
-        if (tid == 0) atomicOr(err, ERR_SMEM_ALIGN);
-        return;
-    }
-    uint8_t *sm = smem_raw;
-    ChainMisc *m = reinterpret_cast<ChainMisc *>(sm + K::MISC);
-    if (tid == 0) {
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(&m->full_a1[s], 1);
-            mbar_init(&m->full_u[s], 1);
-            mbar_init(&m->full_kp[s], 1);
-            mbar_init(&m->empty_a1[s], 1);
-            mbar_init(&m->empty_u[s], 64 * K::kSets);
-            mbar_init(&m->empty_kp[s], 1);
-            mbar_init(&m->bar4[s], 1);
-            mbar_init(&m->o_free[s], 64 * K::kSets);
-            mbar_init(&m->osc_full[s], 64 * K::kSets);
-        }
-        mbar_init(&m->bar1, 1);
-        mbar_init(&m->bar2, 1);
-        mbar_init(&m->s_ready, 32 * K::kSW);
-        mbar_init(&m->u_ready, 64 * K::kSets);
-        m->abort_flag = 0;
-        fence_barrier_init();
-    }
-    if (warp == 0) {
-        tmem_alloc(&m->tmem_base, K::TCOLS);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = m->tmem_base;
-    volatile int *abort_flag = &m->abort_flag;
-    auto fail = [&](uint32_t code) {
-        *abort_flag = 1;
-        atomicOr(err, code);
-    };
-    auto rec_of = [&](int lc) {
-        return recs + ((size_t)lc * chains + chain) * REC_BYTES;
-    };
-
-    if (warp < K::kSW) {
-        // ================================== state block S_b^T, thread = d_k row ====
-        const int sub = warp & 3, cg = warp >> 2;
-        const int t = sub * 32 + lane;
-        const int c0 = cg * K::kCS;
-        const uint32_t lane_off = static_cast<uint32_t>(sub * 32) << 16;
-        float S[K::kCS];
-#pragma unroll
-        for (int j = 0; j < K::kCS; ++j)
-            S[j] = s_in != nullptr ? s_in[sg + (size_t)(c0 + j) * D + t] : 0.f;
-        // fp16 image of the state block for chunk lc (MN-major: row t holds the 32
-        // channels of d_k index t), with its scale exponent
-        const uint32_t srow = sbase + K::SB + t * 64;
-        bool stop = false;
-        auto publish = [&](int lc) {
-            float mx = 0.f;
-#pragma unroll
-            for (int j = 0; j < K::kCS; ++j) mx = fmaxf(mx, fabsf(S[j]));
-            const int sS = role_scale(mx, m->red_s[lc & 1], warp, K::kSW, 1, stop, abort_flag);
-            const float f = exp2i(sS);
-#pragma unroll
-            for (int c = 0; c < 4; ++c)
-                st_shared_v4(srow + ((c ^ ((t >> 1) & 3)) << 4), f2h2_bits(S[8 * c] * f, S[8 * c + 1] * f),
-                             f2h2_bits(S[8 * c + 2] * f, S[8 * c + 3] * f), f2h2_bits(S[8 * c + 4] * f, S[8 * c + 5] * f),
-                             f2h2_bits(S[8 * c + 6] * f, S[8 * c + 7] * f));
-            if (tid == 0) m->es[lc & 3] = sS;
-            fence_proxy_async();
-            mbar_arrive(&m->s_ready);
-        };
-        publish(0);
-        for (int lc = 0; lc < nl && !stop; ++lc) {
-            const float gc =
-                *reinterpret_cast<const float *>(rec_of(lc) + REC_GC + (CHANNEL ? t * 4 : 0));
-            // u_ready publishes the ΔS exponents; M2 done gives ΔS.  A failed wait
-            // still takes part in the role's barrier below.
-            if (!warp_wait(&m->u_ready, lc & 1)) { fail(ERR_TIMEOUT_HANDOFF); stop = true; }
-            if (!stop && !warp_wait(&m->bar2, lc & 1)) { fail(ERR_TIMEOUT_MMA); stop = true; }
-            if (!stop) {
-                tc_fence_after();
-                const float f1 = exp2i(-m->dsx[lc & 1][0]), f2 = exp2i(-m->dsx[lc & 1][1]);
-#pragma unroll
-                for (int p = 0; p < K::kCS / 16; ++p) {
-                    uint32_t x[16];
-                    tmem_ld16(tmem + lane_off + K::TD2 + c0 + p * 16, x);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int jj = 0; jj < 16; ++jj)
-                        S[p * 16 + jj] = fmaf(gc, S[p * 16 + jj], __uint_as_float(x[jj]) * f1 * f2);
-                }
-                tc_fence_before();
-            }
-            if (lc + 1 < nl) publish(lc + 1);
-        }
-        if (s_out != nullptr) {
-#pragma unroll
-            for (int j = 0; j < K::kCS; ++j) s_out[sg + (size_t)(c0 + j) * D + t] = S[j];
-        }
-    } else if (warp < K::kIssuer) {
-        const int set = (warp - K::kSW) >> 2, r = (warp - K::kSW) & 3;
-        const int c0 = set * K::kCU;
-        const uint32_t lane_off = static_cast<uint32_t>(r * 32) << 16;
-        if (r < 2) {
-            // ===================================== U_b = Ũ_b + X, thread = token i ====
-            const int i = r * 32 + lane;
-            const uint32_t urow_img = sbase + K::UB + i * 64;   // MN-major: row i = token
-            bool stop = false;
-            for (int lc = 0; lc < nl && !stop; ++lc) {
-                const uint32_t s = lc & 1;
-                const uint32_t b = K::kDB ? (lc & 1) : 0;
-                // a failed wait still takes part in the role's barrier below
-                if (!warp_wait(&m->full_u[s], (lc >> 1) & 1)) { fail(ERR_TIMEOUT_TMA); stop = true; }
-                if (!stop && !warp_wait(&m->s_ready, lc & 1)) { fail(ERR_TIMEOUT_HANDOFF); stop = true; }
-                if (!stop && !warp_wait(&m->bar1, lc & 1)) { fail(ERR_TIMEOUT_MMA); stop = true; }
-                if (!stop) tc_fence_after();
-                const int sW = m->ex[s][0], sQ = m->ex[s][1], sK = m->ex[s][2], sP = m->ex[s][3];
-                const int sS = m->es[lc & 3];
-                const float fa = exp2i(-sW), fb = exp2i(-sS);
-                // U = Ũ + X in fp32 (this thread's token row, 32 channels)
-                float u[32];
-                float mx = 0.f;
-                if (!stop) {
-                    uint32_t x[32];
-                    tmem_ld32(tmem + lane_off + K::TD1 + b * NB, x);
-                    const uint32_t urow = sbase + K::UT + s * (256 * NB) + i * 128;
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const uint4 v = ld_shared_v4(urow + ((q ^ (i & 7)) << 4));
-                        const float w[4] = {__uint_as_float(v.x), __uint_as_float(v.y),
-                                            __uint_as_float(v.z), __uint_as_float(v.w)};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            u[q * 4 + e] = w[e] + __uint_as_float(x[q * 4 + e]) * fa * fb;
-                            mx = fmaxf(mx, fabsf(u[q * 4 + e]));
-                        }
-                    }
-                }
-                const int sU = role_scale(mx, m->red_u[lc & 1], set * 2 + r, 2 * K::kSets, 2, stop,
-                                          abort_flag);
-                if (stop) break;
-                const float fu = exp2i(sU);
-#pragma unroll
-                for (int c = 0; c < 4; ++c)
-                    st_shared_v4(urow_img + ((c ^ ((i >> 1) & 3)) << 4), f2h2_bits(u[8 * c] * fu, u[8 * c + 1] * fu),
-                                 f2h2_bits(u[8 * c + 2] * fu, u[8 * c + 3] * fu),
-                                 f2h2_bits(u[8 * c + 4] * fu, u[8 * c + 5] * fu),
-                                 f2h2_bits(u[8 * c + 6] * fu, u[8 * c + 7] * fu));
-                if (i == 0 && set == 0) {
-                    m->dsx[lc & 1][0] = sK;
-                    m->dsx[lc & 1][1] = sU;
-                    m->osx[lc & 1][0] = sQ;
-                    m->osx[lc & 1][1] = sS;
-                    m->osx[lc & 1][2] = sP;
-                    m->osx[lc & 1][3] = sU;
-                }
-                fence_proxy_async();
-                tc_fence_before();
-                mbar_arrive(&m->u_ready);
-                mbar_arrive(&m->empty_u[s]);   // this Ũ stage (and its exponents) is read
-                mbar_arrive(&m->osc_full[lc & 1]);
-            }
-        } else {
-            // ====================== output rows (token i = TMEM lane - 64), NB/kSets channels ====
-            const int i = (r - 2) * 32 + lane;
-            for (int lc = 0; lc < nl; ++lc) {
-                if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
-                const uint32_t b = K::kDB ? (lc & 1) : 0;
-                const uint32_t bph = K::kDB ? ((lc >> 1) & 1) : (lc & 1);
-                if (!warp_wait(&m->osc_full[lc & 1], (lc >> 1) & 1)) { fail(ERR_TIMEOUT_HANDOFF); break; }
-                if (!warp_wait(&m->bar4[b], bph)) { fail(ERR_TIMEOUT_MMA); break; }
-                tc_fence_after();
-                const int *sx = m->osx[lc & 1];
-                const float fq1 = exp2i(-sx[0]), fq2 = exp2i(-sx[1]);
-                const float fp1 = exp2i(-sx[2]), fp2 = exp2i(-sx[3]);
-                const int cc = c_begin + lc;
-                const bool live = i < min(C, len - cc * C);
-                uint4 *dst = reinterpret_cast<uint4 *>(o + ((size_t)(t0 + cc * C + i) * H + h) * D + dv0 + c0);
-#pragma unroll
-                for (int p = 0; p < K::kCU / 32; ++p) {
-                    uint32_t x1[32], x4[32];
-                    tmem_ld32(tmem + lane_off + K::TD1 + b * NB + c0 + p * 32, x1);
-                    tmem_ld32(tmem + lane_off + K::TD4 + b * NB + c0 + p * 32, x4);
-                    tmem_wait_ld();
-                    if (live) {
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            uint32_t w[4];
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const int j = q * 8 + 2 * e;
-                                const float a = __uint_as_float(x1[j]) * fq1 * fq2 + __uint_as_float(x4[j]) * fp1 * fp2;
-                                const float c2 = __uint_as_float(x1[j + 1]) * fq1 * fq2 + __uint_as_float(x4[j + 1]) * fp1 * fp2;
-                                const __nv_bfloat162 b2 = __floats2bfloat162_rn(a, c2);
-                                w[e] = *reinterpret_cast<const uint32_t *>(&b2);
-                            }
-                            dst[p * 4 + q] = make_uint4(w[0], w[1], w[2], w[3]);
-                        }
-                    }
-                }
-                tc_fence_before();
-                mbar_arrive(&m->o_free[b]);
-            }
-        }
-    } else if (warp == K::kIssuer) {
-        // ======================================================= MMA issuer ====
-        if (lane == 0) {
-            // MN-major images: 8-row K groups 512 bytes apart, 16 K rows per MMA
-            const uint64_t d_sb = sw64_mnmajor_desc(sbase + K::SB, 8192, 512);
-            const uint64_t d_ub = sw64_mnmajor_desc(sbase + K::UB, 8192, 512);
-            for (int lc = 0; lc < nl; ++lc) {
-                if (*abort_flag) break;
-                const uint32_t s = lc & 1, sph = (lc >> 1) & 1;
-                const uint32_t b = K::kDB ? (lc & 1) : 0;                 // K̂/P stage = O buffer
-                const uint32_t bph = K::kDB ? ((lc >> 1) & 1) : (lc & 1);
-                // the buffers are normally ready long before the state block
-                if (!mbar_wait_sleep(&m->full_a1[s], sph)) { fail(ERR_TIMEOUT_TMA); break; }
-                const int prev = K::kDB ? lc - 2 : lc - 1;                // last user of O buffer b
-                if (prev >= 0 && !mbar_wait_sleep(&m->o_free[b], K::kDB ? ((prev >> 1) & 1) : (prev & 1))) {
-                    fail(ERR_TIMEOUT_HANDOFF);
-                    break;
-                }
-                if (!mbar_wait_sleep(&m->s_ready, lc & 1)) { fail(ERR_TIMEOUT_HANDOFF); break; }
-                tc_fence_after();
-                const uint64_t d_a1 = sw128_kmajor_desc(sbase + K::A1 + s * 32768);
-                // descriptors advance by (bytes >> 4) in their start-address field
-#pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    mma_f16_ss(tmem + K::TD1 + b * NB, d_a1 + (((k >> 2) * 16384 + (k & 3) * 32) >> 4),
-                               d_sb + ((k * 1024) >> 4), K::IDESC, k != 0);
-                mma_commit(&m->bar1);
-                mma_commit(&m->empty_a1[s]);
-                if (!mbar_wait_sleep(&m->full_kp[b], bph)) { fail(ERR_TIMEOUT_TMA); break; }
-                if (!mbar_wait_sleep(&m->u_ready, lc & 1)) { fail(ERR_TIMEOUT_HANDOFF); break; }
-                tc_fence_after();
-                const uint64_t d_kh = sw128_kmajor_desc(sbase + K::KH + b * 16384);
-                const uint64_t d_a4 = sw128_kmajor_desc(sbase + K::A4 + b * 16384);
-#pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    mma_f16_ss(tmem + K::TD2, d_kh + ((k * 32) >> 4), d_ub + ((k * 1024) >> 4), K::IDESC, k != 0);
-                mma_commit(&m->bar2);
-#pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    mma_f16_ss(tmem + K::TD4 + b * NB, d_a4 + ((k * 32) >> 4), d_ub + ((k * 1024) >> 4), K::IDESC,
-                               k != 0);
-                mma_commit(&m->bar4[b]);
-                mma_commit(&m->empty_kp[b]);
-            }
-        }
-    } else if (lane == 0) {
-        // ==================================================== record loader ====
-        uint32_t issued[6] = {0, 0, 0, 0, 0, 0};
-        uint64_t *bars[6] = {&m->full_a1[0], &m->full_a1[1], &m->full_u[0], &m->full_u[1],
-                             &m->full_kp[0], &m->full_kp[1]};
-        auto load_a1 = [&](int lc) {
-            const int s = lc & 1;
-            mbar_arrive_expect_tx(&m->full_a1[s], 32768);
-            bulk_load(sm + K::A1 + s * 32768, rec_of(lc) + REC_A1, 32768, &m->full_a1[s]);
-            ++issued[s];
-        };
-        auto load_u = [&](int lc) {   // this CTA's channel blocks of Ũ, and the exponents
-            const int s = lc & 1;
-            const uint8_t *r = rec_of(lc);
-            mbar_arrive_expect_tx(&m->full_u[s], 256 * NB + 16);
-            bulk_load(sm + K::UT + s * (256 * NB), r + REC_UT + part * (NB / 32) * 8192, 256 * NB,
-                      &m->full_u[s]);
-            bulk_load(m->ex[s], r + REC_EX, 16, &m->full_u[s]);
-            ++issued[2 + s];
-        };
-        auto load_kp = [&](int lc) {
-            const int b = K::kDB ? (lc & 1) : 0;
-            const uint8_t *r = rec_of(lc);
-            mbar_arrive_expect_tx(&m->full_kp[b], 16384 + 8192);
-            bulk_load(sm + K::KH + b * 16384, r + REC_KH, 16384, &m->full_kp[b]);
-            bulk_load(sm + K::A4 + b * 16384 + 8192, r + REC_PM, 8192, &m->full_kp[b]);
-            ++issued[4 + b];
-        };
-        auto prefetch_rec = [&](int lc) {
-            if (lc < nl) {
-                const uint8_t *r = rec_of(lc);
-#pragma unroll
-                for (int q = 0; q < 5; ++q) bulk_prefetch_l2(r + q * 18128, 18128);
-            }
-        };
-        constexpr int kKPAhead = K::kDB ? 2 : 1;   // K̂/P stages in flight
-        load_a1(0);
-        load_kp(0);
-        load_u(0);
-        if (nl > 1) {
-            load_a1(1);
-            load_u(1);
-            if (K::kDB) load_kp(1);
-        }
-        prefetch_rec(1);
-        prefetch_rec(2);
-        // each buffer is refilled as soon as the step reading it has finished,
-        // in the order those steps finish within a chunk
-        for (int lc = 0; lc < nl; ++lc) {
-            if (*abort_flag) break;
-            const uint32_t s = lc & 1, sph = (lc >> 1) & 1;
-            const uint32_t b = K::kDB ? (lc & 1) : 0;
-            const uint32_t bph = K::kDB ? ((lc >> 1) & 1) : (lc & 1);
-            if (!mbar_wait_sleep(&m->empty_a1[s], sph)) { fail(ERR_TIMEOUT_MMA); break; }
-            if (lc + 2 < nl) load_a1(lc + 2);
-            if (!mbar_wait_sleep(&m->empty_u[s], sph)) { fail(ERR_TIMEOUT_HANDOFF); break; }
-            if (lc + 2 < nl) load_u(lc + 2);
-            if (!mbar_wait_sleep(&m->empty_kp[b], bph)) { fail(ERR_TIMEOUT_MMA); break; }
-            if (lc + kKPAhead < nl) load_kp(lc + kKPAhead);
-            prefetch_rec(lc + 3);
-        }
-        // never leave a bulk copy in flight into this CTA's shared memory
-        for (int q = 0; q < 6; ++q)
-            if (issued[q] > 0) (void)mbar_wait_sleep(bars[q], (issued[q] - 1) & 1);
-    }
-
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 0) {
-        tc_fence_after();
-        tmem_dealloc(tmem, K::TCOLS);
-    }
-}
-
-// ------------------------------------------- chain kernel, transposed form ----
-// One CTA per (sequence, head).  The products are written transposed so that
-// the value channel n is the TMEM lane and the state-side operand is the A
-// operand, read from TMEM as packed fp16:
-//
-//   M1  D1^T = S_h [-W; Q̃]^T      (A = S fp16 in TMEM, B = the record's [-W; Q̃])
-//                                  columns 0-63: X^T, 64-127: inter-chunk output
-//   M2  ΔS   = U^T_h K̂            (A = U^T fp16 in TMEM, B = the record's K̂^T)
-//   M4  O4^T = U^T_h (P ⊙ causal)^T   (B = the record's P)
-//
-// Each row of an fp16 A operand (one value channel) carries its own
-// power-of-two scale, so the threads that share a row only exchange one
-// value; there are no shared-memory operand writes.  4 kRQ row warps (warp
-// w: lanes of sub-partition w % 4, part w / 4 of each row) run U, the state
-// update and the output, meeting at one barrier per step that also carries
-// the decision to stop; the next warp issues the MMAs, the last one loads the
-// records.  The output tile goes through shared memory so that it leaves in
-// 16-byte row segments.
-// TMEM loads / stores of N consecutive columns (N = 8, 16 or 32), as many
-// calls as needed for larger N.
-template <int N>
-__device__ __forceinline__ void tmem_ldn(uint32_t taddr, uint32_t (&r)[N]) {
-    if constexpr (N == 16) {
-        tmem_ld16(taddr, r);
-    } else {
-        static_assert(N % 32 == 0, "column count");
-#pragma unroll
-        for (int p = 0; p < N / 32; ++p) tmem_ld32(taddr + p * 32, *reinterpret_cast<uint32_t (*)[32]>(r + p * 32));
-    }
-}
-template <int N>
-__device__ __forceinline__ void tmem_stn(uint32_t taddr, const uint32_t (&r)[N]) {
-    if constexpr (N == 8) {
-        tmem_st8(taddr, r);
-    } else if constexpr (N == 16) {
-        tmem_st16(taddr, r);
-    } else {
-        static_assert(N % 32 == 0, "column count");
-#pragma unroll
-        for (int p = 0; p < N / 32; ++p)
-            tmem_st32(taddr + p * 32, *reinterpret_cast<const uint32_t (*)[32]>(r + p * 32));
-    }
-}
-
-constexpr int kRQ = 2;                     // threads per row (value channel)
-constexpr int kRowWarps = 4 * kRQ;
-constexpr int kRowThreads = 32 * kRowWarps;
-constexpr int kSC = D / kRQ;               // state columns per thread
-constexpr int kTK = C / kRQ;               // tokens per thread (U and output)
-constexpr int kTThreads = kRowThreads + 64;
-constexpr uint32_t TO_A1 = 0;          // [-W; Q̃] fp16 images, 2 stages of 32 KiB
-constexpr uint32_t TO_KH = 65536;      // K̂^T fp16, 2 stages of 16 KiB
-constexpr uint32_t TO_PM = 98304;      // P fp16, 2 stages of 8 KiB
-constexpr uint32_t TO_UT = 114688;     // Ũ fp32, 2 stages of 32 KiB
-constexpr uint32_t TO_OS = 180224;     // output tile [64 tok][128 ch] bf16, 2 buffers of 16 KiB
-constexpr uint32_t TO_MISC = 212992;
-constexpr uint32_t TSMEM = TO_MISC + 12288;
-constexpr uint32_t TT_D1 = 0, TT_DS = 128, TT_O4 = 256, TT_SA = 320, TT_UA = 384, TT_COLS = 512;
-constexpr uint32_t IDESC_H128 = make_idesc(0, 128, 128), IDESC_H64 = make_idesc(0, 128, 64);
-
-struct TMisc {
-    uint64_t full_a1[2], full_u[2], full_kp[2];
-    uint64_t empty_a1[2], empty_u[2], empty_kp[2];
-    uint64_t bar1, bar2, bar4;
-    uint64_t u_ready, s_ready;
-    uint32_t tmem_base;
-    int abort_flag;
-    alignas(16) int ex[2][4];      // record exponents {s_W, s_Q, s_K, s_P}, with the Ũ stage
-    alignas(16) float gam[2][D];   // exp(G_C), with the Ũ stage
-    float xu[2][kRQ * D], xs[2][kRQ * D];   // part-row maxima exchanged between a row's threads
-};
-static_assert(sizeof(TMisc) <= 12288 && TSMEM <= 232448, "chain smem overflow");
-
-template <bool CHANNEL>
-__global__ void __launch_bounds__(kTThreads, 1)
-chain_t_kernel(const uint8_t *__restrict__ recs, const float *h0, float *fin, float *ws_state,
-               const int32_t *__restrict__ cu, int num_seqs, int total_T, int H, int c_begin,
-               int c_end, __nv_bfloat16 *__restrict__ o, uint32_t *err) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t sbase = smem_u32(smem_raw);
     const int chain = blockIdx.x, chains = gridDim.x;
@@ -1197,15 +941,16 @@ chain_t_kernel(const uint8_t *__restrict__ recs, const float *h0, float *fin, fl
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
-    const int sub = warp & 3, qp = (warp >> 2) % kRQ;   // TMEM sub-partition, row quarter
-    const int row = sub * 32 + lane;                     // value channel = TMEM lane
+    const int sub = warp & 3;                          // TMEM sub-partition of this warp
+    const int r = sub * 32 + lane;                     // value channel = TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>(sub * 32) << 16;
-    const size_t sg = (((size_t)n * H + h) * D + row) * D + qp * kSC;
+    const int qc = (warp >> 2) & 3;                    // state warps: key-channel quarter
+    const size_t sg = (((size_t)n * H + h) * D + r) * D + qc * 32;
 
     if (nl == 0) {   // empty sequence: the state passes through
-        if (s_out != nullptr && warp < kRowWarps) {
+        if (s_out != nullptr && warp < kStateWarps) {
 #pragma unroll
-            for (int j = 0; j < kSC; j += 4) {
+            for (int j = 0; j < 32; j += 4) {
                 float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
                 if (s_in != nullptr) x = *reinterpret_cast<const float4 *>(s_in + sg + j);
                 *reinterpret_cast<float4 *>(s_out + sg + j) = x;
@@ -1218,26 +963,24 @@ chain_t_kernel(const uint8_t *__restrict__ recs, const float *h0, float *fin, fl
         return;
     }
     uint8_t *sm = smem_raw;
-    TMisc *m = reinterpret_cast<TMisc *>(sm + TO_MISC);
+    ChainMisc *m = reinterpret_cast<ChainMisc *>(sm + CO_MISC);
     if (tid == 0) {
         for (int s = 0; s < 2; ++s) {
-            mbar_init(&m->full_a1[s], 1);
-            mbar_init(&m->full_u[s], 1);
-            mbar_init(&m->full_kp[s], 1);
-            mbar_init(&m->empty_a1[s], 1);
-            mbar_init(&m->empty_u[s], kRowThreads);
-            mbar_init(&m->empty_kp[s], 1);
+            mbar_init(&m->full[s], 1);
+            mbar_init(&m->empty[s], 1 + kStateThreads + kOutThreads);
         }
-        mbar_init(&m->bar1, 1);
-        mbar_init(&m->bar2, 1);
-        mbar_init(&m->bar4, 1);
-        mbar_init(&m->u_ready, kRowThreads);
-        mbar_init(&m->s_ready, kRowThreads);
+        mbar_init(&m->bar_s, 1);
+        mbar_init(&m->bar_o, 1);
+        mbar_init(&m->o_free, kOutThreads);
+        mbar_init(&m->bar_end, 1);
+        mbar_init(&m->s_hi, kStateThreads);
+        mbar_init(&m->s_lo, kStateThreads);
+        mbar_init(&m->d_free, kStateThreads);
         m->abort_flag = 0;
         fence_barrier_init();
     }
     if (warp == 0) {
-        tmem_alloc(&m->tmem_base, TT_COLS);
+        tmem_alloc(&m->tmem_base, CT_COLS);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -1253,250 +996,233 @@ chain_t_kernel(const uint8_t *__restrict__ recs, const float *h0, float *fin, fl
         return recs + ((size_t)lc * chains + chain) * REC_BYTES;
     };
 
-    if (warp < kRowWarps) {
-        // ============================= row warps: channel `row`, quarter `qp` ====
-        bool stop = false;
-        // Barrier over the row warps; every row warp passes the same sequence of
-        // them, and `stop` leaves it the same in all threads.
-        auto rows_sync = [&]() { stop = named_sync_or(1, kRowThreads, stop || *abort_flag != 0); };
-        // the row's largest |value| over its kRQ parts
-        auto row_max = [&](float mx, float *slots) {
-            slots[qp * D + row] = mx;
-            rows_sync();
+    if (warp < kStateWarps) {
+        // ========= state warps: value channel r, key channels qc*32 .. +31 ========
+        float S[32];
 #pragma unroll
-            for (int k = 0; k < kRQ; ++k) mx = fmaxf(mx, slots[k * D + row]);
-            return mx;
-        };
-        float S[kSC];
-#pragma unroll
-        for (int j = 0; j < kSC; j += 4) {
+        for (int j = 0; j < 32; j += 4) {
             float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
             if (s_in != nullptr) x = *reinterpret_cast<const float4 *>(s_in + sg + j);
             S[j] = x.x; S[j + 1] = x.y; S[j + 2] = x.z; S[j + 3] = x.w;
         }
-        // fp16 copy of the state row (A of M1) with the row's own scale
+        bool stop = false;
+        // S entering chunk lc -> fp16 high and low parts in TMEM with the row's
+        // own scale (the four quarters of a row agree on it through the
+        // barrier, which also agrees on stopping)
         auto publish = [&](int lc) {
             float mx = 0.f;
 #pragma unroll
-            for (int j = 0; j < kSC; ++j) mx = fmaxf(mx, fabsf(S[j]));
-            const int sS = scale_exp(row_max(mx, m->xs[lc & 1]));
-            const float f = exp2i(sS);
-            uint32_t w[kSC / 2];
+            for (int j = 0; j < 32; ++j) mx = fmaxf(mx, fabsf(S[j]));
+            m->xs[lc & 1][qc][r] = mx;
+            stop = named_sync_or(1, kStateThreads, stop || *abort_flag != 0);
 #pragma unroll
-            for (int j = 0; j < kSC / 2; ++j) w[j] = f2h2_bits(S[2 * j] * f, S[2 * j + 1] * f);
-            tmem_stn<kSC / 2>(tmem + lane_off + TT_SA + qp * (kSC / 2), w);
+            for (int k = 0; k < 4; ++k) mx = fmaxf(mx, m->xs[lc & 1][k][r]);
+            const int s = scale_exp(mx);
+            const float f = exp2i(s);
+            // the high part goes first: its MMAs start while the low part is stored
+            uint32_t hi[16], lo[16];
+#pragma unroll
+            for (int jj = 0; jj < 16; ++jj) hi[jj] = f2h2_bits(S[2 * jj] * f, S[2 * jj + 1] * f);
+            tmem_st16(tmem + lane_off + CT_SH + (lc & 1) * 64 + qc * 16, hi);
+            tmem_wait_st();
+            if (qc == 0) m->rowscale[lc & 3][r] = s;
+            tc_fence_before();
+            mbar_arrive(&m->s_hi);
+#pragma unroll
+            for (int jj = 0; jj < 16; ++jj) {
+                const float2 hv = __half22float2(*reinterpret_cast<const __half2 *>(&hi[jj]));
+                lo[jj] = f2h2_bits(fmaf(S[2 * jj], f, -hv.x), fmaf(S[2 * jj + 1], f, -hv.y));
+            }
+            tmem_st16(tmem + lane_off + CT_SL + qc * 16, lo);
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(&m->s_ready);
-            return sS;
+            mbar_arrive(&m->s_lo);
+            return s;
         };
         int sS = publish(0);
         for (int lc = 0; lc < nl && !stop; ++lc) {
-            const uint32_t s = lc & 1, sph = (lc >> 1) & 1;
-            // (a) D1^T: X^T and the inter-chunk output of this thread's tokens
-            if (!warp_wait(&m->bar1, lc & 1)) { fail(ERR_TIMEOUT_MMA); stop = true; }
-            if (!stop && !warp_wait(&m->full_u[s], sph)) { fail(ERR_TIMEOUT_TMA); stop = true; }
-            uint32_t x[kTK], oi[kTK];
-            int sW = 0, sQ = 0, sK = 0, sP = 0;
-            float mx = 0.f;
+            const uint32_t s = lc & 1;
+            const uint8_t *stg = sm + s * CSTAGE;
+            if (!warp_wait(&m->full[s], (lc >> 1) & 1)) { fail(ERR_TIMEOUT_TMA); stop = true; }
+            if (!stop && !warp_wait(&m->bar_s, lc & 1)) { fail(ERR_TIMEOUT_MMA); stop = true; }
             if (!stop) {
                 tc_fence_after();
-                tmem_ldn<kTK>(tmem + lane_off + TT_D1 + qp * kTK, x);
-                tmem_ldn<kTK>(tmem + lane_off + TT_D1 + 64 + qp * kTK, oi);
-                sW = m->ex[s][0]; sQ = m->ex[s][1]; sK = m->ex[s][2]; sP = m->ex[s][3];
-                const float fa = exp2i(-sW), fb = exp2i(-sS);
-                const uint8_t *ut = sm + TO_UT + s * 32768 - REC_UT;
-                tmem_wait_ld();
+                const int *ex = reinterpret_cast<const int *>(stg + REC_EX);
+                const float fs = exp2i(-sS) * exp2i(-ex[0]), fb = exp2i(-ex[2]) * exp2i(-ex[1]);
+                const float *gc = reinterpret_cast<const float *>(stg + REC_GC) + (CHANNEL ? qc * 32 : 0);
 #pragma unroll
-                for (int jj = 0; jj < kTK; ++jj) {
-                    const float u = *reinterpret_cast<const float *>(ut + rec_ut_offset(qp * kTK + jj, row)) +
-                                    __uint_as_float(x[jj]) * fa * fb;
-                    x[jj] = __float_as_uint(u);
-                    mx = fmaxf(mx, fabsf(u));
+                for (int p = 0; p < 2; ++p) {
+                    uint32_t xd[16], xb[16];
+                    tmem_ld16(tmem + lane_off + CT_DS + qc * 32 + p * 16, xd);
+                    tmem_ld16(tmem + lane_off + CT_DB + qc * 32 + p * 16, xb);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const int j = p * 16 + e;
+                        const float gcj = CHANNEL ? gc[j] : gc[0];
+                        S[j] = fmaf(gcj, S[j],
+                                    fmaf(__uint_as_float(xd[e]), fs, __uint_as_float(xb[e]) * fb));
+                    }
                 }
             }
-            const int sU = scale_exp(row_max(mx, m->xu[lc & 1]));
-            if (stop) break;
-            {   // U^T row part (A of M2 and M4): kTK tokens = kTK / 2 packed columns
-                const float f = exp2i(sU);
-                uint32_t w[kTK / 2];
+            tc_fence_before();
+            mbar_arrive(&m->d_free);     // D_S and D_B are read
+            mbar_arrive(&m->empty[s]);   // this stage's gates and exponents are read
+            // S entering chunk lc + 1: its high part goes to the buffer that
+            // chunk lc - 1 read.  This chunk's MMA_O may still read the other one;
+            // MMA_S and MMA_O of chunk lc - 1 were issued before the commit of
+            // bar_s above, so they are complete.
+            if (lc + 1 < nl) sS = publish(lc + 1);
+        }
+        if (s_out != nullptr) {
 #pragma unroll
-                for (int j = 0; j < kTK / 2; ++j)
-                    w[j] = f2h2_bits(__uint_as_float(x[2 * j]) * f, __uint_as_float(x[2 * j + 1]) * f);
-                tmem_stn<kTK / 2>(tmem + lane_off + TT_UA + qp * (kTK / 2), w);
-                tmem_wait_st();
-                tc_fence_before();
-                mbar_arrive(&m->u_ready);
+            for (int j = 0; j < 32; j += 4)
+                *reinterpret_cast<float4 *>(s_out + sg + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+        }
+    } else if (warp < kIssuerWarp) {
+        // ================== output warps: value channel r, all 64 tokens ==========
+        const int otid = tid - kStateThreads;
+        bool stop = false;
+        for (int lc = 0; lc < nl; ++lc) {
+            const uint32_t s = lc & 1;
+            const uint8_t *stg = sm + s * CSTAGE;
+            // take this chunk's O⁰ column r and exponents, then free the record
+            // stage at once, so the loader can refill it early
+            if (!warp_wait(&m->full[s], (lc >> 1) & 1)) { fail(ERR_TIMEOUT_TMA); stop = true; }
+            uint32_t zp[32];
+            int eq = 0, eo = 0;
+            if (!stop) {
+                const uint16_t *oz = reinterpret_cast<const uint16_t *>(stg + REC_OZ) + r;
+#pragma unroll
+                for (int e = 0; e < 32; ++e)
+                    zp[e] = (uint32_t)oz[(2 * e) * 128] | ((uint32_t)oz[(2 * e + 1) * 128] << 16);
+                const int *ex = reinterpret_cast<const int *>(stg + REC_EX);
+                eq = ex[3];
+                eo = ex[4];
             }
-            // (b) S = S Diag(exp(G_C)) + ΔS
-            if (!warp_wait(&m->bar2, lc & 1)) { fail(ERR_TIMEOUT_MMA); stop = true; }
+            mbar_arrive(&m->empty[s]);
+            if (!stop && !warp_wait(&m->bar_o, lc & 1)) { fail(ERR_TIMEOUT_MMA); stop = true; }
             if (!stop) {
                 tc_fence_after();
-                const float f1 = exp2i(-sK), f2 = exp2i(-sU);
-                const float *gam = m->gam[s] + qp * kSC;
-                uint32_t d[kSC];
-                tmem_ldn<kSC>(tmem + lane_off + TT_DS + qp * kSC, d);
-                tmem_wait_ld();
+                const float fo = exp2i(-m->rowscale[lc & 3][r]) * exp2i(-eq), fz = exp2i(-eo);
+                __nv_bfloat16 *tile = reinterpret_cast<__nv_bfloat16 *>(sm + CO_OT) + r;
 #pragma unroll
-                for (int jj = 0; jj < kSC; ++jj) {
-                    const float gc = CHANNEL ? gam[jj] : m->gam[s][0];
-                    S[jj] = fmaf(gc, S[jj], __uint_as_float(d[jj]) * f1 * f2);
-                }
-                tc_fence_before();
-                mbar_arrive(&m->empty_u[s]);   // Ũ, exponents and gate of this stage are read
-            }
-            // (stop may differ between warps here; the barrier in (c) settles it)
-            const int sS_next = (lc + 1 < nl) ? publish(lc + 1) : 0;
-            // (c) output rows: O^T = O_inter^T + O4^T, unscaled, for this thread's
-            //     tokens, staged as a [token][channel] tile
-            if (!warp_wait(&m->bar4, lc & 1)) { fail(ERR_TIMEOUT_MMA); stop = true; }
-            if (!stop) {
-                uint32_t o4[kTK];
-                tc_fence_after();
-                tmem_ldn<kTK>(tmem + lane_off + TT_O4 + qp * kTK, o4);
-                tmem_wait_ld();
-                const float fq1 = exp2i(-sQ), fq2 = exp2i(-sS), fp1 = exp2i(-sP), fp2 = exp2i(-sU);
-                const uint32_t stile = sbase + TO_OS + s * 16384 + qp * kTK * 256 + row * 2;
+                for (int p = 0; p < 4; ++p) {
+                    uint32_t x[16];
+                    tmem_ld16(tmem + lane_off + CT_DO + p * 16, x);
+                    tmem_wait_ld();
 #pragma unroll
-                for (int jj = 0; jj < kTK; ++jj) {
-                    const __nv_bfloat16 b = __float2bfloat16_rn(__uint_as_float(oi[jj]) * fq1 * fq2 +
-                                                                __uint_as_float(o4[jj]) * fp1 * fp2);
-                    st_shared_b16(stile + jj * 256, *reinterpret_cast<const uint16_t *>(&b));
+                    for (int e = 0; e < 16; e += 2) {
+                        const float2 z = __half22float2(*reinterpret_cast<const __half2 *>(&zp[(p * 16 + e) / 2]));
+                        tile[(p * 16 + e) * 128] = __float2bfloat16_rn(fmaf(__uint_as_float(x[e]), fo, z.x * fz));
+                        tile[(p * 16 + e + 1) * 128] =
+                            __float2bfloat16_rn(fmaf(__uint_as_float(x[e + 1]), fo, z.y * fz));
+                    }
                 }
             }
-            rows_sync();
+            tc_fence_before();
+            mbar_arrive(&m->o_free);
+            stop = named_sync_or(3, kOutThreads, stop || *abort_flag != 0);
             if (stop) break;
             {   // 64 rows x 256 bytes leave as 16-byte segments; rows past the end stay
                 const int cc = c_begin + lc;
                 const int cl = min(C, len - cc * C);
-                const uint32_t tile = sbase + TO_OS + s * 16384;
+                const uint4 *tile = reinterpret_cast<const uint4 *>(sm + CO_OT);
 #pragma unroll
-                for (int q = 0; q < 1024 / kRowThreads; ++q) {
-                    const int e = q * kRowThreads + tid;   // segment: row e / 16, 16 bytes e % 16
+                for (int q = 0; q < 1024 / kOutThreads; ++q) {
+                    const int e = q * kOutThreads + otid;   // row e / 16, segment e % 16
                     const int i = e >> 4, seg = e & 15;
-                    if (i < cl) {
-                        const uint4 v = ld_shared_v4(tile + i * 256 + seg * 16);
-                        *reinterpret_cast<uint4 *>(o + ((size_t)(t0 + cc * C + i) * H + h) * D + seg * 8) = v;
-                    }
+                    if (i < cl)
+                        *reinterpret_cast<uint4 *>(o + ((size_t)(t0 + cc * C + i) * H + h) * D + seg * 8) = tile[e];
                 }
             }
-            sS = sS_next;
+            named_sync(3, kOutThreads);   // the tile is free again
         }
-        if (s_out != nullptr) {
-#pragma unroll
-            for (int j = 0; j < kSC; j += 4)
-                *reinterpret_cast<float4 *>(s_out + sg + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
-        }
-    } else if (warp == kRowWarps) {
+    } else if (warp == kIssuerWarp) {
         // ======================================================= MMA issuer ====
         if (lane == 0) {
             for (int lc = 0; lc < nl; ++lc) {
                 if (*abort_flag) break;
-                const uint32_t s = lc & 1, sph = (lc >> 1) & 1;
-                if (!mbar_wait_sleep(&m->full_a1[s], sph)) { fail(ERR_TIMEOUT_TMA); break; }
-                if (!mbar_wait_sleep(&m->s_ready, lc & 1)) { fail(ERR_TIMEOUT_HANDOFF); break; }
+                const uint32_t s = lc & 1;
+                const uint32_t stg = sbase + s * CSTAGE;
+                if (!mbar_wait_sleep(&m->full[s], (lc >> 1) & 1)) { fail(ERR_TIMEOUT_TMA); break; }
+                if (lc > 0 && !mbar_wait_sleep(&m->d_free, (lc - 1) & 1)) { fail(ERR_TIMEOUT_HANDOFF); break; }
                 tc_fence_after();
-                const uint64_t d_a1 = sw128_kmajor_desc(sbase + TO_A1 + s * 32768);
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    mma_f16_ss(tmem + CT_DB, sw128_kmajor_desc(stg + REC_UT + k * 32),
+                               sw128_mnmajor_desc(stg + REC_KH + k * 2048, 8192, 1024), IDESC_DB, k != 0);
+                if (!mbar_wait_sleep(&m->s_hi, lc & 1)) { fail(ERR_TIMEOUT_HANDOFF); break; }
+                tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < 8; ++k)
-                    mma_f16_ts(tmem + TT_D1, tmem + TT_SA + k * 8,
-                               d_a1 + (((k >> 2) * 16384 + (k & 3) * 32) >> 4), IDESC_H128, k != 0);
-                mma_commit(&m->bar1);
-                mma_commit(&m->empty_a1[s]);
-                if (!mbar_wait_sleep(&m->full_kp[s], sph)) { fail(ERR_TIMEOUT_TMA); break; }
-                if (!mbar_wait_sleep(&m->u_ready, lc & 1)) { fail(ERR_TIMEOUT_HANDOFF); break; }
+                    mma_f16_ts(tmem + CT_DS, tmem + CT_SH + s * 64 + k * 8,
+                               sw128_kmajor_desc(stg + REC_NT + (k >> 2) * 16384 + (k & 3) * 32),
+                               IDESC_H128, k != 0);
+                if (!mbar_wait_sleep(&m->s_lo, lc & 1)) { fail(ERR_TIMEOUT_HANDOFF); break; }
                 tc_fence_after();
-                const uint64_t d_kh = sw128_kmajor_desc(sbase + TO_KH + s * 16384);
-                const uint64_t d_pm = sw128_kmajor_desc(sbase + TO_PM + s * 8192);
 #pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    mma_f16_ts(tmem + TT_DS, tmem + TT_UA + k * 8, d_kh + ((k * 32) >> 4), IDESC_H128, k != 0);
-                mma_commit(&m->bar2);
+                for (int k = 0; k < 8; ++k)
+                    mma_f16_ts(tmem + CT_DS, tmem + CT_SL + k * 8,
+                               sw128_kmajor_desc(stg + REC_NT + (k >> 2) * 16384 + (k & 3) * 32),
+                               IDESC_H128, 1);
+                mma_commit(&m->bar_s);
+                if (lc >= 1 && !mbar_wait_sleep(&m->o_free, (lc - 1) & 1)) {
+                    fail(ERR_TIMEOUT_HANDOFF);
+                    break;
+                }
+                tc_fence_after();
 #pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    mma_f16_ts(tmem + TT_O4, tmem + TT_UA + k * 8, d_pm + ((k * 32) >> 4), IDESC_H64, k != 0);
-                mma_commit(&m->bar4);
-                mma_commit(&m->empty_kp[s]);
+                for (int k = 0; k < 8; ++k)
+                    mma_f16_ts(tmem + CT_DO, tmem + CT_SH + s * 64 + k * 8,
+                               sw128_kmajor_desc(stg + REC_QP + (k >> 2) * 8192 + (k & 3) * 32),
+                               IDESC_H64, k != 0);
+                mma_commit(&m->bar_o);
+                mma_commit(&m->empty[s]);
             }
+            // every MMA issued here is complete before TMEM is freed
+            mma_commit(&m->bar_end);
+            (void)mbar_wait_sleep(&m->bar_end, 0);
         }
     } else if (lane == 0) {
         // ==================================================== record loader ====
-        const uint32_t gbytes = CHANNEL ? 512u : 16u;
-        uint32_t issued[6] = {0, 0, 0, 0, 0, 0};
-        uint64_t *bars[6] = {&m->full_a1[0], &m->full_a1[1], &m->full_u[0], &m->full_u[1],
-                             &m->full_kp[0], &m->full_kp[1]};
-        auto load_a1 = [&](int lc) {
-            const int s = lc & 1;
-            mbar_arrive_expect_tx(&m->full_a1[s], 32768);
-            bulk_load(sm + TO_A1 + s * 32768, rec_of(lc) + REC_A1, 32768, &m->full_a1[s]);
-            ++issued[s];
-        };
-        auto load_u = [&](int lc) {
-            const int s = lc & 1;
-            const uint8_t *r = rec_of(lc);
-            mbar_arrive_expect_tx(&m->full_u[s], 32768 + 16 + gbytes);
-            bulk_load(sm + TO_UT + s * 32768, r + REC_UT, 32768, &m->full_u[s]);
-            bulk_load(m->ex[s], r + REC_EX, 16, &m->full_u[s]);
-            bulk_load(m->gam[s], r + REC_GC, gbytes, &m->full_u[s]);
-            ++issued[2 + s];
-        };
-        auto load_kp = [&](int lc) {
-            const int s = lc & 1;
-            const uint8_t *r = rec_of(lc);
-            mbar_arrive_expect_tx(&m->full_kp[s], 16384 + 8192);
-            bulk_load(sm + TO_KH + s * 16384, r + REC_KH, 16384, &m->full_kp[s]);
-            bulk_load(sm + TO_PM + s * 8192, r + REC_PM, 8192, &m->full_kp[s]);
-            ++issued[4 + s];
-        };
-        auto prefetch_rec = [&](int lc) {
-            if (lc < nl) {
-                const uint8_t *r = rec_of(lc);
-#pragma unroll
-                for (int q = 0; q < 5; ++q) bulk_prefetch_l2(r + q * 18128, 18128);
-            }
-        };
-        load_a1(0);
-        load_kp(0);
-        load_u(0);
-        if (nl > 1) {
-            load_a1(1);
-            load_u(1);
-            load_kp(1);
-        }
-        prefetch_rec(2);
-        prefetch_rec(3);
+        uint32_t issued[2] = {0, 0};
         for (int lc = 0; lc < nl; ++lc) {
             if (*abort_flag) break;
-            const uint32_t s = lc & 1, sph = (lc >> 1) & 1;
-            if (!mbar_wait_sleep(&m->empty_a1[s], sph)) { fail(ERR_TIMEOUT_MMA); break; }
-            if (lc + 2 < nl) load_a1(lc + 2);
-            if (!mbar_wait_sleep(&m->empty_kp[s], sph)) { fail(ERR_TIMEOUT_MMA); break; }
-            if (lc + 2 < nl) load_kp(lc + 2);
-            if (!mbar_wait_sleep(&m->empty_u[s], sph)) { fail(ERR_TIMEOUT_HANDOFF); break; }
-            if (lc + 2 < nl) load_u(lc + 2);
-            prefetch_rec(lc + 4);
+            const int s = lc & 1;
+            if (lc >= 2 && !mbar_wait_sleep(&m->empty[s], ((lc - 2) >> 1) & 1)) {
+                fail(ERR_TIMEOUT_HANDOFF);
+                break;
+            }
+            mbar_arrive_expect_tx(&m->full[s], REC_BYTES);
+            bulk_load(sm + s * CSTAGE, rec_of(lc), REC_BYTES, &m->full[s]);
+            ++issued[s];
+            if (lc + 2 < nl) {
+                const uint8_t *pr = rec_of(lc + 2);
+                bulk_prefetch_l2(pr, REC_BYTES / 2);
+                bulk_prefetch_l2(pr + REC_BYTES / 2, REC_BYTES / 2);
+            }
         }
         // never leave a bulk copy in flight into this CTA's shared memory
-        for (int q = 0; q < 6; ++q)
-            if (issued[q] > 0) (void)mbar_wait_sleep(bars[q], (issued[q] - 1) & 1);
+        for (int s = 0; s < 2; ++s)
+            if (issued[s] > 0) (void)mbar_wait_sleep(&m->full[s], (issued[s] - 1) & 1);
     }
 
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
-        tmem_dealloc(tmem, TT_COLS);
+        tmem_dealloc(tmem, CT_COLS);
     }
 }
 
 // ------------------------------------------------------------------ host ----
 
 constexpr size_t kHeaderBytes = 256;                        // error word
-constexpr size_t kMaxRecordBytes = size_t(1) << 30;         // records per window
+constexpr size_t kMaxRecordBytes = size_t(4) << 30;         // records per window
 // Up to 64 chains the two kernels beat the single-kernel plan: its chunk
 // period is set by the chunk-local work, which the prep kernel spreads over
-// all SMs.  With more chains that plan already keeps most SMs busy and the
-// prep kernel's extra record traffic no longer pays (measured on B200).
+// all SMs.
 constexpr int kSplitMaxChains = 64;
 
 struct SplitPlan {
@@ -1506,10 +1232,9 @@ struct SplitPlan {
 };
 
 // Pipeline pieces of one window: the prep kernel of piece k + 1 runs beside
-// the chain kernel of piece k, and on the SMs the chain leaves free a chunk's
-// prep takes about 3/4 of a chunk's chain step, so each piece may be 1.3 times
-// the one before: 12, 16, 21, 27, 35, ... chunks, the last one the remainder.
-// Writes the piece boundaries (count + 1 of them) and returns the count.
+// the chain kernel of piece k; each piece is 1.3 times the one before:
+// 12, 16, 21, 27, 35, ... chunks, the last one the remainder.  Writes the
+// piece boundaries (count + 1 of them) and returns the count.
 constexpr int kMaxPieces = 32;
 int piece_schedule(int max_chunks, int *bounds) {
     int n = 0, c = 0, size = 12;
@@ -1546,7 +1271,6 @@ bool make_split_plan(int num_seqs, int total_T, int H, SplitPlan &p, bool equal_
     return true;
 }
 
-
 // Per-device helper streams for the pipelined plan: chain kernels on a
 // high-priority stream, prep kernels on a low-priority one, forked from and
 // joined back into the caller's stream with events (capturable in a graph).
@@ -1580,19 +1304,6 @@ cudaError_t get_helpers(Helpers **out) {
     return cudaSuccess;
 }
 
-template <int NB>
-cudaError_t launch_chain(bool channel, int chains, const uint8_t *recs, const float *h0, float *fin,
-                         float *state, const int32_t *cu, int num_seqs, int total_T, int H, int c0,
-                         int c1, __nv_bfloat16 *o, uint32_t *err, cudaStream_t stream) {
-    using K = Chain<NB>;
-    auto kern = channel ? chain_kernel<true, NB> : chain_kernel<false, NB>;
-    cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void *>(kern), (int)K::SMEM);
-    if (e != cudaSuccess) return e;
-    kern<<<(unsigned)(chains * (D / NB)), K::kThreads, K::SMEM, stream>>>(
-        recs, h0, fin, state, cu, num_seqs, total_T, H, c0, c1, o, err);
-    return cudaGetLastError();
-}
-
 }  // namespace
 
 size_t tcgen05_split_workspace_bytes(int num_seqs, int total_T, int H) {
@@ -1617,21 +1328,15 @@ cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, co
     auto prep = channel ? prep_kernel<true> : prep_kernel<false>;
     e = ensure_dynamic_smem(reinterpret_cast<const void *>(prep), (int)PREP_SMEM);
     if (e != cudaSuccess) return e;
+    auto chain_k = channel ? chain_kernel<true> : chain_kernel<false>;
+    e = ensure_dynamic_smem(reinterpret_cast<const void *>(chain_k), (int)CHAIN_SMEM);
+    if (e != cudaSuccess) return e;
     float *state = (p.windows > 1 || p.pieces > 1) ? reinterpret_cast<float *>(ws + p.state_off) : nullptr;
     uint8_t *recs = ws + p.rec_off;
     __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(o);
-    // Few chains: split d_v over four CTAs each (NB = 32), so that more SMs
-    // share the chain work; otherwise one CTA per chain, transposed form.
-    const bool dv_split = p.chains * 4 <= 148;
-    auto chain_t = channel ? chain_t_kernel<true> : chain_t_kernel<false>;
-    e = ensure_dynamic_smem(reinterpret_cast<const void *>(chain_t), (int)TSMEM);
-    if (e != cudaSuccess) return e;
     auto run_chain = [&](int c0, int c1, const uint8_t *r, cudaStream_t st) {
-        if (dv_split)
-            return launch_chain<32>(channel, p.chains, r, h0, fin, state, cu, num_seqs, total_T, H, c0, c1,
-                                    out, err, st);
-        chain_t<<<(unsigned)p.chains, kTThreads, TSMEM, st>>>(r, h0, fin, state, cu, num_seqs, total_T, H,
-                                                                c0, c1, out, err);
+        chain_k<<<(unsigned)p.chains, kChainThreads, CHAIN_SMEM, st>>>(r, h0, fin, state, cu, num_seqs,
+                                                                        total_T, H, c0, c1, out, err);
         return cudaGetLastError();
     };
     auto run_prep = [&](int c0, int c1, uint8_t *r, cudaStream_t st) {

@@ -308,6 +308,23 @@ __device__ __forceinline__ uint64_t sw64_mnmajor_desc(uint32_t addr, uint32_t lb
     return d;
 }
 
+// Shared-memory matrix descriptor for an MN-major 16-bit operand in the
+// 128-byte swizzled canonical layout: rows of 128 bytes (64 elements along M
+// or N), one row per K index, 16-byte chunks XOR-swizzled by row % 8 within
+// 1024-byte atoms of 8 rows; `lbo` is the byte distance between 64-element
+// blocks along M/N, `sbo` the distance between groups of 8 rows along K.
+// This is the layout a 128-byte-swizzled TMA box of 64 elements per row
+// lands in, so such a tile can feed an MMA without being transposed.
+__device__ __forceinline__ uint64_t sw128_mnmajor_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+    uint64_t d = 0;
+    d |= (uint64_t)((addr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1u << 46;                       // descriptor version (sm_100)
+    d |= (uint64_t)2u << 61;                       // layout: 128-byte swizzle
+    return d;
+}
+
 // Instruction descriptor: fp32 accumulate, K-major A and B.
 // ab_format: 1 = bf16, 2 = tf32.
 __host__ __device__ constexpr uint32_t make_idesc(uint32_t ab_format, uint32_t M, uint32_t N) {
@@ -317,6 +334,8 @@ __host__ __device__ constexpr uint32_t make_idesc(uint32_t ab_format, uint32_t M
            | ((N >> 3) << 17)        // N / 8
            | ((M >> 4) << 24);       // M / 16
 }
+constexpr uint32_t kIdescAMN = 1u << 15;   // A is MN-major (transposed)
+constexpr uint32_t kIdescBMN = 1u << 16;   // B is MN-major (transposed)
 
 // Byte offset of element (row, 16-byte chunk, byte-in-chunk) inside a block
 // stored in the 128-byte swizzled layout (rows of 128 bytes).

@@ -63,8 +63,9 @@ def rel_frob(a: np.ndarray, b: np.ndarray) -> float:
     return float(np.linalg.norm(a - b) / den) if den > 0 else float(np.linalg.norm(a - b))
 
 
-def check(inp, o_gpu, fin_gpu, o_ref, fin_ref, label=""):
-    """Assert the contract tolerances; returns the error summary."""
+def check(inp, o_gpu, fin_gpu, o_ref, fin_ref, label="", state_rel_tol=TOL_BF16_STATE_REL):
+    """Assert the contract tolerances (a case may pass a derived state
+    tolerance, stating why); returns the error summary."""
     o = o_gpu.float().cpu().numpy().astype(np.float64) if torch.is_tensor(o_gpu) else o_gpu
     f = fin_gpu.float().cpu().numpy().astype(np.float64) if torch.is_tensor(fin_gpu) else fin_gpu
     assert o.shape == o_ref.shape, (o.shape, o_ref.shape)
@@ -86,6 +87,6 @@ def check(inp, o_gpu, fin_gpu, o_ref, fin_ref, label=""):
     else:
         assert err_o <= TOL_BF16_O, f"{label}: o max-abs {err_o}"
         if fin_ref is not None:
-            assert out["rel_frob_state_max"] <= TOL_BF16_STATE_REL, f"{label}: {out}"
-            assert out["rel_frob_state"] <= TOL_BF16_STATE_REL, f"{label}: {out}"
+            assert out["rel_frob_state_max"] <= state_rel_tol, f"{label}: {out}"
+            assert out["rel_frob_state"] <= state_rel_tol, f"{label}: {out}"
     return out

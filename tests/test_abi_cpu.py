@@ -113,10 +113,10 @@ def test_workspace_and_path_queries(lib):
 
 def test_plan_selection_and_workspace_sizes(lib):
     """The tcgen05 family runs as two plans: the chunk-parallel one with the
-    reported workspace (90,640 bytes of chunk records per chunk and head, in
-    windows of at most 1 GiB), the single-kernel one with 16 bytes."""
+    reported workspace (98,848 bytes of chunk records per chunk and head, in
+    windows of at most 4 GiB), the single-kernel one with 16 bytes."""
     S, CH, BF = gdr.GDR_GATE_SCALAR, gdr.GDR_GATE_CHANNEL, gdr.GDR_BF16
-    rec = 90640
+    rec = 98848
     # one window of 128 chunks, run as 4 pipelined pieces: 64 KiB of state per
     # head between pieces
     nb = gdr.gdr_prefill_workspace_size(1, 8192, 16, 128, 128, S, BF)
@@ -134,11 +134,11 @@ def test_plan_selection_and_workspace_sizes(lib):
     # fp32 I/O and other head sizes: the CUDA-core kernel, no workspace
     assert gdr.gdr_prefill_plan(1, 8192, 16, 128, 128, S, gdr.GDR_F32, 0) == gdr.GDR_PATH_SIMT
     assert gdr.gdr_prefill_plan(1, 8192, 16, 64, 64, S, BF, 0) == gdr.GDR_PATH_SIMT
-    # 64 heads x 250 chunks: records beyond 1 GiB -> windows of 185 chunks with
+    # 64 heads x 700 chunks: records beyond 4 GiB -> windows of 678 chunks with
     # 64 KiB of state per head between them
-    nb = gdr.gdr_prefill_workspace_size(1, 16000, 64, 128, 128, S, BF)
+    nb = gdr.gdr_prefill_workspace_size(1, 44800, 64, 128, 128, S, BF)
     state = 64 * 128 * 128 * 4
-    assert nb == ((256 + state + 1023) // 1024) * 1024 + 185 * 64 * rec
+    assert nb == ((256 + state + 1023) // 1024) * 1024 + 678 * 64 * rec
     # a tcgen05 problem without any workspace is refused before any launch
     assert _prefill(lib, dk=128, dv=128, io=1) == gdr.GDR_ERR_WORKSPACE
 

@@ -36,13 +36,14 @@ def test_pipelined_plan_launch_accounting():
     # 128 chunks in one window: pieces of 12, 16, 21, 27, 35 and the last 17;
     # each piece is one prep and one chain launch
     assert bench.split_launches(I.workload("gdn_prefill")) == 12
-    # 64 chains of 90,640-byte records in 1 GiB windows: 185 chunks per
+    # 64 chains of 98,848-byte records in 4 GiB windows: 678 chunks per
     # window.  The two equal sequences go without cu_seqlens, so the plan
-    # knows each has 512 chunks: 3 windows, one piece each
+    # knows each has 512 chunks: one window, in 10 pipelined pieces (12, 16,
+    # 21, 27, 35, 46, 60, 78, 101 and the last 116)
     kda = I.workload("kda_prefill")
-    window = (1 << 30) // (64 * 90640)
-    assert window == 185
-    assert bench.split_launches(kda) == 2 * -(-512 // window) == 6
+    window = (4 << 30) // (64 * 98848)
+    assert window == 678
+    assert bench.split_launches(kda) == 2 * 10
     # with packed lengths only total_T bounds a sequence: varlen has 128
     # chains, beyond the plan, so only the counting is checked here
     assert bench.split_launches(I.workload("gqa_prefill")) == 12

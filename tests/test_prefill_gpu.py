@@ -238,14 +238,14 @@ def test_channel_gate_decay_strengths(c_gate, plan):
 
 @pytest.mark.parametrize("mode", [I.SCALAR, I.CHANNEL])
 def test_chunk_parallel_plan_in_windows(mode):
-    """64 heads x 16,000 tokens: the chunk records exceed the 1 GiB window,
+    """64 heads x 44,800 tokens: the chunk records exceed the 4 GiB window,
     so the chunk-parallel plan runs in two windows of chunks with the state
-    handed between them through the workspace (sequence of 250 chunks, a
-    window of 185).  Sampled heads against the oracle, in-place state."""
-    T, H = 16000, 64
+    handed between them through the workspace (sequence of 700 chunks, a
+    window of 678).  Sampled heads against the oracle, in-place state."""
+    T, H = 44800, 64
     nb = gdr.gdr_prefill_workspace_size(1, T, H, 128, 128, 0 if mode == I.SCALAR else 1,
                                         gdr.GDR_BF16)
-    assert nb > (1 << 30)
+    assert (1 << 30) < nb < 700 * H * 98848   # the workspace holds one window, not all records
     inp = I.make_inputs(total_T=T, H=H, d_k=128, gate_mode=mode, io_dtype=torch.bfloat16,
                         c=0.1, h0_std=0.02, seed=51)
     d = to_device(inp)
@@ -261,14 +261,15 @@ def test_chunk_parallel_plan_in_windows(mode):
 
 @pytest.mark.parametrize("mode", [I.SCALAR, I.CHANNEL])
 def test_plans_agree(mode):
-    """Both tcgen05 plans compute the same chunk algebra in the same
-    precisions: their outputs agree far inside the oracle tolerance."""
+    """Both tcgen05 plans compute the same chunk algebra (the chunk-parallel
+    plan with more of its operands split into high and low halves): their
+    outputs agree within the contract tolerances."""
     inp = I.make_inputs(total_T=1000, H=4, d_k=128, gate_mode=mode, io_dtype=torch.bfloat16,
                         cu_seqlens=[0, 333, 334, 1000], c=0.1, h0_std=0.02, seed=52)
     o1, f1 = gpu_prefill(inp, plan="split")
     o2, f2 = gpu_prefill(inp, plan="single")
-    assert float((o1.float() - o2.float()).abs().max()) <= 4e-3
-    assert float((f1 - f2).norm() / f2.norm()) <= 1e-4
+    assert float((o1.float() - o2.float()).abs().max()) <= TOL_BF16_O
+    assert float((f1 - f2).norm() / f2.norm()) <= 1e-3
 
 
 @pytest.mark.parametrize("mode", [I.SCALAR, I.CHANNEL])
@@ -291,9 +292,9 @@ def test_chunk_parallel_plan_in_pipelined_pieces(mode):
 @pytest.mark.parametrize("mode", [I.SCALAR, I.CHANNEL])
 def test_equal_lengths_plan_knows_each_sequence_length(mode):
     # 2 x 6000 tokens x 32 heads: with cu_seqlens the plan bounds a sequence
-    # by all 12000 tokens (188 chunks: two windows of 185); without it each
-    # sequence has 94 chunks (one window, pipelined pieces).  Both match the
-    # oracle, and the two runs agree.
+    # by all 12000 tokens (188 chunks, pipelined pieces past the second
+    # sequence's end); without it each sequence has 94 chunks.  Both match
+    # the oracle, and the two runs agree.
     inp = I.make_inputs(total_T=12000, H=32, d_k=128, num_seqs=2, gate_mode=mode,
                         io_dtype=torch.bfloat16, c=0.05, h0_std=0.02, seed=90)
     o1, f1 = gpu_prefill(inp, use_cu=True)
