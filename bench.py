@@ -255,25 +255,28 @@ def decode_work(inp):
 
 
 def split_launches(inp):
-    """Kernel launches of the chunk-parallel plan: a prep and a chain kernel
-    per window of chunks (the library bounds the chunk records of one window
-    to 4 GiB at 98,848 bytes per chunk and head), and per pipeline piece when
-    a single window is cut into pieces."""
+    """Kernel launches of the chunk-parallel plan, mirroring its plan: one
+    launch that numbers every sequence's chunks, then a prep and a chain kernel
+    per window of chunks (a window holds at most 8 GiB of records at 98,848
+    bytes per chunk and head), or, when one window holds every record and
+    there are at most 64 (sequence, head) chains, per pipeline piece."""
     chains = inp.num_seqs * inp.H
     # equal lengths go without cu_seqlens, so the library knows each
     # sequence's length; otherwise total_T bounds it
-    longest = inp.total_T // inp.num_seqs if inp.equal_lengths() else inp.total_T
+    equal = inp.equal_lengths()
+    longest = inp.total_T // inp.num_seqs if equal else inp.total_T
     max_chunks = -(-longest // 64)
-    window = max(1, min(max_chunks, (4 << 30) // (chains * 98848)))
-    windows = -(-max_chunks // window)
-    pieces = 1
-    if windows == 1:   # pipelined pieces of 12, 16, 21, 27, ... chunks (1.3x growth)
-        pieces, c, size = 0, 0, 12
-        while c < max_chunks and pieces < 32:
-            c = max_chunks if pieces + 1 == 32 else min(c + size, max_chunks)
-            pieces += 1
-            size = (size * 13 + 9) // 10
-    return 2 * windows * pieces
+    max_total = inp.num_seqs * max_chunks if equal else -(-inp.total_T // 64) + inp.num_seqs
+    window = min(max_total, (8 << 30) // (inp.H * 98848))
+    windows = -(-max_total // window)
+    if windows > 1 or chains > 64:
+        return 1 + 2 * windows
+    pieces, c, size = 0, 0, 12   # pieces of 12, 16, 21, 27, ... chunks (1.3x growth)
+    while c < max_chunks and pieces < 32:
+        c = max_chunks if pieces + 1 == 32 else min(c + size, max_chunks)
+        pieces += 1
+        size = (size * 13 + 9) // 10
+    return 1 + 2 * pieces
 
 
 class PrefillCase:

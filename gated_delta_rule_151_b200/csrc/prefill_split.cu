@@ -43,7 +43,7 @@
 // rounding at about 2^-22 where a single fp16 or tf32 rounding per chunk
 // would be amplified by the conditioning of I + A (up to ~10 at beta = 2).
 // Records take 98,848 bytes per (chunk, head); problems whose records exceed
-// 4 GiB run in windows of chunks, the state passing between windows
+// 8 GiB run in windows of chunks, the state passing between windows
 // through the workspace.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -133,6 +133,65 @@ __device__ __forceinline__ uint16_t bf16_bits(float x) {
 __device__ __forceinline__ void st_global_v4(uint8_t *p, uint32_t a, uint32_t b, uint32_t c,
                                              uint32_t d) {
     *reinterpret_cast<uint4 *>(p) = make_uint4(a, b, c, d);
+}
+
+// ------------------------------------------------------------- chunk map ----
+// Chunks are numbered globally, sequence after sequence: sequence n owns
+// global chunks base[n] .. base[n+1] - 1, base computed on the device from
+// cu_seqlens (or the equal lengths).  The record of (global chunk, head) sits
+// at slot (gc - w0) * H + h of the resident window [w0, w1).  A launch covers
+// either a window of global chunks (by_window) or the local chunks c0 .. c1-1
+// of every sequence (a pipeline piece, when one window holds every record).
+struct ChunkMap {
+    const int32_t *base;   // device [num_seqs + 1]
+    int w0, w1;            // resident global chunks
+    int c0, c1;            // local chunks of every sequence
+    int win;               // window index (state slots between windows)
+    int by_window;
+};
+
+// base[n] = sum over m < n of the chunk count of sequence m (exclusive
+// prefix sum, one CTA of 1024 threads); base[num_seqs] = total chunks.
+__global__ void __launch_bounds__(1024)
+chunk_base_kernel(const int32_t *__restrict__ cu, int num_seqs, int total_T, int32_t *base) {
+    __shared__ int wsum[32];
+    __shared__ int carry;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (tid == 0) carry = 0;
+    __syncthreads();
+    for (int start = 0; start < num_seqs; start += 1024) {
+        const int n = start + tid;
+        int v = 0;
+        if (n < num_seqs) {
+            int t0, len;
+            sequence_range(cu, n, num_seqs, total_T, t0, len);
+            v = (len + C - 1) / C;
+        }
+        int x = v;   // inclusive scan within the warp
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, off);
+            if (lane >= off) x += y;
+        }
+        if (lane == 31) wsum[warp] = x;
+        __syncthreads();
+        if (warp == 0) {
+            int w = wsum[lane];
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, w, off);
+                if (lane >= off) w += y;
+            }
+            wsum[lane] = w;   // inclusive over warps
+        }
+        __syncthreads();
+        const int before = carry + (warp > 0 ? wsum[warp - 1] : 0);
+        if (n < num_seqs) base[n] = before + x - v;
+        __syncthreads();
+        if (tid == 0) carry += wsum[31];
+        __syncthreads();
+    }
+    if (tid == 0) base[num_seqs] = carry;
 }
 
 // ------------------------------------------------------------ prep kernel ----
@@ -237,24 +296,41 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
 prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
             const __grid_constant__ CUtensorMap tm_v, const float *__restrict__ g,
             const float *__restrict__ beta, const int32_t *__restrict__ cu, int num_seqs,
-            int total_T, int Hqk, int H, int c_begin, uint8_t *__restrict__ recs,
+            int total_T, int Hqk, int H, const ChunkMap map, uint8_t *__restrict__ recs,
             uint32_t *err) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t sbase = smem_u32(smem_raw);
-    const int chain = blockIdx.y;
-    const int h = chain % H, n = chain / H;
+    int n, h, c, gc;
+    if (map.by_window) {
+        gc = map.w0 + static_cast<int>(blockIdx.x);
+        h = blockIdx.y;
+        if (gc >= map.w1 || gc >= map.base[num_seqs]) return;
+        int lo = 0, hi = num_seqs;   // base[lo] <= gc < base[hi]
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (map.base[mid] <= gc) lo = mid;
+            else hi = mid;
+        }
+        n = lo;
+        c = gc - map.base[n];
+    } else {
+        h = blockIdx.y % H;
+        n = blockIdx.y / H;
+        c = map.c0 + static_cast<int>(blockIdx.x);
+        if (c >= map.base[n + 1] - map.base[n]) return;   // past this sequence's last chunk
+        gc = map.base[n] + c;
+    }
     const int hq = h / (H / Hqk);
     int t0, len;
     sequence_range(cu, n, num_seqs, total_T, t0, len);
-    const int c = c_begin + static_cast<int>(blockIdx.x);
-    if (c * C >= len) return;          // past this sequence's last chunk
+    if (c * C >= len) return;
     if ((sbase & 1023u) != 0) {
         if (threadIdx.x == 0) atomicOr(err, ERR_SMEM_ALIGN);
         return;
     }
     uint8_t *sm = smem_raw;
     PrepMisc *m = reinterpret_cast<PrepMisc *>(sm + PO_MISC);
-    uint8_t *rec = recs + ((size_t)blockIdx.x * gridDim.y + chain) * REC_BYTES;
+    uint8_t *rec = recs + ((size_t)(gc - map.w0) * H + h) * REC_BYTES;
     const int tok0 = t0 + c * C;
     const int cl = min(C, len - c * C);
 
@@ -924,20 +1000,31 @@ __device__ __forceinline__ void named_sync(int id, int nthreads) {
 template <bool CHANNEL>
 __global__ void __launch_bounds__(kChainThreads, 1)
 chain_kernel(const uint8_t *__restrict__ recs, const float *h0, float *fin, float *ws_state,
-             const int32_t *__restrict__ cu, int num_seqs, int total_T, int H, int c_begin,
-             int c_end, __nv_bfloat16 *__restrict__ o, uint32_t *err) {
+             const int32_t *__restrict__ cu, int num_seqs, int total_T, int H, const ChunkMap map,
+             __nv_bfloat16 *__restrict__ o, uint32_t *err) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t sbase = smem_u32(smem_raw);
-    const int chain = blockIdx.x, chains = gridDim.x;
+    const int chain = blockIdx.x;
     const int h = chain % H, n = chain / H;
     int t0, len;
     sequence_range(cu, n, num_seqs, total_T, t0, len);
-    const int nchunks = (len + C - 1) / C;
-    if (c_begin > 0 && c_begin >= nchunks) return;   // finished in an earlier window
-    const int c_stop = min(c_end, nchunks);
+    const int b0 = map.base[n];
+    const int nchunks = map.base[n + 1] - b0;
+    // this launch's local chunks of the sequence
+    const int c_begin = max(map.c0, map.w0 - b0);
+    const int c_stop = min(min(map.c1, map.w1 - b0), nchunks);
+    const bool first_launch = map.c0 == 0 && map.w0 == 0;
+    if (c_stop <= c_begin && !(nchunks == 0 && first_launch)) return;   // nothing here
     const int nl = max(c_stop - c_begin, 0);
+    // the state enters from the initial state or from the launch before; it
+    // leaves to the final state or to the launch after (pieces: one slot per
+    // chain; windows: one slot per window boundary, which one sequence crosses)
+    const size_t slot_in = map.by_window ? ((size_t)(map.win - 1) * H + h) : (size_t)chain;
+    const size_t slot_out = map.by_window ? ((size_t)map.win * H + h) : (size_t)chain;
     const float *s_in = c_begin == 0 ? h0 : ws_state;
     float *s_out = c_stop == nchunks ? fin : ws_state;
+    const size_t in_off = (c_begin == 0 ? (size_t)chain : slot_in) * D * D;
+    const size_t out_off = (c_stop == nchunks ? (size_t)chain : slot_out) * D * D;
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
@@ -945,15 +1032,15 @@ chain_kernel(const uint8_t *__restrict__ recs, const float *h0, float *fin, floa
     const int r = sub * 32 + lane;                     // value channel = TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>(sub * 32) << 16;
     const int qc = (warp >> 2) & 3;                    // state warps: key-channel quarter
-    const size_t sg = (((size_t)n * H + h) * D + r) * D + qc * 32;
+    const size_t tsg = (size_t)r * D + qc * 32;   // this thread's part of a state
 
     if (nl == 0) {   // empty sequence: the state passes through
         if (s_out != nullptr && warp < kStateWarps) {
 #pragma unroll
             for (int j = 0; j < 32; j += 4) {
                 float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (s_in != nullptr) x = *reinterpret_cast<const float4 *>(s_in + sg + j);
-                *reinterpret_cast<float4 *>(s_out + sg + j) = x;
+                if (s_in != nullptr) x = *reinterpret_cast<const float4 *>(s_in + in_off + tsg + j);
+                *reinterpret_cast<float4 *>(s_out + out_off + tsg + j) = x;
             }
         }
         return;
@@ -993,7 +1080,7 @@ chain_kernel(const uint8_t *__restrict__ recs, const float *h0, float *fin, floa
         atomicOr(err, code);
     };
     auto rec_of = [&](int lc) {
-        return recs + ((size_t)lc * chains + chain) * REC_BYTES;
+        return recs + ((size_t)(b0 + c_begin + lc - map.w0) * H + h) * REC_BYTES;
     };
 
     if (warp < kStateWarps) {
@@ -1002,7 +1089,7 @@ chain_kernel(const uint8_t *__restrict__ recs, const float *h0, float *fin, floa
 #pragma unroll
         for (int j = 0; j < 32; j += 4) {
             float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (s_in != nullptr) x = *reinterpret_cast<const float4 *>(s_in + sg + j);
+            if (s_in != nullptr) x = *reinterpret_cast<const float4 *>(s_in + in_off + tsg + j);
             S[j] = x.x; S[j + 1] = x.y; S[j + 2] = x.z; S[j + 3] = x.w;
         }
         bool stop = false;
@@ -1077,7 +1164,7 @@ chain_kernel(const uint8_t *__restrict__ recs, const float *h0, float *fin, floa
         if (s_out != nullptr) {
 #pragma unroll
             for (int j = 0; j < 32; j += 4)
-                *reinterpret_cast<float4 *>(s_out + sg + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+                *reinterpret_cast<float4 *>(s_out + out_off + tsg + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
         }
     } else if (warp < kIssuerWarp) {
         // ================== output warps: value channel r, all 64 tokens ==========
@@ -1219,16 +1306,19 @@ chain_kernel(const uint8_t *__restrict__ recs, const float *h0, float *fin, floa
 // ------------------------------------------------------------------ host ----
 
 constexpr size_t kHeaderBytes = 256;                        // error word
-constexpr size_t kMaxRecordBytes = size_t(4) << 30;         // records per window
-// Up to 64 chains the two kernels beat the single-kernel plan: its chunk
-// period is set by the chunk-local work, which the prep kernel spreads over
-// all SMs.
-constexpr int kSplitMaxChains = 64;
+constexpr size_t kMaxRecordBytes = size_t(8) << 30;         // records per window
+// Pipelined pieces need the chain CTAs to leave most SMs to the prep kernel;
+// beyond this many (sequence, head) chains the plan runs the prep kernel over
+// a whole window first, then the chain kernel.
+constexpr int kPipeChains = 64;
 
 struct SplitPlan {
-    int chains = 0, max_chunks = 0, window = 0, windows = 0;
-    int pieces = 1;   // pipeline pieces of a single window (prep of piece k + 1 beside chain k)
-    size_t state_off = 0, rec_off = 0, bytes = 0;
+    int chains = 0, max_chunks = 0;
+    long long max_total = 0;        // bound on the number of global chunks
+    int window = 0, windows = 0;    // global chunks per window, windows
+    int pieces = 1;                 // pipeline pieces of a single window
+    bool by_window = false;
+    size_t base_off = 0, state_off = 0, rec_off = 0, bytes = 0;
 };
 
 // Pipeline pieces of one window: the prep kernel of piece k + 1 runs beside
@@ -1248,25 +1338,30 @@ int piece_schedule(int max_chunks, int *bounds) {
 }
 
 // With equal lengths (no cu_seqlens) every sequence has total_T / num_seqs
-// tokens; otherwise the lengths live on the device and total_T bounds them.
-// The equal-length plan never needs more workspace than the general one (its
-// window is no larger, and it needs the state area only when that one does).
+// tokens; otherwise the lengths live on the device, and the number of
+// chunks of all sequences together is at most total_T / 64 + num_seqs.
 bool make_split_plan(int num_seqs, int total_T, int H, SplitPlan &p, bool equal_lengths = false) {
     const long long chains = (long long)num_seqs * H;
-    if (chains < 1 || chains > kSplitMaxChains || total_T <= 0) return false;
+    if (chains < 1 || chains > (1ll << 24) || total_T <= 0) return false;
     p.chains = (int)chains;
     const int longest = equal_lengths ? total_T / num_seqs : total_T;
     p.max_chunks = (longest + C - 1) / C;   // no sequence has more chunks
-    const size_t per = (size_t)p.chains * REC_BYTES;
-    const size_t fit = kMaxRecordBytes / per;
-    p.window = (int)(fit < 1 ? 1 : (fit < (size_t)p.max_chunks ? fit : (size_t)p.max_chunks));
-    p.windows = (p.max_chunks + p.window - 1) / p.window;
+    p.max_total = equal_lengths ? (long long)num_seqs * p.max_chunks
+                                : (long long)(total_T + C - 1) / C + num_seqs;
+    const size_t per = (size_t)H * REC_BYTES;
+    const long long fit = (long long)(kMaxRecordBytes / per);
+    if (fit < 1) return false;
+    p.window = (int)std::min(p.max_total, fit);
+    p.windows = (int)((p.max_total + p.window - 1) / p.window);
     int bounds[kMaxPieces + 1];
-    p.pieces = p.windows == 1 ? piece_schedule(p.max_chunks, bounds) : 1;
-    const size_t state =
-        (p.windows > 1 || p.pieces > 1) ? (size_t)p.chains * D * D * sizeof(float) : 0;
-    p.state_off = kHeaderBytes;
-    p.rec_off = (kHeaderBytes + state + 1023) & ~size_t(1023);
+    p.by_window = !(p.windows == 1 && chains <= kPipeChains);
+    p.pieces = p.by_window ? 1 : piece_schedule(p.max_chunks, bounds);
+    size_t state = 0;   // slots for states between launches
+    if (p.by_window) state = (size_t)(p.windows - 1) * H * D * D * sizeof(float);
+    else if (p.pieces > 1) state = (size_t)p.chains * D * D * sizeof(float);
+    p.base_off = kHeaderBytes;
+    p.state_off = (p.base_off + (size_t)(num_seqs + 1) * sizeof(int32_t) + 255) & ~size_t(255);
+    p.rec_off = (p.state_off + state + 1023) & ~size_t(1023);
     p.bytes = p.rec_off + (size_t)p.window * per;
     return true;
 }
@@ -1307,8 +1402,11 @@ cudaError_t get_helpers(Helpers **out) {
 }  // namespace
 
 size_t tcgen05_split_workspace_bytes(int num_seqs, int total_T, int H) {
-    SplitPlan p;
-    return make_split_plan(num_seqs, total_T, H, p) ? p.bytes : 0;
+    // the caller may pass cu_seqlens or not: room for either plan
+    SplitPlan p, pe;
+    if (!make_split_plan(num_seqs, total_T, H, p)) return 0;
+    const bool equal_ok = total_T % num_seqs == 0 && make_split_plan(num_seqs, total_T, H, pe, true);
+    return equal_ok ? std::max(p.bytes, pe.bytes) : p.bytes;
 }
 
 cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, const float *g,
@@ -1319,6 +1417,7 @@ cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, co
     if (!make_split_plan(num_seqs, total_T, H, p, cu == nullptr)) return cudaErrorInvalidValue;
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     uint32_t *err = reinterpret_cast<uint32_t *>(ws);
+    int32_t *base = reinterpret_cast<int32_t *>(ws + p.base_off);
     cudaError_t e = cudaMemsetAsync(err, 0, sizeof(uint32_t), stream);
     if (e != cudaSuccess) return e;
     CUtensorMap mq, mk, mv;
@@ -1331,49 +1430,63 @@ cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, co
     auto chain_k = channel ? chain_kernel<true> : chain_kernel<false>;
     e = ensure_dynamic_smem(reinterpret_cast<const void *>(chain_k), (int)CHAIN_SMEM);
     if (e != cudaSuccess) return e;
-    float *state = (p.windows > 1 || p.pieces > 1) ? reinterpret_cast<float *>(ws + p.state_off) : nullptr;
+    float *state = reinterpret_cast<float *>(ws + p.state_off);
     uint8_t *recs = ws + p.rec_off;
     __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(o);
-    auto run_chain = [&](int c0, int c1, const uint8_t *r, cudaStream_t st) {
-        chain_k<<<(unsigned)p.chains, kChainThreads, CHAIN_SMEM, st>>>(r, h0, fin, state, cu, num_seqs,
-                                                                        total_T, H, c0, c1, out, err);
+    chunk_base_kernel<<<1, 1024, 0, stream>>>(cu, num_seqs, total_T, base);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    auto run_chain = [&](const ChunkMap &map, cudaStream_t st) {
+        chain_k<<<(unsigned)p.chains, kChainThreads, CHAIN_SMEM, st>>>(recs, h0, fin, state, cu, num_seqs,
+                                                                        total_T, H, map, out, err);
         return cudaGetLastError();
     };
-    auto run_prep = [&](int c0, int c1, uint8_t *r, cudaStream_t st) {
-        prep<<<dim3((unsigned)(c1 - c0), (unsigned)p.chains), kPrepThreads, PREP_SMEM, st>>>(
-            mq, mk, mv, g, beta, cu, num_seqs, total_T, Hqk, H, c0, r, err);
+    auto run_prep = [&](const ChunkMap &map, unsigned gx, unsigned gy, cudaStream_t st) {
+        prep<<<dim3(gx, gy), kPrepThreads, PREP_SMEM, st>>>(mq, mk, mv, g, beta, cu, num_seqs, total_T,
+                                                            Hqk, H, map, recs, err);
         return cudaGetLastError();
     };
-    if (p.pieces > 1) {
-        // every record has its own slot: the prep kernel of piece k + 1 runs on
-        // the SMs the chain kernel of piece k leaves free
+    constexpr int kAll = 1 << 30;
+    if (!p.by_window) {
+        // one window holds every record; pieces of every sequence's chunks
+        int bounds[kMaxPieces + 1];
+        piece_schedule(p.max_chunks, bounds);
+        auto piece = [&](int k) {
+            // w1 = the records' capacity: a malformed cu_seqlens with more chunks
+            // than total_T allows never writes past it
+            return ChunkMap{base, 0, (int)p.max_total, bounds[k], bounds[k + 1], 0, 0};
+        };
+        if (p.pieces == 1) {
+            e = run_prep(piece(0), (unsigned)(bounds[1] - bounds[0]), (unsigned)p.chains, stream);
+            return e == cudaSuccess ? run_chain(piece(0), stream) : e;
+        }
+        // the prep kernel of piece k + 1 runs on the SMs the chain kernel of
+        // piece k leaves free
         std::lock_guard<std::mutex> lock(g_helpers_mutex);
         Helpers *hs = nullptr;
         e = get_helpers(&hs);
         if (e != cudaSuccess) return e;
-        int bounds[kMaxPieces + 1];
-        piece_schedule(p.max_chunks, bounds);
         e = cudaEventRecord(hs->fork, stream);
         if (e == cudaSuccess) e = cudaStreamWaitEvent(hs->prep_s, hs->fork, 0);
         if (e == cudaSuccess) e = cudaStreamWaitEvent(hs->chain_s, hs->fork, 0);
-        for (int k = 0; k < p.pieces && e == cudaSuccess; ++k) {
-            const int c0 = bounds[k], c1 = bounds[k + 1];
-            uint8_t *r = recs + (size_t)c0 * p.chains * REC_BYTES;
-            e = run_prep(c0, c1, r, hs->prep_s);
+        for (int kk = 0; kk < p.pieces && e == cudaSuccess; ++kk) {
+            e = run_prep(piece(kk), (unsigned)(bounds[kk + 1] - bounds[kk]), (unsigned)p.chains, hs->prep_s);
             if (e == cudaSuccess) e = cudaEventRecord(hs->prep_done, hs->prep_s);
             if (e == cudaSuccess) e = cudaStreamWaitEvent(hs->chain_s, hs->prep_done, 0);
-            if (e == cudaSuccess) e = run_chain(c0, c1, r, hs->chain_s);
+            if (e == cudaSuccess) e = run_chain(piece(kk), hs->chain_s);
         }
         if (e == cudaSuccess) e = cudaEventRecord(hs->join, hs->chain_s);
         if (e == cudaSuccess) e = cudaStreamWaitEvent(stream, hs->join, 0);
         return e;
     }
+    // windows of global chunks: the prep kernel over a window, then the chain
     for (int w = 0; w < p.windows; ++w) {
-        const int c0 = w * p.window;
-        const int c1 = c0 + p.window < p.max_chunks ? c0 + p.window : p.max_chunks;
-        e = run_prep(c0, c1, recs, stream);
+        const long long w0 = (long long)w * p.window;
+        const long long w1 = std::min(w0 + p.window, p.max_total);
+        const ChunkMap map{base, (int)w0, (int)w1, 0, kAll, w, 1};
+        e = run_prep(map, (unsigned)(w1 - w0), (unsigned)H, stream);
         if (e != cudaSuccess) return e;
-        e = run_chain(c0, c1, recs, stream);
+        e = run_chain(map, stream);
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;

@@ -111,34 +111,56 @@ def test_workspace_and_path_queries(lib):
         gdr.gdr_prefill_workspace_size(-1, 64, 2, 16, 16, 0, 0)
 
 
+def _split_bytes(N, T, H, equal):
+    """The chunk-parallel plan's workspace layout: a 256-byte header (error
+    word), the chunk numbering (N + 1 int32), the state slots, then one
+    window of 98,848-byte records per (global chunk, head)."""
+    rec = 98848
+    longest = T // N if equal else T
+    max_chunks = -(-longest // 64)
+    max_total = N * max_chunks if equal else -(-T // 64) + N
+    window = min(max_total, (8 << 30) // (H * rec))
+    windows = -(-max_total // window)
+    by_window = windows > 1 or N * H > 64
+    pieces = 1
+    if not by_window:
+        pieces, c, size = 0, 0, 12
+        while c < max_chunks and pieces < 32:
+            c = max_chunks if pieces + 1 == 32 else min(c + size, max_chunks)
+            pieces += 1
+            size = (size * 13 + 9) // 10
+    state = (windows - 1) * H * 65536 if by_window else (N * H * 65536 if pieces > 1 else 0)
+    state_off = (256 + (N + 1) * 4 + 255) // 256 * 256
+    rec_off = (state_off + state + 1023) // 1024 * 1024
+    return rec_off + window * H * rec, windows
+
+
 def test_plan_selection_and_workspace_sizes(lib):
     """The tcgen05 family runs as two plans: the chunk-parallel one with the
     reported workspace (98,848 bytes of chunk records per chunk and head, in
-    windows of at most 4 GiB), the single-kernel one with 16 bytes."""
+    windows of at most 8 GiB), the single-kernel one with 16 bytes."""
     S, CH, BF = gdr.GDR_GATE_SCALAR, gdr.GDR_GATE_CHANNEL, gdr.GDR_BF16
-    rec = 98848
-    # one window of 128 chunks, run as 4 pipelined pieces: 64 KiB of state per
-    # head between pieces
+    # room for the packed-length plan and the equal-length one
     nb = gdr.gdr_prefill_workspace_size(1, 8192, 16, 128, 128, S, BF)
-    assert nb == ((256 + 16 * 65536 + 1023) // 1024) * 1024 + 128 * 16 * rec
+    assert nb == max(_split_bytes(1, 8192, 16, False)[0], _split_bytes(1, 8192, 16, True)[0])
     assert gdr.gdr_prefill_plan(1, 8192, 16, 128, 128, S, BF, nb) == gdr.GDR_PATH_TCGEN05_SPLIT
     assert gdr.gdr_prefill_plan(1, 8192, 16, 128, 128, CH, BF, nb) == gdr.GDR_PATH_TCGEN05_SPLIT
     assert gdr.gdr_prefill_plan(1, 8192, 16, 128, 128, S, BF, nb - 1) == gdr.GDR_PATH_TCGEN05
     assert gdr.gdr_prefill_plan(1, 8192, 16, 128, 128, S, BF, 16) == gdr.GDR_PATH_TCGEN05
     with pytest.raises(gdr.GdrError):
         gdr.gdr_prefill_plan(1, 8192, 16, 128, 128, S, BF, 8)
-    # more than 64 (sequence, head) pairs: the single-kernel plan only
-    assert gdr.gdr_prefill_workspace_size(2, 8192, 33, 128, 128, S, BF) == 16
-    assert gdr.gdr_prefill_plan(2, 8192, 33, 128, 128, S, BF, 1 << 40) == gdr.GDR_PATH_TCGEN05
-    assert gdr.gdr_prefill_workspace_size(1, 8192, 64, 128, 128, S, BF) > 16
+    # more than 64 (sequence, head) chains: a window of global chunks
+    nb = gdr.gdr_prefill_workspace_size(8, 262144, 16, 128, 128, S, BF)
+    assert nb == _split_bytes(8, 262144, 16, False)[0]
+    assert _split_bytes(8, 262144, 16, False)[1] == 1
+    assert gdr.gdr_prefill_plan(8, 262144, 16, 128, 128, S, BF, nb) == gdr.GDR_PATH_TCGEN05_SPLIT
     # fp32 I/O and other head sizes: the CUDA-core kernel, no workspace
     assert gdr.gdr_prefill_plan(1, 8192, 16, 128, 128, S, gdr.GDR_F32, 0) == gdr.GDR_PATH_SIMT
     assert gdr.gdr_prefill_plan(1, 8192, 16, 64, 64, S, BF, 0) == gdr.GDR_PATH_SIMT
-    # 64 heads x 700 chunks: records beyond 4 GiB -> windows of 678 chunks with
-    # 64 KiB of state per head between them
-    nb = gdr.gdr_prefill_workspace_size(1, 44800, 64, 128, 128, S, BF)
-    state = 64 * 128 * 128 * 4
-    assert nb == ((256 + state + 1023) // 1024) * 1024 + 678 * 64 * rec
+    # 64 heads x 1400 chunks: records beyond 8 GiB -> windows of global chunks
+    nb = gdr.gdr_prefill_workspace_size(1, 89600, 64, 128, 128, S, BF)
+    assert nb == max(_split_bytes(1, 89600, 64, False)[0], _split_bytes(1, 89600, 64, True)[0])
+    assert _split_bytes(1, 89600, 64, True)[1] == 2
     # a tcgen05 problem without any workspace is refused before any launch
     assert _prefill(lib, dk=128, dv=128, io=1) == gdr.GDR_ERR_WORKSPACE
 

@@ -33,20 +33,23 @@ def test_reference_arm_prints_one_contract_line():
 
 
 def test_pipelined_plan_launch_accounting():
-    # 128 chunks in one window: pieces of 12, 16, 21, 27, 35 and the last 17;
-    # each piece is one prep and one chain launch
-    assert bench.split_launches(I.workload("gdn_prefill")) == 12
-    # 64 chains of 98,848-byte records in 4 GiB windows: 678 chunks per
-    # window.  The two equal sequences go without cu_seqlens, so the plan
-    # knows each has 512 chunks: one window, in 10 pipelined pieces (12, 16,
-    # 21, 27, 35, 46, 60, 78, 101 and the last 116)
+    # one launch numbers the chunks; then 128 chunks in one window: pieces of
+    # 12, 16, 21, 27, 35 and the last 17, each one prep and one chain launch
+    assert bench.split_launches(I.workload("gdn_prefill")) == 1 + 12
+    # 64 chains of 98,848-byte records, at most 8 GiB per window: 2715 global
+    # chunks of 32 heads.  The two equal sequences go without cu_seqlens, so
+    # the plan knows each has 512 chunks (1024 in all): one window, in 10
+    # pipelined pieces (12, 16, 21, 27, 35, 46, 60, 78, 101 and the last 116)
     kda = I.workload("kda_prefill")
-    window = (4 << 30) // (64 * 98848)
-    assert window == 678
-    assert bench.split_launches(kda) == 2 * 10
-    # with packed lengths only total_T bounds a sequence: varlen has 128
-    # chains, beyond the plan, so only the counting is checked here
-    assert bench.split_launches(I.workload("gqa_prefill")) == 12
+    assert (8 << 30) // (32 * 98848) == 2715
+    assert bench.split_launches(kda) == 1 + 2 * 10
+    # 48 chains at the gdn_prefill length: the same pieces
+    assert bench.split_launches(I.workload("gqa_prefill")) == 1 + 12
+    # varlen: 128 chains run by windows; packed lengths bound the chunks by
+    # 262144 / 64 + 8 = 4104, within one window of 5431 global chunks of 16
+    # heads
+    assert (8 << 30) // (16 * 98848) == 5431
+    assert bench.split_launches(I.workload("varlen_gdn")) == 1 + 2
 
 
 def test_prologue_bytes_per_launch():

@@ -238,14 +238,15 @@ def test_channel_gate_decay_strengths(c_gate, plan):
 
 @pytest.mark.parametrize("mode", [I.SCALAR, I.CHANNEL])
 def test_chunk_parallel_plan_in_windows(mode):
-    """64 heads x 44,800 tokens: the chunk records exceed the 4 GiB window,
-    so the chunk-parallel plan runs in two windows of chunks with the state
-    handed between them through the workspace (sequence of 700 chunks, a
-    window of 678).  Sampled heads against the oracle, in-place state."""
-    T, H = 44800, 64
+    """64 heads x 89,600 tokens: the chunk records exceed the 8 GiB window,
+    so the chunk-parallel plan runs in two windows of global chunks with the
+    state handed between them through the workspace (a sequence of 1400
+    chunks, windows of 1357).  Sampled heads against the oracle, in-place
+    state."""
+    T, H = 89600, 64
     nb = gdr.gdr_prefill_workspace_size(1, T, H, 128, 128, 0 if mode == I.SCALAR else 1,
                                         gdr.GDR_BF16)
-    assert (1 << 30) < nb < 700 * H * 98848   # the workspace holds one window, not all records
+    assert (1 << 30) < nb < 1400 * H * 98848   # the workspace holds one window, not all records
     inp = I.make_inputs(total_T=T, H=H, d_k=128, gate_mode=mode, io_dtype=torch.bfloat16,
                         c=0.1, h0_std=0.02, seed=51)
     d = to_device(inp)
@@ -303,3 +304,25 @@ def test_equal_lengths_plan_knows_each_sequence_length(mode):
     check(inp, o1, f1, o_ref, fin_ref, "with cu_seqlens")
     check(inp, o2, f2, o_ref, fin_ref, "equal lengths")
     assert float((o1.float() - o2.float()).abs().max()) <= 2e-2
+
+
+@pytest.mark.parametrize("mode", [I.SCALAR, I.CHANNEL])
+def test_many_chains_run_by_windows_with_empty_sequences(mode):
+    """40 sequences x 2 heads (more than 64 chains): the chunk-parallel plan
+    numbers every sequence's chunks on the device and runs the prep kernel
+    over the window of global chunks, then one chain CTA per (sequence, head).
+    Empty, one-token and multi-chunk sequences, against the oracle."""
+    rng = np.random.default_rng(np.random.SeedSequence(71, spawn_key=(99,)))
+    lens = rng.choice([0, 1, 5, 63, 64, 65, 130, 200], size=40)
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    inp = I.make_inputs(total_T=int(cu[-1]), H=2, d_k=128, cu_seqlens=cu, gate_mode=mode,
+                        io_dtype=torch.bfloat16, c=0.1, h0_std=0.02, seed=71)
+    nb = gdr.gdr_prefill_workspace_size(40, int(cu[-1]), 2, 128, 128,
+                                        0 if mode == I.SCALAR else 1, gdr.GDR_BF16)
+    assert gdr.gdr_prefill_plan(40, int(cu[-1]), 2, 128, 128, 0 if mode == I.SCALAR else 1,
+                                gdr.GDR_BF16, nb) == gdr.GDR_PATH_TCGEN05_SPLIT
+    o, fin = gpu_prefill(inp)
+    o_ref, fin_ref = oracle_prefill(inp)
+    check(inp, o, fin, o_ref, fin_ref, "windows, many chains")
+    for n in np.nonzero(lens == 0)[0]:
+        assert torch.equal(fin[n].cpu(), inp.h0[n])
