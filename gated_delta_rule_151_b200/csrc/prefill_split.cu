@@ -135,6 +135,27 @@ __device__ __forceinline__ void st_global_v4(uint8_t *p, uint32_t a, uint32_t b,
     *reinterpret_cast<uint4 *>(p) = make_uint4(a, b, c, d);
 }
 
+// Shared-memory accesses through ordinary pointers (byte offsets into the
+// CTA's dynamic shared memory), so that the compiler may batch and reorder
+// them; every hand-off to the tensor cores or to other threads still goes
+// through a fence or barrier that orders memory.
+__device__ __forceinline__ float smb16(const uint8_t *sm, uint32_t off) {
+    return __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sm + off));
+}
+__device__ __forceinline__ void smh16(uint8_t *sm, uint32_t off, float v) {
+    *reinterpret_cast<__half *>(sm + off) = __float2half_rn(v);
+}
+__device__ __forceinline__ void smu16(uint8_t *sm, uint32_t off, uint16_t v) {
+    *reinterpret_cast<uint16_t *>(sm + off) = v;
+}
+__device__ __forceinline__ uint4 smv4(const uint8_t *sm, uint32_t off) {
+    return *reinterpret_cast<const uint4 *>(sm + off);
+}
+__device__ __forceinline__ void smv4(uint8_t *sm, uint32_t off, uint32_t a, uint32_t b, uint32_t c,
+                                     uint32_t d) {
+    *reinterpret_cast<uint4 *>(sm + off) = make_uint4(a, b, c, d);
+}
+
 // ------------------------------------------------------------- chunk map ----
 // Chunks are numbered globally, sequence after sequence: sequence n owns
 // global chunks base[n] .. base[n+1] - 1, base computed on the device from
@@ -432,23 +453,20 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             bool bad = false;
             const uint32_t kcol = (ch >> 6) * 16384, bcol = (ch >> 6) * 8192;
             const uint32_t cch = (ch & 63) >> 3, cel = (ch & 7) * 2;
-#pragma unroll 4
+#pragma unroll
             for (int k = 0; k < 32; ++k) {
                 const int i = hh * 32 + k;
-                const uint32_t src = sbase + PO_KQ + kcol + sw128_offset(i, cch) + cel;
-                const float kv = ld_shared_bf16(src), qv = ld_shared_bf16(src + 8192);
+                const uint32_t src = PO_KQ + kcol + sw128_offset(i, cch) + cel;
+                const float kv = smb16(sm, src), qv = smb16(sm, src + 8192);
                 kmax = fmaxf(kmax, fabsf(kv));
                 qmax = fmaxf(qmax, fabsf(qv));
                 const float up = __expf(gr[k] - R), dn = __expf(R - gr[k]);
                 const float a = kv * up, b = qv * up, e = kv * dn;
                 bad |= !(fabsf(a) < kF16Limit) || !(fabsf(b) < kF16Limit) ||
                        !(fabsf(e) < kF16Limit);
-                st_shared_b16(sbase + PO_RA + kcol + sw128_offset(i, cch) + cel,
-                              __half_as_ushort(__float2half_rn(a)));
-                st_shared_b16(sbase + PO_RA + kcol + sw128_offset(64 + i, cch) + cel,
-                              __half_as_ushort(__float2half_rn(b)));
-                st_shared_b16(sbase + PO_RX + bcol + sw128_offset(i, cch) + cel,
-                              __half_as_ushort(__float2half_rn(e)));
+                smh16(sm, PO_RA + kcol + sw128_offset(i, cch) + cel, a);
+                smh16(sm, PO_RA + kcol + sw128_offset(64 + i, cch) + cel, b);
+                smh16(sm, PO_RX + bcol + sw128_offset(i, cch) + cel, e);
             }
             if (bad) m->slow = 1;
             fence_proxy_async();
@@ -556,7 +574,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 #pragma unroll
                     for (int c8 = 0; c8 < 8; ++c8) {
                         float qf[8];
-                        bf16x8_to_f32(ld_shared_v4(sbase + PO_KQ + 8192 + half * 16384 + sw128_offset(i, c8)), qf);
+                        bf16x8_to_f32(smv4(sm, PO_KQ + 8192 + half * 16384 + sw128_offset(i, c8)), qf);
 #pragma unroll
                         for (int e = 0; e < 8; ++e) mx3[2] = fmaxf(mx3[2], fabsf(qf[e]) * gq);
                     }
@@ -674,11 +692,11 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     }
                 }
                 const uint32_t off = t * 128 + (((cq ^ (t & 7)) & 7) << 4);
-                st_shared_v4(sbase + PO_RA + off, h1[0], h1[1], h1[2], h1[3]);
-                st_shared_v4(sbase + PO_RA + 8192 + off, l1[0], l1[1], l1[2], l1[3]);
+                smv4(sm, PO_RA + off, h1[0], h1[1], h1[2], h1[3]);
+                smv4(sm, PO_RA + 8192 + off, l1[0], l1[1], l1[2], l1[3]);
                 if (!CHANNEL) {
-                    st_shared_v4(sbase + PO_RX + off, h2[0], h2[1], h2[2], h2[3]);
-                    st_shared_v4(sbase + PO_RX + 8192 + off, l2[0], l2[1], l2[2], l2[3]);
+                    smv4(sm, PO_RX + off, h2[0], h2[1], h2[2], h2[3]);
+                    smv4(sm, PO_RX + 8192 + off, l2[0], l2[1], l2[2], l2[3]);
                 }
             }
         }
@@ -696,9 +714,9 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 const int item = tid + it * kPrepThreads;
                 const int blk = item >> 9, t = (item >> 3) & 63, cq = item & 7;
                 float kf[8];
-                bf16x8_to_f32(ld_shared_v4(sbase + PO_KQ + blk * 16384 + sw128_offset(t, cq)), kf);
+                bf16x8_to_f32(smv4(sm, PO_KQ + blk * 16384 + sw128_offset(t, cq)), kf);
                 const float f = m->u.s.kh[t] * fs;
-                st_shared_v4(sbase + PO_RT + blk * 8192 + sw128_offset(t, cq),
+                smv4(sm, PO_RT + blk * 8192 + sw128_offset(t, cq),
                              f2h2_bits(kf[0] * f, kf[1] * f), f2h2_bits(kf[2] * f, kf[3] * f),
                              f2h2_bits(kf[4] * f, kf[5] * f), f2h2_bits(kf[6] * f, kf[7] * f));
             }
@@ -706,19 +724,19 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             const float fk = exp2i(sK), fq = exp2i(sQ);
             const uint32_t kcol = (ch >> 6) * 16384, tcol = (ch >> 6) * 8192;
             const uint32_t cch = (ch & 63) >> 3, cel = (ch & 7) * 2;
-#pragma unroll 4
+#pragma unroll
             for (int k = 0; k < 32; ++k) {
                 const int i = hh * 32 + k;
-                const uint32_t src = sbase + PO_KQ + kcol + sw128_offset(i, cch) + cel;
+                const uint32_t src = PO_KQ + kcol + sw128_offset(i, cch) + cel;
                 const uint32_t dst = tcol + sw128_offset(i, cch) + cel;
-                const float kv = ld_shared_bf16(src), qv = ld_shared_bf16(src + 8192);
+                const float kv = smb16(sm, src), qv = smb16(sm, src + 8192);
                 const float eg = __expf(gr[k]);
-                st_shared_b16(sbase + PO_RT + dst, f2h_bits(kv * __expf(GC - gr[k]) * fk));
+                smh16(sm, PO_RT + dst, kv * __expf(GC - gr[k]) * fk);
                 const float kp = kv * eg;
                 const uint16_t khi = bf16_bits(kp);
-                st_shared_b16(src, khi);
-                st_shared_b16(sbase + PO_RX + dst, bf16_bits(kp - __uint_as_float((uint32_t)khi << 16)));
-                st_shared_b16(src + 8192, f2h_bits(qv * eg * fq));
+                smu16(sm, src, khi);
+                smu16(sm, PO_RX + dst, bf16_bits(kp - __uint_as_float((uint32_t)khi << 16)));
+                smh16(sm, src + 8192, qv * eg * fq);
             }
         }
         fence_proxy_async();
@@ -744,11 +762,11 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             }
             mma_commit(&m->bar_mma);
         }
-        // the K̂ tile goes to the record while the MMAs run
-#pragma unroll
-        for (int it = 0; it < 4; ++it) {
-            const int e = tid + it * kPrepThreads;
-            *reinterpret_cast<uint4 *>(rec + REC_KH + e * 16) = ld_shared_v4(sbase + PO_RT + e * 16);
+        // the K̂ tile goes to the record while the MMAs run (the pass that
+        // wrote it ended with a proxy fence and a barrier)
+        if (tid == 0) {
+            bulk_store(rec + REC_KH, sbase + PO_RT, 16384);
+            bulk_commit();
         }
         if (!block_wait(&m->bar_mma, mph, &m->abort_flag, err, ERR_TIMEOUT_MMA)) break;
         mph ^= 1u;
@@ -780,15 +798,18 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     f2h2_hilo(__uint_as_float(x[i]) * fw, __uint_as_float(x[i + 1]) * fw, hw[e], lw[e]);
                     hu[e] = f2h2_bits(__uint_as_float(y[i]) * fu, __uint_as_float(y[i + 1]) * fu);
                 }
-                st_shared_v4(sbase + PO_RA + off, hw[0], hw[1], hw[2], hw[3]);
-                st_shared_v4(sbase + PO_RX + off, lw[0], lw[1], lw[2], lw[3]);
-                st_shared_v4(sbase + PO_V + off, hu[0], hu[1], hu[2], hu[3]);
-                st_global_v4(rec + REC_UT + off, hu[0], hu[1], hu[2], hu[3]);
+                smv4(sm, PO_RA + off, hw[0], hw[1], hw[2], hw[3]);
+                smv4(sm, PO_RX + off, lw[0], lw[1], lw[2], lw[3]);
+                smv4(sm, PO_V + off, hu[0], hu[1], hu[2], hu[3]);
             }
         }
         fence_proxy_async();
         tc_fence_before();
         __syncthreads();
+        if (tid == 0) {   // Ũ^T is also the record's image
+            bulk_store(rec + REC_UT, sbase + PO_V, 16384);
+            bulk_commit();
+        }
 
         // ---- N^T = K̂^T (-W) (columns 0-127) and P (-W) (rows 64-127 of
         //      columns 128-255), -W as fp16 high + low ------------------------------
@@ -823,9 +844,9 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             const int t = row - C;
             // Q̃ for columns half*64 + p*32 + 8*c8 .. +7 (p < 2, c8 < 4)
             auto qtilde = [&](int p, int c8, float (&qv)[8]) {
-                const uint32_t a = sbase + PO_KQ + 8192 + half * 16384 + sw128_offset(t, p * 4 + c8);
+                const uint32_t a = PO_KQ + 8192 + half * 16384 + sw128_offset(t, p * 4 + c8);
                 if (CHANNEL) {
-                    const uint4 w = ld_shared_v4(a);
+                    const uint4 w = smv4(sm, a);
                     const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
                     const float f = exp2i(-sQ);
 #pragma unroll
@@ -835,7 +856,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                         qv[2 * e + 1] = v.y * f;
                     }
                 } else {
-                    bf16x8_to_f32(ld_shared_v4(a), qv);
+                    bf16x8_to_f32(smv4(sm, a), qv);
                     const float gq2 = m->u.s.gam[t];
 #pragma unroll
                     for (int e = 0; e < 8; ++e) qv[e] *= gq2;
@@ -853,9 +874,9 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     for (int e = 0; e < 4; ++e)
                         w[e] = f2h2_bits(__uint_as_float(x[c8 * 8 + 2 * e]) * gn,
                                          __uint_as_float(x[c8 * 8 + 2 * e + 1]) * gn);
-                    st_global_v4(rec + REC_NT + half * 16384 + row * 128 +
-                                     ((((p * 4 + c8) ^ (row & 7)) & 7) << 4),
-                                 w[0], w[1], w[2], w[3]);
+                    smv4(sm, (half ? PO_RX : PO_RA) + row * 128 +
+                                 ((((p * 4 + c8) ^ (row & 7)) & 7) << 4),
+                         w[0], w[1], w[2], w[3]);
                 }
                 if (qrow) {
                     tmem_ld32(tmem + lane_off + 128 + half * 64 + p * 32, x);
@@ -867,16 +888,23 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 #pragma unroll
                         for (int e = 0; e < 8; ++e)
                             qv[e] = (qv[e] + __uint_as_float(x[c8 * 8 + e]) * fpw) * gq;
-                        st_global_v4(rec + REC_QP + half * 8192 + t * 128 +
-                                         ((((p * 4 + c8) ^ (t & 7)) & 7) << 4),
-                                     f2h2_bits(qv[0], qv[1]), f2h2_bits(qv[2], qv[3]),
-                                     f2h2_bits(qv[4], qv[5]), f2h2_bits(qv[6], qv[7]));
+                        smv4(sm, PO_KQ + half * 16384 + t * 128 + ((((p * 4 + c8) ^ (t & 7)) & 7) << 4),
+                             f2h2_bits(qv[0], qv[1]), f2h2_bits(qv[2], qv[3]),
+                             f2h2_bits(qv[4], qv[5]), f2h2_bits(qv[6], qv[7]));
                     }
                 }
             }
         }
+        fence_proxy_async();
         tc_fence_before();
-        __syncthreads();   // TMEM columns 0-127 are read
+        __syncthreads();   // TMEM columns 0-127 are read; N^T and Q' are staged
+        if (tid == 0) {
+            bulk_store(rec + REC_NT, sbase + PO_RA, 16384);
+            bulk_store(rec + REC_NT + 16384, sbase + PO_RX, 16384);
+            bulk_store(rec + REC_QP, sbase + PO_KQ, 8192);
+            bulk_store(rec + REC_QP + 8192, sbase + PO_KQ + 16384, 8192);
+            bulk_commit();
+        }
 
         // ---- O⁰ = P Ũ (rows 64-127 of columns 0-127) ------------------------------
         if (tid == 0) {
@@ -907,17 +935,27 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                         for (int e = 0; e < 4; ++e)
                             w[e] = f2h2_bits(__uint_as_float(x[c8 * 8 + 2 * e]) * go,
                                              __uint_as_float(x[c8 * 8 + 2 * e + 1]) * go);
-                        st_global_v4(rec + REC_OZ + t * 256 + (half * 64 + p * 32 + c8 * 8) * 2,
-                                     w[0], w[1], w[2], w[3]);
+                        // rows 0-31 over Q d0-63, rows 32-63 over Q d64-127 (Q̃ is consumed)
+                        smv4(sm, PO_KQ + 8192 + (t >> 5) * 16384 + (t & 31) * 256 +
+                                     (half * 64 + p * 32 + c8 * 8) * 2,
+                             w[0], w[1], w[2], w[3]);
                     }
                 }
             }
+            fence_proxy_async();
+            __syncthreads();
             if (tid == 0) {
+                bulk_store(rec + REC_OZ, sbase + PO_KQ + 8192, 8192);
+                bulk_store(rec + REC_OZ + 8192, sbase + PO_KQ + 24576, 8192);
+                bulk_commit();
                 *reinterpret_cast<int4 *>(rec + REC_EX) = make_int4(sN, sK, sU, sQP);
                 *reinterpret_cast<int4 *>(rec + REC_EX + 16) = make_int4(sO, 0, 0, 0);
             }
         }
     } while (0);
+    // the record's bulk stores read this CTA's shared memory: they complete
+    // before the CTA ends
+    if (tid == 0) bulk_wait_all();
 
     tc_fence_before();
     __syncthreads();
