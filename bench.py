@@ -259,7 +259,9 @@ def split_launches(inp):
     launch that numbers every sequence's chunks, then a prep and a chain kernel
     per window of chunks (a window holds at most 8 GiB of records at 98,848
     bytes per chunk and head), or, when one window holds every record and
-    there are at most 64 (sequence, head) chains, per pipeline piece."""
+    there are at most 64 (sequence, head) chains, per pipeline piece, or, with
+    at most 24 chains, one prep launch and the three launches of the
+    segmented scan."""
     chains = inp.num_seqs * inp.H
     # equal lengths go without cu_seqlens, so the library knows each
     # sequence's length; otherwise total_T bounds it
@@ -271,6 +273,12 @@ def split_launches(inp):
     windows = -(-max_total // window)
     if windows > 1 or chains > 64:
         return 1 + 2 * windows
+    nseg = min(8, (148 // chains + 3) // 2)
+    if nseg >= 4 and max_chunks >= 2 * nseg:
+        # few chains: the prep kernel over every chunk, then the segmented scan
+        # (segments from zero and their transitions, composition, segments in
+        # full from their incoming states)
+        return 1 + 1 + 3
     pieces, c, size = 0, 0, 12   # pieces of 12, 16, 21, 27, ... chunks (1.3x growth)
     while c < max_chunks and pieces < 32:
         c = max_chunks if pieces + 1 == 32 else min(c + size, max_chunks)

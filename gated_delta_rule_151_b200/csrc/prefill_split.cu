@@ -130,11 +130,6 @@ __device__ __forceinline__ uint16_t bf16_bits(float x) {
     return __bfloat16_as_ushort(__float2bfloat16_rn(x));
 }
 
-__device__ __forceinline__ void st_global_v4(uint8_t *p, uint32_t a, uint32_t b, uint32_t c,
-                                             uint32_t d) {
-    *reinterpret_cast<uint4 *>(p) = make_uint4(a, b, c, d);
-}
-
 // Shared-memory accesses through ordinary pointers (byte offsets into the
 // CTA's dynamic shared memory), so that the compiler may batch and reorder
 // them; every hand-off to the tensor cores or to other threads still goes
@@ -169,6 +164,14 @@ struct ChunkMap {
     int c0, c1;            // local chunks of every sequence
     int win;               // window index (state slots between windows)
     int by_window;
+    // Segmented scan (few chains): every sequence is cut into nseg segments of
+    // ceil(chunks / nseg) chunks.  Phase 1 runs segment 0 in full from the
+    // initial state and, for segments 1 .. nseg-2, the chain from a zero state
+    // (its B) and the transition from the identity without B (its M); phase 2
+    // runs segments 1 .. nseg-1 in full from their composed incoming states.
+    int nseg;              // 0: no segments
+    int phase;             // 1 or 2
+    float *slots;          // [chains][nseg][3][D * D]: incoming state, B, M
 };
 
 // base[n] = sum over m < n of the chunk count of sequence m (exclusive
@@ -213,6 +216,87 @@ chunk_base_kernel(const int32_t *__restrict__ cu, int num_seqs, int total_T, int
         __syncthreads();
     }
     if (tid == 0) base[num_seqs] = carry;
+}
+
+// Segment composition: S_in(s + 1) = S_in(s) M_s + B_s for s = 1 .. nseg-2,
+// in fp32.  The rows of a state are independent, so CTA (chain, rb) owns rows
+// 16 rb .. 16 rb + 15 for the whole recurrence and keeps them in shared
+// memory, transposed (st[k][16]), from one step to the next; thread tid holds
+// rows 4 (tid / 32) .. +3 by columns 4 (tid % 32) .. +3 in registers.  M_s is
+// staged in shared memory with 16-byte asynchronous copies, the next step's
+// while this step multiplies.
+constexpr int kComposeThreads = 128;
+constexpr uint32_t COMPOSE_SMEM = (2 * D * D + 16 * D) * sizeof(float);   // 136 KiB
+__device__ __forceinline__ void async_copy16(void *dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N> __device__ __forceinline__ void async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+__global__ void __launch_bounds__(kComposeThreads)
+segment_compose_kernel(float *__restrict__ slots, int nseg) {
+    extern __shared__ __align__(16) float csm[];
+    float *st = csm + 2 * D * D;
+    const int chain = blockIdx.x, rb = blockIdx.y, tid = threadIdx.x;
+    const int r0 = (tid >> 5) * 4, c0 = (tid & 31) * 4;
+    auto slot = [&](int sg, int kind) {
+        return slots + (((size_t)chain * nseg + sg) * 3 + kind) * D * D;
+    };
+    auto stage_m = [&](int sg) {
+        const float *M = slot(sg, 2);
+        float *dst = csm + (sg & 1) * D * D;
+#pragma unroll 8
+        for (int e = tid; e < D * D / 4; e += kComposeThreads) async_copy16(dst + 4 * e, M + 4 * e);
+        async_commit();
+    };
+    stage_m(1);
+    {   // incoming rows of segment 1 (segment 0's final state), transposed
+        const float *Sin = slot(1, 0) + (size_t)rb * 16 * D;
+        float4 x[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            x[i] = *reinterpret_cast<const float4 *>(Sin + (size_t)(r0 + i) * D + c0);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            st[(c0 + 0) * 16 + r0 + i] = x[i].x; st[(c0 + 1) * 16 + r0 + i] = x[i].y;
+            st[(c0 + 2) * 16 + r0 + i] = x[i].z; st[(c0 + 3) * 16 + r0 + i] = x[i].w;
+        }
+    }
+    for (int sg = 1; sg + 1 < nseg; ++sg) {
+        const float *B = slot(sg, 1) + (size_t)rb * 16 * D;
+        float acc[4][4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float4 b = *reinterpret_cast<const float4 *>(B + (size_t)(r0 + i) * D + c0);
+            acc[i][0] = b.x; acc[i][1] = b.y; acc[i][2] = b.z; acc[i][3] = b.w;
+        }
+        if (sg + 2 < nseg) { stage_m(sg + 1); async_wait<1>(); }
+        else async_wait<0>();
+        __syncthreads();   // M_sg and the incoming rows are in shared memory
+        const float *Ms = csm + (sg & 1) * D * D;
+#pragma unroll 8
+        for (int k = 0; k < D; ++k) {
+            const float4 a = *reinterpret_cast<const float4 *>(st + k * 16 + r0);
+            const float4 m = *reinterpret_cast<const float4 *>(Ms + k * D + c0);
+            const float av[4] = {a.x, a.y, a.z, a.w}, mv[4] = {m.x, m.y, m.z, m.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], mv[j], acc[i][j]);
+        }
+        __syncthreads();   // every thread is done with st and M_sg
+        float *Sout = slot(sg + 1, 0) + (size_t)rb * 16 * D;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            *reinterpret_cast<float4 *>(Sout + (size_t)(r0 + i) * D + c0) =
+                make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) st[(c0 + j) * 16 + r0 + i] = acc[i][j];
+        }
+    }
 }
 
 // ------------------------------------------------------------ prep kernel ----
@@ -1042,27 +1126,62 @@ chain_kernel(const uint8_t *__restrict__ recs, const float *h0, float *fin, floa
              __nv_bfloat16 *__restrict__ o, uint32_t *err) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t sbase = smem_u32(smem_raw);
-    const int chain = blockIdx.x;
+    // segmented scan: which segment of which chain, and in which role
+    // (0: the chain in full, 1: from a zero state without outputs, 2: the
+    // transition from the identity, without B and outputs)
+    int chain = blockIdx.x, seg = 0, role = 0;
+    if (map.nseg > 0) {
+        const int per = map.phase == 1 ? 2 * map.nseg - 3 : map.nseg - 1;
+        chain = blockIdx.x / per;
+        const int k = blockIdx.x % per;
+        if (map.phase == 1) {
+            seg = k == 0 ? 0 : 1 + (k - 1) / 2;
+            role = k == 0 ? 0 : 1 + ((k - 1) & 1);
+        } else {
+            seg = 1 + k;
+        }
+    }
     const int h = chain % H, n = chain / H;
     int t0, len;
     sequence_range(cu, n, num_seqs, total_T, t0, len);
     const int b0 = map.base[n];
     const int nchunks = map.base[n + 1] - b0;
-    // this launch's local chunks of the sequence
-    const int c_begin = max(map.c0, map.w0 - b0);
-    const int c_stop = min(min(map.c1, map.w1 - b0), nchunks);
-    const bool first_launch = map.c0 == 0 && map.w0 == 0;
-    if (c_stop <= c_begin && !(nchunks == 0 && first_launch)) return;   // nothing here
+    const bool outputs = role == 0, use_b = role != 2, identity = role == 2;
+    int c_begin, c_stop;
+    const float *s_in;
+    float *s_out;
+    size_t in_off = 0, out_off = 0;
+    if (map.nseg > 0) {
+        const int L = (nchunks + map.nseg - 1) / map.nseg;
+        c_begin = min(seg * L, nchunks);
+        c_stop = min(c_begin + L, nchunks);
+        auto slot = [&](int sg, int kind) { return (((size_t)chain * map.nseg + sg) * 3 + kind) * D * D; };
+        s_in = role != 0 ? nullptr : (seg == 0 ? h0 : map.slots);
+        in_off = seg == 0 ? (size_t)chain * D * D : slot(seg, 0);
+        if (map.phase == 1) {
+            s_out = map.slots;
+            out_off = role == 0 ? slot(1, 0) : slot(seg, role);
+        } else {
+            s_out = seg == map.nseg - 1 ? fin : nullptr;
+            out_off = (size_t)chain * D * D;
+        }
+    } else {
+        // this launch's local chunks of the sequence
+        c_begin = max(map.c0, map.w0 - b0);
+        c_stop = min(min(map.c1, map.w1 - b0), nchunks);
+        const bool first_launch = map.c0 == 0 && map.w0 == 0;
+        if (c_stop <= c_begin && !(nchunks == 0 && first_launch)) return;   // nothing here
+        // the state enters from the initial state or from the launch before; it
+        // leaves to the final state or to the launch after (pieces: one slot per
+        // chain; windows: one slot per window boundary, which one sequence crosses)
+        const size_t slot_in = map.by_window ? ((size_t)(map.win - 1) * H + h) : (size_t)chain;
+        const size_t slot_out = map.by_window ? ((size_t)map.win * H + h) : (size_t)chain;
+        s_in = c_begin == 0 ? h0 : ws_state;
+        s_out = c_stop == nchunks ? fin : ws_state;
+        in_off = (c_begin == 0 ? (size_t)chain : slot_in) * D * D;
+        out_off = (c_stop == nchunks ? (size_t)chain : slot_out) * D * D;
+    }
     const int nl = max(c_stop - c_begin, 0);
-    // the state enters from the initial state or from the launch before; it
-    // leaves to the final state or to the launch after (pieces: one slot per
-    // chain; windows: one slot per window boundary, which one sequence crosses)
-    const size_t slot_in = map.by_window ? ((size_t)(map.win - 1) * H + h) : (size_t)chain;
-    const size_t slot_out = map.by_window ? ((size_t)map.win * H + h) : (size_t)chain;
-    const float *s_in = c_begin == 0 ? h0 : ws_state;
-    float *s_out = c_stop == nchunks ? fin : ws_state;
-    const size_t in_off = (c_begin == 0 ? (size_t)chain : slot_in) * D * D;
-    const size_t out_off = (c_stop == nchunks ? (size_t)chain : slot_out) * D * D;
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
@@ -1072,12 +1191,18 @@ chain_kernel(const uint8_t *__restrict__ recs, const float *h0, float *fin, floa
     const int qc = (warp >> 2) & 3;                    // state warps: key-channel quarter
     const size_t tsg = (size_t)r * D + qc * 32;   // this thread's part of a state
 
-    if (nl == 0) {   // empty sequence: the state passes through
+    if (nl == 0) {   // no chunks: the state (or the identity) passes through
         if (s_out != nullptr && warp < kStateWarps) {
 #pragma unroll
             for (int j = 0; j < 32; j += 4) {
                 float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
                 if (s_in != nullptr) x = *reinterpret_cast<const float4 *>(s_in + in_off + tsg + j);
+                if (identity) {
+                    x.x = r == qc * 32 + j ? 1.f : 0.f;
+                    x.y = r == qc * 32 + j + 1 ? 1.f : 0.f;
+                    x.z = r == qc * 32 + j + 2 ? 1.f : 0.f;
+                    x.w = r == qc * 32 + j + 3 ? 1.f : 0.f;
+                }
                 *reinterpret_cast<float4 *>(s_out + out_off + tsg + j) = x;
             }
         }
@@ -1092,7 +1217,7 @@ chain_kernel(const uint8_t *__restrict__ recs, const float *h0, float *fin, floa
     if (tid == 0) {
         for (int s = 0; s < 2; ++s) {
             mbar_init(&m->full[s], 1);
-            mbar_init(&m->empty[s], 1 + kStateThreads + kOutThreads);
+            mbar_init(&m->empty[s], 1 + kStateThreads + (outputs ? kOutThreads : 0));
         }
         mbar_init(&m->bar_s, 1);
         mbar_init(&m->bar_o, 1);
@@ -1129,6 +1254,10 @@ chain_kernel(const uint8_t *__restrict__ recs, const float *h0, float *fin, floa
             float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
             if (s_in != nullptr) x = *reinterpret_cast<const float4 *>(s_in + in_off + tsg + j);
             S[j] = x.x; S[j + 1] = x.y; S[j + 2] = x.z; S[j + 3] = x.w;
+        }
+        if (identity) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) S[j] = r == qc * 32 + j ? 1.f : 0.f;
         }
         bool stop = false;
         // S entering chunk lc -> fp16 high and low parts in TMEM with the row's
@@ -1179,7 +1308,12 @@ chain_kernel(const uint8_t *__restrict__ recs, const float *h0, float *fin, floa
                 for (int p = 0; p < 2; ++p) {
                     uint32_t xd[16], xb[16];
                     tmem_ld16(tmem + lane_off + CT_DS + qc * 32 + p * 16, xd);
-                    tmem_ld16(tmem + lane_off + CT_DB + qc * 32 + p * 16, xb);
+                    if (use_b) {
+                        tmem_ld16(tmem + lane_off + CT_DB + qc * 32 + p * 16, xb);
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) xb[e] = 0u;
+                    }
                     tmem_wait_ld();
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
@@ -1208,7 +1342,7 @@ chain_kernel(const uint8_t *__restrict__ recs, const float *h0, float *fin, floa
         // ================== output warps: value channel r, all 64 tokens ==========
         const int otid = tid - kStateThreads;
         bool stop = false;
-        for (int lc = 0; lc < nl; ++lc) {
+        for (int lc = 0; lc < (outputs ? nl : 0); ++lc) {
             const uint32_t s = lc & 1;
             const uint8_t *stg = sm + s * CSTAGE;
             // take this chunk's O⁰ column r and exponents, then free the record
@@ -1273,10 +1407,12 @@ chain_kernel(const uint8_t *__restrict__ recs, const float *h0, float *fin, floa
                 if (!mbar_wait_sleep(&m->full[s], (lc >> 1) & 1)) { fail(ERR_TIMEOUT_TMA); break; }
                 if (lc > 0 && !mbar_wait_sleep(&m->d_free, (lc - 1) & 1)) { fail(ERR_TIMEOUT_HANDOFF); break; }
                 tc_fence_after();
+                if (use_b) {
 #pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    mma_f16_ss(tmem + CT_DB, sw128_kmajor_desc(stg + REC_UT + k * 32),
-                               sw128_mnmajor_desc(stg + REC_KH + k * 2048, 8192, 1024), IDESC_DB, k != 0);
+                    for (int k = 0; k < 4; ++k)
+                        mma_f16_ss(tmem + CT_DB, sw128_kmajor_desc(stg + REC_UT + k * 32),
+                                   sw128_mnmajor_desc(stg + REC_KH + k * 2048, 8192, 1024), IDESC_DB, k != 0);
+                }
                 if (!mbar_wait_sleep(&m->s_hi, lc & 1)) { fail(ERR_TIMEOUT_HANDOFF); break; }
                 tc_fence_after();
 #pragma unroll
@@ -1292,6 +1428,10 @@ chain_kernel(const uint8_t *__restrict__ recs, const float *h0, float *fin, floa
                                sw128_kmajor_desc(stg + REC_NT + (k >> 2) * 16384 + (k & 3) * 32),
                                IDESC_H128, 1);
                 mma_commit(&m->bar_s);
+                if (!outputs) {
+                    mma_commit(&m->empty[s]);
+                    continue;
+                }
                 if (lc >= 1 && !mbar_wait_sleep(&m->o_free, (lc - 1) & 1)) {
                     fail(ERR_TIMEOUT_HANDOFF);
                     break;
@@ -1349,12 +1489,16 @@ constexpr size_t kMaxRecordBytes = size_t(8) << 30;         // records per windo
 // beyond this many (sequence, head) chains the plan runs the prep kernel over
 // a whole window first, then the chain kernel.
 constexpr int kPipeChains = 64;
+// Segmented scan: at most this many segments per sequence, and phase-1 CTAs
+// (2 per segment) within about one per SM.
+constexpr int kMaxSegments = 8, kSegCTAs = 148;
 
 struct SplitPlan {
     int chains = 0, max_chunks = 0;
     long long max_total = 0;        // bound on the number of global chunks
     int window = 0, windows = 0;    // global chunks per window, windows
     int pieces = 1;                 // pipeline pieces of a single window
+    int nseg = 0;                   // segments per sequence of the segmented scan
     bool by_window = false;
     size_t base_off = 0, state_off = 0, rec_off = 0, bytes = 0;
 };
@@ -1394,8 +1538,19 @@ bool make_split_plan(int num_seqs, int total_T, int H, SplitPlan &p, bool equal_
     int bounds[kMaxPieces + 1];
     p.by_window = !(p.windows == 1 && chains <= kPipeChains);
     p.pieces = p.by_window ? 1 : piece_schedule(p.max_chunks, bounds);
+    // Few chains: the segmented scan, sized so that its first phase (one CTA
+    // for the first segment, two for each later one but the last:
+    // chains (2 nseg - 3) CTAs) fits the 148 SMs at once
+    if (!p.by_window) {
+        const int ns = std::min(kMaxSegments, (kSegCTAs / p.chains + 3) / 2);
+        if (ns >= 4 && p.max_chunks >= 2 * ns) {
+            p.nseg = ns;
+            p.pieces = 1;
+        }
+    }
     size_t state = 0;   // slots for states between launches
     if (p.by_window) state = (size_t)(p.windows - 1) * H * D * D * sizeof(float);
+    else if (p.nseg > 0) state = (size_t)p.chains * p.nseg * 3 * D * D * sizeof(float);
     else if (p.pieces > 1) state = (size_t)p.chains * D * D * sizeof(float);
     p.base_off = kHeaderBytes;
     p.state_off = (p.base_off + (size_t)(num_seqs + 1) * sizeof(int32_t) + 255) & ~size_t(255);
@@ -1485,6 +1640,27 @@ cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, co
         return cudaGetLastError();
     };
     constexpr int kAll = 1 << 30;
+    if (p.nseg > 0) {
+        // the prep kernel over every chunk, then the segmented scan
+        const ChunkMap all{base, 0, (int)p.max_total, 0, p.max_chunks, 0, 0};
+        e = run_prep(all, (unsigned)p.max_chunks, (unsigned)p.chains, stream);
+        if (e != cudaSuccess) return e;
+        ChunkMap seg{base, 0, (int)p.max_total, 0, kAll, 0, 0, p.nseg, 1, state};
+        chain_k<<<(unsigned)(p.chains * (2 * p.nseg - 3)), kChainThreads, CHAIN_SMEM, stream>>>(
+            recs, h0, fin, state, cu, num_seqs, total_T, H, seg, out, err);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        e = ensure_dynamic_smem(reinterpret_cast<const void *>(segment_compose_kernel), (int)COMPOSE_SMEM);
+        if (e != cudaSuccess) return e;
+        segment_compose_kernel<<<dim3((unsigned)p.chains, D / 16), kComposeThreads, COMPOSE_SMEM, stream>>>(
+            state, p.nseg);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        seg.phase = 2;
+        chain_k<<<(unsigned)(p.chains * (p.nseg - 1)), kChainThreads, CHAIN_SMEM, stream>>>(
+            recs, h0, fin, state, cu, num_seqs, total_T, H, seg, out, err);
+        return cudaGetLastError();
+    }
     if (!p.by_window) {
         // one window holds every record; pieces of every sequence's chunks
         int bounds[kMaxPieces + 1];

@@ -122,14 +122,22 @@ def _split_bytes(N, T, H, equal):
     window = min(max_total, (8 << 30) // (H * rec))
     windows = -(-max_total // window)
     by_window = windows > 1 or N * H > 64
-    pieces = 1
+    pieces, nseg = 1, 0
     if not by_window:
         pieces, c, size = 0, 0, 12
         while c < max_chunks and pieces < 32:
             c = max_chunks if pieces + 1 == 32 else min(c + size, max_chunks)
             pieces += 1
             size = (size * 13 + 9) // 10
-    state = (windows - 1) * H * 65536 if by_window else (N * H * 65536 if pieces > 1 else 0)
+        ns = min(8, (148 // (N * H) + 3) // 2)   # few chains: the segmented scan
+        if ns >= 4 and max_chunks >= 2 * ns:
+            nseg, pieces = ns, 1
+    if by_window:
+        state = (windows - 1) * H * 65536
+    elif nseg:
+        state = N * H * nseg * 3 * 65536   # incoming state, B and M of every segment
+    else:
+        state = N * H * 65536 if pieces > 1 else 0
     state_off = (256 + (N + 1) * 4 + 255) // 256 * 256
     rec_off = (state_off + state + 1023) // 1024 * 1024
     return rec_off + window * H * rec, windows

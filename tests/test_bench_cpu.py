@@ -33,9 +33,10 @@ def test_reference_arm_prints_one_contract_line():
 
 
 def test_pipelined_plan_launch_accounting():
-    # one launch numbers the chunks; then 128 chunks in one window: pieces of
-    # 12, 16, 21, 27, 35 and the last 17, each one prep and one chain launch
-    assert bench.split_launches(I.workload("gdn_prefill")) == 1 + 12
+    # one launch numbers the chunks; 16 chains of 128 chunks: one prep launch
+    # over every chunk, then the segmented scan (6 segments): phase 1, the
+    # composition, phase 2
+    assert bench.split_launches(I.workload("gdn_prefill")) == 1 + 1 + 3
     # 64 chains of 98,848-byte records, at most 8 GiB per window: 2715 global
     # chunks of 32 heads.  The two equal sequences go without cu_seqlens, so
     # the plan knows each has 512 chunks (1024 in all): one window, in 10
@@ -43,7 +44,8 @@ def test_pipelined_plan_launch_accounting():
     kda = I.workload("kda_prefill")
     assert (8 << 30) // (32 * 98848) == 2715
     assert bench.split_launches(kda) == 1 + 2 * 10
-    # 48 chains at the gdn_prefill length: the same pieces
+    # 48 chains at the gdn_prefill length: too many for segments, pieces of
+    # 12, 16, 21, 27, 35 and the last 17, each one prep and one chain launch
     assert bench.split_launches(I.workload("gqa_prefill")) == 1 + 12
     # varlen: 128 chains run by windows; packed lengths bound the chunks by
     # 262144 / 64 + 8 = 4104, within one window of 5431 global chunks of 16

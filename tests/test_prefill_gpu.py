@@ -275,19 +275,22 @@ def test_plans_agree(mode):
 
 @pytest.mark.parametrize("mode", [I.SCALAR, I.CHANNEL])
 def test_chunk_parallel_plan_in_pipelined_pieces(mode):
-    """100 chunks of records fit one window, which runs as three pipelined
-    pieces (prep of the next piece beside the chain of this one, the state
-    handed between pieces through the workspace).  Sequences of 32 chunks, one
-    token and 69 chunks, so pieces end inside and after sequences."""
-    inp = I.make_inputs(total_T=6400, H=4, d_k=128, gate_mode=mode, io_dtype=torch.bfloat16,
+    """16 heads x 3 sequences (48 chains, too many for the segmented scan):
+    the records of up to 100 chunks per sequence fit one window, which runs as
+    pipelined pieces (prep of the next piece beside the chain of this one,
+    the state handed between pieces through the workspace).  Sequences of 32
+    chunks, one token and 69 chunks, so pieces end inside and after
+    sequences.  Sampled heads against the oracle."""
+    inp = I.make_inputs(total_T=6400, H=16, d_k=128, gate_mode=mode, io_dtype=torch.bfloat16,
                         cu_seqlens=[0, 2048, 2049, 6400], c=0.1, h0_std=0.02, seed=53)
-    nb = gdr.gdr_prefill_workspace_size(3, 6400, 4, 128, 128, 0 if mode == I.SCALAR else 1,
+    nb = gdr.gdr_prefill_workspace_size(3, 6400, 16, 128, 128, 0 if mode == I.SCALAR else 1,
                                         gdr.GDR_BF16)
-    assert gdr.gdr_prefill_plan(3, 6400, 4, 128, 128, 0 if mode == I.SCALAR else 1, gdr.GDR_BF16,
+    assert gdr.gdr_prefill_plan(3, 6400, 16, 128, 128, 0 if mode == I.SCALAR else 1, gdr.GDR_BF16,
                                 nb) == gdr.GDR_PATH_TCGEN05_SPLIT
     o, fin = gpu_prefill(inp)
-    o_ref, fin_ref = oracle_prefill(inp)
-    check(inp, o, fin, o_ref, fin_ref, "pieces")
+    heads = [0, 9, 15]
+    o_ref, fin_ref = oracle_prefill(inp, heads=heads)
+    check(inp, o[:, heads], fin[:, heads], o_ref, fin_ref, "pieces")
 
 
 @pytest.mark.parametrize("mode", [I.SCALAR, I.CHANNEL])
@@ -326,3 +329,27 @@ def test_many_chains_run_by_windows_with_empty_sequences(mode):
     check(inp, o, fin, o_ref, fin_ref, "windows, many chains")
     for n in np.nonzero(lens == 0)[0]:
         assert torch.equal(fin[n].cpu(), inp.h0[n])
+
+
+
+@pytest.mark.parametrize("mode", [I.SCALAR, I.CHANNEL])
+@pytest.mark.parametrize("case", ["equal", "varlen", "ungated", "strong decay"])
+def test_segmented_scan(mode, case):
+    """Few chains (here 2 heads): each sequence is cut into 8 segments; the
+    segments run from a zero state and their transitions from the identity
+    in parallel, the incoming states are composed segment by segment, and the
+    segments run again from their true incoming states with outputs.  Segment
+    boundaries fall inside chunks' sequences and, with cu_seqlens, sequences
+    end inside segments; the ungated rule (the transitions carry the state
+    undecayed) and strong decays (transitions near zero) are the extremes."""
+    c, cu, T = 0.1, None, 4000
+    if case == "varlen":
+        cu = [0, 1000, 1001, 2500, 4000]
+    inp = I.make_inputs(total_T=T, H=2, d_k=128, gate_mode=mode, io_dtype=torch.bfloat16,
+                        cu_seqlens=cu, num_seqs=1, c=(3.0 if case == "strong decay" else c),
+                        h0_std=0.05, seed=81)
+    if case == "ungated":
+        inp.g = torch.zeros_like(inp.g)
+    o, fin = gpu_prefill(inp, use_cu=cu is not None)
+    o_ref, fin_ref = oracle_prefill(inp)
+    check(inp, o, fin, o_ref, fin_ref, f"segments {case} {mode}")
