@@ -883,7 +883,10 @@ def main():
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": head["dtype"], "data": "synthetic (seeded PCG64; see inputs.py)",
             "config": head["config"], "roofline": head["roofline"], "e2e": head["e2e"],
-            "gpu_launches": sum(r["gpu_launches"] for r in results.values()),
+            "gpu_launches": head["gpu_launches"],
+            # every workload's timed steps together (each line under
+            # "workloads" carries its own count)
+            "gpu_launches_all_workloads": sum(r["gpu_launches"] for r in results.values()),
             "clocks": head["clocks"],
         }
         if "cpu_baseline" in head:

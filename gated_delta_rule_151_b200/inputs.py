@@ -50,6 +50,9 @@ varlen_gdn         8 packed sequences, 262144 tokens, H=16, d=128, bf16,
                    scalar gate c=0.1, h0=0
 gqa_prefill        1 sequence, 8192 tokens, 16 query/key heads shared by 48
                    value heads (3 each), d=128, bf16, scalar gate c=0.05
+kda_prefill_small  kda_prefill at 2 x 2048 tokens (the same 64 chains and
+                   plan at a sixteenth of the length; a profiler capture
+                   holds a few hundred MB on the device instead of 7 GB)
 =================  ==========================================================
 
 With grouped heads (``H_qk`` < ``H``), q and k carry ``H_qk`` heads and value
@@ -360,7 +363,7 @@ def make_prologue_inputs(*, total_T: int, H: int, d_k: int, d_v: int | None = No
 
 WORKLOADS = ("tiny_gdn", "gdn_prefill", "kda_prefill", "decode_gdn",
              "decode_kda", "varlen_gdn", "gqa_prefill", "decode_spec_gdn", "prologue_gdn",
-             "backward_gdn")
+             "backward_gdn", "kda_prefill_small")
 
 SPEC_DRAFT = 4   # tokens verified per sequence per step in decode_spec_gdn
 
@@ -382,8 +385,9 @@ def workload(name: str, seed: int = 0) -> Inputs:
         return make_inputs(total_T=8192, H=16, d_k=128, num_seqs=1, gate_mode=SCALAR,
                            io_dtype=torch.bfloat16, c=0.05, seed=seed,
                            meta={"workload": name})
-    if name == "kda_prefill":
-        return make_inputs(total_T=65536, H=32, d_k=128, num_seqs=2, gate_mode=CHANNEL,
+    if name in ("kda_prefill", "kda_prefill_small"):
+        T = 65536 if name == "kda_prefill" else 4096
+        return make_inputs(total_T=T, H=32, d_k=128, num_seqs=2, gate_mode=CHANNEL,
                            io_dtype=torch.bfloat16, c=0.05, h0_std=0.02, seed=seed,
                            meta={"workload": name})
     if name in ("decode_gdn", "decode_kda", "decode_spec_gdn"):
