@@ -7,15 +7,16 @@ Prints ONE JSON line on rank 0.  The headline (`value`) is the first
 workload; by default that is the largest single-GPU configuration, the
 long-context variable-length GDN prefill (8 packed sequences, 262,144 tokens,
 16 heads, d = 128, bf16).  The other benchmark configurations (the 1 x 8192
-GDN prefill, the 2 x 32768 KDA prefill with an initial state, and the
-256-sequence x 512-step GDN and KDA decodes) follow under "workloads", each
-with the same fields: its own roofline, end-to-end figure, clock record and
-CPU baseline.
+GDN prefill, the 2 x 32768 KDA prefill with an initial state, the
+256-sequence x 512-step GDN and KDA decodes, and the 1 x 8192 GDN prefill
+from raw projections with the input-side prologue fused into it) follow
+under "workloads", each with the same fields: its own roofline, end-to-end
+figure, clock record and (where the recurrence oracle runs it) CPU baseline.
 
 A "step" is one pass of the whole hot path over one batch of synthetic input:
 one gdr_prefill_chunked call for a prefill workload, the 512 consecutive
 gdr_decode_step calls for a decode workload, one gdr_prologue call for the
-prologue workload.  Timing: W untimed warm-up steps, then one step is
+prologue workload, one gdr_prefill_fused call for the fused workload.  Timing: W untimed warm-up steps, then one step is
 captured as a CUDA graph, and K replays of it are each timed with CUDA events
 on the stream the kernels are launched on (--no-graph times eager calls
 instead, which adds the host's per-call time whenever it exceeds the GPU's);
@@ -57,7 +58,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 CHUNK = 64
 # the five benchmark configurations that run on the GPU (the tiny GDN case is
 # a parity-only configuration); the first is the headline
-DEFAULT_WORKLOADS = "varlen_gdn,gdn_prefill,kda_prefill,decode_gdn,decode_kda"
+DEFAULT_WORKLOADS = "varlen_gdn,gdn_prefill,kda_prefill,decode_gdn,decode_kda,prefill_fused_gdn"
 
 
 # ------------------------------------------------------------ plumbing ----
@@ -516,6 +517,67 @@ class PrologueCase:
         return "f32 arithmetic, bf16 in and out"
 
 
+class FusedPrefillCase:
+    """The prologue fused into the chunked prefill at the gdn_prefill shape:
+    one gdr_prefill_fused call per step from the raw projections (the
+    prologue_gdn inputs: convolution with state, SiLU, q/k norms, gate and
+    beta maps) to o, the final state and the outgoing convolution state."""
+    kind = "prefill"
+    kernel_label = "tcgen05 chunk-parallel prefill with the prologue fused into its stage step"
+
+    def __init__(self, name, device, seed):
+        self.name = name
+        self.inp = inp = I.prologue_workload(name, seed=seed)
+        self.dev = device
+        self.d = {k: getattr(inp, k).to(device) for k in
+                  ("xq", "xk", "xv", "wq", "wk", "wv", "xg", "gscale", "xb", "conv_state")}
+        N, T, H = inp.num_seqs, inp.total_T, inp.xv.shape[1]
+        self.N, self.T, self.H = N, T, H
+        self.Call = inp.wq.shape[0] * 2 + inp.wv.shape[0]
+        self.state_out = torch.empty((N, self.Call, 3), dtype=torch.float32, device=device)
+        self.o = torch.empty((T, H, 128), dtype=torch.bfloat16, device=device)
+        self.fin = torch.empty((N, H, 128, 128), dtype=torch.float32, device=device)
+        nb = gdr.gdr_prefill_workspace_size(N, T, H, 128, 128, gdr.GDR_GATE_SCALAR, gdr.GDR_BF16)
+        self.ws = torch.empty(max(nb, 16), dtype=torch.uint8, device=device)
+        e = io_bytes(inp.io_dtype)
+        # read the raw projections, taps, raw gate and beta, coefficients and
+        # the incoming convolution state; write o, the final state and the
+        # outgoing convolution state
+        self.bytes = (T * self.Call * e + self.Call * 16 + inp.xg.numel() * 4 + T * H * 4
+                      + H * 4 + 2 * N * self.Call * 12 + T * H * 128 * e + N * H * 128 * 128 * 4)
+        self.flops = T * H * (5 * CHUNK * 128 + 6 * 128 * 128)
+        self.tokens = T
+        self.launches = 6
+        self.path = None
+
+    def _call(self, d, stream):
+        gdr.gdr_prefill_fused(d["xq"], d["xk"], d["xv"], d["wq"], d["wk"], d["wv"], d["xg"],
+                              d["gscale"], d["xb"], d["conv_state"], None, None,
+                              num_seqs=self.N, conv_state_out=self.state_out, silu=True,
+                              normalize_qk=True, o=self.o, final_state=self.fin,
+                              workspace=self.ws, stream=stream)
+
+    def step(self, stream=None):
+        self._call(self.d, stream)
+
+    def e2e_buffers(self):
+        host = {k: v.cpu().pin_memory() for k, v in self.d.items()}
+        outs = [self.o, self.fin, self.state_out]
+        ho = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
+        h2d = sum(v.numel() * v.element_size() for v in host.values())
+        d2h = sum(o.numel() * o.element_size() for o in ho)
+        return host, ho, None, h2d, d2h
+
+    def e2e_step(self, host, host_o, host_fin, stream):
+        dev = {k: v.to(self.dev, non_blocking=True) for k, v in host.items()}
+        self._call(dev, stream)
+        for h, o in zip(host_o, [self.o, self.fin, self.state_out]):
+            h.copy_(o, non_blocking=True)
+
+    def dtype_label(self):
+        return "bf16/fp16 tensor-core operands, fp32 accumulate, state and prologue arithmetic"
+
+
 class BackwardCase:
     """The gradient of the recurrence at the gdn_prefill shape: one
     gdr_backward call per step (upstream gradients dO and dS_final drawn by
@@ -581,6 +643,8 @@ def make_case(name, device, seed):
         return BackwardCase(name, device, seed)
     if name == "prologue_gdn":
         return PrologueCase(name, device, seed)
+    if name == "prefill_fused_gdn":
+        return FusedPrefillCase(name, device, seed)
     if name == "decode_spec_gdn":
         return SpecDecodeCase(name, device, seed)
     if name.startswith("decode"):

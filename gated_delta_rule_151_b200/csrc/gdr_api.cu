@@ -279,6 +279,102 @@ gdr_status_t gdr_prologue(const void *xq, const void *xk, const void *xv, const 
         beta, static_cast<cudaStream_t>(stream)));
 }
 
+gdr_status_t gdr_prefill_fused(const void *xq, const void *xk, const void *xv, const float *wq,
+                               const float *wk, const float *wv, const float *xg,
+                               const float *gscale, const float *xb, const float *conv_state_in,
+                               float *conv_state_out, const float *initial_state,
+                               const int32_t *cu_seqlens, int32_t num_seqs, int32_t total_T,
+                               int32_t H_qk, int32_t H, int32_t d_k, int32_t d_v,
+                               gdr_gate_mode_t gate_mode, gdr_dtype_t io_dtype, uint32_t flags,
+                               void *o, float *final_state, void *workspace,
+                               size_t workspace_bytes, void *stream) {
+    if (num_seqs < 1 || total_T < 0 || H < 1 || H_qk < 1 || H % H_qk != 0)
+        return GDR_ERR_INVALID_ARG;
+    if (!valid_dim(d_k) || !valid_dim(d_v)) return GDR_ERR_INVALID_ARG;
+    if (gate_mode != GDR_GATE_SCALAR && gate_mode != GDR_GATE_CHANNEL) return GDR_ERR_INVALID_ARG;
+    if (io_dtype != GDR_F32 && io_dtype != GDR_BF16) return GDR_ERR_INVALID_ARG;
+    if ((flags & ~(GDR_PROLOGUE_SILU | GDR_PROLOGUE_NORMALIZE_QK)) != 0) return GDR_ERR_INVALID_ARG;
+    if (cu_seqlens == nullptr && total_T % num_seqs != 0) return GDR_ERR_INVALID_ARG;
+    if ((int64_t)total_T * H > (int64_t)INT32_MAX) return GDR_ERR_INVALID_ARG;
+    const int64_t Cq = (int64_t)H_qk * d_k, Cv = (int64_t)H * d_v, Call = 2 * Cq + Cv;
+    if ((int64_t)num_seqs * Call > INT32_MAX) return GDR_ERR_INVALID_ARG;
+    if (conv_state_out != nullptr && !aligned4(conv_state_out)) return GDR_ERR_INVALID_ARG;
+    if (conv_state_in != nullptr && !aligned4(conv_state_in)) return GDR_ERR_INVALID_ARG;
+    if (!ok_ptr(wq) || !ok_ptr(wk) || !ok_ptr(wv)) return GDR_ERR_INVALID_ARG;
+    if (!ok_opt_ptr(initial_state) || !ok_opt_ptr(final_state) || !ok_opt_ptr(cu_seqlens))
+        return GDR_ERR_INVALID_ARG;
+    if (total_T > 0) {
+        if (!ok_ptr(xq) || !ok_ptr(xk) || !ok_ptr(xv) || !ok_ptr(o) ||
+            !ok_gate_ptr(xg, gate_mode) || !ok_beta_ptr(xb) || gscale == nullptr ||
+            !aligned4(gscale))
+            return GDR_ERR_INVALID_ARG;
+    }
+    // outputs overlap no input (final_state may be initial_state itself, as
+    // for gdr_prefill_chunked) and no other output
+    const size_t T = (size_t)total_T;
+    const size_t gsz = T * H * (gate_mode == GDR_GATE_CHANNEL ? d_k : 1) * 4;
+    const size_t ssz = (size_t)num_seqs * Call * 3 * 4, hsz = (size_t)num_seqs * H * d_v * d_k * 4;
+    struct Range {
+        const void *p;
+        size_t n;
+    };
+    const Range in[] = {{xq, T * Cq * 2}, {xk, T * Cq * 2}, {xv, T * Cv * 2},
+                        {wq, (size_t)Cq * 16}, {wk, (size_t)Cq * 16}, {wv, (size_t)Cv * 16},
+                        {xg, gsz}, {gscale, (size_t)H * 4}, {xb, T * H * 4},
+                        {conv_state_in, ssz},
+                        {initial_state == final_state ? nullptr : initial_state, hsz},
+                        {cu_seqlens, ((size_t)num_seqs + 1) * 4}};
+    const Range out[] = {{o, T * Cv * 2}, {final_state, hsz}, {conv_state_out, ssz}};
+    for (const Range &r : out) {
+        if (r.p == nullptr || r.n == 0) continue;
+        const uintptr_t o0 = reinterpret_cast<uintptr_t>(r.p), o1 = o0 + r.n;
+        for (const Range &i : in) {
+            if (i.p == nullptr || i.n == 0) continue;
+            const uintptr_t i0 = reinterpret_cast<uintptr_t>(i.p), i1 = i0 + i.n;
+            if (o0 < i1 && i0 < o1) return GDR_ERR_INVALID_ARG;
+        }
+        for (const Range &r2 : out) {
+            if (&r2 == &r || r2.p == nullptr || r2.n == 0) continue;
+            const uintptr_t a0 = reinterpret_cast<uintptr_t>(r2.p), a1 = a0 + r2.n;
+            if (o0 < a1 && a0 < o1) return GDR_ERR_INVALID_ARG;
+        }
+    }
+    // the fused staging lives in the chunk-parallel tensor-core plan only
+    if (!uses_tcgen05(d_k, d_v, gate_mode, io_dtype)) return GDR_ERR_UNSUPPORTED;
+    if (workspace_bytes > 0 && (workspace == nullptr || !aligned16(workspace)))
+        return GDR_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (total_T > 0) {
+        gdr_prefill_path_t plan;
+        gdr_status_t st = gdr_prefill_plan(num_seqs, total_T, H, d_k, d_v, gate_mode, io_dtype,
+                                           workspace == nullptr ? 0 : workspace_bytes, &plan);
+        if (st != GDR_OK) return st;
+        if (plan != GDR_PATH_TCGEN05_SPLIT) return GDR_ERR_WORKSPACE;
+    }
+    cudaError_t e = gdr::launch_prologue_state(xq, xk, xv, conv_state_in, conv_state_out,
+                                               cu_seqlens, num_seqs, total_T, H_qk, H, d_k, d_v,
+                                               true, s);
+    if (e != cudaSuccess) return GDR_ERR_CUDA;
+    if (total_T == 0)   // no tokens: the states pass through (or start at zero)
+        return gdr_prefill_chunked_gqa(nullptr, nullptr, nullptr, nullptr, nullptr, initial_state,
+                                       cu_seqlens, num_seqs, 0, H_qk, H, d_k, d_v, gate_mode,
+                                       io_dtype, nullptr, final_state, workspace, workspace_bytes,
+                                       stream);
+    gdr::PrologueIn pin;
+    pin.xq = xq; pin.xk = xk; pin.xv = xv;
+    pin.wq = wq; pin.wk = wk; pin.wv = wv;
+    pin.xg = xg; pin.gscale = gscale; pin.xb = xb;
+    pin.state_in = conv_state_in;
+    pin.Cq = (int)Cq;
+    pin.Call = (int)Call;
+    pin.silu = (flags & GDR_PROLOGUE_SILU) != 0;
+    pin.norm = (flags & GDR_PROLOGUE_NORMALIZE_QK) != 0;
+    return from_cuda(gdr::launch_prefill_split(nullptr, nullptr, nullptr, nullptr, nullptr,
+                                               initial_state, cu_seqlens, num_seqs, total_T, H_qk,
+                                               H, gate_mode == GDR_GATE_CHANNEL, o, final_state,
+                                               workspace, s, &pin));
+}
+
 gdr_status_t gdr_backward_workspace_size(int32_t num_seqs, int32_t total_T, int32_t H,
                                          int32_t d_k, int32_t d_v, size_t *bytes) {
     if (bytes == nullptr || num_seqs < 0 || total_T < 0 || H < 0 || !valid_dim(d_k) ||

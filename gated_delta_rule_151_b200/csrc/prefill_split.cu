@@ -45,6 +45,16 @@
 // Records take 98,848 bytes per (chunk, head); problems whose records exceed
 // 8 GiB run in windows of chunks, the state passing between windows
 // through the workspace.
+//
+// Because the chunk map is affine, a run of chunks composes into one affine
+// map as well.  With few (sequence, head) chains the chain is cut into
+// segments: a first launch runs segment 0 from the initial state and every
+// middle segment twice, from a zero state (its B_s) and from the identity
+// without B (its transition M_s); a small fp32 kernel chains
+// S_in(s + 1) = S_in(s) M_s + B_s; a second launch runs every later segment
+// in full from its incoming state.  With at most 64 chains and one window,
+// the step is instead cut into pieces of chunks whose prep runs beside the
+// previous piece's chain on helper streams.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
@@ -396,13 +406,140 @@ __device__ __forceinline__ bool block_wait(uint64_t *bar, uint32_t phase, int *a
     return *reinterpret_cast<volatile int *>(abort_flag) == 0;
 }
 
-template <bool CHANNEL>
+// Fused input-side prologue: the chunk's q, k (query/key head hq) and v
+// (value head h) tiles computed from the raw projections instead of loaded.
+// Each token is the depthwise causal convolution of kernel size four (page
+// "Qwen3.8-Flash-Next and GLM-5.3-Flash share a 3:1 long-context pattern",
+// section "Kimi Delta Attention extends recurrent memory control") of the
+// token and the three before it, with the incoming convolution state before
+// the sequence's first token; then the optional SiLU and the q/k L2 norms
+// over the head's 128 channels.
+//
+// The raw rows of the chunk and the three before it (those inside the
+// sequence) are staged in the scratch regions with 16-byte asynchronous
+// copies, all in flight together, issued before the CTA sets up its barriers
+// and TMEM.  Then warp w computes tokens 8w .. 8w + 7, lane l channels
+// 4l .. 4l + 3, with the standalone prologue kernel's arithmetic (packed
+// fp32x2 convolution and SiLU, the eight tokens' norms reduced together:
+// the same bits), and writes bf16 into the 128-byte-swizzled tile layout the
+// TMA loads produce.  Rows past the sequence's end are zero.
+constexpr int kStageRows = C + 3;                      // rows c C - 3 .. c C + 63
+constexpr uint32_t PO_STAGE = PO_RA;                   // [k, q, v][kStageRows][128] bf16
+static_assert(PO_STAGE + 3 * kStageRows * 256 <= PO_MISC, "fused prologue staging overflow");
+
+__device__ __forceinline__ void fused_prologue_stage(const PrologueIn &P, uint8_t *sm, int t0,
+                                                     int len, int c, int hq, int h, int Hqk,
+                                                     int H) {
+#pragma unroll 1
+    for (int which = 0; which < 3; ++which) {   // k, q, v
+        const __nv_bfloat16 *x =
+            static_cast<const __nv_bfloat16 *>(which == 0 ? P.xk : which == 1 ? P.xq : P.xv);
+        const int width = which == 2 ? H * D : Hqk * D;
+        const __nv_bfloat16 *src = x + (which == 2 ? h : hq) * D;
+        uint8_t *dst = sm + PO_STAGE + (uint32_t)which * kStageRows * 256u;
+        for (int e = threadIdx.x; e < kStageRows * 16; e += kPrepThreads) {   // 16-byte pieces
+            const int r = e >> 4, piece = e & 15;
+            const int tau = c * C - 3 + r;
+            if (tau >= 0 && tau < len)
+                async_copy16(dst + r * 256 + piece * 16, src + (size_t)(t0 + tau) * width + piece * 8);
+        }
+    }
+    async_commit();
+}
+
+__device__ __forceinline__ void fused_prologue_tiles(const PrologueIn &P, uint8_t *sm, int n,
+                                                     int len, int c, int hq, int h) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int cl = min(C, len - c * C);
+    async_wait<0>();
+    __syncthreads();   // every thread's staged rows have landed
+
+    const int i0 = warp * 8;
+    const uint32_t lane_ch = (uint32_t)(lane & 15) >> 1, lane_b = (uint32_t)(lane & 1) * 8u;
+#pragma unroll 1
+    for (int which = 0; which < 3; ++which) {   // k, q, v
+        const bool isv = which == 2;
+        const int col = (isv ? h : hq) * D + 4 * lane;            // this lane's first channel
+        const float *w = which == 0 ? P.wk : which == 1 ? P.wq : P.wv;
+        const int choff = which == 0 ? P.Cq : which == 1 ? 0 : 2 * P.Cq;
+        float2 tp[2][4];                                          // [channel pair][tap]
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const float4 a = *reinterpret_cast<const float4 *>(w + (size_t)(col + 2 * j) * 4);
+            const float4 b = *reinterpret_cast<const float4 *>(w + (size_t)(col + 2 * j + 1) * 4);
+            tp[j][0] = make_float2(a.x, b.x); tp[j][1] = make_float2(a.y, b.y);
+            tp[j][2] = make_float2(a.z, b.z); tp[j][3] = make_float2(a.w, b.w);
+        }
+        // window rows: tokens i0 - 3 .. i0 + 7 of the chunk (sequence positions
+        // tau = c C + i); before the sequence the incoming state, past its end 0
+        const uint8_t *rows = sm + PO_STAGE + (uint32_t)(which * kStageRows + i0) * 256u + lane * 8;
+        float2 xp[11][2];
+#pragma unroll
+        for (int r = 0; r < 11; ++r) {
+            const int tau = c * C + i0 - 3 + r;
+            if (tau >= 0 && tau < len) {
+                const uint2 raw = *reinterpret_cast<const uint2 *>(rows + r * 256);
+                xp[r][0] = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.x));
+                xp[r][1] = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.y));
+            } else {
+                float v4[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    v4[j] = (tau < 0 && P.state_in != nullptr)
+                                ? P.state_in[((size_t)n * P.Call + choff + col + j) * 3 + (tau + 3)]
+                                : 0.f;
+                xp[r][0] = make_float2(v4[0], v4[1]);
+                xp[r][1] = make_float2(v4[2], v4[3]);
+            }
+        }
+        float ss[8];
+#pragma unroll
+        for (int s = 0; s < 8; ++s) {
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                float2 acc = __fmul2_rn(tp[j][0], xp[s][j]);
+                acc = __ffma2_rn(tp[j][1], xp[s + 1][j], acc);
+                acc = __ffma2_rn(tp[j][2], xp[s + 2][j], acc);
+                acc = __ffma2_rn(tp[j][3], xp[s + 3][j], acc);
+                xp[s][j] = P.silu ? silu2(acc) : acc;   // row s is not read again
+            }
+            const float2 q2 = __ffma2_rn(xp[s][1], xp[s][1], __fmul2_rn(xp[s][0], xp[s][0]));
+            ss[s] = q2.x + q2.y;
+        }
+        if (P.norm != 0 && !isv) {
+            float tot[8];
+            norm_sums8(ss, lane, tot);
+#pragma unroll
+            for (int s = 0; s < 8; ++s) {
+                const float rn = rsqrt_approx(tot[s] + kNormEps);
+                xp[s][0] = __fmul2_rn(xp[s][0], make_float2(rn, rn));
+                xp[s][1] = __fmul2_rn(xp[s][1], make_float2(rn, rn));
+            }
+        }
+        uint8_t *tile = sm + (which == 0 ? PO_KQ : which == 1 ? PO_KQ + 8192 : PO_V);
+        const uint32_t blk = (uint32_t)(lane >> 4) * (isv ? 8192u : 16384u);
+#pragma unroll
+        for (int s = 0; s < 8; ++s) {
+            const int i = i0 + s;
+            const float2 z = make_float2(0.f, 0.f);
+            const bool live = i < cl;
+            const __nv_bfloat162 lo = __float22bfloat162_rn(live ? xp[s][0] : z);
+            const __nv_bfloat162 hi = __float22bfloat162_rn(live ? xp[s][1] : z);
+            uint2 st;
+            st.x = *reinterpret_cast<const uint32_t *>(&lo);
+            st.y = *reinterpret_cast<const uint32_t *>(&hi);
+            *reinterpret_cast<uint2 *>(tile + blk + sw128_offset(i, lane_ch) + lane_b) = st;
+        }
+    }
+}
+
+template <bool CHANNEL, bool FUSED>
 __global__ void __launch_bounds__(kPrepThreads, 2)
 prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
             const __grid_constant__ CUtensorMap tm_v, const float *__restrict__ g,
             const float *__restrict__ beta, const int32_t *__restrict__ cu, int num_seqs,
             int total_T, int Hqk, int H, const ChunkMap map, uint8_t *__restrict__ recs,
-            uint32_t *err) {
+            const PrologueIn pin, uint32_t *err) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t sbase = smem_u32(smem_raw);
     int n, h, c, gc;
@@ -439,6 +576,8 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     const int tok0 = t0 + c * C;
     const int cl = min(C, len - c * C);
 
+    if (FUSED) fused_prologue_stage(pin, sm, t0, len, c, hq, h, Hqk, H);
+
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
     const int sub = warp & 3;           // TMEM sub-partition of this warp
@@ -462,7 +601,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = m->tmem_base;
-    if (tid == 0) {
+    if (!FUSED && tid == 0) {
         mbar_arrive_expect_tx(&m->bar_tma, 6 * 8192);
         tma_load_3d(sm + PO_KQ + 0, &tm_k, &m->bar_tma, 0, hq, tok0);
         tma_load_3d(sm + PO_KQ + 16384, &tm_k, &m->bar_tma, 64, hq, tok0);
@@ -480,9 +619,15 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         if (tid < 32) {
             const int i0 = 2 * tid, i1 = 2 * tid + 1;
             const size_t r0 = (size_t)(tok0 + i0) * H + h, r1 = (size_t)(tok0 + i1) * H + h;
-            const float b0 = i0 < cl ? beta[r0] : 0.f, b1 = i1 < cl ? beta[r1] : 0.f;
-            const float g0 = i0 < cl ? clamp_log_gate(g[r0]) : 0.f;
-            const float g1 = i1 < cl ? clamp_log_gate(g[r1]) : 0.f;
+            float b0 = 0.f, b1 = 0.f, g0 = 0.f, g1 = 0.f;
+            if (FUSED) {
+                const float cg = pin.gscale[h];
+                if (i0 < cl) { b0 = beta_of(pin.xb[r0]); g0 = clamp_log_gate(log_gate_of(cg, pin.xg[r0])); }
+                if (i1 < cl) { b1 = beta_of(pin.xb[r1]); g1 = clamp_log_gate(log_gate_of(cg, pin.xg[r1])); }
+            } else {
+                if (i0 < cl) { b0 = beta[r0]; g0 = clamp_log_gate(g[r0]); }
+                if (i1 < cl) { b1 = beta[r1]; g1 = clamp_log_gate(g[r1]); }
+            }
             const float pair = g0 + g1;
             float incl = pair;
 #pragma unroll
@@ -505,21 +650,34 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             }
         }
     } else {
+        const float cg = FUSED ? pin.gscale[h] : 0.f;
 #pragma unroll
         for (int k = 0; k < 32; ++k) {
             const int i = hh * 32 + k;
-            gr[k] = i < cl ? g[((size_t)(tok0 + i) * H + h) * D + ch] : 0.f;
+            const size_t gi = ((size_t)(tok0 + i) * H + h) * D + ch;
+            gr[k] = i < cl ? (FUSED ? log_gate_of(cg, pin.xg[gi]) : g[gi]) : 0.f;
         }
         gr[0] = clamp_log_gate(gr[0]);
 #pragma unroll
         for (int k = 1; k < 32; ++k) gr[k] = clamp_log_gate(gr[k]) + gr[k - 1];
         if (hh == 0) m->u.c.T0[ch] = gr[31];
         else m->u.c.T1[ch] = gr[31];
-        if (tid < C) m->u.c.beta[tid] = tid < cl ? beta[(size_t)(tok0 + tid) * H + h] : 0.f;
+        if (tid < C) {
+            const size_t bi = (size_t)(tok0 + tid) * H + h;
+            m->u.c.beta[tid] = tid < cl ? (FUSED ? beta_of(pin.xb[bi]) : beta[bi]) : 0.f;
+        }
     }
 
     do {
-        if (!block_wait(&m->bar_tma, 0, &m->abort_flag, err, ERR_TIMEOUT_TMA)) break;
+        if (FUSED) {
+            // the tiles from the staged raw rows (their copies overlapped the
+            // set-up and the gate loads above)
+            fused_prologue_tiles(pin, sm, n, len, c, hq, h);
+            fence_proxy_async();   // the tiles are MMA operands
+            __syncthreads();
+        } else if (!block_wait(&m->bar_tma, 0, &m->abort_flag, err, ERR_TIMEOUT_TMA)) {
+            break;
+        }
 
         float GC = 0.f;
         float kmax = 0.f, qmax = 0.f;   // channel gate: this thread's largest |k| and |q|
@@ -1605,7 +1763,8 @@ size_t tcgen05_split_workspace_bytes(int num_seqs, int total_T, int H) {
 cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, const float *g,
                                  const float *beta, const float *h0, const int32_t *cu,
                                  int num_seqs, int total_T, int Hqk, int H, bool channel, void *o,
-                                 float *fin, void *workspace, cudaStream_t stream) {
+                                 float *fin, void *workspace, cudaStream_t stream,
+                                 const PrologueIn *pin) {
     SplitPlan p;
     if (!make_split_plan(num_seqs, total_T, H, p, cu == nullptr)) return cudaErrorInvalidValue;
     uint8_t *ws = static_cast<uint8_t *>(workspace);
@@ -1613,11 +1772,22 @@ cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, co
     int32_t *base = reinterpret_cast<int32_t *>(ws + p.base_off);
     cudaError_t e = cudaMemsetAsync(err, 0, sizeof(uint32_t), stream);
     if (e != cudaSuccess) return e;
+    // with the fused prologue the tiles are computed, not loaded: the maps
+    // (over the raw projections, of the same shape) are passed but unused
+    const bool fused = pin != nullptr;
+    PrologueIn pi = {};
+    if (fused) {
+        pi = *pin;
+        q = pi.xq;
+        k = pi.xk;
+        v = pi.xv;
+    }
     CUtensorMap mq, mk, mv;
     if (!make_map(&mq, q, total_T, Hqk) || !make_map(&mk, k, total_T, Hqk) ||
         !make_map(&mv, v, total_T, H))
         return cudaErrorInvalidValue;
-    auto prep = channel ? prep_kernel<true> : prep_kernel<false>;
+    auto prep = channel ? (fused ? prep_kernel<true, true> : prep_kernel<true, false>)
+                        : (fused ? prep_kernel<false, true> : prep_kernel<false, false>);
     e = ensure_dynamic_smem(reinterpret_cast<const void *>(prep), (int)PREP_SMEM);
     if (e != cudaSuccess) return e;
     auto chain_k = channel ? chain_kernel<true> : chain_kernel<false>;
@@ -1636,7 +1806,7 @@ cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, co
     };
     auto run_prep = [&](const ChunkMap &map, unsigned gx, unsigned gy, cudaStream_t st) {
         prep<<<dim3(gx, gy), kPrepThreads, PREP_SMEM, st>>>(mq, mk, mv, g, beta, cu, num_seqs, total_T,
-                                                            Hqk, H, map, recs, err);
+                                                            Hqk, H, map, recs, pi, err);
         return cudaGetLastError();
     };
     constexpr int kAll = 1 << 30;

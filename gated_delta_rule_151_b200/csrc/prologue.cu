@@ -48,7 +48,6 @@ constexpr int kProThreads = 32 * kProWarps;
 // shared memory of one block: every warp's ring of window rows, 128 channels
 template <typename IoT>
 constexpr int pro_smem_bytes() { return kProWarps * kProStages * kProRows * 128 * (int)sizeof(IoT); }
-constexpr float kNormEps = 1e-6f;
 
 struct ProArgs {
     const void *xq, *xk, *xv;
@@ -112,41 +111,6 @@ __device__ __forceinline__ int seq_of(const ProArgs &A, int t, int &a, int &b) {
     sequence_range(A.cu, lo, A.num_seqs, A.total_T, a, b);
     b += a;
     return lo;
-}
-
-// Single-instruction approximations (denormals flushed: every operand here is
-// either normal or its exact result is 0 or 1 to fp32 precision).
-__device__ __forceinline__ float ex2_approx(float x) {
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-
-__device__ __forceinline__ float rcp_approx(float x) {
-    float y;
-    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-
-__device__ __forceinline__ float rsqrt_approx(float x) {   // x >= 1e-6 here
-    float y;
-    asm("rsqrt.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-
-constexpr float kLog2e = 1.4426950408889634f;
-
-// SiLU y / (1 + e^-y) = y * 1 / (1 + 2^(-y log2 e)), on a pair of channels.
-// For y -> -inf the power overflows to inf and the reciprocal to 0.
-__device__ __forceinline__ float2 silu2(float2 y) {
-    float2 t = __fmul2_rn(y, make_float2(-kLog2e, -kLog2e));
-    t = make_float2(ex2_approx(t.x), ex2_approx(t.y));
-    t = __fadd2_rn(t, make_float2(1.f, 1.f));
-    return __fmul2_rn(y, make_float2(rcp_approx(t.x), rcp_approx(t.y)));
-}
-
-__device__ __forceinline__ float silu_f(float y) {
-    return y * rcp_approx(1.0f + ex2_approx(-kLog2e * y));
 }
 
 __device__ __forceinline__ void cp_async16(void *dst, const void *src) {
@@ -323,28 +287,7 @@ __device__ __forceinline__ void compute_run(const ProArgs &A, const ProItem &it,
     if (normed) {
         float tot[kProRun];
         if (group == 32) {
-            // transposed butterfly: halve the tokens a lane carries at each of
-            // the xor-16/8/4 steps, finish with xor 2/1, then fetch each
-            // token's total from a lane that holds it (token of lane l:
-            // 4 bit4(l) + 2 bit3(l) + bit2(l))
-            const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
-            float v4[4], v2[2];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const float send = b4 ? ss[k] : ss[k + 4], keep = b4 ? ss[k + 4] : ss[k];
-                v4[k] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
-            }
-#pragma unroll
-            for (int k = 0; k < 2; ++k) {
-                const float send = b3 ? v4[k] : v4[k + 2], keep = b3 ? v4[k + 2] : v4[k];
-                v2[k] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
-            }
-            float v = (b2 ? v2[1] : v2[0]) + __shfl_xor_sync(0xffffffffu, b2 ? v2[0] : v2[1], 4);
-            v += __shfl_xor_sync(0xffffffffu, v, 2);
-            v += __shfl_xor_sync(0xffffffffu, v, 1);
-#pragma unroll
-            for (int k = 0; k < kProRun; ++k)
-                tot[k] = __shfl_sync(0xffffffffu, v, ((k >> 2) & 1) * 16 + ((k >> 1) & 1) * 8 + (k & 1) * 4);
+            norm_sums8(ss, lane, tot);
         } else {
 #pragma unroll
             for (int k = 0; k < kProRun; ++k) tot[k] = ss[k];
@@ -433,10 +376,6 @@ __device__ void conv_warps(const ProArgs &A, uint8_t *smem) {
     }
 }
 
-__device__ __forceinline__ float softplus_f(float x) {
-    return x > 20.f ? x : log1pf(expf(x));
-}
-
 template <typename IoT>
 __global__ void __launch_bounds__(kProThreads, 4)
 prologue_kernel(const __grid_constant__ ProArgs A) {
@@ -453,9 +392,9 @@ prologue_kernel(const __grid_constant__ ProArgs A) {
         const size_t ng = A.channel ? nb * A.dk : nb;
         for (size_t i = first; i < ng; i += stride) {
             const int h = A.channel ? (int)((i / A.dk) % A.H) : (int)(i % A.H);
-            A.g[i] = -A.gscale[h] * softplus_f(A.xg[i]);
+            A.g[i] = log_gate_of(A.gscale[h], A.xg[i]);
         }
-        for (size_t i = first; i < nb; i += stride) A.beta[i] = 1.0f / (1.0f + expf(-A.xb[i]));
+        for (size_t i = first; i < nb; i += stride) A.beta[i] = beta_of(A.xb[i]);
         return;
     }
     // convolution state out: the inputs at b-3, b-2, b-1 of every sequence
@@ -484,6 +423,24 @@ prologue_kernel(const __grid_constant__ ProArgs A) {
     }
 #pragma unroll
     for (int j = 0; j < 3; ++j) A.state_out[i * 3 + j] = s[j];
+}
+
+// One launch of the prologue kernel with the roles A sizes.
+cudaError_t run_prologue(const ProArgs &A, bool bf16, cudaStream_t stream) {
+    const long long blocks = (long long)A.conv_blocks + A.gate_blocks + A.state_blocks;
+    cudaError_t e;
+    if (bf16) {
+        constexpr int smem = pro_smem_bytes<__nv_bfloat16>();
+        e = ensure_dynamic_smem(reinterpret_cast<const void *>(prologue_kernel<__nv_bfloat16>), smem);
+        if (e != cudaSuccess) return e;
+        prologue_kernel<__nv_bfloat16><<<(unsigned)blocks, kProThreads, smem, stream>>>(A);
+    } else {
+        constexpr int smem = pro_smem_bytes<float>();
+        e = ensure_dynamic_smem(reinterpret_cast<const void *>(prologue_kernel<float>), smem);
+        if (e != cudaSuccess) return e;
+        prologue_kernel<float><<<(unsigned)blocks, kProThreads, smem, stream>>>(A);
+    }
+    return cudaGetLastError();
 }
 
 }  // namespace
@@ -524,18 +481,25 @@ cudaError_t launch_prologue(const void *xq, const void *xk, const void *xv, cons
     const long long blocks = (long long)A.conv_blocks + A.gate_blocks + A.state_blocks;
     if (blocks == 0) return cudaSuccess;
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-    if (bf16) {
-        constexpr int smem = pro_smem_bytes<__nv_bfloat16>();
-        e = ensure_dynamic_smem(reinterpret_cast<const void *>(prologue_kernel<__nv_bfloat16>), smem);
-        if (e != cudaSuccess) return e;
-        prologue_kernel<__nv_bfloat16><<<(unsigned)blocks, kProThreads, smem, stream>>>(A);
-    } else {
-        constexpr int smem = pro_smem_bytes<float>();
-        e = ensure_dynamic_smem(reinterpret_cast<const void *>(prologue_kernel<float>), smem);
-        if (e != cudaSuccess) return e;
-        prologue_kernel<float><<<(unsigned)blocks, kProThreads, smem, stream>>>(A);
-    }
-    return cudaGetLastError();
+    return run_prologue(A, bf16, stream);
+}
+
+cudaError_t launch_prologue_state(const void *xq, const void *xk, const void *xv,
+                                  const float *state_in, float *state_out, const int32_t *cu,
+                                  int num_seqs, int total_T, int Hqk, int H, int dk, int dv,
+                                  bool bf16, cudaStream_t stream) {
+    ProArgs A = {};
+    A.xq = xq; A.xk = xk; A.xv = xv;
+    A.state_in = state_in; A.state_out = state_out; A.cu = cu;
+    A.num_seqs = num_seqs; A.total_T = total_T; A.Hqk = Hqk; A.H = H; A.dk = dk; A.dv = dv;
+    A.Cq = Hqk * dk; A.Cv = H * dv; A.Call = 2 * A.Cq + A.Cv;
+    A.conv_blocks = 0;
+    A.gate_blocks = 0;
+    A.state_blocks = state_out != nullptr
+                         ? (int)(((long long)num_seqs * A.Call + kProThreads - 1) / kProThreads)
+                         : 0;
+    if (A.state_blocks == 0) return cudaSuccess;
+    return run_prologue(A, bf16, stream);
 }
 
 }  // namespace gdr

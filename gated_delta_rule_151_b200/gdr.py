@@ -40,7 +40,7 @@ EXPORTED = ("gdr_status_string", "gdr_prefill_workspace_size", "gdr_prefill_path
             "gdr_prefill_chunked_noalloc", "gdr_prefill_chunked_gqa", "gdr_decode_step_gqa",
             "gdr_decode_multi", "gdr_prefill_plan", "gdr_prologue", "gdr_backward",
             "gdr_backward_workspace_size", "gdr_prefill_noalloc_check",
-            "gdr_test_noalloc_wait_timeout")
+            "gdr_test_noalloc_wait_timeout", "gdr_prefill_fused")
 
 
 class GdrError(RuntimeError):
@@ -99,6 +99,9 @@ def load_library():
         lib.gdr_decode_multi.restype = ST
         lib.gdr_prologue.argtypes = [P] * 12 + [I32] * 6 + [ST, ST, ctypes.c_uint32] + [P] * 6
         lib.gdr_prologue.restype = ST
+        lib.gdr_prefill_fused.argtypes = ([P] * 13 + [I32] * 6 + [ST, ST, ctypes.c_uint32] +
+                                          [P, P, P, SZ, P])
+        lib.gdr_prefill_fused.restype = ST
         lib.gdr_backward_workspace_size.argtypes = [I32, I32, I32, I32, I32, ctypes.POINTER(SZ)]
         lib.gdr_backward_workspace_size.restype = ST
         lib.gdr_backward.argtypes = [P] * 7 + [I32] * 6 + [ST, ST] + [P] * 9 + [SZ, P]
@@ -411,6 +414,56 @@ def gdr_prologue(xq, xk, xv, wq, wk, wv, xg, gscale, xb, conv_state_in=None, cu_
         _stream_ptr(stream))
     _check(st, "gdr_prologue")
     return q, k, v, g, beta
+
+
+def gdr_prefill_fused(xq, xk, xv, wq, wk, wv, xg, gscale, xb, conv_state_in=None,
+                      initial_state=None, cu_seqlens=None, *, num_seqs=None, conv_state_out=None,
+                      silu=False, normalize_qk=True, o=None, final_state=None,
+                      output_final_state=True, workspace=None, stream=None):
+    """The prologue fused into the chunked prefill (see include/gdr.h):
+    raw inputs as for gdr_prologue, the state and outputs as for
+    gdr_prefill_chunked_gqa.  Returns (o, final_state)."""
+    _need(xq, "xq", torch.bfloat16, 3)
+    _need(xk, "xk", torch.bfloat16, 3)
+    _need(xv, "xv", torch.bfloat16, 3)
+    for t, name in ((wq, "wq"), (wk, "wk"), (wv, "wv")):
+        _need(t, name, torch.float32, 2)
+    _need(xg, "xg", torch.float32)
+    _need(gscale, "gscale", torch.float32, 1)
+    _need(xb, "xb", torch.float32, 2)
+    T, Hqk, dk = xq.shape
+    H, dv = xv.shape[1], xv.shape[2]
+    gate = GDR_GATE_SCALAR if xg.dim() == 2 else GDR_GATE_CHANNEL
+    if cu_seqlens is not None:
+        _need(cu_seqlens, "cu_seqlens", torch.int32, 1)
+        N = cu_seqlens.numel() - 1
+    else:
+        N = 1 if num_seqs is None else int(num_seqs)
+    for t, name in ((conv_state_in, "conv_state_in"), (conv_state_out, "conv_state_out")):
+        if t is not None:
+            _need(t, name, torch.float32, 3)
+    if initial_state is not None:
+        _need(initial_state, "initial_state", torch.float32, 4)
+    dev = xq.device
+    if o is None:
+        o = torch.empty((T, H, dv), dtype=torch.bfloat16, device=dev)
+    _need(o, "o", torch.bfloat16, 3)
+    if final_state is None and output_final_state:
+        final_state = torch.empty((N, H, dv, dk), dtype=torch.float32, device=dev)
+    if final_state is not None:
+        _need(final_state, "final_state", torch.float32, 4)
+    ws_bytes = gdr_prefill_workspace_size(N, T, H, dk, dv, gate, GDR_BF16)
+    if ws_bytes and workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    flags = (GDR_PROLOGUE_SILU if silu else 0) | (GDR_PROLOGUE_NORMALIZE_QK if normalize_qk else 0)
+    st = load_library().gdr_prefill_fused(
+        _ptr(xq), _ptr(xk), _ptr(xv), _ptr(wq), _ptr(wk), _ptr(wv), _ptr(xg), _ptr(gscale),
+        _ptr(xb), _ptr(conv_state_in), _ptr(conv_state_out), _ptr(initial_state),
+        _ptr(cu_seqlens), N, T, Hqk, H, dk, dv, gate, GDR_BF16, flags, _ptr(o),
+        _ptr(final_state), _ptr(workspace), workspace.numel() if workspace is not None else 0,
+        _stream_ptr(stream))
+    _check(st, "gdr_prefill_fused")
+    return o, final_state
 
 
 def gdr_backward_workspace_size(num_seqs, total_T, H, d_k, d_v) -> int:

@@ -50,6 +50,8 @@ varlen_gdn         8 packed sequences, 262144 tokens, H=16, d=128, bf16,
                    scalar gate c=0.1, h0=0
 gqa_prefill        1 sequence, 8192 tokens, 16 query/key heads shared by 48
                    value heads (3 each), d=128, bf16, scalar gate c=0.05
+prefill_fused_gdn  the prologue_gdn raw inputs through the prologue fused into
+                   the chunked prefill (o and the final state out)
 kda_prefill_small  kda_prefill at 2 x 2048 tokens (the same 64 chains and
                    plan at a sixteenth of the length; a profiler capture
                    holds a few hundred MB on the device instead of 7 GB)
@@ -363,7 +365,7 @@ def make_prologue_inputs(*, total_T: int, H: int, d_k: int, d_v: int | None = No
 
 WORKLOADS = ("tiny_gdn", "gdn_prefill", "kda_prefill", "decode_gdn",
              "decode_kda", "varlen_gdn", "gqa_prefill", "decode_spec_gdn", "prologue_gdn",
-             "backward_gdn", "kda_prefill_small")
+             "backward_gdn", "kda_prefill_small", "prefill_fused_gdn")
 
 SPEC_DRAFT = 4   # tokens verified per sequence per step in decode_spec_gdn
 
@@ -424,8 +426,9 @@ def make_grad_inputs(inp: Inputs, seed: int = 0, dsf_std: float = 1.0):
 
 
 def prologue_workload(name: str = "prologue_gdn", seed: int = 0) -> PrologueInputs:
-    """Raw prologue inputs at the gdn_prefill shape (module docstring table)."""
-    if name != "prologue_gdn":
+    """Raw prologue inputs at the gdn_prefill shape (module docstring table);
+    the fused prefill workload takes the same inputs."""
+    if name not in ("prologue_gdn", "prefill_fused_gdn"):
         raise KeyError(name)
     return make_prologue_inputs(total_T=8192, H=16, d_k=128, num_seqs=1, gate_mode=SCALAR,
                                 io_dtype=torch.bfloat16, c=0.05, tap_std=0.5, state_std=1.0,

@@ -360,6 +360,41 @@ GDR_API gdr_status_t gdr_prologue(const void *xq, const void *xk, const void *xv
                                   void *q, void *k, void *v, float *g, float *beta, void *stream);
 
 /*
+ * The prologue above fused into the chunked prefill: the raw projections go
+ * in, o and the final state come out, and q, k, v, g and beta never reach
+ * HBM.  The prefill's stage step applies the convolution (with the incoming
+ * convolution state before each sequence's first token), the optional SiLU,
+ * the q/k L2 norms and the gate and beta maps to each chunk while it stages
+ * the chunk's tiles, with the same arithmetic as gdr_prologue; the result is
+ * the recurrence of gdr_prefill_chunked_gqa applied to gdr_prologue's outputs
+ * (page "How the New Flash Models Work", section "Serving: prefill and
+ * decode are different problems": the convolution state and the recurrent
+ * state are what a decode continuing the sequence starts from).
+ *
+ * Arguments: those of gdr_prologue (raw inputs, taps, maps, convolution
+ * states, flags) followed by those of gdr_prefill_chunked_gqa's state and
+ * outputs: initial_state / final_state [num_seqs, H, d_v, d_k] fp32 or NULL
+ * (final_state may be initial_state itself), o [total_T, H, d_v] bf16, and
+ * the workspace of gdr_prefill_workspace_size.  Served for bf16 I/O with
+ * d_k = d_v = 128 on the chunk-parallel tensor-core plan only:
+ * GDR_ERR_UNSUPPORTED for other shapes or types (run gdr_prologue and then
+ * gdr_prefill_chunked_gqa there), GDR_ERR_WORKSPACE when the workspace is
+ * smaller than gdr_prefill_workspace_size reports.  No output may overlap an
+ * input or another output (GDR_ERR_INVALID_ARG).  Device-side timeouts are
+ * reported by gdr_prefill_check_workspace, as for gdr_prefill_chunked.
+ */
+GDR_API gdr_status_t gdr_prefill_fused(const void *xq, const void *xk, const void *xv,
+                                       const float *wq, const float *wk, const float *wv,
+                                       const float *xg, const float *gscale, const float *xb,
+                                       const float *conv_state_in, float *conv_state_out,
+                                       const float *initial_state, const int32_t *cu_seqlens,
+                                       int32_t num_seqs, int32_t total_T, int32_t H_qk,
+                                       int32_t H, int32_t d_k, int32_t d_v,
+                                       gdr_gate_mode_t gate_mode, gdr_dtype_t io_dtype,
+                                       uint32_t flags, void *o, float *final_state,
+                                       void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * Gradient of the recurrence (training).  The pages train these layers but
  * print no backward pass; this is the gradient of the rule at the top of this
  * header, for the loss

@@ -245,6 +245,52 @@ def test_prologue_empty_problem_is_a_no_op(lib):
                      g=None, xb=None, beta=None) == gdr.GDR_OK
 
 
+_FU_NAMES = ("xq", "xk", "xv", "wq", "wk", "wv", "xg", "gs", "xb", "sin", "sout", "h0", "cu",
+             "o", "fin", "ws")
+_FU = {n: _PRO_BASE + ((i + 40) << 30) for i, n in enumerate(_FU_NAMES)}
+
+
+def _fused(lib, **kw):
+    args = dict(_FU)
+    args.update(cu=None, sin=None, sout=None, h0=None, N=1, T=64, Hqk=2, H=2, dk=128, dv=128,
+                gate=0, io=1, flags=2, wsb=1 << 30)
+    args.update(kw)
+    P = lambda x: None if x is None else ctypes.c_void_p(x)
+    return lib.gdr_prefill_fused(*(P(args[n]) for n in _FU_NAMES[:13]), args["N"], args["T"],
+                                 args["Hqk"], args["H"], args["dk"], args["dv"], args["gate"],
+                                 args["io"], args["flags"], P(args["o"]), P(args["fin"]),
+                                 P(args["ws"]), args["wsb"], None)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(xq=None), dict(xv=None), dict(o=None), dict(wq=None), dict(gs=None), dict(xb=None),
+    dict(xg=None), dict(xq=_FU["xq"] + 2), dict(o=_FU["o"] + 8), dict(fin=_FU["fin"] + 4),
+    dict(h0=_FU["h0"] + 8), dict(cu=_FU["cu"] + 2), dict(wv=_FU["wv"] + 4),
+    dict(xg=_FU["xg"] + 4, gate=1), dict(sout=_FU["sout"] + 1),
+    dict(dk=48), dict(H=0), dict(Hqk=3), dict(N=0), dict(T=-1), dict(N=3, T=64), dict(gate=2),
+    dict(io=5), dict(flags=4),
+    # outputs overlapping inputs or each other
+    dict(o=_FU["xv"]), dict(o=_FU["xq"] + 64), dict(h0=_FU["h0"], fin=_FU["h0"] + 64),
+    dict(sin=_FU["sin"], sout=_FU["sin"]),
+    dict(sout=_FU["o"]), dict(fin=_FU["wq"]),
+])
+def test_fused_prefill_rejects_invalid_arguments(lib, kw):
+    assert _fused(lib, **kw) == gdr.GDR_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("kw", [dict(dk=64, dv=64), dict(io=0)])
+def test_fused_prefill_serves_only_the_tensor_core_shape(lib, kw):
+    # fp32 I/O or d != 128: run gdr_prologue and gdr_prefill_chunked_gqa instead
+    assert _fused(lib, **kw) == gdr.GDR_ERR_UNSUPPORTED
+
+
+def test_fused_prefill_final_state_may_be_the_initial_state(lib):
+    # aliasing passes validation; without a B200 the call then stops at the
+    # tensor-core check, before anything is launched
+    st = _fused(lib, h0=_FU["h0"], fin=_FU["h0"])
+    assert st != gdr.GDR_ERR_INVALID_ARG
+
+
 _BW_NAMES = ("q", "k", "v", "g", "beta", "h0", "cu", "do", "dsf", "gq", "gk", "gv", "gg", "gb",
              "gh0", "ws")   # gX: the gradient output for X
 _BW = {n: _PRO_BASE + ((i + 20) << 30) for i, n in enumerate(_BW_NAMES)}
@@ -292,6 +338,11 @@ def test_bindings_reject_host_tensors_before_any_call():
                          torch.zeros(8, 2), torch.ones(2), torch.zeros(8, 2))
     with pytest.raises(ValueError, match="CUDA"):
         gdr.gdr_backward(x, x, x, torch.zeros(8, 2), torch.zeros(8, 2), d_o=x)
+    xb = torch.zeros(8, 2, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        gdr.gdr_prefill_fused(xb, xb, xb, torch.zeros(256, 4), torch.zeros(256, 4),
+                              torch.zeros(256, 4), torch.zeros(8, 2), torch.ones(2),
+                              torch.zeros(8, 2))
     with pytest.raises(ValueError, match="CUDA"):
         gdr.gdr_decode_multi(torch.zeros(1, 2, 2, 16), torch.zeros(1, 2, 2, 16),
                              torch.zeros(1, 2, 2, 16), torch.zeros(1, 2, 2), torch.zeros(1, 2, 2),
