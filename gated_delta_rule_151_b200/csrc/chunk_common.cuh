@@ -224,5 +224,20 @@ bool make_map(CUtensorMap *map, const void *base, int total_T, int H) {
     return r == CUDA_SUCCESS;
 }
 
+// [total_T, H, 128] fp32 per-channel gates viewed as {128, H, total_T}; box
+// {32, 1, 64} without swizzle: 64 tokens x 32 channels as rows of 128 bytes.
+bool make_gate_map(CUtensorMap *map, const float *base, int total_T, int H) {
+    auto enc = get_encode();
+    if (enc == nullptr) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)total_T};
+    cuuint64_t strides[2] = {(cuuint64_t)D * 4, (cuuint64_t)H * D * 4};
+    cuuint32_t box[3] = {32, 1, 64};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float *>(base), dims,
+                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 }  // namespace
 }  // namespace gdr

@@ -536,7 +536,8 @@ __device__ __forceinline__ void fused_prologue_tiles(const PrologueIn &P, uint8_
 template <bool CHANNEL, bool FUSED>
 __global__ void __launch_bounds__(kPrepThreads, 2)
 prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-            const __grid_constant__ CUtensorMap tm_v, const float *__restrict__ g,
+            const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
+            const float *__restrict__ g,
             const float *__restrict__ beta, const int32_t *__restrict__ cu, int num_seqs,
             int total_T, int Hqk, int H, const ChunkMap map, uint8_t *__restrict__ recs,
             const PrologueIn pin, uint32_t *err) {
@@ -601,8 +602,15 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = m->tmem_base;
+    // channel gate: the chunk's gates [64 tokens][128 channels] fp32 land in
+    // RT and RX (free until the P1 operand pass) with the tiles
+    constexpr bool kGateTma = CHANNEL && !FUSED;
     if (!FUSED && tid == 0) {
-        mbar_arrive_expect_tx(&m->bar_tma, 6 * 8192);
+        mbar_arrive_expect_tx(&m->bar_tma, 6 * 8192 + (kGateTma ? 32768 : 0));
+        if (kGateTma) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) tma_load_3d(sm + PO_RT + j * 8192, &tm_g, &m->bar_tma, 32 * j, h, tok0);
+        }
         tma_load_3d(sm + PO_KQ + 0, &tm_k, &m->bar_tma, 0, hq, tok0);
         tma_load_3d(sm + PO_KQ + 16384, &tm_k, &m->bar_tma, 64, hq, tok0);
         tma_load_3d(sm + PO_KQ + 8192, &tm_q, &m->bar_tma, 0, hq, tok0);
@@ -650,18 +658,20 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             }
         }
     } else {
-        const float cg = FUSED ? pin.gscale[h] : 0.f;
+        if (FUSED) {
+            const float cg = pin.gscale[h];
 #pragma unroll
-        for (int k = 0; k < 32; ++k) {
-            const int i = hh * 32 + k;
-            const size_t gi = ((size_t)(tok0 + i) * H + h) * D + ch;
-            gr[k] = i < cl ? (FUSED ? log_gate_of(cg, pin.xg[gi]) : g[gi]) : 0.f;
+            for (int k = 0; k < 32; ++k) {
+                const int i = hh * 32 + k;
+                const size_t gi = ((size_t)(tok0 + i) * H + h) * D + ch;
+                gr[k] = i < cl ? log_gate_of(cg, pin.xg[gi]) : 0.f;
+            }
+            gr[0] = clamp_log_gate(gr[0]);
+#pragma unroll
+            for (int k = 1; k < 32; ++k) gr[k] = clamp_log_gate(gr[k]) + gr[k - 1];
+            if (hh == 0) m->u.c.T0[ch] = gr[31];
+            else m->u.c.T1[ch] = gr[31];
         }
-        gr[0] = clamp_log_gate(gr[0]);
-#pragma unroll
-        for (int k = 1; k < 32; ++k) gr[k] = clamp_log_gate(gr[k]) + gr[k - 1];
-        if (hh == 0) m->u.c.T0[ch] = gr[31];
-        else m->u.c.T1[ch] = gr[31];
         if (tid < C) {
             const size_t bi = (size_t)(tok0 + tid) * H + h;
             m->u.c.beta[tid] = tid < cl ? (FUSED ? beta_of(pin.xb[bi]) : beta[bi]) : 0.f;
@@ -681,6 +691,22 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 
         float GC = 0.f;
         float kmax = 0.f, qmax = 0.f;   // channel gate: this thread's largest |k| and |q|
+        if (kGateTma) {
+            // this thread's 32 gates from the staged rows (row = token, 128
+            // bytes per 32 channels), masked past the sequence's end
+            const float *gs = reinterpret_cast<const float *>(sm + PO_RT + (ch >> 5) * 8192) + (ch & 31);
+#pragma unroll
+            for (int k = 0; k < 32; ++k) {
+                const int i = hh * 32 + k;
+                gr[k] = i < cl ? gs[i * 32] : 0.f;
+            }
+            gr[0] = clamp_log_gate(gr[0]);
+#pragma unroll
+            for (int k = 1; k < 32; ++k) gr[k] = clamp_log_gate(gr[k]) + gr[k - 1];
+            if (hh == 0) m->u.c.T0[ch] = gr[31];
+            else m->u.c.T1[ch] = gr[31];
+            __syncthreads();   // T0, T1 for every thread; the staged gates are read
+        }
         if (CHANNEL) {
             // chunk-cumulative gate of this thread's tokens; reference R = G_31
             const float T0 = m->u.c.T0[ch], T1 = m->u.c.T1[ch];
@@ -1782,10 +1808,15 @@ cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, co
         k = pi.xk;
         v = pi.xv;
     }
-    CUtensorMap mq, mk, mv;
+    CUtensorMap mq, mk, mv, mg;
     if (!make_map(&mq, q, total_T, Hqk) || !make_map(&mk, k, total_T, Hqk) ||
         !make_map(&mv, v, total_T, H))
         return cudaErrorInvalidValue;
+    if (channel && !fused) {
+        if (!make_gate_map(&mg, g, total_T, H)) return cudaErrorInvalidValue;
+    } else {
+        mg = mq;   // not read
+    }
     auto prep = channel ? (fused ? prep_kernel<true, true> : prep_kernel<true, false>)
                         : (fused ? prep_kernel<false, true> : prep_kernel<false, false>);
     e = ensure_dynamic_smem(reinterpret_cast<const void *>(prep), (int)PREP_SMEM);
@@ -1805,7 +1836,7 @@ cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, co
         return cudaGetLastError();
     };
     auto run_prep = [&](const ChunkMap &map, unsigned gx, unsigned gy, cudaStream_t st) {
-        prep<<<dim3(gx, gy), kPrepThreads, PREP_SMEM, st>>>(mq, mk, mv, g, beta, cu, num_seqs, total_T,
+        prep<<<dim3(gx, gy), kPrepThreads, PREP_SMEM, st>>>(mq, mk, mv, mg, g, beta, cu, num_seqs, total_T,
                                                             Hqk, H, map, recs, pi, err);
         return cudaGetLastError();
     };
