@@ -261,7 +261,7 @@ def split_launches(inp):
     per window of chunks (a window holds at most 8 GiB of records at 98,848
     bytes per chunk and head), or, when one window holds every record and
     there are at most 64 (sequence, head) chains, per pipeline piece, or, with
-    at most 24 chains, one prep launch and the three launches of the
+    at most 49 chains, one prep launch and the three launches of the
     segmented scan."""
     chains = inp.num_seqs * inp.H
     # equal lengths go without cu_seqlens, so the library knows each
@@ -275,7 +275,7 @@ def split_launches(inp):
     if windows > 1 or chains > 64:
         return 1 + 2 * windows
     nseg = min(8, (148 // chains + 3) // 2)
-    if nseg >= 4 and max_chunks >= 2 * nseg:
+    if nseg >= 3 and max_chunks >= 2 * nseg:
         # few chains: the prep kernel over every chunk, then the segmented scan
         # (segments from zero and their transitions, composition, segments in
         # full from their incoming states)

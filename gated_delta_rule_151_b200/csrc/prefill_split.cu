@@ -1727,7 +1727,7 @@ bool make_split_plan(int num_seqs, int total_T, int H, SplitPlan &p, bool equal_
     // chains (2 nseg - 3) CTAs) fits the 148 SMs at once
     if (!p.by_window) {
         const int ns = std::min(kMaxSegments, (kSegCTAs / p.chains + 3) / 2);
-        if (ns >= 4 && p.max_chunks >= 2 * ns) {
+        if (ns >= 3 && p.max_chunks >= 2 * ns) {
             p.nseg = ns;
             p.pieces = 1;
         }

@@ -130,7 +130,7 @@ def _split_bytes(N, T, H, equal):
             pieces += 1
             size = (size * 13 + 9) // 10
         ns = min(8, (148 // (N * H) + 3) // 2)   # few chains: the segmented scan
-        if ns >= 4 and max_chunks >= 2 * ns:
+        if ns >= 3 and max_chunks >= 2 * ns:
             nseg, pieces = ns, 1
     if by_window:
         state = (windows - 1) * H * 65536

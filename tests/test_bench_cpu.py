@@ -44,9 +44,14 @@ def test_pipelined_plan_launch_accounting():
     kda = I.workload("kda_prefill")
     assert (8 << 30) // (32 * 98848) == 2715
     assert bench.split_launches(kda) == 1 + 2 * 10
-    # 48 chains at the gdn_prefill length: too many for segments, pieces of
-    # 12, 16, 21, 27, 35 and the last 17, each one prep and one chain launch
-    assert bench.split_launches(I.workload("gqa_prefill")) == 1 + 12
+    # 48 chains at the gdn_prefill length: three segments (48 x 3 = 144 CTAs
+    # in the first phase fit the 148 SMs), the same five launches
+    assert bench.split_launches(I.workload("gqa_prefill")) == 1 + 1 + 3
+    # 50 chains: three segments no longer fit, pieces of 12, 16, 21, 28, 37
+    # and the last 14, each one prep and one chain launch
+    wide = I.make_inputs(total_T=8192, H=50, d_k=16, num_seqs=1, gate_mode=I.SCALAR,
+                         io_dtype=torch.bfloat16, seed=0)
+    assert bench.split_launches(wide) == 1 + 12
     # varlen: 128 chains run by windows; packed lengths bound the chunks by
     # 262144 / 64 + 8 = 4104, within one window of 5431 global chunks of 16
     # heads
