@@ -324,7 +324,7 @@ constexpr uint32_t PO_RX = 81920;   // inverse scratch / channel P1 B operand / 
 constexpr uint32_t PO_P = 98304;    // P fp16 [i][j] (rows 64-127 of the M = 128 A operand whose
                                     //   rows 0-63 are the 8 KiB before it, never read back)
 constexpr uint32_t PO_MISC = 106496;
-constexpr uint32_t PREP_SMEM = PO_MISC + 2048;   // 108544: two CTAs per SM
+constexpr uint32_t PREP_SMEM = PO_MISC + 2560;   // 109056: two CTAs per SM
 constexpr uint32_t PT_W = 0, PREP_TMEM_COLS = 256;   // P1 accumulates at column 0
 constexpr uint32_t IDESC_P2 = make_idesc(1, 128, 64) | kIdescAMN;     // bf16, A MN-major
 constexpr uint32_t IDESC_NT = make_idesc(0, 128, 128) | kIdescAMN;    // fp16, A MN-major
@@ -342,12 +342,12 @@ struct PrepMisc {
             float beta[C], G[C], gam[C], kp[C], kh[C], ieg[C];
         } s;
         struct {
-            float beta[C], T0[D], T1[D];
+            float beta[C], T[4][D];    // chunk gate totals of each 16-token quarter
         } c;
     } u;                               // beta comes first in both layouts
     float red[3][8];                   // per-warp maxima for the image scales
 };
-static_assert(sizeof(PrepMisc) <= 2048, "prep misc area overflow");
+static_assert(sizeof(PrepMisc) <= 2560, "prep misc area overflow");
 static_assert(offsetof(PrepMisc, u) % 16 == 0, "prep misc arrays misaligned");
 
 // Scale exponents of two blocks from every thread's largest |value| of each
@@ -533,6 +533,21 @@ __device__ __forceinline__ void fused_prologue_tiles(const PrologueIn &P, uint8_
     }
 }
 
+// A bf16 pair (low half first) as two floats.
+__device__ __forceinline__ float2 bf2_to_f2(uint32_t v) {
+    return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&v));
+}
+
+// Clamped log-gates of 16 consecutive tokens of two channels -> their running
+// sums; the sums' last values (the quarter's totals) go to tot[0..1].
+__device__ __forceinline__ void gate_scan16(float2 (&gr)[16], float *tot) {
+    gr[0] = make_float2(clamp_log_gate(gr[0].x), clamp_log_gate(gr[0].y));
+#pragma unroll
+    for (int k = 1; k < 16; ++k)
+        gr[k] = make_float2(clamp_log_gate(gr[k].x) + gr[k - 1].x, clamp_log_gate(gr[k].y) + gr[k - 1].y);
+    *reinterpret_cast<float2 *>(tot) = gr[15];
+}
+
 template <bool CHANNEL, bool FUSED>
 __global__ void __launch_bounds__(kPrepThreads, 2)
 prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -621,8 +636,10 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 
     // ---- gates (overlap the tile loads); rows past the sequence end get
     //      beta = 0 and g = 0 ------------------------------------------------
-    const int ch = tid & 127, hh = tid >> 7;   // channel gate: channel, token half
-    float gr[32];
+    // channel gate: this thread's channel pair 2 cp, 2 cp + 1 and token quarter
+    // qq (tokens 16 qq .. 16 qq + 15); gr = their chunk-cumulative gates
+    const int cp = tid & 63, qq = tid >> 6, c0 = 2 * cp;
+    float2 gr[16];
     if (!CHANNEL) {
         if (tid < 32) {
             const int i0 = 2 * tid, i1 = 2 * tid + 1;
@@ -661,16 +678,16 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         if (FUSED) {
             const float cg = pin.gscale[h];
 #pragma unroll
-            for (int k = 0; k < 32; ++k) {
-                const int i = hh * 32 + k;
-                const size_t gi = ((size_t)(tok0 + i) * H + h) * D + ch;
-                gr[k] = i < cl ? log_gate_of(cg, pin.xg[gi]) : 0.f;
+            for (int k = 0; k < 16; ++k) {
+                const int i = qq * 16 + k;
+                float2 x = make_float2(0.f, 0.f);
+                if (i < cl) {
+                    x = *reinterpret_cast<const float2 *>(pin.xg + ((size_t)(tok0 + i) * H + h) * D + c0);
+                    x = make_float2(log_gate_of(cg, x.x), log_gate_of(cg, x.y));
+                }
+                gr[k] = x;
             }
-            gr[0] = clamp_log_gate(gr[0]);
-#pragma unroll
-            for (int k = 1; k < 32; ++k) gr[k] = clamp_log_gate(gr[k]) + gr[k - 1];
-            if (hh == 0) m->u.c.T0[ch] = gr[31];
-            else m->u.c.T1[ch] = gr[31];
+            gate_scan16(gr, m->u.c.T[qq] + c0);
         }
         if (tid < C) {
             const size_t bi = (size_t)(tok0 + tid) * H + h;
@@ -689,52 +706,58 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             break;
         }
 
-        float GC = 0.f;
         float kmax = 0.f, qmax = 0.f;   // channel gate: this thread's largest |k| and |q|
         if (kGateTma) {
-            // this thread's 32 gates from the staged rows (row = token, 128
+            // this thread's 2 x 16 gates from the staged rows (row = token, 128
             // bytes per 32 channels), masked past the sequence's end
-            const float *gs = reinterpret_cast<const float *>(sm + PO_RT + (ch >> 5) * 8192) + (ch & 31);
+            const float *gs = reinterpret_cast<const float *>(sm + PO_RT + (cp >> 4) * 8192) + (c0 & 31);
 #pragma unroll
-            for (int k = 0; k < 32; ++k) {
-                const int i = hh * 32 + k;
-                gr[k] = i < cl ? gs[i * 32] : 0.f;
+            for (int k = 0; k < 16; ++k) {
+                const int i = qq * 16 + k;
+                gr[k] = i < cl ? *reinterpret_cast<const float2 *>(gs + i * 32) : make_float2(0.f, 0.f);
             }
-            gr[0] = clamp_log_gate(gr[0]);
-#pragma unroll
-            for (int k = 1; k < 32; ++k) gr[k] = clamp_log_gate(gr[k]) + gr[k - 1];
-            if (hh == 0) m->u.c.T0[ch] = gr[31];
-            else m->u.c.T1[ch] = gr[31];
-            __syncthreads();   // T0, T1 for every thread; the staged gates are read
+            gate_scan16(gr, m->u.c.T[qq] + c0);
+            __syncthreads();   // every quarter's total; the staged gates are read
         }
+        float2 GC2 = make_float2(0.f, 0.f);
         if (CHANNEL) {
-            // chunk-cumulative gate of this thread's tokens; reference R = G_31
-            const float T0 = m->u.c.T0[ch], T1 = m->u.c.T1[ch];
-            if (hh == 1) {
+            // chunk-cumulative gates: the quarters before this one, then the
+            // thread's own; reference R = G at token 31 (the end of quarter 1)
+            float2 pre = make_float2(0.f, 0.f), R = make_float2(0.f, 0.f);
 #pragma unroll
-                for (int k = 0; k < 32; ++k) gr[k] += T0;
+            for (int q = 0; q < 4; ++q) {
+                const float2 t = *reinterpret_cast<const float2 *>(m->u.c.T[q] + c0);
+                if (q < qq) pre = make_float2(pre.x + t.x, pre.y + t.y);
+                if (q < 2) R = make_float2(R.x + t.x, R.y + t.y);
+                GC2 = make_float2(GC2.x + t.x, GC2.y + t.y);
             }
-            const float R = T0;
-            GC = T0 + T1;
-            if (hh == 0) *reinterpret_cast<float *>(rec + REC_GC + ch * 4) = __expf(GC);
+#pragma unroll
+            for (int k = 0; k < 16; ++k) gr[k] = make_float2(gr[k].x + pre.x, gr[k].y + pre.y);
+            if (qq == 0)
+                *reinterpret_cast<float2 *>(rec + REC_GC + c0 * 4) = make_float2(__expf(GC2.x), __expf(GC2.y));
             // fp16 P1 operands: rows [K e^{G-R}; Q e^{G-R}] (RA..RT), K e^{R-G} (RX)
             bool bad = false;
-            const uint32_t kcol = (ch >> 6) * 16384, bcol = (ch >> 6) * 8192;
-            const uint32_t cch = (ch & 63) >> 3, cel = (ch & 7) * 2;
+            const uint32_t kcol = (cp >> 5) * 16384, bcol = (cp >> 5) * 8192;
+            const uint32_t cch = (cp & 31) >> 2, cel = (cp & 3) * 4;
 #pragma unroll
-            for (int k = 0; k < 32; ++k) {
-                const int i = hh * 32 + k;
-                const uint32_t src = PO_KQ + kcol + sw128_offset(i, cch) + cel;
-                const float kv = smb16(sm, src), qv = smb16(sm, src + 8192);
-                kmax = fmaxf(kmax, fabsf(kv));
-                qmax = fmaxf(qmax, fabsf(qv));
-                const float up = __expf(gr[k] - R), dn = __expf(R - gr[k]);
-                const float a = kv * up, b = qv * up, e = kv * dn;
-                bad |= !(fabsf(a) < kF16Limit) || !(fabsf(b) < kF16Limit) ||
-                       !(fabsf(e) < kF16Limit);
-                smh16(sm, PO_RA + kcol + sw128_offset(i, cch) + cel, a);
-                smh16(sm, PO_RA + kcol + sw128_offset(64 + i, cch) + cel, b);
-                smh16(sm, PO_RX + bcol + sw128_offset(i, cch) + cel, e);
+            for (int k = 0; k < 16; ++k) {
+                const int i = qq * 16 + k;
+                const uint32_t so = sw128_offset(i, cch) + cel;
+                const float2 kv = bf2_to_f2(*reinterpret_cast<const uint32_t *>(sm + PO_KQ + kcol + so));
+                const float2 qv = bf2_to_f2(*reinterpret_cast<const uint32_t *>(sm + PO_KQ + kcol + 8192 + so));
+                kmax = fmaxf(kmax, fmaxf(fabsf(kv.x), fabsf(kv.y)));
+                qmax = fmaxf(qmax, fmaxf(fabsf(qv.x), fabsf(qv.y)));
+                const float2 up = make_float2(__expf(gr[k].x - R.x), __expf(gr[k].y - R.y));
+                const float2 dn = make_float2(__expf(R.x - gr[k].x), __expf(R.y - gr[k].y));
+                const float2 a = __fmul2_rn(kv, up), b = __fmul2_rn(qv, up), e = __fmul2_rn(kv, dn);
+                // every value checked on its own: a NaN fails the comparison
+                bad |= !(fabsf(a.x) < kF16Limit) || !(fabsf(a.y) < kF16Limit) ||
+                       !(fabsf(b.x) < kF16Limit) || !(fabsf(b.y) < kF16Limit) ||
+                       !(fabsf(e.x) < kF16Limit) || !(fabsf(e.y) < kF16Limit);
+                *reinterpret_cast<uint32_t *>(sm + PO_RA + kcol + so) = f2h2_bits(a.x, a.y);
+                *reinterpret_cast<uint32_t *>(sm + PO_RA + kcol + sw128_offset(64 + i, cch) + cel) =
+                    f2h2_bits(b.x, b.y);
+                *reinterpret_cast<uint32_t *>(sm + PO_RX + bcol + so) = f2h2_bits(e.x, e.y);
             }
             if (bad) m->slow = 1;
             fence_proxy_async();
@@ -777,9 +800,9 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         if (CHANNEL) {
             float dk = -3.0e38f, dq = -3.0e38f;
 #pragma unroll
-            for (int k = 0; k < 32; ++k) {
-                dk = fmaxf(dk, GC - gr[k]);
-                dq = fmaxf(dq, gr[k]);
+            for (int k = 0; k < 16; ++k) {
+                dk = fmaxf(dk, fmaxf(GC2.x - gr[k].x, GC2.y - gr[k].y));
+                dq = fmaxf(dq, fmaxf(gr[k].x, gr[k].y));
             }
             kbnd = kmax * __expf(dk);
             qbnd = qmax * __expf(dq);
@@ -872,7 +895,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             Tf = reinterpret_cast<float *>(sm + PO_RT);
             Xs = reinterpret_cast<float *>(sm + PO_RA);
 #pragma unroll
-            for (int k = 0; k < 32; ++k) Gs[(hh * 32 + k) * D + ch] = gr[k];
+            for (int k = 0; k < 16; ++k) *reinterpret_cast<float2 *>(Gs + (qq * 16 + k) * D + c0) = gr[k];
             __syncthreads();
             // pair pr = i (i + 1) / 2 + j (j <= i); each thread keeps its P values
             // until the block's scale is known
@@ -990,21 +1013,26 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             }
         } else {
             const float fk = exp2i(sK), fq = exp2i(sQ);
-            const uint32_t kcol = (ch >> 6) * 16384, tcol = (ch >> 6) * 8192;
-            const uint32_t cch = (ch & 63) >> 3, cel = (ch & 7) * 2;
+            const uint32_t kcol = (cp >> 5) * 16384, tcol = (cp >> 5) * 8192;
+            const uint32_t cch = (cp & 31) >> 2, cel = (cp & 3) * 4;
 #pragma unroll
-            for (int k = 0; k < 32; ++k) {
-                const int i = hh * 32 + k;
-                const uint32_t src = PO_KQ + kcol + sw128_offset(i, cch) + cel;
-                const uint32_t dst = tcol + sw128_offset(i, cch) + cel;
-                const float kv = smb16(sm, src), qv = smb16(sm, src + 8192);
-                const float eg = __expf(gr[k]);
-                smh16(sm, PO_RT + dst, kv * __expf(GC - gr[k]) * fk);
-                const float kp = kv * eg;
-                const uint16_t khi = bf16_bits(kp);
-                smu16(sm, src, khi);
-                smu16(sm, PO_RX + dst, bf16_bits(kp - __uint_as_float((uint32_t)khi << 16)));
-                smh16(sm, src + 8192, qv * eg * fq);
+            for (int k = 0; k < 16; ++k) {
+                const int i = qq * 16 + k;
+                const uint32_t so = sw128_offset(i, cch) + cel;
+                const uint32_t src = PO_KQ + kcol + so, dst = tcol + so;
+                const float2 kv = bf2_to_f2(*reinterpret_cast<const uint32_t *>(sm + src));
+                const float2 qv = bf2_to_f2(*reinterpret_cast<const uint32_t *>(sm + src + 8192));
+                const float2 eg = make_float2(__expf(gr[k].x), __expf(gr[k].y));
+                const float2 kh = make_float2(__expf(GC2.x - gr[k].x) * fk, __expf(GC2.y - gr[k].y) * fk);
+                const float2 khat = __fmul2_rn(kv, kh);
+                *reinterpret_cast<uint32_t *>(sm + PO_RT + dst) = f2h2_bits(khat.x, khat.y);
+                const float2 kp = __fmul2_rn(kv, eg);
+                uint32_t khi, klo;
+                bf2_hilo(kp.x, kp.y, khi, klo);
+                *reinterpret_cast<uint32_t *>(sm + src) = khi;
+                *reinterpret_cast<uint32_t *>(sm + PO_RX + dst) = klo;
+                const float2 qt = __fmul2_rn(__fmul2_rn(qv, eg), make_float2(fq, fq));
+                *reinterpret_cast<uint32_t *>(sm + src + 8192) = f2h2_bits(qt.x, qt.y);
             }
         }
         fence_proxy_async();
