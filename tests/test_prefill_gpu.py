@@ -353,3 +353,24 @@ def test_segmented_scan(mode, case):
     o, fin = gpu_prefill(inp, use_cu=cu is not None)
     o_ref, fin_ref = oracle_prefill(inp)
     check(inp, o, fin, o_ref, fin_ref, f"segments {case} {mode}")
+
+
+@pytest.mark.parametrize("mode", [I.SCALAR, I.CHANNEL])
+def test_three_segments(mode):
+    """40 chains (2 sequences x 20 heads): four segments no longer fit the
+    SMs in the first phase, three do (40 x 3 = 120 CTAs): segment 0 from the
+    initial state, the middle segment from zero and from the identity, one
+    composition step, then the middle and last segments from their incoming
+    states.  A ragged tail and unequal lengths put the segment boundaries at
+    different chunks for the two sequences."""
+    inp = I.make_inputs(total_T=1500, H=20, d_k=128, gate_mode=mode, io_dtype=torch.bfloat16,
+                        cu_seqlens=[0, 1100, 1500], c=0.1, h0_std=0.05, seed=83)
+    nb = gdr.gdr_prefill_workspace_size(2, 1500, 20, 128, 128,
+                                        gdr.GDR_GATE_SCALAR if mode == I.SCALAR else gdr.GDR_GATE_CHANNEL,
+                                        gdr.GDR_BF16)
+    assert gdr.gdr_prefill_plan(2, 1500, 20, 128, 128,
+                                gdr.GDR_GATE_SCALAR if mode == I.SCALAR else gdr.GDR_GATE_CHANNEL,
+                                gdr.GDR_BF16, nb) == gdr.GDR_PATH_TCGEN05_SPLIT
+    o, fin = gpu_prefill(inp)
+    o_ref, fin_ref = oracle_prefill(inp)
+    check(inp, o, fin, o_ref, fin_ref, f"three segments {mode}")
