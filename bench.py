@@ -583,7 +583,8 @@ class BackwardCase:
     gdr_backward call per step (upstream gradients dO and dS_final drawn by
     the input module)."""
     kind = "backward"
-    kernel_label = "backward (forward sweep with a checkpoint every 16 tokens, reverse sweep)"
+    kernel_label = ("backward in chunked form: chunk prep, forward and reverse state chains, "
+                    "chunk-local gradients")
 
     def __init__(self, name, device, seed):
         self.name = name
@@ -607,7 +608,7 @@ class BackwardCase:
                       + T * (2 * Hqk * dk + H * dv) * 4 + state)
         self.flops = 0
         self.tokens = T
-        self.launches = 1
+        self.launches = 5   # chunk numbering, prep, forward chain, reverse chain, local gradients
         self.path = None
         self.out = None
 

@@ -1,0 +1,720 @@
+// Gradient of the recurrence in chunked form (scalar gate, d_k = d_v = 128):
+// the chunk algebra of the prefill (page "How the New Flash Models Work:
+// Inside GLM-5.3-Flash and Qwen3.8-Flash-Next", section "Linear attention: a
+// fixed-size memory in place of the cache", rearranged per chunk of C = 64
+// tokens) run backwards.  Per chunk, with S the state entering it, G the
+// chunk-cumulative log-gate, gamma = e^G and R_ij = e^{G_i - G_j}:
+//
+//   A = strictly-lower(diag(beta) (K K^T) o R),  T = (I + A)^-1
+//   W = T diag(beta gamma) K,  U~ = T diag(beta) V,  U = U~ - W S^T
+//   P = causal((Q K^T) o R),  O = diag(gamma) Q S^T + P U
+//   S' = e^{G_C} S + U^T K^,   K^_j = k_j e^{G_C - G_j}
+//
+// With L' the adjoint of S' (dS_final after a sequence's last chunk), the
+// adjoint of the state entering the chunk is
+//
+//   dU = K^ L'^T + P^T dO,   L = e^{G_C} L' + dO^T diag(gamma) Q - dU^T W
+//
+// and the chunk-local gradients follow from S, L', dO and the chunk's own
+// quantities: dK^ = U L', dW = -dU S, dP = causal(dO U^T), d(gamma Q) = dO S,
+// dT = dU (beta V)^T + dW (beta gamma K)^T, dA = -T^T dT T^T (strictly
+// lower), and from these dq, dk, dv, dbeta and the adjoints of G, whose
+// reverse cumulative sum within the chunk is dg.  Four launches:
+//
+//   prep    one CTA per (chunk, head): A, T, W, U~, P, G, beta (fp32).
+//   forward one CTA per (sequence, head, 16 state rows): the state entering
+//           every chunk and U, chunk after chunk.
+//   reverse the same CTAs, chunks last to first: L' of every chunk and dU;
+//           the adjoint of the initial state at the end.
+//   local   one CTA per (chunk, head): every gradient of the chunk's tokens.
+//
+// Everything is fp32 on CUDA cores: a register-tiled product over padded
+// shared-memory operands (rows of 129 or 65 floats, so rows and columns are
+// both read without bank conflicts).  The chunk records live in the
+// workspace: 311,808 bytes per (chunk, head).
+#include <cuda_bf16.h>
+
+#include <algorithm>
+#include <cstddef>
+
+#include "common.cuh"
+#include "internal.h"
+#include "chunk_common.cuh"
+
+namespace gdr {
+namespace {
+
+// per (chunk, head) record of floats
+constexpr size_t R_W = 0;                       // W [64][128]
+constexpr size_t R_UT = R_W + C * D;            // U~ [64][128]
+constexpr size_t R_P = R_UT + C * D;            // P [64][64], causal
+constexpr size_t R_T = R_P + C * C;             // T [64][64], lower with the unit diagonal
+constexpr size_t R_AR = R_T + C * C;            // (K K^T) o R [64][64], strictly lower
+constexpr size_t R_G = R_AR + C * C;            // G [64] (the chunk's cumulative log-gate)
+constexpr size_t R_B = R_G + C;                 // beta [64] (0 past the sequence's end)
+constexpr size_t R_U = R_B + C;                 // U [64][128]
+constexpr size_t R_DU = R_U + C * D;            // dU [64][128]
+constexpr size_t R_S = R_DU + C * D;            // state entering the chunk [128][128]
+constexpr size_t R_L = R_S + D * D;             // adjoint of the state leaving it [128][128]
+constexpr size_t R_FLOATS = R_L + D * D;        // 77,952 floats
+constexpr size_t kBaseBytes = 256;              // sequence chunk offsets precede the records
+
+constexpr int LW = D + 1;    // padded row of 128 floats
+constexpr int LN = C + 1;    // padded row of 64 floats
+constexpr int kRowBlock = 16;                   // state rows per forward / reverse CTA
+constexpr int kChainThreadsB = 128;
+constexpr int kLocalThreads = 256;
+
+__device__ __forceinline__ float ldio(const float *p) { return *p; }
+__device__ __forceinline__ float ldio(const __nv_bfloat16 *p) { return __bfloat162float(*p); }
+
+// The product tile of one thread: out(m, n) = sum_k a(m, k) b(k, n) for
+// rows m = gr + GR r and columns n = gc + GC c, (gr, gc) = (tid / GC, tid % GC),
+// GC = min(N, 16), GR = NT / GC; epi(m, n, value) takes each result.
+template <int M, int N, int NT, class AF, class BF, class EPI>
+__device__ __forceinline__ void gemm(int K, AF a, BF b, EPI epi) {
+    constexpr int GC = N < 16 ? N : 16;
+    constexpr int GR = NT / GC;
+    constexpr int TM = M / GR, TN = N / GC;
+    static_assert(GR * GC == NT && TM * GR == M && TN * GC == N, "product tiling");
+    const int tid = threadIdx.x, gr = tid / GC, gc = tid % GC;
+    float acc[TM][TN];
+#pragma unroll
+    for (int r = 0; r < TM; ++r)
+#pragma unroll
+        for (int c = 0; c < TN; ++c) acc[r][c] = 0.f;
+#pragma unroll 4
+    for (int k = 0; k < K; ++k) {
+        float av[TM], bv[TN];
+#pragma unroll
+        for (int r = 0; r < TM; ++r) av[r] = a(gr + GR * r, k);
+#pragma unroll
+        for (int c = 0; c < TN; ++c) bv[c] = b(k, gc + GC * c);
+#pragma unroll
+        for (int r = 0; r < TM; ++r)
+#pragma unroll
+            for (int c = 0; c < TN; ++c) acc[r][c] = fmaf(av[r], bv[c], acc[r][c]);
+    }
+#pragma unroll
+    for (int r = 0; r < TM; ++r)
+#pragma unroll
+        for (int c = 0; c < TN; ++c) epi(gr + GR * r, gc + GC * c, acc[r][c]);
+}
+
+// base[n] = first global chunk of sequence n (exclusive prefix sum of the
+// sequences' chunk counts); base[num_seqs] = all chunks.
+__global__ void __launch_bounds__(1024)
+bwd_chunk_base_kernel(const int32_t *__restrict__ cu, int num_seqs, int total_T, int32_t *base) {
+    __shared__ int wsum[32];
+    __shared__ int carry;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (tid == 0) carry = 0;
+    __syncthreads();
+    for (int start = 0; start < num_seqs; start += 1024) {
+        const int n = start + tid;
+        int v = 0;
+        if (n < num_seqs) {
+            int t0, len;
+            sequence_range(cu, n, num_seqs, total_T, t0, len);
+            v = (len + C - 1) / C;
+        }
+        int x = v;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, off);
+            if (lane >= off) x += y;
+        }
+        if (lane == 31) wsum[warp] = x;
+        __syncthreads();
+        if (warp == 0) {
+            int w = wsum[lane];
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, w, off);
+                if (lane >= off) w += y;
+            }
+            wsum[lane] = w;
+        }
+        __syncthreads();
+        const int incl = x + (warp > 0 ? wsum[warp - 1] : 0) + carry;
+        if (n < num_seqs) base[n] = incl - v;
+        __syncthreads();
+        if (tid == 1023) carry = incl;
+        __syncthreads();
+    }
+    if (tid == 0) base[num_seqs] = carry;
+}
+
+// (sequence, local chunk) of global chunk gc: base[n] <= gc < base[n + 1].
+__device__ __forceinline__ bool chunk_of(const int32_t *base, int num_seqs, int gc, int &n, int &c) {
+    if (gc >= base[num_seqs]) return false;
+    int lo = 0, hi = num_seqs;
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (base[mid] <= gc) lo = mid;
+        else hi = mid;
+    }
+    n = lo;
+    c = gc - base[n];
+    return true;
+}
+
+// ---------------------------------------------------------------- prep ----
+// One CTA per (global chunk, value head): G, beta, A (via the strictly
+// lower (K K^T) o R), T = (I + A)^-1, W, U~ and P, written to the record.
+constexpr int kPrepB = 256;
+constexpr uint32_t PB_K = 0;                        // K [64][129] fp32 (then beta gamma K)
+constexpr uint32_t PB_Q = PB_K + C * LW;            // Q [64][129]
+constexpr uint32_t PB_V = PB_Q + C * LW;            // V [64][129] (then beta V)
+constexpr uint32_t PB_A = PB_V + C * LW;            // A, swizzled 64 x 64 (the inverse's layout)
+constexpr uint32_t PB_T = PB_A + C * C;             // T, swizzled 64 x 64
+constexpr uint32_t PB_X = PB_T + C * C;             // the inverse's 1024-float scratch
+constexpr uint32_t PB_TP = PB_X + 1024;             // T [64][65], zero above the diagonal
+constexpr uint32_t PB_G = PB_TP + C * LN;           // G [64], gamma [64], beta [64]
+constexpr uint32_t PB_FLOATS = PB_G + 3 * C;
+constexpr uint32_t PB_SMEM = PB_FLOATS * sizeof(float);
+
+template <typename IoT>
+__global__ void __launch_bounds__(kPrepB, 1)
+bwd_prep_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT *__restrict__ v,
+                const float *__restrict__ g, const float *__restrict__ beta,
+                const int32_t *__restrict__ cu, int num_seqs, int total_T, int Hqk, int H,
+                const int32_t *__restrict__ base, float *__restrict__ recs) {
+    extern __shared__ __align__(16) float fs[];
+    int n, c;
+    const int gc = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
+    if (!chunk_of(base, num_seqs, gc, n, c)) return;
+    int t0, len;
+    sequence_range(cu, n, num_seqs, total_T, t0, len);
+    const int tok0 = t0 + c * C, cl = min(C, len - c * C), hq = h / (H / Hqk);
+    float *rec = recs + ((size_t)gc * H + h) * R_FLOATS;
+    float *Ks = fs + PB_K, *Qs = fs + PB_Q, *Vs = fs + PB_V, *Tp = fs + PB_TP;
+    float *Gs = fs + PB_G, *gam = Gs + C, *Bs = gam + C;
+    for (int e = tid; e < C * D; e += kPrepB) {
+        const int i = e >> 7, d = e & 127;
+        float kv = 0.f, qv = 0.f, vv = 0.f;
+        if (i < cl) {
+            const size_t rq = ((size_t)(tok0 + i) * Hqk + hq) * D + d;
+            kv = ldio(k + rq);
+            qv = ldio(q + rq);
+            vv = ldio(v + ((size_t)(tok0 + i) * H + h) * D + d);
+        }
+        Ks[i * LW + d] = kv;
+        Qs[i * LW + d] = qv;
+        Vs[i * LW + d] = vv;
+    }
+    if (tid < 32) {   // gates of tokens 2 tid, 2 tid + 1: clamped, cumulated, 0 past the end
+        const int i0 = 2 * tid, i1 = i0 + 1;
+        const float g0 = i0 < cl ? clamp_log_gate(g[(size_t)(tok0 + i0) * H + h]) : 0.f;
+        const float g1 = i1 < cl ? clamp_log_gate(g[(size_t)(tok0 + i1) * H + h]) : 0.f;
+        float incl = g0 + g1;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const float y = __shfl_up_sync(0xffffffffu, incl, off);
+            if (tid >= off) incl += y;
+        }
+        Gs[i0] = incl - g1;
+        Gs[i1] = incl;
+        gam[i0] = __expf(incl - g1);
+        gam[i1] = __expf(incl);
+        Bs[i0] = i0 < cl ? beta[(size_t)(tok0 + i0) * H + h] : 0.f;
+        Bs[i1] = i1 < cl ? beta[(size_t)(tok0 + i1) * H + h] : 0.f;
+    }
+    __syncthreads();
+    // (K K^T) o R (strictly lower) -> record and A = diag(beta) of it; P -> record
+    float *Af = fs + PB_A;
+    gemm<C, C, kPrepB>(D, [&](int i, int d) { return Ks[i * LW + d]; },
+                       [&](int d, int j) { return Ks[j * LW + d]; },
+                       [&](int i, int j, float x) {
+                           const float ar = j < i ? x * __expf(Gs[i] - Gs[j]) : 0.f;
+                           rec[R_AR + i * C + j] = ar;
+                           Af[ax(i, j)] = Bs[i] * ar;
+                       });
+    gemm<C, C, kPrepB>(D, [&](int i, int d) { return Qs[i * LW + d]; },
+                       [&](int d, int j) { return Ks[j * LW + d]; },
+                       [&](int i, int j, float x) {
+                           rec[R_P + i * C + j] = j <= i ? x * __expf(Gs[i] - Gs[j]) : 0.f;
+                       });
+    __syncthreads();
+    unit_lower_inverse_f32(Af, fs + PB_T, fs + PB_X, tid);   // ends synchronised
+    for (int e = tid; e < C * C; e += kPrepB) {
+        const int i = e >> 6, j = e & 63;
+        const float t = j <= i ? (fs + PB_T)[ax(i, j)] : 0.f;
+        Tp[i * LN + j] = t;
+        rec[R_T + e] = t;
+    }
+    // the scaled operands of W and U~ in place
+    for (int e = tid; e < C * D; e += kPrepB) {
+        const int i = e >> 7, d = e & 127;
+        Ks[i * LW + d] *= Bs[i] * gam[i];
+        Vs[i * LW + d] *= Bs[i];
+    }
+    if (tid < C) {
+        rec[R_G + tid] = Gs[tid];
+        rec[R_B + tid] = Bs[tid];
+    }
+    __syncthreads();
+    gemm<C, D, kPrepB>(C, [&](int i, int j) { return Tp[i * LN + j]; },
+                       [&](int j, int d) { return Ks[j * LW + d]; },
+                       [&](int i, int d, float x) { rec[R_W + i * D + d] = x; });
+    gemm<C, D, kPrepB>(C, [&](int i, int j) { return Tp[i * LN + j]; },
+                       [&](int j, int d) { return Vs[j * LW + d]; },
+                       [&](int i, int d, float x) { rec[R_UT + i * D + d] = x; });
+}
+
+// ------------------------------------------------------ forward / reverse ----
+// One CTA per (sequence, value head, block of 16 state rows); the rows of
+// the state and of its adjoint are independent, so the CTAs of a chain share
+// nothing.  Shared memory (floats): the rows [16][129], two [64][129]
+// operands, one [64][65] operand and [64][17] row-block columns.
+constexpr uint32_t CB_ROWS = 0;                          // S or L rows [16][129]
+constexpr uint32_t CB_M1 = CB_ROWS + kRowBlock * LW;      // [64][129]
+constexpr uint32_t CB_M2 = CB_M1 + C * LW;                // [64][129]
+constexpr uint32_t CB_M3 = CB_M2 + C * LW;                // [64][129]
+constexpr uint32_t CB_P = CB_M3 + C * LW;                 // [64][65]
+constexpr uint32_t CB_C1 = CB_P + C * LN;                 // [64][17]
+constexpr uint32_t CB_C2 = CB_C1 + C * (kRowBlock + 1);   // [64][17]
+constexpr uint32_t CB_G = CB_C2 + C * (kRowBlock + 1);    // G [64]
+constexpr uint32_t CB_FLOATS = CB_G + C;
+constexpr uint32_t CB_SMEM = CB_FLOATS * sizeof(float);
+
+// The chunk's K^ rows k_j e^{G_C - G_j} (0 past the sequence's end) into dst
+// [64][129], and, when Qt is given, gamma_i q_i into Qt; G from the record.
+template <typename IoT>
+__device__ __forceinline__ void load_khat(const IoT *k, const IoT *q, const float *rec, float *Gs,
+                                          float *dst, float *Qt, int tok0, int cl, int Hqk, int hq) {
+    for (int e = threadIdx.x; e < C * D; e += blockDim.x) {
+        const int i = e >> 7, d = e & 127;
+        float kv = 0.f, qv = 0.f;
+        if (i < cl) {
+            const size_t r = ((size_t)(tok0 + i) * Hqk + hq) * D + d;
+            kv = ldio(k + r);
+            if (Qt != nullptr) qv = ldio(q + r);
+        }
+        const float Gi = rec[R_G + i], GC = rec[R_G + C - 1];
+        dst[i * LW + d] = kv * __expf(GC - Gi);
+        if (Qt != nullptr) Qt[i * LW + d] = qv * __expf(Gi);
+    }
+    if (threadIdx.x < C) Gs[threadIdx.x] = rec[R_G + threadIdx.x];
+}
+
+template <typename IoT>
+__global__ void __launch_bounds__(kChainThreadsB, 1)
+bwd_forward_kernel(const IoT *__restrict__ k, const float *__restrict__ h0,
+                   const int32_t *__restrict__ cu, int num_seqs, int total_T, int Hqk, int H,
+                   const int32_t *__restrict__ base, long long slots, float *__restrict__ recs) {
+    extern __shared__ __align__(16) float fs[];
+    const int chain = blockIdx.x, h = chain % H, n = chain / H, r0 = blockIdx.y * kRowBlock;
+    const int tid = threadIdx.x, hq = h / (H / Hqk);
+    int t0, len;
+    sequence_range(cu, n, num_seqs, total_T, t0, len);
+    const int b0 = base[n];
+    // a malformed cu_seqlens can claim more chunks than the records hold
+    const int nch = (int)min((long long)(len + C - 1) / C, max(slots - b0, 0ll));
+    float *Sr = fs + CB_ROWS, *Ws = fs + CB_M1, *Kh = fs + CB_M2, *Us = fs + CB_C1, *Gs = fs + CB_G;
+    for (int e = tid; e < kRowBlock * D; e += kChainThreadsB) {
+        const int r = e >> 7, d = e & 127;
+        Sr[r * LW + d] = h0 != nullptr ? h0[((size_t)chain * D + r0 + r) * D + d] : 0.f;
+    }
+    for (int c = 0; c < nch; ++c) {
+        float *rec = recs + ((size_t)(b0 + c) * H + h) * R_FLOATS;
+        const int tok0 = t0 + c * C, cl = min(C, len - c * C);
+        __syncthreads();   // the rows of the last chunk's update are in place
+        for (int e = tid; e < kRowBlock * D; e += kChainThreadsB) {
+            const int r = e >> 7, d = e & 127;
+            rec[R_S + (size_t)(r0 + r) * D + d] = Sr[r * LW + d];
+        }
+        for (int e = tid; e < C * D; e += kChainThreadsB) Ws[(e >> 7) * LW + (e & 127)] = rec[R_W + e];
+        load_khat<IoT>(k, static_cast<const IoT *>(nullptr), rec, Gs, Kh, nullptr, tok0, cl, Hqk, hq);
+        __syncthreads();
+        // U[j][r0 + r] = U~[j][r0 + r] - sum_d W[j][d] S[r0 + r][d]
+        gemm<C, kRowBlock, kChainThreadsB>(D, [&](int j, int d) { return Ws[j * LW + d]; },
+                                           [&](int d, int r) { return Sr[r * LW + d]; },
+                                           [&](int j, int r, float x) {
+                                               const float u = rec[R_UT + j * D + r0 + r] - x;
+                                               Us[j * (kRowBlock + 1) + r] = u;
+                                               rec[R_U + j * D + r0 + r] = u;
+                                           });
+        __syncthreads();
+        // S[r][d] = e^{G_C} S[r][d] + sum_j U[j][r] K^[j][d]
+        const float gC = __expf(Gs[C - 1]);
+        gemm<kRowBlock, D, kChainThreadsB>(C, [&](int r, int j) { return Us[j * (kRowBlock + 1) + r]; },
+                                           [&](int j, int d) { return Kh[j * LW + d]; },
+                                           [&](int r, int d, float x) { Sr[r * LW + d] = fmaf(gC, Sr[r * LW + d], x); });
+    }
+}
+
+template <typename IoT>
+__global__ void __launch_bounds__(kChainThreadsB, 1)
+bwd_reverse_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT *__restrict__ dO,
+                   const float *__restrict__ dSf, float *__restrict__ dh0,
+                   const int32_t *__restrict__ cu, int num_seqs, int total_T, int Hqk, int H,
+                   const int32_t *__restrict__ base, long long slots, float *__restrict__ recs) {
+    extern __shared__ __align__(16) float fs[];
+    const int chain = blockIdx.x, h = chain % H, n = chain / H, r0 = blockIdx.y * kRowBlock;
+    const int tid = threadIdx.x, hq = h / (H / Hqk);
+    int t0, len;
+    sequence_range(cu, n, num_seqs, total_T, t0, len);
+    const int b0 = base[n];
+    const int nch = (int)min((long long)(len + C - 1) / C, max(slots - b0, 0ll));
+    float *Lr = fs + CB_ROWS, *Ws = fs + CB_M1, *Kh = fs + CB_M2, *Qt = fs + CB_M3, *Ps = fs + CB_P;
+    float *dOr = fs + CB_C1, *dUr = fs + CB_C2, *Gs = fs + CB_G;
+    for (int e = tid; e < kRowBlock * D; e += kChainThreadsB) {
+        const int r = e >> 7, d = e & 127;
+        Lr[r * LW + d] = dSf != nullptr ? dSf[((size_t)chain * D + r0 + r) * D + d] : 0.f;
+    }
+    for (int c = nch - 1; c >= 0; --c) {
+        float *rec = recs + ((size_t)(b0 + c) * H + h) * R_FLOATS;
+        const int tok0 = t0 + c * C, cl = min(C, len - c * C);
+        __syncthreads();
+        for (int e = tid; e < kRowBlock * D; e += kChainThreadsB) {
+            const int r = e >> 7, d = e & 127;
+            rec[R_L + (size_t)(r0 + r) * D + d] = Lr[r * LW + d];
+        }
+        for (int e = tid; e < C * D; e += kChainThreadsB) Ws[(e >> 7) * LW + (e & 127)] = rec[R_W + e];
+        for (int e = tid; e < C * C; e += kChainThreadsB) Ps[(e >> 6) * LN + (e & 63)] = rec[R_P + e];
+        for (int e = tid; e < C * kRowBlock; e += kChainThreadsB) {
+            const int i = e / kRowBlock, r = e % kRowBlock;
+            dOr[i * (kRowBlock + 1) + r] =
+                i < cl ? ldio(dO + ((size_t)(tok0 + i) * H + h) * D + r0 + r) : 0.f;
+        }
+        load_khat<IoT>(k, q, rec, Gs, Kh, Qt, tok0, cl, Hqk, hq);
+        __syncthreads();
+        // dU[j][r] = sum_d K^[j][d] L[r][d] + sum_i P[i][j] dO[i][r]
+        gemm<C, kRowBlock, kChainThreadsB>(D, [&](int j, int d) { return Kh[j * LW + d]; },
+                                           [&](int d, int r) { return Lr[r * LW + d]; },
+                                           [&](int j, int r, float x) { dUr[j * (kRowBlock + 1) + r] = x; });
+        gemm<C, kRowBlock, kChainThreadsB>(C, [&](int j, int i) { return Ps[i * LN + j]; },
+                                           [&](int i, int r) { return dOr[i * (kRowBlock + 1) + r]; },
+                                           [&](int j, int r, float x) {
+                                               const float du = dUr[j * (kRowBlock + 1) + r] + x;
+                                               dUr[j * (kRowBlock + 1) + r] = du;
+                                               rec[R_DU + j * D + r0 + r] = du;
+                                           });
+        __syncthreads();
+        // L[r][d] = e^{G_C} L[r][d] + sum_i dO[i][r] gamma_i q_i[d] - sum_j dU[j][r] W[j][d]
+        const float gC = __expf(Gs[C - 1]);
+        gemm<kRowBlock, D, kChainThreadsB>(C, [&](int r, int i) { return dOr[i * (kRowBlock + 1) + r]; },
+                                           [&](int i, int d) { return Qt[i * LW + d]; },
+                                           [&](int r, int d, float x) { Lr[r * LW + d] = fmaf(gC, Lr[r * LW + d], x); });
+        gemm<kRowBlock, D, kChainThreadsB>(C, [&](int r, int j) { return dUr[j * (kRowBlock + 1) + r]; },
+                                           [&](int j, int d) { return Ws[j * LW + d]; },
+                                           [&](int r, int d, float x) { Lr[r * LW + d] -= x; });
+    }
+    __syncthreads();
+    if (dh0 != nullptr) {
+        for (int e = tid; e < kRowBlock * D; e += kChainThreadsB) {
+            const int r = e >> 7, d = e & 127;
+            dh0[((size_t)chain * D + r0 + r) * D + d] = Lr[r * LW + d];
+        }
+    }
+}
+
+// --------------------------------------------------------------- local ----
+// One CTA per (global chunk, value head): every gradient of the chunk's
+// tokens.  Shared memory (floats) is reused phase by phase:
+//   RA [128][129]: L', then S, then U [64][129], then K [64][129]
+//   RB [64][129]:  U, then dU, then T dT^T... ([64][65]), then Q
+//   RC [64][129]:  K^, then dW, then (K K^T) o R ([64][65])
+//   RD [64][129]:  dO, then V
+//   N1, N2, N3 [64][65]: T then P; dP then its product form; dT then dA
+// and the per-token adjoints dG, dbeta (shared atomics).
+constexpr uint32_t LB_RA = 0;
+constexpr uint32_t LB_RB = LB_RA + D * LW;
+constexpr uint32_t LB_RC = LB_RB + C * LW;
+constexpr uint32_t LB_RD = LB_RC + C * LW;
+constexpr uint32_t LB_N1 = LB_RD + C * LW;
+constexpr uint32_t LB_N2 = LB_N1 + C * LN;
+constexpr uint32_t LB_N3 = LB_N2 + C * LN;
+constexpr uint32_t LB_G = LB_N3 + C * LN;     // G, gamma, beta, dG, dbeta [64] each
+constexpr uint32_t LB_MISC = LB_G + 5 * C;    // dG_C, <S, L'>
+constexpr uint32_t LB_FLOATS = LB_MISC + 8;
+constexpr uint32_t LB_SMEM = LB_FLOATS * sizeof(float);
+
+template <typename IoT>
+__device__ __forceinline__ void load_rows(float *dst, const IoT *src, int tok0, int cl, int heads,
+                                          int head) {
+    for (int e = threadIdx.x; e < C * D; e += kLocalThreads) {
+        const int i = e >> 7, d = e & 127;
+        dst[i * LW + d] = i < cl ? ldio(src + ((size_t)(tok0 + i) * heads + head) * D + d) : 0.f;
+    }
+}
+
+template <typename IoT>
+__global__ void __launch_bounds__(kLocalThreads, 1)
+bwd_local_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT *__restrict__ v,
+                 const float *__restrict__ g, const IoT *__restrict__ dO,
+                 const int32_t *__restrict__ cu, int num_seqs, int total_T, int Hqk, int H,
+                 const int32_t *__restrict__ base, const float *__restrict__ recs,
+                 float *__restrict__ dq, float *__restrict__ dk, float *__restrict__ dv,
+                 float *__restrict__ dg, float *__restrict__ dbeta) {
+    extern __shared__ __align__(16) float fs[];
+    int n, c;
+    const int gc = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
+    if (!chunk_of(base, num_seqs, gc, n, c)) return;
+    int t0, len;
+    sequence_range(cu, n, num_seqs, total_T, t0, len);
+    const int tok0 = t0 + c * C, cl = min(C, len - c * C), hq = h / (H / Hqk);
+    const float *rec = recs + ((size_t)gc * H + h) * R_FLOATS;
+    float *RA = fs + LB_RA, *RB = fs + LB_RB, *RC = fs + LB_RC, *RD = fs + LB_RD;
+    float *N1 = fs + LB_N1, *N2 = fs + LB_N2, *N3 = fs + LB_N3;
+    float *Gs = fs + LB_G, *gam = Gs + C, *Bs = gam + C, *dG = Bs + C, *dB = dG + C;
+    float *misc = fs + LB_MISC;
+    auto qk_at = [&](float *base_, int i, int d) { return base_ + ((size_t)(tok0 + i) * Hqk + hq) * D + d; };
+
+    // ---- phase A: dK^ = U L' and <S, L'> --------------------------------------
+    for (int e = tid; e < D * D; e += kLocalThreads) RA[(e >> 7) * LW + (e & 127)] = rec[R_L + e];
+    for (int e = tid; e < C * D; e += kLocalThreads) RB[(e >> 7) * LW + (e & 127)] = rec[R_U + e];
+    if (tid < C) {
+        Gs[tid] = rec[R_G + tid];
+        gam[tid] = __expf(rec[R_G + tid]);
+        Bs[tid] = rec[R_B + tid];
+        dG[tid] = 0.f;
+        dB[tid] = 0.f;
+    }
+    if (tid < 8) misc[tid] = 0.f;
+    __syncthreads();
+    const float GC = Gs[C - 1], gC = __expf(GC);
+    for (int e = tid; e < C * D; e += kLocalThreads) {   // K^ rows
+        const int i = e >> 7, d = e & 127;
+        const float kv = i < cl ? ldio(k + ((size_t)(tok0 + i) * Hqk + hq) * D + d) : 0.f;
+        RC[i * LW + d] = kv * __expf(GC - Gs[i]);
+    }
+    {
+        float part = 0.f;   // <S, L'> over this thread's entries
+        for (int e = tid; e < D * D; e += kLocalThreads) part = fmaf(rec[R_S + e], RA[(e >> 7) * LW + (e & 127)], part);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+        if ((tid & 31) == 0) atomicAdd(&misc[1], part);
+    }
+    __syncthreads();
+    {
+        float rowacc[4] = {0.f, 0.f, 0.f, 0.f}, gcacc = 0.f;
+        gemm<C, D, kLocalThreads>(D, [&](int j, int r) { return RB[j * LW + r]; },
+                                  [&](int r, int d) { return RA[r * LW + d]; },
+                                  [&](int j, int d, float x) {
+                                      if (j < cl) atomicAdd(qk_at(dk, j, d), __expf(GC - Gs[j]) * x);
+                                      const float t = RC[j * LW + d] * x;
+                                      rowacc[j >> 4] -= t;   // rows j = gr + 16 r
+                                      gcacc += t;
+                                  });
+        const int gr = tid >> 4;
+#pragma unroll
+        for (int r = 0; r < 4; ++r) atomicAdd(&dG[gr + 16 * r], rowacc[r]);
+        atomicAdd(&misc[0], gcacc);
+    }
+    __syncthreads();
+
+    // ---- phase B: dW = -dU S, d(gamma Q) = dO S ---------------------------------
+    for (int e = tid; e < D * D; e += kLocalThreads) RA[(e >> 7) * LW + (e & 127)] = rec[R_S + e];
+    for (int e = tid; e < C * D; e += kLocalThreads) RB[(e >> 7) * LW + (e & 127)] = rec[R_DU + e];
+    load_rows<IoT>(RD, dO, tok0, cl, H, h);
+    __syncthreads();
+    gemm<C, D, kLocalThreads>(D, [&](int j, int r) { return RB[j * LW + r]; },
+                              [&](int r, int d) { return RA[r * LW + d]; },
+                              [&](int j, int d, float x) { RC[j * LW + d] = -x; });
+    {
+        float rowacc[4] = {0.f, 0.f, 0.f, 0.f};
+        gemm<C, D, kLocalThreads>(D, [&](int i, int r) { return RD[i * LW + r]; },
+                                  [&](int r, int d) { return RA[r * LW + d]; },
+                                  [&](int i, int d, float x) {
+                                      if (i < cl) {
+                                          atomicAdd(qk_at(dq, i, d), gam[i] * x);
+                                          rowacc[i >> 4] += gam[i] * ldio(q + ((size_t)(tok0 + i) * Hqk + hq) * D + d) * x;
+                                      }
+                                  });
+        const int gr = tid >> 4;
+#pragma unroll
+        for (int r = 0; r < 4; ++r) atomicAdd(&dG[gr + 16 * r], rowacc[r]);
+    }
+    __syncthreads();
+
+    // ---- phase C: dP, T^T dU, T^T dW, dT ---------------------------------------
+    for (int e = tid; e < C * D; e += kLocalThreads) RA[(e >> 7) * LW + (e & 127)] = rec[R_U + e];
+    for (int e = tid; e < C * C; e += kLocalThreads) N1[(e >> 6) * LN + (e & 63)] = rec[R_T + e];
+    __syncthreads();
+    gemm<C, C, kLocalThreads>(D, [&](int i, int r) { return RD[i * LW + r]; },
+                              [&](int r, int j) { return RA[j * LW + r]; },
+                              [&](int i, int j, float x) { N2[i * LN + j] = j <= i ? x : 0.f; });
+    __syncthreads();
+    load_rows<IoT>(RD, v, tok0, cl, H, h);
+    for (int e = tid; e < C * D; e += kLocalThreads) {
+        const int i = e >> 7, d = e & 127;
+        RA[i * LW + d] = i < cl ? ldio(k + ((size_t)(tok0 + i) * Hqk + hq) * D + d) : 0.f;
+    }
+    __syncthreads();
+    {
+        float rowacc[4] = {0.f, 0.f, 0.f, 0.f};
+        gemm<C, D, kLocalThreads>(C, [&](int j, int i) { return N1[i * LN + j]; },
+                                  [&](int i, int r) { return RB[i * LW + r]; },
+                                  [&](int j, int r, float x) {
+                                      if (j < cl) dv[((size_t)(tok0 + j) * H + h) * D + r] = Bs[j] * x;
+                                      rowacc[j >> 4] += RD[j * LW + r] * x;
+                                  });
+        const int gr = tid >> 4;
+#pragma unroll
+        for (int r = 0; r < 4; ++r) atomicAdd(&dB[gr + 16 * r], rowacc[r]);
+    }
+    {
+        float bacc[4] = {0.f, 0.f, 0.f, 0.f}, gacc[4] = {0.f, 0.f, 0.f, 0.f};
+        gemm<C, D, kLocalThreads>(C, [&](int j, int i) { return N1[i * LN + j]; },
+                                  [&](int i, int d) { return RC[i * LW + d]; },
+                                  [&](int j, int d, float x) {
+                                      if (j < cl) atomicAdd(qk_at(dk, j, d), Bs[j] * gam[j] * x);
+                                      const float t = RA[j * LW + d] * x;
+                                      bacc[j >> 4] += gam[j] * t;
+                                      gacc[j >> 4] += Bs[j] * gam[j] * t;
+                                  });
+        const int gr = tid >> 4;
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            atomicAdd(&dB[gr + 16 * r], bacc[r]);
+            atomicAdd(&dG[gr + 16 * r], gacc[r]);
+        }
+    }
+    gemm<C, C, kLocalThreads>(D, [&](int i, int r) { return RB[i * LW + r]; },
+                              [&](int r, int j) { return Bs[j] * RD[j * LW + r]; },
+                              [&](int i, int j, float x) { N3[i * LN + j] = x; });
+    gemm<C, C, kLocalThreads>(D, [&](int i, int d) { return RC[i * LW + d]; },
+                              [&](int d, int j) { return Bs[j] * gam[j] * RA[j * LW + d]; },
+                              [&](int i, int j, float x) { N3[i * LN + j] += x; });
+    __syncthreads();
+
+    // ---- phase D: dA = -T^T dT T^T, then the A and P terms ------------------------
+    float *Y = RB;   // [64][65]
+    gemm<C, C, kLocalThreads>(C, [&](int i, int m) { return N3[i * LN + m]; },
+                              [&](int m, int j) { return N1[j * LN + m]; },
+                              [&](int i, int j, float x) { Y[i * LN + j] = x; });
+    __syncthreads();
+    gemm<C, C, kLocalThreads>(C, [&](int i, int m) { return N1[m * LN + i]; },
+                              [&](int m, int j) { return Y[m * LN + j]; },
+                              [&](int i, int j, float x) { N3[i * LN + j] = j < i ? -x : 0.f; });
+    __syncthreads();
+    float *AR = RC;   // [64][65]
+    for (int e = tid; e < C * C; e += kLocalThreads) {
+        AR[(e >> 6) * LN + (e & 63)] = rec[R_AR + e];
+        N1[(e >> 6) * LN + (e & 63)] = rec[R_P + e];
+    }
+    __syncthreads();
+    for (int e = tid; e < C * C; e += kLocalThreads) {
+        const int i = e >> 6, j = e & 63;
+        const float R = j <= i ? __expf(Gs[i] - Gs[j]) : 0.f;
+        const float da = N3[i * LN + j], ar = AR[i * LN + j];
+        const float ea = da * Bs[i] * ar;            // dA o A
+        const float dp = N2[i * LN + j], ep = dp * N1[i * LN + j];   // dP o P
+        if (da != 0.f || dp != 0.f) {
+            atomicAdd(&dB[i], da * ar);
+            atomicAdd(&dG[i], ea + ep);
+            atomicAdd(&dG[j], -(ea + ep));
+        }
+        N3[i * LN + j] = da * Bs[i] * R;             // M = dA o beta_i R
+        N2[i * LN + j] = dp * R;                     // dP o R
+    }
+    for (int e = tid; e < C * D; e += kLocalThreads) {   // Q rows over the finished Y
+        const int i = e >> 7, d = e & 127;
+        RB[i * LW + d] = i < cl ? ldio(q + ((size_t)(tok0 + i) * Hqk + hq) * D + d) : 0.f;
+    }
+    __syncthreads();
+    gemm<C, D, kLocalThreads>(C, [&](int i, int j) { return N3[i * LN + j]; },
+                              [&](int j, int d) { return RA[j * LW + d]; },
+                              [&](int i, int d, float x) { if (i < cl) atomicAdd(qk_at(dk, i, d), x); });
+    gemm<C, D, kLocalThreads>(C, [&](int j, int i) { return N3[i * LN + j]; },
+                              [&](int i, int d) { return RA[i * LW + d]; },
+                              [&](int j, int d, float x) { if (j < cl) atomicAdd(qk_at(dk, j, d), x); });
+    gemm<C, D, kLocalThreads>(C, [&](int i, int j) { return N2[i * LN + j]; },
+                              [&](int j, int d) { return RA[j * LW + d]; },
+                              [&](int i, int d, float x) { if (i < cl) atomicAdd(qk_at(dq, i, d), x); });
+    gemm<C, D, kLocalThreads>(C, [&](int j, int i) { return N2[i * LN + j]; },
+                              [&](int i, int d) { return RB[i * LW + d]; },
+                              [&](int j, int d, float x) { if (j < cl) atomicAdd(qk_at(dk, j, d), x); });
+    __syncthreads();
+
+    // ---- phase E: dg as the reverse cumulative sum of dG, and dbeta -----------------
+    if (tid == 0) dG[C - 1] += misc[0] + gC * misc[1];
+    __syncthreads();
+    if (tid < C && tid < cl) {
+        float acc = 0.f;
+        for (int i = C - 1; i >= tid; --i) acc += dG[i];
+        const size_t r = (size_t)(tok0 + tid) * H + h;
+        dg[r] = g[r] < kLogGateMin ? 0.f : acc;
+        dbeta[r] = dB[tid];
+    }
+}
+
+template <typename IoT>
+cudaError_t launch_chunked(const IoT *q, const IoT *k, const IoT *v, const float *g,
+                           const float *beta, const float *h0, const int32_t *cu, int num_seqs,
+                           int total_T, int Hqk, int H, const IoT *dO, const float *dSf,
+                           float *dq, float *dk, float *dv, float *dg, float *dbeta, float *dh0,
+                           uint8_t *ws, long long max_total, size_t base_bytes,
+                           cudaStream_t stream) {
+    int32_t *base = reinterpret_cast<int32_t *>(ws);
+    float *recs = reinterpret_cast<float *>(ws + base_bytes);
+    cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void *>(bwd_prep_kernel<IoT>), (int)PB_SMEM);
+    if (e == cudaSuccess)
+        e = ensure_dynamic_smem(reinterpret_cast<const void *>(bwd_forward_kernel<IoT>), (int)CB_SMEM);
+    if (e == cudaSuccess)
+        e = ensure_dynamic_smem(reinterpret_cast<const void *>(bwd_reverse_kernel<IoT>), (int)CB_SMEM);
+    if (e == cudaSuccess)
+        e = ensure_dynamic_smem(reinterpret_cast<const void *>(bwd_local_kernel<IoT>), (int)LB_SMEM);
+    if (e != cudaSuccess) return e;
+    bwd_chunk_base_kernel<<<1, 1024, 0, stream>>>(cu, num_seqs, total_T, base);
+    const dim3 per_chunk((unsigned)max_total, (unsigned)H);
+    const dim3 per_rows((unsigned)(num_seqs * H), D / kRowBlock);
+    bwd_prep_kernel<IoT><<<per_chunk, kPrepB, PB_SMEM, stream>>>(q, k, v, g, beta, cu, num_seqs,
+                                                                  total_T, Hqk, H, base, recs);
+    bwd_forward_kernel<IoT><<<per_rows, kChainThreadsB, CB_SMEM, stream>>>(
+        k, h0, cu, num_seqs, total_T, Hqk, H, base, max_total, recs);
+    bwd_reverse_kernel<IoT><<<per_rows, kChainThreadsB, CB_SMEM, stream>>>(
+        q, k, dO, dSf, dh0, cu, num_seqs, total_T, Hqk, H, base, max_total, recs);
+    bwd_local_kernel<IoT><<<per_chunk, kLocalThreads, LB_SMEM, stream>>>(
+        q, k, v, g, dO, cu, num_seqs, total_T, Hqk, H, base, recs, dq, dk, dv, dg, dbeta);
+    return cudaGetLastError();
+}
+
+// Global chunks the records must hold: exact for equal lengths, else every
+// sequence may end with a partial chunk.
+long long chunk_slots(int num_seqs, int total_T, bool equal) {
+    if (num_seqs <= 0 || total_T <= 0) return 0;
+    if (equal) return (long long)num_seqs * ((total_T / num_seqs + C - 1) / C);
+    return (long long)(total_T + C - 1) / C + num_seqs;
+}
+
+size_t base_bytes_of(int num_seqs) { return ((size_t)(num_seqs + 1) * 4 + kBaseBytes - 1) & ~(kBaseBytes - 1); }
+
+}  // namespace
+
+size_t chunked_backward_workspace_bytes(int num_seqs, int total_T, int H, bool equal) {
+    const long long slots = chunk_slots(num_seqs, total_T, equal);
+    if (slots == 0) return 0;
+    return base_bytes_of(num_seqs) + (size_t)slots * H * R_FLOATS * sizeof(float);
+}
+
+cudaError_t launch_backward_chunked(const void *q, const void *k, const void *v, const float *g,
+                                    const float *beta, const float *h0, const int32_t *cu,
+                                    int num_seqs, int total_T, int Hqk, int H, bool bf16,
+                                    const void *dO, const float *dSf, float *dq, float *dk,
+                                    float *dv, float *dg, float *dbeta, float *dh0,
+                                    void *workspace, cudaStream_t stream) {
+    const long long slots = chunk_slots(num_seqs, total_T, cu == nullptr);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    // dq and dk sum over the value heads of a group and over the product
+    // terms: atomics into zeroed outputs; dv, dg, dbeta are written once
+    const size_t nq = (size_t)total_T * Hqk * D * sizeof(float);
+    cudaError_t e = cudaMemsetAsync(dq, 0, nq, stream);
+    if (e == cudaSuccess) e = cudaMemsetAsync(dk, 0, nq, stream);
+    if (e != cudaSuccess) return e;
+    const size_t bb = base_bytes_of(num_seqs);
+    if (bf16)
+        return launch_chunked<__nv_bfloat16>(
+            static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
+            static_cast<const __nv_bfloat16 *>(v), g, beta, h0, cu, num_seqs, total_T, Hqk, H,
+            static_cast<const __nv_bfloat16 *>(dO), dSf, dq, dk, dv, dg, dbeta, dh0, ws, slots, bb,
+            stream);
+    return launch_chunked<float>(static_cast<const float *>(q), static_cast<const float *>(k),
+                                 static_cast<const float *>(v), g, beta, h0, cu, num_seqs, total_T,
+                                 Hqk, H, static_cast<const float *>(dO), dSf, dq, dk, dv, dg, dbeta,
+                                 dh0, ws, slots, bb, stream);
+}
+
+}  // namespace gdr

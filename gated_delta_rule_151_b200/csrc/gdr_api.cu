@@ -381,6 +381,12 @@ gdr_status_t gdr_backward_workspace_size(int32_t num_seqs, int32_t total_T, int3
         !valid_dim(d_v))
         return GDR_ERR_INVALID_ARG;
     *bytes = gdr::backward_workspace_bytes(num_seqs, total_T, H, d_k, d_v);
+    // the chunked form (scalar gate, d_k = d_v = 128) needs more; with it the
+    // gradient takes the chunked form where it applies
+    if (d_k == 128 && d_v == 128) {
+        const size_t chunked = gdr::chunked_backward_workspace_bytes(num_seqs, total_T, H, false);
+        if (chunked > *bytes) *bytes = chunked;
+    }
     return GDR_OK;
 }
 
@@ -407,7 +413,15 @@ gdr_status_t gdr_backward(const void *q, const void *k, const void *v, const flo
             !ok_beta_ptr(beta) || !ok_beta_ptr(dbeta))
             return GDR_ERR_INVALID_ARG;
     }
-    const size_t need = gdr::backward_workspace_bytes(num_seqs, total_T, H, d_k, d_v);
+    // the chunked form where it applies and the workspace holds its records,
+    // else the token loop
+    const size_t chunked_need =
+        (gate_mode == GDR_GATE_SCALAR && d_k == 128 && d_v == 128)
+            ? gdr::chunked_backward_workspace_bytes(num_seqs, total_T, H, cu_seqlens == nullptr)
+            : 0;
+    const bool chunked = chunked_need > 0 && workspace != nullptr && workspace_bytes >= chunked_need &&
+                         aligned16(workspace);
+    const size_t need = chunked ? chunked_need : gdr::backward_workspace_bytes(num_seqs, total_T, H, d_k, d_v);
     if (need > 0 && (workspace == nullptr || workspace_bytes < need || !aligned16(workspace)))
         return GDR_ERR_WORKSPACE;
     // no output may overlap an input or another output
@@ -437,6 +451,11 @@ gdr_status_t gdr_backward(const void *q, const void *k, const void *v, const flo
             if (o0 < a1 && a0 < o1) return GDR_ERR_INVALID_ARG;
         }
     }
+    if (chunked)
+        return from_cuda(gdr::launch_backward_chunked(
+            q, k, v, g, beta, initial_state, cu_seqlens, num_seqs, total_T, H_qk, H,
+            io_dtype == GDR_BF16, d_o, d_final_state, dq, dk, dv, dg, dbeta, d_initial_state,
+            workspace, static_cast<cudaStream_t>(stream)));
     return from_cuda(gdr::launch_backward(
         q, k, v, g, beta, initial_state, cu_seqlens, num_seqs, total_T, H_qk, H, d_k, d_v,
         gate_mode == GDR_GATE_CHANNEL, io_dtype == GDR_BF16, d_o, d_final_state, dq, dk, dv, dg,

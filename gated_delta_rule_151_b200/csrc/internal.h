@@ -22,6 +22,16 @@ cudaError_t launch_backward(const void *q, const void *k, const void *v, const f
                             float *dg, float *dbeta, float *dh0, void *workspace,
                             cudaStream_t stream);
 
+// Gradient in chunked form (scalar gate, d_k = d_v = 128): workspace bytes
+// (equal: the sequences have equal lengths and no cu_seqlens), launcher.
+size_t chunked_backward_workspace_bytes(int num_seqs, int total_T, int H, bool equal);
+cudaError_t launch_backward_chunked(const void *q, const void *k, const void *v, const float *g,
+                                    const float *beta, const float *h0, const int32_t *cu,
+                                    int num_seqs, int total_T, int Hqk, int H, bool bf16,
+                                    const void *dO, const float *dSf, float *dq, float *dk,
+                                    float *dv, float *dg, float *dbeta, float *dh0,
+                                    void *workspace, cudaStream_t stream);
+
 // Input-side prologue: short causal convolution with state, q/k
 // normalisation, gate and beta maps (arguments validated by the C ABI).
 cudaError_t launch_prologue(const void *xq, const void *xk, const void *xv, const float *wq,
