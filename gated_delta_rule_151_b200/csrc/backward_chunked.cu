@@ -31,7 +31,7 @@
 // Everything is fp32 on CUDA cores: a register-tiled product over padded
 // shared-memory operands (rows of 129 or 65 floats, so rows and columns are
 // both read without bank conflicts).  The chunk records live in the
-// workspace: 311,808 bytes per (chunk, head).
+// workspace: 377,344 bytes per (chunk, head).
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -56,7 +56,9 @@ constexpr size_t R_U = R_B + C;                 // U [64][128]
 constexpr size_t R_DU = R_U + C * D;            // dU [64][128]
 constexpr size_t R_S = R_DU + C * D;            // state entering the chunk [128][128]
 constexpr size_t R_L = R_S + D * D;             // adjoint of the state leaving it [128][128]
-constexpr size_t R_FLOATS = R_L + D * D;        // 77,952 floats
+constexpr size_t R_KH = R_L + D * D;            // K^ [64][128]
+constexpr size_t R_QT = R_KH + C * D;           // diag(gamma) Q [64][128]
+constexpr size_t R_FLOATS = R_QT + C * D;       // 94,336 floats
 constexpr size_t kBaseBytes = 256;              // sequence chunk offsets precede the records
 
 constexpr int LW = D + 1;    // padded row of 128 floats
@@ -65,8 +67,46 @@ constexpr int kRowBlock = 16;                   // state rows per forward / reve
 constexpr int kChainThreadsB = 128;
 constexpr int kLocalThreads = 256;
 
-__device__ __forceinline__ float ldio(const float *p) { return *p; }
-__device__ __forceinline__ float ldio(const __nv_bfloat16 *p) { return __bfloat162float(*p); }
+// rows x cols fp32 (cols a multiple of 4, 16-byte aligned) from the record
+// into padded shared rows of `ld` floats: 16-byte loads, eight in flight per
+// thread before their stores.
+template <int NT>
+__device__ __forceinline__ void copy_rows(float *dst, int ld, const float *src, int rows, int cols) {
+    const int q4 = cols / 4, total = rows * q4;
+    const float4 *s4 = reinterpret_cast<const float4 *>(src);
+#pragma unroll 8
+    for (int e = threadIdx.x; e < total; e += NT) {
+        const float4 x = __ldg(s4 + e);
+        float *d = dst + (e / q4) * ld + (e % q4) * 4;
+        d[0] = x.x; d[1] = x.y; d[2] = x.z; d[3] = x.w;
+    }
+}
+
+// The chunk's 64 rows of a [T, heads, 128] input (0 past the sequence's end)
+// into padded shared rows: four values per load (8 bytes of bf16 or 16 of
+// fp32), eight loads in flight per thread.
+__device__ __forceinline__ void ld4io(const float *p, float (&x)[4]) {
+    const float4 v = __ldg(reinterpret_cast<const float4 *>(p));
+    x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
+}
+__device__ __forceinline__ void ld4io(const __nv_bfloat16 *p, float (&x)[4]) {
+    const uint2 raw = __ldg(reinterpret_cast<const uint2 *>(p));
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.x));
+    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.y));
+    x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y;
+}
+template <int NT, typename IoT>
+__device__ __forceinline__ void load_io_rows(float *dst, const IoT *src, int tok0, int cl, int heads,
+                                             int head) {
+#pragma unroll 8
+    for (int e = threadIdx.x; e < C * D / 4; e += NT) {
+        const int i = e >> 5, d = (e & 31) * 4;
+        float x[4] = {0.f, 0.f, 0.f, 0.f};
+        if (i < cl) ld4io(src + ((size_t)(tok0 + i) * heads + head) * D + d, x);
+        float *o = dst + i * LW + d;
+        o[0] = x[0]; o[1] = x[1]; o[2] = x[2]; o[3] = x[3];
+    }
+}
 
 // The product tile of one thread: out(m, n) = sum_k a(m, k) b(k, n) for
 // rows m = gr + GR r and columns n = gc + GC c, (gr, gc) = (tid / GC, tid % GC),
@@ -190,19 +230,9 @@ bwd_prep_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT 
     float *rec = recs + ((size_t)gc * H + h) * R_FLOATS;
     float *Ks = fs + PB_K, *Qs = fs + PB_Q, *Vs = fs + PB_V, *Tp = fs + PB_TP;
     float *Gs = fs + PB_G, *gam = Gs + C, *Bs = gam + C;
-    for (int e = tid; e < C * D; e += kPrepB) {
-        const int i = e >> 7, d = e & 127;
-        float kv = 0.f, qv = 0.f, vv = 0.f;
-        if (i < cl) {
-            const size_t rq = ((size_t)(tok0 + i) * Hqk + hq) * D + d;
-            kv = ldio(k + rq);
-            qv = ldio(q + rq);
-            vv = ldio(v + ((size_t)(tok0 + i) * H + h) * D + d);
-        }
-        Ks[i * LW + d] = kv;
-        Qs[i * LW + d] = qv;
-        Vs[i * LW + d] = vv;
-    }
+    load_io_rows<kPrepB>(Ks, k, tok0, cl, Hqk, hq);
+    load_io_rows<kPrepB>(Qs, q, tok0, cl, Hqk, hq);
+    load_io_rows<kPrepB>(Vs, v, tok0, cl, H, h);
     if (tid < 32) {   // gates of tokens 2 tid, 2 tid + 1: clamped, cumulated, 0 past the end
         const int i0 = 2 * tid, i1 = i0 + 1;
         const float g0 = i0 < cl ? clamp_log_gate(g[(size_t)(tok0 + i0) * H + h]) : 0.f;
@@ -243,10 +273,15 @@ bwd_prep_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT 
         Tp[i * LN + j] = t;
         rec[R_T + e] = t;
     }
-    // the scaled operands of W and U~ in place
+    // K^ and diag(gamma) Q to the record, then the scaled operands of W and
+    // U~ in place
+    const float GCp = Gs[C - 1];
     for (int e = tid; e < C * D; e += kPrepB) {
         const int i = e >> 7, d = e & 127;
-        Ks[i * LW + d] *= Bs[i] * gam[i];
+        const float kv = Ks[i * LW + d];
+        rec[R_KH + e] = kv * __expf(GCp - Gs[i]);
+        rec[R_QT + e] = Qs[i * LW + d] * gam[i];
+        Ks[i * LW + d] = kv * Bs[i] * gam[i];
         Vs[i * LW + d] *= Bs[i];
     }
     if (tid < C) {
@@ -278,34 +313,13 @@ constexpr uint32_t CB_G = CB_C2 + C * (kRowBlock + 1);    // G [64]
 constexpr uint32_t CB_FLOATS = CB_G + C;
 constexpr uint32_t CB_SMEM = CB_FLOATS * sizeof(float);
 
-// The chunk's K^ rows k_j e^{G_C - G_j} (0 past the sequence's end) into dst
-// [64][129], and, when Qt is given, gamma_i q_i into Qt; G from the record.
-template <typename IoT>
-__device__ __forceinline__ void load_khat(const IoT *k, const IoT *q, const float *rec, float *Gs,
-                                          float *dst, float *Qt, int tok0, int cl, int Hqk, int hq) {
-    for (int e = threadIdx.x; e < C * D; e += blockDim.x) {
-        const int i = e >> 7, d = e & 127;
-        float kv = 0.f, qv = 0.f;
-        if (i < cl) {
-            const size_t r = ((size_t)(tok0 + i) * Hqk + hq) * D + d;
-            kv = ldio(k + r);
-            if (Qt != nullptr) qv = ldio(q + r);
-        }
-        const float Gi = rec[R_G + i], GC = rec[R_G + C - 1];
-        dst[i * LW + d] = kv * __expf(GC - Gi);
-        if (Qt != nullptr) Qt[i * LW + d] = qv * __expf(Gi);
-    }
-    if (threadIdx.x < C) Gs[threadIdx.x] = rec[R_G + threadIdx.x];
-}
-
-template <typename IoT>
 __global__ void __launch_bounds__(kChainThreadsB, 1)
-bwd_forward_kernel(const IoT *__restrict__ k, const float *__restrict__ h0,
+bwd_forward_kernel(const float *__restrict__ h0,
                    const int32_t *__restrict__ cu, int num_seqs, int total_T, int Hqk, int H,
                    const int32_t *__restrict__ base, long long slots, float *__restrict__ recs) {
     extern __shared__ __align__(16) float fs[];
     const int chain = blockIdx.x, h = chain % H, n = chain / H, r0 = blockIdx.y * kRowBlock;
-    const int tid = threadIdx.x, hq = h / (H / Hqk);
+    const int tid = threadIdx.x;
     int t0, len;
     sequence_range(cu, n, num_seqs, total_T, t0, len);
     const int b0 = base[n];
@@ -318,14 +332,14 @@ bwd_forward_kernel(const IoT *__restrict__ k, const float *__restrict__ h0,
     }
     for (int c = 0; c < nch; ++c) {
         float *rec = recs + ((size_t)(b0 + c) * H + h) * R_FLOATS;
-        const int tok0 = t0 + c * C, cl = min(C, len - c * C);
         __syncthreads();   // the rows of the last chunk's update are in place
         for (int e = tid; e < kRowBlock * D; e += kChainThreadsB) {
             const int r = e >> 7, d = e & 127;
             rec[R_S + (size_t)(r0 + r) * D + d] = Sr[r * LW + d];
         }
-        for (int e = tid; e < C * D; e += kChainThreadsB) Ws[(e >> 7) * LW + (e & 127)] = rec[R_W + e];
-        load_khat<IoT>(k, static_cast<const IoT *>(nullptr), rec, Gs, Kh, nullptr, tok0, cl, Hqk, hq);
+        copy_rows<kChainThreadsB>(Ws, LW, rec + R_W, C, D);
+        copy_rows<kChainThreadsB>(Kh, LW, rec + R_KH, C, D);
+        if (tid < C) Gs[tid] = rec[R_G + tid];
         __syncthreads();
         // U[j][r0 + r] = U~[j][r0 + r] - sum_d W[j][d] S[r0 + r][d]
         gemm<C, kRowBlock, kChainThreadsB>(D, [&](int j, int d) { return Ws[j * LW + d]; },
@@ -346,13 +360,13 @@ bwd_forward_kernel(const IoT *__restrict__ k, const float *__restrict__ h0,
 
 template <typename IoT>
 __global__ void __launch_bounds__(kChainThreadsB, 1)
-bwd_reverse_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT *__restrict__ dO,
+bwd_reverse_kernel(const IoT *__restrict__ dO,
                    const float *__restrict__ dSf, float *__restrict__ dh0,
                    const int32_t *__restrict__ cu, int num_seqs, int total_T, int Hqk, int H,
                    const int32_t *__restrict__ base, long long slots, float *__restrict__ recs) {
     extern __shared__ __align__(16) float fs[];
     const int chain = blockIdx.x, h = chain % H, n = chain / H, r0 = blockIdx.y * kRowBlock;
-    const int tid = threadIdx.x, hq = h / (H / Hqk);
+    const int tid = threadIdx.x;
     int t0, len;
     sequence_range(cu, n, num_seqs, total_T, t0, len);
     const int b0 = base[n];
@@ -371,14 +385,18 @@ bwd_reverse_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const I
             const int r = e >> 7, d = e & 127;
             rec[R_L + (size_t)(r0 + r) * D + d] = Lr[r * LW + d];
         }
-        for (int e = tid; e < C * D; e += kChainThreadsB) Ws[(e >> 7) * LW + (e & 127)] = rec[R_W + e];
-        for (int e = tid; e < C * C; e += kChainThreadsB) Ps[(e >> 6) * LN + (e & 63)] = rec[R_P + e];
-        for (int e = tid; e < C * kRowBlock; e += kChainThreadsB) {
-            const int i = e / kRowBlock, r = e % kRowBlock;
-            dOr[i * (kRowBlock + 1) + r] =
-                i < cl ? ldio(dO + ((size_t)(tok0 + i) * H + h) * D + r0 + r) : 0.f;
+        copy_rows<kChainThreadsB>(Ws, LW, rec + R_W, C, D);
+        copy_rows<kChainThreadsB>(Kh, LW, rec + R_KH, C, D);
+        copy_rows<kChainThreadsB>(Qt, LW, rec + R_QT, C, D);
+        copy_rows<kChainThreadsB>(Ps, LN, rec + R_P, C, C);
+        for (int e = tid; e < C * kRowBlock / 4; e += kChainThreadsB) {   // dO[:, r0 .. r0 + 15]
+            const int i = e >> 2, r = (e & 3) * 4;
+            float x[4] = {0.f, 0.f, 0.f, 0.f};
+            if (i < cl) ld4io(dO + ((size_t)(tok0 + i) * H + h) * D + r0 + r, x);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) dOr[i * (kRowBlock + 1) + r + u] = x[u];
         }
-        load_khat<IoT>(k, q, rec, Gs, Kh, Qt, tok0, cl, Hqk, hq);
+        if (tid < C) Gs[tid] = rec[R_G + tid];
         __syncthreads();
         // dU[j][r] = sum_d K^[j][d] L[r][d] + sum_i P[i][j] dO[i][r]
         gemm<C, kRowBlock, kChainThreadsB>(D, [&](int j, int d) { return Kh[j * LW + d]; },
@@ -432,15 +450,6 @@ constexpr uint32_t LB_FLOATS = LB_MISC + 8;
 constexpr uint32_t LB_SMEM = LB_FLOATS * sizeof(float);
 
 template <typename IoT>
-__device__ __forceinline__ void load_rows(float *dst, const IoT *src, int tok0, int cl, int heads,
-                                          int head) {
-    for (int e = threadIdx.x; e < C * D; e += kLocalThreads) {
-        const int i = e >> 7, d = e & 127;
-        dst[i * LW + d] = i < cl ? ldio(src + ((size_t)(tok0 + i) * heads + head) * D + d) : 0.f;
-    }
-}
-
-template <typename IoT>
 __global__ void __launch_bounds__(kLocalThreads, 1)
 bwd_local_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT *__restrict__ v,
                  const float *__restrict__ g, const IoT *__restrict__ dO,
@@ -463,8 +472,9 @@ bwd_local_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT
     auto qk_at = [&](float *base_, int i, int d) { return base_ + ((size_t)(tok0 + i) * Hqk + hq) * D + d; };
 
     // ---- phase A: dK^ = U L' and <S, L'> --------------------------------------
-    for (int e = tid; e < D * D; e += kLocalThreads) RA[(e >> 7) * LW + (e & 127)] = rec[R_L + e];
-    for (int e = tid; e < C * D; e += kLocalThreads) RB[(e >> 7) * LW + (e & 127)] = rec[R_U + e];
+    copy_rows<kLocalThreads>(RA, LW, rec + R_L, D, D);
+    copy_rows<kLocalThreads>(RB, LW, rec + R_U, C, D);
+    copy_rows<kLocalThreads>(RC, LW, rec + R_KH, C, D);
     if (tid < C) {
         Gs[tid] = rec[R_G + tid];
         gam[tid] = __expf(rec[R_G + tid]);
@@ -475,11 +485,6 @@ bwd_local_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT
     if (tid < 8) misc[tid] = 0.f;
     __syncthreads();
     const float GC = Gs[C - 1], gC = __expf(GC);
-    for (int e = tid; e < C * D; e += kLocalThreads) {   // K^ rows
-        const int i = e >> 7, d = e & 127;
-        const float kv = i < cl ? ldio(k + ((size_t)(tok0 + i) * Hqk + hq) * D + d) : 0.f;
-        RC[i * LW + d] = kv * __expf(GC - Gs[i]);
-    }
     {
         float part = 0.f;   // <S, L'> over this thread's entries
         for (int e = tid; e < D * D; e += kLocalThreads) part = fmaf(rec[R_S + e], RA[(e >> 7) * LW + (e & 127)], part);
@@ -506,9 +511,9 @@ bwd_local_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT
     __syncthreads();
 
     // ---- phase B: dW = -dU S, d(gamma Q) = dO S ---------------------------------
-    for (int e = tid; e < D * D; e += kLocalThreads) RA[(e >> 7) * LW + (e & 127)] = rec[R_S + e];
-    for (int e = tid; e < C * D; e += kLocalThreads) RB[(e >> 7) * LW + (e & 127)] = rec[R_DU + e];
-    load_rows<IoT>(RD, dO, tok0, cl, H, h);
+    copy_rows<kLocalThreads>(RA, LW, rec + R_S, D, D);
+    copy_rows<kLocalThreads>(RB, LW, rec + R_DU, C, D);
+    load_io_rows<kLocalThreads>(RD, dO, tok0, cl, H, h);
     __syncthreads();
     gemm<C, D, kLocalThreads>(D, [&](int j, int r) { return RB[j * LW + r]; },
                               [&](int r, int d) { return RA[r * LW + d]; },
@@ -520,7 +525,7 @@ bwd_local_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT
                                   [&](int i, int d, float x) {
                                       if (i < cl) {
                                           atomicAdd(qk_at(dq, i, d), gam[i] * x);
-                                          rowacc[i >> 4] += gam[i] * ldio(q + ((size_t)(tok0 + i) * Hqk + hq) * D + d) * x;
+                                          rowacc[i >> 4] += rec[R_QT + i * D + d] * x;
                                       }
                                   });
         const int gr = tid >> 4;
@@ -530,18 +535,15 @@ bwd_local_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT
     __syncthreads();
 
     // ---- phase C: dP, T^T dU, T^T dW, dT ---------------------------------------
-    for (int e = tid; e < C * D; e += kLocalThreads) RA[(e >> 7) * LW + (e & 127)] = rec[R_U + e];
-    for (int e = tid; e < C * C; e += kLocalThreads) N1[(e >> 6) * LN + (e & 63)] = rec[R_T + e];
+    copy_rows<kLocalThreads>(RA, LW, rec + R_U, C, D);
+    copy_rows<kLocalThreads>(N1, LN, rec + R_T, C, C);
     __syncthreads();
     gemm<C, C, kLocalThreads>(D, [&](int i, int r) { return RD[i * LW + r]; },
                               [&](int r, int j) { return RA[j * LW + r]; },
                               [&](int i, int j, float x) { N2[i * LN + j] = j <= i ? x : 0.f; });
     __syncthreads();
-    load_rows<IoT>(RD, v, tok0, cl, H, h);
-    for (int e = tid; e < C * D; e += kLocalThreads) {
-        const int i = e >> 7, d = e & 127;
-        RA[i * LW + d] = i < cl ? ldio(k + ((size_t)(tok0 + i) * Hqk + hq) * D + d) : 0.f;
-    }
+    load_io_rows<kLocalThreads>(RD, v, tok0, cl, H, h);
+    load_io_rows<kLocalThreads>(RA, k, tok0, cl, Hqk, hq);
     __syncthreads();
     {
         float rowacc[4] = {0.f, 0.f, 0.f, 0.f};
@@ -591,10 +593,8 @@ bwd_local_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT
                               [&](int i, int j, float x) { N3[i * LN + j] = j < i ? -x : 0.f; });
     __syncthreads();
     float *AR = RC;   // [64][65]
-    for (int e = tid; e < C * C; e += kLocalThreads) {
-        AR[(e >> 6) * LN + (e & 63)] = rec[R_AR + e];
-        N1[(e >> 6) * LN + (e & 63)] = rec[R_P + e];
-    }
+    copy_rows<kLocalThreads>(AR, LN, rec + R_AR, C, C);
+    copy_rows<kLocalThreads>(N1, LN, rec + R_P, C, C);
     __syncthreads();
     for (int e = tid; e < C * C; e += kLocalThreads) {
         const int i = e >> 6, j = e & 63;
@@ -610,10 +610,7 @@ bwd_local_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT
         N3[i * LN + j] = da * Bs[i] * R;             // M = dA o beta_i R
         N2[i * LN + j] = dp * R;                     // dP o R
     }
-    for (int e = tid; e < C * D; e += kLocalThreads) {   // Q rows over the finished Y
-        const int i = e >> 7, d = e & 127;
-        RB[i * LW + d] = i < cl ? ldio(q + ((size_t)(tok0 + i) * Hqk + hq) * D + d) : 0.f;
-    }
+    load_io_rows<kLocalThreads>(RB, q, tok0, cl, Hqk, hq);   // Q rows over the finished Y
     __syncthreads();
     gemm<C, D, kLocalThreads>(C, [&](int i, int j) { return N3[i * LN + j]; },
                               [&](int j, int d) { return RA[j * LW + d]; },
@@ -652,7 +649,7 @@ cudaError_t launch_chunked(const IoT *q, const IoT *k, const IoT *v, const float
     float *recs = reinterpret_cast<float *>(ws + base_bytes);
     cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void *>(bwd_prep_kernel<IoT>), (int)PB_SMEM);
     if (e == cudaSuccess)
-        e = ensure_dynamic_smem(reinterpret_cast<const void *>(bwd_forward_kernel<IoT>), (int)CB_SMEM);
+        e = ensure_dynamic_smem(reinterpret_cast<const void *>(bwd_forward_kernel), (int)CB_SMEM);
     if (e == cudaSuccess)
         e = ensure_dynamic_smem(reinterpret_cast<const void *>(bwd_reverse_kernel<IoT>), (int)CB_SMEM);
     if (e == cudaSuccess)
@@ -663,10 +660,10 @@ cudaError_t launch_chunked(const IoT *q, const IoT *k, const IoT *v, const float
     const dim3 per_rows((unsigned)(num_seqs * H), D / kRowBlock);
     bwd_prep_kernel<IoT><<<per_chunk, kPrepB, PB_SMEM, stream>>>(q, k, v, g, beta, cu, num_seqs,
                                                                   total_T, Hqk, H, base, recs);
-    bwd_forward_kernel<IoT><<<per_rows, kChainThreadsB, CB_SMEM, stream>>>(
-        k, h0, cu, num_seqs, total_T, Hqk, H, base, max_total, recs);
+    bwd_forward_kernel<<<per_rows, kChainThreadsB, CB_SMEM, stream>>>(
+        h0, cu, num_seqs, total_T, Hqk, H, base, max_total, recs);
     bwd_reverse_kernel<IoT><<<per_rows, kChainThreadsB, CB_SMEM, stream>>>(
-        q, k, dO, dSf, dh0, cu, num_seqs, total_T, Hqk, H, base, max_total, recs);
+        dO, dSf, dh0, cu, num_seqs, total_T, Hqk, H, base, max_total, recs);
     bwd_local_kernel<IoT><<<per_chunk, kLocalThreads, LB_SMEM, stream>>>(
         q, k, v, g, dO, cu, num_seqs, total_T, Hqk, H, base, recs, dq, dk, dv, dg, dbeta);
     return cudaGetLastError();
