@@ -40,6 +40,7 @@
 #include "common.cuh"
 #include "internal.h"
 #include "chunk_common.cuh"
+#include "tc_ptx.cuh"
 
 namespace gdr {
 namespace {
@@ -110,10 +111,11 @@ __device__ __forceinline__ void load_io_rows(float *dst, const IoT *src, int tok
 
 // The product tile of one thread: out(m, n) = sum_k a(m, k) b(k, n) for
 // rows m = gr + GR r and columns n = gc + GC c, (gr, gc) = (tid / GC, tid % GC),
-// GC = min(N, 16), GR = NT / GC; epi(m, n, value) takes each result.
-template <int M, int N, int NT, class AF, class BF, class EPI>
+// GC = min(N, 16) unless given, GR = NT / GC; epi(m, n, value) takes each
+// result.
+template <int M, int N, int NT, int GCX = 0, class AF, class BF, class EPI>
 __device__ __forceinline__ void gemm(int K, AF a, BF b, EPI epi) {
-    constexpr int GC = N < 16 ? N : 16;
+    constexpr int GC = GCX > 0 ? GCX : (N < 16 ? N : 16);
     constexpr int GR = NT / GC;
     constexpr int TM = M / GR, TN = N / GC;
     static_assert(GR * GC == NT && TM * GR == M && TN * GC == N, "product tiling");
@@ -337,12 +339,17 @@ bwd_forward_kernel(const float *__restrict__ h0,
             const int r = e >> 7, d = e & 127;
             rec[R_S + (size_t)(r0 + r) * D + d] = Sr[r * LW + d];
         }
+        if (tid == 0 && c + 1 < nch) {   // the next chunk's operands towards L2
+            const float *nx = rec + (size_t)H * R_FLOATS;
+            tc::bulk_prefetch_l2(nx + R_W, 2 * C * D * sizeof(float));   // W and U~
+            tc::bulk_prefetch_l2(nx + R_KH, C * D * sizeof(float));
+        }
         copy_rows<kChainThreadsB>(Ws, LW, rec + R_W, C, D);
         copy_rows<kChainThreadsB>(Kh, LW, rec + R_KH, C, D);
         if (tid < C) Gs[tid] = rec[R_G + tid];
         __syncthreads();
         // U[j][r0 + r] = U~[j][r0 + r] - sum_d W[j][d] S[r0 + r][d]
-        gemm<C, kRowBlock, kChainThreadsB>(D, [&](int j, int d) { return Ws[j * LW + d]; },
+        gemm<C, kRowBlock, kChainThreadsB, 4>(D, [&](int j, int d) { return Ws[j * LW + d]; },
                                            [&](int d, int r) { return Sr[r * LW + d]; },
                                            [&](int j, int r, float x) {
                                                const float u = rec[R_UT + j * D + r0 + r] - x;
@@ -385,6 +392,12 @@ bwd_reverse_kernel(const IoT *__restrict__ dO,
             const int r = e >> 7, d = e & 127;
             rec[R_L + (size_t)(r0 + r) * D + d] = Lr[r * LW + d];
         }
+        if (tid == 0 && c > 0) {   // the previous chunk's operands towards L2
+            const float *pv = rec - (size_t)H * R_FLOATS;
+            tc::bulk_prefetch_l2(pv + R_W, C * D * sizeof(float));
+            tc::bulk_prefetch_l2(pv + R_P, C * C * sizeof(float));
+            tc::bulk_prefetch_l2(pv + R_KH, 2 * C * D * sizeof(float));   // K^ and gamma Q
+        }
         copy_rows<kChainThreadsB>(Ws, LW, rec + R_W, C, D);
         copy_rows<kChainThreadsB>(Kh, LW, rec + R_KH, C, D);
         copy_rows<kChainThreadsB>(Qt, LW, rec + R_QT, C, D);
@@ -399,10 +412,10 @@ bwd_reverse_kernel(const IoT *__restrict__ dO,
         if (tid < C) Gs[tid] = rec[R_G + tid];
         __syncthreads();
         // dU[j][r] = sum_d K^[j][d] L[r][d] + sum_i P[i][j] dO[i][r]
-        gemm<C, kRowBlock, kChainThreadsB>(D, [&](int j, int d) { return Kh[j * LW + d]; },
+        gemm<C, kRowBlock, kChainThreadsB, 4>(D, [&](int j, int d) { return Kh[j * LW + d]; },
                                            [&](int d, int r) { return Lr[r * LW + d]; },
                                            [&](int j, int r, float x) { dUr[j * (kRowBlock + 1) + r] = x; });
-        gemm<C, kRowBlock, kChainThreadsB>(C, [&](int j, int i) { return Ps[i * LN + j]; },
+        gemm<C, kRowBlock, kChainThreadsB, 4>(C, [&](int j, int i) { return Ps[i * LN + j]; },
                                            [&](int i, int r) { return dOr[i * (kRowBlock + 1) + r]; },
                                            [&](int j, int r, float x) {
                                                const float du = dUr[j * (kRowBlock + 1) + r] + x;
