@@ -71,3 +71,29 @@ def test_backward_without_d_initial_state_and_repeatable_per_row_outputs():
     torch.cuda.synchronize()
     assert a[5] is None
     assert torch.equal(a[2], b[2])          # dv: written per row, no atomics
+
+
+@pytest.mark.parametrize("io", [torch.bfloat16, torch.float32])
+def test_chunked_and_token_forms_agree_with_the_oracle(io):
+    """Scalar gate, d = 128: with the workspace gdr_backward_workspace_size
+    reports the gradient takes the chunked form (chunk prep, forward and
+    reverse state chains, chunk-local gradients); with only the token loop's
+    checkpoints it takes the token loop.  Both against the oracle, on grouped
+    heads, an initial state, a final-state adjoint and sequences with partial
+    and single-token chunks."""
+    cu = [0, 70, 200, 201]
+    inp = I.make_inputs(total_T=cu[-1], H=4, H_qk=2, d_k=128, d_v=128, cu_seqlens=cu,
+                        gate_mode=I.SCALAR, io_dtype=io, c=0.1, h0_std=0.1, seed=86)
+    dO, dsf = I.make_grad_inputs(inp, seed=87, dsf_std=1.0)
+    d = lambda x: None if x is None else x.cuda()
+    ref = B.backward(inp.q, inp.k, inp.v, inp.g, inp.beta, inp.h0, inp.cu_seqlens.numpy(), dO, dsf)
+    full = gdr.gdr_backward_workspace_size(3, cu[-1], 4, 128, 128)
+    token = (3 + (cu[-1] + 15) // 16) * 4 * 128 * 128 * 4
+    assert full > token
+    for nbytes in (full, token):
+        ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+        got = gdr.gdr_backward(d(inp.q), d(inp.k), d(inp.v), d(inp.g), d(inp.beta), d(inp.h0),
+                               d(inp.cu_seqlens), d_o=d(dO), d_final_state=d(dsf), workspace=ws)
+        torch.cuda.synchronize()
+        for x, name in zip(got, ("dq", "dk", "dv", "dg", "dbeta", "dh0")):
+            _check(x, ref[name], f"{name} ({nbytes} workspace bytes)")
