@@ -777,9 +777,10 @@ def bench_case(case, args, ws, rank, flush, stream, pk, pk_kind):
         del graph
     value, ms = aggregate_throughput(case.tokens, sum(times) / len(times), ws)
     tokens_all = case.tokens * ws
-    # decode: bytes per launch over the time per launch; prefill: the whole
-    # step's bytes (every kernel of the plan) over the step time
-    launch_ms = ms if case.kind == "prefill" else ms / case.launches
+    # decode and the prologue: bytes per launch over the time per launch;
+    # prefill and the chunked gradient: the whole step's bytes (every kernel of
+    # the plan) over the step time
+    launch_ms = ms if case.kind in ("prefill", "backward") else ms / case.launches
     achieved = case.bytes / (launch_ms / 1e3) / 1e9
     hbm_peak = float(pk["hbm_gbs"])
     roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
