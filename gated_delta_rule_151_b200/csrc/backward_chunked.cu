@@ -48,7 +48,7 @@ namespace {
 // per (chunk, head) record of floats
 constexpr size_t R_W = 0;                       // W [64][128]
 constexpr size_t R_UT = R_W + C * D;            // U~ [64][128]
-constexpr size_t R_P = R_UT + C * D;            // P [64][64], causal
+constexpr size_t R_P = R_UT + C * D;            // P^T [64][64] (P causal)
 constexpr size_t R_T = R_P + C * C;             // T [64][64], lower with the unit diagonal
 constexpr size_t R_AR = R_T + C * C;            // (K K^T) o R [64][64], strictly lower
 constexpr size_t R_G = R_AR + C * C;            // G [64] (the chunk's cumulative log-gate)
@@ -65,8 +65,8 @@ constexpr size_t kBaseBytes = 256;              // sequence chunk offsets preced
 constexpr int LW = D + 1;    // padded row of 128 floats
 constexpr int LN = C + 1;    // padded row of 64 floats
 constexpr int kRowBlock = 16;                   // state rows per forward / reverse CTA
-constexpr int kChainThreadsB = 128;
 constexpr int kLocalThreads = 256;
+constexpr int kLocTM = C / (kLocalThreads / 16), kLocTN = D / 16;   // <C, D> product tile
 
 // rows x cols fp32 (cols a multiple of 4, 16-byte aligned) from the record
 // into padded shared rows of `ld` floats: 16-byte loads, eight in flight per
@@ -141,6 +141,39 @@ __device__ __forceinline__ void gemm(int K, AF a, BF b, EPI epi) {
     for (int r = 0; r < TM; ++r)
 #pragma unroll
         for (int c = 0; c < TN; ++c) epi(gr + GR * r, gc + GC * c, acc[r][c]);
+}
+
+// The same tile, its results handed to epi(r, c, m, n, value) with (r, c) the
+// tile position, so that a caller can keep per-thread sums over several
+// products (every <M, N, NT> product maps (m, n) to the same thread and slot).
+template <int M, int N, int NT, class AF, class BF, class EPI>
+__device__ __forceinline__ void gemm_rc(int K, AF a, BF b, EPI epi) {
+    constexpr int GC = N < 16 ? N : 16;
+    constexpr int GR = NT / GC;
+    constexpr int TM = M / GR, TN = N / GC;
+    static_assert(GR * GC == NT && TM * GR == M && TN * GC == N, "product tiling");
+    const int tid = threadIdx.x, gr = tid / GC, gc = tid % GC;
+    float acc[TM][TN];
+#pragma unroll
+    for (int r = 0; r < TM; ++r)
+#pragma unroll
+        for (int c = 0; c < TN; ++c) acc[r][c] = 0.f;
+#pragma unroll 4
+    for (int k = 0; k < K; ++k) {
+        float av[TM], bv[TN];
+#pragma unroll
+        for (int r = 0; r < TM; ++r) av[r] = a(gr + GR * r, k);
+#pragma unroll
+        for (int c = 0; c < TN; ++c) bv[c] = b(k, gc + GC * c);
+#pragma unroll
+        for (int r = 0; r < TM; ++r)
+#pragma unroll
+            for (int c = 0; c < TN; ++c) acc[r][c] = fmaf(av[r], bv[c], acc[r][c]);
+    }
+#pragma unroll
+    for (int r = 0; r < TM; ++r)
+#pragma unroll
+        for (int c = 0; c < TN; ++c) epi(r, c, gr + GR * r, gc + GC * c, acc[r][c]);
 }
 
 // base[n] = first global chunk of sequence n (exclusive prefix sum of the
@@ -265,7 +298,7 @@ bwd_prep_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT 
     gemm<C, C, kPrepB>(D, [&](int i, int d) { return Qs[i * LW + d]; },
                        [&](int d, int j) { return Ks[j * LW + d]; },
                        [&](int i, int j, float x) {
-                           rec[R_P + i * C + j] = j <= i ? x * __expf(Gs[i] - Gs[j]) : 0.f;
+                           rec[R_P + j * C + i] = j <= i ? x * __expf(Gs[i] - Gs[j]) : 0.f;
                        });
     __syncthreads();
     unit_lower_inverse_f32(Af, fs + PB_T, fs + PB_X, tid);   // ends synchronised
@@ -300,25 +333,118 @@ bwd_prep_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT 
 }
 
 // ------------------------------------------------------ forward / reverse ----
-// One CTA per (sequence, value head, block of 16 state rows); the rows of
-// the state and of its adjoint are independent, so the CTAs of a chain share
-// nothing.  Shared memory (floats): the rows [16][129], two [64][129]
-// operands, one [64][65] operand and [64][17] row-block columns.
-constexpr uint32_t CB_ROWS = 0;                          // S or L rows [16][129]
-constexpr uint32_t CB_M1 = CB_ROWS + kRowBlock * LW;      // [64][129]
-constexpr uint32_t CB_M2 = CB_M1 + C * LW;                // [64][129]
-constexpr uint32_t CB_M3 = CB_M2 + C * LW;                // [64][129]
-constexpr uint32_t CB_P = CB_M3 + C * LW;                 // [64][65]
-constexpr uint32_t CB_C1 = CB_P + C * LN;                 // [64][17]
-constexpr uint32_t CB_C2 = CB_C1 + C * (kRowBlock + 1);   // [64][17]
-constexpr uint32_t CB_G = CB_C2 + C * (kRowBlock + 1);    // G [64]
-constexpr uint32_t CB_FLOATS = CB_G + C;
-constexpr uint32_t CB_SMEM = CB_FLOATS * sizeof(float);
+// One CTA of 256 threads per (sequence, value head, block of 16 state rows);
+// the rows of the state and of its adjoint are independent, so the CTAs of a
+// chain share nothing.  Each chunk takes two products over operands staged
+// in shared memory by 16-byte asynchronous copies.  An operand is reloaded
+// for the next chunk as soon as its product is done, so that its copy runs
+// during the other product and the next chunk's first one.  Rows are padded
+// to 132 or 68 floats: 16-byte aligned for the copies, and the float4 reads
+// of 8 different rows by a quarter warp fall in 8 different bank groups.
+constexpr int kChainThreads = 256;
+constexpr int LW4 = D + 4;
+constexpr int LN4 = C + 4;
+static_assert(kChainThreads == C * 4, "one 16-byte piece of a column strip per thread");
 
-__global__ void __launch_bounds__(kChainThreadsB, 1)
-bwd_forward_kernel(const float *__restrict__ h0,
-                   const int32_t *__restrict__ cu, int num_seqs, int total_T, int Hqk, int H,
-                   const int32_t *__restrict__ base, long long slots, float *__restrict__ recs) {
+__device__ __forceinline__ void cp16(void *dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(tc::smem_u32(dst)), "l"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N> __device__ __forceinline__ void cp_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// 64 x 128 floats of a record field into rows of LW4 floats.
+__device__ __forceinline__ void stage_c_by_d(float *dst, const float *src) {
+#pragma unroll 8
+    for (int e = threadIdx.x; e < C * D / 4; e += kChainThreads)
+        cp16(dst + (e >> 5) * LW4 + (e & 31) * 4, src + e * 4);
+}
+// 64 x 64 floats into rows of LN4 floats.
+__device__ __forceinline__ void stage_c_by_c(float *dst, const float *src) {
+#pragma unroll 4
+    for (int e = threadIdx.x; e < C * C / 4; e += kChainThreads)
+        cp16(dst + (e >> 4) * LN4 + (e & 15) * 4, src + e * 4);
+}
+// Columns r0 .. r0 + 15 of a 64 x 128 record field into rows of 16 floats.
+__device__ __forceinline__ void stage_strip(float *dst, const float *src, int r0) {
+    const int e = threadIdx.x;
+    cp16(dst + (e >> 2) * kRowBlock + (e & 3) * 4, src + (e >> 2) * D + r0 + (e & 3) * 4);
+}
+// The chunk's 64 floats of G.
+__device__ __forceinline__ void stage_g(float *dst, const float *src) {
+    if (threadIdx.x < C / 4) cp16(dst + threadIdx.x * 4, src + threadIdx.x * 4);
+}
+
+__device__ __forceinline__ float4 lds4(const float *p) { return *reinterpret_cast<const float4 *>(p); }
+__device__ __forceinline__ float dot4(float4 a, float4 b, float c) {
+    return fmaf(a.w, b.w, fmaf(a.z, b.z, fmaf(a.y, b.y, fmaf(a.x, b.x, c))));
+}
+
+// 64 x 16 product with both operands read along K: acc[t][u] += sum_k
+// A[j][k] B[r][k] for j = gr + 32 t, r = gc + 8 u, (gr, gc) = (tid / 8, tid % 8).
+__device__ __forceinline__ void prod_narrow(float (&acc)[2][2], const float *A, int lda,
+                                            const float *B, int ldb, int K) {
+    const int gr = threadIdx.x >> 3, gc = threadIdx.x & 7;
+    const float *a0 = A + gr * lda, *a1 = A + (gr + 32) * lda;
+    const float *b0 = B + gc * ldb, *b1 = B + (gc + 8) * ldb;
+#pragma unroll 4
+    for (int k = 0; k < K; k += 4) {
+        const float4 x0 = lds4(a0 + k), x1 = lds4(a1 + k), y0 = lds4(b0 + k), y1 = lds4(b1 + k);
+        acc[0][0] = dot4(x0, y0, acc[0][0]);
+        acc[0][1] = dot4(x0, y1, acc[0][1]);
+        acc[1][0] = dot4(x1, y0, acc[1][0]);
+        acc[1][1] = dot4(x1, y1, acc[1][1]);
+    }
+}
+
+// 16 x 128 product: acc[t][e] += sum_k A[r][k] B[k][4 gc + e] for
+// r = gr + 8 t, (gr, gc) = (tid / 32, tid % 32).
+__device__ __forceinline__ void prod_wide(float (&acc)[2][4], const float *A, int lda,
+                                          const float *B, int ldb, int K) {
+    const int gr = threadIdx.x >> 5, gc = threadIdx.x & 31;
+    const float *a0 = A + gr * lda, *a1 = A + (gr + 8) * lda, *b = B + 4 * gc;
+#pragma unroll 2
+    for (int k = 0; k < K; k += 4) {
+        const float4 x0 = lds4(a0 + k), x1 = lds4(a1 + k);
+        const float xa[4] = {x0.x, x0.y, x0.z, x0.w}, xb[4] = {x1.x, x1.y, x1.z, x1.w};
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+            const float4 y = lds4(b + (k + kk) * ldb);
+            acc[0][0] = fmaf(xa[kk], y.x, acc[0][0]);
+            acc[0][1] = fmaf(xa[kk], y.y, acc[0][1]);
+            acc[0][2] = fmaf(xa[kk], y.z, acc[0][2]);
+            acc[0][3] = fmaf(xa[kk], y.w, acc[0][3]);
+            acc[1][0] = fmaf(xb[kk], y.x, acc[1][0]);
+            acc[1][1] = fmaf(xb[kk], y.y, acc[1][1]);
+            acc[1][2] = fmaf(xb[kk], y.z, acc[1][2]);
+            acc[1][3] = fmaf(xb[kk], y.w, acc[1][3]);
+        }
+    }
+}
+
+// The CTA's 16 rows (padded) -> rows r0 .. r0 + 15 of a [128][128] field.
+__device__ __forceinline__ void store_rows(float *dst, const float *rows, int r0) {
+#pragma unroll
+    for (int e = threadIdx.x; e < kRowBlock * D / 4; e += kChainThreads) {
+        const int r = e >> 5, q = e & 31;
+        *reinterpret_cast<float4 *>(dst + (size_t)(r0 + r) * D + 4 * q) = lds4(rows + r * LW4 + 4 * q);
+    }
+}
+
+constexpr uint32_t CF_S = 0;                             // S rows [16][LW4]
+constexpr uint32_t CF_UT = CF_S + kRowBlock * LW4;       // U^T [16][LN4]
+constexpr uint32_t CF_W = CF_UT + kRowBlock * LN4;       // W [64][LW4]
+constexpr uint32_t CF_KH = CF_W + C * LW4;               // K^ [64][LW4]
+constexpr uint32_t CF_US = CF_KH + C * LW4;              // U~ columns r0 .. r0 + 15 [64][16]
+constexpr uint32_t CF_G = CF_US + C * kRowBlock;         // G [64]
+constexpr uint32_t CF_SMEM = (CF_G + C) * sizeof(float);
+
+__global__ void __launch_bounds__(kChainThreads, 1)
+bwd_forward_kernel(const float *__restrict__ h0, const int32_t *__restrict__ cu, int num_seqs,
+                   int total_T, int H, const int32_t *__restrict__ base, long long slots,
+                   float *__restrict__ recs) {
     extern __shared__ __align__(16) float fs[];
     const int chain = blockIdx.x, h = chain % H, n = chain / H, r0 = blockIdx.y * kRowBlock;
     const int tid = threadIdx.x;
@@ -327,50 +453,90 @@ bwd_forward_kernel(const float *__restrict__ h0,
     const int b0 = base[n];
     // a malformed cu_seqlens can claim more chunks than the records hold
     const int nch = (int)min((long long)(len + C - 1) / C, max(slots - b0, 0ll));
-    float *Sr = fs + CB_ROWS, *Ws = fs + CB_M1, *Kh = fs + CB_M2, *Us = fs + CB_C1, *Gs = fs + CB_G;
-    for (int e = tid; e < kRowBlock * D; e += kChainThreadsB) {
+    float *Sr = fs + CF_S, *Ut = fs + CF_UT, *Ws = fs + CF_W, *Kh = fs + CF_KH, *Us = fs + CF_US,
+          *Gs = fs + CF_G;
+    auto rec_of = [&](int c) { return recs + ((size_t)(b0 + c) * H + h) * R_FLOATS; };
+    for (int e = tid; e < kRowBlock * D; e += kChainThreads) {
         const int r = e >> 7, d = e & 127;
-        Sr[r * LW + d] = h0 != nullptr ? h0[((size_t)chain * D + r0 + r) * D + d] : 0.f;
+        Sr[r * LW4 + d] = h0 != nullptr ? h0[((size_t)chain * D + r0 + r) * D + d] : 0.f;
     }
+    // copy groups, in order: {W, U~} and {K^, G} of every chunk
+    if (nch > 0) {
+        stage_c_by_d(Ws, rec_of(0) + R_W);
+        stage_strip(Us, rec_of(0) + R_UT, r0);
+        cp_commit();
+        stage_c_by_d(Kh, rec_of(0) + R_KH);
+        stage_g(Gs, rec_of(0) + R_G);
+        cp_commit();
+    }
+    const int gr1 = tid >> 3, gc1 = tid & 7, gr2 = tid >> 5, gc2 = tid & 31;
     for (int c = 0; c < nch; ++c) {
-        float *rec = recs + ((size_t)(b0 + c) * H + h) * R_FLOATS;
-        __syncthreads();   // the rows of the last chunk's update are in place
-        for (int e = tid; e < kRowBlock * D; e += kChainThreadsB) {
-            const int r = e >> 7, d = e & 127;
-            rec[R_S + (size_t)(r0 + r) * D + d] = Sr[r * LW + d];
+        float *rec = rec_of(c);
+        cp_wait<1>();
+        __syncthreads();   // W, U~ of chunk c and the state rows in place
+        store_rows(rec + R_S, Sr, r0);
+        {   // U[j][r0 + r] = U~[j][r0 + r] - sum_d W[j][d] S[r][d]
+            float acc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+            prod_narrow(acc, Ws, LW4, Sr, LW4, D);
+#pragma unroll
+            for (int t = 0; t < 2; ++t)
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const int j = gr1 + 32 * t, r = gc1 + 8 * u;
+                    const float x = Us[j * kRowBlock + r] - acc[t][u];
+                    Ut[r * LN4 + j] = x;
+                    rec[R_U + j * D + r0 + r] = x;
+                }
         }
-        if (tid == 0 && c + 1 < nch) {   // the next chunk's operands towards L2
-            const float *nx = rec + (size_t)H * R_FLOATS;
-            tc::bulk_prefetch_l2(nx + R_W, 2 * C * D * sizeof(float));   // W and U~
-            tc::bulk_prefetch_l2(nx + R_KH, C * D * sizeof(float));
+        __syncthreads();   // W and U~ consumed, U^T complete
+        if (c + 1 < nch) {
+            stage_c_by_d(Ws, rec_of(c + 1) + R_W);
+            stage_strip(Us, rec_of(c + 1) + R_UT, r0);
         }
-        copy_rows<kChainThreadsB>(Ws, LW, rec + R_W, C, D);
-        copy_rows<kChainThreadsB>(Kh, LW, rec + R_KH, C, D);
-        if (tid < C) Gs[tid] = rec[R_G + tid];
-        __syncthreads();
-        // U[j][r0 + r] = U~[j][r0 + r] - sum_d W[j][d] S[r0 + r][d]
-        gemm<C, kRowBlock, kChainThreadsB, 4>(D, [&](int j, int d) { return Ws[j * LW + d]; },
-                                           [&](int d, int r) { return Sr[r * LW + d]; },
-                                           [&](int j, int r, float x) {
-                                               const float u = rec[R_UT + j * D + r0 + r] - x;
-                                               Us[j * (kRowBlock + 1) + r] = u;
-                                               rec[R_U + j * D + r0 + r] = u;
-                                           });
-        __syncthreads();
-        // S[r][d] = e^{G_C} S[r][d] + sum_j U[j][r] K^[j][d]
-        const float gC = __expf(Gs[C - 1]);
-        gemm<kRowBlock, D, kChainThreadsB>(C, [&](int r, int j) { return Us[j * (kRowBlock + 1) + r]; },
-                                           [&](int j, int d) { return Kh[j * LW + d]; },
-                                           [&](int r, int d, float x) { Sr[r * LW + d] = fmaf(gC, Sr[r * LW + d], x); });
+        cp_commit();
+        cp_wait<1>();
+        __syncthreads();   // K^ and G of chunk c in place
+        {   // S[r][d] = e^{G_C} S[r][d] + sum_j U[j][r] K^[j][d]
+            float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+            prod_wide(acc, Ut, LN4, Kh, LW4, C);
+            const float gC = __expf(Gs[C - 1]);
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+                float4 *p = reinterpret_cast<float4 *>(Sr + (gr2 + 8 * t) * LW4 + 4 * gc2);
+                float4 s = *p;
+                s.x = fmaf(gC, s.x, acc[t][0]);
+                s.y = fmaf(gC, s.y, acc[t][1]);
+                s.z = fmaf(gC, s.z, acc[t][2]);
+                s.w = fmaf(gC, s.w, acc[t][3]);
+                *p = s;
+            }
+        }
+        __syncthreads();   // K^ and G consumed
+        if (c + 1 < nch) {
+            stage_c_by_d(Kh, rec_of(c + 1) + R_KH);
+            stage_g(Gs, rec_of(c + 1) + R_G);
+        }
+        cp_commit();
     }
+    cp_wait<0>();
 }
 
+constexpr uint32_t CR_L = 0;                             // L rows [16][LW4]
+constexpr uint32_t CR_DUT = CR_L + kRowBlock * LW4;      // dU^T [16][LN4]
+constexpr uint32_t CR_DOT = CR_DUT + kRowBlock * LN4;    // dO^T, columns r0 .. r0 + 15 [16][LN4]
+constexpr uint32_t CR_KH = CR_DOT + kRowBlock * LN4;     // K^ [64][LW4]
+constexpr uint32_t CR_PT = CR_KH + C * LW4;              // P^T [64][LN4]
+constexpr uint32_t CR_QT = CR_PT + C * LN4;              // diag(gamma) Q [64][LW4]
+constexpr uint32_t CR_W = CR_QT + C * LW4;               // W [64][LW4]
+constexpr uint32_t CR_G = CR_W + C * LW4;                // G [64]
+constexpr uint32_t CR_SMEM = (CR_G + C) * sizeof(float);
+
 template <typename IoT>
-__global__ void __launch_bounds__(kChainThreadsB, 1)
-bwd_reverse_kernel(const IoT *__restrict__ dO,
-                   const float *__restrict__ dSf, float *__restrict__ dh0,
-                   const int32_t *__restrict__ cu, int num_seqs, int total_T, int Hqk, int H,
-                   const int32_t *__restrict__ base, long long slots, float *__restrict__ recs) {
+__global__ void __launch_bounds__(kChainThreads, 1)
+bwd_reverse_kernel(const IoT *__restrict__ dO, const float *__restrict__ dSf,
+                   float *__restrict__ dh0, const int32_t *__restrict__ cu, int num_seqs,
+                   int total_T, int H, const int32_t *__restrict__ base, long long slots,
+                   float *__restrict__ recs) {
     extern __shared__ __align__(16) float fs[];
     const int chain = blockIdx.x, h = chain % H, n = chain / H, r0 = blockIdx.y * kRowBlock;
     const int tid = threadIdx.x;
@@ -378,65 +544,98 @@ bwd_reverse_kernel(const IoT *__restrict__ dO,
     sequence_range(cu, n, num_seqs, total_T, t0, len);
     const int b0 = base[n];
     const int nch = (int)min((long long)(len + C - 1) / C, max(slots - b0, 0ll));
-    float *Lr = fs + CB_ROWS, *Ws = fs + CB_M1, *Kh = fs + CB_M2, *Qt = fs + CB_M3, *Ps = fs + CB_P;
-    float *dOr = fs + CB_C1, *dUr = fs + CB_C2, *Gs = fs + CB_G;
-    for (int e = tid; e < kRowBlock * D; e += kChainThreadsB) {
-        const int r = e >> 7, d = e & 127;
-        Lr[r * LW + d] = dSf != nullptr ? dSf[((size_t)chain * D + r0 + r) * D + d] : 0.f;
-    }
-    for (int c = nch - 1; c >= 0; --c) {
-        float *rec = recs + ((size_t)(b0 + c) * H + h) * R_FLOATS;
-        const int tok0 = t0 + c * C, cl = min(C, len - c * C);
-        __syncthreads();
-        for (int e = tid; e < kRowBlock * D; e += kChainThreadsB) {
-            const int r = e >> 7, d = e & 127;
-            rec[R_L + (size_t)(r0 + r) * D + d] = Lr[r * LW + d];
-        }
-        if (tid == 0 && c > 0) {   // the previous chunk's operands towards L2
-            const float *pv = rec - (size_t)H * R_FLOATS;
-            tc::bulk_prefetch_l2(pv + R_W, C * D * sizeof(float));
-            tc::bulk_prefetch_l2(pv + R_P, C * C * sizeof(float));
-            tc::bulk_prefetch_l2(pv + R_KH, 2 * C * D * sizeof(float));   // K^ and gamma Q
-        }
-        copy_rows<kChainThreadsB>(Ws, LW, rec + R_W, C, D);
-        copy_rows<kChainThreadsB>(Kh, LW, rec + R_KH, C, D);
-        copy_rows<kChainThreadsB>(Qt, LW, rec + R_QT, C, D);
-        copy_rows<kChainThreadsB>(Ps, LN, rec + R_P, C, C);
-        for (int e = tid; e < C * kRowBlock / 4; e += kChainThreadsB) {   // dO[:, r0 .. r0 + 15]
-            const int i = e >> 2, r = (e & 3) * 4;
-            float x[4] = {0.f, 0.f, 0.f, 0.f};
-            if (i < cl) ld4io(dO + ((size_t)(tok0 + i) * H + h) * D + r0 + r, x);
+    float *Lr = fs + CR_L, *dUt = fs + CR_DUT, *dOt = fs + CR_DOT, *Kh = fs + CR_KH,
+          *PT = fs + CR_PT, *Qt = fs + CR_QT, *Ws = fs + CR_W, *Gs = fs + CR_G;
+    auto rec_of = [&](int c) { return recs + ((size_t)(b0 + c) * H + h) * R_FLOATS; };
+    // dO[i][r0 + 4 e .. r0 + 4 e + 3] of chunk c, i = tid / 4, e = tid % 4 (0
+    // past the sequence's end), and its place in dO^T
+    const int di = tid >> 2, dr = (tid & 3) * 4;
+    auto load_dO = [&](int c, float (&x)[4]) {
+        x[0] = x[1] = x[2] = x[3] = 0.f;
+        if (di < min(C, len - c * C)) ld4io(dO + ((size_t)(t0 + c * C + di) * H + h) * D + r0 + dr, x);
+    };
+    auto put_dO = [&](const float (&x)[4]) {
 #pragma unroll
-            for (int u = 0; u < 4; ++u) dOr[i * (kRowBlock + 1) + r + u] = x[u];
-        }
-        if (tid < C) Gs[tid] = rec[R_G + tid];
-        __syncthreads();
-        // dU[j][r] = sum_d K^[j][d] L[r][d] + sum_i P[i][j] dO[i][r]
-        gemm<C, kRowBlock, kChainThreadsB, 4>(D, [&](int j, int d) { return Kh[j * LW + d]; },
-                                           [&](int d, int r) { return Lr[r * LW + d]; },
-                                           [&](int j, int r, float x) { dUr[j * (kRowBlock + 1) + r] = x; });
-        gemm<C, kRowBlock, kChainThreadsB, 4>(C, [&](int j, int i) { return Ps[i * LN + j]; },
-                                           [&](int i, int r) { return dOr[i * (kRowBlock + 1) + r]; },
-                                           [&](int j, int r, float x) {
-                                               const float du = dUr[j * (kRowBlock + 1) + r] + x;
-                                               dUr[j * (kRowBlock + 1) + r] = du;
-                                               rec[R_DU + j * D + r0 + r] = du;
-                                           });
-        __syncthreads();
-        // L[r][d] = e^{G_C} L[r][d] + sum_i dO[i][r] gamma_i q_i[d] - sum_j dU[j][r] W[j][d]
-        const float gC = __expf(Gs[C - 1]);
-        gemm<kRowBlock, D, kChainThreadsB>(C, [&](int r, int i) { return dOr[i * (kRowBlock + 1) + r]; },
-                                           [&](int i, int d) { return Qt[i * LW + d]; },
-                                           [&](int r, int d, float x) { Lr[r * LW + d] = fmaf(gC, Lr[r * LW + d], x); });
-        gemm<kRowBlock, D, kChainThreadsB>(C, [&](int r, int j) { return dUr[j * (kRowBlock + 1) + r]; },
-                                           [&](int j, int d) { return Ws[j * LW + d]; },
-                                           [&](int r, int d, float x) { Lr[r * LW + d] -= x; });
+        for (int u = 0; u < 4; ++u) dOt[(dr + u) * LN4 + di] = x[u];
+    };
+    for (int e = tid; e < kRowBlock * D; e += kChainThreads) {
+        const int r = e >> 7, d = e & 127;
+        Lr[r * LW4 + d] = dSf != nullptr ? dSf[((size_t)chain * D + r0 + r) * D + d] : 0.f;
     }
+    // copy groups, in order: {K^, P^T} and {gamma Q, W, G} of every chunk
+    if (nch > 0) {
+        stage_c_by_d(Kh, rec_of(nch - 1) + R_KH);
+        stage_c_by_c(PT, rec_of(nch - 1) + R_P);
+        cp_commit();
+        stage_c_by_d(Qt, rec_of(nch - 1) + R_QT);
+        stage_c_by_d(Ws, rec_of(nch - 1) + R_W);
+        stage_g(Gs, rec_of(nch - 1) + R_G);
+        cp_commit();
+        float x[4];
+        load_dO(nch - 1, x);
+        put_dO(x);
+    }
+    const int gr1 = tid >> 3, gc1 = tid & 7, gr2 = tid >> 5, gc2 = tid & 31;
+    for (int c = nch - 1; c >= 0; --c) {
+        float *rec = rec_of(c);
+        cp_wait<1>();
+        __syncthreads();   // K^, P^T, dO^T of chunk c and the adjoint rows in place
+        store_rows(rec + R_L, Lr, r0);
+        {   // dU[j][r] = sum_d K^[j][d] L[r][d] + sum_i P[i][j] dO[i][r]
+            float acc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+            prod_narrow(acc, Kh, LW4, Lr, LW4, D);
+            prod_narrow(acc, PT, LN4, dOt, LN4, C);
+#pragma unroll
+            for (int t = 0; t < 2; ++t)
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const int j = gr1 + 32 * t, r = gc1 + 8 * u;
+                    dUt[r * LN4 + j] = acc[t][u];
+                    rec[R_DU + j * D + r0 + r] = acc[t][u];
+                }
+        }
+        __syncthreads();   // K^ and P^T consumed, dU^T complete
+        float x[4] = {0.f, 0.f, 0.f, 0.f};
+        if (c > 0) {
+            stage_c_by_d(Kh, rec_of(c - 1) + R_KH);
+            stage_c_by_c(PT, rec_of(c - 1) + R_P);
+            load_dO(c - 1, x);
+        }
+        cp_commit();
+        cp_wait<1>();
+        __syncthreads();   // gamma Q, W and G of chunk c in place
+        {   // L[r][d] = e^{G_C} L[r][d] + sum_i dO[i][r] gamma_i q_i[d] - sum_j dU[j][r] W[j][d]
+            float a1[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+            float a2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+            prod_wide(a1, dOt, LN4, Qt, LW4, C);
+            prod_wide(a2, dUt, LN4, Ws, LW4, C);
+            const float gC = __expf(Gs[C - 1]);
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+                float4 *p = reinterpret_cast<float4 *>(Lr + (gr2 + 8 * t) * LW4 + 4 * gc2);
+                float4 s = *p;
+                s.x = fmaf(gC, s.x, a1[t][0] - a2[t][0]);
+                s.y = fmaf(gC, s.y, a1[t][1] - a2[t][1]);
+                s.z = fmaf(gC, s.z, a1[t][2] - a2[t][2]);
+                s.w = fmaf(gC, s.w, a1[t][3] - a2[t][3]);
+                *p = s;
+            }
+        }
+        __syncthreads();   // gamma Q, W, G and dO^T consumed
+        if (c > 0) {
+            stage_c_by_d(Qt, rec_of(c - 1) + R_QT);
+            stage_c_by_d(Ws, rec_of(c - 1) + R_W);
+            stage_g(Gs, rec_of(c - 1) + R_G);
+            put_dO(x);
+        }
+        cp_commit();
+    }
+    cp_wait<0>();
     __syncthreads();
     if (dh0 != nullptr) {
-        for (int e = tid; e < kRowBlock * D; e += kChainThreadsB) {
+        for (int e = tid; e < kRowBlock * D; e += kChainThreads) {
             const int r = e >> 7, d = e & 127;
-            dh0[((size_t)chain * D + r0 + r) * D + d] = Lr[r * LW + d];
+            dh0[((size_t)chain * D + r0 + r) * D + d] = Lr[r * LW4 + d];
         }
     }
 }
@@ -483,6 +682,25 @@ bwd_local_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT
     float *Gs = fs + LB_G, *gam = Gs + C, *Bs = gam + C, *dG = Bs + C, *dB = dG + C;
     float *misc = fs + LB_MISC;
     auto qk_at = [&](float *base_, int i, int d) { return base_ + ((size_t)(tok0 + i) * Hqk + hq) * D + d; };
+    // dk and dq of the chunk's rows, summed over the product terms in the
+    // registers of the <C, D> product tile (rows gr + 16 r, columns gc + 16 c)
+    float dkacc[kLocTM][kLocTN], dqacc[kLocTM][kLocTN];
+    // everything the later phases read towards L2 while phase A runs: the
+    // record's P, T, (K K^T) o R, G, beta and U .. gamma Q (64 KiB pieces),
+    // and the chunk's rows of q, k, v and dO
+    if (tid == 0) {
+        tc::bulk_prefetch_l2(rec + R_P, (3 * C * C + 2 * C) * sizeof(float));
+        for (size_t o = R_U; o < R_FLOATS; o += 16384)
+            tc::bulk_prefetch_l2(rec + o, (uint32_t)(min((size_t)16384, R_FLOATS - o) * sizeof(float)));
+    } else if (tid >= 64 && tid < 64 + 3 * C) {
+        const int w = (tid - 64) / C, i = (tid - 64) % C;
+        if (i < cl) {
+            const IoT *src = w == 0 ? q + ((size_t)(tok0 + i) * Hqk + hq) * D
+                           : w == 1 ? k + ((size_t)(tok0 + i) * Hqk + hq) * D
+                                    : v + ((size_t)(tok0 + i) * H + h) * D;
+            tc::bulk_prefetch_l2(src, D * sizeof(IoT));
+        }
+    }
 
     // ---- phase A: dK^ = U L' and <S, L'> --------------------------------------
     copy_rows<kLocalThreads>(RA, LW, rec + R_L, D, D);
@@ -508,10 +726,10 @@ bwd_local_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT
     __syncthreads();
     {
         float rowacc[4] = {0.f, 0.f, 0.f, 0.f}, gcacc = 0.f;
-        gemm<C, D, kLocalThreads>(D, [&](int j, int r) { return RB[j * LW + r]; },
+        gemm_rc<C, D, kLocalThreads>(D, [&](int j, int r) { return RB[j * LW + r]; },
                                   [&](int r, int d) { return RA[r * LW + d]; },
-                                  [&](int j, int d, float x) {
-                                      if (j < cl) atomicAdd(qk_at(dk, j, d), __expf(GC - Gs[j]) * x);
+                                  [&](int tr, int tc, int j, int d, float x) {
+                                      dkacc[tr][tc] = __expf(GC - Gs[j]) * x;
                                       const float t = RC[j * LW + d] * x;
                                       rowacc[j >> 4] -= t;   // rows j = gr + 16 r
                                       gcacc += t;
@@ -533,13 +751,11 @@ bwd_local_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT
                               [&](int j, int d, float x) { RC[j * LW + d] = -x; });
     {
         float rowacc[4] = {0.f, 0.f, 0.f, 0.f};
-        gemm<C, D, kLocalThreads>(D, [&](int i, int r) { return RD[i * LW + r]; },
+        gemm_rc<C, D, kLocalThreads>(D, [&](int i, int r) { return RD[i * LW + r]; },
                                   [&](int r, int d) { return RA[r * LW + d]; },
-                                  [&](int i, int d, float x) {
-                                      if (i < cl) {
-                                          atomicAdd(qk_at(dq, i, d), gam[i] * x);
-                                          rowacc[i >> 4] += rec[R_QT + i * D + d] * x;
-                                      }
+                                  [&](int tr, int tc, int i, int d, float x) {
+                                      dqacc[tr][tc] = gam[i] * x;
+                                      if (i < cl) rowacc[i >> 4] += rec[R_QT + i * D + d] * x;
                                   });
         const int gr = tid >> 4;
 #pragma unroll
@@ -572,10 +788,10 @@ bwd_local_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT
     }
     {
         float bacc[4] = {0.f, 0.f, 0.f, 0.f}, gacc[4] = {0.f, 0.f, 0.f, 0.f};
-        gemm<C, D, kLocalThreads>(C, [&](int j, int i) { return N1[i * LN + j]; },
+        gemm_rc<C, D, kLocalThreads>(C, [&](int j, int i) { return N1[i * LN + j]; },
                                   [&](int i, int d) { return RC[i * LW + d]; },
-                                  [&](int j, int d, float x) {
-                                      if (j < cl) atomicAdd(qk_at(dk, j, d), Bs[j] * gam[j] * x);
+                                  [&](int tr, int tc, int j, int d, float x) {
+                                      dkacc[tr][tc] += Bs[j] * gam[j] * x;
                                       const float t = RA[j * LW + d] * x;
                                       bacc[j >> 4] += gam[j] * t;
                                       gacc[j >> 4] += Bs[j] * gam[j] * t;
@@ -614,7 +830,7 @@ bwd_local_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT
         const float R = j <= i ? __expf(Gs[i] - Gs[j]) : 0.f;
         const float da = N3[i * LN + j], ar = AR[i * LN + j];
         const float ea = da * Bs[i] * ar;            // dA o A
-        const float dp = N2[i * LN + j], ep = dp * N1[i * LN + j];   // dP o P
+        const float dp = N2[i * LN + j], ep = dp * N1[j * LN + i];   // dP o P (N1 holds P^T)
         if (da != 0.f || dp != 0.f) {
             atomicAdd(&dB[i], da * ar);
             atomicAdd(&dG[i], ea + ep);
@@ -625,18 +841,38 @@ bwd_local_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT
     }
     load_io_rows<kLocalThreads>(RB, q, tok0, cl, Hqk, hq);   // Q rows over the finished Y
     __syncthreads();
-    gemm<C, D, kLocalThreads>(C, [&](int i, int j) { return N3[i * LN + j]; },
-                              [&](int j, int d) { return RA[j * LW + d]; },
-                              [&](int i, int d, float x) { if (i < cl) atomicAdd(qk_at(dk, i, d), x); });
-    gemm<C, D, kLocalThreads>(C, [&](int j, int i) { return N3[i * LN + j]; },
-                              [&](int i, int d) { return RA[i * LW + d]; },
-                              [&](int j, int d, float x) { if (j < cl) atomicAdd(qk_at(dk, j, d), x); });
-    gemm<C, D, kLocalThreads>(C, [&](int i, int j) { return N2[i * LN + j]; },
-                              [&](int j, int d) { return RA[j * LW + d]; },
-                              [&](int i, int d, float x) { if (i < cl) atomicAdd(qk_at(dq, i, d), x); });
-    gemm<C, D, kLocalThreads>(C, [&](int j, int i) { return N2[i * LN + j]; },
-                              [&](int i, int d) { return RB[i * LW + d]; },
-                              [&](int j, int d, float x) { if (j < cl) atomicAdd(qk_at(dk, j, d), x); });
+    auto add_dk = [&](int tr, int tc, int, int, float x) { dkacc[tr][tc] += x; };
+    gemm_rc<C, D, kLocalThreads>(C, [&](int i, int j) { return N3[i * LN + j]; },
+                                 [&](int j, int d) { return RA[j * LW + d]; }, add_dk);
+    gemm_rc<C, D, kLocalThreads>(C, [&](int j, int i) { return N3[i * LN + j]; },
+                                 [&](int i, int d) { return RA[i * LW + d]; }, add_dk);
+    gemm_rc<C, D, kLocalThreads>(C, [&](int i, int j) { return N2[i * LN + j]; },
+                                 [&](int j, int d) { return RA[j * LW + d]; },
+                                 [&](int tr, int tc, int, int, float x) { dqacc[tr][tc] += x; });
+    gemm_rc<C, D, kLocalThreads>(C, [&](int j, int i) { return N2[i * LN + j]; },
+                                 [&](int i, int d) { return RB[i * LW + d]; }, add_dk);
+    {
+        // one sum per element: a store when the chunk's head owns its q/k
+        // head, else an atomic (the value heads of a group share it)
+        const int gr = tid >> 4, gcol = tid & 15;
+        const bool sole = H == Hqk;
+#pragma unroll
+        for (int r = 0; r < kLocTM; ++r) {
+            const int i = gr + 16 * r;
+            if (i >= cl) continue;
+#pragma unroll
+            for (int c = 0; c < kLocTN; ++c) {
+                const int d = gcol + 16 * c;
+                if (sole) {
+                    *qk_at(dk, i, d) = dkacc[r][c];
+                    *qk_at(dq, i, d) = dqacc[r][c];
+                } else {
+                    atomicAdd(qk_at(dk, i, d), dkacc[r][c]);
+                    atomicAdd(qk_at(dq, i, d), dqacc[r][c]);
+                }
+            }
+        }
+    }
     __syncthreads();
 
     // ---- phase E: dg as the reverse cumulative sum of dG, and dbeta -----------------
@@ -662,9 +898,9 @@ cudaError_t launch_chunked(const IoT *q, const IoT *k, const IoT *v, const float
     float *recs = reinterpret_cast<float *>(ws + base_bytes);
     cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void *>(bwd_prep_kernel<IoT>), (int)PB_SMEM);
     if (e == cudaSuccess)
-        e = ensure_dynamic_smem(reinterpret_cast<const void *>(bwd_forward_kernel), (int)CB_SMEM);
+        e = ensure_dynamic_smem(reinterpret_cast<const void *>(bwd_forward_kernel), (int)CF_SMEM);
     if (e == cudaSuccess)
-        e = ensure_dynamic_smem(reinterpret_cast<const void *>(bwd_reverse_kernel<IoT>), (int)CB_SMEM);
+        e = ensure_dynamic_smem(reinterpret_cast<const void *>(bwd_reverse_kernel<IoT>), (int)CR_SMEM);
     if (e == cudaSuccess)
         e = ensure_dynamic_smem(reinterpret_cast<const void *>(bwd_local_kernel<IoT>), (int)LB_SMEM);
     if (e != cudaSuccess) return e;
@@ -673,10 +909,10 @@ cudaError_t launch_chunked(const IoT *q, const IoT *k, const IoT *v, const float
     const dim3 per_rows((unsigned)(num_seqs * H), D / kRowBlock);
     bwd_prep_kernel<IoT><<<per_chunk, kPrepB, PB_SMEM, stream>>>(q, k, v, g, beta, cu, num_seqs,
                                                                   total_T, Hqk, H, base, recs);
-    bwd_forward_kernel<<<per_rows, kChainThreadsB, CB_SMEM, stream>>>(
-        h0, cu, num_seqs, total_T, Hqk, H, base, max_total, recs);
-    bwd_reverse_kernel<IoT><<<per_rows, kChainThreadsB, CB_SMEM, stream>>>(
-        dO, dSf, dh0, cu, num_seqs, total_T, Hqk, H, base, max_total, recs);
+    bwd_forward_kernel<<<per_rows, kChainThreads, CF_SMEM, stream>>>(
+        h0, cu, num_seqs, total_T, H, base, max_total, recs);
+    bwd_reverse_kernel<IoT><<<per_rows, kChainThreads, CR_SMEM, stream>>>(
+        dO, dSf, dh0, cu, num_seqs, total_T, H, base, max_total, recs);
     bwd_local_kernel<IoT><<<per_chunk, kLocalThreads, LB_SMEM, stream>>>(
         q, k, v, g, dO, cu, num_seqs, total_T, Hqk, H, base, recs, dq, dk, dv, dg, dbeta);
     return cudaGetLastError();
