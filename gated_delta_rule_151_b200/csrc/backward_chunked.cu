@@ -62,11 +62,11 @@ constexpr size_t R_QT = R_KH + C * D;           // diag(gamma) Q [64][128]
 constexpr size_t R_FLOATS = R_QT + C * D;       // 94,336 floats
 constexpr size_t kBaseBytes = 256;              // sequence chunk offsets precede the records
 
-constexpr int LW = D + 1;    // padded row of 128 floats
-constexpr int LN = C + 1;    // padded row of 64 floats
+constexpr int LW = D + 4;    // padded row of 128 floats (4 mod 32: see the products)
+constexpr int LN = C + 4;    // padded row of 64 floats
 constexpr int kRowBlock = 16;                   // state rows per forward / reverse CTA
 constexpr int kLocalThreads = 256;
-constexpr int kLocTM = C / (kLocalThreads / 16), kLocTN = D / 16;   // <C, D> product tile
+constexpr int kLocTM = 4, kLocTN = 8;   // slots of a thread in a <C, D> product over 8 warps
 
 // rows x cols fp32 (cols a multiple of 4, 16-byte aligned) from the record
 // into padded shared rows of `ld` floats: 16-byte loads, eight in flight per
@@ -109,71 +109,115 @@ __device__ __forceinline__ void load_io_rows(float *dst, const IoT *src, int tok
     }
 }
 
-// The product tile of one thread: out(m, n) = sum_k a(m, k) b(k, n) for
-// rows m = gr + GR r and columns n = gc + GC c, (gr, gc) = (tid / GC, tid % GC),
-// GC = min(N, 16) unless given, GR = NT / GC; epi(m, n, value) takes each
-// result.
-template <int M, int N, int NT, int GCX = 0, class AF, class BF, class EPI>
-__device__ __forceinline__ void gemm(int K, AF a, BF b, EPI epi) {
-    constexpr int GC = GCX > 0 ? GCX : (N < 16 ? N : 16);
-    constexpr int GR = NT / GC;
-    constexpr int TM = M / GR, TN = N / GC;
-    static_assert(GR * GC == NT && TM * GR == M && TN * GC == N, "product tiling");
-    const int tid = threadIdx.x, gr = tid / GC, gc = tid % GC;
-    float acc[TM][TN];
-#pragma unroll
-    for (int r = 0; r < TM; ++r)
-#pragma unroll
-        for (int c = 0; c < TN; ++c) acc[r][c] = 0.f;
-#pragma unroll 4
-    for (int k = 0; k < K; ++k) {
-        float av[TM], bv[TN];
-#pragma unroll
-        for (int r = 0; r < TM; ++r) av[r] = a(gr + GR * r, k);
-#pragma unroll
-        for (int c = 0; c < TN; ++c) bv[c] = b(k, gc + GC * c);
-#pragma unroll
-        for (int r = 0; r < TM; ++r)
-#pragma unroll
-            for (int c = 0; c < TN; ++c) acc[r][c] = fmaf(av[r], bv[c], acc[r][c]);
-    }
-#pragma unroll
-    for (int r = 0; r < TM; ++r)
-#pragma unroll
-        for (int c = 0; c < TN; ++c) epi(gr + GR * r, gc + GC * c, acc[r][c]);
+// ---------------------------------------------------- tensor-core products ----
+// Products in fp32 accuracy on the tensor cores: each operand value x is
+// split into x_hi = tf32(x) and x_lo = tf32(x - x_hi), and the product is
+// accumulated in fp32 as lo*hi + hi*lo + hi*hi (the dropped lo*lo term is
+// below 2^-21 of it).  Warp-level m16n8k8 tf32 tiles whose fragments are
+// read from shared memory through the accessors a(m, k) and b(k, n), so a
+// stored matrix serves in either orientation; rows padded to 4 mod 32 floats
+// keep every fragment read within two-way bank conflicts.
+
+__device__ __forceinline__ void split_tf32(float x, uint32_t &hi, uint32_t &lo) {
+    hi = tc::to_tf32(x);
+    lo = tc::to_tf32(x - __uint_as_float(hi));
 }
 
-// The same tile, its results handed to epi(r, c, m, n, value) with (r, c) the
-// tile position, so that a caller can keep per-thread sums over several
-// products (every <M, N, NT> product maps (m, n) to the same thread and slot).
-template <int M, int N, int NT, class AF, class BF, class EPI>
-__device__ __forceinline__ void gemm_rc(int K, AF a, BF b, EPI epi) {
-    constexpr int GC = N < 16 ? N : 16;
-    constexpr int GR = NT / GC;
-    constexpr int TM = M / GR, TN = N / GC;
-    static_assert(GR * GC == NT && TM * GR == M && TN * GC == N, "product tiling");
-    const int tid = threadIdx.x, gr = tid / GC, gc = tid % GC;
-    float acc[TM][TN];
+// d (16 x 8, fp32) += a (16 x 8, tf32, row) * b (8 x 8, tf32, column).
+__device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+    asm("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+        "{%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+// How NW warps share an M x N result: GM x GN warp blocks of WM x WN, each
+// MT x NT tiles of 16 x 8.
+template <int M, int N, int NW>
+struct WarpGrid {
+    static constexpr int pick() {
+        return (M % 32 == 0 && NW % 2 == 0 && N % (8 * (NW / 2)) == 0)   ? 2
+               : (M % 64 == 0 && NW % 4 == 0 && N % (8 * (NW / 4)) == 0) ? 4
+                                                                          : 1;
+    }
+    static constexpr int GM = pick(), GN = NW / GM;
+    static constexpr int WM = M / GM, WN = N / GN;
+    static constexpr int MT = WM / 16, NT = WN / 8;
+    static_assert(GM * GN == NW && MT * 16 * GM == M && NT * 8 * GN == N, "warp tiling");
+};
+
+// out(m, n) = sum_k a(m, k) b(k, n) (K a multiple of 8) over NTH threads;
+// every result goes to epi(r, c, m, n, value) with (r, c) its slot in the
+// calling thread's part (r < 2 MT, c < 2 NT).  Every <M, N, NTH> product
+// hands a thread the same (m, n) in the same slot, so that a caller can sum
+// several products in registers.
+template <int M, int N, int NTH, class AF, class BF, class EPI>
+__device__ __forceinline__ void tgemm_rc(int K, AF a, BF b, EPI epi) {
+    using G = WarpGrid<M, N, NTH / 32>;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int gid = lane >> 2, tig = lane & 3;
+    const int m0 = (warp / G::GN) * G::WM, n0 = (warp % G::GN) * G::WN;
+    float acc[G::MT][G::NT][4];
 #pragma unroll
-    for (int r = 0; r < TM; ++r)
+    for (int mt = 0; mt < G::MT; ++mt)
 #pragma unroll
-        for (int c = 0; c < TN; ++c) acc[r][c] = 0.f;
-#pragma unroll 4
-    for (int k = 0; k < K; ++k) {
-        float av[TM], bv[TN];
+        for (int nt = 0; nt < G::NT; ++nt)
 #pragma unroll
-        for (int r = 0; r < TM; ++r) av[r] = a(gr + GR * r, k);
+            for (int e = 0; e < 4; ++e) acc[mt][nt][e] = 0.f;
+#pragma unroll 2
+    for (int k0 = 0; k0 < K; k0 += 8) {
+        uint32_t ah[G::MT][4], al[G::MT][4], bh[G::NT][2], bl[G::NT][2];
 #pragma unroll
-        for (int c = 0; c < TN; ++c) bv[c] = b(k, gc + GC * c);
+        for (int mt = 0; mt < G::MT; ++mt) {
+            const int m = m0 + mt * 16 + gid;
+            split_tf32(a(m, k0 + tig), ah[mt][0], al[mt][0]);
+            split_tf32(a(m + 8, k0 + tig), ah[mt][1], al[mt][1]);
+            split_tf32(a(m, k0 + tig + 4), ah[mt][2], al[mt][2]);
+            split_tf32(a(m + 8, k0 + tig + 4), ah[mt][3], al[mt][3]);
+        }
 #pragma unroll
-        for (int r = 0; r < TM; ++r)
+        for (int nt = 0; nt < G::NT; ++nt) {
+            const int n = n0 + nt * 8 + gid;
+            split_tf32(b(k0 + tig, n), bh[nt][0], bl[nt][0]);
+            split_tf32(b(k0 + tig + 4, n), bh[nt][1], bl[nt][1]);
+        }
 #pragma unroll
-            for (int c = 0; c < TN; ++c) acc[r][c] = fmaf(av[r], bv[c], acc[r][c]);
+        for (int mt = 0; mt < G::MT; ++mt)
+#pragma unroll
+            for (int nt = 0; nt < G::NT; ++nt) {
+                mma_tf32(acc[mt][nt], al[mt], bh[nt]);
+                mma_tf32(acc[mt][nt], ah[mt], bl[nt]);
+                mma_tf32(acc[mt][nt], ah[mt], bh[nt]);
+            }
     }
 #pragma unroll
-    for (int r = 0; r < TM; ++r)
+    for (int mt = 0; mt < G::MT; ++mt)
 #pragma unroll
-        for (int c = 0; c < TN; ++c) epi(r, c, gr + GR * r, gc + GC * c, acc[r][c]);
+        for (int nt = 0; nt < G::NT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                epi(mt * 2 + (e >> 1), nt * 2 + (e & 1), m0 + mt * 16 + gid + 8 * (e >> 1),
+                    n0 + nt * 8 + 2 * tig + (e & 1), acc[mt][nt][e]);
+}
+
+template <int M, int N, int NTH, class AF, class BF, class EPI>
+__device__ __forceinline__ void tgemm(int K, AF a, BF b, EPI epi) {
+    tgemm_rc<M, N, NTH>(K, a, b, [&](int, int, int m, int n, float v) { epi(m, n, v); });
+}
+
+// Row of slot r and column of slot c of the calling thread in a <M, N, NTH>
+// product.
+template <int M, int N, int NTH>
+__device__ __forceinline__ int tslot_row(int r) {
+    using G = WarpGrid<M, N, NTH / 32>;
+    const int warp = threadIdx.x >> 5, gid = (threadIdx.x & 31) >> 2;
+    return (warp / G::GN) * G::WM + (r >> 1) * 16 + gid + 8 * (r & 1);
+}
+template <int M, int N, int NTH>
+__device__ __forceinline__ int tslot_col(int c) {
+    using G = WarpGrid<M, N, NTH / 32>;
+    const int warp = threadIdx.x >> 5, tig = threadIdx.x & 3;
+    return (warp % G::GN) * G::WN + (c >> 1) * 8 + 2 * tig + (c & 1);
 }
 
 // base[n] = first global chunk of sequence n (exclusive prefix sum of the
@@ -288,14 +332,14 @@ bwd_prep_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT 
     __syncthreads();
     // (K K^T) o R (strictly lower) -> record and A = diag(beta) of it; P -> record
     float *Af = fs + PB_A;
-    gemm<C, C, kPrepB>(D, [&](int i, int d) { return Ks[i * LW + d]; },
+    tgemm<C, C, kPrepB>(D, [&](int i, int d) { return Ks[i * LW + d]; },
                        [&](int d, int j) { return Ks[j * LW + d]; },
                        [&](int i, int j, float x) {
                            const float ar = j < i ? x * __expf(Gs[i] - Gs[j]) : 0.f;
                            rec[R_AR + i * C + j] = ar;
                            Af[ax(i, j)] = Bs[i] * ar;
                        });
-    gemm<C, C, kPrepB>(D, [&](int i, int d) { return Qs[i * LW + d]; },
+    tgemm<C, C, kPrepB>(D, [&](int i, int d) { return Qs[i * LW + d]; },
                        [&](int d, int j) { return Ks[j * LW + d]; },
                        [&](int i, int j, float x) {
                            rec[R_P + j * C + i] = j <= i ? x * __expf(Gs[i] - Gs[j]) : 0.f;
@@ -324,10 +368,10 @@ bwd_prep_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT 
         rec[R_B + tid] = Bs[tid];
     }
     __syncthreads();
-    gemm<C, D, kPrepB>(C, [&](int i, int j) { return Tp[i * LN + j]; },
+    tgemm<C, D, kPrepB>(C, [&](int i, int j) { return Tp[i * LN + j]; },
                        [&](int j, int d) { return Ks[j * LW + d]; },
                        [&](int i, int d, float x) { rec[R_W + i * D + d] = x; });
-    gemm<C, D, kPrepB>(C, [&](int i, int j) { return Tp[i * LN + j]; },
+    tgemm<C, D, kPrepB>(C, [&](int i, int j) { return Tp[i * LN + j]; },
                        [&](int j, int d) { return Vs[j * LW + d]; },
                        [&](int i, int d, float x) { rec[R_UT + i * D + d] = x; });
 }
@@ -342,7 +386,8 @@ bwd_prep_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT 
 // to 132 or 68 floats: 16-byte aligned for the copies, and the float4 reads
 // of 8 different rows by a quarter warp fall in 8 different bank groups.
 constexpr int kChainThreads = 256;
-constexpr int LW4 = D + 4;
+constexpr int LW4 = D + 4;   // rows read as the A operand or along K
+constexpr int LW8 = D + 8;   // rows read as a K x N B operand
 constexpr int LN4 = C + 4;
 static_assert(kChainThreads == C * 4, "one 16-byte piece of a column strip per thread");
 
@@ -355,11 +400,11 @@ template <int N> __device__ __forceinline__ void cp_wait() {
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-// 64 x 128 floats of a record field into rows of LW4 floats.
-__device__ __forceinline__ void stage_c_by_d(float *dst, const float *src) {
+// 64 x 128 floats of a record field into rows of ld floats.
+__device__ __forceinline__ void stage_c_by_d(float *dst, int ld, const float *src) {
 #pragma unroll 8
     for (int e = threadIdx.x; e < C * D / 4; e += kChainThreads)
-        cp16(dst + (e >> 5) * LW4 + (e & 31) * 4, src + e * 4);
+        cp16(dst + (e >> 5) * ld + (e & 31) * 4, src + e * 4);
 }
 // 64 x 64 floats into rows of LN4 floats.
 __device__ __forceinline__ void stage_c_by_c(float *dst, const float *src) {
@@ -378,52 +423,6 @@ __device__ __forceinline__ void stage_g(float *dst, const float *src) {
 }
 
 __device__ __forceinline__ float4 lds4(const float *p) { return *reinterpret_cast<const float4 *>(p); }
-__device__ __forceinline__ float dot4(float4 a, float4 b, float c) {
-    return fmaf(a.w, b.w, fmaf(a.z, b.z, fmaf(a.y, b.y, fmaf(a.x, b.x, c))));
-}
-
-// 64 x 16 product with both operands read along K: acc[t][u] += sum_k
-// A[j][k] B[r][k] for j = gr + 32 t, r = gc + 8 u, (gr, gc) = (tid / 8, tid % 8).
-__device__ __forceinline__ void prod_narrow(float (&acc)[2][2], const float *A, int lda,
-                                            const float *B, int ldb, int K) {
-    const int gr = threadIdx.x >> 3, gc = threadIdx.x & 7;
-    const float *a0 = A + gr * lda, *a1 = A + (gr + 32) * lda;
-    const float *b0 = B + gc * ldb, *b1 = B + (gc + 8) * ldb;
-#pragma unroll 4
-    for (int k = 0; k < K; k += 4) {
-        const float4 x0 = lds4(a0 + k), x1 = lds4(a1 + k), y0 = lds4(b0 + k), y1 = lds4(b1 + k);
-        acc[0][0] = dot4(x0, y0, acc[0][0]);
-        acc[0][1] = dot4(x0, y1, acc[0][1]);
-        acc[1][0] = dot4(x1, y0, acc[1][0]);
-        acc[1][1] = dot4(x1, y1, acc[1][1]);
-    }
-}
-
-// 16 x 128 product: acc[t][e] += sum_k A[r][k] B[k][4 gc + e] for
-// r = gr + 8 t, (gr, gc) = (tid / 32, tid % 32).
-__device__ __forceinline__ void prod_wide(float (&acc)[2][4], const float *A, int lda,
-                                          const float *B, int ldb, int K) {
-    const int gr = threadIdx.x >> 5, gc = threadIdx.x & 31;
-    const float *a0 = A + gr * lda, *a1 = A + (gr + 8) * lda, *b = B + 4 * gc;
-#pragma unroll 2
-    for (int k = 0; k < K; k += 4) {
-        const float4 x0 = lds4(a0 + k), x1 = lds4(a1 + k);
-        const float xa[4] = {x0.x, x0.y, x0.z, x0.w}, xb[4] = {x1.x, x1.y, x1.z, x1.w};
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-            const float4 y = lds4(b + (k + kk) * ldb);
-            acc[0][0] = fmaf(xa[kk], y.x, acc[0][0]);
-            acc[0][1] = fmaf(xa[kk], y.y, acc[0][1]);
-            acc[0][2] = fmaf(xa[kk], y.z, acc[0][2]);
-            acc[0][3] = fmaf(xa[kk], y.w, acc[0][3]);
-            acc[1][0] = fmaf(xb[kk], y.x, acc[1][0]);
-            acc[1][1] = fmaf(xb[kk], y.y, acc[1][1]);
-            acc[1][2] = fmaf(xb[kk], y.z, acc[1][2]);
-            acc[1][3] = fmaf(xb[kk], y.w, acc[1][3]);
-        }
-    }
-}
-
 // The CTA's 16 rows (padded) -> rows r0 .. r0 + 15 of a [128][128] field.
 __device__ __forceinline__ void store_rows(float *dst, const float *rows, int r0) {
 #pragma unroll
@@ -436,8 +435,8 @@ __device__ __forceinline__ void store_rows(float *dst, const float *rows, int r0
 constexpr uint32_t CF_S = 0;                             // S rows [16][LW4]
 constexpr uint32_t CF_UT = CF_S + kRowBlock * LW4;       // U^T [16][LN4]
 constexpr uint32_t CF_W = CF_UT + kRowBlock * LN4;       // W [64][LW4]
-constexpr uint32_t CF_KH = CF_W + C * LW4;               // K^ [64][LW4]
-constexpr uint32_t CF_US = CF_KH + C * LW4;              // U~ columns r0 .. r0 + 15 [64][16]
+constexpr uint32_t CF_KH = CF_W + C * LW4;               // K^ [64][LW8]
+constexpr uint32_t CF_US = CF_KH + C * LW8;              // U~ columns r0 .. r0 + 15 [64][16]
 constexpr uint32_t CF_G = CF_US + C * kRowBlock;         // G [64]
 constexpr uint32_t CF_SMEM = (CF_G + C) * sizeof(float);
 
@@ -462,58 +461,51 @@ bwd_forward_kernel(const float *__restrict__ h0, const int32_t *__restrict__ cu,
     }
     // copy groups, in order: {W, U~} and {K^, G} of every chunk
     if (nch > 0) {
-        stage_c_by_d(Ws, rec_of(0) + R_W);
+        stage_c_by_d(Ws, LW4, rec_of(0) + R_W);
         stage_strip(Us, rec_of(0) + R_UT, r0);
         cp_commit();
-        stage_c_by_d(Kh, rec_of(0) + R_KH);
+        stage_c_by_d(Kh, LW8, rec_of(0) + R_KH);
         stage_g(Gs, rec_of(0) + R_G);
         cp_commit();
     }
-    const int gr1 = tid >> 3, gc1 = tid & 7, gr2 = tid >> 5, gc2 = tid & 31;
     for (int c = 0; c < nch; ++c) {
         float *rec = rec_of(c);
         cp_wait<1>();
         __syncthreads();   // W, U~ of chunk c and the state rows in place
-        store_rows(rec + R_S, Sr, r0);
-        {   // U[j][r0 + r] = U~[j][r0 + r] - sum_d W[j][d] S[r][d]
-            float acc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
-            prod_narrow(acc, Ws, LW4, Sr, LW4, D);
-#pragma unroll
-            for (int t = 0; t < 2; ++t)
-#pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    const int j = gr1 + 32 * t, r = gc1 + 8 * u;
-                    const float x = Us[j * kRowBlock + r] - acc[t][u];
-                    Ut[r * LN4 + j] = x;
-                    rec[R_U + j * D + r0 + r] = x;
-                }
+        if (tid == 0 && blockIdx.y == 0 && c + 2 < nch) {   // chunk c + 2 towards L2
+            const float *nx = rec_of(c + 2);
+            tc::bulk_prefetch_l2(nx + R_W, 2 * C * D * sizeof(float));   // W and U~
+            tc::bulk_prefetch_l2(nx + R_KH, C * D * sizeof(float));
+            tc::bulk_prefetch_l2(nx + R_G, C * sizeof(float));
         }
+        store_rows(rec + R_S, Sr, r0);
+        // U[j][r0 + r] = U~[j][r0 + r] - sum_d W[j][d] S[r][d]
+        tgemm<C, kRowBlock, kChainThreads>(D, [&](int j, int d) { return Ws[j * LW4 + d]; },
+                                           [&](int d, int r) { return Sr[r * LW4 + d]; },
+                                           [&](int j, int r, float x) {
+                                               const float u = Us[j * kRowBlock + r] - x;
+                                               Ut[r * LN4 + j] = u;
+                                               rec[R_U + j * D + r0 + r] = u;
+                                           });
         __syncthreads();   // W and U~ consumed, U^T complete
         if (c + 1 < nch) {
-            stage_c_by_d(Ws, rec_of(c + 1) + R_W);
+            stage_c_by_d(Ws, LW4, rec_of(c + 1) + R_W);
             stage_strip(Us, rec_of(c + 1) + R_UT, r0);
         }
         cp_commit();
         cp_wait<1>();
         __syncthreads();   // K^ and G of chunk c in place
         {   // S[r][d] = e^{G_C} S[r][d] + sum_j U[j][r] K^[j][d]
-            float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-            prod_wide(acc, Ut, LN4, Kh, LW4, C);
             const float gC = __expf(Gs[C - 1]);
-#pragma unroll
-            for (int t = 0; t < 2; ++t) {
-                float4 *p = reinterpret_cast<float4 *>(Sr + (gr2 + 8 * t) * LW4 + 4 * gc2);
-                float4 s = *p;
-                s.x = fmaf(gC, s.x, acc[t][0]);
-                s.y = fmaf(gC, s.y, acc[t][1]);
-                s.z = fmaf(gC, s.z, acc[t][2]);
-                s.w = fmaf(gC, s.w, acc[t][3]);
-                *p = s;
-            }
+            tgemm<kRowBlock, D, kChainThreads>(C, [&](int r, int j) { return Ut[r * LN4 + j]; },
+                                               [&](int j, int d) { return Kh[j * LW8 + d]; },
+                                               [&](int r, int d, float x) {
+                                                   Sr[r * LW4 + d] = fmaf(gC, Sr[r * LW4 + d], x);
+                                               });
         }
         __syncthreads();   // K^ and G consumed
         if (c + 1 < nch) {
-            stage_c_by_d(Kh, rec_of(c + 1) + R_KH);
+            stage_c_by_d(Kh, LW8, rec_of(c + 1) + R_KH);
             stage_g(Gs, rec_of(c + 1) + R_G);
         }
         cp_commit();
@@ -526,9 +518,9 @@ constexpr uint32_t CR_DUT = CR_L + kRowBlock * LW4;      // dU^T [16][LN4]
 constexpr uint32_t CR_DOT = CR_DUT + kRowBlock * LN4;    // dO^T, columns r0 .. r0 + 15 [16][LN4]
 constexpr uint32_t CR_KH = CR_DOT + kRowBlock * LN4;     // K^ [64][LW4]
 constexpr uint32_t CR_PT = CR_KH + C * LW4;              // P^T [64][LN4]
-constexpr uint32_t CR_QT = CR_PT + C * LN4;              // diag(gamma) Q [64][LW4]
-constexpr uint32_t CR_W = CR_QT + C * LW4;               // W [64][LW4]
-constexpr uint32_t CR_G = CR_W + C * LW4;                // G [64]
+constexpr uint32_t CR_QT = CR_PT + C * LN4;              // diag(gamma) Q [64][LW8]
+constexpr uint32_t CR_W = CR_QT + C * LW8;               // W [64][LW8]
+constexpr uint32_t CR_G = CR_W + C * LW8;                // G [64]
 constexpr uint32_t CR_SMEM = (CR_G + C) * sizeof(float);
 
 template <typename IoT>
@@ -564,40 +556,51 @@ bwd_reverse_kernel(const IoT *__restrict__ dO, const float *__restrict__ dSf,
     }
     // copy groups, in order: {K^, P^T} and {gamma Q, W, G} of every chunk
     if (nch > 0) {
-        stage_c_by_d(Kh, rec_of(nch - 1) + R_KH);
+        stage_c_by_d(Kh, LW4, rec_of(nch - 1) + R_KH);
         stage_c_by_c(PT, rec_of(nch - 1) + R_P);
         cp_commit();
-        stage_c_by_d(Qt, rec_of(nch - 1) + R_QT);
-        stage_c_by_d(Ws, rec_of(nch - 1) + R_W);
+        stage_c_by_d(Qt, LW8, rec_of(nch - 1) + R_QT);
+        stage_c_by_d(Ws, LW8, rec_of(nch - 1) + R_W);
         stage_g(Gs, rec_of(nch - 1) + R_G);
         cp_commit();
         float x[4];
         load_dO(nch - 1, x);
         put_dO(x);
     }
-    const int gr1 = tid >> 3, gc1 = tid & 7, gr2 = tid >> 5, gc2 = tid & 31;
     for (int c = nch - 1; c >= 0; --c) {
         float *rec = rec_of(c);
         cp_wait<1>();
         __syncthreads();   // K^, P^T, dO^T of chunk c and the adjoint rows in place
+        if (blockIdx.y == 0 && c >= 2) {   // chunk c - 2 towards L2
+            const float *pv = rec_of(c - 2);
+            if (tid == 0) {
+                tc::bulk_prefetch_l2(pv + R_KH, 2 * C * D * sizeof(float));   // K^ and gamma Q
+                tc::bulk_prefetch_l2(pv + R_W, C * D * sizeof(float));
+                tc::bulk_prefetch_l2(pv + R_P, C * C * sizeof(float));
+                tc::bulk_prefetch_l2(pv + R_G, C * sizeof(float));
+            } else if (tid >= 32 && tid < 32 + C && tid - 32 < min(C, len - (c - 2) * C)) {
+                tc::bulk_prefetch_l2(dO + ((size_t)(t0 + (c - 2) * C + tid - 32) * H + h) * D,
+                                     D * sizeof(IoT));
+            }
+        }
         store_rows(rec + R_L, Lr, r0);
         {   // dU[j][r] = sum_d K^[j][d] L[r][d] + sum_i P[i][j] dO[i][r]
-            float acc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
-            prod_narrow(acc, Kh, LW4, Lr, LW4, D);
-            prod_narrow(acc, PT, LN4, dOt, LN4, C);
-#pragma unroll
-            for (int t = 0; t < 2; ++t)
-#pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    const int j = gr1 + 32 * t, r = gc1 + 8 * u;
-                    dUt[r * LN4 + j] = acc[t][u];
-                    rec[R_DU + j * D + r0 + r] = acc[t][u];
-                }
+            float du[2][2];
+            tgemm_rc<C, kRowBlock, kChainThreads>(D, [&](int j, int d) { return Kh[j * LW4 + d]; },
+                                                  [&](int d, int r) { return Lr[r * LW4 + d]; },
+                                                  [&](int sr, int sc, int, int, float x) { du[sr][sc] = x; });
+            tgemm_rc<C, kRowBlock, kChainThreads>(C, [&](int j, int i) { return PT[j * LN4 + i]; },
+                                                  [&](int i, int r) { return dOt[r * LN4 + i]; },
+                                                  [&](int sr, int sc, int j, int r, float x) {
+                                                      const float v = du[sr][sc] + x;
+                                                      dUt[r * LN4 + j] = v;
+                                                      rec[R_DU + j * D + r0 + r] = v;
+                                                  });
         }
         __syncthreads();   // K^ and P^T consumed, dU^T complete
         float x[4] = {0.f, 0.f, 0.f, 0.f};
         if (c > 0) {
-            stage_c_by_d(Kh, rec_of(c - 1) + R_KH);
+            stage_c_by_d(Kh, LW4, rec_of(c - 1) + R_KH);
             stage_c_by_c(PT, rec_of(c - 1) + R_P);
             load_dO(c - 1, x);
         }
@@ -605,26 +608,21 @@ bwd_reverse_kernel(const IoT *__restrict__ dO, const float *__restrict__ dSf,
         cp_wait<1>();
         __syncthreads();   // gamma Q, W and G of chunk c in place
         {   // L[r][d] = e^{G_C} L[r][d] + sum_i dO[i][r] gamma_i q_i[d] - sum_j dU[j][r] W[j][d]
-            float a1[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-            float a2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-            prod_wide(a1, dOt, LN4, Qt, LW4, C);
-            prod_wide(a2, dUt, LN4, Ws, LW4, C);
+            float la[2][4];
+            tgemm_rc<kRowBlock, D, kChainThreads>(C, [&](int r, int i) { return dOt[r * LN4 + i]; },
+                                                  [&](int i, int d) { return Qt[i * LW8 + d]; },
+                                                  [&](int sr, int sc, int, int, float x) { la[sr][sc] = x; });
             const float gC = __expf(Gs[C - 1]);
-#pragma unroll
-            for (int t = 0; t < 2; ++t) {
-                float4 *p = reinterpret_cast<float4 *>(Lr + (gr2 + 8 * t) * LW4 + 4 * gc2);
-                float4 s = *p;
-                s.x = fmaf(gC, s.x, a1[t][0] - a2[t][0]);
-                s.y = fmaf(gC, s.y, a1[t][1] - a2[t][1]);
-                s.z = fmaf(gC, s.z, a1[t][2] - a2[t][2]);
-                s.w = fmaf(gC, s.w, a1[t][3] - a2[t][3]);
-                *p = s;
-            }
+            tgemm_rc<kRowBlock, D, kChainThreads>(C, [&](int r, int j) { return dUt[r * LN4 + j]; },
+                                                  [&](int j, int d) { return Ws[j * LW8 + d]; },
+                                                  [&](int sr, int sc, int r, int d, float x) {
+                                                      Lr[r * LW4 + d] = fmaf(gC, Lr[r * LW4 + d], la[sr][sc] - x);
+                                                  });
         }
         __syncthreads();   // gamma Q, W, G and dO^T consumed
         if (c > 0) {
-            stage_c_by_d(Qt, rec_of(c - 1) + R_QT);
-            stage_c_by_d(Ws, rec_of(c - 1) + R_W);
+            stage_c_by_d(Qt, LW8, rec_of(c - 1) + R_QT);
+            stage_c_by_d(Ws, LW8, rec_of(c - 1) + R_W);
             stage_g(Gs, rec_of(c - 1) + R_G);
             put_dO(x);
         }
@@ -682,9 +680,22 @@ bwd_local_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT
     float *Gs = fs + LB_G, *gam = Gs + C, *Bs = gam + C, *dG = Bs + C, *dB = dG + C;
     float *misc = fs + LB_MISC;
     auto qk_at = [&](float *base_, int i, int d) { return base_ + ((size_t)(tok0 + i) * Hqk + hq) * D + d; };
+    static_assert(2 * WarpGrid<C, D, kLocalThreads / 32>::MT == kLocTM &&
+                      2 * WarpGrid<C, D, kLocalThreads / 32>::NT == kLocTN,
+                  "slots of a <C, D> product");
     // dk and dq of the chunk's rows, summed over the product terms in the
-    // registers of the <C, D> product tile (rows gr + 16 r, columns gc + 16 c)
+    // registers of the <C, D> product slots
     float dkacc[kLocTM][kLocTN], dqacc[kLocTM][kLocTN];
+    // per-row sums over the slots of a <C, D> product -> dst[row] (shared)
+    auto flush_rows = [&](float *dst, const float (&acc)[kLocTM]) {
+#pragma unroll
+        for (int r = 0; r < kLocTM; ++r) {
+            float x = acc[r];
+            x += __shfl_xor_sync(0xffffffffu, x, 1);
+            x += __shfl_xor_sync(0xffffffffu, x, 2);
+            if ((tid & 3) == 0) atomicAdd(&dst[tslot_row<C, D, kLocalThreads>(r)], x);
+        }
+    };
     // everything the later phases read towards L2 while phase A runs: the
     // record's P, T, (K K^T) o R, G, beta and U .. gamma Q (64 KiB pieces),
     // and the chunk's rows of q, k, v and dO
@@ -726,17 +737,15 @@ bwd_local_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT
     __syncthreads();
     {
         float rowacc[4] = {0.f, 0.f, 0.f, 0.f}, gcacc = 0.f;
-        gemm_rc<C, D, kLocalThreads>(D, [&](int j, int r) { return RB[j * LW + r]; },
+        tgemm_rc<C, D, kLocalThreads>(D, [&](int j, int r) { return RB[j * LW + r]; },
                                   [&](int r, int d) { return RA[r * LW + d]; },
                                   [&](int tr, int tc, int j, int d, float x) {
                                       dkacc[tr][tc] = __expf(GC - Gs[j]) * x;
                                       const float t = RC[j * LW + d] * x;
-                                      rowacc[j >> 4] -= t;   // rows j = gr + 16 r
+                                      rowacc[tr] -= t;
                                       gcacc += t;
                                   });
-        const int gr = tid >> 4;
-#pragma unroll
-        for (int r = 0; r < 4; ++r) atomicAdd(&dG[gr + 16 * r], rowacc[r]);
+        flush_rows(dG, rowacc);
         atomicAdd(&misc[0], gcacc);
     }
     __syncthreads();
@@ -746,20 +755,18 @@ bwd_local_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT
     copy_rows<kLocalThreads>(RB, LW, rec + R_DU, C, D);
     load_io_rows<kLocalThreads>(RD, dO, tok0, cl, H, h);
     __syncthreads();
-    gemm<C, D, kLocalThreads>(D, [&](int j, int r) { return RB[j * LW + r]; },
+    tgemm<C, D, kLocalThreads>(D, [&](int j, int r) { return RB[j * LW + r]; },
                               [&](int r, int d) { return RA[r * LW + d]; },
                               [&](int j, int d, float x) { RC[j * LW + d] = -x; });
     {
         float rowacc[4] = {0.f, 0.f, 0.f, 0.f};
-        gemm_rc<C, D, kLocalThreads>(D, [&](int i, int r) { return RD[i * LW + r]; },
+        tgemm_rc<C, D, kLocalThreads>(D, [&](int i, int r) { return RD[i * LW + r]; },
                                   [&](int r, int d) { return RA[r * LW + d]; },
                                   [&](int tr, int tc, int i, int d, float x) {
                                       dqacc[tr][tc] = gam[i] * x;
-                                      if (i < cl) rowacc[i >> 4] += rec[R_QT + i * D + d] * x;
+                                      if (i < cl) rowacc[tr] += rec[R_QT + i * D + d] * x;
                                   });
-        const int gr = tid >> 4;
-#pragma unroll
-        for (int r = 0; r < 4; ++r) atomicAdd(&dG[gr + 16 * r], rowacc[r]);
+        flush_rows(dG, rowacc);
     }
     __syncthreads();
 
@@ -767,7 +774,7 @@ bwd_local_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT
     copy_rows<kLocalThreads>(RA, LW, rec + R_U, C, D);
     copy_rows<kLocalThreads>(N1, LN, rec + R_T, C, C);
     __syncthreads();
-    gemm<C, C, kLocalThreads>(D, [&](int i, int r) { return RD[i * LW + r]; },
+    tgemm<C, C, kLocalThreads>(D, [&](int i, int r) { return RD[i * LW + r]; },
                               [&](int r, int j) { return RA[j * LW + r]; },
                               [&](int i, int j, float x) { N2[i * LN + j] = j <= i ? x : 0.f; });
     __syncthreads();
@@ -776,48 +783,42 @@ bwd_local_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT
     __syncthreads();
     {
         float rowacc[4] = {0.f, 0.f, 0.f, 0.f};
-        gemm<C, D, kLocalThreads>(C, [&](int j, int i) { return N1[i * LN + j]; },
+        tgemm_rc<C, D, kLocalThreads>(C, [&](int j, int i) { return N1[i * LN + j]; },
                                   [&](int i, int r) { return RB[i * LW + r]; },
-                                  [&](int j, int r, float x) {
+                                  [&](int tr, int, int j, int r, float x) {
                                       if (j < cl) dv[((size_t)(tok0 + j) * H + h) * D + r] = Bs[j] * x;
-                                      rowacc[j >> 4] += RD[j * LW + r] * x;
+                                      rowacc[tr] += RD[j * LW + r] * x;
                                   });
-        const int gr = tid >> 4;
-#pragma unroll
-        for (int r = 0; r < 4; ++r) atomicAdd(&dB[gr + 16 * r], rowacc[r]);
+        flush_rows(dB, rowacc);
     }
     {
         float bacc[4] = {0.f, 0.f, 0.f, 0.f}, gacc[4] = {0.f, 0.f, 0.f, 0.f};
-        gemm_rc<C, D, kLocalThreads>(C, [&](int j, int i) { return N1[i * LN + j]; },
+        tgemm_rc<C, D, kLocalThreads>(C, [&](int j, int i) { return N1[i * LN + j]; },
                                   [&](int i, int d) { return RC[i * LW + d]; },
                                   [&](int tr, int tc, int j, int d, float x) {
                                       dkacc[tr][tc] += Bs[j] * gam[j] * x;
                                       const float t = RA[j * LW + d] * x;
-                                      bacc[j >> 4] += gam[j] * t;
-                                      gacc[j >> 4] += Bs[j] * gam[j] * t;
+                                      bacc[tr] += gam[j] * t;
+                                      gacc[tr] += Bs[j] * gam[j] * t;
                                   });
-        const int gr = tid >> 4;
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-            atomicAdd(&dB[gr + 16 * r], bacc[r]);
-            atomicAdd(&dG[gr + 16 * r], gacc[r]);
-        }
+        flush_rows(dB, bacc);
+        flush_rows(dG, gacc);
     }
-    gemm<C, C, kLocalThreads>(D, [&](int i, int r) { return RB[i * LW + r]; },
+    tgemm<C, C, kLocalThreads>(D, [&](int i, int r) { return RB[i * LW + r]; },
                               [&](int r, int j) { return Bs[j] * RD[j * LW + r]; },
                               [&](int i, int j, float x) { N3[i * LN + j] = x; });
-    gemm<C, C, kLocalThreads>(D, [&](int i, int d) { return RC[i * LW + d]; },
+    tgemm<C, C, kLocalThreads>(D, [&](int i, int d) { return RC[i * LW + d]; },
                               [&](int d, int j) { return Bs[j] * gam[j] * RA[j * LW + d]; },
                               [&](int i, int j, float x) { N3[i * LN + j] += x; });
     __syncthreads();
 
     // ---- phase D: dA = -T^T dT T^T, then the A and P terms ------------------------
     float *Y = RB;   // [64][65]
-    gemm<C, C, kLocalThreads>(C, [&](int i, int m) { return N3[i * LN + m]; },
+    tgemm<C, C, kLocalThreads>(C, [&](int i, int m) { return N3[i * LN + m]; },
                               [&](int m, int j) { return N1[j * LN + m]; },
                               [&](int i, int j, float x) { Y[i * LN + j] = x; });
     __syncthreads();
-    gemm<C, C, kLocalThreads>(C, [&](int i, int m) { return N1[m * LN + i]; },
+    tgemm<C, C, kLocalThreads>(C, [&](int i, int m) { return N1[m * LN + i]; },
                               [&](int m, int j) { return Y[m * LN + j]; },
                               [&](int i, int j, float x) { N3[i * LN + j] = j < i ? -x : 0.f; });
     __syncthreads();
@@ -842,27 +843,26 @@ bwd_local_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT
     load_io_rows<kLocalThreads>(RB, q, tok0, cl, Hqk, hq);   // Q rows over the finished Y
     __syncthreads();
     auto add_dk = [&](int tr, int tc, int, int, float x) { dkacc[tr][tc] += x; };
-    gemm_rc<C, D, kLocalThreads>(C, [&](int i, int j) { return N3[i * LN + j]; },
+    tgemm_rc<C, D, kLocalThreads>(C, [&](int i, int j) { return N3[i * LN + j]; },
                                  [&](int j, int d) { return RA[j * LW + d]; }, add_dk);
-    gemm_rc<C, D, kLocalThreads>(C, [&](int j, int i) { return N3[i * LN + j]; },
+    tgemm_rc<C, D, kLocalThreads>(C, [&](int j, int i) { return N3[i * LN + j]; },
                                  [&](int i, int d) { return RA[i * LW + d]; }, add_dk);
-    gemm_rc<C, D, kLocalThreads>(C, [&](int i, int j) { return N2[i * LN + j]; },
+    tgemm_rc<C, D, kLocalThreads>(C, [&](int i, int j) { return N2[i * LN + j]; },
                                  [&](int j, int d) { return RA[j * LW + d]; },
                                  [&](int tr, int tc, int, int, float x) { dqacc[tr][tc] += x; });
-    gemm_rc<C, D, kLocalThreads>(C, [&](int j, int i) { return N2[i * LN + j]; },
+    tgemm_rc<C, D, kLocalThreads>(C, [&](int j, int i) { return N2[i * LN + j]; },
                                  [&](int i, int d) { return RB[i * LW + d]; }, add_dk);
     {
         // one sum per element: a store when the chunk's head owns its q/k
         // head, else an atomic (the value heads of a group share it)
-        const int gr = tid >> 4, gcol = tid & 15;
         const bool sole = H == Hqk;
 #pragma unroll
         for (int r = 0; r < kLocTM; ++r) {
-            const int i = gr + 16 * r;
+            const int i = tslot_row<C, D, kLocalThreads>(r);
             if (i >= cl) continue;
 #pragma unroll
             for (int c = 0; c < kLocTN; ++c) {
-                const int d = gcol + 16 * c;
+                const int d = tslot_col<C, D, kLocalThreads>(c);
                 if (sole) {
                     *qk_at(dk, i, d) = dkacc[r][c];
                     *qk_at(dq, i, d) = dqacc[r][c];
