@@ -36,6 +36,7 @@
 
 #include <algorithm>
 #include <cstddef>
+#include <type_traits>
 
 #include "common.cuh"
 #include "internal.h"
@@ -110,6 +111,9 @@ __device__ __forceinline__ void load_io_rows(float *dst, const IoT *src, int tok
 }
 
 // ---------------------------------------------------- tensor-core products ----
+// An input held as bf16 is exact in tf32.
+template <typename IoT> constexpr bool kIoExact = std::is_same<IoT, __nv_bfloat16>::value;
+
 // Products in fp32 accuracy on the tensor cores: each operand value x is
 // split into x_hi = tf32(x) and x_lo = tf32(x - x_hi), and the product is
 // accumulated in fp32 as lo*hi + hi*lo + hi*hi (the dropped lo*lo term is
@@ -146,63 +150,94 @@ struct WarpGrid {
     static_assert(GM * GN == NW && MT * 16 * GM == M && NT * 8 * GN == N, "warp tiling");
 };
 
-// out(m, n) = sum_k a(m, k) b(k, n) (K a multiple of 8) over NTH threads;
-// every result goes to epi(r, c, m, n, value) with (r, c) its slot in the
-// calling thread's part (r < 2 MT, c < 2 NT).  Every <M, N, NTH> product
-// hands a thread the same (m, n) in the same slot, so that a caller can sum
-// several products in registers.
-template <int M, int N, int NTH, class AF, class BF, class EPI>
+// out(m, n) = sum_k a(m, k) b(k, n) over NTH threads; every result goes to
+// epi(r, c, m, n, value) with (r, c) its slot in the calling thread's part
+// (r < 2 MT, c < 2 NT).  Every <M, N, NTH> product hands a thread the same
+// (m, n) in the same slot, so that a caller can sum several products in
+// registers.  A warp with few tiles would wait on one long chain of
+// dependent MMAs: KPAR = 2 alternates the k-steps between two sets of
+// accumulators and PSPLIT gives each tf32 pass its own set, the sets summed
+// at the end.  K is a multiple of 8 KPAR.  AEX (BEX) states that every
+// value a (b) returns is exact in tf32 (a bf16 input), so that its low part
+// and the pass that multiplies it are skipped.
+template <int M, int N, int NTH, int KPAR = 1, bool PSPLIT = false, bool AEX = false,
+          bool BEX = false, class AF, class BF, class EPI>
 __device__ __forceinline__ void tgemm_rc(int K, AF a, BF b, EPI epi) {
     using G = WarpGrid<M, N, NTH / 32>;
+    constexpr int NP = PSPLIT ? 3 : 1;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int gid = lane >> 2, tig = lane & 3;
     const int m0 = (warp / G::GN) * G::WM, n0 = (warp % G::GN) * G::WN;
-    float acc[G::MT][G::NT][4];
+    float acc[KPAR][NP][G::MT][G::NT][4];
 #pragma unroll
-    for (int mt = 0; mt < G::MT; ++mt)
+    for (int s = 0; s < KPAR; ++s)
 #pragma unroll
-        for (int nt = 0; nt < G::NT; ++nt)
+        for (int p = 0; p < NP; ++p)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) acc[mt][nt][e] = 0.f;
-#pragma unroll 2
-    for (int k0 = 0; k0 < K; k0 += 8) {
+            for (int mt = 0; mt < G::MT; ++mt)
+#pragma unroll
+                for (int nt = 0; nt < G::NT; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) acc[s][p][mt][nt][e] = 0.f;
+    auto kstep = [&](int k0, float (&ac)[NP][G::MT][G::NT][4]) {
         uint32_t ah[G::MT][4], al[G::MT][4], bh[G::NT][2], bl[G::NT][2];
+        auto take = [](float x, uint32_t &hi, uint32_t &lo, bool exact) {
+            if (exact) hi = __float_as_uint(x);
+            else split_tf32(x, hi, lo);
+        };
 #pragma unroll
         for (int mt = 0; mt < G::MT; ++mt) {
             const int m = m0 + mt * 16 + gid;
-            split_tf32(a(m, k0 + tig), ah[mt][0], al[mt][0]);
-            split_tf32(a(m + 8, k0 + tig), ah[mt][1], al[mt][1]);
-            split_tf32(a(m, k0 + tig + 4), ah[mt][2], al[mt][2]);
-            split_tf32(a(m + 8, k0 + tig + 4), ah[mt][3], al[mt][3]);
+            take(a(m, k0 + tig), ah[mt][0], al[mt][0], AEX);
+            take(a(m + 8, k0 + tig), ah[mt][1], al[mt][1], AEX);
+            take(a(m, k0 + tig + 4), ah[mt][2], al[mt][2], AEX);
+            take(a(m + 8, k0 + tig + 4), ah[mt][3], al[mt][3], AEX);
         }
 #pragma unroll
         for (int nt = 0; nt < G::NT; ++nt) {
             const int n = n0 + nt * 8 + gid;
-            split_tf32(b(k0 + tig, n), bh[nt][0], bl[nt][0]);
-            split_tf32(b(k0 + tig + 4, n), bh[nt][1], bl[nt][1]);
+            take(b(k0 + tig, n), bh[nt][0], bl[nt][0], BEX);
+            take(b(k0 + tig + 4, n), bh[nt][1], bl[nt][1], BEX);
         }
 #pragma unroll
         for (int mt = 0; mt < G::MT; ++mt)
 #pragma unroll
             for (int nt = 0; nt < G::NT; ++nt) {
-                mma_tf32(acc[mt][nt], al[mt], bh[nt]);
-                mma_tf32(acc[mt][nt], ah[mt], bl[nt]);
-                mma_tf32(acc[mt][nt], ah[mt], bh[nt]);
+                if (!AEX) mma_tf32(ac[NP - 1][mt][nt], al[mt], bh[nt]);
+                if (!BEX) mma_tf32(ac[NP > 1 ? 1 : 0][mt][nt], ah[mt], bl[nt]);
+                mma_tf32(ac[0][mt][nt], ah[mt], bh[nt]);
             }
+    };
+#pragma unroll 2
+    for (int k0 = 0; k0 < K; k0 += 8 * KPAR) {
+        kstep(k0, acc[0]);
+        if (KPAR > 1) kstep(k0 + 8, acc[KPAR - 1]);
     }
 #pragma unroll
     for (int mt = 0; mt < G::MT; ++mt)
 #pragma unroll
         for (int nt = 0; nt < G::NT; ++nt)
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
+            for (int e = 0; e < 4; ++e) {
+                float x = acc[0][0][mt][nt][e], corr = 0.f;
+#pragma unroll
+                for (int s = 0; s < KPAR; ++s)
+#pragma unroll
+                    for (int p = 0; p < NP; ++p)
+                        if (s + p > 0) {
+                            if (p > 0) corr += acc[s][p][mt][nt][e];
+                            else x += acc[s][p][mt][nt][e];
+                        }
                 epi(mt * 2 + (e >> 1), nt * 2 + (e & 1), m0 + mt * 16 + gid + 8 * (e >> 1),
-                    n0 + nt * 8 + 2 * tig + (e & 1), acc[mt][nt][e]);
+                    n0 + nt * 8 + 2 * tig + (e & 1), x + corr);
+            }
 }
 
-template <int M, int N, int NTH, class AF, class BF, class EPI>
+template <int M, int N, int NTH, int KPAR = 1, bool PSPLIT = false, bool AEX = false,
+          bool BEX = false, class AF, class BF, class EPI>
 __device__ __forceinline__ void tgemm(int K, AF a, BF b, EPI epi) {
-    tgemm_rc<M, N, NTH>(K, a, b, [&](int, int, int m, int n, float v) { epi(m, n, v); });
+    tgemm_rc<M, N, NTH, KPAR, PSPLIT, AEX, BEX>(K, a, b,
+                                                [&](int, int, int m, int n, float v) { epi(m, n, v); });
 }
 
 // Row of slot r and column of slot c of the calling thread in a <M, N, NTH>
@@ -332,14 +367,15 @@ bwd_prep_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT 
     __syncthreads();
     // (K K^T) o R (strictly lower) -> record and A = diag(beta) of it; P -> record
     float *Af = fs + PB_A;
-    tgemm<C, C, kPrepB>(D, [&](int i, int d) { return Ks[i * LW + d]; },
+    constexpr bool kX = kIoExact<IoT>;
+    tgemm<C, C, kPrepB, 1, false, kX, kX>(D, [&](int i, int d) { return Ks[i * LW + d]; },
                        [&](int d, int j) { return Ks[j * LW + d]; },
                        [&](int i, int j, float x) {
                            const float ar = j < i ? x * __expf(Gs[i] - Gs[j]) : 0.f;
                            rec[R_AR + i * C + j] = ar;
                            Af[ax(i, j)] = Bs[i] * ar;
                        });
-    tgemm<C, C, kPrepB>(D, [&](int i, int d) { return Qs[i * LW + d]; },
+    tgemm<C, C, kPrepB, 1, false, kX, kX>(D, [&](int i, int d) { return Qs[i * LW + d]; },
                        [&](int d, int j) { return Ks[j * LW + d]; },
                        [&](int i, int j, float x) {
                            rec[R_P + j * C + i] = j <= i ? x * __expf(Gs[i] - Gs[j]) : 0.f;
@@ -352,26 +388,24 @@ bwd_prep_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT 
         Tp[i * LN + j] = t;
         rec[R_T + e] = t;
     }
-    // K^ and diag(gamma) Q to the record, then the scaled operands of W and
-    // U~ in place
+    // K^ and diag(gamma) Q to the record
     const float GCp = Gs[C - 1];
     for (int e = tid; e < C * D; e += kPrepB) {
         const int i = e >> 7, d = e & 127;
-        const float kv = Ks[i * LW + d];
-        rec[R_KH + e] = kv * __expf(GCp - Gs[i]);
+        rec[R_KH + e] = Ks[i * LW + d] * __expf(GCp - Gs[i]);
         rec[R_QT + e] = Qs[i * LW + d] * gam[i];
-        Ks[i * LW + d] = kv * Bs[i] * gam[i];
-        Vs[i * LW + d] *= Bs[i];
     }
     if (tid < C) {
         rec[R_G + tid] = Gs[tid];
         rec[R_B + tid] = Bs[tid];
     }
     __syncthreads();
-    tgemm<C, D, kPrepB>(C, [&](int i, int j) { return Tp[i * LN + j]; },
+    // W = T diag(beta gamma) K and U~ = T diag(beta) V, the scales taken
+    // with T so that K and V stay exact operands
+    tgemm<C, D, kPrepB, 1, false, false, kX>(C, [&](int i, int j) { return Tp[i * LN + j] * Bs[j] * gam[j]; },
                        [&](int j, int d) { return Ks[j * LW + d]; },
                        [&](int i, int d, float x) { rec[R_W + i * D + d] = x; });
-    tgemm<C, D, kPrepB>(C, [&](int i, int j) { return Tp[i * LN + j]; },
+    tgemm<C, D, kPrepB, 1, false, false, kX>(C, [&](int i, int j) { return Tp[i * LN + j] * Bs[j]; },
                        [&](int j, int d) { return Vs[j * LW + d]; },
                        [&](int i, int d, float x) { rec[R_UT + i * D + d] = x; });
 }
@@ -480,7 +514,7 @@ bwd_forward_kernel(const float *__restrict__ h0, const int32_t *__restrict__ cu,
         }
         store_rows(rec + R_S, Sr, r0);
         // U[j][r0 + r] = U~[j][r0 + r] - sum_d W[j][d] S[r][d]
-        tgemm<C, kRowBlock, kChainThreads>(D, [&](int j, int d) { return Ws[j * LW4 + d]; },
+        tgemm<C, kRowBlock, kChainThreads, 2, true>(D, [&](int j, int d) { return Ws[j * LW4 + d]; },
                                            [&](int d, int r) { return Sr[r * LW4 + d]; },
                                            [&](int j, int r, float x) {
                                                const float u = Us[j * kRowBlock + r] - x;
@@ -497,7 +531,7 @@ bwd_forward_kernel(const float *__restrict__ h0, const int32_t *__restrict__ cu,
         __syncthreads();   // K^ and G of chunk c in place
         {   // S[r][d] = e^{G_C} S[r][d] + sum_j U[j][r] K^[j][d]
             const float gC = __expf(Gs[C - 1]);
-            tgemm<kRowBlock, D, kChainThreads>(C, [&](int r, int j) { return Ut[r * LN4 + j]; },
+            tgemm<kRowBlock, D, kChainThreads, 2, true>(C, [&](int r, int j) { return Ut[r * LN4 + j]; },
                                                [&](int j, int d) { return Kh[j * LW8 + d]; },
                                                [&](int r, int d, float x) {
                                                    Sr[r * LW4 + d] = fmaf(gC, Sr[r * LW4 + d], x);
@@ -586,10 +620,10 @@ bwd_reverse_kernel(const IoT *__restrict__ dO, const float *__restrict__ dSf,
         store_rows(rec + R_L, Lr, r0);
         {   // dU[j][r] = sum_d K^[j][d] L[r][d] + sum_i P[i][j] dO[i][r]
             float du[2][2];
-            tgemm_rc<C, kRowBlock, kChainThreads>(D, [&](int j, int d) { return Kh[j * LW4 + d]; },
+            tgemm_rc<C, kRowBlock, kChainThreads, 2, true>(D, [&](int j, int d) { return Kh[j * LW4 + d]; },
                                                   [&](int d, int r) { return Lr[r * LW4 + d]; },
                                                   [&](int sr, int sc, int, int, float x) { du[sr][sc] = x; });
-            tgemm_rc<C, kRowBlock, kChainThreads>(C, [&](int j, int i) { return PT[j * LN4 + i]; },
+            tgemm_rc<C, kRowBlock, kChainThreads, 2, true, false, kIoExact<IoT>>(C, [&](int j, int i) { return PT[j * LN4 + i]; },
                                                   [&](int i, int r) { return dOt[r * LN4 + i]; },
                                                   [&](int sr, int sc, int j, int r, float x) {
                                                       const float v = du[sr][sc] + x;
@@ -609,11 +643,11 @@ bwd_reverse_kernel(const IoT *__restrict__ dO, const float *__restrict__ dSf,
         __syncthreads();   // gamma Q, W and G of chunk c in place
         {   // L[r][d] = e^{G_C} L[r][d] + sum_i dO[i][r] gamma_i q_i[d] - sum_j dU[j][r] W[j][d]
             float la[2][4];
-            tgemm_rc<kRowBlock, D, kChainThreads>(C, [&](int r, int i) { return dOt[r * LN4 + i]; },
+            tgemm_rc<kRowBlock, D, kChainThreads, 2, true, kIoExact<IoT>>(C, [&](int r, int i) { return dOt[r * LN4 + i]; },
                                                   [&](int i, int d) { return Qt[i * LW8 + d]; },
                                                   [&](int sr, int sc, int, int, float x) { la[sr][sc] = x; });
             const float gC = __expf(Gs[C - 1]);
-            tgemm_rc<kRowBlock, D, kChainThreads>(C, [&](int r, int j) { return dUt[r * LN4 + j]; },
+            tgemm_rc<kRowBlock, D, kChainThreads, 2, true>(C, [&](int r, int j) { return dUt[r * LN4 + j]; },
                                                   [&](int j, int d) { return Ws[j * LW8 + d]; },
                                                   [&](int sr, int sc, int r, int d, float x) {
                                                       Lr[r * LW4 + d] = fmaf(gC, Lr[r * LW4 + d], la[sr][sc] - x);
@@ -760,7 +794,7 @@ bwd_local_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT
                               [&](int j, int d, float x) { RC[j * LW + d] = -x; });
     {
         float rowacc[4] = {0.f, 0.f, 0.f, 0.f};
-        tgemm_rc<C, D, kLocalThreads>(D, [&](int i, int r) { return RD[i * LW + r]; },
+        tgemm_rc<C, D, kLocalThreads, 1, false, kIoExact<IoT>>(D, [&](int i, int r) { return RD[i * LW + r]; },
                                   [&](int r, int d) { return RA[r * LW + d]; },
                                   [&](int tr, int tc, int i, int d, float x) {
                                       dqacc[tr][tc] = gam[i] * x;
@@ -774,7 +808,7 @@ bwd_local_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT
     copy_rows<kLocalThreads>(RA, LW, rec + R_U, C, D);
     copy_rows<kLocalThreads>(N1, LN, rec + R_T, C, C);
     __syncthreads();
-    tgemm<C, C, kLocalThreads>(D, [&](int i, int r) { return RD[i * LW + r]; },
+    tgemm<C, C, kLocalThreads, 1, false, kIoExact<IoT>>(D, [&](int i, int r) { return RD[i * LW + r]; },
                               [&](int r, int j) { return RA[j * LW + r]; },
                               [&](int i, int j, float x) { N2[i * LN + j] = j <= i ? x : 0.f; });
     __syncthreads();
@@ -804,12 +838,12 @@ bwd_local_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT
         flush_rows(dB, bacc);
         flush_rows(dG, gacc);
     }
-    tgemm<C, C, kLocalThreads>(D, [&](int i, int r) { return RB[i * LW + r]; },
-                              [&](int r, int j) { return Bs[j] * RD[j * LW + r]; },
-                              [&](int i, int j, float x) { N3[i * LN + j] = x; });
-    tgemm<C, C, kLocalThreads>(D, [&](int i, int d) { return RC[i * LW + d]; },
-                              [&](int d, int j) { return Bs[j] * gam[j] * RA[j * LW + d]; },
-                              [&](int i, int j, float x) { N3[i * LN + j] += x; });
+    tgemm<C, C, kLocalThreads, 1, false, false, kIoExact<IoT>>(
+        D, [&](int i, int r) { return RB[i * LW + r]; }, [&](int r, int j) { return RD[j * LW + r]; },
+        [&](int i, int j, float x) { N3[i * LN + j] = Bs[j] * x; });
+    tgemm<C, C, kLocalThreads, 1, false, false, kIoExact<IoT>>(
+        D, [&](int i, int d) { return RC[i * LW + d]; }, [&](int d, int j) { return RA[j * LW + d]; },
+        [&](int i, int j, float x) { N3[i * LN + j] += Bs[j] * gam[j] * x; });
     __syncthreads();
 
     // ---- phase D: dA = -T^T dT T^T, then the A and P terms ------------------------
@@ -826,32 +860,48 @@ bwd_local_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT
     copy_rows<kLocalThreads>(AR, LN, rec + R_AR, C, C);
     copy_rows<kLocalThreads>(N1, LN, rec + R_P, C, C);
     __syncthreads();
-    for (int e = tid; e < C * C; e += kLocalThreads) {
-        const int i = e >> 6, j = e & 63;
-        const float R = j <= i ? __expf(Gs[i] - Gs[j]) : 0.f;
-        const float da = N3[i * LN + j], ar = AR[i * LN + j];
-        const float ea = da * Bs[i] * ar;            // dA o A
-        const float dp = N2[i * LN + j], ep = dp * N1[j * LN + i];   // dP o P (N1 holds P^T)
-        if (da != 0.f || dp != 0.f) {
-            atomicAdd(&dB[i], da * ar);
-            atomicAdd(&dG[i], ea + ep);
-            atomicAdd(&dG[j], -(ea + ep));
+    {
+        // a warp takes half a row i per step: the row sums of dA o A (for
+        // dbeta_i) and of dA o A + dP o P (for dG_i) are reduced over the
+        // warp; a thread's column j = tid % 64 is the same at every step, so
+        // its sum for dG_j stays in a register
+        const int j = tid & (C - 1);
+        float colacc = 0.f;
+        for (int e = tid; e < C * C; e += kLocalThreads) {
+            const int i = e >> 6;
+            const float R = j <= i ? __expf(Gs[i] - Gs[j]) : 0.f;
+            const float da = N3[i * LN + j], ar = AR[i * LN + j];
+            const float ea = da * Bs[i] * ar;                           // dA o A
+            const float dp = N2[i * LN + j], ep = dp * N1[j * LN + i];   // dP o P (N1 holds P^T)
+            float rb = da * ar, rg = ea + ep;
+            colacc -= rg;
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                rb += __shfl_xor_sync(0xffffffffu, rb, off);
+                rg += __shfl_xor_sync(0xffffffffu, rg, off);
+            }
+            if ((tid & 31) == 0) {
+                atomicAdd(&dB[i], rb);
+                atomicAdd(&dG[i], rg);
+            }
+            N3[i * LN + j] = da * Bs[i] * R;             // M = dA o beta_i R
+            N2[i * LN + j] = dp * R;                     // dP o R
         }
-        N3[i * LN + j] = da * Bs[i] * R;             // M = dA o beta_i R
-        N2[i * LN + j] = dp * R;                     // dP o R
+        atomicAdd(&dG[j], colacc);
     }
     load_io_rows<kLocalThreads>(RB, q, tok0, cl, Hqk, hq);   // Q rows over the finished Y
     __syncthreads();
     auto add_dk = [&](int tr, int tc, int, int, float x) { dkacc[tr][tc] += x; };
-    tgemm_rc<C, D, kLocalThreads>(C, [&](int i, int j) { return N3[i * LN + j]; },
-                                 [&](int j, int d) { return RA[j * LW + d]; }, add_dk);
-    tgemm_rc<C, D, kLocalThreads>(C, [&](int j, int i) { return N3[i * LN + j]; },
-                                 [&](int i, int d) { return RA[i * LW + d]; }, add_dk);
-    tgemm_rc<C, D, kLocalThreads>(C, [&](int i, int j) { return N2[i * LN + j]; },
-                                 [&](int j, int d) { return RA[j * LW + d]; },
-                                 [&](int tr, int tc, int, int, float x) { dqacc[tr][tc] += x; });
-    tgemm_rc<C, D, kLocalThreads>(C, [&](int j, int i) { return N2[i * LN + j]; },
-                                 [&](int i, int d) { return RB[i * LW + d]; }, add_dk);
+    constexpr bool kX = kIoExact<IoT>;
+    tgemm_rc<C, D, kLocalThreads, 1, false, false, kX>(C, [&](int i, int j) { return N3[i * LN + j]; },
+                                                        [&](int j, int d) { return RA[j * LW + d]; }, add_dk);
+    tgemm_rc<C, D, kLocalThreads, 1, false, false, kX>(C, [&](int j, int i) { return N3[i * LN + j]; },
+                                                        [&](int i, int d) { return RA[i * LW + d]; }, add_dk);
+    tgemm_rc<C, D, kLocalThreads, 1, false, false, kX>(C, [&](int i, int j) { return N2[i * LN + j]; },
+                                                        [&](int j, int d) { return RA[j * LW + d]; },
+                                                        [&](int tr, int tc, int, int, float x) { dqacc[tr][tc] += x; });
+    tgemm_rc<C, D, kLocalThreads, 1, false, false, kX>(C, [&](int j, int i) { return N2[i * LN + j]; },
+                                                        [&](int i, int d) { return RB[i * LW + d]; }, add_dk);
     {
         // one sum per element: a store when the chunk's head owns its q/k
         // head, else an atomic (the value heads of a group share it)
