@@ -60,7 +60,9 @@ constexpr size_t R_S = R_DU + C * D;            // state entering the chunk [128
 constexpr size_t R_L = R_S + D * D;             // adjoint of the state leaving it [128][128]
 constexpr size_t R_KH = R_L + D * D;            // K^ [64][128]
 constexpr size_t R_QT = R_KH + C * D;           // diag(gamma) Q [64][128]
-constexpr size_t R_FLOATS = R_QT + C * D;       // 94,336 floats
+constexpr size_t R_Y = R_QT + C * D;            // dO^T diag(gamma) Q [128][128]
+constexpr size_t R_Z = R_Y + D * D;             // P^T dO [64][128]
+constexpr size_t R_FLOATS = R_Z + C * D;        // 118,912 floats
 constexpr size_t kBaseBytes = 256;              // sequence chunk offsets precede the records
 
 constexpr int LW = D + 4;    // padded row of 128 floats (4 mod 32: see the products)
@@ -324,14 +326,16 @@ constexpr uint32_t PB_A = PB_V + C * LW;            // A, swizzled 64 x 64 (the 
 constexpr uint32_t PB_T = PB_A + C * C;             // T, swizzled 64 x 64
 constexpr uint32_t PB_X = PB_T + C * C;             // the inverse's 1024-float scratch
 constexpr uint32_t PB_TP = PB_X + 1024;             // T [64][65], zero above the diagonal
-constexpr uint32_t PB_G = PB_TP + C * LN;           // G [64], gamma [64], beta [64]
+constexpr uint32_t PB_DO = PB_TP + C * LN;          // dO [64][LW]
+constexpr uint32_t PB_P = PB_DO + C * LW;           // P [64][LN]
+constexpr uint32_t PB_G = PB_P + C * LN;            // G [64], gamma [64], beta [64]
 constexpr uint32_t PB_FLOATS = PB_G + 3 * C;
 constexpr uint32_t PB_SMEM = PB_FLOATS * sizeof(float);
 
 template <typename IoT>
 __global__ void __launch_bounds__(kPrepB, 1)
 bwd_prep_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT *__restrict__ v,
-                const float *__restrict__ g, const float *__restrict__ beta,
+                const float *__restrict__ g, const float *__restrict__ beta, const IoT *__restrict__ dO,
                 const int32_t *__restrict__ cu, int num_seqs, int total_T, int Hqk, int H,
                 const int32_t *__restrict__ base, float *__restrict__ recs) {
     extern __shared__ __align__(16) float fs[];
@@ -342,11 +346,13 @@ bwd_prep_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT 
     sequence_range(cu, n, num_seqs, total_T, t0, len);
     const int tok0 = t0 + c * C, cl = min(C, len - c * C), hq = h / (H / Hqk);
     float *rec = recs + ((size_t)gc * H + h) * R_FLOATS;
-    float *Ks = fs + PB_K, *Qs = fs + PB_Q, *Vs = fs + PB_V, *Tp = fs + PB_TP;
+    float *Ks = fs + PB_K, *Qs = fs + PB_Q, *Vs = fs + PB_V, *Tp = fs + PB_TP, *DOs = fs + PB_DO,
+          *Ps = fs + PB_P;
     float *Gs = fs + PB_G, *gam = Gs + C, *Bs = gam + C;
     load_io_rows<kPrepB>(Ks, k, tok0, cl, Hqk, hq);
     load_io_rows<kPrepB>(Qs, q, tok0, cl, Hqk, hq);
     load_io_rows<kPrepB>(Vs, v, tok0, cl, H, h);
+    load_io_rows<kPrepB>(DOs, dO, tok0, cl, H, h);
     if (tid < 32) {   // gates of tokens 2 tid, 2 tid + 1: clamped, cumulated, 0 past the end
         const int i0 = 2 * tid, i1 = i0 + 1;
         const float g0 = i0 < cl ? clamp_log_gate(g[(size_t)(tok0 + i0) * H + h]) : 0.f;
@@ -378,7 +384,9 @@ bwd_prep_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT 
     tgemm<C, C, kPrepB, 1, false, kX, kX>(D, [&](int i, int d) { return Qs[i * LW + d]; },
                        [&](int d, int j) { return Ks[j * LW + d]; },
                        [&](int i, int j, float x) {
-                           rec[R_P + j * C + i] = j <= i ? x * __expf(Gs[i] - Gs[j]) : 0.f;
+                           const float pv = j <= i ? x * __expf(Gs[i] - Gs[j]) : 0.f;
+                           rec[R_P + j * C + i] = pv;
+                           Ps[i * LN + j] = pv;
                        });
     __syncthreads();
     unit_lower_inverse_f32(Af, fs + PB_T, fs + PB_X, tid);   // ends synchronised
@@ -408,6 +416,14 @@ bwd_prep_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT 
     tgemm<C, D, kPrepB, 1, false, false, kX>(C, [&](int i, int j) { return Tp[i * LN + j] * Bs[j]; },
                        [&](int j, int d) { return Vs[j * LW + d]; },
                        [&](int i, int d, float x) { rec[R_UT + i * D + d] = x; });
+    // the upstream gradient's terms of the adjoint chain, which depend on the
+    // chunk alone: Y = dO^T diag(gamma) Q and Z = P^T dO
+    tgemm<D, D, kPrepB, 1, false, kX>(C, [&](int r, int i) { return DOs[i * LW + r]; },
+                                      [&](int i, int d) { return Qs[i * LW + d] * gam[i]; },
+                                      [&](int r, int d, float x) { rec[R_Y + r * D + d] = x; });
+    tgemm<C, D, kPrepB, 1, false, false, kX>(C, [&](int j, int i) { return Ps[i * LN + j]; },
+                                             [&](int i, int r) { return DOs[i * LW + r]; },
+                                             [&](int j, int r, float x) { rec[R_Z + j * D + r] = x; });
 }
 
 // ------------------------------------------------------ forward / reverse ----
@@ -439,12 +455,6 @@ __device__ __forceinline__ void stage_c_by_d(float *dst, int ld, const float *sr
 #pragma unroll 8
     for (int e = threadIdx.x; e < C * D / 4; e += kChainThreads)
         cp16(dst + (e >> 5) * ld + (e & 31) * 4, src + e * 4);
-}
-// 64 x 64 floats into rows of LN4 floats.
-__device__ __forceinline__ void stage_c_by_c(float *dst, const float *src) {
-#pragma unroll 4
-    for (int e = threadIdx.x; e < C * C / 4; e += kChainThreads)
-        cp16(dst + (e >> 4) * LN4 + (e & 15) * 4, src + e * 4);
 }
 // Columns r0 .. r0 + 15 of a 64 x 128 record field into rows of 16 floats.
 __device__ __forceinline__ void stage_strip(float *dst, const float *src, int r0) {
@@ -549,20 +559,28 @@ bwd_forward_kernel(const float *__restrict__ h0, const int32_t *__restrict__ cu,
 
 constexpr uint32_t CR_L = 0;                             // L rows [16][LW4]
 constexpr uint32_t CR_DUT = CR_L + kRowBlock * LW4;      // dU^T [16][LN4]
-constexpr uint32_t CR_DOT = CR_DUT + kRowBlock * LN4;    // dO^T, columns r0 .. r0 + 15 [16][LN4]
-constexpr uint32_t CR_KH = CR_DOT + kRowBlock * LN4;     // K^ [64][LW4]
-constexpr uint32_t CR_PT = CR_KH + C * LW4;              // P^T [64][LN4]
-constexpr uint32_t CR_QT = CR_PT + C * LN4;              // diag(gamma) Q [64][LW8]
-constexpr uint32_t CR_W = CR_QT + C * LW8;               // W [64][LW8]
-constexpr uint32_t CR_G = CR_W + C * LW8;                // G [64]
+constexpr uint32_t CR_KH = CR_DUT + kRowBlock * LN4;     // K^ [64][LW4]
+constexpr uint32_t CR_ZS = CR_KH + C * LW4;              // Z columns r0 .. r0 + 15 [64][16]
+constexpr uint32_t CR_W = CR_ZS + C * kRowBlock;         // W [64][LW8]
+constexpr uint32_t CR_YS = CR_W + C * LW8;               // Y rows r0 .. r0 + 15 [16][LW4]
+constexpr uint32_t CR_G = CR_YS + kRowBlock * LW4;       // G [64]
 constexpr uint32_t CR_SMEM = (CR_G + C) * sizeof(float);
 
-template <typename IoT>
+// Rows r0 .. r0 + 15 of a [128][128] record field into rows of LW4 floats.
+__device__ __forceinline__ void stage_row_block(float *dst, const float *src, int r0) {
+#pragma unroll
+    for (int e = threadIdx.x; e < kRowBlock * D / 4; e += kChainThreads)
+        cp16(dst + (e >> 5) * LW4 + (e & 31) * 4, src + (size_t)r0 * D + e * 4);
+}
+
+// The adjoint chain, chunks last to first: with the chunk's upstream terms
+// Y = dO^T diag(gamma) Q and Z = P^T dO taken from the record,
+//   dU = Z + K^ L'^T,   L = e^{G_C} L' + Y - dU^T W
+// (L' the adjoint of the state leaving the chunk, L of the one entering it).
 __global__ void __launch_bounds__(kChainThreads, 1)
-bwd_reverse_kernel(const IoT *__restrict__ dO, const float *__restrict__ dSf,
-                   float *__restrict__ dh0, const int32_t *__restrict__ cu, int num_seqs,
-                   int total_T, int H, const int32_t *__restrict__ base, long long slots,
-                   float *__restrict__ recs) {
+bwd_reverse_kernel(const float *__restrict__ dSf, float *__restrict__ dh0,
+                   const int32_t *__restrict__ cu, int num_seqs, int total_T, int H,
+                   const int32_t *__restrict__ base, long long slots, float *__restrict__ recs) {
     extern __shared__ __align__(16) float fs[];
     const int chain = blockIdx.x, h = chain % H, n = chain / H, r0 = blockIdx.y * kRowBlock;
     const int tid = threadIdx.x;
@@ -570,95 +588,65 @@ bwd_reverse_kernel(const IoT *__restrict__ dO, const float *__restrict__ dSf,
     sequence_range(cu, n, num_seqs, total_T, t0, len);
     const int b0 = base[n];
     const int nch = (int)min((long long)(len + C - 1) / C, max(slots - b0, 0ll));
-    float *Lr = fs + CR_L, *dUt = fs + CR_DUT, *dOt = fs + CR_DOT, *Kh = fs + CR_KH,
-          *PT = fs + CR_PT, *Qt = fs + CR_QT, *Ws = fs + CR_W, *Gs = fs + CR_G;
+    float *Lr = fs + CR_L, *dUt = fs + CR_DUT, *Kh = fs + CR_KH, *Zs = fs + CR_ZS, *Ws = fs + CR_W,
+          *Ys = fs + CR_YS, *Gs = fs + CR_G;
     auto rec_of = [&](int c) { return recs + ((size_t)(b0 + c) * H + h) * R_FLOATS; };
-    // dO[i][r0 + 4 e .. r0 + 4 e + 3] of chunk c, i = tid / 4, e = tid % 4 (0
-    // past the sequence's end), and its place in dO^T
-    const int di = tid >> 2, dr = (tid & 3) * 4;
-    auto load_dO = [&](int c, float (&x)[4]) {
-        x[0] = x[1] = x[2] = x[3] = 0.f;
-        if (di < min(C, len - c * C)) ld4io(dO + ((size_t)(t0 + c * C + di) * H + h) * D + r0 + dr, x);
-    };
-    auto put_dO = [&](const float (&x)[4]) {
-#pragma unroll
-        for (int u = 0; u < 4; ++u) dOt[(dr + u) * LN4 + di] = x[u];
-    };
     for (int e = tid; e < kRowBlock * D; e += kChainThreads) {
         const int r = e >> 7, d = e & 127;
         Lr[r * LW4 + d] = dSf != nullptr ? dSf[((size_t)chain * D + r0 + r) * D + d] : 0.f;
     }
-    // copy groups, in order: {K^, P^T} and {gamma Q, W, G} of every chunk
+    // copy groups, in order: {K^, Z} and {W, Y, G} of every chunk
     if (nch > 0) {
         stage_c_by_d(Kh, LW4, rec_of(nch - 1) + R_KH);
-        stage_c_by_c(PT, rec_of(nch - 1) + R_P);
+        stage_strip(Zs, rec_of(nch - 1) + R_Z, r0);
         cp_commit();
-        stage_c_by_d(Qt, LW8, rec_of(nch - 1) + R_QT);
         stage_c_by_d(Ws, LW8, rec_of(nch - 1) + R_W);
+        stage_row_block(Ys, rec_of(nch - 1) + R_Y, r0);
         stage_g(Gs, rec_of(nch - 1) + R_G);
         cp_commit();
-        float x[4];
-        load_dO(nch - 1, x);
-        put_dO(x);
     }
     for (int c = nch - 1; c >= 0; --c) {
         float *rec = rec_of(c);
         cp_wait<1>();
-        __syncthreads();   // K^, P^T, dO^T of chunk c and the adjoint rows in place
-        if (blockIdx.y == 0 && c >= 2) {   // chunk c - 2 towards L2
+        __syncthreads();   // K^ and Z of chunk c and the adjoint rows in place
+        if (tid == 0 && blockIdx.y == 0 && c >= 2) {   // chunk c - 2 towards L2
             const float *pv = rec_of(c - 2);
-            if (tid == 0) {
-                tc::bulk_prefetch_l2(pv + R_KH, 2 * C * D * sizeof(float));   // K^ and gamma Q
-                tc::bulk_prefetch_l2(pv + R_W, C * D * sizeof(float));
-                tc::bulk_prefetch_l2(pv + R_P, C * C * sizeof(float));
-                tc::bulk_prefetch_l2(pv + R_G, C * sizeof(float));
-            } else if (tid >= 32 && tid < 32 + C && tid - 32 < min(C, len - (c - 2) * C)) {
-                tc::bulk_prefetch_l2(dO + ((size_t)(t0 + (c - 2) * C + tid - 32) * H + h) * D,
-                                     D * sizeof(IoT));
-            }
+            tc::bulk_prefetch_l2(pv + R_KH, C * D * sizeof(float));
+            tc::bulk_prefetch_l2(pv + R_W, C * D * sizeof(float));
+            tc::bulk_prefetch_l2(pv + R_Y, D * D * sizeof(float));
+            tc::bulk_prefetch_l2(pv + R_Z, C * D * sizeof(float));
+            tc::bulk_prefetch_l2(pv + R_G, C * sizeof(float));
         }
         store_rows(rec + R_L, Lr, r0);
-        {   // dU[j][r] = sum_d K^[j][d] L[r][d] + sum_i P[i][j] dO[i][r]
-            float du[2][2];
-            tgemm_rc<C, kRowBlock, kChainThreads, 2, true>(D, [&](int j, int d) { return Kh[j * LW4 + d]; },
-                                                  [&](int d, int r) { return Lr[r * LW4 + d]; },
-                                                  [&](int sr, int sc, int, int, float x) { du[sr][sc] = x; });
-            tgemm_rc<C, kRowBlock, kChainThreads, 2, true, false, kIoExact<IoT>>(C, [&](int j, int i) { return PT[j * LN4 + i]; },
-                                                  [&](int i, int r) { return dOt[r * LN4 + i]; },
-                                                  [&](int sr, int sc, int j, int r, float x) {
-                                                      const float v = du[sr][sc] + x;
-                                                      dUt[r * LN4 + j] = v;
-                                                      rec[R_DU + j * D + r0 + r] = v;
-                                                  });
-        }
-        __syncthreads();   // K^ and P^T consumed, dU^T complete
-        float x[4] = {0.f, 0.f, 0.f, 0.f};
+        // dU[j][r0 + r] = Z[j][r0 + r] + sum_d K^[j][d] L[r][d]
+        tgemm<C, kRowBlock, kChainThreads, 2, true>(D, [&](int j, int d) { return Kh[j * LW4 + d]; },
+                                                    [&](int d, int r) { return Lr[r * LW4 + d]; },
+                                                    [&](int j, int r, float x) {
+                                                        const float v = Zs[j * kRowBlock + r] + x;
+                                                        dUt[r * LN4 + j] = v;
+                                                        rec[R_DU + j * D + r0 + r] = v;
+                                                    });
+        __syncthreads();   // K^ and Z consumed, dU^T complete
         if (c > 0) {
             stage_c_by_d(Kh, LW4, rec_of(c - 1) + R_KH);
-            stage_c_by_c(PT, rec_of(c - 1) + R_P);
-            load_dO(c - 1, x);
+            stage_strip(Zs, rec_of(c - 1) + R_Z, r0);
         }
         cp_commit();
         cp_wait<1>();
-        __syncthreads();   // gamma Q, W and G of chunk c in place
-        {   // L[r][d] = e^{G_C} L[r][d] + sum_i dO[i][r] gamma_i q_i[d] - sum_j dU[j][r] W[j][d]
-            float la[2][4];
-            tgemm_rc<kRowBlock, D, kChainThreads, 2, true, kIoExact<IoT>>(C, [&](int r, int i) { return dOt[r * LN4 + i]; },
-                                                  [&](int i, int d) { return Qt[i * LW8 + d]; },
-                                                  [&](int sr, int sc, int, int, float x) { la[sr][sc] = x; });
+        __syncthreads();   // W, Y and G of chunk c in place
+        {   // L[r][d] = e^{G_C} L[r][d] + Y[r0 + r][d] - sum_j dU[j][r] W[j][d]
             const float gC = __expf(Gs[C - 1]);
-            tgemm_rc<kRowBlock, D, kChainThreads, 2, true>(C, [&](int r, int j) { return dUt[r * LN4 + j]; },
-                                                  [&](int j, int d) { return Ws[j * LW8 + d]; },
-                                                  [&](int sr, int sc, int r, int d, float x) {
-                                                      Lr[r * LW4 + d] = fmaf(gC, Lr[r * LW4 + d], la[sr][sc] - x);
-                                                  });
+            tgemm<kRowBlock, D, kChainThreads, 2, true>(C, [&](int r, int j) { return dUt[r * LN4 + j]; },
+                                                        [&](int j, int d) { return Ws[j * LW8 + d]; },
+                                                        [&](int r, int d, float x) {
+                                                            Lr[r * LW4 + d] = fmaf(gC, Lr[r * LW4 + d], Ys[r * LW4 + d] - x);
+                                                        });
         }
-        __syncthreads();   // gamma Q, W, G and dO^T consumed
+        __syncthreads();   // W, Y and G consumed
         if (c > 0) {
-            stage_c_by_d(Qt, LW8, rec_of(c - 1) + R_QT);
             stage_c_by_d(Ws, LW8, rec_of(c - 1) + R_W);
+            stage_row_block(Ys, rec_of(c - 1) + R_Y, r0);
             stage_g(Gs, rec_of(c - 1) + R_G);
-            put_dO(x);
         }
         cp_commit();
     }
@@ -893,10 +881,10 @@ bwd_local_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT
     __syncthreads();
     auto add_dk = [&](int tr, int tc, int, int, float x) { dkacc[tr][tc] += x; };
     constexpr bool kX = kIoExact<IoT>;
-    tgemm_rc<C, D, kLocalThreads, 1, false, false, kX>(C, [&](int i, int j) { return N3[i * LN + j]; },
-                                                        [&](int j, int d) { return RA[j * LW + d]; }, add_dk);
-    tgemm_rc<C, D, kLocalThreads, 1, false, false, kX>(C, [&](int j, int i) { return N3[i * LN + j]; },
-                                                        [&](int i, int d) { return RA[i * LW + d]; }, add_dk);
+    // dk_i += sum_j M_ij k_j and dk_j += sum_i M_ij k_i: one product with M + M^T
+    tgemm_rc<C, D, kLocalThreads, 1, false, false, kX>(
+        C, [&](int i, int j) { return N3[i * LN + j] + N3[j * LN + i]; },
+        [&](int j, int d) { return RA[j * LW + d]; }, add_dk);
     tgemm_rc<C, D, kLocalThreads, 1, false, false, kX>(C, [&](int i, int j) { return N2[i * LN + j]; },
                                                         [&](int j, int d) { return RA[j * LW + d]; },
                                                         [&](int tr, int tc, int, int, float x) { dqacc[tr][tc] += x; });
@@ -950,19 +938,19 @@ cudaError_t launch_chunked(const IoT *q, const IoT *k, const IoT *v, const float
     if (e == cudaSuccess)
         e = ensure_dynamic_smem(reinterpret_cast<const void *>(bwd_forward_kernel), (int)CF_SMEM);
     if (e == cudaSuccess)
-        e = ensure_dynamic_smem(reinterpret_cast<const void *>(bwd_reverse_kernel<IoT>), (int)CR_SMEM);
+        e = ensure_dynamic_smem(reinterpret_cast<const void *>(bwd_reverse_kernel), (int)CR_SMEM);
     if (e == cudaSuccess)
         e = ensure_dynamic_smem(reinterpret_cast<const void *>(bwd_local_kernel<IoT>), (int)LB_SMEM);
     if (e != cudaSuccess) return e;
     bwd_chunk_base_kernel<<<1, 1024, 0, stream>>>(cu, num_seqs, total_T, base);
     const dim3 per_chunk((unsigned)max_total, (unsigned)H);
     const dim3 per_rows((unsigned)(num_seqs * H), D / kRowBlock);
-    bwd_prep_kernel<IoT><<<per_chunk, kPrepB, PB_SMEM, stream>>>(q, k, v, g, beta, cu, num_seqs,
+    bwd_prep_kernel<IoT><<<per_chunk, kPrepB, PB_SMEM, stream>>>(q, k, v, g, beta, dO, cu, num_seqs,
                                                                   total_T, Hqk, H, base, recs);
     bwd_forward_kernel<<<per_rows, kChainThreads, CF_SMEM, stream>>>(
         h0, cu, num_seqs, total_T, H, base, max_total, recs);
-    bwd_reverse_kernel<IoT><<<per_rows, kChainThreads, CR_SMEM, stream>>>(
-        dO, dSf, dh0, cu, num_seqs, total_T, H, base, max_total, recs);
+    bwd_reverse_kernel<<<per_rows, kChainThreads, CR_SMEM, stream>>>(
+        dSf, dh0, cu, num_seqs, total_T, H, base, max_total, recs);
     bwd_local_kernel<IoT><<<per_chunk, kLocalThreads, LB_SMEM, stream>>>(
         q, k, v, g, dO, cu, num_seqs, total_T, Hqk, H, base, recs, dq, dk, dv, dg, dbeta);
     return cudaGetLastError();

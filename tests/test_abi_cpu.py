@@ -327,11 +327,11 @@ def test_backward_rejects_a_missing_or_small_workspace(lib, kw):
 def test_backward_workspace_size(lib):
     # one state checkpoint per 16 tokens of every sequence, plus one per sequence
     assert gdr.gdr_backward_workspace_size(2, 100, 3, 64, 32) == (2 + 7) * 3 * 32 * 64 * 4
-    # d_k = d_v = 128: room for the chunked form, one 377,344-byte record per
+    # d_k = d_v = 128: room for the chunked form, one 475,648-byte record per
     # (chunk, head) for up to ceil(T / 64) + N chunks, after 256 bytes of
     # chunk offsets (more than the token loop's checkpoints)
-    assert gdr.gdr_backward_workspace_size(1, 8192, 16, 128, 128) == 256 + (128 + 1) * 16 * 377344
-    assert 256 + (128 + 1) * 16 * 377344 > (1 + 512) * 16 * 65536
+    assert gdr.gdr_backward_workspace_size(1, 8192, 16, 128, 128) == 256 + (128 + 1) * 16 * 475648
+    assert 256 + (128 + 1) * 16 * 475648 > (1 + 512) * 16 * 65536
 
 
 def test_bindings_reject_host_tensors_before_any_call():

@@ -82,9 +82,9 @@ def test_backward_bytes_per_launch():
               + 3 * act * 4          # dq, dk, dv (fp32)
               + H * d * d * 4)       # d_initial_state
     assert case.bytes == expect
-    # the chunked form's records: 377,344 bytes per (chunk, head) for up to
+    # the chunked form's records: 475,648 bytes per (chunk, head) for up to
     # T / 64 + 1 chunks (cu_seqlens given), after 256 bytes of chunk offsets
-    assert case.ws.numel() == 256 + (T // 64 + 1) * H * 377344
+    assert case.ws.numel() == 256 + (T // 64 + 1) * H * 475648
 
 
 def test_reference_arm_under_two_ranks_prints_once():
