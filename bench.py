@@ -608,7 +608,7 @@ class BackwardCase:
                       + T * (2 * Hqk * dk + H * dv) * 4 + state)
         self.flops = 0
         self.tokens = T
-        self.launches = 5   # chunk numbering, prep, forward chain, reverse chain, local gradients
+        self.launches = 4   # chunk numbering, prep, the two chains in one launch, local gradients
         self.path = None
         self.out = None
 

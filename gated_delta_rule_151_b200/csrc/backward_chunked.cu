@@ -484,8 +484,7 @@ constexpr uint32_t CF_US = CF_KH + C * LW8;              // U~ columns r0 .. r0 
 constexpr uint32_t CF_G = CF_US + C * kRowBlock;         // G [64]
 constexpr uint32_t CF_SMEM = (CF_G + C) * sizeof(float);
 
-__global__ void __launch_bounds__(kChainThreads, 1)
-bwd_forward_kernel(const float *__restrict__ h0, const int32_t *__restrict__ cu, int num_seqs,
+__device__ __forceinline__ void forward_chain(const float *__restrict__ h0, const int32_t *__restrict__ cu, int num_seqs,
                    int total_T, int H, const int32_t *__restrict__ base, long long slots,
                    float *__restrict__ recs) {
     extern __shared__ __align__(16) float fs[];
@@ -577,8 +576,7 @@ __device__ __forceinline__ void stage_row_block(float *dst, const float *src, in
 // Y = dO^T diag(gamma) Q and Z = P^T dO taken from the record,
 //   dU = Z + K^ L'^T,   L = e^{G_C} L' + Y - dU^T W
 // (L' the adjoint of the state leaving the chunk, L of the one entering it).
-__global__ void __launch_bounds__(kChainThreads, 1)
-bwd_reverse_kernel(const float *__restrict__ dSf, float *__restrict__ dh0,
+__device__ __forceinline__ void reverse_chain(const float *__restrict__ dSf, float *__restrict__ dh0,
                    const int32_t *__restrict__ cu, int num_seqs, int total_T, int H,
                    const int32_t *__restrict__ base, long long slots, float *__restrict__ recs) {
     extern __shared__ __align__(16) float fs[];
@@ -660,6 +658,20 @@ bwd_reverse_kernel(const float *__restrict__ dSf, float *__restrict__ dh0,
     }
 }
 
+// Both chains in one launch: blockIdx.z = 0 carries the state forward, 1 the
+// adjoint backward.  They share nothing (the chunk-local gradients need both,
+// afterwards), so a forward and a reverse CTA run side by side on an SM and
+// the tensor pipe serves both.
+constexpr uint32_t CH_SMEM = CF_SMEM > CR_SMEM ? CF_SMEM : CR_SMEM;
+__global__ void __launch_bounds__(kChainThreads, 2)
+bwd_chains_kernel(const float *__restrict__ h0, const float *__restrict__ dSf,
+                  float *__restrict__ dh0, const int32_t *__restrict__ cu, int num_seqs,
+                  int total_T, int H, const int32_t *__restrict__ base, long long slots,
+                  float *__restrict__ recs) {
+    if (blockIdx.z == 0) forward_chain(h0, cu, num_seqs, total_T, H, base, slots, recs);
+    else reverse_chain(dSf, dh0, cu, num_seqs, total_T, H, base, slots, recs);
+}
+
 // --------------------------------------------------------------- local ----
 // One CTA per (global chunk, value head): every gradient of the chunk's
 // tokens.  Shared memory (floats) is reused phase by phase:
@@ -720,11 +732,11 @@ bwd_local_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT
     };
     // everything the later phases read towards L2 while phase A runs: the
     // record's P, T, (K K^T) o R, G, beta and U .. gamma Q (64 KiB pieces),
-    // and the chunk's rows of q, k, v and dO
+    // and the chunk's rows of q, k and v
     if (tid == 0) {
         tc::bulk_prefetch_l2(rec + R_P, (3 * C * C + 2 * C) * sizeof(float));
-        for (size_t o = R_U; o < R_FLOATS; o += 16384)
-            tc::bulk_prefetch_l2(rec + o, (uint32_t)(min((size_t)16384, R_FLOATS - o) * sizeof(float)));
+        for (size_t o = R_U; o < R_Y; o += 16384)
+            tc::bulk_prefetch_l2(rec + o, (uint32_t)(min((size_t)16384, R_Y - o) * sizeof(float)));
     } else if (tid >= 64 && tid < 64 + 3 * C) {
         const int w = (tid - 64) / C, i = (tid - 64) % C;
         if (i < cl) {
@@ -750,8 +762,14 @@ bwd_local_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT
     __syncthreads();
     const float GC = Gs[C - 1], gC = __expf(GC);
     {
-        float part = 0.f;   // <S, L'> over this thread's entries
-        for (int e = tid; e < D * D; e += kLocalThreads) part = fmaf(rec[R_S + e], RA[(e >> 7) * LW + (e & 127)], part);
+        float part = 0.f;   // <S, L'> over this thread's entries, 16-byte loads
+        const float4 *s4 = reinterpret_cast<const float4 *>(rec + R_S);
+#pragma unroll 8
+        for (int e = tid; e < D * D / 4; e += kLocalThreads) {
+            const float4 x = __ldg(s4 + e);
+            const float4 y = *reinterpret_cast<const float4 *>(RA + (e >> 5) * LW + (e & 31) * 4);
+            part = fmaf(x.x, y.x, fmaf(x.y, y.y, fmaf(x.z, y.z, fmaf(x.w, y.w, part))));
+        }
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
         if ((tid & 31) == 0) atomicAdd(&misc[1], part);
@@ -855,6 +873,7 @@ bwd_local_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT
         // its sum for dG_j stays in a register
         const int j = tid & (C - 1);
         float colacc = 0.f;
+#pragma unroll 4
         for (int e = tid; e < C * C; e += kLocalThreads) {
             const int i = e >> 6;
             const float R = j <= i ? __expf(Gs[i] - Gs[j]) : 0.f;
@@ -936,21 +955,17 @@ cudaError_t launch_chunked(const IoT *q, const IoT *k, const IoT *v, const float
     float *recs = reinterpret_cast<float *>(ws + base_bytes);
     cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void *>(bwd_prep_kernel<IoT>), (int)PB_SMEM);
     if (e == cudaSuccess)
-        e = ensure_dynamic_smem(reinterpret_cast<const void *>(bwd_forward_kernel), (int)CF_SMEM);
-    if (e == cudaSuccess)
-        e = ensure_dynamic_smem(reinterpret_cast<const void *>(bwd_reverse_kernel), (int)CR_SMEM);
+        e = ensure_dynamic_smem(reinterpret_cast<const void *>(bwd_chains_kernel), (int)CH_SMEM);
     if (e == cudaSuccess)
         e = ensure_dynamic_smem(reinterpret_cast<const void *>(bwd_local_kernel<IoT>), (int)LB_SMEM);
     if (e != cudaSuccess) return e;
     bwd_chunk_base_kernel<<<1, 1024, 0, stream>>>(cu, num_seqs, total_T, base);
     const dim3 per_chunk((unsigned)max_total, (unsigned)H);
-    const dim3 per_rows((unsigned)(num_seqs * H), D / kRowBlock);
+    const dim3 per_rows((unsigned)(num_seqs * H), D / kRowBlock, 2);
     bwd_prep_kernel<IoT><<<per_chunk, kPrepB, PB_SMEM, stream>>>(q, k, v, g, beta, dO, cu, num_seqs,
                                                                   total_T, Hqk, H, base, recs);
-    bwd_forward_kernel<<<per_rows, kChainThreads, CF_SMEM, stream>>>(
-        h0, cu, num_seqs, total_T, H, base, max_total, recs);
-    bwd_reverse_kernel<<<per_rows, kChainThreads, CR_SMEM, stream>>>(
-        dSf, dh0, cu, num_seqs, total_T, H, base, max_total, recs);
+    bwd_chains_kernel<<<per_rows, kChainThreads, CH_SMEM, stream>>>(
+        h0, dSf, dh0, cu, num_seqs, total_T, H, base, max_total, recs);
     bwd_local_kernel<IoT><<<per_chunk, kLocalThreads, LB_SMEM, stream>>>(
         q, k, v, g, dO, cu, num_seqs, total_T, Hqk, H, base, recs, dq, dk, dv, dg, dbeta);
     return cudaGetLastError();
