@@ -167,7 +167,7 @@ template <int M, int N, int NTH, int KPAR = 1, bool PSPLIT = false, bool AEX = f
 __device__ __forceinline__ void tgemm_rc(int K, AF a, BF b, EPI epi) {
     using G = WarpGrid<M, N, NTH / 32>;
     constexpr int NP = PSPLIT ? 3 : 1;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int t = threadIdx.x & (NTH - 1), lane = t & 31, warp = t >> 5;
     const int gid = lane >> 2, tig = lane & 3;
     const int m0 = (warp / G::GN) * G::WM, n0 = (warp % G::GN) * G::WN;
     float acc[KPAR][NP][G::MT][G::NT][4];
@@ -247,13 +247,13 @@ __device__ __forceinline__ void tgemm(int K, AF a, BF b, EPI epi) {
 template <int M, int N, int NTH>
 __device__ __forceinline__ int tslot_row(int r) {
     using G = WarpGrid<M, N, NTH / 32>;
-    const int warp = threadIdx.x >> 5, gid = (threadIdx.x & 31) >> 2;
+    const int warp = (threadIdx.x & (NTH - 1)) >> 5, gid = (threadIdx.x & 31) >> 2;
     return (warp / G::GN) * G::WM + (r >> 1) * 16 + gid + 8 * (r & 1);
 }
 template <int M, int N, int NTH>
 __device__ __forceinline__ int tslot_col(int c) {
     using G = WarpGrid<M, N, NTH / 32>;
-    const int warp = threadIdx.x >> 5, tig = threadIdx.x & 3;
+    const int warp = (threadIdx.x & (NTH - 1)) >> 5, tig = threadIdx.x & 3;
     return (warp % G::GN) * G::WN + (c >> 1) * 8 + 2 * tig + (c & 1);
 }
 
@@ -453,24 +453,25 @@ template <int N> __device__ __forceinline__ void cp_wait() {
 // 64 x 128 floats of a record field into rows of ld floats.
 __device__ __forceinline__ void stage_c_by_d(float *dst, int ld, const float *src) {
 #pragma unroll 8
-    for (int e = threadIdx.x; e < C * D / 4; e += kChainThreads)
+    for (int e = threadIdx.x & (kChainThreads - 1); e < C * D / 4; e += kChainThreads)
         cp16(dst + (e >> 5) * ld + (e & 31) * 4, src + e * 4);
 }
 // Columns r0 .. r0 + 15 of a 64 x 128 record field into rows of 16 floats.
 __device__ __forceinline__ void stage_strip(float *dst, const float *src, int r0) {
-    const int e = threadIdx.x;
+    const int e = threadIdx.x & (kChainThreads - 1);
     cp16(dst + (e >> 2) * kRowBlock + (e & 3) * 4, src + (e >> 2) * D + r0 + (e & 3) * 4);
 }
 // The chunk's 64 floats of G.
 __device__ __forceinline__ void stage_g(float *dst, const float *src) {
-    if (threadIdx.x < C / 4) cp16(dst + threadIdx.x * 4, src + threadIdx.x * 4);
+    const int e = threadIdx.x & (kChainThreads - 1);
+    if (e < C / 4) cp16(dst + e * 4, src + e * 4);
 }
 
 __device__ __forceinline__ float4 lds4(const float *p) { return *reinterpret_cast<const float4 *>(p); }
 // The CTA's 16 rows (padded) -> rows r0 .. r0 + 15 of a [128][128] field.
 __device__ __forceinline__ void store_rows(float *dst, const float *rows, int r0) {
 #pragma unroll
-    for (int e = threadIdx.x; e < kRowBlock * D / 4; e += kChainThreads) {
+    for (int e = threadIdx.x & (kChainThreads - 1); e < kRowBlock * D / 4; e += kChainThreads) {
         const int r = e >> 5, q = e & 31;
         *reinterpret_cast<float4 *>(dst + (size_t)(r0 + r) * D + 4 * q) = lds4(rows + r * LW4 + 4 * q);
     }
@@ -484,12 +485,11 @@ constexpr uint32_t CF_US = CF_KH + C * LW8;              // U~ columns r0 .. r0 
 constexpr uint32_t CF_G = CF_US + C * kRowBlock;         // G [64]
 constexpr uint32_t CF_SMEM = (CF_G + C) * sizeof(float);
 
-__device__ __forceinline__ void forward_chain(const float *__restrict__ h0, const int32_t *__restrict__ cu, int num_seqs,
+__device__ __forceinline__ void forward_chain(float *fs, const float *__restrict__ h0, const int32_t *__restrict__ cu, int num_seqs,
                    int total_T, int H, const int32_t *__restrict__ base, long long slots,
                    float *__restrict__ recs) {
-    extern __shared__ __align__(16) float fs[];
     const int chain = blockIdx.x, h = chain % H, n = chain / H, r0 = blockIdx.y * kRowBlock;
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x & (kChainThreads - 1);
     int t0, len;
     sequence_range(cu, n, num_seqs, total_T, t0, len);
     const int b0 = base[n];
@@ -514,7 +514,7 @@ __device__ __forceinline__ void forward_chain(const float *__restrict__ h0, cons
     for (int c = 0; c < nch; ++c) {
         float *rec = rec_of(c);
         cp_wait<1>();
-        __syncthreads();   // W, U~ of chunk c and the state rows in place
+        group_sync(1);   // W, U~ of chunk c and the state rows in place
         if (tid == 0 && blockIdx.y == 0 && c + 2 < nch) {   // chunk c + 2 towards L2
             const float *nx = rec_of(c + 2);
             tc::bulk_prefetch_l2(nx + R_W, 2 * C * D * sizeof(float));   // W and U~
@@ -530,14 +530,14 @@ __device__ __forceinline__ void forward_chain(const float *__restrict__ h0, cons
                                                Ut[r * LN4 + j] = u;
                                                rec[R_U + j * D + r0 + r] = u;
                                            });
-        __syncthreads();   // W and U~ consumed, U^T complete
+        group_sync(1);   // W and U~ consumed, U^T complete
         if (c + 1 < nch) {
             stage_c_by_d(Ws, LW4, rec_of(c + 1) + R_W);
             stage_strip(Us, rec_of(c + 1) + R_UT, r0);
         }
         cp_commit();
         cp_wait<1>();
-        __syncthreads();   // K^ and G of chunk c in place
+        group_sync(1);   // K^ and G of chunk c in place
         {   // S[r][d] = e^{G_C} S[r][d] + sum_j U[j][r] K^[j][d]
             const float gC = __expf(Gs[C - 1]);
             tgemm<kRowBlock, D, kChainThreads, 2, true>(C, [&](int r, int j) { return Ut[r * LN4 + j]; },
@@ -546,7 +546,7 @@ __device__ __forceinline__ void forward_chain(const float *__restrict__ h0, cons
                                                    Sr[r * LW4 + d] = fmaf(gC, Sr[r * LW4 + d], x);
                                                });
         }
-        __syncthreads();   // K^ and G consumed
+        group_sync(1);   // K^ and G consumed
         if (c + 1 < nch) {
             stage_c_by_d(Kh, LW8, rec_of(c + 1) + R_KH);
             stage_g(Gs, rec_of(c + 1) + R_G);
@@ -568,7 +568,7 @@ constexpr uint32_t CR_SMEM = (CR_G + C) * sizeof(float);
 // Rows r0 .. r0 + 15 of a [128][128] record field into rows of LW4 floats.
 __device__ __forceinline__ void stage_row_block(float *dst, const float *src, int r0) {
 #pragma unroll
-    for (int e = threadIdx.x; e < kRowBlock * D / 4; e += kChainThreads)
+    for (int e = threadIdx.x & (kChainThreads - 1); e < kRowBlock * D / 4; e += kChainThreads)
         cp16(dst + (e >> 5) * LW4 + (e & 31) * 4, src + (size_t)r0 * D + e * 4);
 }
 
@@ -576,12 +576,11 @@ __device__ __forceinline__ void stage_row_block(float *dst, const float *src, in
 // Y = dO^T diag(gamma) Q and Z = P^T dO taken from the record,
 //   dU = Z + K^ L'^T,   L = e^{G_C} L' + Y - dU^T W
 // (L' the adjoint of the state leaving the chunk, L of the one entering it).
-__device__ __forceinline__ void reverse_chain(const float *__restrict__ dSf, float *__restrict__ dh0,
+__device__ __forceinline__ void reverse_chain(float *fs, const float *__restrict__ dSf, float *__restrict__ dh0,
                    const int32_t *__restrict__ cu, int num_seqs, int total_T, int H,
                    const int32_t *__restrict__ base, long long slots, float *__restrict__ recs) {
-    extern __shared__ __align__(16) float fs[];
     const int chain = blockIdx.x, h = chain % H, n = chain / H, r0 = blockIdx.y * kRowBlock;
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x & (kChainThreads - 1);
     int t0, len;
     sequence_range(cu, n, num_seqs, total_T, t0, len);
     const int b0 = base[n];
@@ -606,7 +605,7 @@ __device__ __forceinline__ void reverse_chain(const float *__restrict__ dSf, flo
     for (int c = nch - 1; c >= 0; --c) {
         float *rec = rec_of(c);
         cp_wait<1>();
-        __syncthreads();   // K^ and Z of chunk c and the adjoint rows in place
+        group_sync(2);   // K^ and Z of chunk c and the adjoint rows in place
         if (tid == 0 && blockIdx.y == 0 && c >= 2) {   // chunk c - 2 towards L2
             const float *pv = rec_of(c - 2);
             tc::bulk_prefetch_l2(pv + R_KH, C * D * sizeof(float));
@@ -624,14 +623,14 @@ __device__ __forceinline__ void reverse_chain(const float *__restrict__ dSf, flo
                                                         dUt[r * LN4 + j] = v;
                                                         rec[R_DU + j * D + r0 + r] = v;
                                                     });
-        __syncthreads();   // K^ and Z consumed, dU^T complete
+        group_sync(2);   // K^ and Z consumed, dU^T complete
         if (c > 0) {
             stage_c_by_d(Kh, LW4, rec_of(c - 1) + R_KH);
             stage_strip(Zs, rec_of(c - 1) + R_Z, r0);
         }
         cp_commit();
         cp_wait<1>();
-        __syncthreads();   // W, Y and G of chunk c in place
+        group_sync(2);   // W, Y and G of chunk c in place
         {   // L[r][d] = e^{G_C} L[r][d] + Y[r0 + r][d] - sum_j dU[j][r] W[j][d]
             const float gC = __expf(Gs[C - 1]);
             tgemm<kRowBlock, D, kChainThreads, 2, true>(C, [&](int r, int j) { return dUt[r * LN4 + j]; },
@@ -640,7 +639,7 @@ __device__ __forceinline__ void reverse_chain(const float *__restrict__ dSf, flo
                                                             Lr[r * LW4 + d] = fmaf(gC, Lr[r * LW4 + d], Ys[r * LW4 + d] - x);
                                                         });
         }
-        __syncthreads();   // W, Y and G consumed
+        group_sync(2);   // W, Y and G consumed
         if (c > 0) {
             stage_c_by_d(Ws, LW8, rec_of(c - 1) + R_W);
             stage_row_block(Ys, rec_of(c - 1) + R_Y, r0);
@@ -649,7 +648,7 @@ __device__ __forceinline__ void reverse_chain(const float *__restrict__ dSf, flo
         cp_commit();
     }
     cp_wait<0>();
-    __syncthreads();
+    group_sync(2);
     if (dh0 != nullptr) {
         for (int e = tid; e < kRowBlock * D; e += kChainThreads) {
             const int r = e >> 7, d = e & 127;
@@ -658,18 +657,21 @@ __device__ __forceinline__ void reverse_chain(const float *__restrict__ dSf, flo
     }
 }
 
-// Both chains in one launch: blockIdx.z = 0 carries the state forward, 1 the
-// adjoint backward.  They share nothing (the chunk-local gradients need both,
-// afterwards), so a forward and a reverse CTA run side by side on an SM and
-// the tensor pipe serves both.
-constexpr uint32_t CH_SMEM = CF_SMEM > CR_SMEM ? CF_SMEM : CR_SMEM;
-__global__ void __launch_bounds__(kChainThreads, 2)
+// Both chains in one CTA of 512 threads per (sequence, head, 16 rows):
+// warps 0-7 carry the state forward, warps 8-15 the adjoint backward, each
+// half on its own named barrier.  The two share nothing (the chunk-local
+// gradients need both, afterwards), so the SM's tensor pipe serves both.
+constexpr uint32_t CH_SMEM = CF_SMEM + CR_SMEM;
+__global__ void __launch_bounds__(2 * kChainThreads, 1)
 bwd_chains_kernel(const float *__restrict__ h0, const float *__restrict__ dSf,
                   float *__restrict__ dh0, const int32_t *__restrict__ cu, int num_seqs,
                   int total_T, int H, const int32_t *__restrict__ base, long long slots,
                   float *__restrict__ recs) {
-    if (blockIdx.z == 0) forward_chain(h0, cu, num_seqs, total_T, H, base, slots, recs);
-    else reverse_chain(dSf, dh0, cu, num_seqs, total_T, H, base, slots, recs);
+    extern __shared__ __align__(16) float fs[];
+    if (threadIdx.x < kChainThreads)
+        forward_chain(fs, h0, cu, num_seqs, total_T, H, base, slots, recs);
+    else
+        reverse_chain(fs + CF_SMEM / sizeof(float), dSf, dh0, cu, num_seqs, total_T, H, base, slots, recs);
 }
 
 // --------------------------------------------------------------- local ----
@@ -961,10 +963,10 @@ cudaError_t launch_chunked(const IoT *q, const IoT *k, const IoT *v, const float
     if (e != cudaSuccess) return e;
     bwd_chunk_base_kernel<<<1, 1024, 0, stream>>>(cu, num_seqs, total_T, base);
     const dim3 per_chunk((unsigned)max_total, (unsigned)H);
-    const dim3 per_rows((unsigned)(num_seqs * H), D / kRowBlock, 2);
+    const dim3 per_rows((unsigned)(num_seqs * H), D / kRowBlock);
     bwd_prep_kernel<IoT><<<per_chunk, kPrepB, PB_SMEM, stream>>>(q, k, v, g, beta, dO, cu, num_seqs,
                                                                   total_T, Hqk, H, base, recs);
-    bwd_chains_kernel<<<per_rows, kChainThreads, CH_SMEM, stream>>>(
+    bwd_chains_kernel<<<per_rows, 2 * kChainThreads, CH_SMEM, stream>>>(
         h0, dSf, dh0, cu, num_seqs, total_T, H, base, max_total, recs);
     bwd_local_kernel<IoT><<<per_chunk, kLocalThreads, LB_SMEM, stream>>>(
         q, k, v, g, dO, cu, num_seqs, total_T, Hqk, H, base, recs, dq, dk, dv, dg, dbeta);
