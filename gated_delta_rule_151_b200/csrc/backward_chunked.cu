@@ -21,17 +21,22 @@
 // lower), and from these dq, dk, dv, dbeta and the adjoints of G, whose
 // reverse cumulative sum within the chunk is dg.  Four launches:
 //
-//   prep    one CTA per (chunk, head): A, T, W, U~, P, G, beta (fp32).
-//   forward one CTA per (sequence, head, 16 state rows): the state entering
-//           every chunk and U, chunk after chunk.
-//   reverse the same CTAs, chunks last to first: L' of every chunk and dU;
-//           the adjoint of the initial state at the end.
-//   local   one CTA per (chunk, head): every gradient of the chunk's tokens.
+//   chunk base  the first global chunk of every sequence.
+//   prep        one CTA per (chunk, head): A, T, W, U~, P, K^, diag(gamma) Q,
+//               G, beta and the upstream terms of the adjoint chain,
+//               Y = dO^T diag(gamma) Q and Z = P^T dO (fp32 record).
+//   chains      one CTA of 512 threads per (sequence, head, 16 state rows):
+//               warps 0-7 carry the state forward (S and U of every chunk),
+//               warps 8-15 the adjoint backward (L' and dU = Z + K^ L'^T of
+//               every chunk, L = e^{G_C} L' + Y - dU^T W, the adjoint of the
+//               initial state at the end).
+//   local       one CTA per (chunk, head): every gradient of the chunk's
+//               tokens.
 //
-// Everything is fp32 on CUDA cores: a register-tiled product over padded
-// shared-memory operands (rows of 129 or 65 floats, so rows and columns are
-// both read without bank conflicts).  The chunk records live in the
-// workspace: 377,344 bytes per (chunk, head).
+// Every product runs on the tensor cores as warp-level tf32 MMAs in up to
+// three passes over tf32-split operands (fp32 accuracy; see the products
+// below).  The chunk records live in the workspace: 475,648 bytes per
+// (chunk, head).
 #include <cuda_bf16.h>
 
 #include <algorithm>
