@@ -58,7 +58,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 CHUNK = 64
 # the five benchmark configurations that run on the GPU (the tiny GDN case is
 # a parity-only configuration); the first is the headline
-DEFAULT_WORKLOADS = "varlen_gdn,gdn_prefill,kda_prefill,decode_gdn,decode_kda,prefill_fused_gdn"
+DEFAULT_WORKLOADS = "varlen_gdn,gdn_prefill,kda_prefill,decode_gdn,decode_kda,prefill_fused_gdn,backward_gdn"
 
 
 # ------------------------------------------------------------ plumbing ----
@@ -834,12 +834,39 @@ def bench_case(case, args, ws, rank, flush, stream, pk, pk_kind):
     }
 
 
+def cpu_baseline_backward(name, budget_s=8.0):
+    """The fp64 backward oracle (numpy, one thread), as it stands, on whole
+    heads of the gradient workload (all tokens) until about budget_s has
+    run; tokens/s scaled to the full workload's head count."""
+    from oracle import backward as B
+    from threadpoolctl import threadpool_limits
+    inp = I.workload("gdn_prefill", seed=0)
+    dO, dsf = I.make_grad_inputs(inp, seed=0)
+    cu = inp.cu_seqlens.numpy()
+    done, dt = 0, 0.0
+    with threadpool_limits(limits=1):
+        while done < inp.H and dt < budget_s:
+            h = slice(done, done + 1)
+            t = time.perf_counter()
+            B.backward(inp.q[:, h], inp.k[:, h], inp.v[:, h], inp.g[:, h], inp.beta[:, h],
+                       None if inp.h0 is None else inp.h0[:, h], cu, dO[:, h],
+                       None if dsf is None else dsf[:, h])
+            dt += time.perf_counter() - t
+            done += 1
+    value = inp.total_T * (done / inp.H) / dt
+    return {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{name}: {done} of {inp.H} heads, all {inp.total_T} tokens, fp64 numpy "
+                      f"backward oracle on one thread, {dt:.2f} s"}
+
+
 def cpu_baseline(name, budget_s=10.0):
     """The oracle, as it stands, on a bounded sample of the workload: whole
     heads (all tokens of every sequence) until the estimated cost reaches the
     budget.  Returns tokens/s scaled to the full workload's head count (a
     decode workload's tokens are its sequences' tokens: the oracle runs the
     same recurrence token by token)."""
+    if name == "backward_gdn":
+        return cpu_baseline_backward(name)
     import oracle
     inp = I.workload(name)
     cores = oracle.loop.default_threads()
@@ -856,10 +883,10 @@ def cpu_baseline(name, budget_s=10.0):
                       f"{inp.num_seqs} sequences, fp64 C loop, {dt:.2f} s"}
 
 
-# workloads whose recurrence the fp64 oracle runs (the prologue and the
-# backward have oracles of their own, not timed here)
+# workloads with a timed oracle: the fp64 C recurrence, or the fp64 backward
+# oracle for the gradient (the prologue's oracle is not timed here)
 CPU_BASELINE_WORKLOADS = ("tiny_gdn", "gdn_prefill", "kda_prefill", "varlen_gdn", "gqa_prefill",
-                          "decode_gdn", "decode_kda", "decode_spec_gdn")
+                          "decode_gdn", "decode_kda", "decode_spec_gdn", "backward_gdn")
 
 
 def run_reference(args, ws, rank):
