@@ -247,6 +247,93 @@ __device__ __forceinline__ void tgemm(int K, AF a, BF b, EPI epi) {
                                                 [&](int, int, int m, int n, float v) { epi(m, n, v); });
 }
 
+// The same products in bf16: each value x splits into x_hi = bf16(x) and
+// x_lo = bf16(x - x_hi) (16 significant bits together, the fp32 exponent
+// range), accumulated in fp32 as lo*hi + hi*lo + hi*hi with m16n8k16 MMAs
+// (twice the k-depth of a tf32 MMA per instruction).  Each product term is
+// off by about 2^-16 of its size, which the chunk-local gradients (one
+// product deep, nothing carried from chunk to chunk) can take; the chains
+// keep the tf32 form.  AEX / BEX as above (a bf16 input is exact).
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo_elem, float hi_elem) {
+    const __nv_bfloat162 p = __floats2bfloat162_rn(lo_elem, hi_elem);
+    return *reinterpret_cast<const uint32_t *>(&p);
+}
+// Two values -> their high pair and low pair.
+__device__ __forceinline__ void split_bf16x2(float x0, float x1, uint32_t &hi, uint32_t &lo) {
+    hi = pack_bf16(x0, x1);
+    const float h0 = __uint_as_float(hi << 16), h1 = __uint_as_float(hi & 0xFFFF0000u);
+    lo = pack_bf16(x0 - h0, x1 - h1);
+}
+
+// d (16 x 8, fp32) += a (16 x 16, bf16, row) * b (16 x 8, bf16, column).
+__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+        "{%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+// tgemm_rc's contract with bf16 products; K a multiple of 16.
+template <int M, int N, int NTH, bool AEX = false, bool BEX = false, class AF, class BF, class EPI>
+__device__ __forceinline__ void bgemm_rc(int K, AF a, BF b, EPI epi) {
+    using G = WarpGrid<M, N, NTH / 32>;
+    const int t = threadIdx.x & (NTH - 1), lane = t & 31, warp = t >> 5;
+    const int gid = lane >> 2, tig = lane & 3;
+    const int m0 = (warp / G::GN) * G::WM, n0 = (warp % G::GN) * G::WN;
+    float acc[G::MT][G::NT][4];
+#pragma unroll
+    for (int mt = 0; mt < G::MT; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < G::NT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[mt][nt][e] = 0.f;
+    auto take = [](float x0, float x1, uint32_t &hi, uint32_t &lo, bool exact) {
+        if (exact) hi = pack_bf16(x0, x1);
+        else split_bf16x2(x0, x1, hi, lo);
+    };
+#pragma unroll 2
+    for (int k0 = 0; k0 < K; k0 += 16) {
+        uint32_t ah[G::MT][4], al[G::MT][4], bh[G::NT][2], bl[G::NT][2];
+        const int ka = k0 + 2 * tig;
+#pragma unroll
+        for (int mt = 0; mt < G::MT; ++mt) {
+            const int m = m0 + mt * 16 + gid;
+            take(a(m, ka), a(m, ka + 1), ah[mt][0], al[mt][0], AEX);
+            take(a(m + 8, ka), a(m + 8, ka + 1), ah[mt][1], al[mt][1], AEX);
+            take(a(m, ka + 8), a(m, ka + 9), ah[mt][2], al[mt][2], AEX);
+            take(a(m + 8, ka + 8), a(m + 8, ka + 9), ah[mt][3], al[mt][3], AEX);
+        }
+#pragma unroll
+        for (int nt = 0; nt < G::NT; ++nt) {
+            const int n = n0 + nt * 8 + gid;
+            take(b(ka, n), b(ka + 1, n), bh[nt][0], bl[nt][0], BEX);
+            take(b(ka + 8, n), b(ka + 9, n), bh[nt][1], bl[nt][1], BEX);
+        }
+#pragma unroll
+        for (int mt = 0; mt < G::MT; ++mt)
+#pragma unroll
+            for (int nt = 0; nt < G::NT; ++nt) {
+                if (!AEX) mma_bf16(acc[mt][nt], al[mt], bh[nt]);
+                if (!BEX) mma_bf16(acc[mt][nt], ah[mt], bl[nt]);
+                mma_bf16(acc[mt][nt], ah[mt], bh[nt]);
+            }
+    }
+#pragma unroll
+    for (int mt = 0; mt < G::MT; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < G::NT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                epi(mt * 2 + (e >> 1), nt * 2 + (e & 1), m0 + mt * 16 + gid + 8 * (e >> 1),
+                    n0 + nt * 8 + 2 * tig + (e & 1), acc[mt][nt][e]);
+}
+
+template <int M, int N, int NTH, bool AEX = false, bool BEX = false, class AF, class BF, class EPI>
+__device__ __forceinline__ void bgemm(int K, AF a, BF b, EPI epi) {
+    bgemm_rc<M, N, NTH, AEX, BEX>(K, a, b, [&](int, int, int m, int n, float v) { epi(m, n, v); });
+}
+
 // Row of slot r and column of slot c of the calling thread in a <M, N, NTH>
 // product.
 template <int M, int N, int NTH>
@@ -415,18 +502,18 @@ bwd_prep_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT 
     __syncthreads();
     // W = T diag(beta gamma) K and U~ = T diag(beta) V, the scales taken
     // with T so that K and V stay exact operands
-    tgemm<C, D, kPrepB, 1, false, false, kX>(C, [&](int i, int j) { return Tp[i * LN + j] * Bs[j] * gam[j]; },
+    bgemm<C, D, kPrepB, false, kX>(C, [&](int i, int j) { return Tp[i * LN + j] * Bs[j] * gam[j]; },
                        [&](int j, int d) { return Ks[j * LW + d]; },
                        [&](int i, int d, float x) { rec[R_W + i * D + d] = x; });
-    tgemm<C, D, kPrepB, 1, false, false, kX>(C, [&](int i, int j) { return Tp[i * LN + j] * Bs[j]; },
+    bgemm<C, D, kPrepB, false, kX>(C, [&](int i, int j) { return Tp[i * LN + j] * Bs[j]; },
                        [&](int j, int d) { return Vs[j * LW + d]; },
                        [&](int i, int d, float x) { rec[R_UT + i * D + d] = x; });
     // the upstream gradient's terms of the adjoint chain, which depend on the
     // chunk alone: Y = dO^T diag(gamma) Q and Z = P^T dO
-    tgemm<D, D, kPrepB, 1, false, kX>(C, [&](int r, int i) { return DOs[i * LW + r]; },
+    bgemm<D, D, kPrepB, kX>(C, [&](int r, int i) { return DOs[i * LW + r]; },
                                       [&](int i, int d) { return Qs[i * LW + d] * gam[i]; },
                                       [&](int r, int d, float x) { rec[R_Y + r * D + d] = x; });
-    tgemm<C, D, kPrepB, 1, false, false, kX>(C, [&](int j, int i) { return Ps[i * LN + j]; },
+    bgemm<C, D, kPrepB, false, kX>(C, [&](int j, int i) { return Ps[i * LN + j]; },
                                              [&](int i, int r) { return DOs[i * LW + r]; },
                                              [&](int j, int r, float x) { rec[R_Z + j * D + r] = x; });
 }
@@ -528,7 +615,7 @@ __device__ __forceinline__ void forward_chain(float *fs, const float *__restrict
         }
         store_rows(rec + R_S, Sr, r0);
         // U[j][r0 + r] = U~[j][r0 + r] - sum_d W[j][d] S[r][d]
-        tgemm<C, kRowBlock, kChainThreads, 2, true>(D, [&](int j, int d) { return Ws[j * LW4 + d]; },
+        bgemm<C, kRowBlock, kChainThreads>(D, [&](int j, int d) { return Ws[j * LW4 + d]; },
                                            [&](int d, int r) { return Sr[r * LW4 + d]; },
                                            [&](int j, int r, float x) {
                                                const float u = Us[j * kRowBlock + r] - x;
@@ -545,7 +632,7 @@ __device__ __forceinline__ void forward_chain(float *fs, const float *__restrict
         group_sync(1);   // K^ and G of chunk c in place
         {   // S[r][d] = e^{G_C} S[r][d] + sum_j U[j][r] K^[j][d]
             const float gC = __expf(Gs[C - 1]);
-            tgemm<kRowBlock, D, kChainThreads, 2, true>(C, [&](int r, int j) { return Ut[r * LN4 + j]; },
+            bgemm<kRowBlock, D, kChainThreads>(C, [&](int r, int j) { return Ut[r * LN4 + j]; },
                                                [&](int j, int d) { return Kh[j * LW8 + d]; },
                                                [&](int r, int d, float x) {
                                                    Sr[r * LW4 + d] = fmaf(gC, Sr[r * LW4 + d], x);
@@ -621,7 +708,7 @@ __device__ __forceinline__ void reverse_chain(float *fs, const float *__restrict
         }
         store_rows(rec + R_L, Lr, r0);
         // dU[j][r0 + r] = Z[j][r0 + r] + sum_d K^[j][d] L[r][d]
-        tgemm<C, kRowBlock, kChainThreads, 2, true>(D, [&](int j, int d) { return Kh[j * LW4 + d]; },
+        bgemm<C, kRowBlock, kChainThreads>(D, [&](int j, int d) { return Kh[j * LW4 + d]; },
                                                     [&](int d, int r) { return Lr[r * LW4 + d]; },
                                                     [&](int j, int r, float x) {
                                                         const float v = Zs[j * kRowBlock + r] + x;
@@ -638,7 +725,7 @@ __device__ __forceinline__ void reverse_chain(float *fs, const float *__restrict
         group_sync(2);   // W, Y and G of chunk c in place
         {   // L[r][d] = e^{G_C} L[r][d] + Y[r0 + r][d] - sum_j dU[j][r] W[j][d]
             const float gC = __expf(Gs[C - 1]);
-            tgemm<kRowBlock, D, kChainThreads, 2, true>(C, [&](int r, int j) { return dUt[r * LN4 + j]; },
+            bgemm<kRowBlock, D, kChainThreads>(C, [&](int r, int j) { return dUt[r * LN4 + j]; },
                                                         [&](int j, int d) { return Ws[j * LW8 + d]; },
                                                         [&](int r, int d, float x) {
                                                             Lr[r * LW4 + d] = fmaf(gC, Lr[r * LW4 + d], Ys[r * LW4 + d] - x);
@@ -784,7 +871,7 @@ bwd_local_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT
     __syncthreads();
     {
         float rowacc[4] = {0.f, 0.f, 0.f, 0.f}, gcacc = 0.f;
-        tgemm_rc<C, D, kLocalThreads>(D, [&](int j, int r) { return RB[j * LW + r]; },
+        bgemm_rc<C, D, kLocalThreads>(D, [&](int j, int r) { return RB[j * LW + r]; },
                                   [&](int r, int d) { return RA[r * LW + d]; },
                                   [&](int tr, int tc, int j, int d, float x) {
                                       dkacc[tr][tc] = __expf(GC - Gs[j]) * x;
@@ -802,12 +889,12 @@ bwd_local_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT
     copy_rows<kLocalThreads>(RB, LW, rec + R_DU, C, D);
     load_io_rows<kLocalThreads>(RD, dO, tok0, cl, H, h);
     __syncthreads();
-    tgemm<C, D, kLocalThreads>(D, [&](int j, int r) { return RB[j * LW + r]; },
+    bgemm<C, D, kLocalThreads>(D, [&](int j, int r) { return RB[j * LW + r]; },
                               [&](int r, int d) { return RA[r * LW + d]; },
                               [&](int j, int d, float x) { RC[j * LW + d] = -x; });
     {
         float rowacc[4] = {0.f, 0.f, 0.f, 0.f};
-        tgemm_rc<C, D, kLocalThreads, 1, false, kIoExact<IoT>>(D, [&](int i, int r) { return RD[i * LW + r]; },
+        bgemm_rc<C, D, kLocalThreads, kIoExact<IoT>>(D, [&](int i, int r) { return RD[i * LW + r]; },
                                   [&](int r, int d) { return RA[r * LW + d]; },
                                   [&](int tr, int tc, int i, int d, float x) {
                                       dqacc[tr][tc] = gam[i] * x;
@@ -821,7 +908,7 @@ bwd_local_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT
     copy_rows<kLocalThreads>(RA, LW, rec + R_U, C, D);
     copy_rows<kLocalThreads>(N1, LN, rec + R_T, C, C);
     __syncthreads();
-    tgemm<C, C, kLocalThreads, 1, false, kIoExact<IoT>>(D, [&](int i, int r) { return RD[i * LW + r]; },
+    bgemm<C, C, kLocalThreads, kIoExact<IoT>>(D, [&](int i, int r) { return RD[i * LW + r]; },
                               [&](int r, int j) { return RA[j * LW + r]; },
                               [&](int i, int j, float x) { N2[i * LN + j] = j <= i ? x : 0.f; });
     __syncthreads();
@@ -830,7 +917,7 @@ bwd_local_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT
     __syncthreads();
     {
         float rowacc[4] = {0.f, 0.f, 0.f, 0.f};
-        tgemm_rc<C, D, kLocalThreads>(C, [&](int j, int i) { return N1[i * LN + j]; },
+        bgemm_rc<C, D, kLocalThreads>(C, [&](int j, int i) { return N1[i * LN + j]; },
                                   [&](int i, int r) { return RB[i * LW + r]; },
                                   [&](int tr, int, int j, int r, float x) {
                                       if (j < cl) dv[((size_t)(tok0 + j) * H + h) * D + r] = Bs[j] * x;
@@ -840,7 +927,7 @@ bwd_local_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT
     }
     {
         float bacc[4] = {0.f, 0.f, 0.f, 0.f}, gacc[4] = {0.f, 0.f, 0.f, 0.f};
-        tgemm_rc<C, D, kLocalThreads>(C, [&](int j, int i) { return N1[i * LN + j]; },
+        bgemm_rc<C, D, kLocalThreads>(C, [&](int j, int i) { return N1[i * LN + j]; },
                                   [&](int i, int d) { return RC[i * LW + d]; },
                                   [&](int tr, int tc, int j, int d, float x) {
                                       dkacc[tr][tc] += Bs[j] * gam[j] * x;
@@ -851,21 +938,21 @@ bwd_local_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT
         flush_rows(dB, bacc);
         flush_rows(dG, gacc);
     }
-    tgemm<C, C, kLocalThreads, 1, false, false, kIoExact<IoT>>(
+    bgemm<C, C, kLocalThreads, false, kIoExact<IoT>>(
         D, [&](int i, int r) { return RB[i * LW + r]; }, [&](int r, int j) { return RD[j * LW + r]; },
         [&](int i, int j, float x) { N3[i * LN + j] = Bs[j] * x; });
-    tgemm<C, C, kLocalThreads, 1, false, false, kIoExact<IoT>>(
+    bgemm<C, C, kLocalThreads, false, kIoExact<IoT>>(
         D, [&](int i, int d) { return RC[i * LW + d]; }, [&](int d, int j) { return RA[j * LW + d]; },
         [&](int i, int j, float x) { N3[i * LN + j] += Bs[j] * gam[j] * x; });
     __syncthreads();
 
     // ---- phase D: dA = -T^T dT T^T, then the A and P terms ------------------------
     float *Y = RB;   // [64][65]
-    tgemm<C, C, kLocalThreads>(C, [&](int i, int m) { return N3[i * LN + m]; },
+    bgemm<C, C, kLocalThreads>(C, [&](int i, int m) { return N3[i * LN + m]; },
                               [&](int m, int j) { return N1[j * LN + m]; },
                               [&](int i, int j, float x) { Y[i * LN + j] = x; });
     __syncthreads();
-    tgemm<C, C, kLocalThreads>(C, [&](int i, int m) { return N1[m * LN + i]; },
+    bgemm<C, C, kLocalThreads>(C, [&](int i, int m) { return N1[m * LN + i]; },
                               [&](int m, int j) { return Y[m * LN + j]; },
                               [&](int i, int j, float x) { N3[i * LN + j] = j < i ? -x : 0.f; });
     __syncthreads();
@@ -908,13 +995,13 @@ bwd_local_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT
     auto add_dk = [&](int tr, int tc, int, int, float x) { dkacc[tr][tc] += x; };
     constexpr bool kX = kIoExact<IoT>;
     // dk_i += sum_j M_ij k_j and dk_j += sum_i M_ij k_i: one product with M + M^T
-    tgemm_rc<C, D, kLocalThreads, 1, false, false, kX>(
+    bgemm_rc<C, D, kLocalThreads, false, kX>(
         C, [&](int i, int j) { return N3[i * LN + j] + N3[j * LN + i]; },
         [&](int j, int d) { return RA[j * LW + d]; }, add_dk);
-    tgemm_rc<C, D, kLocalThreads, 1, false, false, kX>(C, [&](int i, int j) { return N2[i * LN + j]; },
+    bgemm_rc<C, D, kLocalThreads, false, kX>(C, [&](int i, int j) { return N2[i * LN + j]; },
                                                         [&](int j, int d) { return RA[j * LW + d]; },
                                                         [&](int tr, int tc, int, int, float x) { dqacc[tr][tc] += x; });
-    tgemm_rc<C, D, kLocalThreads, 1, false, false, kX>(C, [&](int j, int i) { return N2[i * LN + j]; },
+    bgemm_rc<C, D, kLocalThreads, false, kX>(C, [&](int j, int i) { return N2[i * LN + j]; },
                                                         [&](int i, int d) { return RB[i * LW + d]; }, add_dk);
     {
         // one sum per element: a store when the chunk's head owns its q/k

@@ -97,3 +97,27 @@ def test_chunked_and_token_forms_agree_with_the_oracle(io):
         torch.cuda.synchronize()
         for x, name in zip(got, ("dq", "dk", "dv", "dg", "dbeta", "dh0")):
             _check(x, ref[name], f"{name} ({nbytes} workspace bytes)")
+
+
+def test_chunked_form_at_the_backward_gdn_shape_on_sampled_heads():
+    """The gradient at the bench's shape (the gdn_prefill inputs, 8192 tokens,
+    16 heads, 128 chunks per chain, dO and dS_final ~ N(0, 1)), run the way
+    the bench runs it; every element of two sampled heads (the first and the
+    last) against the oracle on those heads alone (heads do not interact:
+    H_qk = H, no shared q/k)."""
+    inp = I.workload("gdn_prefill", seed=0)
+    dO, dsf = I.make_grad_inputs(inp, seed=0)
+    assert inp.H == inp.H_qk and inp.h0 is None
+    d = lambda x: None if x is None else x.cuda()
+    ws = torch.empty(gdr.gdr_backward_workspace_size(inp.num_seqs, inp.total_T, inp.H, 128, 128),
+                     dtype=torch.uint8, device="cuda")
+    got = gdr.gdr_backward(d(inp.q), d(inp.k), d(inp.v), d(inp.g), d(inp.beta), None,
+                           d(inp.cu_seqlens), d_o=d(dO), d_final_state=d(dsf), workspace=ws)
+    torch.cuda.synchronize()
+    cu = inp.cu_seqlens.numpy()
+    for head in (0, inp.H - 1):
+        h = slice(head, head + 1)
+        ref = B.backward(inp.q[:, h], inp.k[:, h], inp.v[:, h], inp.g[:, h], inp.beta[:, h], None,
+                         cu, dO[:, h], dsf[:, h])
+        for x, name in zip(got, ("dq", "dk", "dv", "dg", "dbeta", "dh0")):
+            _check(x[:, h], ref[name], f"{name} head {head}")
