@@ -76,21 +76,6 @@ constexpr int kRowBlock = 16;                   // state rows per forward / reve
 constexpr int kLocalThreads = 256;
 constexpr int kLocTM = 4, kLocTN = 8;   // slots of a thread in a <C, D> product over 8 warps
 
-// rows x cols fp32 (cols a multiple of 4, 16-byte aligned) from the record
-// into padded shared rows of `ld` floats: 16-byte loads, eight in flight per
-// thread before their stores.
-template <int NT>
-__device__ __forceinline__ void copy_rows(float *dst, int ld, const float *src, int rows, int cols) {
-    const int q4 = cols / 4, total = rows * q4;
-    const float4 *s4 = reinterpret_cast<const float4 *>(src);
-#pragma unroll 8
-    for (int e = threadIdx.x; e < total; e += NT) {
-        const float4 x = __ldg(s4 + e);
-        float *d = dst + (e / q4) * ld + (e % q4) * 4;
-        d[0] = x.x; d[1] = x.y; d[2] = x.z; d[3] = x.w;
-    }
-}
-
 // The chunk's 64 rows of a [T, heads, 128] input (0 past the sequence's end)
 // into padded shared rows: four values per load (8 bytes of bf16 or 16 of
 // fp32), eight loads in flight per thread.
@@ -548,6 +533,15 @@ __device__ __forceinline__ void stage_c_by_d(float *dst, int ld, const float *sr
     for (int e = threadIdx.x & (kChainThreads - 1); e < C * D / 4; e += kChainThreads)
         cp16(dst + (e >> 5) * ld + (e & 31) * 4, src + e * 4);
 }
+// rows x cols fp32 (cols a multiple of 4) from the record into rows of ld
+// floats (16-byte aligned), by 16-byte asynchronous copies over NT threads.
+template <int NT>
+__device__ __forceinline__ void copy_rows_async(float *dst, int ld, const float *src, int rows, int cols) {
+    const int q4 = cols / 4, total = rows * q4;
+    for (int e = threadIdx.x & (NT - 1); e < total; e += NT)
+        cp16(dst + (e / q4) * ld + (e % q4) * 4, src + e * 4);
+}
+
 // Columns r0 .. r0 + 15 of a 64 x 128 record field into rows of 16 floats.
 __device__ __forceinline__ void stage_strip(float *dst, const float *src, int r0) {
     const int e = threadIdx.x & (kChainThreads - 1);
@@ -842,9 +836,13 @@ bwd_local_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT
     }
 
     // ---- phase A: dK^ = U L' and <S, L'> --------------------------------------
-    copy_rows<kLocalThreads>(RA, LW, rec + R_L, D, D);
-    copy_rows<kLocalThreads>(RB, LW, rec + R_U, C, D);
-    copy_rows<kLocalThreads>(RC, LW, rec + R_KH, C, D);
+    copy_rows_async<kLocalThreads>(RA, LW, rec + R_L, D, D);
+    copy_rows_async<kLocalThreads>(RB, LW, rec + R_U, C, D);
+    copy_rows_async<kLocalThreads>(RC, LW, rec + R_KH, C, D);
+    float *Sd = RD;   // S, dense 128 x 128, in the buffers phase A leaves free (RD .. N3)
+    static_assert(LB_G - LB_RD >= D * D, "room for S");
+    copy_rows_async<kLocalThreads>(Sd, D, rec + R_S, D, D);
+    cp_commit();
     if (tid < C) {
         Gs[tid] = rec[R_G + tid];
         gam[tid] = __expf(rec[R_G + tid]);
@@ -853,14 +851,14 @@ bwd_local_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT
         dB[tid] = 0.f;
     }
     if (tid < 8) misc[tid] = 0.f;
+    cp_wait<0>();
     __syncthreads();
     const float GC = Gs[C - 1], gC = __expf(GC);
     {
-        float part = 0.f;   // <S, L'> over this thread's entries, 16-byte loads
-        const float4 *s4 = reinterpret_cast<const float4 *>(rec + R_S);
+        float part = 0.f;   // <S, L'> over this thread's entries
 #pragma unroll 8
         for (int e = tid; e < D * D / 4; e += kLocalThreads) {
-            const float4 x = __ldg(s4 + e);
+            const float4 x = *reinterpret_cast<const float4 *>(Sd + e * 4);
             const float4 y = *reinterpret_cast<const float4 *>(RA + (e >> 5) * LW + (e & 31) * 4);
             part = fmaf(x.x, y.x, fmaf(x.y, y.y, fmaf(x.z, y.z, fmaf(x.w, y.w, part))));
         }
@@ -885,9 +883,11 @@ bwd_local_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT
     __syncthreads();
 
     // ---- phase B: dW = -dU S, d(gamma Q) = dO S ---------------------------------
-    copy_rows<kLocalThreads>(RA, LW, rec + R_S, D, D);
-    copy_rows<kLocalThreads>(RB, LW, rec + R_DU, C, D);
+    copy_rows_async<kLocalThreads>(RA, LW, rec + R_S, D, D);
+    copy_rows_async<kLocalThreads>(RB, LW, rec + R_DU, C, D);
+    cp_commit();
     load_io_rows<kLocalThreads>(RD, dO, tok0, cl, H, h);
+    cp_wait<0>();
     __syncthreads();
     bgemm<C, D, kLocalThreads>(D, [&](int j, int r) { return RB[j * LW + r]; },
                               [&](int r, int d) { return RA[r * LW + d]; },
@@ -905,8 +905,10 @@ bwd_local_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT
     __syncthreads();
 
     // ---- phase C: dP, T^T dU, T^T dW, dT ---------------------------------------
-    copy_rows<kLocalThreads>(RA, LW, rec + R_U, C, D);
-    copy_rows<kLocalThreads>(N1, LN, rec + R_T, C, C);
+    copy_rows_async<kLocalThreads>(RA, LW, rec + R_U, C, D);
+    copy_rows_async<kLocalThreads>(N1, LN, rec + R_T, C, C);
+    cp_commit();
+    cp_wait<0>();
     __syncthreads();
     bgemm<C, C, kLocalThreads, kIoExact<IoT>>(D, [&](int i, int r) { return RD[i * LW + r]; },
                               [&](int r, int j) { return RA[j * LW + r]; },
@@ -957,38 +959,45 @@ bwd_local_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT
                               [&](int i, int j, float x) { N3[i * LN + j] = j < i ? -x : 0.f; });
     __syncthreads();
     float *AR = RC;   // [64][65]
-    copy_rows<kLocalThreads>(AR, LN, rec + R_AR, C, C);
-    copy_rows<kLocalThreads>(N1, LN, rec + R_P, C, C);
+    copy_rows_async<kLocalThreads>(AR, LN, rec + R_AR, C, C);
+    copy_rows_async<kLocalThreads>(N1, LN, rec + R_P, C, C);
+    cp_commit();
+    cp_wait<0>();
     __syncthreads();
     {
-        // a warp takes half a row i per step: the row sums of dA o A (for
-        // dbeta_i) and of dA o A + dP o P (for dG_i) are reduced over the
-        // warp; a thread's column j = tid % 64 is the same at every step, so
-        // its sum for dG_j stays in a register
-        const int j = tid & (C - 1);
-        float colacc = 0.f;
-#pragma unroll 4
+        // dA o A + dP o P over AR (each element read, then written, by one
+        // thread) and dA o A / beta_i over the finished Y; then their row
+        // sums (dG_i, dbeta_i) and column sums (dG_j), each by one thread
+        float *Es = AR, *Bq = RB;
         for (int e = tid; e < C * C; e += kLocalThreads) {
-            const int i = e >> 6;
+            const int i = e >> 6, j = e & 63;
             const float R = j <= i ? __expf(Gs[i] - Gs[j]) : 0.f;
             const float da = N3[i * LN + j], ar = AR[i * LN + j];
-            const float ea = da * Bs[i] * ar;                           // dA o A
             const float dp = N2[i * LN + j], ep = dp * N1[j * LN + i];   // dP o P (N1 holds P^T)
-            float rb = da * ar, rg = ea + ep;
-            colacc -= rg;
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) {
-                rb += __shfl_xor_sync(0xffffffffu, rb, off);
-                rg += __shfl_xor_sync(0xffffffffu, rg, off);
-            }
-            if ((tid & 31) == 0) {
-                atomicAdd(&dB[i], rb);
-                atomicAdd(&dG[i], rg);
-            }
+            Es[i * LN + j] = da * Bs[i] * ar + ep;
+            Bq[i * LN + j] = da * ar;
             N3[i * LN + j] = da * Bs[i] * R;             // M = dA o beta_i R
             N2[i * LN + j] = dp * R;                     // dP o R
         }
-        atomicAdd(&dG[j], colacc);
+        __syncthreads();
+        if (tid < C) {   // row tid, columns in a staggered order (no bank conflicts)
+            float se = 0.f, sb = 0.f;
+#pragma unroll 8
+            for (int s_ = 0; s_ < C; ++s_) {
+                const int j = (s_ + tid) & (C - 1);
+                se += Es[tid * LN + j];
+                sb += Bq[tid * LN + j];
+            }
+            atomicAdd(&dG[tid], se);
+            atomicAdd(&dB[tid], sb);
+        } else if (tid < 2 * C) {   // column tid - C
+            const int j = tid - C;
+            float se = 0.f;
+#pragma unroll 8
+            for (int i = 0; i < C; ++i) se += Es[i * LN + j];
+            atomicAdd(&dG[j], -se);
+        }
+        __syncthreads();
     }
     load_io_rows<kLocalThreads>(RB, q, tok0, cl, Hqk, hq);   // Q rows over the finished Y
     __syncthreads();
