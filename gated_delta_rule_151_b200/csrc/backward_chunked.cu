@@ -259,8 +259,11 @@ __device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], 
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
-// tgemm_rc's contract with bf16 products; K a multiple of 16.
-template <int M, int N, int NTH, bool AEX = false, bool BEX = false, class AF, class BF, class EPI>
+// tgemm_rc's contract with bf16 products; K a multiple of 16.  With PAIRS
+// the results go out two at a time, epi(m, n, value(m, n), value(m, n + 1))
+// with n even, so that a store can take both.
+template <int M, int N, int NTH, bool AEX = false, bool BEX = false, bool PAIRS = false, class AF,
+          class BF, class EPI>
 __device__ __forceinline__ void bgemm_rc(int K, AF a, BF b, EPI epi) {
     using G = WarpGrid<M, N, NTH / 32>;
     const int t = threadIdx.x & (NTH - 1), lane = t & 31, warp = t >> 5;
@@ -307,16 +310,32 @@ __device__ __forceinline__ void bgemm_rc(int K, AF a, BF b, EPI epi) {
 #pragma unroll
     for (int mt = 0; mt < G::MT; ++mt)
 #pragma unroll
-        for (int nt = 0; nt < G::NT; ++nt)
+        for (int nt = 0; nt < G::NT; ++nt) {
+            if constexpr (PAIRS) {
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-                epi(mt * 2 + (e >> 1), nt * 2 + (e & 1), m0 + mt * 16 + gid + 8 * (e >> 1),
-                    n0 + nt * 8 + 2 * tig + (e & 1), acc[mt][nt][e]);
+                for (int h = 0; h < 2; ++h)
+                    epi(m0 + mt * 16 + gid + 8 * h, n0 + nt * 8 + 2 * tig, acc[mt][nt][2 * h],
+                        acc[mt][nt][2 * h + 1]);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    epi(mt * 2 + (e >> 1), nt * 2 + (e & 1), m0 + mt * 16 + gid + 8 * (e >> 1),
+                        n0 + nt * 8 + 2 * tig + (e & 1), acc[mt][nt][e]);
+            }
+        }
 }
 
 template <int M, int N, int NTH, bool AEX = false, bool BEX = false, class AF, class BF, class EPI>
 __device__ __forceinline__ void bgemm(int K, AF a, BF b, EPI epi) {
     bgemm_rc<M, N, NTH, AEX, BEX>(K, a, b, [&](int, int, int m, int n, float v) { epi(m, n, v); });
+}
+
+// bgemm storing out(m, n) row-major with ld floats: two results per 8-byte store.
+template <int M, int N, int NTH, bool AEX = false, bool BEX = false, class AF, class BF>
+__device__ __forceinline__ void bgemm_store(int K, AF a, BF b, float *out, int ld) {
+    bgemm_rc<M, N, NTH, AEX, BEX, true>(K, a, b, [&](int m, int n, float x0, float x1) {
+        *reinterpret_cast<float2 *>(out + (size_t)m * ld + n) = make_float2(x0, x1);
+    });
 }
 
 // Row of slot r and column of slot c of the calling thread in a <M, N, NTH>
@@ -426,6 +445,18 @@ bwd_prep_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT 
     float *Ks = fs + PB_K, *Qs = fs + PB_Q, *Vs = fs + PB_V, *Tp = fs + PB_TP, *DOs = fs + PB_DO,
           *Ps = fs + PB_P;
     float *Gs = fs + PB_G, *gam = Gs + C, *Bs = gam + C;
+    {   // the chunk's rows of k, q, v and dO towards L2, one row per thread,
+        // so that the loads below after the first find them there
+        const int w = tid / C, i = tid % C;
+        if (i < cl) {
+            const IoT *src = w == 0 ? k + ((size_t)(tok0 + i) * Hqk + hq) * D
+                           : w == 1 ? q + ((size_t)(tok0 + i) * Hqk + hq) * D
+                           : w == 2 ? v + ((size_t)(tok0 + i) * H + h) * D
+                                    : dO + ((size_t)(tok0 + i) * H + h) * D;
+            tc::bulk_prefetch_l2(src, D * sizeof(IoT));
+        }
+    }
+    static_assert(kPrepB == 4 * C, "one input row per thread");
     load_io_rows<kPrepB>(Ks, k, tok0, cl, Hqk, hq);
     load_io_rows<kPrepB>(Qs, q, tok0, cl, Hqk, hq);
     load_io_rows<kPrepB>(Vs, v, tok0, cl, H, h);
@@ -487,20 +518,16 @@ bwd_prep_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT 
     __syncthreads();
     // W = T diag(beta gamma) K and U~ = T diag(beta) V, the scales taken
     // with T so that K and V stay exact operands
-    bgemm<C, D, kPrepB, false, kX>(C, [&](int i, int j) { return Tp[i * LN + j] * Bs[j] * gam[j]; },
-                       [&](int j, int d) { return Ks[j * LW + d]; },
-                       [&](int i, int d, float x) { rec[R_W + i * D + d] = x; });
-    bgemm<C, D, kPrepB, false, kX>(C, [&](int i, int j) { return Tp[i * LN + j] * Bs[j]; },
-                       [&](int j, int d) { return Vs[j * LW + d]; },
-                       [&](int i, int d, float x) { rec[R_UT + i * D + d] = x; });
+    bgemm_store<C, D, kPrepB, false, kX>(C, [&](int i, int j) { return Tp[i * LN + j] * Bs[j] * gam[j]; },
+                                          [&](int j, int d) { return Ks[j * LW + d]; }, rec + R_W, D);
+    bgemm_store<C, D, kPrepB, false, kX>(C, [&](int i, int j) { return Tp[i * LN + j] * Bs[j]; },
+                                          [&](int j, int d) { return Vs[j * LW + d]; }, rec + R_UT, D);
     // the upstream gradient's terms of the adjoint chain, which depend on the
     // chunk alone: Y = dO^T diag(gamma) Q and Z = P^T dO
-    bgemm<D, D, kPrepB, kX>(C, [&](int r, int i) { return DOs[i * LW + r]; },
-                                      [&](int i, int d) { return Qs[i * LW + d] * gam[i]; },
-                                      [&](int r, int d, float x) { rec[R_Y + r * D + d] = x; });
-    bgemm<C, D, kPrepB, false, kX>(C, [&](int j, int i) { return Ps[i * LN + j]; },
-                                             [&](int i, int r) { return DOs[i * LW + r]; },
-                                             [&](int j, int r, float x) { rec[R_Z + j * D + r] = x; });
+    bgemm_store<D, D, kPrepB, kX>(C, [&](int r, int i) { return DOs[i * LW + r]; },
+                                   [&](int i, int d) { return Qs[i * LW + d] * gam[i]; }, rec + R_Y, D);
+    bgemm_store<C, D, kPrepB, false, kX>(C, [&](int j, int i) { return Ps[i * LN + j]; },
+                                          [&](int i, int r) { return DOs[i * LW + r]; }, rec + R_Z, D);
 }
 
 // ------------------------------------------------------ forward / reverse ----
@@ -820,17 +847,20 @@ bwd_local_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT
     };
     // everything the later phases read towards L2 while phase A runs: the
     // record's P, T, (K K^T) o R, G, beta and U .. gamma Q (64 KiB pieces),
-    // and the chunk's rows of q, k and v
+    // and the chunk's rows of q, k, v and dO
     if (tid == 0) {
         tc::bulk_prefetch_l2(rec + R_P, (3 * C * C + 2 * C) * sizeof(float));
         for (size_t o = R_U; o < R_Y; o += 16384)
             tc::bulk_prefetch_l2(rec + o, (uint32_t)(min((size_t)16384, R_Y - o) * sizeof(float)));
-    } else if (tid >= 64 && tid < 64 + 3 * C) {
-        const int w = (tid - 64) / C, i = (tid - 64) % C;
+    }
+    static_assert(kLocalThreads == 4 * C, "one input row per thread");
+    {
+        const int w = tid / C, i = tid % C;   // one row of q, k, v or dO per thread
         if (i < cl) {
             const IoT *src = w == 0 ? q + ((size_t)(tok0 + i) * Hqk + hq) * D
                            : w == 1 ? k + ((size_t)(tok0 + i) * Hqk + hq) * D
-                                    : v + ((size_t)(tok0 + i) * H + h) * D;
+                           : w == 2 ? v + ((size_t)(tok0 + i) * H + h) * D
+                                    : dO + ((size_t)(tok0 + i) * H + h) * D;
             tc::bulk_prefetch_l2(src, D * sizeof(IoT));
         }
     }
