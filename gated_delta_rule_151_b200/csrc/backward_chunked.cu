@@ -259,29 +259,35 @@ __device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], 
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
-// tgemm_rc's contract with bf16 products; K a multiple of 16.  With PAIRS
-// the results go out two at a time, epi(m, n, value(m, n), value(m, n + 1))
-// with n even, so that a store can take both.
-template <int M, int N, int NTH, bool AEX = false, bool BEX = false, bool PAIRS = false, class AF,
-          class BF, class EPI>
+// tgemm_rc's contract with bf16 products; K a multiple of 16 KPAR.  With
+// PAIRS the results go out two at a time, epi(m, n, value(m, n),
+// value(m, n + 1)) with n even, so that a store can take both.  KPAR and
+// PSPLIT as for tgemm_rc (independent accumulator sets for warps with few
+// tiles).
+template <int M, int N, int NTH, bool AEX = false, bool BEX = false, bool PAIRS = false,
+          int KPAR = 1, bool PSPLIT = false, class AF, class BF, class EPI>
 __device__ __forceinline__ void bgemm_rc(int K, AF a, BF b, EPI epi) {
     using G = WarpGrid<M, N, NTH / 32>;
+    constexpr int NP = PSPLIT ? 3 : 1;
     const int t = threadIdx.x & (NTH - 1), lane = t & 31, warp = t >> 5;
     const int gid = lane >> 2, tig = lane & 3;
     const int m0 = (warp / G::GN) * G::WM, n0 = (warp % G::GN) * G::WN;
-    float acc[G::MT][G::NT][4];
+    float acc[KPAR][NP][G::MT][G::NT][4];
 #pragma unroll
-    for (int mt = 0; mt < G::MT; ++mt)
+    for (int s = 0; s < KPAR; ++s)
 #pragma unroll
-        for (int nt = 0; nt < G::NT; ++nt)
+        for (int p = 0; p < NP; ++p)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) acc[mt][nt][e] = 0.f;
+            for (int mt = 0; mt < G::MT; ++mt)
+#pragma unroll
+                for (int nt = 0; nt < G::NT; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) acc[s][p][mt][nt][e] = 0.f;
     auto take = [](float x0, float x1, uint32_t &hi, uint32_t &lo, bool exact) {
         if (exact) hi = pack_bf16(x0, x1);
         else split_bf16x2(x0, x1, hi, lo);
     };
-#pragma unroll 2
-    for (int k0 = 0; k0 < K; k0 += 16) {
+    auto kstep = [&](int k0, float (&ac)[NP][G::MT][G::NT][4]) {
         uint32_t ah[G::MT][4], al[G::MT][4], bh[G::NT][2], bl[G::NT][2];
         const int ka = k0 + 2 * tig;
 #pragma unroll
@@ -302,11 +308,28 @@ __device__ __forceinline__ void bgemm_rc(int K, AF a, BF b, EPI epi) {
         for (int mt = 0; mt < G::MT; ++mt)
 #pragma unroll
             for (int nt = 0; nt < G::NT; ++nt) {
-                if (!AEX) mma_bf16(acc[mt][nt], al[mt], bh[nt]);
-                if (!BEX) mma_bf16(acc[mt][nt], ah[mt], bl[nt]);
-                mma_bf16(acc[mt][nt], ah[mt], bh[nt]);
+                if (!AEX) mma_bf16(ac[NP - 1][mt][nt], al[mt], bh[nt]);
+                if (!BEX) mma_bf16(ac[NP > 1 ? 1 : 0][mt][nt], ah[mt], bl[nt]);
+                mma_bf16(ac[0][mt][nt], ah[mt], bh[nt]);
             }
+    };
+#pragma unroll 2
+    for (int k0 = 0; k0 < K; k0 += 16 * KPAR) {
+        kstep(k0, acc[0]);
+        if (KPAR > 1) kstep(k0 + 16, acc[KPAR - 1]);
     }
+    auto total = [&](int mt, int nt, int e) {
+        float x = acc[0][0][mt][nt][e], corr = 0.f;
+#pragma unroll
+        for (int s = 0; s < KPAR; ++s)
+#pragma unroll
+            for (int p = 0; p < NP; ++p)
+                if (s + p > 0) {
+                    if (p > 0) corr += acc[s][p][mt][nt][e];
+                    else x += acc[s][p][mt][nt][e];
+                }
+        return x + corr;
+    };
 #pragma unroll
     for (int mt = 0; mt < G::MT; ++mt)
 #pragma unroll
@@ -314,13 +337,13 @@ __device__ __forceinline__ void bgemm_rc(int K, AF a, BF b, EPI epi) {
             if constexpr (PAIRS) {
 #pragma unroll
                 for (int h = 0; h < 2; ++h)
-                    epi(m0 + mt * 16 + gid + 8 * h, n0 + nt * 8 + 2 * tig, acc[mt][nt][2 * h],
-                        acc[mt][nt][2 * h + 1]);
+                    epi(m0 + mt * 16 + gid + 8 * h, n0 + nt * 8 + 2 * tig, total(mt, nt, 2 * h),
+                        total(mt, nt, 2 * h + 1));
             } else {
 #pragma unroll
                 for (int e = 0; e < 4; ++e)
                     epi(mt * 2 + (e >> 1), nt * 2 + (e & 1), m0 + mt * 16 + gid + 8 * (e >> 1),
-                        n0 + nt * 8 + 2 * tig + (e & 1), acc[mt][nt][e]);
+                        n0 + nt * 8 + 2 * tig + (e & 1), total(mt, nt, e));
             }
         }
 }
@@ -636,13 +659,14 @@ __device__ __forceinline__ void forward_chain(float *fs, const float *__restrict
         }
         store_rows(rec + R_S, Sr, r0);
         // U[j][r0 + r] = U~[j][r0 + r] - sum_d W[j][d] S[r][d]
-        bgemm<C, kRowBlock, kChainThreads>(D, [&](int j, int d) { return Ws[j * LW4 + d]; },
-                                           [&](int d, int r) { return Sr[r * LW4 + d]; },
-                                           [&](int j, int r, float x) {
-                                               const float u = Us[j * kRowBlock + r] - x;
-                                               Ut[r * LN4 + j] = u;
-                                               rec[R_U + j * D + r0 + r] = u;
-                                           });
+        bgemm_rc<C, kRowBlock, kChainThreads, false, false, true, 2, true>(
+            D, [&](int j, int d) { return Ws[j * LW4 + d]; }, [&](int d, int r) { return Sr[r * LW4 + d]; },
+            [&](int j, int r, float x0, float x1) {
+                const float u0 = Us[j * kRowBlock + r] - x0, u1 = Us[j * kRowBlock + r + 1] - x1;
+                Ut[r * LN4 + j] = u0;
+                Ut[(r + 1) * LN4 + j] = u1;
+                *reinterpret_cast<float2 *>(rec + R_U + j * D + r0 + r) = make_float2(u0, u1);
+            });
         group_sync(1);   // W and U~ consumed, U^T complete
         if (c + 1 < nch) {
             stage_c_by_d(Ws, LW4, rec_of(c + 1) + R_W);
@@ -653,10 +677,12 @@ __device__ __forceinline__ void forward_chain(float *fs, const float *__restrict
         group_sync(1);   // K^ and G of chunk c in place
         {   // S[r][d] = e^{G_C} S[r][d] + sum_j U[j][r] K^[j][d]
             const float gC = __expf(Gs[C - 1]);
-            bgemm<kRowBlock, D, kChainThreads>(C, [&](int r, int j) { return Ut[r * LN4 + j]; },
+            bgemm_rc<kRowBlock, D, kChainThreads, false, false, true, 2, true>(C, [&](int r, int j) { return Ut[r * LN4 + j]; },
                                                [&](int j, int d) { return Kh[j * LW8 + d]; },
-                                               [&](int r, int d, float x) {
-                                                   Sr[r * LW4 + d] = fmaf(gC, Sr[r * LW4 + d], x);
+                                               [&](int r, int d, float x0, float x1) {
+                                                   float2 *p = reinterpret_cast<float2 *>(Sr + r * LW4 + d);
+                                                   const float2 s = *p;
+                                                   *p = make_float2(fmaf(gC, s.x, x0), fmaf(gC, s.y, x1));
                                                });
         }
         group_sync(1);   // K^ and G consumed
@@ -729,13 +755,14 @@ __device__ __forceinline__ void reverse_chain(float *fs, const float *__restrict
         }
         store_rows(rec + R_L, Lr, r0);
         // dU[j][r0 + r] = Z[j][r0 + r] + sum_d K^[j][d] L[r][d]
-        bgemm<C, kRowBlock, kChainThreads>(D, [&](int j, int d) { return Kh[j * LW4 + d]; },
-                                                    [&](int d, int r) { return Lr[r * LW4 + d]; },
-                                                    [&](int j, int r, float x) {
-                                                        const float v = Zs[j * kRowBlock + r] + x;
-                                                        dUt[r * LN4 + j] = v;
-                                                        rec[R_DU + j * D + r0 + r] = v;
-                                                    });
+        bgemm_rc<C, kRowBlock, kChainThreads, false, false, true, 2, true>(
+            D, [&](int j, int d) { return Kh[j * LW4 + d]; }, [&](int d, int r) { return Lr[r * LW4 + d]; },
+            [&](int j, int r, float x0, float x1) {
+                const float v0 = Zs[j * kRowBlock + r] + x0, v1 = Zs[j * kRowBlock + r + 1] + x1;
+                dUt[r * LN4 + j] = v0;
+                dUt[(r + 1) * LN4 + j] = v1;
+                *reinterpret_cast<float2 *>(rec + R_DU + j * D + r0 + r) = make_float2(v0, v1);
+            });
         group_sync(2);   // K^ and Z consumed, dU^T complete
         if (c > 0) {
             stage_c_by_d(Kh, LW4, rec_of(c - 1) + R_KH);
@@ -746,11 +773,13 @@ __device__ __forceinline__ void reverse_chain(float *fs, const float *__restrict
         group_sync(2);   // W, Y and G of chunk c in place
         {   // L[r][d] = e^{G_C} L[r][d] + Y[r0 + r][d] - sum_j dU[j][r] W[j][d]
             const float gC = __expf(Gs[C - 1]);
-            bgemm<kRowBlock, D, kChainThreads>(C, [&](int r, int j) { return dUt[r * LN4 + j]; },
-                                                        [&](int j, int d) { return Ws[j * LW8 + d]; },
-                                                        [&](int r, int d, float x) {
-                                                            Lr[r * LW4 + d] = fmaf(gC, Lr[r * LW4 + d], Ys[r * LW4 + d] - x);
-                                                        });
+            bgemm_rc<kRowBlock, D, kChainThreads, false, false, true, 2, true>(
+                C, [&](int r, int j) { return dUt[r * LN4 + j]; }, [&](int j, int d) { return Ws[j * LW8 + d]; },
+                [&](int r, int d, float x0, float x1) {
+                    float2 *p = reinterpret_cast<float2 *>(Lr + r * LW4 + d);
+                    const float2 l = *p, y = *reinterpret_cast<const float2 *>(Ys + r * LW4 + d);
+                    *p = make_float2(fmaf(gC, l.x, y.x - x0), fmaf(gC, l.y, y.y - x1));
+                });
         }
         group_sync(2);   // W, Y and G consumed
         if (c > 0) {
