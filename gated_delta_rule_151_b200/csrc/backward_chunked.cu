@@ -434,6 +434,74 @@ __device__ __forceinline__ bool chunk_of(const int32_t *base, int num_seqs, int 
     return true;
 }
 
+__device__ __forceinline__ void cp16(void *dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(tc::smem_u32(dst)), "l"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N> __device__ __forceinline__ void cp_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// The chunk's 64 rows of a [T, heads, 128] input (0 past the sequence's end)
+// into padded fp32 rows by 16-byte asynchronous copies: fp32 rows straight
+// into place; bf16 rows into the second half of the destination (rows
+// 32 .. 63 of it are not yet written), converted by finish_io_rows.
+template <int NT, typename IoT>
+__device__ __forceinline__ void stage_io_rows(float *dst, const IoT *src, int tok0, int cl, int heads,
+                                              int head) {
+    const int t = threadIdx.x & (NT - 1);
+    if constexpr (std::is_same<IoT, float>::value) {
+        for (int e = t; e < C * D / 4; e += NT) {
+            const int i = e >> 5, q = e & 31;
+            float *o = dst + i * LW + 4 * q;
+            if (i < cl) cp16(o, src + ((size_t)(tok0 + i) * heads + head) * D + 4 * q);
+            else *reinterpret_cast<float4 *>(o) = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    } else {
+        char *raw = reinterpret_cast<char *>(dst + C * LW / 2);
+        for (int e = t; e < C * D / 8; e += NT) {
+            const int i = e >> 4, q = e & 15;
+            if (i < cl) cp16(raw + i * 256 + q * 16, src + ((size_t)(tok0 + i) * heads + head) * D + 8 * q);
+        }
+    }
+}
+// The bf16 rows staged in four destinations, converted in place: every
+// thread reads its raw pieces, the block synchronises, then writes the fp32
+// rows.  Called by every thread after the copies are waited for and
+// synchronised; ends synchronised.
+template <int NT, typename IoT>
+__device__ __forceinline__ void finish_io_rows(float *d0, float *d1, float *d2, float *d3, int cl) {
+    if constexpr (!std::is_same<IoT, float>::value) {
+        constexpr int PER = C * D / 8 / NT;
+        float *dst[4] = {d0, d1, d2, d3};
+        uint4 raw[4][PER];
+        const int t = threadIdx.x & (NT - 1);
+#pragma unroll
+        for (int w = 0; w < 4; ++w)
+#pragma unroll
+            for (int p = 0; p < PER; ++p) {
+                const int e = t + p * NT, i = e >> 4, q = e & 15;
+                raw[w][p] = i < cl ? *reinterpret_cast<const uint4 *>(
+                                         reinterpret_cast<const char *>(dst[w] + C * LW / 2) + i * 256 + q * 16)
+                                   : make_uint4(0u, 0u, 0u, 0u);
+            }
+        __syncthreads();
+#pragma unroll
+        for (int w = 0; w < 4; ++w)
+#pragma unroll
+            for (int p = 0; p < PER; ++p) {
+                const int e = t + p * NT, i = e >> 4, q = e & 15;
+                float f[8];
+                bf16x8_to_f32(raw[w][p], f);
+                float4 *o = reinterpret_cast<float4 *>(dst[w] + i * LW + 8 * q);
+                o[0] = make_float4(f[0], f[1], f[2], f[3]);
+                o[1] = make_float4(f[4], f[5], f[6], f[7]);
+            }
+    }
+    __syncthreads();
+}
+
 // ---------------------------------------------------------------- prep ----
 // One CTA per (global chunk, value head): G, beta, A (via the strictly
 // lower (K K^T) o R), T = (I + A)^-1, W, U~ and P, written to the record.
@@ -468,22 +536,12 @@ bwd_prep_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT 
     float *Ks = fs + PB_K, *Qs = fs + PB_Q, *Vs = fs + PB_V, *Tp = fs + PB_TP, *DOs = fs + PB_DO,
           *Ps = fs + PB_P;
     float *Gs = fs + PB_G, *gam = Gs + C, *Bs = gam + C;
-    {   // the chunk's rows of k, q, v and dO towards L2, one row per thread,
-        // so that the loads below after the first find them there
-        const int w = tid / C, i = tid % C;
-        if (i < cl) {
-            const IoT *src = w == 0 ? k + ((size_t)(tok0 + i) * Hqk + hq) * D
-                           : w == 1 ? q + ((size_t)(tok0 + i) * Hqk + hq) * D
-                           : w == 2 ? v + ((size_t)(tok0 + i) * H + h) * D
-                                    : dO + ((size_t)(tok0 + i) * H + h) * D;
-            tc::bulk_prefetch_l2(src, D * sizeof(IoT));
-        }
-    }
-    static_assert(kPrepB == 4 * C, "one input row per thread");
-    load_io_rows<kPrepB>(Ks, k, tok0, cl, Hqk, hq);
-    load_io_rows<kPrepB>(Qs, q, tok0, cl, Hqk, hq);
-    load_io_rows<kPrepB>(Vs, v, tok0, cl, H, h);
-    load_io_rows<kPrepB>(DOs, dO, tok0, cl, H, h);
+    // the chunk's rows of k, q, v and dO, every copy in flight at once
+    stage_io_rows<kPrepB>(Ks, k, tok0, cl, Hqk, hq);
+    stage_io_rows<kPrepB>(Qs, q, tok0, cl, Hqk, hq);
+    stage_io_rows<kPrepB>(Vs, v, tok0, cl, H, h);
+    stage_io_rows<kPrepB>(DOs, dO, tok0, cl, H, h);
+    cp_commit();
     if (tid < 32) {   // gates of tokens 2 tid, 2 tid + 1: clamped, cumulated, 0 past the end
         const int i0 = 2 * tid, i1 = i0 + 1;
         const float g0 = i0 < cl ? clamp_log_gate(g[(size_t)(tok0 + i0) * H + h]) : 0.f;
@@ -501,7 +559,9 @@ bwd_prep_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT 
         Bs[i0] = i0 < cl ? beta[(size_t)(tok0 + i0) * H + h] : 0.f;
         Bs[i1] = i1 < cl ? beta[(size_t)(tok0 + i1) * H + h] : 0.f;
     }
+    cp_wait<0>();
     __syncthreads();
+    finish_io_rows<kPrepB, IoT>(Ks, Qs, Vs, DOs, cl);   // ends synchronised
     // (K K^T) o R (strictly lower) -> record and A = diag(beta) of it; P -> record
     float *Af = fs + PB_A;
     constexpr bool kX = kIoExact<IoT>;
@@ -567,15 +627,6 @@ constexpr int LW4 = D + 4;   // rows read as the A operand or along K
 constexpr int LW8 = D + 8;   // rows read as a K x N B operand
 constexpr int LN4 = C + 4;
 static_assert(kChainThreads == C * 4, "one 16-byte piece of a column strip per thread");
-
-__device__ __forceinline__ void cp16(void *dst, const void *src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(tc::smem_u32(dst)), "l"(src)
-                 : "memory");
-}
-__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N> __device__ __forceinline__ void cp_wait() {
-    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
 
 // 64 x 128 floats of a record field into rows of ld floats.
 __device__ __forceinline__ void stage_c_by_d(float *dst, int ld, const float *src) {
