@@ -260,8 +260,9 @@ __device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], 
 }
 
 // tgemm_rc's contract with bf16 products; K a multiple of 16 KPAR.  With
-// PAIRS the results go out two at a time, epi(m, n, value(m, n),
-// value(m, n + 1)) with n even, so that a store can take both.  KPAR and
+// PAIRS the results go out two at a time, epi(r, m, n, value(m, n),
+// value(m, n + 1)) with n even and r the row's slot, so that a store can
+// take both.  KPAR and
 // PSPLIT as for tgemm_rc (independent accumulator sets for warps with few
 // tiles).
 template <int M, int N, int NTH, bool AEX = false, bool BEX = false, bool PAIRS = false,
@@ -337,8 +338,8 @@ __device__ __forceinline__ void bgemm_rc(int K, AF a, BF b, EPI epi) {
             if constexpr (PAIRS) {
 #pragma unroll
                 for (int h = 0; h < 2; ++h)
-                    epi(m0 + mt * 16 + gid + 8 * h, n0 + nt * 8 + 2 * tig, total(mt, nt, 2 * h),
-                        total(mt, nt, 2 * h + 1));
+                    epi(mt * 2 + h, m0 + mt * 16 + gid + 8 * h, n0 + nt * 8 + 2 * tig,
+                        total(mt, nt, 2 * h), total(mt, nt, 2 * h + 1));
             } else {
 #pragma unroll
                 for (int e = 0; e < 4; ++e)
@@ -356,7 +357,7 @@ __device__ __forceinline__ void bgemm(int K, AF a, BF b, EPI epi) {
 // bgemm storing out(m, n) row-major with ld floats: two results per 8-byte store.
 template <int M, int N, int NTH, bool AEX = false, bool BEX = false, class AF, class BF>
 __device__ __forceinline__ void bgemm_store(int K, AF a, BF b, float *out, int ld) {
-    bgemm_rc<M, N, NTH, AEX, BEX, true>(K, a, b, [&](int m, int n, float x0, float x1) {
+    bgemm_rc<M, N, NTH, AEX, BEX, true>(K, a, b, [&](int, int m, int n, float x0, float x1) {
         *reinterpret_cast<float2 *>(out + (size_t)m * ld + n) = make_float2(x0, x1);
     });
 }
@@ -712,7 +713,7 @@ __device__ __forceinline__ void forward_chain(float *fs, const float *__restrict
         // U[j][r0 + r] = U~[j][r0 + r] - sum_d W[j][d] S[r][d]
         bgemm_rc<C, kRowBlock, kChainThreads, false, false, true, 2, true>(
             D, [&](int j, int d) { return Ws[j * LW4 + d]; }, [&](int d, int r) { return Sr[r * LW4 + d]; },
-            [&](int j, int r, float x0, float x1) {
+            [&](int, int j, int r, float x0, float x1) {
                 const float u0 = Us[j * kRowBlock + r] - x0, u1 = Us[j * kRowBlock + r + 1] - x1;
                 Ut[r * LN4 + j] = u0;
                 Ut[(r + 1) * LN4 + j] = u1;
@@ -730,7 +731,7 @@ __device__ __forceinline__ void forward_chain(float *fs, const float *__restrict
             const float gC = __expf(Gs[C - 1]);
             bgemm_rc<kRowBlock, D, kChainThreads, false, false, true, 2, true>(C, [&](int r, int j) { return Ut[r * LN4 + j]; },
                                                [&](int j, int d) { return Kh[j * LW8 + d]; },
-                                               [&](int r, int d, float x0, float x1) {
+                                               [&](int, int r, int d, float x0, float x1) {
                                                    float2 *p = reinterpret_cast<float2 *>(Sr + r * LW4 + d);
                                                    const float2 s = *p;
                                                    *p = make_float2(fmaf(gC, s.x, x0), fmaf(gC, s.y, x1));
@@ -808,7 +809,7 @@ __device__ __forceinline__ void reverse_chain(float *fs, const float *__restrict
         // dU[j][r0 + r] = Z[j][r0 + r] + sum_d K^[j][d] L[r][d]
         bgemm_rc<C, kRowBlock, kChainThreads, false, false, true, 2, true>(
             D, [&](int j, int d) { return Kh[j * LW4 + d]; }, [&](int d, int r) { return Lr[r * LW4 + d]; },
-            [&](int j, int r, float x0, float x1) {
+            [&](int, int j, int r, float x0, float x1) {
                 const float v0 = Zs[j * kRowBlock + r] + x0, v1 = Zs[j * kRowBlock + r + 1] + x1;
                 dUt[r * LN4 + j] = v0;
                 dUt[(r + 1) * LN4 + j] = v1;
@@ -826,7 +827,7 @@ __device__ __forceinline__ void reverse_chain(float *fs, const float *__restrict
             const float gC = __expf(Gs[C - 1]);
             bgemm_rc<kRowBlock, D, kChainThreads, false, false, true, 2, true>(
                 C, [&](int r, int j) { return dUt[r * LN4 + j]; }, [&](int j, int d) { return Ws[j * LW8 + d]; },
-                [&](int r, int d, float x0, float x1) {
+                [&](int, int r, int d, float x0, float x1) {
                     float2 *p = reinterpret_cast<float2 *>(Lr + r * LW4 + d);
                     const float2 l = *p, y = *reinterpret_cast<const float2 *>(Ys + r * LW4 + d);
                     *p = make_float2(fmaf(gC, l.x, y.x - x0), fmaf(gC, l.y, y.y - x1));
@@ -1029,12 +1030,14 @@ bwd_local_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT
     __syncthreads();
     {
         float rowacc[4] = {0.f, 0.f, 0.f, 0.f};
-        bgemm_rc<C, D, kLocalThreads>(C, [&](int j, int i) { return N1[i * LN + j]; },
-                                  [&](int i, int r) { return RB[i * LW + r]; },
-                                  [&](int tr, int, int j, int r, float x) {
-                                      if (j < cl) dv[((size_t)(tok0 + j) * H + h) * D + r] = Bs[j] * x;
-                                      rowacc[tr] += RD[j * LW + r] * x;
-                                  });
+        bgemm_rc<C, D, kLocalThreads, false, false, true>(
+            C, [&](int j, int i) { return N1[i * LN + j]; }, [&](int i, int r) { return RB[i * LW + r]; },
+            [&](int tr, int j, int r, float x0, float x1) {
+                if (j < cl)
+                    *reinterpret_cast<float2 *>(dv + ((size_t)(tok0 + j) * H + h) * D + r) =
+                        make_float2(Bs[j] * x0, Bs[j] * x1);
+                rowacc[tr] += RD[j * LW + r] * x0 + RD[j * LW + r + 1] * x1;
+            });
         flush_rows(dB, rowacc);
     }
     {
@@ -1131,12 +1134,14 @@ bwd_local_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT
             const int i = tslot_row<C, D, kLocalThreads>(r);
             if (i >= cl) continue;
 #pragma unroll
-            for (int c = 0; c < kLocTN; ++c) {
+            for (int c = 0; c < kLocTN; c += 2) {   // slots c, c + 1: columns d, d + 1
                 const int d = tslot_col<C, D, kLocalThreads>(c);
                 if (sole) {
-                    *qk_at(dk, i, d) = dkacc[r][c];
-                    *qk_at(dq, i, d) = dqacc[r][c];
+                    *reinterpret_cast<float2 *>(qk_at(dk, i, d)) = make_float2(dkacc[r][c], dkacc[r][c + 1]);
+                    *reinterpret_cast<float2 *>(qk_at(dq, i, d)) = make_float2(dqacc[r][c], dqacc[r][c + 1]);
                 } else {
+                    atomicAdd(qk_at(dk, i, d + 1), dkacc[r][c + 1]);
+                    atomicAdd(qk_at(dq, i, d + 1), dqacc[r][c + 1]);
                     atomicAdd(qk_at(dk, i, d), dkacc[r][c]);
                     atomicAdd(qk_at(dq, i, d), dqacc[r][c]);
                 }
