@@ -266,7 +266,8 @@ __device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], 
 // PSPLIT as for tgemm_rc (independent accumulator sets for warps with few
 // tiles).
 template <int M, int N, int NTH, bool AEX = false, bool BEX = false, bool PAIRS = false,
-          int KPAR = 1, bool PSPLIT = false, class AF, class BF, class EPI>
+          int KPAR = 1, bool PSPLIT = false, bool APAIR = false, bool BPAIR = false, class AF,
+          class BF, class EPI>
 __device__ __forceinline__ void bgemm_rc(int K, AF a, BF b, EPI epi) {
     using G = WarpGrid<M, N, NTH / 32>;
     constexpr int NP = PSPLIT ? 3 : 1;
@@ -288,22 +289,34 @@ __device__ __forceinline__ void bgemm_rc(int K, AF a, BF b, EPI epi) {
         if (exact) hi = pack_bf16(x0, x1);
         else split_bf16x2(x0, x1, hi, lo);
     };
+    // a k-pair of an operand: one float2 from the accessor (APAIR / BPAIR:
+    // it returns (x(k), x(k + 1)) for even k, one 8-byte load) or two values
+    auto a2 = [&](int m, int k) {
+        if constexpr (APAIR) return a(m, k);
+        else return make_float2(a(m, k), a(m, k + 1));
+    };
+    auto b2 = [&](int k, int n) {
+        if constexpr (BPAIR) return b(k, n);
+        else return make_float2(b(k, n), b(k + 1, n));
+    };
     auto kstep = [&](int k0, float (&ac)[NP][G::MT][G::NT][4]) {
         uint32_t ah[G::MT][4], al[G::MT][4], bh[G::NT][2], bl[G::NT][2];
         const int ka = k0 + 2 * tig;
 #pragma unroll
         for (int mt = 0; mt < G::MT; ++mt) {
             const int m = m0 + mt * 16 + gid;
-            take(a(m, ka), a(m, ka + 1), ah[mt][0], al[mt][0], AEX);
-            take(a(m + 8, ka), a(m + 8, ka + 1), ah[mt][1], al[mt][1], AEX);
-            take(a(m, ka + 8), a(m, ka + 9), ah[mt][2], al[mt][2], AEX);
-            take(a(m + 8, ka + 8), a(m + 8, ka + 9), ah[mt][3], al[mt][3], AEX);
+            float2 x;
+            x = a2(m, ka);         take(x.x, x.y, ah[mt][0], al[mt][0], AEX);
+            x = a2(m + 8, ka);     take(x.x, x.y, ah[mt][1], al[mt][1], AEX);
+            x = a2(m, ka + 8);     take(x.x, x.y, ah[mt][2], al[mt][2], AEX);
+            x = a2(m + 8, ka + 8); take(x.x, x.y, ah[mt][3], al[mt][3], AEX);
         }
 #pragma unroll
         for (int nt = 0; nt < G::NT; ++nt) {
             const int n = n0 + nt * 8 + gid;
-            take(b(ka, n), b(ka + 1, n), bh[nt][0], bl[nt][0], BEX);
-            take(b(ka + 8, n), b(ka + 9, n), bh[nt][1], bl[nt][1], BEX);
+            float2 y;
+            y = b2(ka, n);     take(y.x, y.y, bh[nt][0], bl[nt][0], BEX);
+            y = b2(ka + 8, n); take(y.x, y.y, bh[nt][1], bl[nt][1], BEX);
         }
 #pragma unroll
         for (int mt = 0; mt < G::MT; ++mt)
@@ -624,9 +637,9 @@ bwd_prep_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT 
 // to 132 or 68 floats: 16-byte aligned for the copies, and the float4 reads
 // of 8 different rows by a quarter warp fall in 8 different bank groups.
 constexpr int kChainThreads = 256;
-constexpr int LW4 = D + 4;   // rows read as the A operand or along K
-constexpr int LW8 = D + 8;   // rows read as a K x N B operand
-constexpr int LN4 = C + 4;
+constexpr int LW4 = D + 4;   // rows of a K x N B operand (read down a column)
+constexpr int LW8 = D + 8;   // rows read in k-pairs by 8-byte loads
+constexpr int LN8 = C + 8;
 static_assert(kChainThreads == C * 4, "one 16-byte piece of a column strip per thread");
 
 // 64 x 128 floats of a record field into rows of ld floats.
@@ -656,20 +669,20 @@ __device__ __forceinline__ void stage_g(float *dst, const float *src) {
 }
 
 __device__ __forceinline__ float4 lds4(const float *p) { return *reinterpret_cast<const float4 *>(p); }
-// The CTA's 16 rows (padded) -> rows r0 .. r0 + 15 of a [128][128] field.
-__device__ __forceinline__ void store_rows(float *dst, const float *rows, int r0) {
+// The CTA's 16 rows (rows of ld floats) -> rows r0 .. r0 + 15 of a [128][128] field.
+__device__ __forceinline__ void store_rows(float *dst, const float *rows, int ld, int r0) {
 #pragma unroll
     for (int e = threadIdx.x & (kChainThreads - 1); e < kRowBlock * D / 4; e += kChainThreads) {
         const int r = e >> 5, q = e & 31;
-        *reinterpret_cast<float4 *>(dst + (size_t)(r0 + r) * D + 4 * q) = lds4(rows + r * LW4 + 4 * q);
+        *reinterpret_cast<float4 *>(dst + (size_t)(r0 + r) * D + 4 * q) = lds4(rows + r * ld + 4 * q);
     }
 }
 
-constexpr uint32_t CF_S = 0;                             // S rows [16][LW4]
-constexpr uint32_t CF_UT = CF_S + kRowBlock * LW4;       // U^T [16][LN4]
-constexpr uint32_t CF_W = CF_UT + kRowBlock * LN4;       // W [64][LW4]
-constexpr uint32_t CF_KH = CF_W + C * LW4;               // K^ [64][LW8]
-constexpr uint32_t CF_US = CF_KH + C * LW8;              // U~ columns r0 .. r0 + 15 [64][16]
+constexpr uint32_t CF_S = 0;                             // S rows [16][LW8]
+constexpr uint32_t CF_UT = CF_S + kRowBlock * LW8;       // U^T [16][LN8]
+constexpr uint32_t CF_W = CF_UT + kRowBlock * LN8;       // W [64][LW8]
+constexpr uint32_t CF_KH = CF_W + C * LW8;               // K^ [64][LW4]
+constexpr uint32_t CF_US = CF_KH + C * LW4;              // U~ columns r0 .. r0 + 15 [64][16]
 constexpr uint32_t CF_G = CF_US + C * kRowBlock;         // G [64]
 constexpr uint32_t CF_SMEM = (CF_G + C) * sizeof(float);
 
@@ -688,14 +701,14 @@ __device__ __forceinline__ void forward_chain(float *fs, const float *__restrict
     auto rec_of = [&](int c) { return recs + ((size_t)(b0 + c) * H + h) * R_FLOATS; };
     for (int e = tid; e < kRowBlock * D; e += kChainThreads) {
         const int r = e >> 7, d = e & 127;
-        Sr[r * LW4 + d] = h0 != nullptr ? h0[((size_t)chain * D + r0 + r) * D + d] : 0.f;
+        Sr[r * LW8 + d] = h0 != nullptr ? h0[((size_t)chain * D + r0 + r) * D + d] : 0.f;
     }
     // copy groups, in order: {W, U~} and {K^, G} of every chunk
     if (nch > 0) {
-        stage_c_by_d(Ws, LW4, rec_of(0) + R_W);
+        stage_c_by_d(Ws, LW8, rec_of(0) + R_W);
         stage_strip(Us, rec_of(0) + R_UT, r0);
         cp_commit();
-        stage_c_by_d(Kh, LW8, rec_of(0) + R_KH);
+        stage_c_by_d(Kh, LW4, rec_of(0) + R_KH);
         stage_g(Gs, rec_of(0) + R_G);
         cp_commit();
     }
@@ -709,19 +722,20 @@ __device__ __forceinline__ void forward_chain(float *fs, const float *__restrict
             tc::bulk_prefetch_l2(nx + R_KH, C * D * sizeof(float));
             tc::bulk_prefetch_l2(nx + R_G, C * sizeof(float));
         }
-        store_rows(rec + R_S, Sr, r0);
+        store_rows(rec + R_S, Sr, LW8, r0);
         // U[j][r0 + r] = U~[j][r0 + r] - sum_d W[j][d] S[r][d]
-        bgemm_rc<C, kRowBlock, kChainThreads, false, false, true, 2, true>(
-            D, [&](int j, int d) { return Ws[j * LW4 + d]; }, [&](int d, int r) { return Sr[r * LW4 + d]; },
+        bgemm_rc<C, kRowBlock, kChainThreads, false, false, true, 2, true, true, true>(
+            D, [&](int j, int d) { return *reinterpret_cast<const float2 *>(Ws + j * LW8 + d); },
+            [&](int d, int r) { return *reinterpret_cast<const float2 *>(Sr + r * LW8 + d); },
             [&](int, int j, int r, float x0, float x1) {
                 const float u0 = Us[j * kRowBlock + r] - x0, u1 = Us[j * kRowBlock + r + 1] - x1;
-                Ut[r * LN4 + j] = u0;
-                Ut[(r + 1) * LN4 + j] = u1;
+                Ut[r * LN8 + j] = u0;
+                Ut[(r + 1) * LN8 + j] = u1;
                 *reinterpret_cast<float2 *>(rec + R_U + j * D + r0 + r) = make_float2(u0, u1);
             });
         group_sync(1);   // W and U~ consumed, U^T complete
         if (c + 1 < nch) {
-            stage_c_by_d(Ws, LW4, rec_of(c + 1) + R_W);
+            stage_c_by_d(Ws, LW8, rec_of(c + 1) + R_W);
             stage_strip(Us, rec_of(c + 1) + R_UT, r0);
         }
         cp_commit();
@@ -729,17 +743,18 @@ __device__ __forceinline__ void forward_chain(float *fs, const float *__restrict
         group_sync(1);   // K^ and G of chunk c in place
         {   // S[r][d] = e^{G_C} S[r][d] + sum_j U[j][r] K^[j][d]
             const float gC = __expf(Gs[C - 1]);
-            bgemm_rc<kRowBlock, D, kChainThreads, false, false, true, 2, true>(C, [&](int r, int j) { return Ut[r * LN4 + j]; },
-                                               [&](int j, int d) { return Kh[j * LW8 + d]; },
+            bgemm_rc<kRowBlock, D, kChainThreads, false, false, true, 2, true, true, false>(
+                C, [&](int r, int j) { return *reinterpret_cast<const float2 *>(Ut + r * LN8 + j); },
+                [&](int j, int d) { return Kh[j * LW4 + d]; },
                                                [&](int, int r, int d, float x0, float x1) {
-                                                   float2 *p = reinterpret_cast<float2 *>(Sr + r * LW4 + d);
+                                                   float2 *p = reinterpret_cast<float2 *>(Sr + r * LW8 + d);
                                                    const float2 s = *p;
                                                    *p = make_float2(fmaf(gC, s.x, x0), fmaf(gC, s.y, x1));
                                                });
         }
         group_sync(1);   // K^ and G consumed
         if (c + 1 < nch) {
-            stage_c_by_d(Kh, LW8, rec_of(c + 1) + R_KH);
+            stage_c_by_d(Kh, LW4, rec_of(c + 1) + R_KH);
             stage_g(Gs, rec_of(c + 1) + R_G);
         }
         cp_commit();
@@ -747,12 +762,12 @@ __device__ __forceinline__ void forward_chain(float *fs, const float *__restrict
     cp_wait<0>();
 }
 
-constexpr uint32_t CR_L = 0;                             // L rows [16][LW4]
-constexpr uint32_t CR_DUT = CR_L + kRowBlock * LW4;      // dU^T [16][LN4]
-constexpr uint32_t CR_KH = CR_DUT + kRowBlock * LN4;     // K^ [64][LW4]
-constexpr uint32_t CR_ZS = CR_KH + C * LW4;              // Z columns r0 .. r0 + 15 [64][16]
-constexpr uint32_t CR_W = CR_ZS + C * kRowBlock;         // W [64][LW8]
-constexpr uint32_t CR_YS = CR_W + C * LW8;               // Y rows r0 .. r0 + 15 [16][LW4]
+constexpr uint32_t CR_L = 0;                             // L rows [16][LW8]
+constexpr uint32_t CR_DUT = CR_L + kRowBlock * LW8;      // dU^T [16][LN8]
+constexpr uint32_t CR_KH = CR_DUT + kRowBlock * LN8;     // K^ [64][LW8]
+constexpr uint32_t CR_ZS = CR_KH + C * LW8;              // Z columns r0 .. r0 + 15 [64][16]
+constexpr uint32_t CR_W = CR_ZS + C * kRowBlock;         // W [64][LW4]
+constexpr uint32_t CR_YS = CR_W + C * LW4;               // Y rows r0 .. r0 + 15 [16][LW4]
 constexpr uint32_t CR_G = CR_YS + kRowBlock * LW4;       // G [64]
 constexpr uint32_t CR_SMEM = (CR_G + C) * sizeof(float);
 
@@ -781,14 +796,14 @@ __device__ __forceinline__ void reverse_chain(float *fs, const float *__restrict
     auto rec_of = [&](int c) { return recs + ((size_t)(b0 + c) * H + h) * R_FLOATS; };
     for (int e = tid; e < kRowBlock * D; e += kChainThreads) {
         const int r = e >> 7, d = e & 127;
-        Lr[r * LW4 + d] = dSf != nullptr ? dSf[((size_t)chain * D + r0 + r) * D + d] : 0.f;
+        Lr[r * LW8 + d] = dSf != nullptr ? dSf[((size_t)chain * D + r0 + r) * D + d] : 0.f;
     }
     // copy groups, in order: {K^, Z} and {W, Y, G} of every chunk
     if (nch > 0) {
-        stage_c_by_d(Kh, LW4, rec_of(nch - 1) + R_KH);
+        stage_c_by_d(Kh, LW8, rec_of(nch - 1) + R_KH);
         stage_strip(Zs, rec_of(nch - 1) + R_Z, r0);
         cp_commit();
-        stage_c_by_d(Ws, LW8, rec_of(nch - 1) + R_W);
+        stage_c_by_d(Ws, LW4, rec_of(nch - 1) + R_W);
         stage_row_block(Ys, rec_of(nch - 1) + R_Y, r0);
         stage_g(Gs, rec_of(nch - 1) + R_G);
         cp_commit();
@@ -805,19 +820,20 @@ __device__ __forceinline__ void reverse_chain(float *fs, const float *__restrict
             tc::bulk_prefetch_l2(pv + R_Z, C * D * sizeof(float));
             tc::bulk_prefetch_l2(pv + R_G, C * sizeof(float));
         }
-        store_rows(rec + R_L, Lr, r0);
+        store_rows(rec + R_L, Lr, LW8, r0);
         // dU[j][r0 + r] = Z[j][r0 + r] + sum_d K^[j][d] L[r][d]
-        bgemm_rc<C, kRowBlock, kChainThreads, false, false, true, 2, true>(
-            D, [&](int j, int d) { return Kh[j * LW4 + d]; }, [&](int d, int r) { return Lr[r * LW4 + d]; },
+        bgemm_rc<C, kRowBlock, kChainThreads, false, false, true, 2, true, true, true>(
+            D, [&](int j, int d) { return *reinterpret_cast<const float2 *>(Kh + j * LW8 + d); },
+            [&](int d, int r) { return *reinterpret_cast<const float2 *>(Lr + r * LW8 + d); },
             [&](int, int j, int r, float x0, float x1) {
                 const float v0 = Zs[j * kRowBlock + r] + x0, v1 = Zs[j * kRowBlock + r + 1] + x1;
-                dUt[r * LN4 + j] = v0;
-                dUt[(r + 1) * LN4 + j] = v1;
+                dUt[r * LN8 + j] = v0;
+                dUt[(r + 1) * LN8 + j] = v1;
                 *reinterpret_cast<float2 *>(rec + R_DU + j * D + r0 + r) = make_float2(v0, v1);
             });
         group_sync(2);   // K^ and Z consumed, dU^T complete
         if (c > 0) {
-            stage_c_by_d(Kh, LW4, rec_of(c - 1) + R_KH);
+            stage_c_by_d(Kh, LW8, rec_of(c - 1) + R_KH);
             stage_strip(Zs, rec_of(c - 1) + R_Z, r0);
         }
         cp_commit();
@@ -825,17 +841,18 @@ __device__ __forceinline__ void reverse_chain(float *fs, const float *__restrict
         group_sync(2);   // W, Y and G of chunk c in place
         {   // L[r][d] = e^{G_C} L[r][d] + Y[r0 + r][d] - sum_j dU[j][r] W[j][d]
             const float gC = __expf(Gs[C - 1]);
-            bgemm_rc<kRowBlock, D, kChainThreads, false, false, true, 2, true>(
-                C, [&](int r, int j) { return dUt[r * LN4 + j]; }, [&](int j, int d) { return Ws[j * LW8 + d]; },
+            bgemm_rc<kRowBlock, D, kChainThreads, false, false, true, 2, true, true, false>(
+                C, [&](int r, int j) { return *reinterpret_cast<const float2 *>(dUt + r * LN8 + j); },
+                [&](int j, int d) { return Ws[j * LW4 + d]; },
                 [&](int, int r, int d, float x0, float x1) {
-                    float2 *p = reinterpret_cast<float2 *>(Lr + r * LW4 + d);
+                    float2 *p = reinterpret_cast<float2 *>(Lr + r * LW8 + d);
                     const float2 l = *p, y = *reinterpret_cast<const float2 *>(Ys + r * LW4 + d);
                     *p = make_float2(fmaf(gC, l.x, y.x - x0), fmaf(gC, l.y, y.y - x1));
                 });
         }
         group_sync(2);   // W, Y and G consumed
         if (c > 0) {
-            stage_c_by_d(Ws, LW8, rec_of(c - 1) + R_W);
+            stage_c_by_d(Ws, LW4, rec_of(c - 1) + R_W);
             stage_row_block(Ys, rec_of(c - 1) + R_Y, r0);
             stage_g(Gs, rec_of(c - 1) + R_G);
         }
@@ -846,7 +863,7 @@ __device__ __forceinline__ void reverse_chain(float *fs, const float *__restrict
     if (dh0 != nullptr) {
         for (int e = tid; e < kRowBlock * D; e += kChainThreads) {
             const int r = e >> 7, d = e & 127;
-            dh0[((size_t)chain * D + r0 + r) * D + d] = Lr[r * LW4 + d];
+            dh0[((size_t)chain * D + r0 + r) * D + d] = Lr[r * LW8 + d];
         }
     }
 }
