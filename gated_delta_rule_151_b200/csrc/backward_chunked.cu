@@ -33,9 +33,9 @@
 //   local       one CTA per (chunk, head): every gradient of the chunk's
 //               tokens.
 //
-// Every product runs on the tensor cores as warp-level tf32 MMAs in up to
-// three passes over tf32-split operands (fp32 accuracy; see the products
-// below).  The chunk records live in the workspace: 475,648 bytes per
+// Every product runs on the tensor cores as warp-level MMAs over operands
+// split into a high and a low part (bf16, or tf32 for K K^T and Q K^T), in up
+// to three passes with fp32 accumulation (see the products below).  The chunk records live in the workspace: 475,648 bytes per
 // (chunk, head).
 #include <cuda_bf16.h>
 
@@ -887,12 +887,13 @@ bwd_chains_kernel(const float *__restrict__ h0, const float *__restrict__ dSf,
 
 // --------------------------------------------------------------- local ----
 // One CTA per (global chunk, value head): every gradient of the chunk's
-// tokens.  Shared memory (floats) is reused phase by phase:
-//   RA [128][129]: L', then S, then U [64][129], then K [64][129]
-//   RB [64][129]:  U, then dU, then T dT^T... ([64][65]), then Q
-//   RC [64][129]:  K^, then dW, then (K K^T) o R ([64][65])
-//   RD [64][129]:  dO, then V
-//   N1, N2, N3 [64][65]: T then P; dP then its product form; dT then dA
+// tokens.  Shared memory (floats, rows of LW = 132 or LN = 68) is reused
+// phase by phase:
+//   RA [128][LW]: L', then S, then U [64][LW], then K [64][LW]
+//   RB [64][LW]:  U, then dU, then Y = dT T^T and dA o A / beta ([64][LN]), then Q
+//   RC [64][LW]:  K^, then dW, then (K K^T) o R and dA o A + dP o P ([64][LN])
+//   RD [64][LW]:  dO, then V (RD .. N3 hold S, dense, during phase A)
+//   N1, N2, N3 [64][LN]: T then P^T; dP then its product form; dT then dA
 // and the per-token adjoints dG, dbeta (shared atomics).
 constexpr uint32_t LB_RA = 0;
 constexpr uint32_t LB_RB = LB_RA + D * LW;
