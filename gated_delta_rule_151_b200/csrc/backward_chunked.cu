@@ -142,41 +142,33 @@ struct WarpGrid {
     static_assert(GM * GN == NW && MT * 16 * GM == M && NT * 8 * GN == N, "warp tiling");
 };
 
-// out(m, n) = sum_k a(m, k) b(k, n) over NTH threads; every result goes to
-// epi(r, c, m, n, value) with (r, c) its slot in the calling thread's part
-// (r < 2 MT, c < 2 NT).  Every <M, N, NTH> product hands a thread the same
-// (m, n) in the same slot, so that a caller can sum several products in
-// registers.  A warp with few tiles would wait on one long chain of
-// dependent MMAs: KPAR = 2 alternates the k-steps between two sets of
-// accumulators and PSPLIT gives each tf32 pass its own set, the sets summed
-// at the end.  K is a multiple of 8 KPAR.  AEX (BEX) states that every
-// value a (b) returns is exact in tf32 (a bf16 input), so that its low part
-// and the pass that multiplies it are skipped.
-template <int M, int N, int NTH, int KPAR = 1, bool PSPLIT = false, bool AEX = false,
-          bool BEX = false, class AF, class BF, class EPI>
+// out(m, n) = sum_k a(m, k) b(k, n) over NTH threads (K a multiple of 8);
+// every result goes to epi(r, c, m, n, value) with (r, c) its slot in the
+// calling thread's part (r < 2 MT, c < 2 NT).  Every <M, N, NTH> product
+// hands a thread the same (m, n) in the same slot, so that a caller can sum
+// several products in registers.  AEX (BEX) states that every value a (b)
+// returns is exact in tf32 (a bf16 input), so that its low part and the pass
+// that multiplies it are skipped.
+template <int M, int N, int NTH, bool AEX = false, bool BEX = false, class AF, class BF, class EPI>
 __device__ __forceinline__ void tgemm_rc(int K, AF a, BF b, EPI epi) {
     using G = WarpGrid<M, N, NTH / 32>;
-    constexpr int NP = PSPLIT ? 3 : 1;
     const int t = threadIdx.x & (NTH - 1), lane = t & 31, warp = t >> 5;
     const int gid = lane >> 2, tig = lane & 3;
     const int m0 = (warp / G::GN) * G::WM, n0 = (warp % G::GN) * G::WN;
-    float acc[KPAR][NP][G::MT][G::NT][4];
+    float acc[G::MT][G::NT][4];
 #pragma unroll
-    for (int s = 0; s < KPAR; ++s)
+    for (int mt = 0; mt < G::MT; ++mt)
 #pragma unroll
-        for (int p = 0; p < NP; ++p)
+        for (int nt = 0; nt < G::NT; ++nt)
 #pragma unroll
-            for (int mt = 0; mt < G::MT; ++mt)
-#pragma unroll
-                for (int nt = 0; nt < G::NT; ++nt)
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) acc[s][p][mt][nt][e] = 0.f;
-    auto kstep = [&](int k0, float (&ac)[NP][G::MT][G::NT][4]) {
+            for (int e = 0; e < 4; ++e) acc[mt][nt][e] = 0.f;
+    auto take = [](float x, uint32_t &hi, uint32_t &lo, bool exact) {
+        if (exact) hi = __float_as_uint(x);
+        else split_tf32(x, hi, lo);
+    };
+#pragma unroll 2
+    for (int k0 = 0; k0 < K; k0 += 8) {
         uint32_t ah[G::MT][4], al[G::MT][4], bh[G::NT][2], bl[G::NT][2];
-        auto take = [](float x, uint32_t &hi, uint32_t &lo, bool exact) {
-            if (exact) hi = __float_as_uint(x);
-            else split_tf32(x, hi, lo);
-        };
 #pragma unroll
         for (int mt = 0; mt < G::MT; ++mt) {
             const int m = m0 + mt * 16 + gid;
@@ -195,41 +187,24 @@ __device__ __forceinline__ void tgemm_rc(int K, AF a, BF b, EPI epi) {
         for (int mt = 0; mt < G::MT; ++mt)
 #pragma unroll
             for (int nt = 0; nt < G::NT; ++nt) {
-                if (!AEX) mma_tf32(ac[NP - 1][mt][nt], al[mt], bh[nt]);
-                if (!BEX) mma_tf32(ac[NP > 1 ? 1 : 0][mt][nt], ah[mt], bl[nt]);
-                mma_tf32(ac[0][mt][nt], ah[mt], bh[nt]);
+                if (!AEX) mma_tf32(acc[mt][nt], al[mt], bh[nt]);
+                if (!BEX) mma_tf32(acc[mt][nt], ah[mt], bl[nt]);
+                mma_tf32(acc[mt][nt], ah[mt], bh[nt]);
             }
-    };
-#pragma unroll 2
-    for (int k0 = 0; k0 < K; k0 += 8 * KPAR) {
-        kstep(k0, acc[0]);
-        if (KPAR > 1) kstep(k0 + 8, acc[KPAR - 1]);
     }
 #pragma unroll
     for (int mt = 0; mt < G::MT; ++mt)
 #pragma unroll
         for (int nt = 0; nt < G::NT; ++nt)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                float x = acc[0][0][mt][nt][e], corr = 0.f;
-#pragma unroll
-                for (int s = 0; s < KPAR; ++s)
-#pragma unroll
-                    for (int p = 0; p < NP; ++p)
-                        if (s + p > 0) {
-                            if (p > 0) corr += acc[s][p][mt][nt][e];
-                            else x += acc[s][p][mt][nt][e];
-                        }
+            for (int e = 0; e < 4; ++e)
                 epi(mt * 2 + (e >> 1), nt * 2 + (e & 1), m0 + mt * 16 + gid + 8 * (e >> 1),
-                    n0 + nt * 8 + 2 * tig + (e & 1), x + corr);
-            }
+                    n0 + nt * 8 + 2 * tig + (e & 1), acc[mt][nt][e]);
 }
 
-template <int M, int N, int NTH, int KPAR = 1, bool PSPLIT = false, bool AEX = false,
-          bool BEX = false, class AF, class BF, class EPI>
+template <int M, int N, int NTH, bool AEX = false, bool BEX = false, class AF, class BF, class EPI>
 __device__ __forceinline__ void tgemm(int K, AF a, BF b, EPI epi) {
-    tgemm_rc<M, N, NTH, KPAR, PSPLIT, AEX, BEX>(K, a, b,
-                                                [&](int, int, int m, int n, float v) { epi(m, n, v); });
+    tgemm_rc<M, N, NTH, AEX, BEX>(K, a, b, [&](int, int, int m, int n, float v) { epi(m, n, v); });
 }
 
 // The same products in bf16: each value x splits into x_hi = bf16(x) and
@@ -259,12 +234,16 @@ __device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], 
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
-// tgemm_rc's contract with bf16 products; K a multiple of 16 KPAR.  With
-// PAIRS the results go out two at a time, epi(r, m, n, value(m, n),
-// value(m, n + 1)) with n even and r the row's slot, so that a store can
-// take both.  KPAR and
-// PSPLIT as for tgemm_rc (independent accumulator sets for warps with few
-// tiles).
+// tgemm_rc's contract with bf16 products; K a multiple of 16 KPAR.
+//   PAIRS: the results go out two at a time, epi(r, m, n, value(m, n),
+//          value(m, n + 1)) with n even and r the row's slot, so that a
+//          store can take both.
+//   KPAR, PSPLIT: a warp with few tiles would wait on one long chain of
+//          dependent MMAs, so KPAR = 2 alternates the k-steps between two
+//          sets of accumulators and PSPLIT gives each pass its own set, the
+//          sets summed at the end.
+//   APAIR, BPAIR: the accessor returns the k-pair (x(k), x(k + 1)) for even
+//          k as a float2 (one 8-byte load from a k-contiguous row).
 template <int M, int N, int NTH, bool AEX = false, bool BEX = false, bool PAIRS = false,
           int KPAR = 1, bool PSPLIT = false, bool APAIR = false, bool BPAIR = false, class AF,
           class BF, class EPI>
@@ -579,14 +558,14 @@ bwd_prep_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT 
     // (K K^T) o R (strictly lower) -> record and A = diag(beta) of it; P -> record
     float *Af = fs + PB_A;
     constexpr bool kX = kIoExact<IoT>;
-    tgemm<C, C, kPrepB, 1, false, kX, kX>(D, [&](int i, int d) { return Ks[i * LW + d]; },
+    tgemm<C, C, kPrepB, kX, kX>(D, [&](int i, int d) { return Ks[i * LW + d]; },
                        [&](int d, int j) { return Ks[j * LW + d]; },
                        [&](int i, int j, float x) {
                            const float ar = j < i ? x * __expf(Gs[i] - Gs[j]) : 0.f;
                            rec[R_AR + i * C + j] = ar;
                            Af[ax(i, j)] = Bs[i] * ar;
                        });
-    tgemm<C, C, kPrepB, 1, false, kX, kX>(D, [&](int i, int d) { return Qs[i * LW + d]; },
+    tgemm<C, C, kPrepB, kX, kX>(D, [&](int i, int d) { return Qs[i * LW + d]; },
                        [&](int d, int j) { return Ks[j * LW + d]; },
                        [&](int i, int j, float x) {
                            const float pv = j <= i ? x * __expf(Gs[i] - Gs[j]) : 0.f;
@@ -628,14 +607,15 @@ bwd_prep_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT 
 }
 
 // ------------------------------------------------------ forward / reverse ----
-// One CTA of 256 threads per (sequence, value head, block of 16 state rows);
-// the rows of the state and of its adjoint are independent, so the CTAs of a
-// chain share nothing.  Each chunk takes two products over operands staged
-// in shared memory by 16-byte asynchronous copies.  An operand is reloaded
-// for the next chunk as soon as its product is done, so that its copy runs
-// during the other product and the next chunk's first one.  Rows are padded
-// to 132 or 68 floats: 16-byte aligned for the copies, and the float4 reads
-// of 8 different rows by a quarter warp fall in 8 different bank groups.
+// 256 threads per (sequence, value head, block of 16 state rows) and chain
+// (the forward chain of the state, the reverse chain of its adjoint; one CTA
+// of 512 threads holds both, see bwd_chains_kernel).  The rows of the state
+// and of its adjoint are independent, so the row blocks share nothing.
+// Each chunk takes two products over operands staged in shared memory by
+// 16-byte asynchronous copies.  An operand is reloaded for the next chunk as
+// soon as its product is done, so that its copy runs during the other
+// product.  Rows read in k-pairs (8-byte loads) are padded to 8 mod 32
+// floats, rows read down a column to 4 mod 32: both without bank conflicts.
 constexpr int kChainThreads = 256;
 constexpr int LW4 = D + 4;   // rows of a K x N B operand (read down a column)
 constexpr int LW8 = D + 8;   // rows read in k-pairs by 8-byte loads
