@@ -482,6 +482,10 @@ def gdr_backward(q, k, v, g, beta, initial_state=None, cu_seqlens=None, *, d_o,
     Inputs as for gdr_prefill_chunked_gqa; d_o [T, H, d_v] in the io dtype;
     d_final_state [N, H, d_v, d_k] fp32 or None.  Returns (dq, dk, dv, dg,
     dbeta, d_initial_state) as fp32 tensors (the last None unless wanted).
+    Without a workspace one of gdr_backward_workspace_size bytes is
+    allocated, which selects the chunked form where it applies (scalar gate,
+    d = 128); a workspace too small for its records selects the per-token
+    form.
     """
     _need(q, "q", ndim=3)
     io = q.dtype

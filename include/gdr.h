@@ -410,14 +410,27 @@ GDR_API gdr_status_t gdr_prefill_fused(const void *xq, const void *xk, const voi
  *   dg                [total_T, H] or [total_T, H, d_k]   (zero where g was clamped at -20)
  *   dbeta             [total_T, H]
  *   d_initial_state   [N, H, d_v, d_k], or NULL to skip
- * The workspace (gdr_backward_workspace_size bytes, 16-byte aligned) holds
- * the state checkpointed every 16 tokens: (N + ceil(total_T / 16)) * H *
- * d_v * d_k * 4 bytes.  Pointers: q, k, v, d_o, the states, dq, dk, dv and
- * channel-mode g/dg 16-byte aligned; the rest 4-byte aligned.  Outputs must
- * not overlap inputs.  Errors: GDR_ERR_INVALID_ARG (size, pointer, overlap),
- * GDR_ERR_WORKSPACE (missing or too small), GDR_ERR_CUDA; nothing is launched
- * on error.  Sums over rows use floating-point atomics, so the last bits of
- * dq, dk, dg and dbeta may differ from run to run.
+ * Two forms, chosen by the workspace (16-byte aligned) the caller passes:
+ *   - chunked (scalar gate, d_k = d_v = 128): chunk records of 475,648
+ *     bytes per (chunk, head), 256 + slots * H * 475,648 bytes with slots =
+ *     N * ceil(total_T / N / 64) for equal lengths (cu_seqlens NULL), else
+ *     ceil(total_T / 64) + N.  Its products run on the tensor cores over
+ *     split operands (high and low bf16 or tf32 parts, fp32 accumulation);
+ *     against an fp64 evaluation the gradients agree to about 1e-5 of each
+ *     tensor's largest magnitude.
+ *   - per token (every other shape, or a workspace too small for the
+ *     records): the state checkpointed every 16 tokens, (N + ceil(total_T /
+ *     16)) * H * d_v * d_k * 4 bytes; fp32 CUDA-core arithmetic.
+ * gdr_backward_workspace_size reports the larger of the two where the
+ * chunked form applies by shape (it does not know the gate mode), so that
+ * the workspace it reports always selects the chunked form for the scalar
+ * gate.  Pointers: q, k, v, d_o, the states, dq, dk, dv and channel-mode
+ * g/dg 16-byte aligned; the rest 4-byte aligned.  Outputs must not overlap
+ * inputs.  Errors: GDR_ERR_INVALID_ARG (size, pointer, overlap),
+ * GDR_ERR_WORKSPACE (missing or too small for the token form), GDR_ERR_CUDA;
+ * nothing is launched on error.  Sums over rows or over the value heads of
+ * a group use floating-point atomics, so the last bits of dq, dk, dg and
+ * dbeta may differ from run to run.
  */
 GDR_API gdr_status_t gdr_backward_workspace_size(int32_t num_seqs, int32_t total_T, int32_t H,
                                                  int32_t d_k, int32_t d_v, size_t *bytes);
