@@ -76,32 +76,6 @@ constexpr int kRowBlock = 16;                   // state rows per forward / reve
 constexpr int kLocalThreads = 256;
 constexpr int kLocTM = 4, kLocTN = 8;   // slots of a thread in a <C, D> product over 8 warps
 
-// The chunk's 64 rows of a [T, heads, 128] input (0 past the sequence's end)
-// into padded shared rows: four values per load (8 bytes of bf16 or 16 of
-// fp32), eight loads in flight per thread.
-__device__ __forceinline__ void ld4io(const float *p, float (&x)[4]) {
-    const float4 v = __ldg(reinterpret_cast<const float4 *>(p));
-    x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
-}
-__device__ __forceinline__ void ld4io(const __nv_bfloat16 *p, float (&x)[4]) {
-    const uint2 raw = __ldg(reinterpret_cast<const uint2 *>(p));
-    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.x));
-    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.y));
-    x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y;
-}
-template <int NT, typename IoT>
-__device__ __forceinline__ void load_io_rows(float *dst, const IoT *src, int tok0, int cl, int heads,
-                                             int head) {
-#pragma unroll 8
-    for (int e = threadIdx.x; e < C * D / 4; e += NT) {
-        const int i = e >> 5, d = (e & 31) * 4;
-        float x[4] = {0.f, 0.f, 0.f, 0.f};
-        if (i < cl) ld4io(src + ((size_t)(tok0 + i) * heads + head) * D + d, x);
-        float *o = dst + i * LW + d;
-        o[0] = x[0]; o[1] = x[1]; o[2] = x[2]; o[3] = x[3];
-    }
-}
-
 // ---------------------------------------------------- tensor-core products ----
 // An input held as bf16 is exact in tf32.
 template <typename IoT> constexpr bool kIoExact = std::is_same<IoT, __nv_bfloat16>::value;
@@ -459,19 +433,18 @@ __device__ __forceinline__ void stage_io_rows(float *dst, const IoT *src, int to
         }
     }
 }
-// The bf16 rows staged in four destinations, converted in place: every
-// thread reads its raw pieces, the block synchronises, then writes the fp32
-// rows.  Called by every thread after the copies are waited for and
-// synchronised; ends synchronised.
-template <int NT, typename IoT>
-__device__ __forceinline__ void finish_io_rows(float *d0, float *d1, float *d2, float *d3, int cl) {
+// The bf16 rows staged in NW destinations, converted in place: every thread
+// reads its raw pieces, the block synchronises, then writes the fp32 rows.
+// Called by every thread after the copies are waited for and synchronised;
+// ends synchronised.
+template <int NT, typename IoT, int NW>
+__device__ __forceinline__ void finish_io_rows(float *const (&dst)[NW], int cl) {
     if constexpr (!std::is_same<IoT, float>::value) {
         constexpr int PER = C * D / 8 / NT;
-        float *dst[4] = {d0, d1, d2, d3};
-        uint4 raw[4][PER];
+        uint4 raw[NW][PER];
         const int t = threadIdx.x & (NT - 1);
 #pragma unroll
-        for (int w = 0; w < 4; ++w)
+        for (int w = 0; w < NW; ++w)
 #pragma unroll
             for (int p = 0; p < PER; ++p) {
                 const int e = t + p * NT, i = e >> 4, q = e & 15;
@@ -481,7 +454,7 @@ __device__ __forceinline__ void finish_io_rows(float *d0, float *d1, float *d2, 
             }
         __syncthreads();
 #pragma unroll
-        for (int w = 0; w < 4; ++w)
+        for (int w = 0; w < NW; ++w)
 #pragma unroll
             for (int p = 0; p < PER; ++p) {
                 const int e = t + p * NT, i = e >> 4, q = e & 15;
@@ -554,7 +527,10 @@ bwd_prep_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT 
     }
     cp_wait<0>();
     __syncthreads();
-    finish_io_rows<kPrepB, IoT>(Ks, Qs, Vs, DOs, cl);   // ends synchronised
+    {
+        float *const rows[4] = {Ks, Qs, Vs, DOs};
+        finish_io_rows<kPrepB, IoT>(rows, cl);   // ends synchronised
+    }
     // (K K^T) o R (strictly lower) -> record and A = diag(beta) of it; P -> record
     float *Af = fs + PB_A;
     constexpr bool kX = kIoExact<IoT>;
@@ -994,10 +970,14 @@ bwd_local_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT
     // ---- phase B: dW = -dU S, d(gamma Q) = dO S ---------------------------------
     copy_rows_async<kLocalThreads>(RA, LW, rec + R_S, D, D);
     copy_rows_async<kLocalThreads>(RB, LW, rec + R_DU, C, D);
+    stage_io_rows<kLocalThreads>(RD, dO, tok0, cl, H, h);
     cp_commit();
-    load_io_rows<kLocalThreads>(RD, dO, tok0, cl, H, h);
     cp_wait<0>();
     __syncthreads();
+    {
+        float *const rows[1] = {RD};
+        finish_io_rows<kLocalThreads, IoT>(rows, cl);
+    }
     bgemm<C, D, kLocalThreads>(D, [&](int j, int r) { return RB[j * LW + r]; },
                               [&](int r, int d) { return RA[r * LW + d]; },
                               [&](int j, int d, float x) { RC[j * LW + d] = -x; });
@@ -1023,9 +1003,15 @@ bwd_local_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT
                               [&](int r, int j) { return RA[j * LW + r]; },
                               [&](int i, int j, float x) { N2[i * LN + j] = j <= i ? x : 0.f; });
     __syncthreads();
-    load_io_rows<kLocalThreads>(RD, v, tok0, cl, H, h);
-    load_io_rows<kLocalThreads>(RA, k, tok0, cl, Hqk, hq);
+    stage_io_rows<kLocalThreads>(RD, v, tok0, cl, H, h);
+    stage_io_rows<kLocalThreads>(RA, k, tok0, cl, Hqk, hq);
+    cp_commit();
+    cp_wait<0>();
     __syncthreads();
+    {
+        float *const rows[2] = {RD, RA};
+        finish_io_rows<kLocalThreads, IoT>(rows, cl);
+    }
     {
         float rowacc[4] = {0.f, 0.f, 0.f, 0.f};
         bgemm_rc<C, D, kLocalThreads, false, false, true>(
@@ -1110,8 +1096,14 @@ bwd_local_kernel(const IoT *__restrict__ q, const IoT *__restrict__ k, const IoT
         }
         __syncthreads();
     }
-    load_io_rows<kLocalThreads>(RB, q, tok0, cl, Hqk, hq);   // Q rows over the finished Y
+    stage_io_rows<kLocalThreads>(RB, q, tok0, cl, Hqk, hq);   // Q rows over the finished Y
+    cp_commit();
+    cp_wait<0>();
     __syncthreads();
+    {
+        float *const rows[1] = {RB};
+        finish_io_rows<kLocalThreads, IoT>(rows, cl);
+    }
     auto add_dk = [&](int tr, int tc, int, int, float x) { dkacc[tr][tc] += x; };
     constexpr bool kX = kIoExact<IoT>;
     // dk_i += sum_j M_ij k_j and dk_j += sum_i M_ij k_i: one product with M + M^T
@@ -1213,12 +1205,15 @@ cudaError_t launch_backward_chunked(const void *q, const void *k, const void *v,
                                     void *workspace, cudaStream_t stream) {
     const long long slots = chunk_slots(num_seqs, total_T, cu == nullptr);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
-    // dq and dk sum over the value heads of a group and over the product
-    // terms: atomics into zeroed outputs; dv, dg, dbeta are written once
-    const size_t nq = (size_t)total_T * Hqk * D * sizeof(float);
-    cudaError_t e = cudaMemsetAsync(dq, 0, nq, stream);
-    if (e == cudaSuccess) e = cudaMemsetAsync(dk, 0, nq, stream);
-    if (e != cudaSuccess) return e;
+    // dq and dk: with grouped heads the value heads of a group add into them
+    // with atomics (zeroed first); otherwise every row of every sequence is
+    // stored once by its chunk's CTA.  dv, dg, dbeta are written once.
+    if (Hqk != H) {
+        const size_t nq = (size_t)total_T * Hqk * D * sizeof(float);
+        cudaError_t e = cudaMemsetAsync(dq, 0, nq, stream);
+        if (e == cudaSuccess) e = cudaMemsetAsync(dk, 0, nq, stream);
+        if (e != cudaSuccess) return e;
+    }
     const size_t bb = base_bytes_of(num_seqs);
     if (bf16)
         return launch_chunked<__nv_bfloat16>(
