@@ -141,3 +141,78 @@ def test_chunk_size_does_not_change_the_gradient():
     b = chunked_gradient(*args, C=16)
     for key in a:
         assert np.allclose(a[key], b[key], rtol=1e-10, atol=1e-12), key
+
+
+def chunked_gradient_channel(q, k, v, g, beta, h0, dO, dSf, C):
+    """The same chunk algebra for a gate per key channel (g [T, dk]), the
+    decays carried by the key-side operands: with G the within-chunk
+    cumulative log-gate per channel, K~ = K o e^G, K- = K o e^-G,
+    Q~ = Q o e^G, K^ = K o e^{G_C - G},
+
+      A = strictly-lower(diag(beta) K~ K-^T), P = causal(Q~ K-^T),
+      W = T diag(beta) K~, S' = S Diag(e^{G_C}) + U^T K^,
+      L = L' Diag(e^{G_C}) + dO^T Q~ - dU^T W,
+
+    and the adjoint of G per channel from each of K~, K-, K^, Q~ and
+    e^{G_C}.  (fp64, moderate gates: e^-G stays in range.)"""
+    T = q.shape[0]
+    n_chunks = (T + C - 1) // C
+    chunks, S = [], h0.copy()
+    for c in range(n_chunks):
+        a, b = c * C, min(T, c * C + C)
+        K, Q, V, bt = k[a:b], q[a:b], v[a:b], beta[a:b]
+        G = np.cumsum(g[a:b], axis=0)
+        GC = G[-1]
+        Kt, Km, Qt = K * np.exp(G), K * np.exp(-G), Q * np.exp(G)
+        Kh = K * np.exp(GC - G)
+        A = np.tril(bt[:, None] * (Kt @ Km.T), -1)
+        Tm = np.linalg.inv(np.eye(b - a) + A)
+        W = Tm @ (bt[:, None] * Kt)
+        Ut = Tm @ (bt[:, None] * V)
+        P = np.tril(Qt @ Km.T)
+        U = Ut - W @ S.T
+        chunks.append(dict(a=a, b=b, K=K, Q=Q, V=V, bt=bt, G=G, GC=GC, Kt=Kt, Km=Km, Qt=Qt,
+                           Kh=Kh, A=A, T=Tm, W=W, P=P, U=U, S=S.copy()))
+        S = S * np.exp(GC)[None, :] + U.T @ Kh
+    dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    dg, db = np.zeros_like(g), np.zeros(T)
+    Lam = dSf.copy()
+    for z in reversed(chunks):
+        a, b = z["a"], z["b"]
+        K, Q, V, bt, G, GC, Tm = z["K"], z["Q"], z["V"], z["bt"], z["G"], z["GC"], z["T"]
+        Kt, Km, Qt, Kh, W, P, U, S = z["Kt"], z["Km"], z["Qt"], z["Kh"], z["W"], z["P"], z["U"], z["S"]
+        dOc = dO[a:b]
+        dU = Kh @ Lam.T + P.T @ dOc
+        dKh = U @ Lam
+        dP = np.tril(dOc @ U.T)
+        dQt = dOc @ S
+        dW = -dU @ S
+        dT = dW @ (bt[:, None] * Kt).T + dU @ (bt[:, None] * V).T
+        X1, X2 = Tm.T @ dU, Tm.T @ dW
+        dA = np.tril(-Tm.T @ dT @ Tm.T, -1)
+        dKt = bt[:, None] * X2 + bt[:, None] * (dA @ Km)
+        dKm = dA.T @ (bt[:, None] * Kt) + dP.T @ Qt
+        dQt = dQt + dP @ Km
+        dv[a:b] += bt[:, None] * X1
+        db[a:b] += np.sum(V * X1, 1) + np.sum(Kt * X2, 1) + np.sum(dA * (Kt @ Km.T), 1)
+        dk[a:b] += dKt * np.exp(G) + dKm * np.exp(-G) + dKh * np.exp(GC - G)
+        dq[a:b] += dQt * np.exp(G)
+        dG = dKt * Kt - dKm * Km - dKh * Kh + dQt * Qt
+        dG[-1] += np.exp(GC) * np.sum(S * Lam, 0) + np.sum(dKh * Kh, 0)
+        dg[a:b] = np.cumsum(dG[::-1], axis=0)[::-1]
+        Lam = Lam * np.exp(GC)[None, :] + dOc.T @ Qt - dU.T @ W
+    return dict(dq=dq, dk=dk, dv=dv, dg=dg, dbeta=db, dh0=Lam)
+
+
+@pytest.mark.parametrize("T, C, dk, dv", [(37, 8, 6, 5), (16, 16, 4, 4), (3, 8, 5, 3)])
+def test_channel_gate_chunk_algebra_matches_the_token_oracle(T, C, dk, dv):
+    q, k, v, _, beta, h0, dO, dSf = _case(11 + T, T, dk, dv, 0.3)
+    rng = np.random.default_rng(100 + T)
+    g = -np.log1p(np.exp(rng.standard_normal((T, dk)))) * 0.2   # one log-gate per key channel
+    got = chunked_gradient_channel(q, k, v, g, beta, h0, dO, dSf, C)
+    ref = OB.backward(q[:, None], k[:, None], v[:, None], g[:, None], beta[:, None],
+                      h0[None, None], None, dO[:, None], dSf[None, None])
+    for key in ("dq", "dk", "dv", "dg", "dbeta", "dh0"):
+        r = np.asarray(ref[key], dtype=np.float64).reshape(got[key].shape)
+        scale = max(float(np.max(np.abs(r))), 1e-30)
+        assert float(np.max(np.abs(got[key] - r))) <= 1e-9 * scale, key
