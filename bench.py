@@ -578,6 +578,27 @@ class FusedPrefillCase:
         return "bf16/fp16 tensor-core operands, fp32 accumulate, state and prologue arithmetic"
 
 
+def backward_flops(inp, C=64):
+    """Flops of the chunked gradient's products per step (2 per multiply-add;
+    the forms the kernels run, each product once whatever its number of
+    split passes).  Per (chunk, head), with d = d_k = d_v:
+      prep    K K^T, Q K^T (C C d each), W, U~ (C d C each), Y (d d C), Z (C d C)
+      chains  forward W S^T, U^T K^ and reverse K^ L'^T, dU^T W (d d C each)
+      local   U L', dU S, dO S (C d d each); dP, T^T dU, T^T dW, the two terms
+              of dT, (M + M^T) K, (dP o R) K, (dP o R)^T Q (C C d each);
+              dT T^T, T^T Y (C C C each)
+    Zero where the chunked form does not apply (it runs the token form)."""
+    if inp.gate_mode != I.SCALAR or inp.d_k != 128 or inp.d_v != 128:
+        return 0
+    d = inp.d_k
+    macs = (2 * C * C * d + 2 * C * d * C + d * d * C + C * d * C      # prep
+            + 4 * d * d * C                                            # chains
+            + 3 * C * d * d + 8 * C * C * d + 2 * C * C * C)           # local
+    cu = inp.cu_seqlens.numpy()
+    chunks = int(sum((int(cu[n + 1]) - int(cu[n]) + C - 1) // C for n in range(len(cu) - 1)))
+    return 2 * macs * chunks * inp.H
+
+
 class BackwardCase:
     """The gradient of the recurrence at the gdn_prefill shape: one
     gdr_backward call per step (upstream gradients dO and dS_final drawn by
@@ -606,7 +627,7 @@ class BackwardCase:
         self.bytes = (T * (2 * Hqk * dk + 2 * H * dv) * e + 2 * gate + 2 * T * H * 4
                       + (2 if inp.h0 is not None else 1) * state
                       + T * (2 * Hqk * dk + H * dv) * 4 + state)
-        self.flops = 0
+        self.flops = backward_flops(inp)
         self.tokens = T
         self.launches = 4   # chunk numbering, prep, the two chains in one launch, local gradients
         self.path = None
@@ -795,6 +816,16 @@ def bench_case(case, args, ws, rank, flush, stream, pk, pk_kind):
     else:
         roof["algorithmic_bytes_per_launch"] = case.bytes
         roof["frac_of_8TBps_nominal"] = round(achieved / 8000.0, 4)
+    if case.kind == "backward" and case.flops:
+        # the gradient's products are fp32-accurate (split operands on the
+        # tensor cores): their useful rate against the CUDA cores' fp32 FMA
+        # rate, 148 SMs x 128 lanes x 2 flops at the maximum SM clock
+        fma_peak = 148 * 128 * 2 * 1965e6 / 1e12
+        rate = case.flops / (launch_ms / 1e3) / 1e12
+        roof["flops_per_launch"] = case.flops
+        roof["fp32_equivalent_tflops"] = round(rate, 2)
+        roof["frac_of_fp32_fma_peak"] = round(rate / fma_peak, 4)
+        roof["fp32_fma_peak_tflops"] = round(fma_peak, 1)
 
     # end to end: pinned host buffers, copies inside the timed region
     host, ho, hf, h2d, d2h = case.e2e_buffers()

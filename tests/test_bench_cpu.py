@@ -85,6 +85,16 @@ def test_backward_bytes_per_launch():
     # the chunked form's records: 475,648 bytes per (chunk, head) for up to
     # T / 64 + 1 chunks (cu_seqlens given), after 256 bytes of chunk offsets
     assert case.ws.numel() == 256 + (T // 64 + 1) * H * 475648
+    # the chunked form's products, per (chunk, head): prep 3.67 M, chains
+    # 4.19 M, local 7.86 M multiply-adds (d = 128, C = 64), over 128 x 16
+    macs = (2 * 64 * 64 * 128 * 2 + 128 * 128 * 64 + 64 * 128 * 64
+            + 4 * 128 * 128 * 64
+            + 3 * 64 * 128 * 128 + 8 * 64 * 64 * 128 + 2 * 64 ** 3)
+    assert macs == 15_728_640
+    assert case.flops == 2 * macs * (T // 64) * H
+    # no chunked form for the channel gate: no flop count
+    kda = I.make_inputs(total_T=128, H=2, d_k=128, num_seqs=1, gate_mode=I.CHANNEL, seed=1)
+    assert bench.backward_flops(kda) == 0
 
 
 def test_reference_arm_under_two_ranks_prints_once():
